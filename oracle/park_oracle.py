@@ -1,0 +1,424 @@
+"""PARK oracle: a plain, slow, float64 CPU statement of what the hot path computes.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` use it.  It shares no code with the
+CUDA library; the only module both sides import is ``synth`` (seeded inputs).
+
+Source: "PARK: Accurate Block Retrieval for Sparse Attention in Video Diffusion
+Transformers" (abstract, AI summary, Figure 1 and Figure 2 captions, Table 1
+caption).  The pages give no equations; every step below is the plainest reading
+of their words, and each reading that fills a gap is marked READING.
+
+Notation, per (batch b, head h): Q, K, V in R^{N x d}; s = 1/sqrt(d); query
+clusters r = 0..NQ-1, key clusters m = 0..NK-1.  All arithmetic is float64.
+Values that the method stores in the input dtype (centroids) are rounded once,
+round-to-nearest-even, from float64.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+# ----------------------------------------------------------------------------
+# rounding to the storage dtype
+# ----------------------------------------------------------------------------
+
+
+def round_to_bf16(x):
+    """Nearest bf16 (8 significant bits, ties to even) of float64 values, taken
+    directly from float64 (no intermediate float32)."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)                      # |x| in [2^(e-1), 2^e)
+    e = np.maximum(e, -125)                 # below 2^-126 the bf16 ulp is fixed at 2^-133
+    return np.ldexp(np.rint(np.ldexp(x, 8 - e)), e - 8)
+
+
+def round_to(x, dtype):
+    """Round float64 values to the storage dtype ("bf16", "f32", or None = keep)."""
+    if dtype is None:
+        return np.asarray(x, dtype=np.float64)
+    if dtype == "bf16":
+        return round_to_bf16(x)
+    if dtype == "f32":
+        return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+    raise ValueError(dtype)
+
+
+# ----------------------------------------------------------------------------
+# QRKC metric
+# ----------------------------------------------------------------------------
+
+
+def metric(Q):
+    """M = (1/N) sum_i q_i q_i^T, the queries' second-moment matrix.
+
+    READING of "transforms keys using a metric derived from the current
+    queries, so that keys receiving similar QK scores are grouped together"
+    (PARK, Figure 2 caption): for any key k and centroid c,
+    (k - c)^T M (k - c) = mean_i (q_i.k - q_i.c)^2, the mean squared QK-score
+    difference under the current queries, which is what the pages want small
+    inside a key cluster.  A library matmul forms the sum."""
+    Q = np.asarray(Q, dtype=np.float64)
+    return (Q.T @ Q) / Q.shape[0]
+
+
+def metric_factor(M):
+    """F with M = F F^T (eigendecomposition, clipped at 0 for a PSD M), so that
+    (x - c)^T M (x - c) = ||F^T x - F^T c||^2: keys transformed before
+    clustering, as the pages put it (PARK abstract)."""
+    lam, V = np.linalg.eigh(np.asarray(M, dtype=np.float64))
+    return V * np.sqrt(np.clip(lam, 0.0, None))
+
+
+# ----------------------------------------------------------------------------
+# K-means (queries: Euclidean; keys: QRKC)
+# ----------------------------------------------------------------------------
+
+
+def strided_init(X, K):
+    """READING (pages silent on initialisation): c_k = x_floor(k N / K)."""
+    N = X.shape[0]
+    return np.asarray(X, dtype=np.float64)[(np.arange(K) * N) // K].copy()
+
+
+def distances(X, C, M=None, row_block=4096):
+    """D[i, k] = (x_i - c_k)^T M (x_i - c_k); M = None means the identity
+    (standard Euclidean K-means, PARK Figure 2 caption).  For a metric the keys
+    and centroids are first transformed by F^T with M = F F^T."""
+    X = np.asarray(X, dtype=np.float64)
+    C = np.asarray(C, dtype=np.float64)
+    if M is not None:
+        F = metric_factor(M)
+        X = X @ F
+        C = C @ F
+    D = np.empty((X.shape[0], C.shape[0]))
+    for i0 in range(0, X.shape[0], row_block):
+        diff = X[i0:i0 + row_block, None, :] - C[None, :, :]
+        D[i0:i0 + row_block] = np.sum(diff * diff, axis=2)
+    return D
+
+
+def assign(X, C, M=None):
+    """a(i) = argmin_k D(x_i, c_k); ties go to the lowest k (READING)."""
+    return np.argmin(distances(X, C, M), axis=1).astype(np.int64)
+
+
+def exact_mean(rows, dtype):
+    """Centroid = round_dtype( fl64(exact sum of the rows) / n ).
+
+    The column sums are exact and rounded once to float64 (math.fsum is
+    correctly rounded), then divided by n in IEEE float64, then rounded to the
+    storage dtype.  READING: the pages only say clusters are represented by
+    their averages (PARK abstract, "averaged representations")."""
+    n = rows.shape[0]
+    sums = np.array([math.fsum(col) for col in np.asarray(rows, dtype=np.float64).T.tolist()])
+    return round_to(sums / float(n), dtype)
+
+
+def update(X, labels, C_prev, dtype):
+    """Centroid update; an empty cluster keeps its previous centroid (READING)."""
+    X = np.asarray(X, dtype=np.float64)
+    C = np.array(C_prev, dtype=np.float64, copy=True)
+    order = np.argsort(labels, kind="stable")
+    counts = np.bincount(labels, minlength=C.shape[0])
+    start = 0
+    for k in range(C.shape[0]):
+        n = counts[k]
+        if n:
+            C[k] = exact_mean(X[order[start:start + n]], dtype)
+        start += n
+    return C
+
+
+def kmeans(X, K, iters, M=None, dtype="bf16", init=None, history=False):
+    """Lloyd K-means: `iters` x (assign, update), no early stop (READING).
+
+    Returns (labels of the last assign, centroids of the last update) and, with
+    history=True, the list of centroids entering each iteration."""
+    if iters < 1:
+        raise ValueError("iters >= 1")
+    C = strided_init(X, K) if init is None else np.array(init, dtype=np.float64, copy=True)
+    hist = []
+    labels = None
+    for _ in range(iters):
+        hist.append(C.copy())
+        labels = assign(X, C, M)
+        C = update(X, labels, C, dtype)
+    return (labels, C, hist) if history else (labels, C)
+
+
+def objective(X, labels, C, M=None):
+    """sum_i D(x_i, c_a(i))."""
+    D = distances(X, C, M)
+    return float(np.sum(D[np.arange(X.shape[0]), labels]))
+
+
+# ----------------------------------------------------------------------------
+# blocks: stable permutation by cluster
+# ----------------------------------------------------------------------------
+
+
+def stable_permutation(labels, K):
+    """Counting sort: perm[pos] = original token index, cluster by cluster,
+    original order inside a cluster; offsets[k] = first position of cluster k.
+    READING: the query/key "blocks" are the clusters (PARK Figure 2)."""
+    labels = np.asarray(labels)
+    counts = [0] * K
+    for a in labels.tolist():
+        counts[a] += 1
+    offsets = [0] * (K + 1)
+    for k in range(K):
+        offsets[k + 1] = offsets[k] + counts[k]
+    cursor = offsets[:-1].copy()
+    perm = [0] * len(labels)
+    for i, a in enumerate(labels.tolist()):
+        perm[cursor[a]] = i
+        cursor[a] += 1
+    return np.array(perm, dtype=np.int64), np.array(offsets, dtype=np.int64)
+
+
+# ----------------------------------------------------------------------------
+# PAMA block importance
+# ----------------------------------------------------------------------------
+
+
+def pama(Q, q_labels, NQ, CK, k_counts, scale, row_block=8192):
+    """Block-importance map I[r, m].
+
+    PARK (abstract; Figure 2 caption): every original query keeps its own
+    Softmax over the key centroids, and these distributions are averaged within
+    each query block:
+        P_im = softmax_m(s q_i . c_m),   I_rm = mean_{i in Q_r} P_im.
+    READING: only non-empty key clusters take part (an empty cluster stands for
+    no keys); rows of empty query clusters are 0."""
+    Q = np.asarray(Q, dtype=np.float64)
+    CK = np.asarray(CK, dtype=np.float64)
+    live = np.nonzero(np.asarray(k_counts) > 0)[0]
+    NK = CK.shape[0]
+    sums = np.zeros((NQ, live.size))
+    q_labels = np.asarray(q_labels)
+    for i0 in range(0, Q.shape[0], row_block):
+        Z = scale * (Q[i0:i0 + row_block] @ CK[live].T)
+        Z -= Z.max(axis=1, keepdims=True)
+        P = np.exp(Z)
+        P /= P.sum(axis=1, keepdims=True)
+        np.add.at(sums, q_labels[i0:i0 + row_block], P)
+    q_counts = np.bincount(q_labels, minlength=NQ)
+    I = np.zeros((NQ, NK))
+    nz = q_counts > 0
+    I[np.ix_(nz, live)] = sums[nz] / q_counts[nz, None]
+    return I
+
+
+def pama_centroid_query(CQ, q_counts, CK, k_counts, scale):
+    """"w/o PAMA" ablation (PARK Table 3; Figure 1(a)): the query centroid is
+    scored instead of every query, i.e. queries are averaged before Softmax:
+    I_rm = softmax_m(s c_r^Q . c_m) for non-empty r, m."""
+    live = np.nonzero(np.asarray(k_counts) > 0)[0]
+    I = np.zeros((CQ.shape[0], CK.shape[0]))
+    for r in range(CQ.shape[0]):
+        if q_counts[r] == 0:
+            continue
+        z = scale * (np.asarray(CK, dtype=np.float64)[live] @ np.asarray(CQ[r], dtype=np.float64))
+        z -= z.max()
+        e = np.exp(z)
+        I[r, live] = e / e.sum()
+    return I
+
+
+# ----------------------------------------------------------------------------
+# top-p selection
+# ----------------------------------------------------------------------------
+
+
+def top_p(I, p, q_counts, k_counts):
+    """Keep, per non-empty query cluster r, the shortest prefix of the key
+    clusters sorted by I[r, m] descending (ties: lower m first) whose float64
+    running sum reaches p; the crossing block is kept (PARK Table 1 caption:
+    top-p block retrieval, p = 0.9).  READING: p >= 1 keeps every non-empty key
+    cluster; empty query clusters keep nothing."""
+    NQ, NK = I.shape
+    mask = np.zeros((NQ, NK), dtype=bool)
+    live = [m for m in range(NK) if k_counts[m] > 0]
+    for r in range(NQ):
+        if q_counts[r] == 0:
+            continue
+        if p >= 1.0:
+            mask[r, live] = True
+            continue
+        order = sorted(live, key=lambda m: (-I[r, m], m))
+        acc = 0.0
+        for m in order:
+            mask[r, m] = True
+            acc += I[r, m]
+            if acc >= p:
+                break
+    return mask
+
+
+def top_k_ratio(I, rho, q_counts, k_counts):
+    """Top-k at a fixed retrieval ratio rho (PARK Table 10): keep the
+    ceil(rho * NK_live) most important key clusters (ties: lower m)."""
+    NQ, NK = I.shape
+    mask = np.zeros((NQ, NK), dtype=bool)
+    live = [m for m in range(NK) if k_counts[m] > 0]
+    k = max(1, int(math.ceil(rho * len(live))))
+    for r in range(NQ):
+        if q_counts[r] == 0:
+            continue
+        order = sorted(live, key=lambda m: (-I[r, m], m))
+        mask[r, order[:k]] = True
+    return mask
+
+
+# ----------------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------------
+
+
+def dense_attention(Q, K, V, scale):
+    """Textbook attention softmax(s Q K^T) V, row by row block."""
+    Q, K, V = (np.asarray(a, dtype=np.float64) for a in (Q, K, V))
+    O = np.empty((Q.shape[0], V.shape[1]))
+    for i0 in range(0, Q.shape[0], 2048):
+        S = scale * (Q[i0:i0 + 2048] @ K.T)
+        S -= S.max(axis=1, keepdims=True)
+        P = np.exp(S)
+        O[i0:i0 + 2048] = (P @ V) / P.sum(axis=1, keepdims=True)
+    return O
+
+
+def sparse_attention(Q, K, V, q_labels, k_labels, mask, scale, rows=None):
+    """Block-sparse attention: query i attends, with a renormalised Softmax,
+    only to keys whose cluster is kept for its query cluster a(i) ("computing
+    attention only within" the retrieved blocks, PARK abstract).  Returns
+    float64 [N, d] in original token order (or only the listed rows)."""
+    Q, K, V = (np.asarray(a, dtype=np.float64) for a in (Q, K, V))
+    q_labels = np.asarray(q_labels)
+    k_labels = np.asarray(k_labels)
+    want = np.arange(Q.shape[0]) if rows is None else np.asarray(rows)
+    O = np.zeros((want.size, V.shape[1]))
+    lab = q_labels[want]
+    for r in np.unique(lab):
+        sel = np.nonzero(lab == r)[0]
+        keys = np.nonzero(mask[r][k_labels])[0]
+        S = scale * (Q[want[sel]] @ K[keys].T)
+        S -= S.max(axis=1, keepdims=True)
+        P = np.exp(S)
+        O[sel] = (P @ V[keys]) / P.sum(axis=1, keepdims=True)
+    return O
+
+
+# ----------------------------------------------------------------------------
+# one layer
+# ----------------------------------------------------------------------------
+
+
+def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full"):
+    """PARK retrieval for one (b, h): query K-means (Euclidean), key K-means
+    with the query-derived metric (QRKC), PAMA importance, top-p mask
+    (PARK Figure 2).  qrkc=False is the "w/o QRKC" ablation (M = I);
+    pama_mode="centroid" is "w/o PAMA"."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    d = Q.shape[1]
+    scale = 1.0 / math.sqrt(d)
+    M = metric(Q)
+    q_labels, CQ = kmeans(Q, NQ, iters, None, dtype)
+    k_labels, CK = kmeans(K, NK, iters, M if qrkc else None, dtype)
+    q_counts = np.bincount(q_labels, minlength=NQ)
+    k_counts = np.bincount(k_labels, minlength=NK)
+    if pama_mode == "full":
+        I = pama(Q, q_labels, NQ, CK, k_counts, scale)
+    else:
+        I = pama_centroid_query(CQ, q_counts, CK, k_counts, scale)
+    mask = top_p(I, p, q_counts, k_counts)
+    q_perm, q_off = stable_permutation(q_labels, NQ)
+    k_perm, k_off = stable_permutation(k_labels, NK)
+    return dict(M=M, q_labels=q_labels, k_labels=k_labels, q_centroids=CQ, k_centroids=CK,
+                q_counts=q_counts, k_counts=k_counts, importance=I, mask=mask,
+                q_perm=q_perm, q_offsets=q_off, k_perm=k_perm, k_offsets=k_off)
+
+
+def layer_head(Q, K, V, NQ, NK, p, iters, dtype, **kw):
+    """Retrieval followed by block-sparse attention for one (b, h)."""
+    r = retrieve_head(Q, K, NQ, NK, p, iters, dtype, **kw)
+    scale = 1.0 / math.sqrt(np.asarray(Q).shape[1])
+    r["O"] = sparse_attention(Q, K, V, r["q_labels"], r["k_labels"], r["mask"], scale)
+    return r
+
+
+def layer(Q, K, V, NQ, NK, p, iters, dtype, **kw):
+    """All (b, h) of [B, H, N, d] inputs; returns a list (row-major over b, h)."""
+    B, H = Q.shape[:2]
+    return [layer_head(Q[b, h], K[b, h], V[b, h], NQ, NK, p, iters, dtype, **kw)
+            for b in range(B) for h in range(H)]
+
+
+# ----------------------------------------------------------------------------
+# diagnostics (PARK Tables 1, 4, 5)
+# ----------------------------------------------------------------------------
+
+
+def block_recall(Q, K, q_labels, k_labels, mask, scale, rows=None):
+    """Attention recall of the kept blocks: (1/|rows|) sum_i sum_{j in J_a(i)} A_ij
+    with A the dense float64 softmax(s Q K^T) (PARK Table 1)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    want = np.arange(Q.shape[0]) if rows is None else np.asarray(rows)
+    q_labels = np.asarray(q_labels)
+    k_labels = np.asarray(k_labels)
+    tot = 0.0
+    for i0 in range(0, want.size, 2048):
+        idx = want[i0:i0 + 2048]
+        S = scale * (Q[idx] @ K.T)
+        S -= S.max(axis=1, keepdims=True)
+        A = np.exp(S)
+        A /= A.sum(axis=1, keepdims=True)
+        keep = mask[q_labels[idx]][:, k_labels]
+        tot += float(np.sum(A * keep))
+    return tot / want.size
+
+
+def exact_block_mass(Q, K, q_labels, NQ, k_labels, NK, scale):
+    """Full-query / full-key block importance: I_rm = mean_{i in Q_r} sum_{j in B_m} A_ij."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    S = scale * (Q @ K.T)
+    S -= S.max(axis=1, keepdims=True)
+    A = np.exp(S)
+    A /= A.sum(axis=1, keepdims=True)
+    mass = np.zeros((Q.shape[0], NK))
+    np.add.at(mass.T, np.asarray(k_labels), A.T)
+    q_counts = np.bincount(q_labels, minlength=NQ)
+    I = np.zeros((NQ, NK))
+    np.add.at(I, np.asarray(q_labels), mass)
+    nz = q_counts > 0
+    I[nz] /= q_counts[nz, None]
+    return I, mass
+
+
+def attention_tv(Q, K, k_labels, NK, CK, scale):
+    """PARK Table 4, full-query / centroid-key row: mean_i (1/2) sum_m |P_im - sum_{j in B_m} A_ij|."""
+    Q = np.asarray(Q, dtype=np.float64)
+    k_counts = np.bincount(k_labels, minlength=NK)
+    live = np.nonzero(k_counts > 0)[0]
+    Z = scale * (Q @ np.asarray(CK, dtype=np.float64)[live].T)
+    Z -= Z.max(axis=1, keepdims=True)
+    P = np.exp(Z)
+    P /= P.sum(axis=1, keepdims=True)
+    _, mass = exact_block_mass(Q, K, np.zeros(Q.shape[0], dtype=np.int64), 1, k_labels, NK, scale)
+    return float(np.mean(0.5 * np.sum(np.abs(P - mass[:, live]), axis=1)))
+
+
+def key_errors(Q, K, k_labels, CK):
+    """PARK Table 5: raw-key MSE mean_j ||k_j - c_a(j)||^2 / d ... reported as the
+    mean over keys of the squared distance, and the QK-score squared error
+    mean_{i,j} (q_i.k_j - q_i.c_a(j))^2, computed directly over queries."""
+    Q = np.asarray(Q, dtype=np.float64)
+    R = np.asarray(K, dtype=np.float64) - np.asarray(CK, dtype=np.float64)[np.asarray(k_labels)]
+    raw = float(np.mean(np.sum(R * R, axis=1)))
+    qk = float(np.mean((Q @ R.T) ** 2))
+    return raw, qk
