@@ -1,0 +1,589 @@
+// PAMA block importance, top-p selection and the kept-block CSR.
+//
+// PAMA (PARK abstract; Figure 2 caption): every query i keeps its own Softmax
+// over the non-empty key clusters, P_im = softmax_m(q_i . c_m / sqrt(D)), and
+// I_rm is the mean of P_im over the members i of query cluster r.
+//
+// Fast path (bf16): one CTA per (query cluster, head) streams the cluster's
+// rows in 64-row tiles through two tensor-core passes over the key centroids:
+// pass 1 finds each row's max logit and Softmax denominator, pass 2 adds the
+// normalised probabilities into per-warp column sums.  Only the NQ x NK map is
+// written; per-query scores never reach memory (O(NQ*NK) extra memory, the
+// streamed form of PARK Appendix Table 6).  The kernel also writes a relative
+// error bound rho_r for the row of I.
+//
+// top-p: per (query cluster, head) a bitonic sort (I descending, ties: lower m
+// first) and a float64 prefix sum give the shortest prefix reaching p.  The
+// decision is certified against rho_r; a row that is not certified is
+// recomputed entirely in float64 (k_pama_f64), which also serves the float32
+// input path for every row.
+#include "kernels.h"
+#include "mma_sync.cuh"
+
+namespace park {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- PAMA (bf16)
+__global__ __launch_bounds__(128) void k_pama_mma(const uint16_t* __restrict__ Q, const int32_t* __restrict__ q_perm,
+                                                  const int32_t* __restrict__ q_off, const uint16_t* __restrict__ CK,
+                                                  const int32_t* __restrict__ k_off, const float* __restrict__ qnorm,
+                                                  const float* __restrict__ ckmax, int N, int NQ, int NK, float sl2e,
+                                                  float delta_scale, float* __restrict__ importance,
+                                                  float* __restrict__ rho) {
+    constexpr int D = 128, CH = 64, LDS = D + 8;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint16_t* Cs = reinterpret_cast<uint16_t*>(smem_raw);                       // [2][CH][LDS]
+    float* live = reinterpret_cast<float*>(smem_raw + 2 * CH * LDS * 2);        // [nch*CH] 0 or -inf
+    const int nch = (NK + CH - 1) / CH;
+    float* colsum = live + nch * CH;                                             // [4][nch*CH]
+    __shared__ float s_dmax[4];
+
+    const int r = blockIdx.x, bh = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    const int qs = q_off[(size_t)bh * (NQ + 1) + r], nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - qs;
+    float* Irow = importance + ((size_t)bh * NQ + r) * NK;
+    if (nr == 0) {
+        for (int m = threadIdx.x; m < NK; m += blockDim.x) Irow[m] = 0.f;
+        if (threadIdx.x == 0) rho[(size_t)bh * NQ + r] = 0.f;
+        return;
+    }
+    const int32_t* ko = k_off + (size_t)bh * (NK + 1);
+    for (int m = threadIdx.x; m < nch * CH; m += blockDim.x) {
+        live[m] = (m < NK && ko[m + 1] > ko[m]) ? 0.f : __int_as_float(0xff800000);
+        for (int w = 0; w < 4; ++w) colsum[w * nch * CH + m] = 0.f;
+    }
+    const uint16_t* Ch = CK + (size_t)bh * NK * D;
+    const uint16_t* Qh = Q + (size_t)bh * N * D;
+    const int32_t* pm = q_perm + (size_t)bh * N + qs;
+    const float cmax = ckmax[bh];
+    float dmax = 0.f;
+
+    auto load_chunk = [&](int c, int stg) {
+        for (int e = threadIdx.x; e < CH * 16; e += 128) {
+            int rr = e >> 4, pc = e & 15, ci = c * CH + rr;
+            cp_async16(Cs + (stg * CH + rr) * LDS + pc * 8, Ch + (size_t)(ci < NK ? ci : NK - 1) * D + pc * 8,
+                       ci < NK ? 16 : 0);
+        }
+    };
+    auto scores = [&](int stg, const uint32_t (&a)[8][4], float (&acc)[8][4]) {
+        const uint16_t* Cst = Cs + stg * CH * LDS;
+        const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[nt][j] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(b0, b1, b2, b3, Cst + (np * 16 + (mi >> 1) * 8 + rr) * LDS + kk * 16 + (mi & 1) * 8);
+                mma_bf16_16816(acc[2 * np], a[kk], b0, b1);
+                mma_bf16_16816(acc[2 * np + 1], a[kk], b2, b3);
+            }
+    };
+
+    for (int t0 = 0; t0 < nr; t0 += 64) {
+        const int lr0 = t0 + warp * 16 + g, lr1 = lr0 + 8;  // rows within the cluster
+        const bool v0 = lr0 < nr, v1 = lr1 < nr;
+        const int tok0 = v0 ? pm[lr0] : 0, tok1 = v1 ? pm[lr1] : 0;
+        uint32_t a[8][4];
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            int c0 = kk * 16 + 2 * tq;
+            a[kk][0] = v0 ? ld_u32(Qh + (size_t)tok0 * D + c0) : 0u;
+            a[kk][1] = v1 ? ld_u32(Qh + (size_t)tok1 * D + c0) : 0u;
+            a[kk][2] = v0 ? ld_u32(Qh + (size_t)tok0 * D + c0 + 8) : 0u;
+            a[kk][3] = v1 ? ld_u32(Qh + (size_t)tok1 * D + c0 + 8) : 0u;
+        }
+        if (tq == 0) {
+            if (v0) dmax = fmaxf(dmax, qnorm[(size_t)bh * N + tok0]);
+            if (v1) dmax = fmaxf(dmax, qnorm[(size_t)bh * N + tok1]);
+        }
+        // pass 1: row max and Softmax denominator (log2 domain)
+        float mrow[2] = {__int_as_float(0xff800000), __int_as_float(0xff800000)};
+        double lrow[2] = {0.0, 0.0};
+        __syncthreads();
+        load_chunk(0, 0);
+        cp_async_commit();
+        for (int c = 0; c < nch; ++c) {
+            const int stg = c & 1;
+            if (c + 1 < nch) load_chunk(c + 1, stg ^ 1);
+            cp_async_commit();
+            cp_async_wait<1>();
+            __syncthreads();
+            float acc[8][4];
+            scores(stg, a, acc);
+            float mloc[2] = {__int_as_float(0xff800000), __int_as_float(0xff800000)};
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float s = acc[nt][j] * sl2e + live[c * CH + nt * 8 + 2 * tq + (j & 1)];
+                    acc[nt][j] = s;
+                    mloc[j >> 1] = fmaxf(mloc[j >> 1], s);
+                }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], 1));
+                mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], 2));
+                float mn = fmaxf(mrow[h], mloc[h]);
+                if (mn != __int_as_float(0xff800000)) {
+                    lrow[h] *= (double)exp2f(mrow[h] - mn);
+                    mrow[h] = mn;
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) lrow[j >> 1] += (double)exp2f(acc[nt][j] - mrow[j >> 1]);
+            __syncthreads();
+        }
+        float inv[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
+            lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
+            inv[h] = (float)(1.0 / lrow[h]);
+        }
+        if (!v0) inv[0] = 0.f;
+        if (!v1) inv[1] = 0.f;
+        // pass 2: normalised probabilities summed over the tile's rows
+        load_chunk(0, 0);
+        cp_async_commit();
+        for (int c = 0; c < nch; ++c) {
+            const int stg = c & 1;
+            if (c + 1 < nch) load_chunk(c + 1, stg ^ 1);
+            cp_async_commit();
+            cp_async_wait<1>();
+            __syncthreads();
+            float acc[8][4];
+            scores(stg, a, acc);
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    int cl = nt * 8 + 2 * tq + j;
+                    float lv = live[c * CH + cl];
+                    float p0 = exp2f(acc[nt][j] * sl2e + lv - mrow[0]) * inv[0];
+                    float p1 = exp2f(acc[nt][j + 2] * sl2e + lv - mrow[1]) * inv[1];
+                    float s = p0 + p1;
+                    s += __shfl_xor_sync(0xffffffffu, s, 4);
+                    s += __shfl_xor_sync(0xffffffffu, s, 8);
+                    s += __shfl_xor_sync(0xffffffffu, s, 16);
+                    if (g == 0) colsum[warp * nch * CH + c * CH + cl] += s;
+                }
+            __syncthreads();
+        }
+    }
+    // importance row and its bound
+    dmax = warp_max(dmax);
+    if (lane == 0) s_dmax[warp] = dmax;
+    __syncthreads();
+    const float invn = 1.0f / (float)nr;
+    for (int m = threadIdx.x; m < NK; m += blockDim.x) {
+        float s = colsum[m] + colsum[nch * CH + m] + colsum[2 * nch * CH + m] + colsum[3 * nch * CH + m];
+        Irow[m] = s * invn;
+    }
+    if (threadIdx.x == 0) {
+        float qm = fmaxf(fmaxf(s_dmax[0], s_dmax[1]), fmaxf(s_dmax[2], s_dmax[3]));
+        double delta = (double)delta_scale * qm * cmax;  // logit error bound (natural log units)
+        double rr = expm1(2.0 * delta) + 1.6e-5 + (24.0 + nr / 64.0) * 1.2e-7;
+        rho[(size_t)bh * NQ + r] = (float)(rr * 1.001);
+    }
+}
+
+int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t* q_perm, const int32_t* q_off,
+                    const void* CK, const int32_t* k_off, const float* qnorm, float* importance, float* rho,
+                    float* ckmax, cudaStream_t st) {
+    const int D = 128;
+    int nch = (NK + 63) / 64;
+    size_t sm = 2 * 64 * (D + 8) * 2 + (size_t)nch * 64 * 4 * 5;
+    cudaFuncSetAttribute(k_pama_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    float scale = 1.0f / sqrtf((float)D);
+    float sl2e = scale * kLog2e;
+    // |logit~ - logit| <= s * (D 2^-23 + 2^-22) ||q|| max||c||  (tensor-core accumulation, scaling)
+    float delta_scale = (float)((1.0 / sqrt((double)D)) * ((double)D * 1.1920929e-7 * 1.01 + 2.4e-7));
+    k_pama_mma<<<dim3(NQ, BH), 128, sm, st>>>((const uint16_t*)Q, q_perm, q_off, (const uint16_t*)CK, k_off, qnorm,
+                                              ckmax, N, NQ, NK, sl2e, delta_scale, importance, rho);
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- sort helpers
+// Bitonic sort of n (power of two) (value, index) pairs: value descending,
+// ties by index ascending.  All threads of the block take part.
+template <typename V>
+__device__ void bitonic_desc(V* v, int32_t* idx, int n) {
+    for (int k = 2; k <= n; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                int ixj = i ^ j;
+                if (ixj > i) {
+                    V a = v[i], b = v[ixj];
+                    int ia = idx[i], ib = idx[ixj];
+                    bool b_first = (b > a) || (b == a && ib < ia);
+                    bool a_first = (a > b) || (a == b && ia < ib);
+                    bool up = (i & k) == 0;
+                    if (up ? b_first : a_first) {
+                        v[i] = b;
+                        v[ixj] = a;
+                        idx[i] = ib;
+                        idx[ixj] = ia;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+static int next_pow2(int x) {
+    int p = 2;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+// ---------------------------------------------------------------- top-p (certified)
+__global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importance, const float* __restrict__ rho,
+                                              const int32_t* __restrict__ q_off, const int32_t* __restrict__ k_off,
+                                              int NQ, int NK, int NKP, float p, uint8_t* __restrict__ mask,
+                                              int32_t* __restrict__ kept_cnt, int32_t* __restrict__ flag_list,
+                                              int32_t* __restrict__ flag_count) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    double* S = reinterpret_cast<double*>(smem_raw);       // [NKP] inclusive prefix sums
+    float* sv = reinterpret_cast<float*>(S + NKP);         // [NKP]
+    int32_t* si = reinterpret_cast<int32_t*>(sv + NKP);    // [NKP]
+    uint8_t* keep = reinterpret_cast<uint8_t*>(si + NKP);  // [NKP]
+    __shared__ double wsum[16];
+    __shared__ int s_cut, s_live;
+
+    const int r = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+    const size_t row = (size_t)bh * NQ + r;
+    uint8_t* mrow = mask + row * NK;
+    const int nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - q_off[(size_t)bh * (NQ + 1) + r];
+    if (nr == 0) {
+        for (int m = t; m < NK; m += blockDim.x) mrow[m] = 0;
+        if (t == 0) kept_cnt[row] = 0;
+        return;
+    }
+    const int32_t* ko = k_off + (size_t)bh * (NK + 1);
+    const float* I = importance + row * NK;
+    if (t == 0) {
+        s_cut = -1;
+        s_live = 0;
+    }
+    __syncthreads();
+    int live_local = 0;
+    for (int m = t; m < NKP; m += blockDim.x) {
+        bool lv = m < NK && ko[m + 1] > ko[m];
+        sv[m] = lv ? I[m] : -1.0f;
+        si[m] = m;
+        keep[m] = 0;
+        live_local += lv;
+    }
+    atomicAdd(&s_live, live_local);
+    __syncthreads();
+    bitonic_desc<float>(sv, si, NKP);
+    const int L = s_live;
+    // inclusive float64 prefix sums of the live sorted values
+    const int seg = NKP / blockDim.x > 0 ? NKP / blockDim.x : 1;
+    const int b0 = t * seg;
+    double loc = 0.0;
+    for (int e = b0; e < b0 + seg && e < NKP; ++e) loc += e < L ? (double)sv[e] : 0.0;
+    // block exclusive scan of loc
+    double incl = loc;
+    const int lane = t & 31, w = t >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    if (t == 0) {
+        double run = 0.0;
+        for (int q = 0; q < (int)(blockDim.x >> 5); ++q) {
+            double x = wsum[q];
+            wsum[q] = run;
+            run += x;
+        }
+    }
+    __syncthreads();
+    double run = wsum[w] + incl - loc;
+    for (int e = b0; e < b0 + seg && e < NKP; ++e) {
+        run += e < L ? (double)sv[e] : 0.0;
+        S[e] = run;
+    }
+    __syncthreads();
+    for (int e = t; e < L; e += blockDim.x)
+        if (S[e] >= (double)p && (e == 0 || S[e - 1] < (double)p)) s_cut = e;
+    __syncthreads();
+    int cut = s_cut;
+    bool ok;
+    if (p >= 1.0f) {
+        cut = L - 1;
+        ok = true;
+    } else if (cut < 0) {
+        ok = false;  // float sums fell short of p: let float64 decide
+    } else {
+        const double rh = (double)rho[row];
+        const double vc = (double)sv[cut];
+        const double eps = 1e-12;
+        bool ord = cut + 1 >= L || vc * (1.0 - rh) > (double)sv[cut + 1] * (1.0 + 2.0 * rh) + 1e-300;
+        bool hi = S[cut] * (1.0 - 2.0 * rh) - eps >= (double)p;
+        bool lo = S[cut] * (1.0 + 2.0 * rh) + eps - vc * (1.0 - rh) < (double)p;
+        ok = ord && hi && lo;
+    }
+    if (!ok) {
+        if (t == 0) {
+            int pos = atomicAdd(flag_count, 1);
+            flag_list[pos] = (int32_t)row;
+        }
+        return;
+    }
+    for (int e = t; e <= cut; e += blockDim.x) keep[si[e]] = 1;
+    __syncthreads();
+    for (int m = t; m < NK; m += blockDim.x) mrow[m] = keep[m];
+    if (t == 0) kept_cnt[row] = cut + 1;
+}
+
+int launch_topp(const float* importance, const float* rho, int BH, int NQ, int NK, const int32_t* q_off,
+                const int32_t* k_off, float p, uint8_t* mask, int32_t* kept_cnt, int32_t* flag_list,
+                int32_t* flag_count, cudaStream_t st) {
+    int NKP = next_pow2(NK);
+    if (NKP < 512) NKP = 512;
+    size_t sm = (size_t)NKP * (8 + 4 + 4 + 1) + 16;
+    cudaFuncSetAttribute(k_topp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_topp<<<dim3(NQ, BH), 512, sm, st>>>(importance, rho, q_off, k_off, NQ, NK, NKP, p, mask, kept_cnt, flag_list,
+                                          flag_count);
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- float64 PAMA + top-p
+// One CTA (256 threads) per listed (head, query cluster), or per cluster of
+// every head when all_clusters is set.  Thread t owns key clusters
+// m = t, t + 256, ...: for each member query it forms s (q . c_m) in float64,
+// the block takes the max and the sum of exp (fixed reduction tree), and the
+// thread adds P_im to its own columns.  Then I is sorted (descending, ties by
+// m) and a sequential float64 running sum finds the cut, exactly as the
+// definition reads.
+template <typename T>
+__global__ __launch_bounds__(256) void k_pama_f64(const T* __restrict__ Q, const int32_t* __restrict__ q_perm,
+                                                  const int32_t* __restrict__ q_off, const T* __restrict__ CK,
+                                                  const int32_t* __restrict__ k_off, int N, int D, int NQ, int NK,
+                                                  int NKP, double scale, float p, const int32_t* __restrict__ list,
+                                                  const int32_t* __restrict__ count_ptr, int all_clusters,
+                                                  int BHNQ, float* __restrict__ importance,
+                                                  uint8_t* __restrict__ mask, int32_t* __restrict__ kept_cnt,
+                                                  int64_t* __restrict__ counters) {
+    constexpr int MAXU = 16;  // NK <= 4096 = 16 * 256
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    double* Iv = reinterpret_cast<double*>(smem_raw);      // [NKP]
+    int32_t* si = reinterpret_cast<int32_t*>(Iv + NKP);    // [NKP]
+    double* qv = reinterpret_cast<double*>(si + NKP);      // [128]
+    __shared__ double red[8];
+    __shared__ int s_cut;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int count = all_clusters ? BHNQ : *count_ptr;
+    if (blockIdx.x == 0 && t == 0 && !all_clusters && counters)
+        atomicAdd((unsigned long long*)(counters + PARK_CNT_PAMA_RECHECK), (unsigned long long)count);
+    for (int e = blockIdx.x; e < count; e += gridDim.x) {
+        const int row = all_clusters ? e : list[e];
+        const int bh = row / NQ, r = row - bh * NQ;
+        const int qs = q_off[(size_t)bh * (NQ + 1) + r], nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - qs;
+        const int32_t* ko = k_off + (size_t)bh * (NK + 1);
+        uint8_t* mrow = mask + (size_t)row * NK;
+        float* Irow = importance + (size_t)row * NK;
+        if (nr == 0) {
+            for (int m = t; m < NK; m += blockDim.x) {
+                mrow[m] = 0;
+                Irow[m] = 0.f;
+            }
+            if (t == 0) kept_cnt[row] = 0;
+            __syncthreads();
+            continue;
+        }
+        double acc[MAXU];
+        bool lv[MAXU];
+#pragma unroll
+        for (int u = 0; u < MAXU; ++u) {
+            int m = t + 256 * u;
+            acc[u] = 0.0;
+            lv[u] = m < NK && ko[m + 1] > ko[m];
+        }
+        const T* Ch = CK + (size_t)bh * NK * D;
+        for (int i = 0; i < nr; ++i) {
+            const int tok = q_perm[(size_t)bh * N + qs + i];
+            __syncthreads();
+            if (t < D) qv[t] = Elem<T>::to_double(Q + ((size_t)bh * N + tok) * D, t);
+            __syncthreads();
+            double z[MAXU];
+            double zm = -1.0 / 0.0;
+#pragma unroll
+            for (int u = 0; u < MAXU; ++u) {
+                int m = t + 256 * u;
+                z[u] = -1.0 / 0.0;
+                if (m < NK && lv[u]) {
+                    const T* c = Ch + (size_t)m * D;
+                    double s = 0.0;
+                    for (int j = 0; j < D; ++j) s = __fma_rn(qv[j], Elem<T>::to_double(c, j), s);
+                    z[u] = scale * s;
+                    zm = fmax(zm, z[u]);
+                }
+            }
+            zm = warp_max(zm);
+            if (lane == 0) red[w] = zm;
+            __syncthreads();
+            zm = red[0];
+            for (int q = 1; q < 8; ++q) zm = fmax(zm, red[q]);
+            __syncthreads();
+            double ls = 0.0;
+#pragma unroll
+            for (int u = 0; u < MAXU; ++u) {
+                z[u] = (t + 256 * u < NK && lv[u]) ? exp(z[u] - zm) : 0.0;
+                ls += z[u];
+            }
+            ls = warp_sum(ls);
+            if (lane == 0) red[w] = ls;
+            __syncthreads();
+            ls = 0.0;
+            for (int q = 0; q < 8; ++q) ls += red[q];
+#pragma unroll
+            for (int u = 0; u < MAXU; ++u) acc[u] += z[u] / ls;
+        }
+        // I row, then sort and cut
+        for (int m = t; m < NKP; m += blockDim.x) {
+            si[m] = m;
+            Iv[m] = -1.0;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < MAXU; ++u) {
+            int m = t + 256 * u;
+            if (m < NK) {
+                double iv = acc[u] / (double)nr;
+                Irow[m] = lv[u] ? (float)iv : 0.f;
+                if (lv[u]) Iv[m] = iv;
+            }
+        }
+        __syncthreads();
+        bitonic_desc<double>(Iv, si, NKP);
+        if (t == 0) {
+            double run = 0.0;
+            int cut = -1;
+            for (int q = 0; q < NKP && Iv[q] >= 0.0; ++q) {
+                cut = q;
+                run += Iv[q];
+                if (p < 1.0f && run >= (double)p) break;
+            }
+            s_cut = cut;
+        }
+        __syncthreads();
+        const int cut = s_cut;
+        for (int m = t; m < NK; m += blockDim.x) mrow[m] = 0;
+        __syncthreads();
+        for (int q = t; q <= cut; q += blockDim.x) mrow[si[q]] = 1;
+        if (t == 0) kept_cnt[row] = cut + 1;
+        __syncthreads();
+    }
+}
+
+int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int NK, const int32_t* q_perm,
+                    const int32_t* q_off, const void* CK, const int32_t* k_off, float p, const int32_t* list,
+                    const int32_t* count, int all_clusters, int num_sms, float* importance, uint8_t* mask,
+                    int32_t* kept_cnt, int64_t* counters, cudaStream_t st) {
+    if (NK > 4096 || D > 128) return PARK_ERR_UNSUPPORTED;
+    int NKP = next_pow2(NK);
+    size_t sm = (size_t)NKP * 12 + 128 * 8;
+    int blocks = num_sms * 4;
+    double scale = 1.0 / sqrt((double)D);
+    if (dtype == PARK_BF16) {
+        cudaFuncSetAttribute(k_pama_f64<bf16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        k_pama_f64<bf16_t><<<blocks, 256, sm, st>>>((const bf16_t*)Q, q_perm, q_off, (const bf16_t*)CK, k_off, N, D,
+                                                    NQ, NK, NKP, scale, p, list, count, all_clusters, BH * NQ,
+                                                    importance, mask, kept_cnt, counters);
+    } else {
+        cudaFuncSetAttribute(k_pama_f64<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        k_pama_f64<float><<<blocks, 256, sm, st>>>((const float*)Q, q_perm, q_off, (const float*)CK, k_off, N, D, NQ,
+                                                   NK, NKP, scale, p, list, count, all_clusters, BH * NQ, importance,
+                                                   mask, kept_cnt, counters);
+    }
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- kept-block CSR
+__global__ __launch_bounds__(1024) void k_kept_scan(const int32_t* __restrict__ cnt, int NQ,
+                                                    int32_t* __restrict__ ptr, int64_t* __restrict__ counters) {
+    __shared__ int wsum[32];
+    const int bh = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int seg = (NQ + 1023) / 1024, b0 = t * seg;
+    const int32_t* c = cnt + (size_t)bh * NQ;
+    int loc = 0;
+    for (int e = b0; e < b0 + seg && e < NQ; ++e) loc += c[e];
+    int incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int x = wsum[lane], xi = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, xi, o);
+            if (lane >= o) xi += y;
+        }
+        wsum[lane] = xi - x;
+    }
+    __syncthreads();
+    int run = wsum[w] + incl - loc;
+    int32_t* pr = ptr + (size_t)bh * (NQ + 1);
+    for (int e = b0; e < b0 + seg && e < NQ; ++e) {
+        pr[e] = run;
+        run += c[e];
+    }
+    if (b0 < NQ && b0 + seg >= NQ) {
+        pr[NQ] = run;
+        if (counters) atomicAdd((unsigned long long*)(counters + PARK_CNT_KEPT_BLOCKS), (unsigned long long)run);
+    }
+}
+
+__global__ __launch_bounds__(256) void k_kept_compact(const uint8_t* __restrict__ mask, const int32_t* __restrict__ ptr,
+                                                      int NQ, int NK, int32_t* __restrict__ idx) {
+    __shared__ int wcnt[8];
+    const int r = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const uint8_t* mrow = mask + ((size_t)bh * NQ + r) * NK;
+    int32_t* out = idx + (size_t)bh * NQ * NK + ptr[(size_t)bh * (NQ + 1) + r];
+    int base = 0;
+    for (int m0 = 0; m0 < NK; m0 += 256) {
+        int m = m0 + t;
+        bool f = m < NK && mrow[m];
+        unsigned bal = __ballot_sync(0xffffffffu, f);
+        if (lane == 0) wcnt[w] = __popc(bal);
+        __syncthreads();
+        int off = base;
+        for (int q = 0; q < w; ++q) off += wcnt[q];
+        if (f) out[off + __popc(bal & ((1u << lane) - 1u))] = m;
+        int tot = 0;
+        for (int q = 0; q < 8; ++q) tot += wcnt[q];
+        base += tot;
+        __syncthreads();
+    }
+}
+
+int launch_kept_csr(const uint8_t* mask, const int32_t* kept_cnt, int BH, int NQ, int NK, int32_t* kept_ptr,
+                    int32_t* kept_idx, int64_t* counters, cudaStream_t st) {
+    k_kept_scan<<<BH, 1024, 0, st>>>(kept_cnt, NQ, kept_ptr, counters);
+    PARK_TRY_LAUNCH();
+    k_kept_compact<<<dim3(NQ, BH), 256, 0, st>>>(mask, kept_ptr, NQ, NK, kept_idx);
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+}  // namespace park

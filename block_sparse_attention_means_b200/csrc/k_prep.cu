@@ -1,0 +1,254 @@
+// Input check, QRKC metric, row norms, strided K-means initialisation and
+// per-iteration centroid operands.
+#include "kernels.h"
+
+namespace park {
+
+// ---------------------------------------------------------------- input check
+// One pass over the tensor with 16-byte loads: every element must be 0 or a
+// finite value with 2^-20 <= |x| < 2^16 (the library's range precondition).
+template <int BYTES>
+__global__ void k_input_check(const uint4* __restrict__ x, size_t n16, int32_t* status) {
+    size_t stride = (size_t)gridDim.x * blockDim.x;
+    bool bad = false;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += stride) {
+        uint4 v = x[i];
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (BYTES == 2) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t b = (w[q] >> (16 * h)) & 0xFFFFu;
+                    uint32_t mag = b & 0x7FFFu;
+                    int e = (b >> 7) & 0xFF;
+                    bad |= !in_range_exp(e, mag);
+                }
+            } else {
+                uint32_t mag = w[q] & 0x7FFFFFFFu;
+                int e = (w[q] >> 23) & 0xFF;
+                bad |= !in_range_exp(e, mag);
+            }
+        }
+    }
+    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) set_status(status, PARK_ERR_RANGE);
+}
+
+int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status, cudaStream_t st) {
+    int eb = dtype == PARK_BF16 ? 2 : 4;
+    size_t n16 = n_elems * eb / 16;
+    int blocks = (int)((n16 + 255) / 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    if (eb == 2)
+        k_input_check<2><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status);
+    else
+        k_input_check<4><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status);
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- metric
+// M = (1/N) sum_i q_i q_i^T in float64.  Pass 1: grid (chunks, BH); each CTA
+// sums the outer products of its row chunk.  Thread t owns entries
+// (a = t/16 + 16u, b = t%16 + 16v).  Entries (a,b) and (b,a) see the same
+// products in the same order, so M is exactly symmetric.  Pass 2 adds the
+// chunk partials in chunk order and divides by N.
+template <typename T>
+__global__ __launch_bounds__(256) void k_metric_partial(const T* __restrict__ Q, int N, int D, int rows_per_chunk,
+                                                        double* __restrict__ part) {
+    constexpr int RB = 32;
+    extern __shared__ double qs[];  // [RB][D]
+    int bh = blockIdx.y, c = blockIdx.x, nch = gridDim.x;
+    const T* X = Q + (size_t)bh * N * D;
+    int r0 = c * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
+    int t = threadIdx.x, ta = t >> 4, tb = t & 15;
+    double acc[8][8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[u][v] = 0.0;
+    for (int base = r0; base < r1; base += RB) {
+        int nr = min(RB, r1 - base);
+        for (int e = t; e < RB * D; e += 256) {
+            int rr = e / D, jj = e - rr * D;
+            qs[e] = rr < nr ? Elem<T>::to_double(X + (size_t)(base + rr) * D, jj) : 0.0;
+        }
+        __syncthreads();
+        for (int rr = 0; rr < nr; ++rr) {
+            const double* q = qs + rr * D;
+            double qa[8], qb[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                int a = ta + 16 * u, b = tb + 16 * u;
+                qa[u] = a < D ? q[a] : 0.0;
+                qb[u] = b < D ? q[b] : 0.0;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                for (int v = 0; v < 8; ++v) acc[u][v] = __fma_rn(qa[u], qb[v], acc[u][v]);
+        }
+        __syncthreads();
+    }
+    double* P = part + ((size_t)bh * nch + c) * D * D;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            int a = ta + 16 * u, b = tb + 16 * v;
+            if (a < D && b < D) P[a * D + b] = acc[u][v];
+        }
+}
+
+__global__ void k_metric_reduce(const double* __restrict__ part, int nch, int N, int D, double* __restrict__ M,
+                                double* __restrict__ M_out) {
+    int bh = blockIdx.y;
+    int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= D * D) return;
+    double s = 0.0;
+    for (int c = 0; c < nch; ++c) s += part[((size_t)bh * nch + c) * D * D + e];
+    double m = s / (double)N;
+    M[(size_t)bh * D * D + e] = m;
+    if (M_out) M_out[(size_t)bh * D * D + e] = m;
+}
+
+int launch_metric(const void* Q, int dtype, int BH, int N, int D, double* part, int nchunks, double* M,
+                  double* M_out, cudaStream_t st) {
+    int rpc = (N + nchunks - 1) / nchunks;
+    dim3 g1(nchunks, BH);
+    size_t sm = 32 * D * sizeof(double);
+    if (dtype == PARK_BF16)
+        k_metric_partial<bf16_t><<<g1, 256, sm, st>>>((const bf16_t*)Q, N, D, rpc, part);
+    else
+        k_metric_partial<float><<<g1, 256, sm, st>>>((const float*)Q, N, D, rpc, part);
+    PARK_TRY_LAUNCH();
+    dim3 g2((D * D + 255) / 256, BH);
+    k_metric_reduce<<<g2, 256, 0, st>>>(part, nchunks, N, D, M, M_out);
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- row norms
+// ||x_i|| (float64 sum of squares, square root rounded up to float): one warp
+// per row.  Used only inside the certified score bound.
+template <typename T>
+__global__ void k_row_norms(const T* __restrict__ X, size_t rows, int D, float* __restrict__ out) {
+    size_t w = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    int lane = threadIdx.x & 31;
+    if (w >= rows) return;
+    const T* x = X + w * D;
+    double s = 0.0;
+    for (int j = lane; j < D; j += 32) {
+        double v = Elem<T>::to_double(x, j);
+        s += v * v;
+    }
+    s = warp_sum(s);
+    if (lane == 0) out[w] = round_up_f(__double2float_ru(sqrt(s)));
+}
+
+int launch_row_norms(const void* X, int dtype, int BH, int N, int D, float* xnorm, cudaStream_t st) {
+    size_t rows = (size_t)BH * N;
+    int blocks = (int)((rows * 32 + 255) / 256);
+    if (dtype == PARK_BF16)
+        k_row_norms<bf16_t><<<blocks, 256, 0, st>>>((const bf16_t*)X, rows, D, xnorm);
+    else
+        k_row_norms<float><<<blocks, 256, 0, st>>>((const float*)X, rows, D, xnorm);
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- strided init
+// c_k = x_floor(k N / K) (pages silent on initialisation; deterministic choice).
+__global__ void k_strided_init(const uint8_t* __restrict__ X, int N, int K, int row_bytes, uint8_t* __restrict__ C) {
+    int k = blockIdx.x, bh = blockIdx.y;
+    long long src = ((long long)k * N) / K;
+    const uint8_t* s = X + ((size_t)bh * N + src) * row_bytes;
+    uint8_t* d = C + ((size_t)bh * K + k) * row_bytes;
+    for (int b = threadIdx.x * 4; b < row_bytes; b += blockDim.x * 4)
+        *(uint32_t*)(d + b) = *(const uint32_t*)(s + b);
+}
+
+int launch_strided_init(const void* X, int dtype, int BH, int N, int D, int K, void* C, cudaStream_t st) {
+    int rb = D * (dtype == PARK_BF16 ? 2 : 4);
+    k_strided_init<<<dim3(K, BH), 64, 0, st>>>((const uint8_t*)X, N, K, rb, (uint8_t*)C);
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- centroid operands
+// Per centroid: bias = ||c||^2 (Euclidean) or c^T M c with w = M c (QRKC),
+// w split as bf16 hi + lo (|w - hi - lo| <= 2^-16 |w|) for the score GEMM,
+// and the per-head maxima ||w|| and |bias| used by the certified bound.
+// One CTA of D threads per (centroid, head); float64 sums in a fixed tree.
+template <typename T, bool METRIC>
+__global__ void k_centroid_prep(const T* __restrict__ C, int K, int D, const double* __restrict__ Mall,
+                                uint16_t* __restrict__ wop, float* __restrict__ bias32,
+                                double* __restrict__ bias64, double* __restrict__ w64, float* __restrict__ wmax,
+                                float* __restrict__ bmax) {
+    __shared__ double cs[128];
+    __shared__ double red[2][128];
+    int k = blockIdx.x, bh = blockIdx.y, a = threadIdx.x;
+    const T* c = C + ((size_t)bh * K + k) * D;
+    double ca = Elem<T>::to_double(c, a);
+    cs[a] = ca;
+    __syncthreads();
+    double wa = ca;
+    if (METRIC) {
+        const double* M = Mall + (size_t)bh * D * D + (size_t)a * D;
+        double s = 0.0;
+        for (int b = 0; b < D; ++b) s = __fma_rn(M[b], cs[b], s);
+        wa = s;
+        w64[((size_t)bh * K + k) * D + a] = wa;
+        if (wop != nullptr) {
+            uint16_t hi = double_to_bf16_bits(wa);
+            double hid = (double)__uint_as_float(((uint32_t)hi) << 16);
+            uint16_t lo = double_to_bf16_bits(wa - hid);  // wa - hid is exact
+            wop[((size_t)bh * K + k) * (2 * D) + a] = hi;
+            wop[((size_t)bh * K + k) * (2 * D) + D + a] = lo;
+        }
+    }
+    red[0][a] = ca * wa;
+    red[1][a] = wa * wa;
+    __syncthreads();
+    for (int s = 64; s > 0; s >>= 1) {
+        if (a < s && a + s < D) {
+            red[0][a] += red[0][a + s];
+            red[1][a] += red[1][a + s];
+        }
+        __syncthreads();
+    }
+    if (a == 0) {
+        double b = red[0][0];
+        bias64[(size_t)bh * K + k] = b;
+        bias32[(size_t)bh * K + k] = __double2float_rn(b);
+        atomic_max_nonneg(wmax + bh, round_up_f(__double2float_ru(sqrt(red[1][0]))));
+        atomic_max_nonneg(bmax + bh, round_up_f(__double2float_ru(fabs(b))));
+    }
+}
+
+int launch_centroid_prep(const void* C, int dtype, int BH, int K, int D, const double* M, CentroidOps ops,
+                         cudaStream_t st) {
+    if (D > 128) return PARK_ERR_UNSUPPORTED;  // one thread per coordinate
+    dim3 g(K, BH);
+    bool metric = M != nullptr;
+    if (dtype == PARK_BF16) {
+        if (metric)
+            k_centroid_prep<bf16_t, true><<<g, D, 0, st>>>((const bf16_t*)C, K, D, M, (uint16_t*)ops.w, ops.bias32,
+                                                          ops.bias64, ops.w64, ops.wmax, ops.bmax);
+        else
+            k_centroid_prep<bf16_t, false><<<g, D, 0, st>>>((const bf16_t*)C, K, D, M, nullptr, ops.bias32,
+                                                           ops.bias64, ops.w64, ops.wmax, ops.bmax);
+    } else {
+        if (metric)
+            k_centroid_prep<float, true><<<g, D, 0, st>>>((const float*)C, K, D, M, (uint16_t*)ops.w, ops.bias32,
+                                                         ops.bias64, ops.w64, ops.wmax, ops.bmax);
+        else
+            k_centroid_prep<float, false><<<g, D, 0, st>>>((const float*)C, K, D, M, nullptr, ops.bias32,
+                                                          ops.bias64, ops.w64, ops.wmax, ops.bmax);
+    }
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+}  // namespace park

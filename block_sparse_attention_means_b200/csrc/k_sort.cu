@@ -1,0 +1,221 @@
+// Stable counting sort of tokens by cluster label (perm, offsets) and the
+// exact K-means centroid update.
+//
+// Sort: tokens are split into chunks of 1024.  (1) per-chunk label histogram
+// in shared memory; (2) one CTA per head turns the [label][chunk] table into
+// exclusive start positions (label-major, so clusters are contiguous and
+// chunks keep token order); (3) each chunk ranks its tokens among equal labels
+// in token order (warp match + warps in sequence) and scatters them.  The
+// result equals a stable argsort of the labels.
+//
+// Update: one CTA per (cluster, head) sums its members' rows exactly in fixed
+// point (x * 2^27 for bf16, x * 2^43 for float32 inputs; integer sums are exact
+// and independent of order), converts the exact sum to float64 with one
+// correct rounding, divides by the member count in IEEE float64 and rounds to
+// the storage dtype (nearest, ties to even).  Empty clusters keep their
+// centroid.
+#include "kernels.h"
+
+namespace park {
+
+constexpr int SORT_CHUNK = 1024;
+
+__global__ void k_label_hist(const int32_t* __restrict__ labels, int N, int K, int nchunks,
+                             int32_t* __restrict__ hist) {
+    extern __shared__ int32_t cnt[];
+    int c = blockIdx.x, bh = blockIdx.y;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) cnt[k] = 0;
+    __syncthreads();
+    int i0 = c * SORT_CHUNK, i1 = min(N, i0 + SORT_CHUNK);
+    const int32_t* lab = labels + (size_t)bh * N;
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) atomicAdd(&cnt[lab[i]], 1);
+    __syncthreads();
+    int32_t* h = hist + (size_t)bh * K * nchunks;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) h[(size_t)k * nchunks + c] = cnt[k];
+}
+
+// Exclusive scan of hist[bh] (K * nchunks entries) in place; offsets[k] = start
+// of cluster k, offsets[K] = N.  1024 threads, each owns a contiguous segment.
+__global__ __launch_bounds__(1024) void k_label_scan(int32_t* __restrict__ hist, int N, int K, int nchunks,
+                                                     int32_t* __restrict__ offsets) {
+    __shared__ int32_t wsum[32];
+    int bh = blockIdx.x, t = threadIdx.x;
+    int total = K * nchunks;
+    int seg = (total + 1023) / 1024;
+    int32_t* h = hist + (size_t)bh * total;
+    int b0 = t * seg, b1 = min(total, b0 + seg);
+    int s = 0;
+    for (int e = b0; e < b1; ++e) s += h[e];
+    // block exclusive scan of s
+    int lane = t & 31, w = t >> 5;
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int x = wsum[lane];
+        int xi = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, xi, o);
+            if (lane >= o) xi += y;
+        }
+        wsum[lane] = xi - x;  // exclusive warp offsets
+    }
+    __syncthreads();
+    int run = wsum[w] + incl - s;
+    for (int e = b0; e < b1; ++e) {
+        int v = h[e];
+        h[e] = run;
+        if (e % nchunks == 0) offsets[(size_t)bh * (K + 1) + e / nchunks] = run;
+        run += v;
+    }
+    if (t == 0) offsets[(size_t)bh * (K + 1) + K] = N;
+}
+
+__global__ __launch_bounds__(1024) void k_label_scatter(const int32_t* __restrict__ labels, int N, int K,
+                                                        int nchunks, const int32_t* __restrict__ hist,
+                                                        int32_t* __restrict__ perm) {
+    extern __shared__ int32_t run[];  // [K] tokens already placed per label in this chunk
+    int c = blockIdx.x, bh = blockIdx.y;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) run[k] = 0;
+    __syncthreads();
+    int i = c * SORT_CHUNK + threadIdx.x;
+    bool valid = i < N;
+    int lab = valid ? labels[(size_t)bh * N + i] : -1;
+    int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned peers = __match_any_sync(0xffffffffu, lab);
+    unsigned lower = peers & ((1u << lane) - 1u);
+    int rank = __popc(lower);
+    bool leader = lower == 0u;
+    int pos = 0;
+    for (int w = 0; w < 32; ++w) {
+        if (warp == w) {
+            int base = valid ? run[lab] : 0;
+            __syncwarp();
+            if (valid && leader) run[lab] = base + __popc(peers);
+            if (valid) pos = hist[((size_t)bh * K + lab) * nchunks + c] + base + rank;
+        }
+        __syncthreads();
+    }
+    if (valid) perm[(size_t)bh * N + pos] = i;
+}
+
+int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist, int nchunks, int32_t* perm,
+                      int32_t* offsets, cudaStream_t st) {
+    size_t sm = (size_t)K * sizeof(int32_t);
+    if (sm > 48 * 1024) {
+        cudaFuncSetAttribute(k_label_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        cudaFuncSetAttribute(k_label_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    }
+    dim3 g(nchunks, BH);
+    k_label_hist<<<g, 256, sm, st>>>(labels, N, K, nchunks, hist);
+    PARK_TRY_LAUNCH();
+    k_label_scan<<<BH, 1024, 0, st>>>(hist, N, K, nchunks, offsets);
+    PARK_TRY_LAUNCH();
+    k_label_scatter<<<g, 1024, sm, st>>>(labels, N, K, nchunks, hist, perm);
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- update
+// 128 threads.  Each thread owns one 16-byte piece of a row: VEC elements at
+// piece p = t % CPR, and rows s, s + RPI, ... of the cluster (s = t / CPR).
+template <typename T>
+__global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const int32_t* __restrict__ perm,
+                                                const int32_t* __restrict__ offsets, int N, int D, int K,
+                                                T* __restrict__ C) {
+    constexpr int VEC = 16 / sizeof(T);
+    constexpr bool TWO_LIMBS = sizeof(T) == 4;
+    extern __shared__ long long red[];  // [RPI][D] (x2 for two limbs)
+    int k = blockIdx.x, bh = blockIdx.y;
+    const int32_t* off = offsets + (size_t)bh * (K + 1);
+    int start = off[k], n = off[k + 1] - start;
+    if (n == 0) return;  // empty cluster keeps its centroid
+    const int CPR = D / VEC, RPI = 128 / CPR;
+    int t = threadIdx.x, piece = t % CPR, slot = t / CPR;
+    long long acc_hi[VEC];
+    unsigned long long acc_lo[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        acc_hi[e] = 0;
+        acc_lo[e] = 0;
+    }
+    const int32_t* pm = perm + (size_t)bh * N + start;
+    const T* Xh = X + (size_t)bh * N * D;
+    if (slot < RPI) {
+        for (int j = slot; j < n; j += RPI) {
+            int tok = pm[j];
+            uint4 v = *reinterpret_cast<const uint4*>(Xh + (size_t)tok * D + piece * VEC);
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            if (!TWO_LIMBS) {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc_hi[e] += fixed_bf16((uint16_t)(w[e >> 1] >> (16 * (e & 1))));
+            } else {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    long long f = fixed_f32(w[e]);
+                    acc_lo[e] += (unsigned long long)(f & 0xFFFFFFFFll);
+                    acc_hi[e] += f >> 32;
+                }
+            }
+        }
+    }
+    long long* red_hi = red;
+    long long* red_lo = red + RPI * D;
+    if (slot < RPI) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            red_hi[slot * D + piece * VEC + e] = acc_hi[e];
+            if (TWO_LIMBS) red_lo[slot * D + piece * VEC + e] = (long long)acc_lo[e];
+        }
+    }
+    __syncthreads();
+    if (t < D) {
+        double mean;
+        if (!TWO_LIMBS) {
+            long long s = 0;
+            for (int q = 0; q < RPI; ++q) s += red_hi[q * D + t];
+            mean = ldexp(__ll2double_rn(s), -Elem<T>::frac_bits) / (double)n;
+        } else {
+            long long sh = 0;
+            unsigned long long sl = 0;
+            for (int q = 0; q < RPI; ++q) {
+                sh += red_hi[q * D + t];
+                sl += (unsigned long long)red_lo[q * D + t];
+            }
+            // exact value = sh * 2^32 + sl (sl < 2^52, |sh| < 2^48): form it in 128 bits
+            __int128 v = ((__int128)sh << 32) + (__int128)sl;
+            long long hi = (long long)(v >> 64);
+            unsigned long long lo = (unsigned long long)v;
+            mean = ldexp(i128_to_double_rn(hi, lo), -Elem<T>::frac_bits) / (double)n;
+        }
+        T* c = C + ((size_t)bh * K + k) * D + t;
+        if (sizeof(T) == 2)
+            reinterpret_cast<uint16_t*>(c)[0] = double_to_bf16_bits(mean);
+        else
+            reinterpret_cast<float*>(c)[0] = __double2float_rn(mean);
+    }
+}
+
+int launch_update(const void* X, int dtype, int BH, int N, int D, int K, const int32_t* perm,
+                  const int32_t* offsets, void* C, cudaStream_t st) {
+    dim3 g(K, BH);
+    if (dtype == PARK_BF16) {
+        if (D % 8 || D / 8 > 128) return PARK_ERR_UNSUPPORTED;
+        int rpi = 128 / (D / 8);
+        k_update<bf16_t><<<g, 128, (size_t)rpi * D * 8, st>>>((const bf16_t*)X, perm, offsets, N, D, K, (bf16_t*)C);
+    } else {
+        if (D % 4 || D / 4 > 128) return PARK_ERR_UNSUPPORTED;
+        int rpi = 128 / (D / 4);
+        k_update<float><<<g, 128, (size_t)rpi * D * 16, st>>>((const float*)X, perm, offsets, N, D, K, (float*)C);
+    }
+    PARK_TRY_LAUNCH();
+    return PARK_OK;
+}
+
+}  // namespace park

@@ -1,0 +1,85 @@
+// Internal launch interface between the C ABI (park_api.cu) and the kernels.
+// Every launcher enqueues on `st`, never synchronises, and returns a PARK_*
+// code (PARK_ERR_CUDA when the launch itself failed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace park {
+
+// K-means centroid operands for the score GEMM: score_k = bias_k - 2 x . w_k.
+struct CentroidOps {
+    const uint16_t* w;  // bf16 [BH][K][kw]   (queries: the centroids themselves, kw = D;
+                        //                     keys: hi/lo split of M c, kw = 2D)
+    int kw;
+    float* bias32;      // [BH][K]  bias rounded to float
+    double* bias64;     // [BH][K]  ||c||^2 (queries) or c^T M c (keys)
+    double* w64;        // [BH][K][D] M c in float64 (keys only)
+    float* wmax;        // [BH] max_k ||w_k||  (rounded up)
+    float* bmax;        // [BH] max_k |bias_k| (rounded up)
+};
+
+struct Lists {
+    int32_t* pair_row;   // [BH*N] bh*N + i of rows whose winner is one of two candidates
+    int32_t* pair_cand;  // [BH*N] the second candidate
+    int32_t* full_row;   // [BH*N] rows rescored against every centroid
+    int32_t* counts;     // [4]: pair count, full count, (spare)
+};
+
+// ---- k_prep.cu
+int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status, cudaStream_t st);
+int launch_metric(const void* Q, int dtype, int BH, int N, int D, double* part, int nchunks, double* M,
+                  double* M_out, cudaStream_t st);
+int launch_row_norms(const void* X, int dtype, int BH, int N, int D, float* xnorm, cudaStream_t st);
+int launch_strided_init(const void* X, int dtype, int BH, int N, int D, int K, void* C, cudaStream_t st);
+int launch_centroid_prep(const void* C, int dtype, int BH, int K, int D, const double* M, CentroidOps ops,
+                         cudaStream_t st);
+
+// ---- k_assign.cu
+int launch_assign_mma(const void* X, int BH, int N, int K, const CentroidOps& ops, const float* xnorm,
+                      float gamma, int32_t* labels, Lists lists, cudaStream_t st);
+int launch_recheck(const void* X, int dtype, int BH, int N, int D, int K, const void* C, const double* w64,
+                   const double* b64, int32_t* labels, Lists lists, int all_rows, int num_sms,
+                   int64_t* counters, int cnt_slot, cudaStream_t st);
+
+// ---- k_sort.cu
+int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist, int nchunks, int32_t* perm,
+                      int32_t* offsets, cudaStream_t st);
+int launch_update(const void* X, int dtype, int BH, int N, int D, int K, const int32_t* perm,
+                  const int32_t* offsets, void* C, cudaStream_t st);
+
+// ---- k_pama.cu
+int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t* q_perm, const int32_t* q_off,
+                    const void* CK, const int32_t* k_off, const float* qnorm, float* importance, float* rho,
+                    float* ckmax, cudaStream_t st);
+int launch_topp(const float* importance, const float* rho, int BH, int NQ, int NK, const int32_t* q_off,
+                const int32_t* k_off, float p, uint8_t* mask, int32_t* kept_cnt, int32_t* flag_list,
+                int32_t* flag_count, cudaStream_t st);
+int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int NK, const int32_t* q_perm,
+                    const int32_t* q_off, const void* CK, const int32_t* k_off, float p, const int32_t* list,
+                    const int32_t* count, int all_clusters, int num_sms, float* importance, uint8_t* mask,
+                    int32_t* kept_cnt, int64_t* counters, cudaStream_t st);
+int launch_kept_csr(const uint8_t* mask, const int32_t* kept_cnt, int BH, int NQ, int NK, int32_t* kept_ptr,
+                    int32_t* kept_idx, int64_t* counters, cudaStream_t st);
+
+// ---- k_attn.cu
+struct WorkItem {
+    int bh, r, q_start, rows;
+};
+int launch_gather(const void* X, int dtype, int BH, int N, int D, const int32_t* perm, void* Xp, cudaStream_t st);
+int launch_attn_schedule(int BH, int NQ, int NK, const int32_t* q_off, const int32_t* k_off,
+                         const int32_t* kept_ptr, const int32_t* kept_idx, int32_t* kv_pre, int32_t* kv_len,
+                         WorkItem* items, int32_t* item_count, int64_t* counters, int tile_rows, cudaStream_t st);
+int launch_sparse_attn_mma(const void* Qp, const void* Kp, const void* Vp, int BH, int N, int NQ, int NK,
+                           const int32_t* q_perm, const int32_t* k_off, const int32_t* kept_ptr,
+                           const int32_t* kept_idx, const int32_t* kv_pre, const int32_t* kv_len,
+                           const WorkItem* items, const int32_t* item_count, int32_t* work_counter, void* O,
+                           int num_sms, cudaStream_t st);
+int launch_sparse_attn_simt(const void* Q, const void* K, const void* V, int dtype, int BH, int N, int D, int NQ,
+                            int NK, const int32_t* q_labels, const int32_t* k_perm, const int32_t* k_off,
+                            const int32_t* kept_ptr, const int32_t* kept_idx, void* O, cudaStream_t st);
+
+}  // namespace park

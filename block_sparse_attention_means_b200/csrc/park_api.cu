@@ -1,0 +1,363 @@
+// C ABI of libpark: argument validation, workspace carving and the launch
+// sequence of park_retrieve / park_sparse_attn / park_layer.  Nothing here
+// allocates or synchronises; every step is a kernel on the caller's stream.
+#include <atomic>
+#include <cmath>
+
+#include "kernels.h"
+
+namespace park {
+
+static std::atomic<unsigned long long> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+namespace {
+
+struct Dims {
+    int B, H, N, D, dtype, BH, elt;
+};
+
+int check_shape(const park_shape* s, int NQ, int NK, Dims* d) {
+    if (!s) return PARK_ERR_INVALID_ARG;
+    if (s->B < 1 || s->H < 1 || s->T < 0 || s->Hg < 0 || s->W < 0 || s->n_text < 0 || s->D < 1)
+        return PARK_ERR_INVALID_ARG;
+    long long nv = (long long)s->T * s->Hg * s->W;
+    long long N = nv + s->n_text;
+    if (N < 1 || N > (1ll << 20)) return N < 1 ? PARK_ERR_INVALID_ARG : PARK_ERR_UNSUPPORTED;
+    long long BH = (long long)s->B * s->H;
+    if (BH * N >= (1ll << 31) || BH > 65535) return PARK_ERR_UNSUPPORTED;
+    if (NQ < 1 || NK < 1 || NQ > N || NK > N) return PARK_ERR_INVALID_ARG;
+    if (NK > 4096 || NQ > 65536) return PARK_ERR_UNSUPPORTED;
+    if (s->dtype == PARK_BF16) {
+        if (s->D != 128) return PARK_ERR_UNSUPPORTED;
+    } else if (s->dtype == PARK_F32) {
+        if (s->D % 32 != 0 || s->D > 128) return PARK_ERR_UNSUPPORTED;
+    } else {
+        return PARK_ERR_INVALID_ARG;
+    }
+    d->B = s->B;
+    d->H = s->H;
+    d->N = (int)N;
+    d->D = s->D;
+    d->dtype = s->dtype;
+    d->BH = (int)BH;
+    d->elt = s->dtype == PARK_BF16 ? 2 : 4;
+    return PARK_OK;
+}
+
+struct Carver {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        size_t o = off;
+        off = align_up(off + (bytes ? bytes : 1), 256);
+        return o;
+    }
+};
+
+constexpr int kSortChunk = 1024;
+constexpr int kAttnTile = 64;
+
+int metric_chunks(const Dims& d) {
+    int c = (2 * 148 + d.BH - 1) / d.BH;
+    int cap = (d.N + 255) / 256;
+    if (c > cap) c = cap;
+    if (c > 64) c = 64;
+    return c < 1 ? 1 : c;
+}
+
+struct RetrievalWs {
+    size_t M, Mpart, xnorm_q, xnorm_k, wop, b32, b64, w64, wmax, bmax, lpair, lcand, lfull, lcnt, hist, rho, plist,
+        pcnt, kcnt, total;
+};
+
+RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
+    RetrievalWs w;
+    Carver c;
+    size_t BH = d.BH, N = d.N, D = d.D, Km = NQ > NK ? NQ : NK;
+    size_t nchunks = (N + kSortChunk - 1) / kSortChunk;
+    w.M = c.take(BH * D * D * 8);
+    w.Mpart = c.take(BH * metric_chunks(d) * D * D * 8);
+    w.xnorm_q = c.take(BH * N * 4);
+    w.xnorm_k = c.take(BH * N * 4);
+    w.wop = c.take(BH * Km * 2 * D * 2);
+    w.b32 = c.take(BH * Km * 4);
+    w.b64 = c.take(BH * Km * 8);
+    w.w64 = c.take(BH * Km * D * 8);
+    w.wmax = c.take(BH * 4);
+    w.bmax = c.take(BH * 4);
+    w.lpair = c.take(BH * N * 4);
+    w.lcand = c.take(BH * N * 4);
+    w.lfull = c.take(BH * N * 4);
+    w.lcnt = c.take(16 * 4);
+    w.hist = c.take(BH * Km * nchunks * 4);
+    w.rho = c.take(BH * NQ * 4);
+    w.plist = c.take(BH * NQ * 4);
+    w.pcnt = c.take(16 * 4);
+    w.kcnt = c.take(BH * NQ * 4);
+    w.total = c.off;
+    return w;
+}
+
+struct AttnWs {
+    size_t Qp, Kp, Vp, items, icnt, kvpre, kvlen, total;
+};
+
+AttnWs plan_attn(const Dims& d, int NQ, int NK) {
+    AttnWs w;
+    Carver c;
+    size_t BH = d.BH, N = d.N, D = d.D;
+    size_t rowbytes = D * d.elt;
+    if (d.dtype == PARK_BF16) {
+        w.Qp = c.take(BH * N * rowbytes);
+        w.Kp = c.take(BH * N * rowbytes);
+        w.Vp = c.take(BH * N * rowbytes);
+    } else {
+        w.Qp = w.Kp = w.Vp = 0;
+    }
+    size_t max_items = BH * ((N + kAttnTile - 1) / kAttnTile + (size_t)NQ);
+    w.items = c.take(max_items * sizeof(WorkItem));
+    w.icnt = c.take(16 * 4);
+    w.kvpre = c.take(BH * (size_t)NQ * NK * 4);
+    w.kvlen = c.take(BH * (size_t)NQ * 4);
+    w.total = c.off;
+    return w;
+}
+
+int num_sms_current() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+    }
+    cudaGetLastError();
+    return n > 0 ? n : 148;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) {
+    return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int memset_async(void* p, size_t n, cudaStream_t st) {
+    if (cudaMemsetAsync(p, 0, n, st) != cudaSuccess) {
+        cudaGetLastError();
+        return PARK_ERR_CUDA;
+    }
+    return PARK_OK;
+}
+
+// Score-bound factors (see k_assign.cu): tensor-core fp32 accumulation of
+// `terms` exact products (worst case terms * 2^-23 of sum |x_j w_j|), doubled
+// because the score is bias - 2 x.w, the bf16 hi/lo split residual of M c
+// (keys), and the rounding of the score itself.
+float gamma_for(int terms, bool split) {
+    double g = 2.0 * terms * 1.1920929e-7 * 1.01 + 2.4e-7;
+    if (split) g += 2.0 * 1.52587890625e-5;
+    return (float)(g * 1.05);
+}
+
+struct Side {
+    const void* X;
+    int K;
+    void* C;
+    int32_t* labels;
+    int32_t* perm;
+    int32_t* offsets;
+    const double* M;  // null: Euclidean
+    bool warm;
+    int cnt_slot;
+    float* xnorm;
+};
+
+int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, void* ws, int64_t* counters,
+               int num_sms, cudaStream_t st) {
+    const bool bf16 = d.dtype == PARK_BF16;
+    const int BH = d.BH, N = d.N, D = d.D, K = s.K;
+    const int nchunks = (N + kSortChunk - 1) / kSortChunk;
+    CentroidOps ops;
+    ops.bias32 = at<float>(ws, w.b32);
+    ops.bias64 = at<double>(ws, w.b64);
+    ops.w64 = s.M ? at<double>(ws, w.w64) : nullptr;
+    ops.wmax = at<float>(ws, w.wmax);
+    ops.bmax = at<float>(ws, w.bmax);
+    if (s.M) {
+        ops.w = bf16 ? at<uint16_t>(ws, w.wop) : nullptr;
+        ops.kw = 2 * D;
+    } else {
+        ops.w = static_cast<const uint16_t*>(s.C);
+        ops.kw = D;
+    }
+    Lists lists;
+    lists.pair_row = at<int32_t>(ws, w.lpair);
+    lists.pair_cand = at<int32_t>(ws, w.lcand);
+    lists.full_row = at<int32_t>(ws, w.lfull);
+    lists.counts = at<int32_t>(ws, w.lcnt);
+    if (bf16) PARK_CHECK(launch_row_norms(s.X, d.dtype, BH, N, D, s.xnorm, st));
+    if (!s.warm) PARK_CHECK(launch_strided_init(s.X, d.dtype, BH, N, D, K, s.C, st));
+    const float gamma = gamma_for(ops.kw, s.M != nullptr);
+    for (int it = 0; it < iters; ++it) {
+        PARK_CHECK(memset_async(ops.wmax, (size_t)BH * 4, st));
+        PARK_CHECK(memset_async(ops.bmax, (size_t)BH * 4, st));
+        PARK_CHECK(memset_async(lists.counts, 16 * 4, st));
+        PARK_CHECK(launch_centroid_prep(s.C, d.dtype, BH, K, D, s.M, ops, st));
+        if (bf16) {
+            PARK_CHECK(launch_assign_mma(s.X, BH, N, K, ops, s.xnorm, gamma, s.labels, lists, st));
+            PARK_CHECK(launch_recheck(s.X, d.dtype, BH, N, D, K, s.C, ops.w64, ops.bias64, s.labels, lists, 0,
+                                      num_sms, counters, s.cnt_slot, st));
+        } else {
+            PARK_CHECK(launch_recheck(s.X, d.dtype, BH, N, D, K, s.C, ops.w64, ops.bias64, s.labels, lists, 1,
+                                      num_sms, counters, s.cnt_slot, st));
+        }
+        PARK_CHECK(launch_label_sort(s.labels, BH, N, K, at<int32_t>(ws, w.hist), nchunks, s.perm, s.offsets, st));
+        PARK_CHECK(launch_update(s.X, d.dtype, BH, N, D, K, s.perm, s.offsets, s.C, st));
+    }
+    return PARK_OK;
+}
+
+bool retrieval_ptrs_ok(const park_retrieval* o) {
+    return o && o->q_labels && o->k_labels && o->q_perm && o->k_perm && o->q_offsets && o->k_offsets &&
+           o->q_centroids && o->k_centroids && o->importance && o->mask && o->kept_ptr && o->kept_idx &&
+           o->counters && o->status;
+}
+
+size_t ws_bytes_for(const Dims& d, int NQ, int NK) {
+    size_t a = plan_retrieval(d, NQ, NK).total, b = plan_attn(d, NQ, NK).total;
+    return a > b ? a : b;
+}
+
+int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, float p, int iters,
+                  park_retrieval* out, void* ws, cudaStream_t st) {
+    const RetrievalWs w = plan_retrieval(d, NQ, NK);
+    const int num_sms = num_sms_current();
+    const int BH = d.BH, N = d.N, D = d.D;
+    const size_t nel = (size_t)BH * N * D;
+    PARK_CHECK(memset_async(out->status, 4, st));
+    PARK_CHECK(memset_async(out->counters, PARK_NUM_COUNTERS * 8, st));
+    PARK_CHECK(memset_async(at<int32_t>(ws, w.pcnt), 16 * 4, st));
+    PARK_CHECK(launch_input_check(Q, nel, d.dtype, out->status, st));
+    PARK_CHECK(launch_input_check(K, nel, d.dtype, out->status, st));
+    double* M = at<double>(ws, w.M);
+    PARK_CHECK(launch_metric(Q, d.dtype, BH, N, D, at<double>(ws, w.Mpart), metric_chunks(d), M, out->metric, st));
+
+    Side sq{Q, NQ, out->q_centroids, out->q_labels, out->q_perm, out->q_offsets, nullptr,
+            (out->flags & PARK_FLAG_WARM_START_Q) != 0, PARK_CNT_Q_RECHECK, at<float>(ws, w.xnorm_q)};
+    Side sk{K, NK, out->k_centroids, out->k_labels, out->k_perm, out->k_offsets, M,
+            (out->flags & PARK_FLAG_WARM_START_K) != 0, PARK_CNT_K_RECHECK, at<float>(ws, w.xnorm_k)};
+    PARK_CHECK(run_kmeans(d, sq, iters, w, ws, out->counters, num_sms, st));
+    PARK_CHECK(run_kmeans(d, sk, iters, w, ws, out->counters, num_sms, st));
+
+    int32_t* kcnt = at<int32_t>(ws, w.kcnt);
+    if (d.dtype == PARK_BF16) {
+        // max ||c_m|| over the final key centroids, for the PAMA bound
+        CentroidOps ops{nullptr, D, at<float>(ws, w.b32), at<double>(ws, w.b64), nullptr, at<float>(ws, w.wmax),
+                        at<float>(ws, w.bmax)};
+        PARK_CHECK(memset_async(ops.wmax, (size_t)BH * 4, st));
+        PARK_CHECK(memset_async(ops.bmax, (size_t)BH * 4, st));
+        PARK_CHECK(launch_centroid_prep(out->k_centroids, d.dtype, BH, NK, D, nullptr, ops, st));
+        PARK_CHECK(launch_pama_mma(Q, BH, N, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids, out->k_offsets,
+                                   at<float>(ws, w.xnorm_q), out->importance, at<float>(ws, w.rho), ops.wmax, st));
+        PARK_CHECK(launch_topp(out->importance, at<float>(ws, w.rho), BH, NQ, NK, out->q_offsets, out->k_offsets, p,
+                               out->mask, kcnt, at<int32_t>(ws, w.plist), at<int32_t>(ws, w.pcnt), st));
+        PARK_CHECK(launch_pama_f64(Q, d.dtype, BH, N, D, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids,
+                                   out->k_offsets, p, at<int32_t>(ws, w.plist), at<int32_t>(ws, w.pcnt), 0, num_sms,
+                                   out->importance, out->mask, kcnt, out->counters, st));
+    } else {
+        PARK_CHECK(launch_pama_f64(Q, d.dtype, BH, N, D, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids,
+                                   out->k_offsets, p, nullptr, nullptr, 1, num_sms, out->importance, out->mask, kcnt,
+                                   out->counters, st));
+    }
+    PARK_CHECK(launch_kept_csr(out->mask, kcnt, BH, NQ, NK, out->kept_ptr, out->kept_idx, out->counters, st));
+    return PARK_OK;
+}
+
+int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ, int NK, const park_retrieval* r,
+              void* O, void* ws, cudaStream_t st) {
+    const AttnWs w = plan_attn(d, NQ, NK);
+    const int BH = d.BH, N = d.N, D = d.D;
+    PARK_CHECK(launch_input_check(V, (size_t)BH * N * D, d.dtype, r->status, st));
+    PARK_CHECK(memset_async(r->counters + PARK_CNT_KEPT_PAIRS, 2 * sizeof(int64_t), st));
+    int32_t* icnt = at<int32_t>(ws, w.icnt);
+    PARK_CHECK(memset_async(icnt, 16 * 4, st));
+    PARK_CHECK(launch_attn_schedule(BH, NQ, NK, r->q_offsets, r->k_offsets, r->kept_ptr, r->kept_idx,
+                                    at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
+                                    icnt, r->counters, kAttnTile, st));
+    if (d.dtype != PARK_BF16) {
+        return launch_sparse_attn_simt(Q, K, V, d.dtype, BH, N, D, NQ, NK, r->q_labels, r->k_perm, r->k_offsets,
+                                       r->kept_ptr, r->kept_idx, O, st);
+    }
+    const int num_sms = num_sms_current();
+    void* Qp = at<void>(ws, w.Qp);
+    void* Kp = at<void>(ws, w.Kp);
+    void* Vp = at<void>(ws, w.Vp);
+    PARK_CHECK(launch_gather(Q, d.dtype, BH, N, D, r->q_perm, Qp, st));
+    PARK_CHECK(launch_gather(K, d.dtype, BH, N, D, r->k_perm, Kp, st));
+    PARK_CHECK(launch_gather(V, d.dtype, BH, N, D, r->k_perm, Vp, st));
+    PARK_CHECK(launch_sparse_attn_mma(Qp, Kp, Vp, BH, N, NQ, NK, r->q_perm, r->k_offsets, r->kept_ptr, r->kept_idx,
+                                      at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
+                                      icnt, icnt + 1, O, num_sms, st));
+    return PARK_OK;
+}
+
+}  // namespace
+}  // namespace park
+
+using namespace park;
+
+extern "C" {
+
+int park_workspace_size(const park_shape* shape, int NQ, int NK, size_t* bytes) {
+    Dims d;
+    if (!bytes) return PARK_ERR_INVALID_ARG;
+    PARK_CHECK(check_shape(shape, NQ, NK, &d));
+    *bytes = ws_bytes_for(d, NQ, NK);
+    return PARK_OK;
+}
+
+int park_retrieve(const void* Q, const void* K, const park_shape* shape, int NQ, int NK, float p, int iters,
+                  park_retrieval* out, void* ws, size_t ws_bytes, void* stream) {
+    Dims d;
+    PARK_CHECK(check_shape(shape, NQ, NK, &d));
+    if (!Q || !K || !ws || !retrieval_ptrs_ok(out)) return PARK_ERR_INVALID_ARG;
+    if (!(p > 0.0f) || !std::isfinite(p) || iters < 1) return PARK_ERR_INVALID_ARG;
+    if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
+    return retrieve_impl(Q, K, d, NQ, NK, p, iters, out, ws, static_cast<cudaStream_t>(stream));
+}
+
+int park_sparse_attn(const void* Q, const void* K, const void* V, const park_shape* shape, int NQ, int NK,
+                     const park_retrieval* r, void* O, void* ws, size_t ws_bytes, void* stream) {
+    Dims d;
+    PARK_CHECK(check_shape(shape, NQ, NK, &d));
+    if (!Q || !K || !V || !O || !ws || !retrieval_ptrs_ok(r)) return PARK_ERR_INVALID_ARG;
+    if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
+    return attn_impl(Q, K, V, d, NQ, NK, r, O, ws, static_cast<cudaStream_t>(stream));
+}
+
+int park_layer(const void* Q, const void* K, const void* V, const park_shape* shape, int NQ, int NK, float p,
+               int iters, void* O, park_retrieval* out, void* ws, size_t ws_bytes, void* stream) {
+    Dims d;
+    PARK_CHECK(check_shape(shape, NQ, NK, &d));
+    if (!Q || !K || !V || !O || !ws || !retrieval_ptrs_ok(out)) return PARK_ERR_INVALID_ARG;
+    if (!(p > 0.0f) || !std::isfinite(p) || iters < 1) return PARK_ERR_INVALID_ARG;
+    if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    PARK_CHECK(retrieve_impl(Q, K, d, NQ, NK, p, iters, out, ws, st));
+    return attn_impl(Q, K, V, d, NQ, NK, out, O, ws, st);
+}
+
+const char* park_status_string(int code) {
+    switch (code) {
+        case PARK_OK: return "ok";
+        case PARK_ERR_INVALID_ARG: return "invalid argument";
+        case PARK_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case PARK_ERR_WORKSPACE: return "workspace too small";
+        case PARK_ERR_CUDA: return "CUDA launch failed";
+        case PARK_ERR_RANGE: return "input outside the range precondition (0 or 2^-20 <= |x| < 2^16, finite)";
+        case PARK_ERR_TIMEOUT: return "a bounded device wait ran out";
+        default: return "unknown status";
+    }
+}
+
+uint64_t park_launch_count(void) { return (uint64_t)g_launches.load(); }
+
+int park_version(void) { return 100; }
+
+}  // extern "C"

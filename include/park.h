@@ -1,0 +1,162 @@
+/*
+ * park.h - C ABI of the PARK block-retrieval + block-sparse attention library
+ * (libpark.so, CUDA, sm_100a).
+ *
+ * The operation is the one described in "PARK: Accurate Block Retrieval for
+ * Sparse Attention in Video Diffusion Transformers" (abstract; Figure 2
+ * caption; Table 1 caption): for one attention layer, cluster the queries with
+ * Euclidean K-means, cluster the keys with K-means under a metric derived from
+ * the current queries (QRKC), give every original query a Softmax over the key
+ * centroids and average these within each query cluster (PAMA), keep key
+ * clusters per query cluster up to cumulative importance p (top-p), and compute
+ * attention only on the kept (query-cluster, key-cluster) pairs.
+ *
+ * Definitions fixed by this library where the pages are silent:
+ *   metric       M = (1/N) sum_i q_i q_i^T (float64); key distance
+ *                (k - c)^T M (k - c) = mean_i (q_i.k - q_i.c)^2.
+ *   K-means      init c_k = x_floor(k N / K); `iters` x (assign, update), no
+ *                early stop; assign ties go to the lowest index; update
+ *                c_k = round_dtype(fl64(exact sum of members) / n_k), empty
+ *                clusters keep their centroid.  Key centroids live in raw key
+ *                space.
+ *   PAMA         P_im = softmax over NON-EMPTY key clusters m of (q_i.c_m)/sqrt(D);
+ *                I_rm = mean over members i of query cluster r of P_im.
+ *   top-p        per non-empty query cluster: key clusters sorted by I_rm
+ *                descending (ties: lower m first); keep the shortest prefix
+ *                whose running sum is >= p (crossing block kept); p >= 1 keeps
+ *                every non-empty key cluster.
+ *   attention    o_i = sum_{j in J_r} softmax_j(q_i.k_j/sqrt(D)) v_j with J_r the
+ *                keys of the kept key clusters of i's query cluster r.
+ *
+ * Conventions
+ *   - Every pointer argument named Q, K, V, O, ws and every pointer inside
+ *     park_retrieval is a DEVICE pointer; shape structs and `bytes` are host.
+ *   - Ownership: the caller allocates and frees everything.  The library never
+ *     allocates, frees or synchronises; all work is enqueued on `stream` (a
+ *     cudaStream_t passed as void*, NULL = legacy default stream).
+ *   - Layout: Q, K, V, O are [B, H, N, D] contiguous, N = T*Hg*W + n_text
+ *     (video tokens in (t, y, w) order, text tokens last).  dtype PARK_BF16
+ *     requires D == 128; PARK_F32 requires D % 32 == 0 and D <= 128.
+ *   - Range precondition: every input element is 0 or has 2^-20 <= |x| < 2^16
+ *     (and is finite).  N <= 2^20, B*H*N < 2^31, 1 <= NQ, NK <= N,
+ *     NK <= 4096, NQ <= 65536, p > 0, iters >= 1.
+ *   - Errors: argument errors are returned synchronously (nothing is enqueued).
+ *     Conditions only the device can see (an input outside the range
+ *     precondition, a bounded wait that ran out) are written to *status; the
+ *     outputs are valid only if *status == PARK_OK after the stream has
+ *     reached the end of the call.  A launch failure returns PARK_ERR_CUDA.
+ */
+#ifndef PARK_H
+#define PARK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define PARK_OK 0
+#define PARK_ERR_INVALID_ARG 1 /* null pointer, bad shape or parameter       */
+#define PARK_ERR_UNSUPPORTED 2 /* valid but not implemented (e.g. bf16, D!=128) */
+#define PARK_ERR_WORKSPACE 3   /* ws_bytes smaller than park_workspace_size   */
+#define PARK_ERR_CUDA 4        /* a kernel launch or memset failed            */
+#define PARK_ERR_RANGE 5       /* device: input outside the range precondition */
+#define PARK_ERR_TIMEOUT 6     /* device: a bounded wait ran out              */
+
+/* ---- element types ----------------------------------------------------- */
+#define PARK_BF16 0
+#define PARK_F32 1
+
+/* ---- park_retrieval.flags (inputs) ------------------------------------- */
+/* Start query / key K-means from the centroids already in q_centroids /
+ * k_centroids instead of the strided initialisation (mask and cluster reuse
+ * across denoising steps, PARK Appendix Table 9). */
+#define PARK_FLAG_WARM_START_Q 0x1u
+#define PARK_FLAG_WARM_START_K 0x2u
+
+/* ---- park_retrieval.counters indices (outputs, int64) ------------------ */
+#define PARK_CNT_Q_RECHECK 0    /* query rows whose bf16 score margin was not
+                                   certified and were rescored in float64    */
+#define PARK_CNT_K_RECHECK 1    /* same for key rows                          */
+#define PARK_CNT_FULL_RESCORE 2 /* rows rescored against every centroid       */
+#define PARK_CNT_PAMA_RECHECK 3 /* query clusters whose top-p cut was not
+                                   certified and were recomputed in float64  */
+#define PARK_CNT_KEPT_BLOCKS 4  /* kept (query cluster, key cluster) pairs    */
+#define PARK_CNT_KEPT_PAIRS 5   /* sum_r |Q_r| * |J_r|: attended query-key pairs */
+#define PARK_CNT_WORK_ITEMS 6   /* query tiles scheduled for attention        */
+#define PARK_CNT_RESERVED 7
+#define PARK_NUM_COUNTERS 8
+
+/* Problem shape.  N = T*Hg*W + n_text. */
+typedef struct {
+    int B, H;          /* batch, heads                                       */
+    int T, Hg, W;      /* video token grid (frames, height, width)           */
+    int n_text;        /* text tokens appended after the video tokens        */
+    int D;             /* head dimension                                     */
+    int dtype;         /* PARK_BF16 or PARK_F32 (Q, K, V, O and centroids)   */
+} park_shape;
+
+/* Retrieval result.  All arrays are caller-allocated DEVICE memory, [B, H, ...]
+ * contiguous; "bh" below is b*H + h.  Written by park_retrieve, read by
+ * park_sparse_attn. */
+typedef struct {
+    uint32_t flags;        /* in: PARK_FLAG_* bits                                */
+    int32_t *q_labels;     /* [B,H,N]      query cluster of each token            */
+    int32_t *k_labels;     /* [B,H,N]      key cluster of each token              */
+    int32_t *q_perm;       /* [B,H,N]      sorted position -> token (stable by cluster) */
+    int32_t *k_perm;       /* [B,H,N]                                             */
+    int32_t *q_offsets;    /* [B,H,NQ+1]   first sorted position of each cluster  */
+    int32_t *k_offsets;    /* [B,H,NK+1]                                          */
+    void *q_centroids;     /* [B,H,NQ,D]   input dtype                            */
+    void *k_centroids;     /* [B,H,NK,D]   input dtype, raw key space             */
+    float *importance;     /* [B,H,NQ,NK]  PAMA block importance I               */
+    uint8_t *mask;         /* [B,H,NQ,NK]  1 = kept                               */
+    int32_t *kept_ptr;     /* [B,H,NQ+1]   CSR row pointers, per (b,h) from 0     */
+    int32_t *kept_idx;     /* [B,H,NQ*NK]  kept m per row, ascending; row r of
+                              head bh starts at bh*NQ*NK + kept_ptr[bh*(NQ+1)+r]   */
+    double *metric;        /* [B,H,D,D]    optional (may be NULL): the metric M   */
+    int64_t *counters;     /* [PARK_NUM_COUNTERS], zeroed by park_retrieve        */
+    int32_t *status;       /* [1] device status word, zeroed by park_retrieve     */
+} park_retrieval;
+
+/* Bytes of device workspace that park_retrieve, park_sparse_attn and
+ * park_layer need for this shape (one buffer serves all three).  Host only;
+ * returns PARK_ERR_INVALID_ARG / PARK_ERR_UNSUPPORTED for bad shapes. */
+int park_workspace_size(const park_shape *shape, int NQ, int NK, size_t *bytes);
+
+/* Block retrieval (PARK Figure 2): metric, query K-means, QRKC key K-means,
+ * PAMA, top-p, CSR of kept blocks.  Q, K: device [B,H,N,D].  Fills every array
+ * of *out except that out->metric is written only when non-NULL. */
+int park_retrieve(const void *Q, const void *K, const park_shape *shape, int NQ, int NK, float p,
+                  int iters, park_retrieval *out, void *ws, size_t ws_bytes, void *stream);
+
+/* Block-sparse attention over the kept blocks of a retrieval result (PARK
+ * abstract: "computing attention only within" the retrieved blocks).  Reads
+ * labels, perms, offsets and the CSR of *r; writes O [B,H,N,D] in the input
+ * dtype, original token order.  Also sets r->counters[PARK_CNT_WORK_ITEMS] and
+ * may set *r->status. */
+int park_sparse_attn(const void *Q, const void *K, const void *V, const park_shape *shape, int NQ,
+                     int NK, const park_retrieval *r, void *O, void *ws, size_t ws_bytes,
+                     void *stream);
+
+/* park_retrieve followed by park_sparse_attn on the same stream. */
+int park_layer(const void *Q, const void *K, const void *V, const park_shape *shape, int NQ, int NK,
+               float p, int iters, void *O, park_retrieval *out, void *ws, size_t ws_bytes,
+               void *stream);
+
+/* Static description of a status code (never NULL). */
+const char *park_status_string(int code);
+
+/* Number of CUDA kernels this library has launched in this process. */
+uint64_t park_launch_count(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int park_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARK_H */
