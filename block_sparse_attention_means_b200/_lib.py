@@ -32,7 +32,7 @@ PARK_NUM_COUNTERS = 8
 
 # Every symbol include/park.h declares (checked by the CPU tests).
 EXPORTS = ("park_workspace_size", "park_retrieve", "park_sparse_attn", "park_layer", "park_status_string",
-           "park_launch_count", "park_version")
+           "park_launch_count", "park_version", "park_profile_enable", "park_profile_collect")
 
 
 class ParkShape(ctypes.Structure):
@@ -49,6 +49,10 @@ class ParkRetrieval(ctypes.Structure):
                 ("importance", ctypes.c_void_p), ("mask", ctypes.c_void_p),
                 ("kept_ptr", ctypes.c_void_p), ("kept_idx", ctypes.c_void_p),
                 ("metric", ctypes.c_void_p), ("counters", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+
+
+class ParkKernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("total_ms", ctypes.c_double), ("launches", ctypes.c_int64)]
 
 
 class ParkError(RuntimeError):
@@ -84,6 +88,10 @@ def load() -> ctypes.CDLL:
     lib.park_launch_count.restype = ctypes.c_uint64
     lib.park_version.argtypes = []
     lib.park_version.restype = i32
+    lib.park_profile_enable.argtypes = [i32]
+    lib.park_profile_enable.restype = i32
+    lib.park_profile_collect.argtypes = [ctypes.POINTER(ParkKernelTime), i32, ctypes.POINTER(i32)]
+    lib.park_profile_collect.restype = i32
     _lib = lib
     return lib
 

@@ -13,9 +13,14 @@ namespace park {
 
 // ---------------------------------------------------------------- host side
 void note_launch(int n = 1);  // counts kernels for park_launch_count()
+// Per-kernel event timing (park_profile_enable): begin before a launch, end
+// (with the kernel's name) right after it, on the launch stream.
+void prof_begin(cudaStream_t st);
+void prof_end(const char* name, cudaStream_t st);
 
-#define PARK_TRY_LAUNCH()                                        \
+#define PARK_TRY_LAUNCH(name, st)                                \
     do {                                                         \
+        ::park::prof_end(name, st);                              \
         ::park::note_launch();                                   \
         if (cudaPeekAtLastError() != cudaSuccess) {              \
             cudaGetLastError();                                  \

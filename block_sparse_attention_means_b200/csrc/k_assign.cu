@@ -186,19 +186,21 @@ __global__ __launch_bounds__(256, 2) void k_assign_mma(const uint16_t* __restric
 int launch_assign_mma(const void* X, int BH, int N, int K, const CentroidOps& ops, const float* xnorm,
                       float gamma, int32_t* labels, Lists lists, cudaStream_t st) {
     dim3 grid((N + 127) / 128, BH);
+    if (ops.kw != 128 && ops.kw != 256) return PARK_ERR_UNSUPPORTED;
+    if (ops.kw == 256)
+        cudaFuncSetAttribute(k_assign_mma<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             2 * 64 * (256 + 8) * 2 + 2 * 64 * 4);
+    ::park::prof_begin(st);
     if (ops.kw == 128) {
         size_t sm = 2 * 64 * (128 + 8) * 2 + 2 * 64 * 4;
         k_assign_mma<128><<<grid, 256, sm, st>>>((const uint16_t*)X, ops.w, ops.bias32, xnorm, ops.wmax, ops.bmax,
                                                  gamma, N, K, labels, lists);
     } else if (ops.kw == 256) {
         size_t sm = 2 * 64 * (256 + 8) * 2 + 2 * 64 * 4;
-        cudaFuncSetAttribute(k_assign_mma<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         k_assign_mma<256><<<grid, 256, sm, st>>>((const uint16_t*)X, ops.w, ops.bias32, xnorm, ops.wmax, ops.bmax,
                                                  gamma, N, K, labels, lists);
-    } else {
-        return PARK_ERR_UNSUPPORTED;
     }
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_assign_mma", st);
     return PARK_OK;
 }
 
@@ -284,6 +286,7 @@ int launch_recheck(const void* X, int dtype, int BH, int N, int D, int K, const 
     const int blocks = num_sms * 8, threads = 256;
     const int total = BH * N;
     auto go = [&](int mode, const int32_t* rows, const int32_t* cand, const int32_t* cnt) {
+        ::park::prof_begin(st);
         if (dtype == PARK_BF16) {
             if (metric)
                 k_recheck<bf16_t, true><<<blocks, threads, 0, st>>>((const bf16_t*)X, (const bf16_t*)C, w64, b64, N,
@@ -306,12 +309,12 @@ int launch_recheck(const void* X, int dtype, int BH, int N, int D, int K, const 
     };
     if (all_rows) {
         go(2, nullptr, nullptr, nullptr);
-        PARK_TRY_LAUNCH();
+        PARK_TRY_LAUNCH("k_recheck", st);
     } else {
         go(0, lists.pair_row, lists.pair_cand, lists.counts + 0);
-        PARK_TRY_LAUNCH();
+        PARK_TRY_LAUNCH("k_recheck", st);
         go(1, lists.full_row, nullptr, lists.counts + 1);
-        PARK_TRY_LAUNCH();
+        PARK_TRY_LAUNCH("k_recheck", st);
     }
     return PARK_OK;
 }

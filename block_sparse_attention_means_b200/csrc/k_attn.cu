@@ -36,9 +36,10 @@ int launch_gather(const void* X, int dtype, int BH, int N, int D, const int32_t*
     size_t rows = (size_t)BH * N;
     size_t total = rows * vpr;
     int blocks = (int)((total + 255) / 256);
+    ::park::prof_begin(st);
     if (blocks > 148 * 32) blocks = 148 * 32;
     k_gather_rows<<<blocks, 256, 0, st>>>((const uint4*)X, perm, (uint4*)Xp, rows, N, vpr);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_gather_rows", st);
     return PARK_OK;
 }
 
@@ -104,9 +105,10 @@ __global__ __launch_bounds__(256) void k_attn_schedule(int NQ, int NK, const int
 int launch_attn_schedule(int BH, int NQ, int NK, const int32_t* q_off, const int32_t* k_off,
                          const int32_t* kept_ptr, const int32_t* kept_idx, int32_t* kv_pre, int32_t* kv_len,
                          WorkItem* items, int32_t* item_count, int64_t* counters, int tile_rows, cudaStream_t st) {
+    ::park::prof_begin(st);
     k_attn_schedule<<<dim3(NQ, BH), 256, 0, st>>>(NQ, NK, q_off, k_off, kept_ptr, kept_idx, kv_pre, kv_len, items,
                                                   item_count, counters, tile_rows);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_attn_schedule", st);
     return PARK_OK;
 }
 
@@ -314,10 +316,11 @@ int launch_sparse_attn_mma(const void* Qp, const void* Kp, const void* Vp, int B
     size_t sm = 2 * 2 * AT_ROWS * AT_LDS * 2 + 2 * AT_ROWS * 4;
     cudaFuncSetAttribute(k_sparse_attn_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     float sl2e = (1.0f / sqrtf(128.f)) * kLog2eA;
+    ::park::prof_begin(st);
     k_sparse_attn_mma<<<num_sms * 3, 128, sm, st>>>((const uint16_t*)Qp, (const uint16_t*)Kp, (const uint16_t*)Vp,
                                                      N, NQ, NK, q_perm, k_off, kept_ptr, kept_idx, kv_pre, kv_len,
                                                      items, item_count, work_counter, (uint16_t*)O, sl2e);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_sparse_attn_mma", st);
     return PARK_OK;
 }
 
@@ -382,11 +385,12 @@ int launch_sparse_attn_simt(const void* Q, const void* K, const void* V, int dty
     if (dtype != PARK_F32 || D > 128) return PARK_ERR_UNSUPPORTED;
     size_t rows = (size_t)BH * N;
     int blocks = (int)((rows * 32 + 255) / 256);
+    ::park::prof_begin(st);
     if (blocks > 148 * 64) blocks = 148 * 64;
     k_sparse_attn_simt<float><<<blocks, 256, 0, st>>>((const float*)Q, (const float*)K, (const float*)V, N, D, NQ, NK,
                                                       q_labels, k_perm, k_off, kept_ptr, kept_idx, (float*)O, rows,
                                                       1.0f / sqrtf((float)D));
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_sparse_attn_simt", st);
     return PARK_OK;
 }
 

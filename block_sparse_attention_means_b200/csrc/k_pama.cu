@@ -134,10 +134,13 @@ __global__ __launch_bounds__(128) void k_pama_mma(const uint16_t* __restrict__ Q
                     mrow[h] = mn;
                 }
             }
+            // rows whose max is still -inf have seen only empty clusters: nothing to add
+            const float mr0 = mrow[0] == __int_as_float(0xff800000) ? 0.f : mrow[0];
+            const float mr1 = mrow[1] == __int_as_float(0xff800000) ? 0.f : mrow[1];
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) lrow[j >> 1] += (double)exp2f(acc[nt][j] - mrow[j >> 1]);
+                for (int j = 0; j < 4; ++j) lrow[j >> 1] += (double)exp2f(acc[nt][j] - (j < 2 ? mr0 : mr1));
             __syncthreads();
         }
         float inv[2];
@@ -205,9 +208,10 @@ int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t*
     float sl2e = scale * kLog2e;
     // |logit~ - logit| <= s * (D 2^-23 + 2^-22) ||q|| max||c||  (tensor-core accumulation, scaling)
     float delta_scale = (float)((1.0 / sqrt((double)D)) * ((double)D * 1.1920929e-7 * 1.01 + 2.4e-7));
+    ::park::prof_begin(st);
     k_pama_mma<<<dim3(NQ, BH), 128, sm, st>>>((const uint16_t*)Q, q_perm, q_off, (const uint16_t*)CK, k_off, qnorm,
                                               ckmax, N, NQ, NK, sl2e, delta_scale, importance, rho);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_pama_mma", st);
     return PARK_OK;
 }
 
@@ -356,9 +360,10 @@ int launch_topp(const float* importance, const float* rho, int BH, int NQ, int N
     if (NKP < 512) NKP = 512;
     size_t sm = (size_t)NKP * (8 + 4 + 4 + 1) + 16;
     cudaFuncSetAttribute(k_topp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    ::park::prof_begin(st);
     k_topp<<<dim3(NQ, BH), 512, sm, st>>>(importance, rho, q_off, k_off, NQ, NK, NKP, p, mask, kept_cnt, flag_list,
                                           flag_count);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_topp", st);
     return PARK_OK;
 }
 
@@ -500,18 +505,21 @@ int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int 
     size_t sm = (size_t)NKP * 12 + 128 * 8;
     int blocks = num_sms * 4;
     double scale = 1.0 / sqrt((double)D);
-    if (dtype == PARK_BF16) {
+    if (dtype == PARK_BF16)
         cudaFuncSetAttribute(k_pama_f64<bf16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    else
+        cudaFuncSetAttribute(k_pama_f64<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    ::park::prof_begin(st);
+    if (dtype == PARK_BF16) {
         k_pama_f64<bf16_t><<<blocks, 256, sm, st>>>((const bf16_t*)Q, q_perm, q_off, (const bf16_t*)CK, k_off, N, D,
                                                     NQ, NK, NKP, scale, p, list, count, all_clusters, BH * NQ,
                                                     importance, mask, kept_cnt, counters);
     } else {
-        cudaFuncSetAttribute(k_pama_f64<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         k_pama_f64<float><<<blocks, 256, sm, st>>>((const float*)Q, q_perm, q_off, (const float*)CK, k_off, N, D, NQ,
                                                    NK, NKP, scale, p, list, count, all_clusters, BH * NQ, importance,
                                                    mask, kept_cnt, counters);
     }
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_pama_f64", st);
     return PARK_OK;
 }
 
@@ -579,10 +587,12 @@ __global__ __launch_bounds__(256) void k_kept_compact(const uint8_t* __restrict_
 
 int launch_kept_csr(const uint8_t* mask, const int32_t* kept_cnt, int BH, int NQ, int NK, int32_t* kept_ptr,
                     int32_t* kept_idx, int64_t* counters, cudaStream_t st) {
+    ::park::prof_begin(st);
     k_kept_scan<<<BH, 1024, 0, st>>>(kept_cnt, NQ, kept_ptr, counters);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_kept_scan", st);
+    ::park::prof_begin(st);
     k_kept_compact<<<dim3(NQ, BH), 256, 0, st>>>(mask, kept_ptr, NQ, NK, kept_idx);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_kept_compact", st);
     return PARK_OK;
 }
 

@@ -38,13 +38,14 @@ int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status
     int eb = dtype == PARK_BF16 ? 2 : 4;
     size_t n16 = n_elems * eb / 16;
     int blocks = (int)((n16 + 255) / 256);
+    ::park::prof_begin(st);
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (blocks < 1) blocks = 1;
     if (eb == 2)
         k_input_check<2><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status);
     else
         k_input_check<4><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_input_check", st);
     return PARK_OK;
 }
 
@@ -118,14 +119,16 @@ int launch_metric(const void* Q, int dtype, int BH, int N, int D, double* part, 
     int rpc = (N + nchunks - 1) / nchunks;
     dim3 g1(nchunks, BH);
     size_t sm = 32 * D * sizeof(double);
+    ::park::prof_begin(st);
     if (dtype == PARK_BF16)
         k_metric_partial<bf16_t><<<g1, 256, sm, st>>>((const bf16_t*)Q, N, D, rpc, part);
     else
         k_metric_partial<float><<<g1, 256, sm, st>>>((const float*)Q, N, D, rpc, part);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_metric_partial", st);
     dim3 g2((D * D + 255) / 256, BH);
+    ::park::prof_begin(st);
     k_metric_reduce<<<g2, 256, 0, st>>>(part, nchunks, N, D, M, M_out);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_metric_reduce", st);
     return PARK_OK;
 }
 
@@ -150,11 +153,12 @@ __global__ void k_row_norms(const T* __restrict__ X, size_t rows, int D, float* 
 int launch_row_norms(const void* X, int dtype, int BH, int N, int D, float* xnorm, cudaStream_t st) {
     size_t rows = (size_t)BH * N;
     int blocks = (int)((rows * 32 + 255) / 256);
+    ::park::prof_begin(st);
     if (dtype == PARK_BF16)
         k_row_norms<bf16_t><<<blocks, 256, 0, st>>>((const bf16_t*)X, rows, D, xnorm);
     else
         k_row_norms<float><<<blocks, 256, 0, st>>>((const float*)X, rows, D, xnorm);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_row_norms", st);
     return PARK_OK;
 }
 
@@ -171,8 +175,9 @@ __global__ void k_strided_init(const uint8_t* __restrict__ X, int N, int K, int 
 
 int launch_strided_init(const void* X, int dtype, int BH, int N, int D, int K, void* C, cudaStream_t st) {
     int rb = D * (dtype == PARK_BF16 ? 2 : 4);
+    ::park::prof_begin(st);
     k_strided_init<<<dim3(K, BH), 64, 0, st>>>((const uint8_t*)X, N, K, rb, (uint8_t*)C);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_strided_init", st);
     return PARK_OK;
 }
 
@@ -232,6 +237,7 @@ int launch_centroid_prep(const void* C, int dtype, int BH, int K, int D, const d
     if (D > 128) return PARK_ERR_UNSUPPORTED;  // one thread per coordinate
     dim3 g(K, BH);
     bool metric = M != nullptr;
+    ::park::prof_begin(st);
     if (dtype == PARK_BF16) {
         if (metric)
             k_centroid_prep<bf16_t, true><<<g, D, 0, st>>>((const bf16_t*)C, K, D, M, (uint16_t*)ops.w, ops.bias32,
@@ -247,7 +253,7 @@ int launch_centroid_prep(const void* C, int dtype, int BH, int K, int D, const d
             k_centroid_prep<float, false><<<g, D, 0, st>>>((const float*)C, K, D, M, nullptr, ops.bias32,
                                                           ops.bias64, ops.w64, ops.wmax, ops.bmax);
     }
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_centroid_prep", st);
     return PARK_OK;
 }
 

@@ -113,12 +113,15 @@ int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist
         cudaFuncSetAttribute(k_label_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     }
     dim3 g(nchunks, BH);
+    ::park::prof_begin(st);
     k_label_hist<<<g, 256, sm, st>>>(labels, N, K, nchunks, hist);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_label_hist", st);
+    ::park::prof_begin(st);
     k_label_scan<<<BH, 1024, 0, st>>>(hist, N, K, nchunks, offsets);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_label_scan", st);
+    ::park::prof_begin(st);
     k_label_scatter<<<g, 1024, sm, st>>>(labels, N, K, nchunks, hist, perm);
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_label_scatter", st);
     return PARK_OK;
 }
 
@@ -205,16 +208,17 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
 int launch_update(const void* X, int dtype, int BH, int N, int D, int K, const int32_t* perm,
                   const int32_t* offsets, void* C, cudaStream_t st) {
     dim3 g(K, BH);
+    const int vec = dtype == PARK_BF16 ? 8 : 4;
+    if (D % vec || D / vec > 128) return PARK_ERR_UNSUPPORTED;
+    ::park::prof_begin(st);
     if (dtype == PARK_BF16) {
-        if (D % 8 || D / 8 > 128) return PARK_ERR_UNSUPPORTED;
         int rpi = 128 / (D / 8);
         k_update<bf16_t><<<g, 128, (size_t)rpi * D * 8, st>>>((const bf16_t*)X, perm, offsets, N, D, K, (bf16_t*)C);
     } else {
-        if (D % 4 || D / 4 > 128) return PARK_ERR_UNSUPPORTED;
         int rpi = 128 / (D / 4);
         k_update<float><<<g, 128, (size_t)rpi * D * 16, st>>>((const float*)X, perm, offsets, N, D, K, (float*)C);
     }
-    PARK_TRY_LAUNCH();
+    PARK_TRY_LAUNCH("k_update", st);
     return PARK_OK;
 }
 

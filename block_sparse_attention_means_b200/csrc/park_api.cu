@@ -3,6 +3,9 @@
 // allocates or synchronises; every step is a kernel on the caller's stream.
 #include <atomic>
 #include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "kernels.h"
 
@@ -10,6 +13,53 @@ namespace park {
 
 static std::atomic<unsigned long long> g_launches{0};
 void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+// ---------------------------------------------------------------- per-kernel timing
+namespace {
+struct ProfRec {
+    const char* name;
+    cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::atomic<bool> g_prof_on{false};
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_prof_pool;
+thread_local cudaEvent_t t_prof_begin = nullptr;
+
+cudaEvent_t prof_event() {
+    if (!g_prof_pool.empty()) {
+        cudaEvent_t e = g_prof_pool.back();
+        g_prof_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return e;
+}
+}  // namespace
+
+void prof_begin(cudaStream_t st) {
+    if (!g_prof_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    t_prof_begin = prof_event();
+    if (t_prof_begin) cudaEventRecord(t_prof_begin, st);
+}
+
+void prof_end(const char* name, cudaStream_t st) {
+    if (!g_prof_on.load(std::memory_order_relaxed) || !t_prof_begin) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    cudaEvent_t b = prof_event();
+    if (b) {
+        cudaEventRecord(b, st);
+        g_prof_recs.push_back({name, t_prof_begin, b});
+    } else {
+        g_prof_pool.push_back(t_prof_begin);
+    }
+    t_prof_begin = nullptr;
+}
 
 namespace {
 
@@ -357,6 +407,41 @@ const char* park_status_string(int code) {
 }
 
 uint64_t park_launch_count(void) { return (uint64_t)g_launches.load(); }
+
+int park_profile_enable(int on) {
+    g_prof_on.store(on != 0);
+    return PARK_OK;
+}
+
+int park_profile_collect(park_kernel_time* out, int cap, int* n) {
+    if (!n || cap < 0 || (cap > 0 && !out)) return PARK_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    int count = 0, rc = PARK_OK;
+    for (const ProfRec& r : g_prof_recs) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+            cudaGetLastError();
+            rc = PARK_ERR_CUDA;
+        }
+        int slot = -1;
+        for (int i = 0; i < count; ++i)
+            if (std::strcmp(out[i].name, r.name) == 0) slot = i;
+        if (slot < 0 && count < cap) {
+            slot = count++;
+            std::memset(&out[slot], 0, sizeof(park_kernel_time));
+            std::strncpy(out[slot].name, r.name, sizeof(out[slot].name) - 1);
+        }
+        if (slot >= 0) {
+            out[slot].total_ms += ms;
+            out[slot].launches += 1;
+        }
+        g_prof_pool.push_back(r.a);
+        g_prof_pool.push_back(r.b);
+    }
+    g_prof_recs.clear();
+    *n = count;
+    return rc;
+}
 
 int park_version(void) { return 100; }
 

@@ -162,3 +162,18 @@ def layer(Q, K, V, shape: Shape, NQ: int, NK: int, p: float, iters: int, O: torc
 
 def launch_count() -> int:
     return int(_lib.load().park_launch_count())
+
+
+def profile_enable(on: bool = True) -> None:
+    """Record a CUDA event pair around every later kernel launch of the library."""
+    _lib.check(_lib.load().park_profile_enable(1 if on else 0), "park_profile_enable")
+
+
+def profile_collect() -> dict:
+    """{kernel name: (total ms, launches)} of the recorded launches (call after a
+    synchronize); clears the record."""
+    cap = 64
+    buf = (_lib.ParkKernelTime * cap)()
+    n = ctypes.c_int(0)
+    _lib.check(_lib.load().park_profile_collect(buf, cap, ctypes.byref(n)), "park_profile_collect")
+    return {buf[i].name.decode(): (buf[i].total_ms, int(buf[i].launches)) for i in range(n.value)}

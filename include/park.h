@@ -155,6 +155,23 @@ uint64_t park_launch_count(void);
 /* Library version, major*10000 + minor*100 + patch. */
 int park_version(void);
 
+/* ---- per-kernel timing for measurement tools --------------------------- */
+typedef struct {
+    char name[48];     /* kernel name                                        */
+    double total_ms;   /* summed device time between its begin/end events    */
+    int64_t launches;  /* number of launches recorded                        */
+} park_kernel_time;
+
+/* on != 0: every later kernel launch of this library records a CUDA event
+ * before and after it on its stream (host state, all threads).  Off by
+ * default; costs two event records per launch. */
+int park_profile_enable(int on);
+
+/* Aggregate the recorded launches by kernel name into out[0..cap) and clear
+ * the record; *n = entries written.  Call only after every recorded stream has
+ * been synchronised.  Returns PARK_ERR_CUDA if an event could not be read. */
+int park_profile_collect(park_kernel_time *out, int cap, int *n);
+
 #ifdef __cplusplus
 }
 #endif
