@@ -32,7 +32,8 @@ PARK_NUM_COUNTERS = 8
 
 # Every symbol include/park.h declares (checked by the CPU tests).
 EXPORTS = ("park_workspace_size", "park_retrieve", "park_sparse_attn", "park_layer", "park_status_string",
-           "park_launch_count", "park_version", "park_profile_enable", "park_profile_collect")
+           "park_launch_count", "park_version", "park_profile_enable", "park_profile_collect",
+           "park_qrkc_metric_static")
 
 
 class ParkShape(ctypes.Structure):
@@ -92,6 +93,8 @@ def load() -> ctypes.CDLL:
     lib.park_profile_enable.restype = i32
     lib.park_profile_collect.argtypes = [ctypes.POINTER(ParkKernelTime), i32, ctypes.POINTER(i32)]
     lib.park_profile_collect.restype = i32
+    lib.park_qrkc_metric_static.argtypes = [vp, shp, vp, vp]
+    lib.park_qrkc_metric_static.restype = i32
     _lib = lib
     return lib
 

@@ -172,6 +172,24 @@ int park_profile_enable(int on);
  * been synchronised.  Returns PARK_ERR_CUDA if an event could not be read. */
 int park_profile_collect(park_kernel_time *out, int cap, int *n);
 
+/* ---- metric without caller workspace ----------------------------------- */
+/* The paper has no counterpart of this entry point: it exists for callers
+ * that cannot allocate device memory where they need the QRKC metric (for
+ * example while a CUDA graph is being captured, where cudaMalloc is not
+ * allowed, or inside a host framework that passes only input and output
+ * buffers).  It computes the same M = (1/N) sum_i q_i q_i^T per (b, h) as
+ * park_retrieve writes to out->metric.
+ *   Q: device [B,H,N,D] (same dtypes and D as park_retrieve); M: device float64
+ *   [B,H,D,D], written; stream: cudaStream_t or NULL.
+ * Scratch comes from a 16 MiB array compiled into the library (held by every
+ * GPU that loads it until exit), so B*H may be at most 16 MiB / (8*D*D)
+ * (128 at D = 128); larger shapes return PARK_ERR_UNSUPPORTED with nothing
+ * enqueued.  No allocation of any kind.  The first call on each device looks
+ * up the array's device address (with that device current): make it before
+ * any stream capture.  All calls share the array, so calls that overlap on the
+ * GPU race; serialise them (one stream, or events). */
+int park_qrkc_metric_static(const void *Q, const park_shape *shape, double *M, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
