@@ -49,7 +49,8 @@ class ParkRetrieval(ctypes.Structure):
                 ("q_centroids", ctypes.c_void_p), ("k_centroids", ctypes.c_void_p),
                 ("importance", ctypes.c_void_p), ("mask", ctypes.c_void_p),
                 ("kept_ptr", ctypes.c_void_p), ("kept_idx", ctypes.c_void_p),
-                ("metric", ctypes.c_void_p), ("counters", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+                ("metric", ctypes.c_void_p), ("importance_bound", ctypes.c_void_p),
+                ("counters", ctypes.c_void_p), ("status", ctypes.c_void_p)]
 
 
 class ParkKernelTime(ctypes.Structure):

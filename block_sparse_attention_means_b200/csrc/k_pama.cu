@@ -191,8 +191,11 @@ __global__ __launch_bounds__(128) void k_pama_mma(const uint16_t* __restrict__ Q
     }
     if (threadIdx.x == 0) {
         float qm = fmaxf(fmaxf(s_dmax[0], s_dmax[1]), fmaxf(s_dmax[2], s_dmax[3]));
-        double delta = (double)delta_scale * qm * cmax;  // logit error bound (natural log units)
-        double rr = expm1(2.0 * delta) + 1.6e-5 + (24.0 + nr / 64.0) * 1.2e-7;
+        // logit error bound (natural log units); then exp2 approximations (2^-21
+        // relative each, numerator and denominator), products, and the float32
+        // column sums (within-warp adds, one add per tile, warp sum, division)
+        double delta = (double)delta_scale * qm * cmax;
+        double rr = expm1(2.0 * delta) + 4.0 * 4.76837158203125e-7 + (16.0 + nr / 64.0) * 5.9604644775390625e-8;
         rho[(size_t)bh * NQ + r] = (float)(rr * 1.001);
     }
 }
@@ -206,8 +209,15 @@ int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t*
     cudaFuncSetAttribute(k_pama_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     float scale = 1.0f / sqrtf((float)D);
     float sl2e = scale * kLog2e;
-    // |logit~ - logit| <= s * (D 2^-23 + 2^-22) ||q|| max||c||  (tensor-core accumulation, scaling)
-    float delta_scale = (float)((1.0 / sqrt((double)D)) * ((double)D * 1.1920929e-7 * 1.01 + 2.4e-7));
+    // |logit~ - logit| <= s (kappa 2^-24 + 2^-23) ||q|| max||c||: tensor-core fp32
+    // accumulation modelled as at most 2 half-ulps of the partial-sum bound per
+    // k-step (kappa = 2 D / 16 = 16 for D = 128; five times the largest error
+    // measured on this GPU over 8.4M bf16 dot products), plus the rounding of
+    // the scaled logit.  The GPU tests check the oracle's importance lies
+    // inside the resulting per-row bound.
+    const double kappa = 2.0 * D / 16.0;
+    float delta_scale =
+        (float)((1.0 / sqrt((double)D)) * (kappa * 5.9604644775390625e-8 + 1.1920928955078125e-7) * 1.01);
     ::park::prof_begin(st);
     k_pama_mma<<<dim3(NQ, BH), 128, sm, st>>>((const uint16_t*)Q, q_perm, q_off, (const uint16_t*)CK, k_off, qnorm,
                                               ckmax, N, NQ, NK, sl2e, delta_scale, importance, rho);
@@ -253,8 +263,8 @@ static int next_pow2(int x) {
 __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importance, const float* __restrict__ rho,
                                               const int32_t* __restrict__ q_off, const int32_t* __restrict__ k_off,
                                               int NQ, int NK, int NKP, float p, uint8_t* __restrict__ mask,
-                                              int32_t* __restrict__ kept_cnt, int32_t* __restrict__ flag_list,
-                                              int32_t* __restrict__ flag_count) {
+                                              int32_t* __restrict__ kept_cnt, float* __restrict__ importance_bound,
+                                              int32_t* __restrict__ flag_list, int32_t* __restrict__ flag_count) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     double* S = reinterpret_cast<double*>(smem_raw);       // [NKP] inclusive prefix sums
     float* sv = reinterpret_cast<float*>(S + NKP);         // [NKP]
@@ -269,7 +279,10 @@ __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importan
     const int nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - q_off[(size_t)bh * (NQ + 1) + r];
     if (nr == 0) {
         for (int m = t; m < NK; m += blockDim.x) mrow[m] = 0;
-        if (t == 0) kept_cnt[row] = 0;
+        if (t == 0) {
+            kept_cnt[row] = 0;
+            if (importance_bound) importance_bound[row] = 0.f;
+        }
         return;
     }
     const int32_t* ko = k_off + (size_t)bh * (NK + 1);
@@ -350,51 +363,64 @@ __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importan
     for (int e = t; e <= cut; e += blockDim.x) keep[si[e]] = 1;
     __syncthreads();
     for (int m = t; m < NK; m += blockDim.x) mrow[m] = keep[m];
-    if (t == 0) kept_cnt[row] = cut + 1;
+    if (t == 0) {
+        kept_cnt[row] = cut + 1;
+        if (importance_bound) importance_bound[row] = rho[row];
+    }
 }
 
 int launch_topp(const float* importance, const float* rho, int BH, int NQ, int NK, const int32_t* q_off,
-                const int32_t* k_off, float p, uint8_t* mask, int32_t* kept_cnt, int32_t* flag_list,
-                int32_t* flag_count, cudaStream_t st) {
+                const int32_t* k_off, float p, uint8_t* mask, int32_t* kept_cnt, float* importance_bound,
+                int32_t* flag_list, int32_t* flag_count, cudaStream_t st) {
     int NKP = next_pow2(NK);
     if (NKP < 512) NKP = 512;
     size_t sm = (size_t)NKP * (8 + 4 + 4 + 1) + 16;
     cudaFuncSetAttribute(k_topp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     ::park::prof_begin(st);
-    k_topp<<<dim3(NQ, BH), 512, sm, st>>>(importance, rho, q_off, k_off, NQ, NK, NKP, p, mask, kept_cnt, flag_list,
-                                          flag_count);
+    k_topp<<<dim3(NQ, BH), 512, sm, st>>>(importance, rho, q_off, k_off, NQ, NK, NKP, p, mask, kept_cnt,
+                                          importance_bound, flag_list, flag_count);
     PARK_TRY_LAUNCH("k_topp", st);
     return PARK_OK;
 }
 
 // ---------------------------------------------------------------- float64 PAMA + top-p
-// One CTA (256 threads) per listed (head, query cluster), or per cluster of
-// every head when all_clusters is set.  Thread t owns key clusters
-// m = t, t + 256, ...: for each member query it forms s (q . c_m) in float64,
-// the block takes the max and the sum of exp (fixed reduction tree), and the
-// thread adds P_im to its own columns.  Then I is sorted (descending, ties by
-// m) and a sequential float64 running sum finds the cut, exactly as the
-// definition reads.
+// One CTA (256 threads, persistent over the list) per listed (head, query
+// cluster), or per cluster of every head when all_clusters is set.  The
+// cluster's rows are staged 64 at a time in shared memory as float64 and the
+// key centroids stream through in chunks of 64.  Thread t owns the 4 x 4 logit
+// block rows 4*(t/16)+i, columns (t%16)+16u of the 64 x 64 tile.
+//   pass 1: per-row max and sum of exp over every non-empty key cluster
+//           (online per thread, then merged over the 16 threads of a row group);
+//   pass 2: P = exp(z - max) / sum, summed over the rows into per-row-group
+//           column partials that are added in a fixed order.
+// Then I = column sums / |Q_r| is sorted (descending, ties by m) and a
+// sequential float64 running sum finds the cut, as the definition reads.
+constexpr int F64_TILE = 64, F64_LD = 129;  // padded rows: conflict-free column reads
+
 template <typename T>
-__global__ __launch_bounds__(256) void k_pama_f64(const T* __restrict__ Q, const int32_t* __restrict__ q_perm,
-                                                  const int32_t* __restrict__ q_off, const T* __restrict__ CK,
-                                                  const int32_t* __restrict__ k_off, int N, int D, int NQ, int NK,
-                                                  int NKP, double scale, float p, const int32_t* __restrict__ list,
-                                                  const int32_t* __restrict__ count_ptr, int all_clusters,
-                                                  int BHNQ, float* __restrict__ importance,
-                                                  uint8_t* __restrict__ mask, int32_t* __restrict__ kept_cnt,
-                                                  int64_t* __restrict__ counters) {
-    constexpr int MAXU = 16;  // NK <= 4096 = 16 * 256
+__global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, const int32_t* __restrict__ q_perm,
+                                                     const int32_t* __restrict__ q_off, const T* __restrict__ CK,
+                                                     const int32_t* __restrict__ k_off, int N, int D, int NQ, int NK,
+                                                     int NKP, double scale, float p, const int32_t* __restrict__ list,
+                                                     const int32_t* __restrict__ count_ptr, int all_clusters,
+                                                     int BHNQ, float* __restrict__ importance,
+                                                     float* __restrict__ importance_bound,
+                                                     uint8_t* __restrict__ mask, int32_t* __restrict__ kept_cnt,
+                                                     int64_t* __restrict__ counters) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    double* Iv = reinterpret_cast<double*>(smem_raw);      // [NKP]
-    int32_t* si = reinterpret_cast<int32_t*>(Iv + NKP);    // [NKP]
-    double* qv = reinterpret_cast<double*>(si + NKP);      // [128]
-    __shared__ double red[8];
+    double* Qs = reinterpret_cast<double*>(smem_raw);         // [64][129]
+    double* Cs = Qs + F64_TILE * F64_LD;                      // [64][129]
+    double* Isum = Cs + F64_TILE * F64_LD;                    // [NKP]
+    double* part = Isum + NKP;                                // [16][64]
+    int32_t* si = reinterpret_cast<int32_t*>(part + 16 * 64); // [NKP]
+    uint8_t* live = reinterpret_cast<uint8_t*>(si + NKP);     // [NKP]
     __shared__ int s_cut;
-    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const double NEG_INF = __longlong_as_double(0xfff0000000000000ll);
+    const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
     const int count = all_clusters ? BHNQ : *count_ptr;
     if (blockIdx.x == 0 && t == 0 && !all_clusters && counters)
         atomicAdd((unsigned long long*)(counters + PARK_CNT_PAMA_RECHECK), (unsigned long long)count);
+    const int nch = (NK + F64_TILE - 1) / F64_TILE;
     for (int e = blockIdx.x; e < count; e += gridDim.x) {
         const int row = all_clusters ? e : list[e];
         const int bh = row / NQ, r = row - bh * NQ;
@@ -402,108 +428,162 @@ __global__ __launch_bounds__(256) void k_pama_f64(const T* __restrict__ Q, const
         const int32_t* ko = k_off + (size_t)bh * (NK + 1);
         uint8_t* mrow = mask + (size_t)row * NK;
         float* Irow = importance + (size_t)row * NK;
+        __syncthreads();  // previous entry's shared memory fully consumed
         if (nr == 0) {
             for (int m = t; m < NK; m += blockDim.x) {
                 mrow[m] = 0;
                 Irow[m] = 0.f;
             }
-            if (t == 0) kept_cnt[row] = 0;
-            __syncthreads();
+            if (t == 0) {
+                kept_cnt[row] = 0;
+                if (importance_bound) importance_bound[row] = 0.f;
+            }
             continue;
         }
-        double acc[MAXU];
-        bool lv[MAXU];
-#pragma unroll
-        for (int u = 0; u < MAXU; ++u) {
-            int m = t + 256 * u;
-            acc[u] = 0.0;
-            lv[u] = m < NK && ko[m + 1] > ko[m];
+        for (int m = t; m < NKP; m += blockDim.x) {
+            Isum[m] = 0.0;
+            live[m] = (m < NK && ko[m + 1] > ko[m]) ? 1 : 0;
         }
         const T* Ch = CK + (size_t)bh * NK * D;
-        for (int i = 0; i < nr; ++i) {
-            const int tok = q_perm[(size_t)bh * N + qs + i];
-            __syncthreads();
-            if (t < D) qv[t] = Elem<T>::to_double(Q + ((size_t)bh * N + tok) * D, t);
-            __syncthreads();
-            double z[MAXU];
-            double zm = -1.0 / 0.0;
+        const T* Qh = Q + (size_t)bh * N * D;
+        const int32_t* pm = q_perm + (size_t)bh * N + qs;
+        auto load_chunk = [&](int c) {
+            for (int idx = t; idx < F64_TILE * D; idx += blockDim.x) {
+                int cc = idx / D, j = idx - cc * D, m = c * F64_TILE + cc;
+                Cs[cc * F64_LD + j] = m < NK ? Elem<T>::to_double(Ch + (size_t)m * D, j) : 0.0;
+            }
+        };
+        auto logits = [&](double (&z)[4][4]) {
 #pragma unroll
-            for (int u = 0; u < MAXU; ++u) {
-                int m = t + 256 * u;
-                z[u] = -1.0 / 0.0;
-                if (m < NK && lv[u]) {
-                    const T* c = Ch + (size_t)m * D;
-                    double s = 0.0;
-                    for (int j = 0; j < D; ++j) s = __fma_rn(qv[j], Elem<T>::to_double(c, j), s);
-                    z[u] = scale * s;
-                    zm = fmax(zm, z[u]);
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) z[i][u] = 0.0;
+            for (int j = 0; j < D; ++j) {
+                double a[4], b[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a[i] = Qs[(ty * 4 + i) * F64_LD + j];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) b[u] = Cs[(tx + 16 * u) * F64_LD + j];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) z[i][u] = __fma_rn(a[i], b[u], z[i][u]);
+            }
+        };
+        for (int t0 = 0; t0 < nr; t0 += F64_TILE) {
+            __syncthreads();  // Qs free
+            for (int idx = t; idx < F64_TILE * D; idx += blockDim.x) {
+                int rr = idx / D, j = idx - rr * D;
+                Qs[rr * F64_LD + j] = t0 + rr < nr ? Elem<T>::to_double(Qh + (size_t)pm[t0 + rr] * D, j) : 0.0;
+            }
+            double mx[4], sm[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                mx[i] = NEG_INF;
+                sm[i] = 0.0;
+            }
+            for (int c = 0; c < nch; ++c) {  // pass 1
+                __syncthreads();
+                load_chunk(c);
+                __syncthreads();
+                double z[4][4];
+                logits(z);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int col = c * F64_TILE + tx + 16 * u;
+                    if (col < NK && live[col]) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            double zz = scale * z[i][u];
+                            if (zz > mx[i]) {
+                                sm[i] = sm[i] * exp(mx[i] - zz) + 1.0;
+                                mx[i] = zz;
+                            } else {
+                                sm[i] += exp(zz - mx[i]);
+                            }
+                        }
+                    }
                 }
             }
-            zm = warp_max(zm);
-            if (lane == 0) red[w] = zm;
-            __syncthreads();
-            zm = red[0];
-            for (int q = 1; q < 8; ++q) zm = fmax(zm, red[q]);
-            __syncthreads();
-            double ls = 0.0;
 #pragma unroll
-            for (int u = 0; u < MAXU; ++u) {
-                z[u] = (t + 256 * u < NK && lv[u]) ? exp(z[u] - zm) : 0.0;
-                ls += z[u];
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) {
+                    double m2 = __shfl_xor_sync(0xffffffffu, mx[i], o, 16);
+                    double s2 = __shfl_xor_sync(0xffffffffu, sm[i], o, 16);
+                    double M = fmax(mx[i], m2);
+                    if (M != NEG_INF) {
+                        sm[i] = sm[i] * exp(mx[i] - M) + s2 * exp(m2 - M);
+                        mx[i] = M;
+                    }
+                }
             }
-            ls = warp_sum(ls);
-            if (lane == 0) red[w] = ls;
-            __syncthreads();
-            ls = 0.0;
-            for (int q = 0; q < 8; ++q) ls += red[q];
+            double inv[4];
 #pragma unroll
-            for (int u = 0; u < MAXU; ++u) acc[u] += z[u] / ls;
+            for (int i = 0; i < 4; ++i) inv[i] = (t0 + ty * 4 + i < nr) ? 1.0 / sm[i] : 0.0;
+            for (int c = 0; c < nch; ++c) {  // pass 2
+                __syncthreads();
+                load_chunk(c);
+                __syncthreads();
+                double z[4][4];
+                logits(z);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int col = c * F64_TILE + tx + 16 * u;
+                    double cs = 0.0;
+                    if (col < NK && live[col]) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) cs += exp(scale * z[i][u] - mx[i]) * inv[i];
+                    }
+                    part[ty * F64_TILE + tx + 16 * u] = cs;
+                }
+                __syncthreads();
+                if (t < F64_TILE) {
+                    double s = 0.0;
+                    for (int q = 0; q < 16; ++q) s += part[q * F64_TILE + t];
+                    const int col = c * F64_TILE + t;
+                    if (col < NK) Isum[col] += s;
+                }
+            }
         }
-        // I row, then sort and cut
+        __syncthreads();
         for (int m = t; m < NKP; m += blockDim.x) {
+            const bool lv = live[m] != 0;
+            const double iv = lv ? Isum[m] / (double)nr : -1.0;
+            if (m < NK) Irow[m] = lv ? (float)iv : 0.f;
+            Isum[m] = iv;
             si[m] = m;
-            Iv[m] = -1.0;
         }
         __syncthreads();
-#pragma unroll
-        for (int u = 0; u < MAXU; ++u) {
-            int m = t + 256 * u;
-            if (m < NK) {
-                double iv = acc[u] / (double)nr;
-                Irow[m] = lv[u] ? (float)iv : 0.f;
-                if (lv[u]) Iv[m] = iv;
-            }
-        }
-        __syncthreads();
-        bitonic_desc<double>(Iv, si, NKP);
+        bitonic_desc<double>(Isum, si, NKP);
         if (t == 0) {
             double run = 0.0;
             int cut = -1;
-            for (int q = 0; q < NKP && Iv[q] >= 0.0; ++q) {
+            for (int q = 0; q < NKP && Isum[q] >= 0.0; ++q) {
                 cut = q;
-                run += Iv[q];
+                run += Isum[q];
                 if (p < 1.0f && run >= (double)p) break;
             }
             s_cut = cut;
+            kept_cnt[row] = cut + 1;
+            if (importance_bound) importance_bound[row] = 0.f;
         }
         __syncthreads();
         const int cut = s_cut;
         for (int m = t; m < NK; m += blockDim.x) mrow[m] = 0;
         __syncthreads();
         for (int q = t; q <= cut; q += blockDim.x) mrow[si[q]] = 1;
-        if (t == 0) kept_cnt[row] = cut + 1;
-        __syncthreads();
     }
 }
 
 int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int NK, const int32_t* q_perm,
                     const int32_t* q_off, const void* CK, const int32_t* k_off, float p, const int32_t* list,
-                    const int32_t* count, int all_clusters, int num_sms, float* importance, uint8_t* mask,
-                    int32_t* kept_cnt, int64_t* counters, cudaStream_t st) {
+                    const int32_t* count, int all_clusters, int num_sms, float* importance, float* importance_bound,
+                    uint8_t* mask, int32_t* kept_cnt, int64_t* counters, cudaStream_t st) {
     if (NK > 4096 || D > 128) return PARK_ERR_UNSUPPORTED;
     int NKP = next_pow2(NK);
-    size_t sm = (size_t)NKP * 12 + 128 * 8;
-    int blocks = num_sms * 4;
+    size_t sm = (size_t)2 * F64_TILE * F64_LD * 8 + (size_t)NKP * 8 + 16 * 64 * 8 + (size_t)NKP * 4 + NKP;
+    int blocks = num_sms;
     double scale = 1.0 / sqrt((double)D);
     if (dtype == PARK_BF16)
         cudaFuncSetAttribute(k_pama_f64<bf16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
@@ -513,11 +593,11 @@ int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int 
     if (dtype == PARK_BF16) {
         k_pama_f64<bf16_t><<<blocks, 256, sm, st>>>((const bf16_t*)Q, q_perm, q_off, (const bf16_t*)CK, k_off, N, D,
                                                     NQ, NK, NKP, scale, p, list, count, all_clusters, BH * NQ,
-                                                    importance, mask, kept_cnt, counters);
+                                                    importance, importance_bound, mask, kept_cnt, counters);
     } else {
         k_pama_f64<float><<<blocks, 256, sm, st>>>((const float*)Q, q_perm, q_off, (const float*)CK, k_off, N, D, NQ,
                                                    NK, NKP, scale, p, list, count, all_clusters, BH * NQ, importance,
-                                                   mask, kept_cnt, counters);
+                                                   importance_bound, mask, kept_cnt, counters);
     }
     PARK_TRY_LAUNCH("k_pama_f64", st);
     return PARK_OK;

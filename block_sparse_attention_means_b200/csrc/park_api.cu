@@ -306,14 +306,15 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
         PARK_CHECK(launch_pama_mma(Q, BH, N, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids, out->k_offsets,
                                    at<float>(ws, w.xnorm_q), out->importance, at<float>(ws, w.rho), ops.wmax, st));
         PARK_CHECK(launch_topp(out->importance, at<float>(ws, w.rho), BH, NQ, NK, out->q_offsets, out->k_offsets, p,
-                               out->mask, kcnt, at<int32_t>(ws, w.plist), at<int32_t>(ws, w.pcnt), st));
+                               out->mask, kcnt, out->importance_bound, at<int32_t>(ws, w.plist),
+                               at<int32_t>(ws, w.pcnt), st));
         PARK_CHECK(launch_pama_f64(Q, d.dtype, BH, N, D, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids,
                                    out->k_offsets, p, at<int32_t>(ws, w.plist), at<int32_t>(ws, w.pcnt), 0, num_sms,
-                                   out->importance, out->mask, kcnt, out->counters, st));
+                                   out->importance, out->importance_bound, out->mask, kcnt, out->counters, st));
     } else {
         PARK_CHECK(launch_pama_f64(Q, d.dtype, BH, N, D, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids,
-                                   out->k_offsets, p, nullptr, nullptr, 1, num_sms, out->importance, out->mask, kcnt,
-                                   out->counters, st));
+                                   out->k_offsets, p, nullptr, nullptr, 1, num_sms, out->importance,
+                                   out->importance_bound, out->mask, kcnt, out->counters, st));
     }
     PARK_CHECK(launch_kept_csr(out->mask, kcnt, BH, NQ, NK, out->kept_ptr, out->kept_idx, out->counters, st));
     return PARK_OK;

@@ -60,6 +60,7 @@ class Retrieval:
     kept_ptr: torch.Tensor
     kept_idx: torch.Tensor
     metric: torch.Tensor | None
+    importance_bound: torch.Tensor | None
     counters: torch.Tensor
     status: torch.Tensor
     flags: int = 0
@@ -69,7 +70,7 @@ class Retrieval:
         return _lib.ParkRetrieval(self.flags, p(self.q_labels), p(self.k_labels), p(self.q_perm), p(self.k_perm),
                                   p(self.q_offsets), p(self.k_offsets), p(self.q_centroids), p(self.k_centroids),
                                   p(self.importance), p(self.mask), p(self.kept_ptr), p(self.kept_idx),
-                                  p(self.metric), p(self.counters), p(self.status))
+                                  p(self.metric), p(self.importance_bound), p(self.counters), p(self.status))
 
     def status_code(self) -> int:
         return int(self.status.item())
@@ -88,6 +89,7 @@ def alloc_retrieval(shape: Shape, NQ: int, NK: int, device, with_metric: bool = 
         mask=torch.empty(B, H, NQ, NK, dtype=torch.uint8, device=device),
         kept_ptr=torch.empty(B, H, NQ + 1, **i32), kept_idx=torch.empty(B, H, NQ * NK, **i32),
         metric=torch.empty(B, H, D, D, dtype=torch.float64, device=device) if with_metric else None,
+        importance_bound=torch.empty(B, H, NQ, dtype=torch.float32, device=device),
         counters=torch.zeros(_lib.PARK_NUM_COUNTERS, dtype=torch.int64, device=device),
         status=torch.zeros(1, dtype=torch.int32, device=device))
 

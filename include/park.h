@@ -117,6 +117,9 @@ typedef struct {
     int32_t *kept_idx;     /* [B,H,NQ*NK]  kept m per row, ascending; row r of
                               head bh starts at bh*NQ*NK + kept_ptr[bh*(NQ+1)+r]   */
     double *metric;        /* [B,H,D,D]    optional (may be NULL): the metric M   */
+    float *importance_bound; /* [B,H,NQ]   optional (may be NULL): relative error
+                              bound of row r of importance; 0 where the row was
+                              computed in float64                              */
     int64_t *counters;     /* [PARK_NUM_COUNTERS], zeroed by park_retrieve        */
     int32_t *status;       /* [1] device status word, zeroed by park_retrieve     */
 } park_retrieval;

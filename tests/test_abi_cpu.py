@@ -29,9 +29,9 @@ def test_library_exports_every_declared_function():
 
 
 def test_struct_layout_matches_header():
-    # park_shape: 8 ints; park_retrieval: uint32 flags + 15 pointers (padded)
+    # park_shape: 8 ints; park_retrieval: uint32 flags + 16 pointers (padded)
     assert ctypes.sizeof(_lib.ParkShape) == 32
-    assert ctypes.sizeof(_lib.ParkRetrieval) == 8 + 15 * 8
+    assert ctypes.sizeof(_lib.ParkRetrieval) == 8 + 16 * 8
     text = open(os.path.join(ROOT, "include", "park.h")).read()
     assert re.search(r"#define PARK_NUM_COUNTERS 8", text)
     for name in ("PARK_OK", "PARK_ERR_INVALID_ARG", "PARK_ERR_UNSUPPORTED", "PARK_ERR_WORKSPACE", "PARK_ERR_CUDA",

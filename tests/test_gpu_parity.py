@@ -33,6 +33,25 @@ def run_layer(park, cfg: LayerConfig, Q, K, V, p=None, NQ=None, NK=None, iters=N
     return O, r
 
 
+def check_importance_bound(r, ref):
+    """Every importance entry is within the row's reported relative bound of
+    the oracle's float64 value (plus the float32 rounding of the output)."""
+    imp = r.importance.cpu().numpy().astype(np.float64)
+    bound = r.importance_bound.cpu().numpy().astype(np.float64)
+    H = imp.shape[1]
+    worst = 0.0
+    for bh, h in enumerate(ref):
+        b, hh = divmod(bh, H)
+        want = h["importance"]
+        slack = (bound[b, hh][:, None] + 2.0 ** -23) * want + 1e-30
+        err = np.abs(imp[b, hh] - want)
+        assert np.all(err <= slack), f"bh={bh}: importance outside its bound"
+        live = (want > 0) & (bound[b, hh][:, None] > 0)  # rows certified in float32
+        if live.any():
+            worst = max(worst, float(np.max(err[live] / (bound[b, hh][:, None] * want + 1e-30)[live])))
+    print(f"importance error / bound: max {worst:.3g}")
+
+
 @pytest.mark.parametrize("name", ["tiny", "small"])
 def test_layer_matches_oracle(park, name):
     cfg = CONFIGS[name]
@@ -47,6 +66,7 @@ def test_layer_matches_oracle(park, name):
     cnt = r.counters.cpu().numpy()
     print(f"\n{name}: counters {cnt.tolist()}")
     assert not fails, "\n".join(fails[:20])
+    check_importance_bound(r, ref)
     worst, mean = pu.assert_output_close(O, ref, cfg.dtype == "f32")
     print(f"{name}: O max abs {worst:.3g} mean abs {mean:.3g}")
     pairs = sum(int(np.sum(np.bincount(h["q_labels"], minlength=cfg.NQ)[:, None] * h["mask"] *
