@@ -45,42 +45,55 @@ int launch_gather(const void* X, int dtype, int BH, int N, int D, const int32_t*
 
 // ---------------------------------------------------------------- schedule
 // One CTA per (query cluster, head): kv_pre[j] = sum of the sizes of the first
-// j kept key clusters; kv_len = their total; query tiles appended to the work
-// list.  Counters: attended query-key pairs and work items.
+// j kept key clusters (rounded up to multiples of 8 when pad8 is set); kv_len =
+// their total; query tiles appended to the work list.  Counters: attended
+// query-key pairs (unpadded) and work items.
 __global__ __launch_bounds__(256) void k_attn_schedule(int NQ, int NK, const int32_t* __restrict__ q_off,
                                                        const int32_t* __restrict__ k_off,
                                                        const int32_t* __restrict__ kept_ptr,
                                                        const int32_t* __restrict__ kept_idx,
                                                        int32_t* __restrict__ kv_pre, int32_t* __restrict__ kv_len,
                                                        WorkItem* __restrict__ items, int32_t* __restrict__ item_count,
-                                                       int64_t* __restrict__ counters, int tile_rows) {
-    __shared__ int wsum[8];
+                                                       int64_t* __restrict__ counters, int tile_rows, int pad8,
+                                                       const int32_t* __restrict__ poff, int Npad,
+                                                       int2* __restrict__ segs) {
+    __shared__ int wsum[8], wsum_u[8];
     const int r = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int qs = q_off[(size_t)bh * (NQ + 1) + r], nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - qs;
     const int kp0 = kept_ptr[(size_t)bh * (NQ + 1) + r], nk = kept_ptr[(size_t)bh * (NQ + 1) + r + 1] - kp0;
     const int32_t* kl = kept_idx + (size_t)bh * NQ * NK + kp0;
     int32_t* pre = kv_pre + (size_t)bh * NQ * NK + kp0;
     const int32_t* ko = k_off + (size_t)bh * (NK + 1);
+    auto padded = [&](int sz) { return pad8 ? (sz + 7) & ~7 : sz; };
     const int seg = (nk + 255) / 256, b0 = t * seg;
-    int loc = 0;
-    for (int e = b0; e < b0 + seg && e < nk; ++e) loc += ko[kl[e] + 1] - ko[kl[e]];
-    int incl = loc;
+    int loc = 0, loc_u = 0;
+    for (int e = b0; e < b0 + seg && e < nk; ++e) {
+        const int sz = ko[kl[e] + 1] - ko[kl[e]];
+        loc += padded(sz);
+        loc_u += sz;
+    }
+    int incl = loc, su = loc_u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
+        su += __shfl_xor_sync(0xffffffffu, su, o);
     }
     if (lane == 31) wsum[w] = incl;
+    if (lane == 0) wsum_u[w] = su;
     __syncthreads();
-    int woff = 0, total = 0;
+    int woff = 0, total = 0, total_u = 0;
     for (int q = 0; q < 8; ++q) {
         if (q < w) woff += wsum[q];
         total += wsum[q];
+        total_u += wsum_u[q];
     }
     int run = woff + incl - loc;
     for (int e = b0; e < b0 + seg && e < nk; ++e) {
+        const int m = kl[e], sz = ko[m + 1] - ko[m];
         pre[e] = run;
-        run += ko[kl[e] + 1] - ko[kl[e]];
+        if (segs) segs[(size_t)bh * NQ * NK + kp0 + e] = make_int2(bh * Npad + poff[(size_t)bh * (NK + 1) + m], sz);
+        run += padded(sz);
     }
     if (t == 0) {
         kv_len[(size_t)bh * NQ + r] = nr > 0 ? total : 0;
@@ -96,7 +109,7 @@ __global__ __launch_bounds__(256) void k_attn_schedule(int NQ, int NK, const int
                 items[base + q] = it;
             }
             atomicAdd((unsigned long long*)(counters + PARK_CNT_KEPT_PAIRS),
-                      (unsigned long long)nr * (unsigned long long)total);
+                      (unsigned long long)nr * (unsigned long long)total_u);
             atomicAdd((unsigned long long*)(counters + PARK_CNT_WORK_ITEMS), (unsigned long long)tiles);
         }
     }
@@ -104,11 +117,95 @@ __global__ __launch_bounds__(256) void k_attn_schedule(int NQ, int NK, const int
 
 int launch_attn_schedule(int BH, int NQ, int NK, const int32_t* q_off, const int32_t* k_off,
                          const int32_t* kept_ptr, const int32_t* kept_idx, int32_t* kv_pre, int32_t* kv_len,
-                         WorkItem* items, int32_t* item_count, int64_t* counters, int tile_rows, cudaStream_t st) {
+                         WorkItem* items, int32_t* item_count, int64_t* counters, int tile_rows, int pad8,
+                         const int32_t* poff, int Npad, int2* segs, cudaStream_t st) {
     ::park::prof_begin(st);
     k_attn_schedule<<<dim3(NQ, BH), 256, 0, st>>>(NQ, NK, q_off, k_off, kept_ptr, kept_idx, kv_pre, kv_len, items,
-                                                  item_count, counters, tile_rows);
+                                                  item_count, counters, tile_rows, pad8, poff, Npad, segs);
     PARK_TRY_LAUNCH("k_attn_schedule", st);
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- padded K/V
+// poff[bh][m] = sum over m' < m of ceil8(|B_m'|) (one CTA per head).
+__global__ __launch_bounds__(1024) void k_kv_pad_offsets(const int32_t* __restrict__ k_off, int NK,
+                                                         int32_t* __restrict__ poff) {
+    __shared__ int wsum[32];
+    const int bh = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int32_t* ko = k_off + (size_t)bh * (NK + 1);
+    int32_t* po = poff + (size_t)bh * (NK + 1);
+    const int seg = (NK + 1023) / 1024, b0 = t * seg;
+    int loc = 0;
+    for (int m = b0; m < b0 + seg && m < NK; ++m) loc += (ko[m + 1] - ko[m] + 7) & ~7;
+    int incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    int woff = 0;
+    for (int q = 0; q < w; ++q) woff += wsum[q];
+    int run = woff + incl - loc;
+    for (int m = b0; m < b0 + seg && m < NK; ++m) {
+        po[m] = run;
+        run += (ko[m + 1] - ko[m] + 7) & ~7;
+    }
+    if (b0 < NK && b0 + seg >= NK) po[NK] = run;
+}
+
+// Row copies into the padded layout (16-byte pieces) and zeros in the pad rows.
+__global__ void k_kv_pad_gather(const uint4* __restrict__ K, const uint4* __restrict__ V, int N, int NK, int Npad,
+                                size_t BH, const int32_t* __restrict__ k_perm, const int32_t* __restrict__ k_labels,
+                                const int32_t* __restrict__ k_off, const int32_t* __restrict__ poff,
+                                uint4* __restrict__ Kp, uint4* __restrict__ Vp) {
+    constexpr int VPR = 16;  // 16-byte pieces per 128-element bf16 row
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    const size_t rows = BH * (size_t)N;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < rows * VPR; e += stride) {
+        const size_t row = e / VPR;
+        const int pc = (int)(e - row * VPR);
+        const size_t bh = row / N;
+        const int pos = (int)(row - bh * N);
+        const int tok = k_perm[row];
+        const int m = k_labels[bh * N + tok];
+        const size_t dst = bh * Npad + poff[bh * (NK + 1) + m] + (pos - k_off[bh * (NK + 1) + m]);
+        Kp[dst * VPR + pc] = K[(bh * N + tok) * VPR + pc];
+        Vp[dst * VPR + pc] = V[(bh * N + tok) * VPR + pc];
+    }
+    // pad rows: at most 7 per cluster
+    const size_t pads = BH * (size_t)NK * 7 * VPR;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < pads; e += stride) {
+        const size_t q = e / VPR;
+        const int pc = (int)(e - q * VPR);
+        const size_t bhm = q / 7;
+        const int i = (int)(q - bhm * 7);
+        const size_t bh = bhm / NK;
+        const int m = (int)(bhm - bh * NK);
+        const int sz = k_off[bh * (NK + 1) + m + 1] - k_off[bh * (NK + 1) + m];
+        const int padn = ((sz + 7) & ~7) - sz;
+        if (i < padn) {
+            const size_t dst = bh * Npad + poff[bh * (NK + 1) + m] + sz + i;
+            Kp[dst * VPR + pc] = make_uint4(0, 0, 0, 0);
+            Vp[dst * VPR + pc] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+int launch_kv_pad_gather(const void* K, const void* V, int BH, int N, int NK, int Npad, const int32_t* k_perm,
+                         const int32_t* k_labels, const int32_t* k_off, int32_t* poff, void* Kpad, void* Vpad,
+                         cudaStream_t st) {
+    ::park::prof_begin(st);
+    k_kv_pad_offsets<<<BH, 1024, 0, st>>>(k_off, NK, poff);
+    PARK_TRY_LAUNCH("k_kv_pad_offsets", st);
+    size_t total = (size_t)BH * N * 16;
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    ::park::prof_begin(st);
+    k_kv_pad_gather<<<blocks, 256, 0, st>>>((const uint4*)K, (const uint4*)V, N, NK, Npad, (size_t)BH, k_perm,
+                                            k_labels, k_off, poff, (uint4*)Kpad, (uint4*)Vpad);
+    PARK_TRY_LAUNCH("k_kv_pad_gather", st);
     return PARK_OK;
 }
 

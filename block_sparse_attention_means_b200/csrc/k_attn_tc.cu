@@ -1,0 +1,475 @@
+// Block-sparse attention on the 5th-generation tensor cores (tcgen05 + TMEM +
+// TMA), bf16 inputs, D = 128.
+//
+// Layout: Q is gathered into cluster order (rows of a query cluster are
+// contiguous).  K and V are gathered into cluster order with every key
+// cluster padded to a multiple of 8 rows (zero rows), so a kept key cluster is
+// a run of whole 8-row groups.  For a query cluster, its kept key clusters are
+// concatenated (padded sizes) into one virtual key sequence that is cut into
+// full 128-row tiles: clusters smaller than a tile share a tile (the
+// gather-into-full-tiles idea of the AB-Attention article).  A 128-row key
+// tile is assembled by 16 TMA loads of 8-row boxes per 64-column half, for K
+// and for V; groups past the end load out of bounds (zero fill) and are masked.
+//
+// One CTA per SM (persistent, work items round-robin), 6 warps:
+//   warp 0     TMA producer: Q tile (128 x 128) per item, K/V tiles into a
+//              2-stage ring;
+//   warp 1     TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into one of
+//              two TMEM buffers (128 x 128 fp32), then O += P_j V_j into a TMEM
+//              accumulator (128 x 128 fp32);
+//   warps 2-5  Softmax: thread = query row = TMEM lane.  Loads S_j, online
+//              Softmax in the log2 domain with a lazily updated reference max
+//              (O is rescaled in TMEM only when the row max grows by more than
+//              2^8), writes P_j as bf16 into shared memory in the swizzled
+//              K-major layout of the next MMA, and finally normalises O and
+//              writes the row in original token order.
+// Every wait is time-bounded; a timeout sets PARK_ERR_TIMEOUT in the status
+// word, the roles leave their loops, outstanding copies and MMAs are waited
+// for (bounded) and TMEM is freed before the CTA exits.
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace park {
+
+using namespace sm100;
+
+namespace {
+constexpr int TC_ROWS = 128;       // query rows and key rows per tile
+constexpr int TC_BLK = 16384;      // one 128-row x 64-column bf16 block (128 B rows)
+constexpr int TC_STAGES = 2;
+constexpr uint32_t TC_TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256,384)
+constexpr float kLog2eT = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
+
+struct TcSmem {
+    uint64_t q_full, q_empty, kv_full[TC_STAGES], kv_empty[TC_STAGES], s_full[2], s_empty[2], p_full, o_done,
+        o_empty, final_bar;
+    uint32_t tmem_base;
+    int abort;
+    uint8_t valid[TC_STAGES][16];  // per-stage validity of the 128 key rows (bit i of byte g: row 8g+i)
+};
+}  // namespace
+
+__device__ __forceinline__ float bits_f(uint32_t u) { return __uint_as_float(u); }
+// warp-uniform view of the abort flag
+__device__ __forceinline__ bool warp_abort(volatile int* abort) { return __any_sync(0xffffffffu, *abort != 0); }
+
+__global__ void __launch_bounds__(192, 1)
+    k_sparse_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, int N, int NQ, int NK, int Npad, int BH,
+                     const int32_t* __restrict__ q_perm, const int2* __restrict__ segs,
+                     const int32_t* __restrict__ kept_ptr, const int32_t* __restrict__ kv_pre,
+                     const int32_t* __restrict__ kv_len, const WorkItem* __restrict__ items,
+                     const int32_t* __restrict__ item_count, uint16_t* __restrict__ O, float sl2e,
+                     int32_t* __restrict__ status) {
+    extern __shared__ __align__(1024) uint8_t dsmem_raw[];
+    __shared__ TcSmem sh;
+    // 1024-byte aligned operand area: Q | K0 V0 K1 V1 | P
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* Qs = base;                                  // 2 blocks
+    uint8_t* KVs = base + 2 * TC_BLK;                    // per stage: K 2 blocks, V 2 blocks
+    uint8_t* Ps = base + 2 * TC_BLK + TC_STAGES * 4 * TC_BLK;  // 2 blocks
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* abort = &sh.abort;
+    if (threadIdx.x == 0) {
+        mbar_init(&sh.q_full, 1);
+        mbar_init(&sh.q_empty, 1);
+        for (int s = 0; s < TC_STAGES; ++s) {
+            mbar_init(&sh.kv_full[s], 1);
+            mbar_init(&sh.kv_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sh.s_full[b], 1);
+            mbar_init(&sh.s_empty[b], 128);
+        }
+        mbar_init(&sh.p_full, 128);
+        mbar_init(&sh.o_done, 1);
+        mbar_init(&sh.o_empty, 128);
+        mbar_init(&sh.final_bar, 1);
+        sh.abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(&sh.tmem_base, TC_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    const int n_items = *item_count;
+    const uint32_t idS = idesc_bf16(128, 128, 0, 0);  // S = Q K^T: both K-major
+    const uint32_t idPV = idesc_bf16(128, 128, 0, 1);  // O += P V: P K-major, V MN-major
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int T = 0, I = 0;
+        int last_parity[TC_STAGES] = {-1, -1};
+        int q_pending = 0, q_parity = 0;
+        for (int it = blockIdx.x; it < n_items && !warp_abort(abort); it += gridDim.x) {
+            const WorkItem wi = items[it];
+            const int L = kv_len[(size_t)wi.bh * NQ + wi.r];
+            const int nkt = (L + TC_ROWS - 1) / TC_ROWS;
+            if (nkt == 0) continue;
+            const int kp0 = kept_ptr[(size_t)wi.bh * (NQ + 1) + wi.r];
+            const int nk = kept_ptr[(size_t)wi.bh * (NQ + 1) + wi.r + 1] - kp0;
+            const int32_t* pre = kv_pre + (size_t)wi.bh * NQ * NK + kp0;
+            const int2* segs_item = segs + (size_t)wi.bh * NQ * NK + kp0;
+            if (lane == 0) {
+                bool ok = I == 0 || mbar_wait(&sh.q_empty, (I - 1) & 1, abort);
+                if (ok) {
+                    mbar_arrive_expect_tx(&sh.q_full, 2 * TC_BLK);
+                    const int y = wi.bh * N + wi.q_start;
+                    tma_load_2d(Qs, &tmQ, &sh.q_full, 0, y);
+                    tma_load_2d(Qs + TC_BLK, &tmQ, &sh.q_full, 64, y);
+                    q_pending = 1;
+                    q_parity = I & 1;
+                }
+            }
+            __syncwarp();
+            if (warp_abort(abort)) break;
+            // Segment cursor: lane l holds entry seg0 + l of the item's kept
+            // segments (prefix of padded sizes, first padded row, size); a tile
+            // spans at most 17 segments (each is >= 8 rows), so 32 lanes cover it.
+            int seg0 = 0, p_l = 0x7fffffff, src_l = 0, sz_l = 0;
+            auto load_entries = [&](int s0) {
+                const int idx = s0 + lane;
+                if (idx < nk) {
+                    p_l = pre[idx];
+                    const int2 e = segs_item[idx];
+                    src_l = e.x;
+                    sz_l = e.y;
+                } else {
+                    p_l = 0x7fffffff;
+                    src_l = 0;
+                    sz_l = 0;
+                }
+            };
+            load_entries(0);
+            for (int j = 0; j < nkt; ++j) {
+                const int stg = T & 1, round = T >> 1;
+                int y = BH * Npad;  // out of bounds: zero fill
+                uint8_t vmask = 0;
+#pragma unroll 4
+                for (int g = 0; g < 16; ++g) {
+                    const int vg = j * TC_ROWS + 8 * g;
+                    const unsigned bal = __ballot_sync(0xffffffffu, p_l <= vg);
+                    const int idx = (__popc(bal) - 1) & 31;
+                    const int pp = __shfl_sync(0xffffffffu, p_l, idx);
+                    const int src = __shfl_sync(0xffffffffu, src_l, idx);
+                    const int sz = __shfl_sync(0xffffffffu, sz_l, idx);
+                    if (lane == g && vg < L) {
+                        const int o0 = vg - pp;
+                        int nv = sz - o0;
+                        nv = nv < 0 ? 0 : (nv > 8 ? 8 : nv);
+                        vmask = (uint8_t)((1u << nv) - 1u);
+                        y = src + o0;
+                    }
+                }
+                {  // advance the cursor and prefetch the next tile's entries
+                    const int vn = (j + 1) * TC_ROWS;
+                    if (vn < L) {
+                        const unsigned bal = __ballot_sync(0xffffffffu, p_l <= vn);
+                        seg0 += __popc(bal) - 1;
+                        load_entries(seg0);
+                    }
+                }
+                bool ok = true;
+                if (lane == 0 && round > 0) ok = mbar_wait(&sh.kv_empty[stg], (round - 1) & 1, abort);
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok || warp_abort(abort)) break;
+                if (lane < 16) sh.valid[stg][lane] = vmask;
+                __syncwarp();
+                if (lane == 0) mbar_arrive_expect_tx(&sh.kv_full[stg], 4 * TC_BLK);
+                __syncwarp();
+                if (lane < 16) {
+                    uint8_t* Kst = KVs + stg * 4 * TC_BLK;
+                    uint8_t* Vst = Kst + 2 * TC_BLK;
+                    tma_load_2d(Kst + lane * 1024, &tmK, &sh.kv_full[stg], 0, y);
+                    tma_load_2d(Kst + TC_BLK + lane * 1024, &tmK, &sh.kv_full[stg], 64, y);
+                    tma_load_2d(Vst + lane * 1024, &tmV, &sh.kv_full[stg], 0, y);
+                    tma_load_2d(Vst + TC_BLK + lane * 1024, &tmV, &sh.kv_full[stg], 64, y);
+                }
+                last_parity[stg] = round & 1;
+                ++T;
+            }
+            ++I;
+        }
+        // drain: copies still in flight complete before the CTA may exit
+        if (lane == 0) {
+            for (int s = 0; s < TC_STAGES; ++s)
+                if (last_parity[s] >= 0) {
+                    int dummy = 0;
+                    mbar_wait(&sh.kv_full[s], last_parity[s], &dummy, 100000000ull);
+                }
+            if (q_pending) {
+                int dummy = 0;
+                mbar_wait(&sh.q_full, q_parity, &dummy, 100000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int G = 0, I = 0;
+            const uint32_t qa = smem_u32(Qs), pa = smem_u32(Ps);
+            auto issue_S = [&](int g) -> bool {
+                const int stg = g & 1, round = g >> 1;
+                if (!mbar_wait(&sh.kv_full[stg], round & 1, abort)) return false;
+                if (round > 0 && !mbar_wait(&sh.s_empty[stg], (round - 1) & 1, abort)) return false;
+                tc_fence_after();
+                const uint32_t ka = smem_u32(KVs + stg * 4 * TC_BLK);
+                const uint32_t d = tmem + (uint32_t)(stg * 128);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (uint32_t)((kk >> 2) * TC_BLK + (kk & 3) * 32);
+                    umma_bf16(d, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
+                }
+                umma_commit(&sh.s_full[stg]);
+                return true;
+            };
+            for (int it = blockIdx.x; it < n_items && !*abort; it += gridDim.x) {
+                const WorkItem wi = items[it];
+                const int L = kv_len[(size_t)wi.bh * NQ + wi.r];
+                const int nkt = (L + TC_ROWS - 1) / TC_ROWS;
+                if (nkt == 0) continue;
+                if (!mbar_wait(&sh.q_full, I & 1, abort)) break;
+                tc_fence_after();
+                if (!issue_S(G)) break;
+                bool ok = true;
+                for (int j = 0; j < nkt && ok; ++j) {
+                    const int g = G + j;
+                    if (j + 1 < nkt && !issue_S(g + 1)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait(&sh.p_full, g & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (j == 0 && I > 0 && !mbar_wait(&sh.o_empty, (I - 1) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t va = smem_u32(KVs + (g & 1) * 4 * TC_BLK + 2 * TC_BLK);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t aoff = (uint32_t)((kk >> 2) * TC_BLK + (kk & 3) * 32);
+                        umma_bf16(tmem + 256, sdesc_sw128(pa + aoff, 16, 1024),
+                                  sdesc_sw128(va + (uint32_t)kk * 2048, TC_BLK, 1024), idPV, (j > 0 || kk > 0));
+                    }
+                    umma_commit(&sh.o_done);
+                    umma_commit(&sh.kv_empty[g & 1]);
+                }
+                if (!ok) break;
+                umma_commit(&sh.q_empty);
+                G += nkt;
+                ++I;
+            }
+            // every MMA issued so far has completed before TMEM is released
+            umma_commit(&sh.final_bar);
+            int dummy = 0;
+            mbar_wait(&sh.final_bar, 0, &dummy, 100000000ull);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int lane_base = 32 * (warp & 3);
+        const int row = lane_base + lane;
+        const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
+        int G = 0, I = 0;
+        // waits are decided per warp: tcgen05.ld and shuffles below are warp-collective
+        auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            const bool ok = mbar_wait(bar, parity, abort);
+            return __all_sync(0xffffffffu, ok);
+        };
+        for (int it = blockIdx.x; it < n_items && !warp_abort(abort); it += gridDim.x) {
+            const WorkItem wi = items[it];
+            const int L = kv_len[(size_t)wi.bh * NQ + wi.r];
+            const int nkt = (L + TC_ROWS - 1) / TC_ROWS;
+            if (nkt == 0) continue;
+            float m_ref = __int_as_float(0xff800000), l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < nkt; ++j) {
+                const int g = G + j, b = g & 1, round = g >> 1;
+                if (!wwait(&sh.s_full[b], round & 1) || !wwait(&sh.kv_full[b], round & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t s[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(trow + (uint32_t)(b * 128 + 32 * c), s[c]);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&sh.s_empty[b]);
+                const uint8_t* vb = sh.valid[b];
+                float tmax = __int_as_float(0xff800000);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int col = 32 * c + e;
+                        const bool v = (vb[col >> 3] >> (col & 7)) & 1;
+                        const float x = v ? bits_f(s[c][e]) * sl2e : __int_as_float(0xff800000);
+                        s[c][e] = __float_as_uint(x);
+                        tmax = fmaxf(tmax, x);
+                    }
+                }
+                bool waited = j == 0;
+                if (j == 0) {
+                    m_ref = tmax;
+                } else if (__any_sync(0xffffffffu, tmax > m_ref + kRescaleThreshold)) {
+                    // decided per warp: the TMEM loads/stores below are warp-collective;
+                    // rows that do not need a new reference keep theirs (alpha = 1)
+                    if (!wwait(&sh.o_done, (g - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    waited = true;
+                    tc_fence_after();
+                    const float m_new = tmax > m_ref + kRescaleThreshold ? tmax : m_ref;
+                    const float alpha = exp2f(m_ref - m_new);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(trow + 256u + 32u * c, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(bits_f(o[e]) * alpha);
+                        tmem_st32(trow + 256u + 32u * c, o);
+                    }
+                    tmem_st_wait();
+                    l *= alpha;
+                    m_ref = m_new;
+                }
+                if (!waited && !wwait(&sh.o_done, (g - 1) & 1)) {  // P buffer free
+                    ok = false;
+                    break;
+                }
+                // P row -> shared memory, K-major, 128-byte swizzle: chunk c16 of row r at c16 ^ (r & 7)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = exp2f(bits_f(s[c][2 * e]) - m_ref);
+                        const float p1 = exp2f(bits_f(s[c][2 * e + 1]) - m_ref);
+                        l += p0 + p1;
+                        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                        pk[e] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    uint8_t* blk = Ps + (c >> 1) * TC_BLK + row * 128;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int c16 = (c & 1) * 4 + q;
+                        *reinterpret_cast<uint4*>(blk + ((c16 ^ (row & 7)) << 4)) =
+                            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&sh.p_full);
+            }
+            if (!ok) break;
+            // epilogue: O / l, original token order
+            if (!wwait(&sh.o_done, (G + nkt - 1) & 1)) break;
+            tc_fence_after();
+            uint32_t o[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(trow + 256u + 32u * c, o[c]);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&sh.o_empty);
+            if (row < wi.rows) {
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+                const int tok = q_perm[(size_t)wi.bh * N + wi.q_start + row];
+                uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)wi.bh * N + tok) * 128);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            __nv_bfloat162 h = __floats2bfloat162_rn(bits_f(o[c][8 * q + 2 * e]) * inv,
+                                                                     bits_f(o[c][8 * q + 2 * e + 1]) * inv);
+                            w4[e] = *reinterpret_cast<uint32_t*>(&h);
+                        }
+                        dst[c * 4 + q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+            }
+            G += nkt;
+            ++I;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TC_TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && sh.abort) set_status(status, PARK_ERR_TIMEOUT);
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encoder() {
+    if (g_encode) return PARK_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn) {
+        cudaGetLastError();
+        return PARK_ERR_CUDA;
+    }
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return PARK_OK;
+}
+
+// 2-D bf16 tensor [rows][128], 128-byte swizzled boxes of 64 columns x box_rows.
+int make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t box_rows) {
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {128 * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PARK_OK : PARK_ERR_CUDA;
+}
+}  // namespace
+
+size_t attn_tc_smem_bytes() { return (size_t)(2 + TC_STAGES * 4 + 2) * TC_BLK + 1024; }
+
+int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
+                          const int32_t* q_perm, const int2* segs, const int32_t* kept_ptr, const int32_t* kv_pre,
+                          const int32_t* kv_len,
+                          const WorkItem* items, const int32_t* item_count, void* O, int32_t* status, int num_sms,
+                          cudaStream_t st) {
+    PARK_CHECK(get_encoder());
+    CUtensorMap mQ, mK, mV;
+    PARK_CHECK(make_map(&mQ, Qp, (uint64_t)BH * N, 128));
+    PARK_CHECK(make_map(&mK, Kpad, (uint64_t)BH * Npad, 8));
+    PARK_CHECK(make_map(&mV, Vpad, (uint64_t)BH * Npad, 8));
+    const size_t sm = attn_tc_smem_bytes();
+    cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    const float sl2e = (1.0f / sqrtf(128.f)) * kLog2eT;
+    ::park::prof_begin(st);
+    k_sparse_attn_tc<<<num_sms, 192, sm, st>>>(mQ, mK, mV, N, NQ, NK, Npad, BH, q_perm, segs, kept_ptr, kv_pre,
+                                                kv_len, items, item_count, (uint16_t*)O, sl2e, status);
+    PARK_TRY_LAUNCH("k_sparse_attn_tc", st);
+    return PARK_OK;
+}
+
+}  // namespace park

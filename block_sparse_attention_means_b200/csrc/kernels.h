@@ -70,9 +70,25 @@ struct WorkItem {
     int bh, r, q_start, rows;
 };
 int launch_gather(const void* X, int dtype, int BH, int N, int D, const int32_t* perm, void* Xp, cudaStream_t st);
+// pad8: key cluster sizes rounded up to multiples of 8 in kv_pre / kv_len (the
+// padded layout of the tensor-core kernel), and segs[j] = (first padded row of
+// the j-th kept cluster, its size) written from poff; the pair counter always
+// counts the unpadded keys.
 int launch_attn_schedule(int BH, int NQ, int NK, const int32_t* q_off, const int32_t* k_off,
                          const int32_t* kept_ptr, const int32_t* kept_idx, int32_t* kv_pre, int32_t* kv_len,
-                         WorkItem* items, int32_t* item_count, int64_t* counters, int tile_rows, cudaStream_t st);
+                         WorkItem* items, int32_t* item_count, int64_t* counters, int tile_rows, int pad8,
+                         const int32_t* poff, int Npad, int2* segs, cudaStream_t st);
+// K and V in key-cluster order with every cluster padded to a multiple of 8
+// rows (zeros): poff[bh][m] = first padded row of cluster m; Npad rows per head.
+int launch_kv_pad_gather(const void* K, const void* V, int BH, int N, int NK, int Npad, const int32_t* k_perm,
+                         const int32_t* k_labels, const int32_t* k_off, int32_t* poff, void* Kpad, void* Vpad,
+                         cudaStream_t st);
+size_t attn_tc_smem_bytes();
+int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
+                          const int32_t* q_perm, const int2* segs, const int32_t* kept_ptr, const int32_t* kv_pre,
+                          const int32_t* kv_len,
+                          const WorkItem* items, const int32_t* item_count, void* O, int32_t* status, int num_sms,
+                          cudaStream_t st);
 int launch_sparse_attn_mma(const void* Qp, const void* Kp, const void* Vp, int BH, int N, int NQ, int NK,
                            const int32_t* q_perm, const int32_t* k_off, const int32_t* kept_ptr,
                            const int32_t* kept_idx, const int32_t* kv_pre, const int32_t* kv_len,

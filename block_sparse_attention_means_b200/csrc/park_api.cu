@@ -105,7 +105,8 @@ struct Carver {
 };
 
 constexpr int kSortChunk = 1024;
-constexpr int kAttnTile = 64;
+constexpr int kAttnTile = 64;     // query rows per work item, float32 path
+constexpr int kAttnTileTc = 128;  // query rows per work item, tensor-core path
 
 int metric_chunks(const Dims& d) {
     int c = (2 * 148 + d.BH - 1) / d.BH;
@@ -149,20 +150,28 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
 }
 
 struct AttnWs {
-    size_t Qp, Kp, Vp, items, icnt, kvpre, kvlen, total;
+    size_t Qp, Kp, Vp, poff, segs, items, icnt, kvpre, kvlen, total;
+    int Npad;
 };
+
+// Rows per head of the padded key layout: every key cluster rounded up to a
+// multiple of 8 rows adds at most 7 rows per cluster.
+int padded_rows(const Dims& d, int NK) { return (int)align_up((size_t)d.N + 7 * (size_t)NK, 8); }
 
 AttnWs plan_attn(const Dims& d, int NQ, int NK) {
     AttnWs w;
     Carver c;
     size_t BH = d.BH, N = d.N, D = d.D;
     size_t rowbytes = D * d.elt;
+    w.Npad = padded_rows(d, NK);
     if (d.dtype == PARK_BF16) {
         w.Qp = c.take(BH * N * rowbytes);
-        w.Kp = c.take(BH * N * rowbytes);
-        w.Vp = c.take(BH * N * rowbytes);
+        w.Kp = c.take(BH * (size_t)w.Npad * rowbytes);
+        w.Vp = c.take(BH * (size_t)w.Npad * rowbytes);
+        w.poff = c.take(BH * (size_t)(NK + 1) * 4);
+        w.segs = c.take(BH * (size_t)NQ * NK * 8);
     } else {
-        w.Qp = w.Kp = w.Vp = 0;
+        w.Qp = w.Kp = w.Vp = w.poff = w.segs = 0;
     }
     size_t max_items = BH * ((N + kAttnTile - 1) / kAttnTile + (size_t)NQ);
     w.items = c.take(max_items * sizeof(WorkItem));
@@ -324,14 +333,15 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
               void* O, void* ws, cudaStream_t st) {
     const AttnWs w = plan_attn(d, NQ, NK);
     const int BH = d.BH, N = d.N, D = d.D;
+    const bool bf16 = d.dtype == PARK_BF16;
     PARK_CHECK(launch_input_check(V, (size_t)BH * N * D, d.dtype, r->status, st));
     PARK_CHECK(memset_async(r->counters + PARK_CNT_KEPT_PAIRS, 2 * sizeof(int64_t), st));
     int32_t* icnt = at<int32_t>(ws, w.icnt);
     PARK_CHECK(memset_async(icnt, 16 * 4, st));
-    PARK_CHECK(launch_attn_schedule(BH, NQ, NK, r->q_offsets, r->k_offsets, r->kept_ptr, r->kept_idx,
-                                    at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
-                                    icnt, r->counters, kAttnTile, st));
-    if (d.dtype != PARK_BF16) {
+    if (!bf16) {
+        PARK_CHECK(launch_attn_schedule(BH, NQ, NK, r->q_offsets, r->k_offsets, r->kept_ptr, r->kept_idx,
+                                        at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
+                                        icnt, r->counters, kAttnTile, 0, nullptr, 0, nullptr, st));
         return launch_sparse_attn_simt(Q, K, V, d.dtype, BH, N, D, NQ, NK, r->q_labels, r->k_perm, r->k_offsets,
                                        r->kept_ptr, r->kept_idx, O, st);
     }
@@ -339,12 +349,16 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
     void* Qp = at<void>(ws, w.Qp);
     void* Kp = at<void>(ws, w.Kp);
     void* Vp = at<void>(ws, w.Vp);
+    int32_t* poff = at<int32_t>(ws, w.poff);
+    int2* segs = at<int2>(ws, w.segs);
     PARK_CHECK(launch_gather(Q, d.dtype, BH, N, D, r->q_perm, Qp, st));
-    PARK_CHECK(launch_gather(K, d.dtype, BH, N, D, r->k_perm, Kp, st));
-    PARK_CHECK(launch_gather(V, d.dtype, BH, N, D, r->k_perm, Vp, st));
-    PARK_CHECK(launch_sparse_attn_mma(Qp, Kp, Vp, BH, N, NQ, NK, r->q_perm, r->k_offsets, r->kept_ptr, r->kept_idx,
-                                      at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
-                                      icnt, icnt + 1, O, num_sms, st));
+    PARK_CHECK(launch_kv_pad_gather(K, V, BH, N, NK, w.Npad, r->k_perm, r->k_labels, r->k_offsets, poff, Kp, Vp, st));
+    PARK_CHECK(launch_attn_schedule(BH, NQ, NK, r->q_offsets, r->k_offsets, r->kept_ptr, r->kept_idx,
+                                    at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
+                                    icnt, r->counters, kAttnTileTc, 1, poff, w.Npad, segs, st));
+    PARK_CHECK(launch_sparse_attn_tc(Qp, Kp, Vp, BH, N, w.Npad, NQ, NK, r->q_perm, segs, r->kept_ptr,
+                                     at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
+                                     icnt, O, r->status, num_sms, st));
     return PARK_OK;
 }
 

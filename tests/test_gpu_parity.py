@@ -175,6 +175,21 @@ def test_identity_clustering_pin(park):
         assert np.abs(pu.np64(O)[0, h] - dense).max() <= pu.O_MAX_ABS
 
 
+def test_large_logits_many_key_tiles(park):
+    """Queries scaled by 4 give logits whose row maxima keep growing across the
+    ~12 key tiles of a query tile, so the attention kernel rescales its
+    accumulator for some rows of a warp but not others."""
+    cfg = LayerConfig("wide", 1, 2, 8, 16, 16, 0, 128, "bf16", 6, 8, 3, 0.95, True, "normal")
+    Q, K, V = gen_layer(cfg, seed=12)
+    Q = (Q * 4.0).astype(np.float32)  # a power of two: still exact in bf16
+    ref = po.layer(Q, K, V, cfg.NQ, cfg.NK, cfg.p, cfg.iters, cfg.dtype)
+    O, r = run_layer(park, cfg, Q, K, V)
+    fails = pu.compare_retrieval(r, ref, cfg.NQ, cfg.NK)
+    assert not fails, "\n".join(fails[:20])
+    assert int(r.counters.cpu()[6]) >= cfg.NQ  # several query tiles
+    pu.assert_output_close(O, ref, False)
+
+
 def test_range_precondition_reported(park):
     cfg = RAGGED
     Q, K, V = gen_layer(cfg, seed=6)
