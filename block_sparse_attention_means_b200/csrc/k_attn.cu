@@ -155,14 +155,26 @@ __global__ __launch_bounds__(1024) void k_kv_pad_offsets(const int32_t* __restri
     if (b0 < NK && b0 + seg >= NK) po[NK] = run;
 }
 
-// Row copies into the padded layout (16-byte pieces) and zeros in the pad rows.
+// Row copies into the padded layout, stored as the byte image of the
+// tensor-core kernel's shared-memory tiles: padded row pp of a head lies in
+// 8-row group q = pp / 8 (2048 bytes at q * 2048), first the 64-column half 0
+// then half 1 (1024 bytes each); inside a half, row r = pp % 8 takes 128 bytes
+// at r * 128 and its 16-byte chunk c sits at chunk position c ^ r (the 128-byte
+// swizzle).  A run of whole groups is then one contiguous bulk copy.  Pad rows
+// are zeros.
+__device__ __forceinline__ size_t kv_image_chunk(size_t head_base_groups, int pp, int c) {
+    const int q = pp >> 3, r = pp & 7, h = c >> 3, c16 = c & 7;
+    return (head_base_groups + (size_t)q) * 128 + (size_t)h * 64 + (size_t)r * 8 + (size_t)(c16 ^ r);
+}
+
 __global__ void k_kv_pad_gather(const uint4* __restrict__ K, const uint4* __restrict__ V, int N, int NK, int Npad,
                                 size_t BH, const int32_t* __restrict__ k_perm, const int32_t* __restrict__ k_labels,
                                 const int32_t* __restrict__ k_off, const int32_t* __restrict__ poff,
                                 uint4* __restrict__ Kp, uint4* __restrict__ Vp) {
-    constexpr int VPR = 16;  // 16-byte pieces per 128-element bf16 row
+    constexpr int VPR = 16;  // 16-byte chunks per 128-element bf16 row
     const size_t stride = (size_t)gridDim.x * blockDim.x;
     const size_t rows = BH * (size_t)N;
+    const size_t gph = (size_t)Npad / 8;  // groups per head
     for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < rows * VPR; e += stride) {
         const size_t row = e / VPR;
         const int pc = (int)(e - row * VPR);
@@ -170,9 +182,10 @@ __global__ void k_kv_pad_gather(const uint4* __restrict__ K, const uint4* __rest
         const int pos = (int)(row - bh * N);
         const int tok = k_perm[row];
         const int m = k_labels[bh * N + tok];
-        const size_t dst = bh * Npad + poff[bh * (NK + 1) + m] + (pos - k_off[bh * (NK + 1) + m]);
-        Kp[dst * VPR + pc] = K[(bh * N + tok) * VPR + pc];
-        Vp[dst * VPR + pc] = V[(bh * N + tok) * VPR + pc];
+        const int pp = poff[bh * (NK + 1) + m] + (pos - k_off[bh * (NK + 1) + m]);
+        const size_t dst = kv_image_chunk(bh * gph, pp, pc);
+        Kp[dst] = K[(bh * N + tok) * VPR + pc];
+        Vp[dst] = V[(bh * N + tok) * VPR + pc];
     }
     // pad rows: at most 7 per cluster
     const size_t pads = BH * (size_t)NK * 7 * VPR;
@@ -186,9 +199,9 @@ __global__ void k_kv_pad_gather(const uint4* __restrict__ K, const uint4* __rest
         const int sz = k_off[bh * (NK + 1) + m + 1] - k_off[bh * (NK + 1) + m];
         const int padn = ((sz + 7) & ~7) - sz;
         if (i < padn) {
-            const size_t dst = bh * Npad + poff[bh * (NK + 1) + m] + sz + i;
-            Kp[dst * VPR + pc] = make_uint4(0, 0, 0, 0);
-            Vp[dst * VPR + pc] = make_uint4(0, 0, 0, 0);
+            const size_t dst = kv_image_chunk(bh * gph, poff[bh * (NK + 1) + m] + sz + i, pc);
+            Kp[dst] = make_uint4(0, 0, 0, 0);
+            Vp[dst] = make_uint4(0, 0, 0, 0);
         }
     }
 }

@@ -7,25 +7,32 @@
 // a run of whole 8-row groups.  For a query cluster, its kept key clusters are
 // concatenated (padded sizes) into one virtual key sequence that is cut into
 // full 128-row tiles: clusters smaller than a tile share a tile (the
-// gather-into-full-tiles idea of the AB-Attention article).  A 128-row key
-// tile is assembled by 16 TMA loads of 8-row boxes per 64-column half, for K
-// and for V; groups past the end load out of bounds (zero fill) and are masked.
+// gather-into-full-tiles idea of the AB-Attention article).  Padded K and V
+// are stored in global memory as the byte image of the shared-memory tiles
+// (8-row groups of 2048 bytes: both 64-column halves, 128-byte swizzled), so
+// the part of a kept cluster that falls in a tile arrives with one bulk copy
+// for K and one for V; pad rows and groups past the end are masked.
 //
 // One CTA per SM (persistent, work items round-robin), 6 warps:
-//   warp 0     TMA producer: Q tile (128 x 128) per item, K/V tiles into a
-//              2-stage ring;
-//   warp 1     TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into one of
-//              two TMEM buffers (128 x 128 fp32), then O += P_j V_j into a TMEM
-//              accumulator (128 x 128 fp32);
+//   warp 0     producer: Q tile (128 x 128, TMA) per item; K and V tiles (bulk
+//              copies, one per kept-cluster piece) into two 2-stage rings with
+//              separate barriers, so K of tile j+2 may arrive while V of tile
+//              j is still in use; a per-tile column bias (0 or -inf) for the
+//              masked rows;
+//   warp 1     TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into TMEM
+//              buffer j%2 (128 x 128 fp32), O += P_j V_j into a TMEM
+//              accumulator (128 x 128 fp32), in the order S0 S1 PV0 S2 PV1 S3 ...
 //   warps 2-5  Softmax: thread = query row = TMEM lane.  Loads S_j, online
 //              Softmax in the log2 domain with a lazily updated reference max
-//              (O is rescaled in TMEM only when the row max grows by more than
-//              2^8), writes P_j as bf16 into shared memory in the swizzled
-//              K-major layout of the next MMA, and finally normalises O and
-//              writes the row in original token order.
+//              (O is rescaled in TMEM only when a row max grows by more than
+//              2^8), writes P_j as bf16 into shared-memory buffer j%2 in the
+//              swizzled K-major layout of the PV MMA (two buffers: writing P_j
+//              only waits for PV_{j-2}), and finally normalises O and writes the
+//              rows in original token order.
 // Every wait is time-bounded; a timeout sets PARK_ERR_TIMEOUT in the status
 // word, the roles leave their loops, outstanding copies and MMAs are waited
-// for (bounded) and TMEM is freed before the CTA exits.
+// for (bounded) and TMEM is freed before the CTA exits.  Decisions that guard
+// warp-collective operations (tcgen05.ld/st, shuffles) are warp-uniform.
 #include <cudaTypedefs.h>
 
 #include "kernels.h"
@@ -36,83 +43,87 @@ namespace park {
 using namespace sm100;
 
 namespace {
-constexpr int TC_ROWS = 128;       // query rows and key rows per tile
-constexpr int TC_BLK = 16384;      // one 128-row x 64-column bf16 block (128 B rows)
-constexpr int TC_STAGES = 2;
+constexpr int TC_ROWS = 128;            // query rows and key rows per tile
+constexpr int TC_BLK = 16384;           // 128 rows x 128 bytes
 constexpr uint32_t TC_TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256,384)
 constexpr float kLog2eT = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
 
 struct TcSmem {
-    uint64_t q_full, q_empty, kv_full[TC_STAGES], kv_empty[TC_STAGES], s_full[2], s_empty[2], p_full, o_done,
-        o_empty, final_bar;
+    uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_empty[2], p_full[2],
+        pv_done[2], o_empty, final_bar;
     uint32_t tmem_base;
     int abort;
-    uint8_t valid[TC_STAGES][16];  // per-stage validity of the 128 key rows (bit i of byte g: row 8g+i)
+    alignas(16) float bias[2][TC_ROWS];  // per stage: 0 for a real key row, -inf for a pad row or past the end
 };
 }  // namespace
 
 __device__ __forceinline__ float bits_f(uint32_t u) { return __uint_as_float(u); }
 // warp-uniform view of the abort flag
 __device__ __forceinline__ bool warp_abort(volatile int* abort) { return __any_sync(0xffffffffu, *abort != 0); }
+__device__ __forceinline__ float fast_ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __global__ void __launch_bounds__(192, 1)
-    k_sparse_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, int N, int NQ, int NK, int Npad, int BH,
-                     const int32_t* __restrict__ q_perm, const int2* __restrict__ segs,
-                     const int32_t* __restrict__ kept_ptr, const int32_t* __restrict__ kv_pre,
-                     const int32_t* __restrict__ kv_len, const WorkItem* __restrict__ items,
-                     const int32_t* __restrict__ item_count, uint16_t* __restrict__ O, float sl2e,
-                     int32_t* __restrict__ status) {
+    k_sparse_attn_tc(const __grid_constant__ CUtensorMap tmQ, const uint8_t* __restrict__ Kimg,
+                     const uint8_t* __restrict__ Vimg, int N, int NQ, int NK, const int32_t* __restrict__ q_perm,
+                     const int2* __restrict__ segs, const int32_t* __restrict__ kept_ptr,
+                     const int32_t* __restrict__ kv_pre, const int32_t* __restrict__ kv_len,
+                     const WorkItem* __restrict__ items, const int32_t* __restrict__ item_count,
+                     uint16_t* __restrict__ O, float sl2e, int32_t* __restrict__ status) {
     extern __shared__ __align__(1024) uint8_t dsmem_raw[];
     __shared__ TcSmem sh;
-    // 1024-byte aligned operand area: Q | K0 V0 K1 V1 | P
+    // 1024-byte aligned operand area: Q | K0 K1 | V0 V1 | P0 P1 (each 32 KB)
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* Qs = base;                                  // 2 blocks
-    uint8_t* KVs = base + 2 * TC_BLK;                    // per stage: K 2 blocks, V 2 blocks
-    uint8_t* Ps = base + 2 * TC_BLK + TC_STAGES * 4 * TC_BLK;  // 2 blocks
+    uint8_t* Qs = base;
+    uint8_t* Ks = base + 2 * TC_BLK;
+    uint8_t* Vs = Ks + 4 * TC_BLK;
+    uint8_t* Ps = Vs + 4 * TC_BLK;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort = &sh.abort;
     if (threadIdx.x == 0) {
         mbar_init(&sh.q_full, 1);
         mbar_init(&sh.q_empty, 1);
-        for (int s = 0; s < TC_STAGES; ++s) {
-            mbar_init(&sh.kv_full[s], 1);
-            mbar_init(&sh.kv_empty[s], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sh.k_full[s], 1);
+            mbar_init(&sh.k_empty[s], 1);
+            mbar_init(&sh.v_full[s], 1);
+            mbar_init(&sh.v_empty[s], 1);
+            mbar_init(&sh.s_full[s], 1);
+            mbar_init(&sh.s_empty[s], 128);
+            mbar_init(&sh.p_full[s], 128);
+            mbar_init(&sh.pv_done[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sh.s_full[b], 1);
-            mbar_init(&sh.s_empty[b], 128);
-        }
-        mbar_init(&sh.p_full, 128);
-        mbar_init(&sh.o_done, 1);
         mbar_init(&sh.o_empty, 128);
         mbar_init(&sh.final_bar, 1);
         sh.abort = 0;
         mbar_fence_init();
     }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmQ);
-        tma_prefetch_desc(&tmK);
-        tma_prefetch_desc(&tmV);
-    }
+    if (warp == 0 && lane == 0) tma_prefetch_desc(&tmQ);
     if (warp == 1) {
         tmem_alloc(&sh.tmem_base, TC_TMEM_COLS);
         tmem_relinquish();
     }
+    // K/V stages start as zeros: groups that are never loaded must hold finite values
+    for (int i = threadIdx.x; i < 8 * TC_BLK / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(Ks)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
     const int n_items = *item_count;
-    const uint32_t idS = idesc_bf16(128, 128, 0, 0);  // S = Q K^T: both K-major
+    const uint32_t idS = idesc_bf16(128, 128, 0, 0);   // S = Q K^T: both K-major
     const uint32_t idPV = idesc_bf16(128, 128, 0, 1);  // O += P V: P K-major, V MN-major
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         int T = 0, I = 0;
-        int last_parity[TC_STAGES] = {-1, -1};
+        int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
         int q_pending = 0, q_parity = 0;
         for (int it = blockIdx.x; it < n_items && !warp_abort(abort); it += gridDim.x) {
             const WorkItem wi = items[it];
@@ -154,26 +165,37 @@ __global__ void __launch_bounds__(192, 1)
                 }
             };
             load_entries(0);
-            for (int j = 0; j < nkt; ++j) {
+            bool ok = true;
+            for (int j = 0; j < nkt && ok; ++j) {
                 const int stg = T & 1, round = T >> 1;
-                int y = BH * Npad;  // out of bounds: zero fill
-                uint8_t vmask = 0;
+                int nvalid = 0;  // real key rows of group `lane` (lanes 0..15)
 #pragma unroll 4
                 for (int g = 0; g < 16; ++g) {
                     const int vg = j * TC_ROWS + 8 * g;
                     const unsigned bal = __ballot_sync(0xffffffffu, p_l <= vg);
                     const int idx = (__popc(bal) - 1) & 31;
                     const int pp = __shfl_sync(0xffffffffu, p_l, idx);
-                    const int src = __shfl_sync(0xffffffffu, src_l, idx);
                     const int sz = __shfl_sync(0xffffffffu, sz_l, idx);
                     if (lane == g && vg < L) {
-                        const int o0 = vg - pp;
-                        int nv = sz - o0;
-                        nv = nv < 0 ? 0 : (nv > 8 ? 8 : nv);
-                        vmask = (uint8_t)((1u << nv) - 1u);
-                        y = src + o0;
+                        int nv = sz - (vg - pp);
+                        nvalid = nv < 0 ? 0 : (nv > 8 ? 8 : nv);
                     }
                 }
+                // this lane's segment (seg0 + lane) as one piece of whole 8-row groups of the tile
+                const int t0 = j * TC_ROWS, t1 = min(t0 + TC_ROWS, L);
+                int pc_start = 0, pc_groups = 0, pc_src = 0;
+                if (p_l < t1) {
+                    const int seg_end = p_l + ((sz_l + 7) & ~7);
+                    const int a = max(p_l, t0), b = min(seg_end, t1);
+                    if (b > a) {
+                        pc_start = a - t0;
+                        pc_groups = (b - a) >> 3;
+                        pc_src = src_l + (a - p_l);
+                    }
+                }
+                const size_t src_off = (size_t)(pc_src >> 3) * 2048;
+                const uint32_t bytes = (uint32_t)pc_groups * 2048u;
+                const uint32_t tile_bytes = (uint32_t)(t1 - t0) * 256u;
                 {  // advance the cursor and prefetch the next tile's entries
                     const int vn = (j + 1) * TC_ROWS;
                     if (vn < L) {
@@ -182,57 +204,73 @@ __global__ void __launch_bounds__(192, 1)
                         load_entries(seg0);
                     }
                 }
-                bool ok = true;
-                if (lane == 0 && round > 0) ok = mbar_wait(&sh.kv_empty[stg], (round - 1) & 1, abort);
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                if (!ok || warp_abort(abort)) break;
-                if (lane < 16) sh.valid[stg][lane] = vmask;
-                __syncwarp();
-                if (lane == 0) mbar_arrive_expect_tx(&sh.kv_full[stg], 4 * TC_BLK);
-                __syncwarp();
-                if (lane < 16) {
-                    uint8_t* Kst = KVs + stg * 4 * TC_BLK;
-                    uint8_t* Vst = Kst + 2 * TC_BLK;
-                    tma_load_2d(Kst + lane * 1024, &tmK, &sh.kv_full[stg], 0, y);
-                    tma_load_2d(Kst + TC_BLK + lane * 1024, &tmK, &sh.kv_full[stg], 64, y);
-                    tma_load_2d(Vst + lane * 1024, &tmV, &sh.kv_full[stg], 0, y);
-                    tma_load_2d(Vst + TC_BLK + lane * 1024, &tmV, &sh.kv_full[stg], 64, y);
+                // K of tile j: stage free once S_{j-2} has completed
+                bool w = true;
+                if (lane == 0 && round > 0) w = mbar_wait(&sh.k_empty[stg], (round - 1) & 1, abort);
+                if (__shfl_sync(0xffffffffu, w ? 1 : 0, 0) == 0 || warp_abort(abort)) {
+                    ok = false;
+                    break;
                 }
-                last_parity[stg] = round & 1;
+                if (lane == 0) mbar_arrive_expect_tx(&sh.k_full[stg], tile_bytes);
+                __syncwarp();
+                if (pc_groups > 0) bulk_load(Ks + stg * 2 * TC_BLK + (pc_start >> 3) * 2048, Kimg + src_off, bytes,
+                                             &sh.k_full[stg]);
+                k_last[stg] = round & 1;
+                // V of tile j and its column bias: free once PV_{j-2} has completed
+                w = true;
+                if (lane == 0 && round > 0) w = mbar_wait(&sh.v_empty[stg], (round - 1) & 1, abort);
+                if (__shfl_sync(0xffffffffu, w ? 1 : 0, 0) == 0 || warp_abort(abort)) {
+                    ok = false;
+                    break;
+                }
+                if (lane < 16) {
+                    float4* bp = reinterpret_cast<float4*>(&sh.bias[stg][8 * lane]);
+                    const float NI = __int_as_float(0xff800000);
+                    bp[0] = make_float4(nvalid > 0 ? 0.f : NI, nvalid > 1 ? 0.f : NI, nvalid > 2 ? 0.f : NI,
+                                        nvalid > 3 ? 0.f : NI);
+                    bp[1] = make_float4(nvalid > 4 ? 0.f : NI, nvalid > 5 ? 0.f : NI, nvalid > 6 ? 0.f : NI,
+                                        nvalid > 7 ? 0.f : NI);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive_expect_tx(&sh.v_full[stg], tile_bytes);
+                __syncwarp();
+                if (pc_groups > 0) bulk_load(Vs + stg * 2 * TC_BLK + (pc_start >> 3) * 2048, Vimg + src_off, bytes,
+                                             &sh.v_full[stg]);
+                v_last[stg] = round & 1;
                 ++T;
             }
+            if (!ok) break;
             ++I;
         }
         // drain: copies still in flight complete before the CTA may exit
         if (lane == 0) {
-            for (int s = 0; s < TC_STAGES; ++s)
-                if (last_parity[s] >= 0) {
-                    int dummy = 0;
-                    mbar_wait(&sh.kv_full[s], last_parity[s], &dummy, 100000000ull);
-                }
-            if (q_pending) {
-                int dummy = 0;
-                mbar_wait(&sh.q_full, q_parity, &dummy, 100000000ull);
+            int dummy = 0;
+            for (int s = 0; s < 2; ++s) {
+                if (k_last[s] >= 0) mbar_wait(&sh.k_full[s], k_last[s], &dummy, 100000000ull);
+                if (v_last[s] >= 0) mbar_wait(&sh.v_full[s], v_last[s], &dummy, 100000000ull);
             }
+            if (q_pending) mbar_wait(&sh.q_full, q_parity, &dummy, 100000000ull);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             int G = 0, I = 0;
-            const uint32_t qa = smem_u32(Qs), pa = smem_u32(Ps);
+            const uint32_t qa = smem_u32(Qs);
             auto issue_S = [&](int g) -> bool {
-                const int stg = g & 1, round = g >> 1;
-                if (!mbar_wait(&sh.kv_full[stg], round & 1, abort)) return false;
-                if (round > 0 && !mbar_wait(&sh.s_empty[stg], (round - 1) & 1, abort)) return false;
+                const int b = g & 1, round = g >> 1;
+                if (!mbar_wait(&sh.k_full[b], round & 1, abort)) return false;
+                if (round > 0 && !mbar_wait(&sh.s_empty[b], (round - 1) & 1, abort)) return false;
                 tc_fence_after();
-                const uint32_t ka = smem_u32(KVs + stg * 4 * TC_BLK);
-                const uint32_t d = tmem + (uint32_t)(stg * 128);
+                const uint32_t ka = smem_u32(Ks + b * 2 * TC_BLK);
+                const uint32_t d = tmem + (uint32_t)(b * 128);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * TC_BLK + (kk & 3) * 32);
-                    umma_bf16(d, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
+                    const uint32_t qoff = (uint32_t)((kk >> 2) * TC_BLK + (kk & 3) * 32);
+                    const uint32_t koff = (uint32_t)((kk >> 2) * 1024 + (kk & 3) * 32);
+                    umma_bf16(d, sdesc_sw128(qa + qoff, 16, 1024), sdesc_sw128(ka + koff, 16, 2048), idS, kk > 0);
                 }
-                umma_commit(&sh.s_full[stg]);
+                umma_commit(&sh.s_full[b]);
+                umma_commit(&sh.k_empty[b]);
                 return true;
             };
             for (int it = blockIdx.x; it < n_items && !*abort; it += gridDim.x) {
@@ -242,32 +280,26 @@ __global__ void __launch_bounds__(192, 1)
                 if (nkt == 0) continue;
                 if (!mbar_wait(&sh.q_full, I & 1, abort)) break;
                 tc_fence_after();
-                if (!issue_S(G)) break;
-                bool ok = true;
+                bool ok = issue_S(G) && (nkt < 2 || issue_S(G + 1));
                 for (int j = 0; j < nkt && ok; ++j) {
-                    const int g = G + j;
-                    if (j + 1 < nkt && !issue_S(g + 1)) {
-                        ok = false;
-                        break;
-                    }
-                    if (!mbar_wait(&sh.p_full, g & 1, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    if (j == 0 && I > 0 && !mbar_wait(&sh.o_empty, (I - 1) & 1, abort)) {
+                    const int g = G + j, b = g & 1, ph = (g >> 1) & 1;
+                    if (!mbar_wait(&sh.p_full[b], ph, abort) ||
+                        (j == 0 && I > 0 && !mbar_wait(&sh.o_empty, (I - 1) & 1, abort)) ||
+                        !mbar_wait(&sh.v_full[b], ph, abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t va = smem_u32(KVs + (g & 1) * 4 * TC_BLK + 2 * TC_BLK);
+                    const uint32_t pa = smem_u32(Ps + b * 2 * TC_BLK), va = smem_u32(Vs + b * 2 * TC_BLK);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t aoff = (uint32_t)((kk >> 2) * TC_BLK + (kk & 3) * 32);
-                        umma_bf16(tmem + 256, sdesc_sw128(pa + aoff, 16, 1024),
-                                  sdesc_sw128(va + (uint32_t)kk * 2048, TC_BLK, 1024), idPV, (j > 0 || kk > 0));
+                        const uint32_t poff = (uint32_t)((kk >> 2) * TC_BLK + (kk & 3) * 32);
+                        umma_bf16(tmem + 256, sdesc_sw128(pa + poff, 16, 1024),
+                                  sdesc_sw128(va + (uint32_t)kk * 4096, 1024, 2048), idPV, (j > 0 || kk > 0));
                     }
-                    umma_commit(&sh.o_done);
-                    umma_commit(&sh.kv_empty[g & 1]);
+                    umma_commit(&sh.pv_done[b]);
+                    umma_commit(&sh.v_empty[b]);
+                    if (j + 2 < nkt && !issue_S(g + 2)) ok = false;
                 }
                 if (!ok) break;
                 umma_commit(&sh.q_empty);
@@ -286,7 +318,7 @@ __global__ void __launch_bounds__(192, 1)
         const int row = lane_base + lane;
         const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
         int G = 0, I = 0;
-        // waits are decided per warp: tcgen05.ld and shuffles below are warp-collective
+        // waits are decided per warp: tcgen05.ld/st and shuffles below are warp-collective
         auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
             const bool ok = mbar_wait(bar, parity, abort);
             return __all_sync(0xffffffffu, ok);
@@ -299,8 +331,8 @@ __global__ void __launch_bounds__(192, 1)
             float m_ref = __int_as_float(0xff800000), l = 0.f;
             bool ok = true;
             for (int j = 0; j < nkt; ++j) {
-                const int g = G + j, b = g & 1, round = g >> 1;
-                if (!wwait(&sh.s_full[b], round & 1) || !wwait(&sh.kv_full[b], round & 1)) {
+                const int g = G + j, b = g & 1, ph = (g >> 1) & 1;
+                if (!wwait(&sh.s_full[b], ph) || !wwait(&sh.v_full[b], ph)) {
                     ok = false;
                     break;
                 }
@@ -311,33 +343,36 @@ __global__ void __launch_bounds__(192, 1)
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&sh.s_empty[b]);
-                const uint8_t* vb = sh.valid[b];
+                const float4* bz = reinterpret_cast<const float4*>(sh.bias[b]);
                 float tmax = __int_as_float(0xff800000);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int col = 32 * c + e;
-                        const bool v = (vb[col >> 3] >> (col & 7)) & 1;
-                        const float x = v ? bits_f(s[c][e]) * sl2e : __int_as_float(0xff800000);
-                        s[c][e] = __float_as_uint(x);
-                        tmax = fmaxf(tmax, x);
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 bb = bz[c * 8 + q];
+                        const float x0 = fmaf(bits_f(s[c][4 * q + 0]), sl2e, bb.x);
+                        const float x1 = fmaf(bits_f(s[c][4 * q + 1]), sl2e, bb.y);
+                        const float x2 = fmaf(bits_f(s[c][4 * q + 2]), sl2e, bb.z);
+                        const float x3 = fmaf(bits_f(s[c][4 * q + 3]), sl2e, bb.w);
+                        s[c][4 * q + 0] = __float_as_uint(x0);
+                        s[c][4 * q + 1] = __float_as_uint(x1);
+                        s[c][4 * q + 2] = __float_as_uint(x2);
+                        s[c][4 * q + 3] = __float_as_uint(x3);
+                        tmax = fmaxf(tmax, fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
                     }
                 }
-                bool waited = j == 0;
                 if (j == 0) {
                     m_ref = tmax;
                 } else if (__any_sync(0xffffffffu, tmax > m_ref + kRescaleThreshold)) {
-                    // decided per warp: the TMEM loads/stores below are warp-collective;
-                    // rows that do not need a new reference keep theirs (alpha = 1)
-                    if (!wwait(&sh.o_done, (g - 1) & 1)) {
+                    // decided per warp (TMEM loads/stores are warp-collective); rows that do
+                    // not need a new reference keep theirs (alpha = 1).  O must hold PV_{j-1}.
+                    if (!wwait(&sh.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) {
                         ok = false;
                         break;
                     }
-                    waited = true;
                     tc_fence_after();
                     const float m_new = tmax > m_ref + kRescaleThreshold ? tmax : m_ref;
-                    const float alpha = exp2f(m_ref - m_new);
+                    const float alpha = fast_ex2(m_ref - m_new);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         uint32_t o[32];
@@ -351,23 +386,26 @@ __global__ void __launch_bounds__(192, 1)
                     l *= alpha;
                     m_ref = m_new;
                 }
-                if (!waited && !wwait(&sh.o_done, (g - 1) & 1)) {  // P buffer free
+                // P buffer b was last read by PV_{j-2} (for j < 2 the previous item's
+                // epilogue already waited for all of its PVs)
+                if (j >= 2 && !wwait(&sh.pv_done[b], ((g - 2) >> 1) & 1)) {
                     ok = false;
                     break;
                 }
                 // P row -> shared memory, K-major, 128-byte swizzle: chunk c16 of row r at c16 ^ (r & 7)
+                uint8_t* Pb = Ps + b * 2 * TC_BLK;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = exp2f(bits_f(s[c][2 * e]) - m_ref);
-                        const float p1 = exp2f(bits_f(s[c][2 * e + 1]) - m_ref);
+                        const float p0 = fast_ex2(bits_f(s[c][2 * e]) - m_ref);
+                        const float p1 = fast_ex2(bits_f(s[c][2 * e + 1]) - m_ref);
                         l += p0 + p1;
                         __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
                         pk[e] = *reinterpret_cast<uint32_t*>(&h);
                     }
-                    uint8_t* blk = Ps + (c >> 1) * TC_BLK + row * 128;
+                    uint8_t* blk = Pb + (c >> 1) * TC_BLK + row * 128;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int c16 = (c & 1) * 4 + q;
@@ -377,11 +415,12 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(&sh.p_full);
+                mbar_arrive(&sh.p_full[b]);
             }
             if (!ok) break;
             // epilogue: O / l, original token order
-            if (!wwait(&sh.o_done, (G + nkt - 1) & 1)) break;
+            const int gl = G + nkt - 1;
+            if (!wwait(&sh.pv_done[gl & 1], (gl >> 1) & 1)) break;
             tc_fence_after();
             uint32_t o[4][32];
 #pragma unroll
@@ -450,7 +489,7 @@ int make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t box_rows
 }
 }  // namespace
 
-size_t attn_tc_smem_bytes() { return (size_t)(2 + TC_STAGES * 4 + 2) * TC_BLK + 1024; }
+size_t attn_tc_smem_bytes() { return (size_t)14 * TC_BLK + 1024; }  // Q, K x2, V x2, P x2
 
 int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
                           const int32_t* q_perm, const int2* segs, const int32_t* kept_ptr, const int32_t* kv_pre,
@@ -458,16 +497,15 @@ int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, in
                           const WorkItem* items, const int32_t* item_count, void* O, int32_t* status, int num_sms,
                           cudaStream_t st) {
     PARK_CHECK(get_encoder());
-    CUtensorMap mQ, mK, mV;
+    CUtensorMap mQ;
     PARK_CHECK(make_map(&mQ, Qp, (uint64_t)BH * N, 128));
-    PARK_CHECK(make_map(&mK, Kpad, (uint64_t)BH * Npad, 8));
-    PARK_CHECK(make_map(&mV, Vpad, (uint64_t)BH * Npad, 8));
     const size_t sm = attn_tc_smem_bytes();
     cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     const float sl2e = (1.0f / sqrtf(128.f)) * kLog2eT;
     ::park::prof_begin(st);
-    k_sparse_attn_tc<<<num_sms, 192, sm, st>>>(mQ, mK, mV, N, NQ, NK, Npad, BH, q_perm, segs, kept_ptr, kv_pre,
-                                                kv_len, items, item_count, (uint16_t*)O, sl2e, status);
+    k_sparse_attn_tc<<<num_sms, 192, sm, st>>>(mQ, (const uint8_t*)Kpad, (const uint8_t*)Vpad, N, NQ, NK, q_perm,
+                                                segs, kept_ptr, kv_pre, kv_len, items, item_count, (uint16_t*)O,
+                                                sl2e, status);
     PARK_TRY_LAUNCH("k_sparse_attn_tc", st);
     return PARK_OK;
 }
