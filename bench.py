@@ -228,18 +228,19 @@ def workload_config(cfg) -> dict:
 
 # ----------------------------------------------------------------------------- roofline of one kernel
 
-KERNEL_SOURCES = {"k_sparse_attn_mma": ["block_sparse_attention_means_b200/csrc/k_attn.cu"],
+KERNEL_SOURCES = {"k_sparse_attn_tc": ["block_sparse_attention_means_b200/csrc/k_attn_tc.cu"],
                   "k_assign_mma": ["block_sparse_attention_means_b200/csrc/k_assign.cu"],
                   "k_pama_mma": ["block_sparse_attention_means_b200/csrc/k_pama.cu"],
                   "k_pama_f64": ["block_sparse_attention_means_b200/csrc/k_pama.cu"],
                   "k_metric_partial": ["block_sparse_attention_means_b200/csrc/k_prep.cu"]}
+ATTENTION_KERNELS = ("k_sparse_attn_tc", "k_gather_rows", "k_attn_schedule", "k_kv_pad_gather", "k_kv_pad_offsets")
 
 
 def kernel_roofline(name: str, ms_per_launch: float, cfg, counters, peaks, peak_kind) -> dict:
     """Algorithmic work per launch of the named kernel and its roofline."""
     BH, N, D, NQ, NK = cfg.B * cfg.H, cfg.N, cfg.D, cfg.NQ, cfg.NK
     sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    if name == "k_sparse_attn_mma":
+    if name == "k_sparse_attn_tc":
         work, bound, peak, unit = 4.0 * D * counters[5], "tensor", sustained, "TFLOP/s"
     elif name == "k_assign_mma":
         work, bound, peak, unit = 2.0 * BH * N * ((NQ + NK) / 2) * D, "tensor", sustained, "TFLOP/s"
@@ -255,8 +256,13 @@ def kernel_roofline(name: str, ms_per_launch: float, cfg, counters, peaks, peak_
         return {"kernel": name, "bound": None}
     achieved = work / (ms_per_launch * 1e-3) / 1e12
     traffic = committed_traffic(name)
+    extra = {}
+    if name == "k_sparse_attn_tc":
+        # tensor work actually issued: every (128-row query tile, 128-row key tile) pair, padding included
+        tile_tf = 4.0 * 128 * 128 * D * counters[7] / (ms_per_launch * 1e-3) / 1e12
+        extra = {"tile_tflops": round(tile_tf, 2), "tensor_pipe_frac_on_tiles": round(tile_tf / peak, 4)}
     return {"kernel": name, "bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": unit,
-            "frac": round(achieved / peak, 4), "traffic": traffic, "ms_per_launch": round(ms_per_launch, 3),
+            "frac": round(achieved / peak, 4), "traffic": traffic, "ms_per_launch": round(ms_per_launch, 3), **extra,
             "peak_source": peak_kind + (" (fp64: 148 SMs x 64 FMA/clk x 1.965 GHz)" if bound == "alu" else
                                         " bf16_tflops_sustained")}
 
@@ -388,11 +394,11 @@ def main():
                for k, v in sorted(prof.items(), key=lambda kv: -kv[1][0])}
     top = next(iter(kernels)) if kernels else None
     roof = kernel_roofline(top, prof[top][0] / prof[top][1], cfg, counters, peaks, peak_kind) if top else None
-    attn = prof.get("k_sparse_attn_mma")
-    attn_roof = kernel_roofline("k_sparse_attn_mma", attn[0] / attn[1], cfg, counters, peaks, peak_kind) \
+    attn = prof.get("k_sparse_attn_tc")
+    attn_roof = kernel_roofline("k_sparse_attn_tc", attn[0] / attn[1], cfg, counters, peaks, peak_kind) \
         if attn else None
     retrieval_ms = sum(v[0] for k, v in prof.items()
-                       if k not in ("k_sparse_attn_mma", "k_gather_rows", "k_attn_schedule")) / args.steps
+                       if k not in ATTENTION_KERNELS) / args.steps
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

@@ -28,6 +28,7 @@ PARK_CNT_PAMA_RECHECK = 3
 PARK_CNT_KEPT_BLOCKS = 4
 PARK_CNT_KEPT_PAIRS = 5
 PARK_CNT_WORK_ITEMS = 6
+PARK_CNT_KEY_TILES = 7
 PARK_NUM_COUNTERS = 8
 
 # Every symbol include/park.h declares (checked by the CPU tests).

@@ -12,11 +12,8 @@
 // Softmax over its virtual key tiles and writes O rows back in original token
 // order.
 #include "kernels.h"
-#include "mma_sync.cuh"
 
 namespace park {
-
-constexpr float kLog2eA = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- gather
 __global__ void k_gather_rows(const uint4* __restrict__ X, const int32_t* __restrict__ perm, uint4* __restrict__ Xp,
@@ -111,6 +108,8 @@ __global__ __launch_bounds__(256) void k_attn_schedule(int NQ, int NK, const int
             atomicAdd((unsigned long long*)(counters + PARK_CNT_KEPT_PAIRS),
                       (unsigned long long)nr * (unsigned long long)total_u);
             atomicAdd((unsigned long long*)(counters + PARK_CNT_WORK_ITEMS), (unsigned long long)tiles);
+            atomicAdd((unsigned long long*)(counters + PARK_CNT_KEY_TILES),
+                      (unsigned long long)tiles * (unsigned long long)((total + tile_rows - 1) / tile_rows));
         }
     }
 }
@@ -219,218 +218,6 @@ int launch_kv_pad_gather(const void* K, const void* V, int BH, int N, int NK, in
     k_kv_pad_gather<<<blocks, 256, 0, st>>>((const uint4*)K, (const uint4*)V, N, NK, Npad, (size_t)BH, k_perm,
                                             k_labels, k_off, poff, (uint4*)Kpad, (uint4*)Vpad);
     PARK_TRY_LAUNCH("k_kv_pad_gather", st);
-    return PARK_OK;
-}
-
-// ---------------------------------------------------------------- attention (bf16, D = 128)
-// 128 threads: 4 warps x 16 query rows.  K/V tiles of 64 rows are staged by
-// cp.async from the row table of the virtual key sequence (double buffered).
-// S = Q K^T and O += P V on tensor cores (fp32 accumulate), Softmax online in
-// the log2 domain.
-constexpr int AT_ROWS = 64, AT_LDS = 128 + 8;
-
-__device__ __forceinline__ int kv_source_row(int v, int L, int nk, const int32_t* pre, const int32_t* kl,
-                                             const int32_t* ko) {
-    if (v >= L) return -1;
-    int lo = 0, hi = nk - 1;
-    while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (pre[mid] <= v)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    return ko[kl[lo]] + (v - pre[lo]);
-}
-
-__global__ __launch_bounds__(128) void k_sparse_attn_mma(
-    const uint16_t* __restrict__ Qp, const uint16_t* __restrict__ Kp, const uint16_t* __restrict__ Vp, int N, int NQ,
-    int NK, const int32_t* __restrict__ q_perm, const int32_t* __restrict__ k_off,
-    const int32_t* __restrict__ kept_ptr, const int32_t* __restrict__ kept_idx, const int32_t* __restrict__ kv_pre,
-    const int32_t* __restrict__ kv_len, const WorkItem* __restrict__ items, const int32_t* __restrict__ item_count,
-    int32_t* __restrict__ work_counter, uint16_t* __restrict__ O, float sl2e) {
-    constexpr int D = 128;
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    uint16_t* Ks = reinterpret_cast<uint16_t*>(smem_raw);          // [2][64][LDS]
-    uint16_t* Vs = Ks + 2 * AT_ROWS * AT_LDS;                      // [2][64][LDS]
-    int32_t* tbl = reinterpret_cast<int32_t*>(Vs + 2 * AT_ROWS * AT_LDS);  // [2][64]
-    __shared__ int s_item;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
-    const int mi = lane >> 3, r8 = lane & 7;
-    const int n_items = *item_count;
-
-    for (;;) {
-        __syncthreads();
-        if (tid == 0) s_item = atomicAdd(work_counter, 1);
-        __syncthreads();
-        const int it = s_item;
-        if (it >= n_items) break;
-        const WorkItem wi = items[it];
-        const int bh = wi.bh, r = wi.r;
-        const int L = kv_len[(size_t)bh * NQ + r];
-        const int kp0 = kept_ptr[(size_t)bh * (NQ + 1) + r];
-        const int nk = kept_ptr[(size_t)bh * (NQ + 1) + r + 1] - kp0;
-        const int32_t* kl = kept_idx + (size_t)bh * NQ * NK + kp0;
-        const int32_t* pre = kv_pre + (size_t)bh * NQ * NK + kp0;
-        const int32_t* ko = k_off + (size_t)bh * (NK + 1);
-        const uint16_t* Kh = Kp + (size_t)bh * N * D;
-        const uint16_t* Vh = Vp + (size_t)bh * N * D;
-        const int nkt = (L + AT_ROWS - 1) / AT_ROWS;
-
-        // Q fragments (rows beyond the tile are computed but never stored)
-        const int qr0 = wi.q_start + warp * 16 + g, qr1 = qr0 + 8;
-        const uint16_t* Qh = Qp + (size_t)bh * N * D;
-        uint32_t qa[8][4];
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            int c0 = kk * 16 + 2 * tq;
-            qa[kk][0] = qr0 < N ? ld_u32(Qh + (size_t)qr0 * D + c0) : 0u;
-            qa[kk][1] = qr1 < N ? ld_u32(Qh + (size_t)qr1 * D + c0) : 0u;
-            qa[kk][2] = qr0 < N ? ld_u32(Qh + (size_t)qr0 * D + c0 + 8) : 0u;
-            qa[kk][3] = qr1 < N ? ld_u32(Qh + (size_t)qr1 * D + c0 + 8) : 0u;
-        }
-        float o[16][4];
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) o[nt][j] = 0.f;
-        float mrow[2] = {__int_as_float(0xff800000), __int_as_float(0xff800000)};
-        float lrow[2] = {0.f, 0.f};
-
-        auto build_table = [&](int kt, int stg) {
-            if (tid < AT_ROWS) tbl[stg * AT_ROWS + tid] = kv_source_row(kt * AT_ROWS + tid, L, nk, pre, kl, ko);
-        };
-        auto issue_loads = [&](int stg) {
-            for (int e = tid; e < AT_ROWS * 16; e += 128) {
-                int rr = e >> 4, pc = e & 15;
-                int src = tbl[stg * AT_ROWS + rr];
-                size_t so = (size_t)(src < 0 ? 0 : src) * D + pc * 8;
-                int nb = src < 0 ? 0 : 16;
-                cp_async16(Ks + (stg * AT_ROWS + rr) * AT_LDS + pc * 8, Kh + so, nb);
-                cp_async16(Vs + (stg * AT_ROWS + rr) * AT_LDS + pc * 8, Vh + so, nb);
-            }
-        };
-
-        if (nkt > 0) {
-            build_table(0, 0);
-            __syncthreads();
-            issue_loads(0);
-            cp_async_commit();
-        }
-        for (int kt = 0; kt < nkt; ++kt) {
-            const int stg = kt & 1;
-            if (kt + 1 < nkt) build_table(kt + 1, stg ^ 1);
-            __syncthreads();
-            if (kt + 1 < nkt) issue_loads(stg ^ 1);
-            cp_async_commit();
-            cp_async_wait<1>();
-            __syncthreads();
-
-            const uint16_t* Kst = Ks + stg * AT_ROWS * AT_LDS;
-            const uint16_t* Vst = Vs + stg * AT_ROWS * AT_LDS;
-            float s[8][4];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) s[nt][j] = 0.f;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-#pragma unroll
-                for (int np = 0; np < 4; ++np) {
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4(b0, b1, b2, b3, Kst + (np * 16 + (mi >> 1) * 8 + r8) * AT_LDS + kk * 16 + (mi & 1) * 8);
-                    mma_bf16_16816(s[2 * np], qa[kk], b0, b1);
-                    mma_bf16_16816(s[2 * np + 1], qa[kk], b2, b3);
-                }
-            const int valid_cols = L - kt * AT_ROWS;
-            float mloc[2] = {__int_as_float(0xff800000), __int_as_float(0xff800000)};
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    int col = nt * 8 + 2 * tq + (j & 1);
-                    float v = col < valid_cols ? s[nt][j] * sl2e : __int_as_float(0xff800000);
-                    s[nt][j] = v;
-                    mloc[j >> 1] = fmaxf(mloc[j >> 1], v);
-                }
-            float alpha[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], 1));
-                mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], 2));
-                float mn = fmaxf(mrow[h], mloc[h]);
-                alpha[h] = mrow[h] == __int_as_float(0xff800000) ? 0.f : exp2f(mrow[h] - mn);
-                mrow[h] = mn;
-                lrow[h] *= alpha[h];
-            }
-#pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                o[nt][0] *= alpha[0];
-                o[nt][1] *= alpha[0];
-                o[nt][2] *= alpha[1];
-                o[nt][3] *= alpha[1];
-            }
-            uint32_t pa[4][4];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                float p0 = exp2f(s[nt][0] - mrow[0]), p1 = exp2f(s[nt][1] - mrow[0]);
-                float p2 = exp2f(s[nt][2] - mrow[1]), p3 = exp2f(s[nt][3] - mrow[1]);
-                lrow[0] += p0 + p1;
-                lrow[1] += p2 + p3;
-                int kk2 = nt >> 1, half = nt & 1;
-                pa[kk2][half * 2 + 0] = pack_bf16x2(p0, p1);
-                pa[kk2][half * 2 + 1] = pack_bf16x2(p2, p3);
-            }
-#pragma unroll
-            for (int kk2 = 0; kk2 < 4; ++kk2)
-#pragma unroll
-                for (int dp = 0; dp < 8; ++dp) {
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4_trans(b0, b1, b2, b3,
-                                      Vst + (kk2 * 16 + (mi & 1) * 8 + r8) * AT_LDS + dp * 16 + (mi >> 1) * 8);
-                    mma_bf16_16816(o[2 * dp], pa[kk2], b0, b1);
-                    mma_bf16_16816(o[2 * dp + 1], pa[kk2], b2, b3);
-                }
-            __syncthreads();
-        }
-        // epilogue: normalise, write rows in original token order
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
-            lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
-        }
-        const float inv0 = lrow[0] > 0.f ? 1.f / lrow[0] : 0.f, inv1 = lrow[1] > 0.f ? 1.f / lrow[1] : 0.f;
-        const int lr0 = warp * 16 + g, lr1 = lr0 + 8;
-        if (lr0 < wi.rows) {
-            int tok = q_perm[(size_t)bh * N + wi.q_start + lr0];
-            uint16_t* orow = O + ((size_t)bh * N + tok) * D;
-#pragma unroll
-            for (int nt = 0; nt < 16; ++nt)
-                *reinterpret_cast<uint32_t*>(orow + nt * 8 + 2 * tq) = pack_bf16x2(o[nt][0] * inv0, o[nt][1] * inv0);
-        }
-        if (lr1 < wi.rows) {
-            int tok = q_perm[(size_t)bh * N + wi.q_start + lr1];
-            uint16_t* orow = O + ((size_t)bh * N + tok) * D;
-#pragma unroll
-            for (int nt = 0; nt < 16; ++nt)
-                *reinterpret_cast<uint32_t*>(orow + nt * 8 + 2 * tq) = pack_bf16x2(o[nt][2] * inv1, o[nt][3] * inv1);
-        }
-    }
-}
-
-int launch_sparse_attn_mma(const void* Qp, const void* Kp, const void* Vp, int BH, int N, int NQ, int NK,
-                           const int32_t* q_perm, const int32_t* k_off, const int32_t* kept_ptr,
-                           const int32_t* kept_idx, const int32_t* kv_pre, const int32_t* kv_len,
-                           const WorkItem* items, const int32_t* item_count, int32_t* work_counter, void* O,
-                           int num_sms, cudaStream_t st) {
-    size_t sm = 2 * 2 * AT_ROWS * AT_LDS * 2 + 2 * AT_ROWS * 4;
-    cudaFuncSetAttribute(k_sparse_attn_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    float sl2e = (1.0f / sqrtf(128.f)) * kLog2eA;
-    ::park::prof_begin(st);
-    k_sparse_attn_mma<<<num_sms * 3, 128, sm, st>>>((const uint16_t*)Qp, (const uint16_t*)Kp, (const uint16_t*)Vp,
-                                                     N, NQ, NK, q_perm, k_off, kept_ptr, kept_idx, kv_pre, kv_len,
-                                                     items, item_count, work_counter, (uint16_t*)O, sl2e);
-    PARK_TRY_LAUNCH("k_sparse_attn_mma", st);
     return PARK_OK;
 }
 

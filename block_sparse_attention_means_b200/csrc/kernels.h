@@ -89,11 +89,6 @@ int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, in
                           const int32_t* kv_len,
                           const WorkItem* items, const int32_t* item_count, void* O, int32_t* status, int num_sms,
                           cudaStream_t st);
-int launch_sparse_attn_mma(const void* Qp, const void* Kp, const void* Vp, int BH, int N, int NQ, int NK,
-                           const int32_t* q_perm, const int32_t* k_off, const int32_t* kept_ptr,
-                           const int32_t* kept_idx, const int32_t* kv_pre, const int32_t* kv_len,
-                           const WorkItem* items, const int32_t* item_count, int32_t* work_counter, void* O,
-                           int num_sms, cudaStream_t st);
 int launch_sparse_attn_simt(const void* Q, const void* K, const void* V, int dtype, int BH, int N, int D, int NQ,
                             int NK, const int32_t* q_labels, const int32_t* k_perm, const int32_t* k_off,
                             const int32_t* kept_ptr, const int32_t* kept_idx, void* O, cudaStream_t st);

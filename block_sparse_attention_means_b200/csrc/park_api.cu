@@ -335,7 +335,7 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
     const int BH = d.BH, N = d.N, D = d.D;
     const bool bf16 = d.dtype == PARK_BF16;
     PARK_CHECK(launch_input_check(V, (size_t)BH * N * D, d.dtype, r->status, st));
-    PARK_CHECK(memset_async(r->counters + PARK_CNT_KEPT_PAIRS, 2 * sizeof(int64_t), st));
+    PARK_CHECK(memset_async(r->counters + PARK_CNT_KEPT_PAIRS, 3 * sizeof(int64_t), st));
     int32_t* icnt = at<int32_t>(ws, w.icnt);
     PARK_CHECK(memset_async(icnt, 16 * 4, st));
     if (!bf16) {

@@ -86,7 +86,7 @@ extern "C" {
 #define PARK_CNT_KEPT_BLOCKS 4  /* kept (query cluster, key cluster) pairs    */
 #define PARK_CNT_KEPT_PAIRS 5   /* sum_r |Q_r| * |J_r|: attended query-key pairs */
 #define PARK_CNT_WORK_ITEMS 6   /* query tiles scheduled for attention        */
-#define PARK_CNT_RESERVED 7
+#define PARK_CNT_KEY_TILES 7   /* (query tile, key tile) pairs computed by attention */
 #define PARK_NUM_COUNTERS 8
 
 /* Problem shape.  N = T*Hg*W + n_text. */
