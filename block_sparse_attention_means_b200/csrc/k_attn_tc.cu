@@ -35,6 +35,8 @@
 // warp-collective operations (tcgen05.ld/st, shuffles) are warp-uniform.
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -462,24 +464,27 @@ __global__ void __launch_bounds__(192, 1)
 // ---------------------------------------------------------------- host side
 namespace {
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_encode_mu;
+}  // namespace
 
-int get_encoder() {
-    if (g_encode) return PARK_OK;
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !fn) {
-        cudaGetLastError();
-        return PARK_ERR_CUDA;
+// 2-D bf16 tensor [rows][cols] (row-major), boxes of 64 columns x box_rows,
+// 128-byte swizzle.  The driver entry point is looked up once.
+int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t cols, uint32_t box_rows) {
+    {
+        std::lock_guard<std::mutex> lk(g_encode_mu);
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn) {
+                cudaGetLastError();
+                return PARK_ERR_CUDA;
+            }
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
     }
-    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    return PARK_OK;
-}
-
-// 2-D bf16 tensor [rows][128], 128-byte swizzled boxes of 64 columns x box_rows.
-int make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t box_rows) {
-    cuuint64_t dims[2] = {128, rows};
-    cuuint64_t strides[1] = {128 * 2};
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
     cuuint32_t box[2] = {64, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -487,7 +492,6 @@ int make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t box_rows
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? PARK_OK : PARK_ERR_CUDA;
 }
-}  // namespace
 
 size_t attn_tc_smem_bytes() { return (size_t)14 * TC_BLK + 1024; }  // Q, K x2, V x2, P x2
 
@@ -496,9 +500,8 @@ int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, in
                           const int32_t* kv_len,
                           const WorkItem* items, const int32_t* item_count, void* O, int32_t* status, int num_sms,
                           cudaStream_t st) {
-    PARK_CHECK(get_encoder());
     CUtensorMap mQ;
-    PARK_CHECK(make_map(&mQ, Qp, (uint64_t)BH * N, 128));
+    PARK_CHECK(make_tma_map_bf16(&mQ, Qp, (uint64_t)BH * N, 128, 128));
     const size_t sm = attn_tc_smem_bytes();
     cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     const float sl2e = (1.0f / sqrtf(128.f)) * kLog2eT;

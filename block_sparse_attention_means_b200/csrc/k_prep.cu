@@ -188,7 +188,7 @@ int launch_strided_init(const void* X, int dtype, int BH, int N, int D, int K, v
 // One CTA of D threads per (centroid, head); float64 sums in a fixed tree.
 template <typename T, bool METRIC>
 __global__ void k_centroid_prep(const T* __restrict__ C, int K, int D, const double* __restrict__ Mall,
-                                uint16_t* __restrict__ wop, float* __restrict__ bias32,
+                                uint16_t* __restrict__ wop, float* __restrict__ bias32, int bias_ld,
                                 double* __restrict__ bias64, double* __restrict__ w64, float* __restrict__ wmax,
                                 float* __restrict__ bmax) {
     __shared__ double cs[128];
@@ -223,10 +223,13 @@ __global__ void k_centroid_prep(const T* __restrict__ C, int K, int D, const dou
         }
         __syncthreads();
     }
+    if (k == 0)  // columns past K read +inf, so a score GEMM over whole 128-column chunks never picks them
+        for (int j = K + a; j < ((K + 127) & ~127); j += blockDim.x)
+            bias32[(size_t)bh * bias_ld + j] = __int_as_float(0x7f800000);
     if (a == 0) {
         double b = red[0][0];
         bias64[(size_t)bh * K + k] = b;
-        bias32[(size_t)bh * K + k] = __double2float_rn(b);
+        bias32[(size_t)bh * bias_ld + k] = __double2float_rn(b);
         atomic_max_nonneg(wmax + bh, round_up_f(__double2float_ru(sqrt(red[1][0]))));
         atomic_max_nonneg(bmax + bh, round_up_f(__double2float_ru(fabs(b))));
     }
@@ -240,17 +243,17 @@ int launch_centroid_prep(const void* C, int dtype, int BH, int K, int D, const d
     ::park::prof_begin(st);
     if (dtype == PARK_BF16) {
         if (metric)
-            k_centroid_prep<bf16_t, true><<<g, D, 0, st>>>((const bf16_t*)C, K, D, M, (uint16_t*)ops.w, ops.bias32,
+            k_centroid_prep<bf16_t, true><<<g, D, 0, st>>>((const bf16_t*)C, K, D, M, (uint16_t*)ops.w, ops.bias32, ops.bias_ld,
                                                           ops.bias64, ops.w64, ops.wmax, ops.bmax);
         else
-            k_centroid_prep<bf16_t, false><<<g, D, 0, st>>>((const bf16_t*)C, K, D, M, nullptr, ops.bias32,
+            k_centroid_prep<bf16_t, false><<<g, D, 0, st>>>((const bf16_t*)C, K, D, M, nullptr, ops.bias32, ops.bias_ld,
                                                            ops.bias64, ops.w64, ops.wmax, ops.bmax);
     } else {
         if (metric)
-            k_centroid_prep<float, true><<<g, D, 0, st>>>((const float*)C, K, D, M, (uint16_t*)ops.w, ops.bias32,
+            k_centroid_prep<float, true><<<g, D, 0, st>>>((const float*)C, K, D, M, (uint16_t*)ops.w, ops.bias32, ops.bias_ld,
                                                          ops.bias64, ops.w64, ops.wmax, ops.bmax);
         else
-            k_centroid_prep<float, false><<<g, D, 0, st>>>((const float*)C, K, D, M, nullptr, ops.bias32,
+            k_centroid_prep<float, false><<<g, D, 0, st>>>((const float*)C, K, D, M, nullptr, ops.bias32, ops.bias_ld,
                                                           ops.bias64, ops.w64, ops.wmax, ops.bmax);
     }
     PARK_TRY_LAUNCH("k_centroid_prep", st);

@@ -3,6 +3,7 @@
 // code (PARK_ERR_CUDA when the launch itself failed).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -15,7 +16,8 @@ struct CentroidOps {
     const uint16_t* w;  // bf16 [BH][K][kw]   (queries: the centroids themselves, kw = D;
                         //                     keys: hi/lo split of M c, kw = 2D)
     int kw;
-    float* bias32;      // [BH][K]  bias rounded to float
+    float* bias32;      // [BH][bias_ld]  bias rounded to float
+    int bias_ld;        // leading dimension of bias32 (multiple of 128, >= K)
     double* bias64;     // [BH][K]  ||c||^2 (queries) or c^T M c (keys)
     double* w64;        // [BH][K][D] M c in float64 (keys only)
     float* wmax;        // [BH] max_k ||w_k||  (rounded up)
@@ -39,8 +41,9 @@ int launch_centroid_prep(const void* C, int dtype, int BH, int K, int D, const d
                          cudaStream_t st);
 
 // ---- k_assign.cu
-int launch_assign_mma(const void* X, int BH, int N, int K, const CentroidOps& ops, const float* xnorm,
-                      float gamma, int32_t* labels, Lists lists, cudaStream_t st);
+// k_assign_tc.cu: tcgen05 score GEMM with the certified top-3 epilogue (bf16, D = 128)
+int launch_assign_tc(const void* X, int BH, int N, int K, const CentroidOps& ops, const float* xnorm, float gamma,
+                     int32_t* labels, Lists lists, int32_t* status, int num_sms, cudaStream_t st);
 int launch_recheck(const void* X, int dtype, int BH, int N, int D, int K, const void* C, const double* w64,
                    const double* b64, int32_t* labels, Lists lists, int all_rows, int num_sms,
                    int64_t* counters, int cnt_slot, cudaStream_t st);
@@ -84,6 +87,9 @@ int launch_kv_pad_gather(const void* K, const void* V, int BH, int N, int NK, in
                          const int32_t* k_labels, const int32_t* k_off, int32_t* poff, void* Kpad, void* Vpad,
                          cudaStream_t st);
 size_t attn_tc_smem_bytes();
+// TMA descriptor for a row-major bf16 [rows][cols] tensor, boxes of 64 columns x
+// box_rows, 128-byte swizzle (k_attn_tc.cu).
+int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t cols, uint32_t box_rows);
 int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
                           const int32_t* q_perm, const int2* segs, const int32_t* kept_ptr, const int32_t* kv_pre,
                           const int32_t* kv_len,

@@ -131,7 +131,7 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
     w.xnorm_q = c.take(BH * N * 4);
     w.xnorm_k = c.take(BH * N * 4);
     w.wop = c.take(BH * Km * 2 * D * 2);
-    w.b32 = c.take(BH * Km * 4);
+    w.b32 = c.take(BH * align_up(Km, 128) * 4);
     w.b64 = c.take(BH * Km * 8);
     w.w64 = c.take(BH * Km * D * 8);
     w.wmax = c.take(BH * 4);
@@ -225,6 +225,8 @@ struct Side {
     bool warm;
     int cnt_slot;
     float* xnorm;
+    int Kmax;          // max(NQ, NK): leading dimension of the shared bias buffer
+    int32_t* status;
 };
 
 int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, void* ws, int64_t* counters,
@@ -234,6 +236,7 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
     const int nchunks = (N + kSortChunk - 1) / kSortChunk;
     CentroidOps ops;
     ops.bias32 = at<float>(ws, w.b32);
+    ops.bias_ld = (int)align_up((size_t)(s.Kmax), 128);
     ops.bias64 = at<double>(ws, w.b64);
     ops.w64 = s.M ? at<double>(ws, w.w64) : nullptr;
     ops.wmax = at<float>(ws, w.wmax);
@@ -259,7 +262,7 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
         PARK_CHECK(memset_async(lists.counts, 16 * 4, st));
         PARK_CHECK(launch_centroid_prep(s.C, d.dtype, BH, K, D, s.M, ops, st));
         if (bf16) {
-            PARK_CHECK(launch_assign_mma(s.X, BH, N, K, ops, s.xnorm, gamma, s.labels, lists, st));
+            PARK_CHECK(launch_assign_tc(s.X, BH, N, K, ops, s.xnorm, gamma, s.labels, lists, s.status, num_sms, st));
             PARK_CHECK(launch_recheck(s.X, d.dtype, BH, N, D, K, s.C, ops.w64, ops.bias64, s.labels, lists, 0,
                                       num_sms, counters, s.cnt_slot, st));
         } else {
@@ -298,17 +301,19 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
     PARK_CHECK(launch_metric(Q, d.dtype, BH, N, D, at<double>(ws, w.Mpart), metric_chunks(d), M, out->metric, st));
 
     Side sq{Q, NQ, out->q_centroids, out->q_labels, out->q_perm, out->q_offsets, nullptr,
-            (out->flags & PARK_FLAG_WARM_START_Q) != 0, PARK_CNT_Q_RECHECK, at<float>(ws, w.xnorm_q)};
+            (out->flags & PARK_FLAG_WARM_START_Q) != 0, PARK_CNT_Q_RECHECK, at<float>(ws, w.xnorm_q),
+            NQ > NK ? NQ : NK, out->status};
     Side sk{K, NK, out->k_centroids, out->k_labels, out->k_perm, out->k_offsets, M,
-            (out->flags & PARK_FLAG_WARM_START_K) != 0, PARK_CNT_K_RECHECK, at<float>(ws, w.xnorm_k)};
+            (out->flags & PARK_FLAG_WARM_START_K) != 0, PARK_CNT_K_RECHECK, at<float>(ws, w.xnorm_k),
+            NQ > NK ? NQ : NK, out->status};
     PARK_CHECK(run_kmeans(d, sq, iters, w, ws, out->counters, num_sms, st));
     PARK_CHECK(run_kmeans(d, sk, iters, w, ws, out->counters, num_sms, st));
 
     int32_t* kcnt = at<int32_t>(ws, w.kcnt);
     if (d.dtype == PARK_BF16) {
         // max ||c_m|| over the final key centroids, for the PAMA bound
-        CentroidOps ops{nullptr, D, at<float>(ws, w.b32), at<double>(ws, w.b64), nullptr, at<float>(ws, w.wmax),
-                        at<float>(ws, w.bmax)};
+        CentroidOps ops{nullptr, D, at<float>(ws, w.b32), (int)align_up((size_t)(NQ > NK ? NQ : NK), 128),
+                        at<double>(ws, w.b64), nullptr, at<float>(ws, w.wmax), at<float>(ws, w.bmax)};
         PARK_CHECK(memset_async(ops.wmax, (size_t)BH * 4, st));
         PARK_CHECK(memset_async(ops.bmax, (size_t)BH * 4, st));
         PARK_CHECK(launch_centroid_prep(out->k_centroids, d.dtype, BH, NK, D, nullptr, ops, st));
