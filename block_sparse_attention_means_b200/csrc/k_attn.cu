@@ -108,8 +108,11 @@ __global__ __launch_bounds__(256) void k_attn_schedule(int NQ, int NK, const int
             atomicAdd((unsigned long long*)(counters + PARK_CNT_KEPT_PAIRS),
                       (unsigned long long)nr * (unsigned long long)total_u);
             atomicAdd((unsigned long long*)(counters + PARK_CNT_WORK_ITEMS), (unsigned long long)tiles);
+            // (query tile, key tile) products: 128 x 128 on the tensor-core path, whose
+            // items are up to two 128-row query halves
+            const int qt = pad8 ? (nr + 127) / 128 : tiles, kt = pad8 ? (total + 127) / 128 : (total + tile_rows - 1) / tile_rows;
             atomicAdd((unsigned long long*)(counters + PARK_CNT_KEY_TILES),
-                      (unsigned long long)tiles * (unsigned long long)((total + tile_rows - 1) / tile_rows));
+                      (unsigned long long)qt * (unsigned long long)kt);
         }
     }
 }

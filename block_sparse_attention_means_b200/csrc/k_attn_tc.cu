@@ -13,7 +13,7 @@
 // the part of a kept cluster that falls in a tile arrives with one bulk copy
 // for K and one for V; pad rows and groups past the end are masked.
 //
-// One CTA per SM (persistent, work items round-robin), 6 warps:
+// One CTA per SM (persistent, work items round-robin), 10 warps:
 //   warp 0     producer: Q tile (128 x 128, TMA) per item; K and V tiles (bulk
 //              copies, one per kept-cluster piece) into two 2-stage rings with
 //              separate barriers, so K of tile j+2 may arrive while V of tile
@@ -21,14 +21,20 @@
 //              masked rows;
 //   warp 1     TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into TMEM
 //              buffer j%2 (128 x 128 fp32), O += P_j V_j into a TMEM
-//              accumulator (128 x 128 fp32), in the order S0 S1 PV0 S2 PV1 S3 ...
-//   warps 2-5  Softmax: thread = query row = TMEM lane.  Loads S_j, online
-//              Softmax in the log2 domain with a lazily updated reference max
-//              (O is rescaled in TMEM only when a row max grows by more than
-//              2^8), writes P_j as bf16 into shared-memory buffer j%2 in the
-//              swizzled K-major layout of the PV MMA (two buffers: writing P_j
-//              only waits for PV_{j-2}), and finally normalises O and writes the
-//              rows in original token order.
+//              accumulator (128 x 128 fp32) with P_j read from TMEM, in the
+//              order S0 S1 PV0 S2 PV1 S3 ...; tcgen05 MMAs of one thread run in
+//              issue order, so S_{j+2} overwrites buffer j%2 only after PV_j has
+//              read P_j from it.
+//   warps 2-9  Softmax, two threads per query row (= TMEM lane; warps w and
+//              w+4 share a lane quadrant), each owning 64 of a tile's 128
+//              columns.  Online Softmax in the log2 domain with a lazily
+//              updated reference max (O is rescaled in TMEM only when a row max
+//              grows by more than 2^8); the two halves exchange their tile
+//              maxima through shared memory so both use the same reference.
+//              P_j is written as bf16 pairs over the first 64 columns of S_j's
+//              TMEM buffer (the A operand of the PV MMA).  At the end the two
+//              partial row sums are added, and each thread normalises and
+//              writes its half of the O row in original token order.
 // Every wait is time-bounded; a timeout sets PARK_ERR_TIMEOUT in the status
 // word, the roles leave their loops, outstanding copies and MMAs are waited
 // for (bounded) and TMEM is freed before the CTA exits.  Decisions that guard
@@ -52,11 +58,13 @@ constexpr float kLog2eT = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
 
 struct TcSmem {
-    uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_empty[2], p_full[2],
-        pv_done[2], o_empty, final_bar;
+    uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], pv_done[2],
+        o_empty, final_bar;
     uint32_t tmem_base;
     int abort;
     alignas(16) float bias[2][TC_ROWS];  // per stage: 0 for a real key row, -inf for a pad row or past the end
+    float xmax[2][2][TC_ROWS];           // [tile parity][column half][row]: tile maxima of the two halves
+    float xl[2][TC_ROWS];                // [column half][row]: partial row sums
 };
 }  // namespace
 
@@ -69,7 +77,7 @@ __device__ __forceinline__ float fast_ex2(float x) {
     return y;
 }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     k_sparse_attn_tc(const __grid_constant__ CUtensorMap tmQ, const uint8_t* __restrict__ Kimg,
                      const uint8_t* __restrict__ Vimg, int N, int NQ, int NK, const int32_t* __restrict__ q_perm,
                      const int2* __restrict__ segs, const int32_t* __restrict__ kept_ptr,
@@ -78,12 +86,11 @@ __global__ void __launch_bounds__(192, 1)
                      uint16_t* __restrict__ O, float sl2e, int32_t* __restrict__ status) {
     extern __shared__ __align__(1024) uint8_t dsmem_raw[];
     __shared__ TcSmem sh;
-    // 1024-byte aligned operand area: Q | K0 K1 | V0 V1 | P0 P1 (each 32 KB)
+    // 1024-byte aligned operand area: Q | K0 K1 | V0 V1 (each 32 KB)
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* Qs = base;
     uint8_t* Ks = base + 2 * TC_BLK;
     uint8_t* Vs = Ks + 4 * TC_BLK;
-    uint8_t* Ps = Vs + 4 * TC_BLK;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort = &sh.abort;
@@ -96,11 +103,10 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&sh.v_full[s], 1);
             mbar_init(&sh.v_empty[s], 1);
             mbar_init(&sh.s_full[s], 1);
-            mbar_init(&sh.s_empty[s], 128);
-            mbar_init(&sh.p_full[s], 128);
+            mbar_init(&sh.p_full[s], 256);
             mbar_init(&sh.pv_done[s], 1);
         }
-        mbar_init(&sh.o_empty, 128);
+        mbar_init(&sh.o_empty, 256);
         mbar_init(&sh.final_bar, 1);
         sh.abort = 0;
         mbar_fence_init();
@@ -120,7 +126,7 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem = sh.tmem_base;
     const int n_items = *item_count;
     const uint32_t idS = idesc_bf16(128, 128, 0, 0);   // S = Q K^T: both K-major
-    const uint32_t idPV = idesc_bf16(128, 128, 0, 1);  // O += P V: P K-major, V MN-major
+    const uint32_t idPV = idesc_bf16(128, 128, 0, 1);  // O += P V: P K-major (TMEM), V MN-major
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -260,8 +266,8 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t qa = smem_u32(Qs);
             auto issue_S = [&](int g) -> bool {
                 const int b = g & 1, round = g >> 1;
+                // buffer b is free: its last reader, PV_{g-2}, was issued before this MMA
                 if (!mbar_wait(&sh.k_full[b], round & 1, abort)) return false;
-                if (round > 0 && !mbar_wait(&sh.s_empty[b], (round - 1) & 1, abort)) return false;
                 tc_fence_after();
                 const uint32_t ka = smem_u32(Ks + b * 2 * TC_BLK);
                 const uint32_t d = tmem + (uint32_t)(b * 128);
@@ -292,13 +298,11 @@ __global__ void __launch_bounds__(192, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t pa = smem_u32(Ps + b * 2 * TC_BLK), va = smem_u32(Vs + b * 2 * TC_BLK);
+                    const uint32_t va = smem_u32(Vs + b * 2 * TC_BLK);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t poff = (uint32_t)((kk >> 2) * TC_BLK + (kk & 3) * 32);
-                        umma_bf16(tmem + 256, sdesc_sw128(pa + poff, 16, 1024),
-                                  sdesc_sw128(va + (uint32_t)kk * 4096, 1024, 2048), idPV, (j > 0 || kk > 0));
-                    }
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16_ts(tmem + 256, tmem + (uint32_t)(b * 128 + 8 * kk),
+                                     sdesc_sw128(va + (uint32_t)kk * 4096, 1024, 2048), idPV, (j > 0 || kk > 0));
                     umma_commit(&sh.pv_done[b]);
                     umma_commit(&sh.v_empty[b]);
                     if (j + 2 < nkt && !issue_S(g + 2)) ok = false;
@@ -316,126 +320,134 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
-        const int lane_base = 32 * (warp & 3);
-        const int row = lane_base + lane;
-        const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
-        int G = 0, I = 0;
-        // waits are decided per warp: tcgen05.ld/st and shuffles below are warp-collective
-        auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
-            const bool ok = mbar_wait(bar, parity, abort);
-            return __all_sync(0xffffffffu, ok);
+        const int quad = warp & 3, hc = (warp - 2) >> 2;  // lane quadrant, column half
+        const int row = 32 * quad + lane;
+        const uint32_t trow = tmem + ((uint32_t)(32 * quad) << 16);
+        const int pair_bar = 1 + quad;  // named barrier of warps w and w+4 (64 threads)
+        int G = 0;
+        // Waits are decided per warp (tcgen05.ld/st and shuffles are warp-collective).
+        // The two warps of a pair pass their named barrier the same number of times
+        // whatever happens: after a failed wait a warp skips every later wait and all
+        // tensor-memory work but still walks the items and meets its barriers.
+        bool failed = false;
+        auto wwait = [&](uint64_t* bar, uint32_t parity) {
+            if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+            return !failed;
         };
-        for (int it = blockIdx.x; it < n_items && !warp_abort(abort); it += gridDim.x) {
+        for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
             const WorkItem wi = items[it];
             const int L = kv_len[(size_t)wi.bh * NQ + wi.r];
             const int nkt = (L + TC_ROWS - 1) / TC_ROWS;
             if (nkt == 0) continue;
             float m_ref = __int_as_float(0xff800000), l = 0.f;
-            bool ok = true;
             for (int j = 0; j < nkt; ++j) {
                 const int g = G + j, b = g & 1, ph = (g >> 1) & 1;
-                if (!wwait(&sh.s_full[b], ph) || !wwait(&sh.v_full[b], ph)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                uint32_t s[4][32];
+                const bool live = wwait(&sh.s_full[b], ph) && wwait(&sh.v_full[b], ph);
+                uint32_t s[2][32];
+                float tm[4] = {__int_as_float(0xff800000), __int_as_float(0xff800000), __int_as_float(0xff800000),
+                               __int_as_float(0xff800000)};
+                if (live) {
+                    tc_fence_after();
+                    tmem_ld32(trow + (uint32_t)(b * 128 + 64 * hc), s[0]);
+                    tmem_ld32(trow + (uint32_t)(b * 128 + 64 * hc + 32), s[1]);
+                    tmem_ld_wait();
+                    tmem_ld_dep(s[0]);
+                    tmem_ld_dep(s[1]);
+                    const float4* bz = reinterpret_cast<const float4*>(sh.bias[b] + 64 * hc);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(trow + (uint32_t)(b * 128 + 32 * c), s[c]);
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(&sh.s_empty[b]);
-                const float4* bz = reinterpret_cast<const float4*>(sh.bias[b]);
-                float tmax = __int_as_float(0xff800000);
+                    for (int c = 0; c < 2; ++c) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 bb = bz[c * 8 + q];
-                        const float x0 = fmaf(bits_f(s[c][4 * q + 0]), sl2e, bb.x);
-                        const float x1 = fmaf(bits_f(s[c][4 * q + 1]), sl2e, bb.y);
-                        const float x2 = fmaf(bits_f(s[c][4 * q + 2]), sl2e, bb.z);
-                        const float x3 = fmaf(bits_f(s[c][4 * q + 3]), sl2e, bb.w);
-                        s[c][4 * q + 0] = __float_as_uint(x0);
-                        s[c][4 * q + 1] = __float_as_uint(x1);
-                        s[c][4 * q + 2] = __float_as_uint(x2);
-                        s[c][4 * q + 3] = __float_as_uint(x3);
-                        tmax = fmaxf(tmax, fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 bb = bz[c * 8 + q];
+                            const float x0 = fmaf(bits_f(s[c][4 * q + 0]), sl2e, bb.x);
+                            const float x1 = fmaf(bits_f(s[c][4 * q + 1]), sl2e, bb.y);
+                            const float x2 = fmaf(bits_f(s[c][4 * q + 2]), sl2e, bb.z);
+                            const float x3 = fmaf(bits_f(s[c][4 * q + 3]), sl2e, bb.w);
+                            s[c][4 * q + 0] = __float_as_uint(x0);
+                            s[c][4 * q + 1] = __float_as_uint(x1);
+                            s[c][4 * q + 2] = __float_as_uint(x2);
+                            s[c][4 * q + 3] = __float_as_uint(x3);
+                            tm[0] = fmaxf(tm[0], x0);
+                            tm[1] = fmaxf(tm[1], x1);
+                            tm[2] = fmaxf(tm[2], x2);
+                            tm[3] = fmaxf(tm[3], x3);
+                        }
                     }
                 }
+                // Both halves of the row agree on the tile max.  The barrier also orders
+                // the partner's S loads before this thread's P stores over them.
+                sh.xmax[j & 1][hc][row] = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+                tc_fence_before();
+                named_bar_sync(pair_bar, 64);
+                tc_fence_after();
+                if (!live) continue;
+                const float tmax = fmaxf(sh.xmax[j & 1][0][row], sh.xmax[j & 1][1][row]);
                 if (j == 0) {
                     m_ref = tmax;
                 } else if (__any_sync(0xffffffffu, tmax > m_ref + kRescaleThreshold)) {
-                    // decided per warp (TMEM loads/stores are warp-collective); rows that do
-                    // not need a new reference keep theirs (alpha = 1).  O must hold PV_{j-1}.
-                    if (!wwait(&sh.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) {
-                        ok = false;
-                        break;
-                    }
+                    // decided per warp, identically in both warps of the pair (same rows,
+                    // same maxima); rows that keep their reference get alpha = 1.  O must
+                    // hold PV_{j-1}.
+                    if (!wwait(&sh.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) continue;
                     tc_fence_after();
                     const float m_new = tmax > m_ref + kRescaleThreshold ? tmax : m_ref;
                     const float alpha = fast_ex2(m_ref - m_new);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 2; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(trow + 256u + 32u * c, o);
+                        tmem_ld32(trow + 256u + (uint32_t)(64 * hc + 32 * c), o);
                         tmem_ld_wait();
+                        tmem_ld_dep(o);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(bits_f(o[e]) * alpha);
-                        tmem_st32(trow + 256u + 32u * c, o);
+                        tmem_st32(trow + 256u + (uint32_t)(64 * hc + 32 * c), o);
                     }
                     tmem_st_wait();
                     l *= alpha;
                     m_ref = m_new;
                 }
-                // P buffer b was last read by PV_{j-2} (for j < 2 the previous item's
-                // epilogue already waited for all of its PVs)
-                if (j >= 2 && !wwait(&sh.pv_done[b], ((g - 2) >> 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                // P row -> shared memory, K-major, 128-byte swizzle: chunk c16 of row r at c16 ^ (r & 7)
-                uint8_t* Pb = Ps + b * 2 * TC_BLK;
+                // P (bf16 pairs) over the first 64 columns of buffer b: this half's 64
+                // keys are packed columns [32 hc, 32 hc + 32)
+                uint32_t pk[32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t pk[16];
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const float p0 = fast_ex2(bits_f(s[c][2 * e]) - m_ref);
                         const float p1 = fast_ex2(bits_f(s[c][2 * e + 1]) - m_ref);
                         l += p0 + p1;
                         __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                        pk[e] = *reinterpret_cast<uint32_t*>(&h);
+                        pk[16 * c + e] = *reinterpret_cast<uint32_t*>(&h);
                     }
-                    uint8_t* blk = Pb + (c >> 1) * TC_BLK + row * 128;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int c16 = (c & 1) * 4 + q;
-                        *reinterpret_cast<uint4*>(blk + ((c16 ^ (row & 7)) << 4)) =
-                            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                    }
-                }
-                fence_proxy_async_smem();
+                tmem_st32(trow + (uint32_t)(b * 128 + 32 * hc), pk);
+                tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&sh.p_full[b]);
             }
-            if (!ok) break;
-            // epilogue: O / l, original token order
+            // epilogue: O / l, original token order; each thread writes its 64 columns.
+            // The partner overwrites xl only after its next item's first pair barrier,
+            // which this thread reaches after reading xl.
+            sh.xl[hc][row] = l;
+            named_bar_sync(pair_bar, 64);
+            const float lt = sh.xl[0][row] + sh.xl[1][row];
             const int gl = G + nkt - 1;
-            if (!wwait(&sh.pv_done[gl & 1], (gl >> 1) & 1)) break;
+            G += nkt;
+            if (!wwait(&sh.pv_done[gl & 1], (gl >> 1) & 1)) continue;
             tc_fence_after();
-            uint32_t o[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(trow + 256u + 32u * c, o[c]);
+            uint32_t o[2][32];
+            tmem_ld32(trow + 256u + (uint32_t)(64 * hc), o[0]);
+            tmem_ld32(trow + 256u + (uint32_t)(64 * hc + 32), o[1]);
             tmem_ld_wait();
+            tmem_ld_dep(o[0]);
+            tmem_ld_dep(o[1]);
             tc_fence_before();
             mbar_arrive(&sh.o_empty);
             if (row < wi.rows) {
-                const float inv = l > 0.f ? 1.f / l : 0.f;
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
                 const int tok = q_perm[(size_t)wi.bh * N + wi.q_start + row];
-                uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)wi.bh * N + tok) * 128);
+                uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)wi.bh * N + tok) * 128 + 64 * hc);
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint32_t w4[4];
@@ -448,8 +460,6 @@ __global__ void __launch_bounds__(192, 1)
                         dst[c * 4 + q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
             }
-            G += nkt;
-            ++I;
         }
     }
     tc_fence_before();
@@ -493,7 +503,7 @@ int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t
     return r == CUDA_SUCCESS ? PARK_OK : PARK_ERR_CUDA;
 }
 
-size_t attn_tc_smem_bytes() { return (size_t)14 * TC_BLK + 1024; }  // Q, K x2, V x2, P x2
+size_t attn_tc_smem_bytes() { return (size_t)10 * TC_BLK + 1024; }  // Q, K x2, V x2
 
 int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
                           const int32_t* q_perm, const int2* segs, const int32_t* kept_ptr, const int32_t* kv_pre,
@@ -506,7 +516,7 @@ int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, in
     cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     const float sl2e = (1.0f / sqrtf(128.f)) * kLog2eT;
     ::park::prof_begin(st);
-    k_sparse_attn_tc<<<num_sms, 192, sm, st>>>(mQ, (const uint8_t*)Kpad, (const uint8_t*)Vpad, N, NQ, NK, q_perm,
+    k_sparse_attn_tc<<<num_sms, 320, sm, st>>>(mQ, (const uint8_t*)Kpad, (const uint8_t*)Vpad, N, NQ, NK, q_perm,
                                                 segs, kept_ptr, kv_pre, kv_len, items, item_count, (uint16_t*)O,
                                                 sl2e, status);
     PARK_TRY_LAUNCH("k_sparse_attn_tc", st);
