@@ -384,51 +384,64 @@ int launch_topp(const float* importance, const float* rho, int BH, int NQ, int N
 }
 
 // ---------------------------------------------------------------- float64 PAMA + top-p
-// One CTA (256 threads, persistent over the list) per listed (head, query
-// cluster), or per cluster of every head when all_clusters is set.  The
-// cluster's rows are staged 64 at a time in shared memory as float64 and the
-// key centroids stream through in chunks of 64.  Thread t owns the 4 x 4 logit
-// block rows 4*(t/16)+i, columns (t%16)+16u of the 64 x 64 tile.
-//   pass 1: per-row max and sum of exp over every non-empty key cluster
-//           (online per thread, then merged over the 16 threads of a row group);
-//   pass 2: P = exp(z - max) / sum, summed over the rows into per-row-group
-//           column partials that are added in a fixed order.
+// One CTA (256 threads) per listed (head, query cluster), or per cluster of
+// every head when all_clusters is set; CTAs take clusters from an atomic work
+// counter.  The cluster's rows are staged RT at a time in shared memory as
+// float64, transposed (Qs[k][row]); the key centroids stream through in
+// chunks of 64 (Cs[k][col]), the next chunk prefetched through registers while
+// the current one is used.  Thread (ty, tx) of a 16 x 16 grid owns the RPT x 4
+// logit block rows ty*RPT + i, columns 4*tx + u of the RT x 64 tile (RT = 16
+// RPT), read with 16-byte shared loads.
+//   pass 1: logits z (scaled; -inf for empty key clusters) into the CTA's
+//           float64 scratch, and the row max;
+//   pass 2: e = exp(z - max) over the scratch, row sums;
+//   pass 3: P = e / sum, summed over the rows into per-row-group column
+//           partials that are added in a fixed order.
 // Then I = column sums / |Q_r| is sorted (descending, ties by m) and a
 // sequential float64 running sum finds the cut, as the definition reads.
-constexpr int F64_TILE = 64, F64_LD = 129;  // padded rows: conflict-free column reads
+constexpr int F64_CH = 64;  // centroids per chunk
 
-template <typename T>
+template <typename T, int RPT>
 __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, const int32_t* __restrict__ q_perm,
                                                      const int32_t* __restrict__ q_off, const T* __restrict__ CK,
                                                      const int32_t* __restrict__ k_off, int N, int D, int NQ, int NK,
                                                      int NKP, double scale, float p, const int32_t* __restrict__ list,
                                                      const int32_t* __restrict__ count_ptr, int all_clusters,
-                                                     int BHNQ, float* __restrict__ importance,
+                                                     int BHNQ, int32_t* __restrict__ work_ctr,
+                                                     double* __restrict__ zscratch, float* __restrict__ importance,
                                                      float* __restrict__ importance_bound,
                                                      uint8_t* __restrict__ mask, int32_t* __restrict__ kept_cnt,
                                                      int64_t* __restrict__ counters) {
+    constexpr int RT = 16 * RPT, DM = 128, ZB = RPT * 4;
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    double* Qs = reinterpret_cast<double*>(smem_raw);         // [64][129]
-    double* Cs = Qs + F64_TILE * F64_LD;                      // [64][129]
-    double* Isum = Cs + F64_TILE * F64_LD;                    // [NKP]
-    double* part = Isum + NKP;                                // [16][64]
-    int32_t* si = reinterpret_cast<int32_t*>(part + 16 * 64); // [NKP]
-    uint8_t* live = reinterpret_cast<uint8_t*>(si + NKP);     // [NKP]
-    __shared__ int s_cut;
+    double* Qs = reinterpret_cast<double*>(smem_raw);          // [DM][RT]
+    double* Cs = Qs + DM * RT;                                 // [DM][F64_CH]
+    double* Isum = Cs + DM * F64_CH;                           // [NKP]
+    double* part = Isum + NKP;                                 // [16][F64_CH]
+    int32_t* si = reinterpret_cast<int32_t*>(part + 16 * F64_CH);  // [NKP]
+    uint8_t* live = reinterpret_cast<uint8_t*>(si + NKP);      // [NKP]
+    __shared__ int s_cut, s_e;
     const double NEG_INF = __longlong_as_double(0xfff0000000000000ll);
     const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
     const int count = all_clusters ? BHNQ : *count_ptr;
     if (blockIdx.x == 0 && t == 0 && !all_clusters && counters)
         atomicAdd((unsigned long long*)(counters + PARK_CNT_PAMA_RECHECK), (unsigned long long)count);
-    const int nch = (NK + F64_TILE - 1) / F64_TILE;
-    for (int e = blockIdx.x; e < count; e += gridDim.x) {
+    const int nch = (NK + F64_CH - 1) / F64_CH;
+    double* zs = zscratch + (size_t)blockIdx.x * nch * 256 * ZB;  // this CTA's scratch
+    // chunk staging: thread t holds centroid (t >> 2) of the chunk, dims (t & 3) + 4 v
+    constexpr int CPT = F64_CH * DM / 256;  // elements per thread (32)
+    for (;;) {
+        __syncthreads();  // previous entry's shared memory fully consumed
+        if (t == 0) s_e = atomicAdd(work_ctr, 1);
+        __syncthreads();
+        const int e = s_e;
+        if (e >= count) break;
         const int row = all_clusters ? e : list[e];
         const int bh = row / NQ, r = row - bh * NQ;
         const int qs = q_off[(size_t)bh * (NQ + 1) + r], nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - qs;
         const int32_t* ko = k_off + (size_t)bh * (NK + 1);
         uint8_t* mrow = mask + (size_t)row * NK;
         float* Irow = importance + (size_t)row * NK;
-        __syncthreads();  // previous entry's shared memory fully consumed
         if (nr == 0) {
             for (int m = t; m < NK; m += blockDim.x) {
                 mrow[m] = 0;
@@ -447,101 +460,127 @@ __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, co
         const T* Ch = CK + (size_t)bh * NK * D;
         const T* Qh = Q + (size_t)bh * N * D;
         const int32_t* pm = q_perm + (size_t)bh * N + qs;
-        auto load_chunk = [&](int c) {
-            for (int idx = t; idx < F64_TILE * D; idx += blockDim.x) {
-                int cc = idx / D, j = idx - cc * D, m = c * F64_TILE + cc;
-                Cs[cc * F64_LD + j] = m < NK ? Elem<T>::to_double(Ch + (size_t)m * D, j) : 0.0;
+        float cpre[CPT];  // inputs are exact in float32 (bf16 or float32)
+        auto fetch_chunk = [&](int c) {  // global -> registers
+            const int m = c * F64_CH + (t >> 2);
+#pragma unroll
+            for (int v = 0; v < CPT; ++v) {
+                const int k = (t & 3) + 4 * v;
+                cpre[v] = (m < NK && k < D) ? Elem<T>::to_float(Ch + (size_t)m * D, k) : 0.f;
             }
         };
-        auto logits = [&](double (&z)[4][4]) {
+        auto store_chunk = [&]() {  // registers -> Cs[k][col]
+            const int col = t >> 2;
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int u = 0; u < 4; ++u) z[i][u] = 0.0;
-            for (int j = 0; j < D; ++j) {
-                double a[4], b[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) a[i] = Qs[(ty * 4 + i) * F64_LD + j];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) b[u] = Cs[(tx + 16 * u) * F64_LD + j];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) z[i][u] = __fma_rn(a[i], b[u], z[i][u]);
-            }
+            for (int v = 0; v < CPT; ++v) Cs[((t & 3) + 4 * v) * F64_CH + col] = (double)cpre[v];
         };
-        for (int t0 = 0; t0 < nr; t0 += F64_TILE) {
+        for (int t0 = 0; t0 < nr; t0 += RT) {
             __syncthreads();  // Qs free
-            for (int idx = t; idx < F64_TILE * D; idx += blockDim.x) {
-                int rr = idx / D, j = idx - rr * D;
-                Qs[rr * F64_LD + j] = t0 + rr < nr ? Elem<T>::to_double(Qh + (size_t)pm[t0 + rr] * D, j) : 0.0;
+            for (int idx = t; idx < RT * DM; idx += blockDim.x) {
+                const int k = idx / RT, rr = idx - k * RT;
+                Qs[k * RT + rr] = (t0 + rr < nr && k < D) ? Elem<T>::to_double(Qh + (size_t)pm[t0 + rr] * D, k) : 0.0;
             }
-            double mx[4], sm[4];
+            // pass 1: logits into the scratch, row max
+            double mx[RPT];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                mx[i] = NEG_INF;
-                sm[i] = 0.0;
-            }
-            for (int c = 0; c < nch; ++c) {  // pass 1
+            for (int i = 0; i < RPT; ++i) mx[i] = NEG_INF;
+            fetch_chunk(0);
+            for (int c = 0; c < nch; ++c) {
+                __syncthreads();  // Cs free (and Qs staged)
+                store_chunk();
                 __syncthreads();
-                load_chunk(c);
-                __syncthreads();
-                double z[4][4];
-                logits(z);
+                if (c + 1 < nch) fetch_chunk(c + 1);  // in flight during the GEMM
+                double z[RPT][4];
+#pragma unroll
+                for (int i = 0; i < RPT; ++i)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) z[i][u] = 0.0;
+#pragma unroll 2
+                for (int k = 0; k < DM; ++k) {
+                    double a[RPT], b[4];
+#pragma unroll
+                    for (int i = 0; i < RPT; i += 2) {
+                        const double2 q2 = *reinterpret_cast<const double2*>(Qs + k * RT + ty * RPT + i);
+                        a[i] = q2.x;
+                        a[i + 1] = q2.y;
+                    }
+                    const double2 c0 = *reinterpret_cast<const double2*>(Cs + k * F64_CH + 4 * tx);
+                    const double2 c1 = *reinterpret_cast<const double2*>(Cs + k * F64_CH + 4 * tx + 2);
+                    b[0] = c0.x;
+                    b[1] = c0.y;
+                    b[2] = c1.x;
+                    b[3] = c1.y;
+#pragma unroll
+                    for (int i = 0; i < RPT; ++i)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) z[i][u] = __fma_rn(a[i], b[u], z[i][u]);
+                }
+                double2* zb = reinterpret_cast<double2*>(zs + ((size_t)c * 256 + t) * ZB);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int col = c * F64_TILE + tx + 16 * u;
-                    if (col < NK && live[col]) {
+                    const int col = c * F64_CH + 4 * tx + u;
+                    const bool lv = col < NK && live[col];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            double zz = scale * z[i][u];
-                            if (zz > mx[i]) {
-                                sm[i] = sm[i] * exp(mx[i] - zz) + 1.0;
-                                mx[i] = zz;
-                            } else {
-                                sm[i] += exp(zz - mx[i]);
-                            }
-                        }
+                    for (int i = 0; i < RPT; ++i) {
+                        z[i][u] = lv ? scale * z[i][u] : NEG_INF;
+                        mx[i] = fmax(mx[i], z[i][u]);
                     }
+                }
+#pragma unroll
+                for (int i = 0; i < RPT; ++i) {
+                    zb[2 * i] = make_double2(z[i][0], z[i][1]);
+                    zb[2 * i + 1] = make_double2(z[i][2], z[i][3]);
                 }
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < RPT; ++i)
 #pragma unroll
-                for (int o = 8; o > 0; o >>= 1) {
-                    double m2 = __shfl_xor_sync(0xffffffffu, mx[i], o, 16);
-                    double s2 = __shfl_xor_sync(0xffffffffu, sm[i], o, 16);
-                    double M = fmax(mx[i], m2);
-                    if (M != NEG_INF) {
-                        sm[i] = sm[i] * exp(mx[i] - M) + s2 * exp(m2 - M);
-                        mx[i] = M;
-                    }
+                for (int o = 8; o > 0; o >>= 1) mx[i] = fmax(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], o, 16));
+            // pass 2: e = exp(z - max) over this thread's own scratch blocks, row sums
+            double sm[RPT];
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) sm[i] = 0.0;
+            for (int c = 0; c < nch; ++c) {
+                double2* zb = reinterpret_cast<double2*>(zs + ((size_t)c * 256 + t) * ZB);
+#pragma unroll
+                for (int i = 0; i < RPT; ++i) {
+                    double2 v0 = zb[2 * i], v1 = zb[2 * i + 1];
+                    v0.x = exp(v0.x - mx[i]);
+                    v0.y = exp(v0.y - mx[i]);
+                    v1.x = exp(v1.x - mx[i]);
+                    v1.y = exp(v1.y - mx[i]);
+                    sm[i] += (v0.x + v0.y) + (v1.x + v1.y);
+                    zb[2 * i] = v0;
+                    zb[2 * i + 1] = v1;
                 }
             }
-            double inv[4];
+            double inv[RPT];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) inv[i] = (t0 + ty * 4 + i < nr) ? 1.0 / sm[i] : 0.0;
-            for (int c = 0; c < nch; ++c) {  // pass 2
-                __syncthreads();
-                load_chunk(c);
-                __syncthreads();
-                double z[4][4];
-                logits(z);
+            for (int i = 0; i < RPT; ++i) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int col = c * F64_TILE + tx + 16 * u;
-                    double cs = 0.0;
-                    if (col < NK && live[col]) {
+                for (int o = 8; o > 0; o >>= 1) sm[i] += __shfl_xor_sync(0xffffffffu, sm[i], o, 16);
+                inv[i] = (t0 + ty * RPT + i < nr) ? 1.0 / sm[i] : 0.0;
+            }
+            // pass 3: normalised probabilities summed over the tile's rows
+            for (int c = 0; c < nch; ++c) {
+                const double2* zb = reinterpret_cast<const double2*>(zs + ((size_t)c * 256 + t) * ZB);
+                double cs[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) cs += exp(scale * z[i][u] - mx[i]) * inv[i];
-                    }
-                    part[ty * F64_TILE + tx + 16 * u] = cs;
+                for (int i = 0; i < RPT; ++i) {
+                    const double2 v0 = zb[2 * i], v1 = zb[2 * i + 1];
+                    cs[0] += v0.x * inv[i];
+                    cs[1] += v0.y * inv[i];
+                    cs[2] += v1.x * inv[i];
+                    cs[3] += v1.y * inv[i];
                 }
+                __syncthreads();  // part free
+#pragma unroll
+                for (int u = 0; u < 4; ++u) part[ty * F64_CH + 4 * tx + u] = cs[u];
                 __syncthreads();
-                if (t < F64_TILE) {
+                if (t < F64_CH) {
                     double s = 0.0;
-                    for (int q = 0; q < 16; ++q) s += part[q * F64_TILE + t];
-                    const int col = c * F64_TILE + t;
+                    for (int q = 0; q < 16; ++q) s += part[q * F64_CH + t];
+                    const int col = c * F64_CH + t;
                     if (col < NK) Isum[col] += s;
                 }
             }
@@ -576,28 +615,56 @@ __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, co
     }
 }
 
+size_t pama_f64_scratch_bytes(int NK) {
+    return (size_t)kPamaF64Slots * ((NK + F64_CH - 1) / F64_CH) * 256 * 32 * sizeof(double);
+}
+
+template <typename T, int RPT>
+static void pama_f64_launch(const void* Q, const int32_t* q_perm, const int32_t* q_off, const void* CK,
+                            const int32_t* k_off, int N, int D, int NQ, int NK, int NKP, double scale, float p,
+                            const int32_t* list, const int32_t* count, int all_clusters, int BHNQ, int32_t* work_ctr,
+                            double* zscratch, float* importance, float* importance_bound, uint8_t* mask,
+                            int32_t* kept_cnt, int64_t* counters, size_t sm, int blocks, cudaStream_t st) {
+    cudaFuncSetAttribute(k_pama_f64<T, RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_pama_f64<T, RPT><<<blocks, 256, sm, st>>>((const T*)Q, q_perm, q_off, (const T*)CK, k_off, N, D, NQ, NK, NKP,
+                                                scale, p, list, count, all_clusters, BHNQ, work_ctr, zscratch,
+                                                importance, importance_bound, mask, kept_cnt, counters);
+}
+
 int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int NK, const int32_t* q_perm,
                     const int32_t* q_off, const void* CK, const int32_t* k_off, float p, const int32_t* list,
-                    const int32_t* count, int all_clusters, int num_sms, float* importance, float* importance_bound,
-                    uint8_t* mask, int32_t* kept_cnt, int64_t* counters, cudaStream_t st) {
+                    const int32_t* count, int all_clusters, int num_sms, int32_t* work_ctr, double* zscratch,
+                    float* importance, float* importance_bound, uint8_t* mask, int32_t* kept_cnt, int64_t* counters,
+                    cudaStream_t st) {
     if (NK > 4096 || D > 128) return PARK_ERR_UNSUPPORTED;
-    int NKP = next_pow2(NK);
-    size_t sm = (size_t)2 * F64_TILE * F64_LD * 8 + (size_t)NKP * 8 + 16 * 64 * 8 + (size_t)NKP * 4 + NKP;
-    int blocks = num_sms;
-    double scale = 1.0 / sqrt((double)D);
-    if (dtype == PARK_BF16)
-        cudaFuncSetAttribute(k_pama_f64<bf16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    else
-        cudaFuncSetAttribute(k_pama_f64<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    const int NKP = next_pow2(NK);
+    auto smem = [&](int RT) {
+        return (size_t)128 * RT * 8 + (size_t)128 * F64_CH * 8 + (size_t)NKP * 8 + 16 * F64_CH * 8 + (size_t)NKP * 4 +
+               NKP;
+    };
+    const bool big = smem(128) <= 227 * 1024;  // 128-row tiles when the sort buffers leave room
+    const size_t sm = smem(big ? 128 : 64);
+    const int blocks = num_sms < kPamaF64Slots ? num_sms : kPamaF64Slots;
+    const double scale = 1.0 / sqrt((double)D);
     ::park::prof_begin(st);
     if (dtype == PARK_BF16) {
-        k_pama_f64<bf16_t><<<blocks, 256, sm, st>>>((const bf16_t*)Q, q_perm, q_off, (const bf16_t*)CK, k_off, N, D,
-                                                    NQ, NK, NKP, scale, p, list, count, all_clusters, BH * NQ,
-                                                    importance, importance_bound, mask, kept_cnt, counters);
+        if (big)
+            pama_f64_launch<bf16_t, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, list, count,
+                                       all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
+                                       kept_cnt, counters, sm, blocks, st);
+        else
+            pama_f64_launch<bf16_t, 4>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, list, count,
+                                       all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
+                                       kept_cnt, counters, sm, blocks, st);
     } else {
-        k_pama_f64<float><<<blocks, 256, sm, st>>>((const float*)Q, q_perm, q_off, (const float*)CK, k_off, N, D, NQ,
-                                                   NK, NKP, scale, p, list, count, all_clusters, BH * NQ, importance,
-                                                   importance_bound, mask, kept_cnt, counters);
+        if (big)
+            pama_f64_launch<float, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, list, count,
+                                      all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
+                                      kept_cnt, counters, sm, blocks, st);
+        else
+            pama_f64_launch<float, 4>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, list, count,
+                                      all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
+                                      kept_cnt, counters, sm, blocks, st);
     }
     PARK_TRY_LAUNCH("k_pama_f64", st);
     return PARK_OK;

@@ -61,10 +61,16 @@ int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t*
 int launch_topp(const float* importance, const float* rho, int BH, int NQ, int NK, const int32_t* q_off,
                 const int32_t* k_off, float p, uint8_t* mask, int32_t* kept_cnt, float* importance_bound,
                 int32_t* flag_list, int32_t* flag_count, cudaStream_t st);
+// Float64 PAMA + top-p for the listed clusters (or all): at most kPamaF64Slots
+// CTAs, each with pama_f64_scratch_bytes(NK) / kPamaF64Slots bytes of float64
+// scratch; work_ctr (zeroed by the caller) hands out the clusters.
+constexpr int kPamaF64Slots = 160;
+size_t pama_f64_scratch_bytes(int NK);
 int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int NK, const int32_t* q_perm,
                     const int32_t* q_off, const void* CK, const int32_t* k_off, float p, const int32_t* list,
-                    const int32_t* count, int all_clusters, int num_sms, float* importance, float* importance_bound,
-                    uint8_t* mask, int32_t* kept_cnt, int64_t* counters, cudaStream_t st);
+                    const int32_t* count, int all_clusters, int num_sms, int32_t* work_ctr, double* zscratch,
+                    float* importance, float* importance_bound, uint8_t* mask, int32_t* kept_cnt, int64_t* counters,
+                    cudaStream_t st);
 int launch_kept_csr(const uint8_t* mask, const int32_t* kept_cnt, int BH, int NQ, int NK, int32_t* kept_ptr,
                     int32_t* kept_idx, int64_t* counters, cudaStream_t st);
 

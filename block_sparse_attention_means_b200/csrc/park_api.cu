@@ -118,7 +118,7 @@ int metric_chunks(const Dims& d) {
 
 struct RetrievalWs {
     size_t M, Mpart, xnorm_q, xnorm_k, wop, b32, b64, w64, wmax, bmax, lpair, lcand, lfull, lcnt, hist, rho, plist,
-        pcnt, kcnt, total;
+        pcnt, kcnt, f64z, total;
 };
 
 RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
@@ -145,6 +145,7 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
     w.plist = c.take(BH * NQ * 4);
     w.pcnt = c.take(16 * 4);
     w.kcnt = c.take(BH * NQ * 4);
+    w.f64z = c.take(pama_f64_scratch_bytes(NK));
     w.total = c.off;
     return w;
 }
@@ -324,11 +325,13 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
                                at<int32_t>(ws, w.pcnt), st));
         PARK_CHECK(launch_pama_f64(Q, d.dtype, BH, N, D, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids,
                                    out->k_offsets, p, at<int32_t>(ws, w.plist), at<int32_t>(ws, w.pcnt), 0, num_sms,
-                                   out->importance, out->importance_bound, out->mask, kcnt, out->counters, st));
+                                   at<int32_t>(ws, w.pcnt) + 4, at<double>(ws, w.f64z), out->importance,
+                                   out->importance_bound, out->mask, kcnt, out->counters, st));
     } else {
         PARK_CHECK(launch_pama_f64(Q, d.dtype, BH, N, D, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids,
-                                   out->k_offsets, p, nullptr, nullptr, 1, num_sms, out->importance,
-                                   out->importance_bound, out->mask, kcnt, out->counters, st));
+                                   out->k_offsets, p, nullptr, nullptr, 1, num_sms, at<int32_t>(ws, w.pcnt) + 4,
+                                   at<double>(ws, w.f64z), out->importance, out->importance_bound, out->mask, kcnt,
+                                   out->counters, st));
     }
     PARK_CHECK(launch_kept_csr(out->mask, kcnt, BH, NQ, NK, out->kept_ptr, out->kept_idx, out->counters, st));
     return PARK_OK;
