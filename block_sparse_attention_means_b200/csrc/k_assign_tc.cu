@@ -9,10 +9,13 @@
 // tile used twice as the A operand ([x, x] . [hi; lo] = x . (hi + lo)).
 // Accumulators live in TMEM (two buffers x two row halves of 128 x 128 fp32).
 // Eight epilogue warps (warps 2-5: rows 0-127, warps 6-9: rows 128-255; one
-// thread per row) keep the three smallest scores of their row and apply the
-// certified decision of k_assign.cu: winner certified when
-// the runner-up is more than 2 beta above it, else the row is listed for a
-// float64 rescore of two candidates or of every centroid.
+// thread per row) track, branch-free, the smallest score of their row, its
+// column and the second smallest score, in four independent copies (one per
+// 32-column group of every chunk) merged once per tile, and apply the
+// certified decision of k_assign.cu: the winner is certified when the
+// runner-up is more than 2 beta above it, else the row is listed for a float64
+// rescore against every centroid.  The head's float bias is staged in shared
+// memory.
 //
 // One CTA per SM, persistent over row tiles; warp 0 loads, warp 1 owns TMEM
 // and issues the MMAs (one thread), warps 2-9 are the epilogue.  Every wait is
@@ -35,26 +38,6 @@ struct AsSmem {
     int abort;
 };
 
-__device__ __forceinline__ void top3(float (&v)[3], int (&id)[3], float s, int k) {
-    if (s < v[2]) {
-        if (s < v[1]) {
-            v[2] = v[1];
-            id[2] = id[1];
-            if (s < v[0]) {
-                v[1] = v[0];
-                id[1] = id[0];
-                v[0] = s;
-                id[0] = k;
-            } else {
-                v[1] = s;
-                id[1] = k;
-            }
-        } else {
-            v[2] = s;
-            id[2] = k;
-        }
-    }
-}
 }  // namespace
 
 template <int KW>
@@ -69,6 +52,7 @@ __global__ void __launch_bounds__(320, 1)
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* Xs = base;               // row halves x 2 column blocks
     uint8_t* Ws = base + 4 * AS_BLK;  // 2 stages x WB blocks
+    float* sbias = reinterpret_cast<float*>(Ws + 2 * WB * AS_BLK);  // [nch * 128] bias of the current head
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort = &sh.abort;
     if (threadIdx.x == 0) {
@@ -182,12 +166,18 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t trow = tmem + ((uint32_t)lane_base << 16) + (uint32_t)(half * 128);
         const float INF = __int_as_float(0x7f800000);
         bool failed = false;
-        int G = 0;
+        int G = 0, cur_bh = -1;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
             const int bh = t / tpr, r0 = (t - bh * tpr) * AS_ROWS;
-            const float* bb = bias + (size_t)bh * bias_ld;
-            float v[3] = {INF, INF, INF};
-            int id[3] = {0, 0, 0};
+            if (bh != cur_bh) {  // stage the head's bias (all epilogue warps take this branch together)
+                named_bar_sync(1, 256);
+                for (int k = threadIdx.x - 64; k < nch * AS_CH; k += 256) sbias[k] = bias[(size_t)bh * bias_ld + k];
+                named_bar_sync(1, 256);
+                cur_bh = bh;
+            }
+            // tracker g covers columns 32 g .. 32 g + 31 of every chunk, in increasing order
+            float v0[4] = {INF, INF, INF, INF}, v1[4] = {INF, INF, INF, INF};
+            int i0[4] = {0, 0, 0, 0};
             for (int c = 0; c < nch; ++c) {
                 const int s = G & 1, round = G >> 1;
                 if (!failed) {
@@ -195,56 +185,53 @@ __global__ void __launch_bounds__(320, 1)
                     failed = !__all_sync(0xffffffffu, ok);
                 }
                 tc_fence_after();
-                uint32_t acc[4][32];
 #pragma unroll
-                for (int g = 0; g < 4; ++g) tmem_ld32(trow + (uint32_t)(2 * s * 128 + 32 * g), acc[g]);
-                tmem_ld_wait();
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    // Scores of 32 columns, then their minimum by a tree; the ordered
-                    // top-3 insertion runs only when that minimum beats the current
-                    // third score (columns past K carry bias +inf and never do).
-                    const int cb = c * AS_CH + 32 * g;
-                    const float4* bp = reinterpret_cast<const float4*>(bb + cb);
-                    float sc[32];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 b4 = __ldg(bp + q);
-                        sc[4 * q + 0] = fmaf(-2.f, __uint_as_float(acc[g][4 * q + 0]), b4.x);
-                        sc[4 * q + 1] = fmaf(-2.f, __uint_as_float(acc[g][4 * q + 1]), b4.y);
-                        sc[4 * q + 2] = fmaf(-2.f, __uint_as_float(acc[g][4 * q + 2]), b4.z);
-                        sc[4 * q + 3] = fmaf(-2.f, __uint_as_float(acc[g][4 * q + 3]), b4.w);
+                for (int gp = 0; gp < 2; ++gp) {  // two 32-column groups at a time
+                    uint32_t acc[2][32];
+                    tmem_ld32(trow + (uint32_t)(2 * s * 128 + 64 * gp), acc[0]);
+                    tmem_ld32(trow + (uint32_t)(2 * s * 128 + 64 * gp + 32), acc[1]);
+                    tmem_ld_wait();
+                    tmem_ld_dep(acc[0]);
+                    tmem_ld_dep(acc[1]);
+                    if (gp == 1) {  // the whole chunk is in registers: release the accumulator
+                        tc_fence_before();
+                        mbar_arrive(&sh.acc_empty[s]);
                     }
-                    float m[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) m[j] = fminf(sc[2 * j], sc[2 * j + 1]);
+                    for (int q = 0; q < 8; ++q)
 #pragma unroll
-                    for (int w = 8; w > 0; w >>= 1)
+                        for (int h = 0; h < 2; ++h) {  // two trackers interleave for ILP
+                            const int g = 2 * gp + h;
+                            const int cb = c * AS_CH + 32 * g + 4 * q;
+                            const float4 b4 = *reinterpret_cast<const float4*>(sbias + cb);
+                            const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-                        for (int j = 0; j < w; ++j) m[j] = fminf(m[j], m[j + w]);
-                    if (m[0] < v[2]) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) top3(v, id, sc[j], cb + j);
-                    }
+                            for (int e = 0; e < 4; ++e) {
+                                const float sc = fmaf(-2.f, __uint_as_float(acc[h][4 * q + e]), bv[e]);
+                                v1[g] = fminf(v1[g], fmaxf(v0[g], sc));
+                                i0[g] = sc < v0[g] ? cb + e : i0[g];  // strict: the first of equal scores stays
+                                v0[g] = fminf(v0[g], sc);
+                            }
+                        }
                 }
-                tc_fence_before();
-                mbar_arrive(&sh.acc_empty[s]);
                 ++G;
             }
+            // merge: smallest (v0, column), then the second smallest of everything else
+            int w = 0;
+#pragma unroll
+            for (int g = 1; g < 4; ++g)
+                if (v0[g] < v0[w] || (v0[g] == v0[w] && i0[g] < i0[w])) w = g;
+            float best = v0[w], second = v1[w];
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                if (g != w) second = fminf(second, v0[g]);
             if (r0 + row < N && !failed) {
                 const size_t gr = (size_t)bh * N + r0 + row;
                 const float beta = gamma * xnorm[gr] * wmax[bh] + 4.8e-7f * bmax[bh] + 1e-30f;
-                const float tb = 2.f * beta;
-                labels[gr] = id[0];
-                if (!(v[1] - v[0] > tb)) {
-                    if (v[2] - v[0] > tb) {
-                        const int pos = atomicAdd(lists.counts + 0, 1);
-                        lists.pair_row[pos] = (int32_t)gr;
-                        lists.pair_cand[pos] = id[1];
-                    } else {
-                        const int pos = atomicAdd(lists.counts + 1, 1);
-                        lists.full_row[pos] = (int32_t)gr;
-                    }
+                labels[gr] = i0[w];
+                if (!(second - best > 2.f * beta)) {
+                    const int pos = atomicAdd(lists.counts + 1, 1);
+                    lists.full_row[pos] = (int32_t)gr;
                 }
             }
         }
@@ -265,7 +252,7 @@ int launch_assign_tc(const void* X, int BH, int N, int K, const CentroidOps& ops
     CUtensorMap mX, mW;
     PARK_CHECK(make_tma_map_bf16(&mX, X, (uint64_t)BH * N, 128, 128));
     PARK_CHECK(make_tma_map_bf16(&mW, ops.w, (uint64_t)BH * K, (uint32_t)ops.kw, AS_CH));
-    const size_t sm = (size_t)(4 + 2 * (ops.kw / 64)) * AS_BLK + 1024;
+    const size_t sm = (size_t)(4 + 2 * (ops.kw / 64)) * AS_BLK + 1024 + (size_t)((K + AS_CH - 1) / AS_CH) * AS_CH * 4;
     if (ops.kw == 128)
         cudaFuncSetAttribute(k_assign_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     else

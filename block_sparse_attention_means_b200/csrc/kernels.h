@@ -25,10 +25,8 @@ struct CentroidOps {
 };
 
 struct Lists {
-    int32_t* pair_row;   // [BH*N] bh*N + i of rows whose winner is one of two candidates
-    int32_t* pair_cand;  // [BH*N] the second candidate
-    int32_t* full_row;   // [BH*N] rows rescored against every centroid
-    int32_t* counts;     // [4]: pair count, full count, (spare)
+    int32_t* full_row;  // [BH*N] bh*N + i of rows rescored against every centroid
+    int32_t* counts;    // [4]: (spare), full count, (spare)
 };
 
 // ---- k_prep.cu

@@ -117,7 +117,7 @@ int metric_chunks(const Dims& d) {
 }
 
 struct RetrievalWs {
-    size_t M, Mpart, xnorm_q, xnorm_k, wop, b32, b64, w64, wmax, bmax, lpair, lcand, lfull, lcnt, hist, rho, plist,
+    size_t M, Mpart, xnorm_q, xnorm_k, wop, b32, b64, w64, wmax, bmax, lfull, lcnt, hist, rho, plist,
         pcnt, kcnt, f64z, total;
 };
 
@@ -136,8 +136,6 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
     w.w64 = c.take(BH * Km * D * 8);
     w.wmax = c.take(BH * 4);
     w.bmax = c.take(BH * 4);
-    w.lpair = c.take(BH * N * 4);
-    w.lcand = c.take(BH * N * 4);
     w.lfull = c.take(BH * N * 4);
     w.lcnt = c.take(16 * 4);
     w.hist = c.take(BH * Km * nchunks * 4);
@@ -250,8 +248,6 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
         ops.kw = D;
     }
     Lists lists;
-    lists.pair_row = at<int32_t>(ws, w.lpair);
-    lists.pair_cand = at<int32_t>(ws, w.lcand);
     lists.full_row = at<int32_t>(ws, w.lfull);
     lists.counts = at<int32_t>(ws, w.lcnt);
     if (bf16) PARK_CHECK(launch_row_norms(s.X, d.dtype, BH, N, D, s.xnorm, st));
