@@ -50,80 +50,98 @@ int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status
 }
 
 // ---------------------------------------------------------------- metric
-// M = (1/N) sum_i q_i q_i^T in float64.  Pass 1: grid (chunks, BH); each CTA
-// sums the outer products of its row chunk.  Thread t owns entries
-// (a = t/16 + 16u, b = t%16 + 16v).  Entries (a,b) and (b,a) see the same
-// products in the same order, so M is exactly symmetric.  Pass 2 adds the
-// chunk partials in chunk order and divides by N.
+// M = (1/N) sum_i q_i q_i^T in float64, exploiting symmetry.  Pass 1: one CTA
+// per (row chunk, head) sums the outer products of its rows into the upper
+// triangle of 8 x 8 blocks (136 blocks for D = 128); thread i owns rows
+// 8 ta + 4 (i & 1) + 0..3 and columns 8 tb + 0..7 of block i >> 1 (ta <= tb),
+// reading the rows from shared memory with 16-byte loads.  Pass 2 adds the
+// chunk partials in chunk order, divides by N and writes M[a][b] = M[b][a], so
+// M is exactly symmetric.
+constexpr int kMetricRB = 32;  // rows staged per step
+
 template <typename T>
-__global__ __launch_bounds__(256) void k_metric_partial(const T* __restrict__ Q, int N, int D, int rows_per_chunk,
+__global__ __launch_bounds__(272) void k_metric_partial(const T* __restrict__ Q, int N, int D, int rows_per_chunk,
                                                         double* __restrict__ part) {
-    constexpr int RB = 32;
-    extern __shared__ double qs[];  // [RB][D]
-    int bh = blockIdx.y, c = blockIdx.x, nch = gridDim.x;
+    __shared__ __align__(16) double qs[kMetricRB][128];
+    const int bh = blockIdx.y, c = blockIdx.x, nch = gridDim.x;
     const T* X = Q + (size_t)bh * N * D;
-    int r0 = c * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
-    int t = threadIdx.x, ta = t >> 4, tb = t & 15;
-    double acc[8][8];
+    const int r0 = c * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
+    const int t = threadIdx.x, bi = t >> 1, hf = t & 1;
+    int tb = (int)((sqrt(8.0 * bi + 1.0) - 1.0) * 0.5);
+    while ((tb + 1) * (tb + 2) / 2 <= bi) ++tb;
+    while (tb * (tb + 1) / 2 > bi) --tb;
+    const int ta = bi - tb * (tb + 1) / 2;
+    const int a0 = 8 * ta + 4 * hf, b0 = 8 * tb;
+    const bool active = b0 < D;  // D is a multiple of 32
+    double acc[4][8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < 4; ++u)
 #pragma unroll
         for (int v = 0; v < 8; ++v) acc[u][v] = 0.0;
-    for (int base = r0; base < r1; base += RB) {
-        int nr = min(RB, r1 - base);
-        for (int e = t; e < RB * D; e += 256) {
-            int rr = e / D, jj = e - rr * D;
-            qs[e] = rr < nr ? Elem<T>::to_double(X + (size_t)(base + rr) * D, jj) : 0.0;
+    for (int base = r0; base < r1; base += kMetricRB) {
+        const int nr = min(kMetricRB, r1 - base);
+        __syncthreads();
+        for (int e = t; e < kMetricRB * 128; e += blockDim.x) {
+            const int rr = e >> 7, jj = e & 127;
+            qs[rr][jj] = (rr < nr && jj < D) ? Elem<T>::to_double(X + (size_t)(base + rr) * D, jj) : 0.0;
         }
         __syncthreads();
-        for (int rr = 0; rr < nr; ++rr) {
-            const double* q = qs + rr * D;
-            double qa[8], qb[8];
+        if (active) {
+            for (int rr = 0; rr < nr; ++rr) {
+                double qa[4], qb[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                int a = ta + 16 * u, b = tb + 16 * u;
-                qa[u] = a < D ? q[a] : 0.0;
-                qb[u] = b < D ? q[b] : 0.0;
+                for (int u = 0; u < 4; u += 2) {
+                    const double2 x = *reinterpret_cast<const double2*>(&qs[rr][a0 + u]);
+                    qa[u] = x.x;
+                    qa[u + 1] = x.y;
+                }
+#pragma unroll
+                for (int v = 0; v < 8; v += 2) {
+                    const double2 x = *reinterpret_cast<const double2*>(&qs[rr][b0 + v]);
+                    qb[v] = x.x;
+                    qb[v + 1] = x.y;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) acc[u][v] = __fma_rn(qa[u], qb[v], acc[u][v]);
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-#pragma unroll
-                for (int v = 0; v < 8; ++v) acc[u][v] = __fma_rn(qa[u], qb[v], acc[u][v]);
         }
-        __syncthreads();
     }
+    if (!active) return;
     double* P = part + ((size_t)bh * nch + c) * D * D;
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            int a = ta + 16 * u, b = tb + 16 * v;
-            if (a < D && b < D) P[a * D + b] = acc[u][v];
-        }
+        for (int v = 0; v < 8; ++v) P[(a0 + u) * D + b0 + v] = acc[u][v];
 }
 
 __global__ void k_metric_reduce(const double* __restrict__ part, int nch, int N, int D, double* __restrict__ M,
                                 double* __restrict__ M_out) {
-    int bh = blockIdx.y;
-    int e = blockIdx.x * blockDim.x + threadIdx.x;
+    const int bh = blockIdx.y;
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= D * D) return;
+    const int a = e / D, b = e - a * D;
+    // entry (a, b) of the upper triangle of 8 x 8 blocks that holds {a, b}
+    const int ua = (a >> 3) <= (b >> 3) ? a : b, ub = (a >> 3) <= (b >> 3) ? b : a;
+    const int src = ua * D + ub;
     double s = 0.0;
-    for (int c = 0; c < nch; ++c) s += part[((size_t)bh * nch + c) * D * D + e];
-    double m = s / (double)N;
+    for (int c = 0; c < nch; ++c) s += part[((size_t)bh * nch + c) * D * D + src];
+    const double m = s / (double)N;
     M[(size_t)bh * D * D + e] = m;
     if (M_out) M_out[(size_t)bh * D * D + e] = m;
 }
 
 int launch_metric(const void* Q, int dtype, int BH, int N, int D, double* part, int nchunks, double* M,
                   double* M_out, cudaStream_t st) {
+    if (D > 128 || D % 32 != 0) return PARK_ERR_UNSUPPORTED;
     int rpc = (N + nchunks - 1) / nchunks;
     dim3 g1(nchunks, BH);
-    size_t sm = 32 * D * sizeof(double);
     ::park::prof_begin(st);
     if (dtype == PARK_BF16)
-        k_metric_partial<bf16_t><<<g1, 256, sm, st>>>((const bf16_t*)Q, N, D, rpc, part);
+        k_metric_partial<bf16_t><<<g1, 272, 0, st>>>((const bf16_t*)Q, N, D, rpc, part);
     else
-        k_metric_partial<float><<<g1, 256, sm, st>>>((const float*)Q, N, D, rpc, part);
+        k_metric_partial<float><<<g1, 272, 0, st>>>((const float*)Q, N, D, rpc, part);
     PARK_TRY_LAUNCH("k_metric_partial", st);
     dim3 g2((D * D + 255) / 256, BH);
     ::park::prof_begin(st);
@@ -235,11 +253,99 @@ __global__ void k_centroid_prep(const T* __restrict__ C, int K, int D, const dou
     }
 }
 
+// QRKC operands for 16 centroids per CTA: M (symmetric, float64) is staged once
+// in shared memory, thread (a, half) forms w_a = sum_b M[b][a] c_b for eight
+// centroids (row b of M: conflict-free), then per centroid bias = c . w and
+// ||w||^2 are reduced over the 128 threads of its half in a fixed order.
+constexpr int kPrepCents = 16;
+
+template <typename T>
+__global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restrict__ C, int K, int D,
+                                                              const double* __restrict__ Mall,
+                                                              uint16_t* __restrict__ wop, float* __restrict__ bias32,
+                                                              int bias_ld, double* __restrict__ bias64,
+                                                              double* __restrict__ w64, float* __restrict__ wmax,
+                                                              float* __restrict__ bmax) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    double* Ms = reinterpret_cast<double*>(smem_raw);  // [D][D]
+    double* Cs = Ms + D * D;                          // [kPrepCents][D]
+    __shared__ double red[kPrepCents][4][2];
+    const int bh = blockIdx.y, k0 = blockIdx.x * kPrepCents, t = threadIdx.x;
+    const int a = t & 127, half = t >> 7, lane = t & 31, wq = (t >> 5) & 3;
+    const double* M = Mall + (size_t)bh * D * D;
+    for (int i = t; i < D * D; i += blockDim.x) Ms[i] = M[i];
+    for (int i = t; i < kPrepCents * D; i += blockDim.x) {
+        const int c = i / D, j = i - c * D, k = k0 + c;
+        Cs[i] = k < K ? Elem<T>::to_double(C + ((size_t)bh * K + k) * D, j) : 0.0;
+    }
+    if (blockIdx.x == 0)  // columns past K read +inf, so a score GEMM over whole 128-column chunks never picks them
+        for (int j = K + t; j < ((K + 127) & ~127); j += blockDim.x)
+            bias32[(size_t)bh * bias_ld + j] = __int_as_float(0x7f800000);
+    __syncthreads();
+    double w[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) w[c] = 0.0;
+    if (a < D) {
+        for (int b = 0; b < D; ++b) {
+            const double m = Ms[b * D + a];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) w[c] = __fma_rn(m, Cs[(half * 8 + c) * D + b], w[c]);
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const int cc = half * 8 + c, k = k0 + cc;
+        const double ca = a < D ? Cs[cc * D + a] : 0.0;
+        if (a < D && k < K) {
+            w64[((size_t)bh * K + k) * D + a] = w[c];
+            if (wop != nullptr) {
+                const uint16_t hi = double_to_bf16_bits(w[c]);
+                const double hid = (double)__uint_as_float(((uint32_t)hi) << 16);
+                const uint16_t lo = double_to_bf16_bits(w[c] - hid);  // w - hi is exact
+                wop[((size_t)bh * K + k) * (2 * D) + a] = hi;
+                wop[((size_t)bh * K + k) * (2 * D) + D + a] = lo;
+            }
+        }
+        const double pb = warp_sum(ca * w[c]), pn = warp_sum(w[c] * w[c]);
+        if (lane == 0) {
+            red[cc][wq][0] = pb;
+            red[cc][wq][1] = pn;
+        }
+    }
+    __syncthreads();
+    if (t < kPrepCents && k0 + t < K) {
+        const int k = k0 + t;
+        const double b = ((red[t][0][0] + red[t][1][0]) + red[t][2][0]) + red[t][3][0];
+        const double n2 = ((red[t][0][1] + red[t][1][1]) + red[t][2][1]) + red[t][3][1];
+        bias64[(size_t)bh * K + k] = b;
+        bias32[(size_t)bh * bias_ld + k] = __double2float_rn(b);
+        atomic_max_nonneg(wmax + bh, round_up_f(__double2float_ru(sqrt(n2))));
+        atomic_max_nonneg(bmax + bh, round_up_f(__double2float_ru(fabs(b))));
+    }
+}
+
 int launch_centroid_prep(const void* C, int dtype, int BH, int K, int D, const double* M, CentroidOps ops,
                          cudaStream_t st) {
     if (D > 128) return PARK_ERR_UNSUPPORTED;  // one thread per coordinate
     dim3 g(K, BH);
     bool metric = M != nullptr;
+    if (metric) {  // tiled form: M staged once per 16 centroids
+        const dim3 gm((K + kPrepCents - 1) / kPrepCents, BH);
+        const size_t sm = (size_t)D * D * 8 + (size_t)kPrepCents * D * 8;
+        ::park::prof_begin(st);
+        if (dtype == PARK_BF16) {
+            cudaFuncSetAttribute(k_centroid_prep_metric<bf16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            k_centroid_prep_metric<bf16_t><<<gm, 256, sm, st>>>((const bf16_t*)C, K, D, M, (uint16_t*)ops.w,
+                                                               ops.bias32, ops.bias_ld, ops.bias64, ops.w64,
+                                                               ops.wmax, ops.bmax);
+        } else {
+            cudaFuncSetAttribute(k_centroid_prep_metric<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            k_centroid_prep_metric<float><<<gm, 256, sm, st>>>((const float*)C, K, D, M, (uint16_t*)ops.w, ops.bias32,
+                                                              ops.bias_ld, ops.bias64, ops.w64, ops.wmax, ops.bmax);
+        }
+        PARK_TRY_LAUNCH("k_centroid_prep_metric", st);
+        return PARK_OK;
+    }
     ::park::prof_begin(st);
     if (dtype == PARK_BF16) {
         if (metric)

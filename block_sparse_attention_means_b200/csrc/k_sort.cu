@@ -2,11 +2,11 @@
 // exact K-means centroid update.
 //
 // Sort: tokens are split into chunks of 1024.  (1) per-chunk label histogram
-// in shared memory; (2) one CTA per head turns the [label][chunk] table into
-// exclusive start positions (label-major, so clusters are contiguous and
-// chunks keep token order); (3) each chunk ranks its tokens among equal labels
-// in token order (warp match + warps in sequence) and scatters them.  The
-// result equals a stable argsort of the labels.
+// in shared memory; (2) the [label][chunk] table becomes start positions
+// (label-major, so clusters are contiguous and chunks keep token order); (3)
+// each chunk ranks its tokens among equal labels in token order (warp match +
+// warps in sequence) and scatters them.  The result equals a stable argsort of
+// the labels.
 //
 // Update: one CTA per (cluster, head) sums its members' rows exactly in fixed
 // point (x * 2^27 for bf16, x * 2^43 for float32 inputs; integer sums are exact
@@ -34,51 +34,73 @@ __global__ void k_label_hist(const int32_t* __restrict__ labels, int N, int K, i
     for (int k = threadIdx.x; k < K; k += blockDim.x) h[(size_t)k * nchunks + c] = cnt[k];
 }
 
-// Exclusive scan of hist[bh] (K * nchunks entries) in place; offsets[k] = start
-// of cluster k, offsets[K] = N.  1024 threads, each owns a contiguous segment.
-__global__ __launch_bounds__(1024) void k_label_scan(int32_t* __restrict__ hist, int N, int K, int nchunks,
-                                                     int32_t* __restrict__ offsets) {
-    __shared__ int32_t wsum[32];
-    int bh = blockIdx.x, t = threadIdx.x;
-    int total = K * nchunks;
-    int seg = (total + 1023) / 1024;
-    int32_t* h = hist + (size_t)bh * total;
-    int b0 = t * seg, b1 = min(total, b0 + seg);
-    int s = 0;
-    for (int e = b0; e < b1; ++e) s += h[e];
-    // block exclusive scan of s
-    int lane = t & 31, w = t >> 5;
-    int incl = s;
+// Positions, in two steps that keep every SM busy.  (2a) one warp per (label,
+// head) turns its row hist[k][*] into exclusive positions within the label and
+// writes the label's size to offsets[k]; (2b) one CTA per head turns the sizes
+// into exclusive starts, offsets[K] = N.  A token's position is offsets[label]
+// + hist[label][chunk] + its rank in the chunk.
+__global__ __launch_bounds__(256) void k_label_rowscan(int32_t* __restrict__ hist, int K, int nchunks,
+                                                       int32_t* __restrict__ offsets) {
+    const int lane = threadIdx.x & 31;
+    const int k = blockIdx.x * 8 + (threadIdx.x >> 5), bh = blockIdx.y;
+    if (k >= K) return;
+    int32_t* h = hist + ((size_t)bh * K + k) * nchunks;
+    const int seg = (nchunks + 31) / 32, b0 = lane * seg, b1 = min(nchunks, b0 + seg);
+    int loc = 0;
+    for (int e = b0; e < b1; ++e) loc += h[e];
+    int incl = loc;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    int run = incl - loc;
+    for (int e = b0; e < b1; ++e) {
+        const int v = h[e];
+        h[e] = run;
+        run += v;
+    }
+    if (lane == 31) offsets[(size_t)bh * (K + 1) + k] = incl;
+}
+
+__global__ __launch_bounds__(1024) void k_label_scan(int N, int K, int32_t* __restrict__ offsets) {
+    __shared__ int32_t wsum[32];
+    const int bh = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+    int32_t* off = offsets + (size_t)bh * (K + 1);
+    const int seg = (K + 1023) / 1024, b0 = t * seg, b1 = min(K, b0 + seg);
+    int loc = 0;
+    for (int e = b0; e < b1; ++e) loc += off[e];
+    int incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
     }
     if (lane == 31) wsum[w] = incl;
     __syncthreads();
     if (w == 0) {
-        int x = wsum[lane];
+        const int x = wsum[lane];
         int xi = x;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            int y = __shfl_up_sync(0xffffffffu, xi, o);
+            const int y = __shfl_up_sync(0xffffffffu, xi, o);
             if (lane >= o) xi += y;
         }
-        wsum[lane] = xi - x;  // exclusive warp offsets
+        wsum[lane] = xi - x;
     }
     __syncthreads();
-    int run = wsum[w] + incl - s;
+    int run = wsum[w] + incl - loc;
     for (int e = b0; e < b1; ++e) {
-        int v = h[e];
-        h[e] = run;
-        if (e % nchunks == 0) offsets[(size_t)bh * (K + 1) + e / nchunks] = run;
+        const int v = off[e];
+        off[e] = run;
         run += v;
     }
-    if (t == 0) offsets[(size_t)bh * (K + 1) + K] = N;
+    if (t == 0) off[K] = N;
 }
 
 __global__ __launch_bounds__(1024) void k_label_scatter(const int32_t* __restrict__ labels, int N, int K,
                                                         int nchunks, const int32_t* __restrict__ hist,
+                                                        const int32_t* __restrict__ offsets,
                                                         int32_t* __restrict__ perm) {
     extern __shared__ int32_t run[];  // [K] tokens already placed per label in this chunk
     int c = blockIdx.x, bh = blockIdx.y;
@@ -98,7 +120,7 @@ __global__ __launch_bounds__(1024) void k_label_scatter(const int32_t* __restric
             int base = valid ? run[lab] : 0;
             __syncwarp();
             if (valid && leader) run[lab] = base + __popc(peers);
-            if (valid) pos = hist[((size_t)bh * K + lab) * nchunks + c] + base + rank;
+            if (valid) pos = offsets[(size_t)bh * (K + 1) + lab] + hist[((size_t)bh * K + lab) * nchunks + c] + base + rank;
         }
         __syncthreads();
     }
@@ -117,10 +139,13 @@ int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist
     k_label_hist<<<g, 256, sm, st>>>(labels, N, K, nchunks, hist);
     PARK_TRY_LAUNCH("k_label_hist", st);
     ::park::prof_begin(st);
-    k_label_scan<<<BH, 1024, 0, st>>>(hist, N, K, nchunks, offsets);
+    k_label_rowscan<<<dim3((K + 7) / 8, BH), 256, 0, st>>>(hist, K, nchunks, offsets);
+    PARK_TRY_LAUNCH("k_label_rowscan", st);
+    ::park::prof_begin(st);
+    k_label_scan<<<BH, 1024, 0, st>>>(N, K, offsets);
     PARK_TRY_LAUNCH("k_label_scan", st);
     ::park::prof_begin(st);
-    k_label_scatter<<<g, 1024, sm, st>>>(labels, N, K, nchunks, hist, perm);
+    k_label_scatter<<<g, 1024, sm, st>>>(labels, N, K, nchunks, hist, offsets, perm);
     PARK_TRY_LAUNCH("k_label_scatter", st);
     return PARK_OK;
 }
