@@ -229,7 +229,7 @@ def workload_config(cfg) -> dict:
 # ----------------------------------------------------------------------------- roofline of one kernel
 
 KERNEL_SOURCES = {"k_sparse_attn_tc": ["block_sparse_attention_means_b200/csrc/k_attn_tc.cu"],
-                  "k_assign_mma": ["block_sparse_attention_means_b200/csrc/k_assign.cu"],
+                  "k_assign_tc": ["block_sparse_attention_means_b200/csrc/k_assign_tc.cu"],
                   "k_pama_mma": ["block_sparse_attention_means_b200/csrc/k_pama.cu"],
                   "k_pama_f64": ["block_sparse_attention_means_b200/csrc/k_pama.cu"],
                   "k_metric_partial": ["block_sparse_attention_means_b200/csrc/k_prep.cu"]}
@@ -242,7 +242,7 @@ def kernel_roofline(name: str, ms_per_launch: float, cfg, counters, peaks, peak_
     sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     if name == "k_sparse_attn_tc":
         work, bound, peak, unit = 4.0 * D * counters[5], "tensor", sustained, "TFLOP/s"
-    elif name == "k_assign_mma":
+    elif name == "k_assign_tc":
         work, bound, peak, unit = 2.0 * BH * N * ((NQ + NK) / 2) * D, "tensor", sustained, "TFLOP/s"
     elif name == "k_pama_mma":
         work, bound, peak, unit = 2.0 * BH * N * NK * D, "tensor", sustained, "TFLOP/s"
