@@ -184,7 +184,7 @@ def stable_permutation(labels, K):
 # ----------------------------------------------------------------------------
 
 
-def pama(Q, q_labels, NQ, CK, k_counts, scale, row_block=8192):
+def pama(Q, q_labels, NQ, CK, k_counts, scale, row_block=8192, size_prior=False):
     """Block-importance map I[r, m].
 
     PARK (abstract; Figure 2 caption): every original query keeps its own
@@ -192,15 +192,19 @@ def pama(Q, q_labels, NQ, CK, k_counts, scale, row_block=8192):
     each query block:
         P_im = softmax_m(s q_i . c_m),   I_rm = mean_{i in Q_r} P_im.
     READING: only non-empty key clusters take part (an empty cluster stands for
-    no keys); rows of empty query clusters are 0."""
+    no keys); rows of empty query clusters are 0.
+    size_prior: a variant that is not on the pages, P_im proportional to
+    |B_m| exp(s q_i . c_m) (the Softmax with a log |B_m| prior); when every key of
+    cluster m equals c_m it is the exact attention mass of the cluster."""
     Q = np.asarray(Q, dtype=np.float64)
     CK = np.asarray(CK, dtype=np.float64)
     live = np.nonzero(np.asarray(k_counts) > 0)[0]
     NK = CK.shape[0]
     sums = np.zeros((NQ, live.size))
     q_labels = np.asarray(q_labels)
+    prior = np.log(np.asarray(k_counts, dtype=np.float64)[live]) if size_prior else 0.0
     for i0 in range(0, Q.shape[0], row_block):
-        Z = scale * (Q[i0:i0 + row_block] @ CK[live].T)
+        Z = scale * (Q[i0:i0 + row_block] @ CK[live].T) + prior
         Z -= Z.max(axis=1, keepdims=True)
         P = np.exp(Z)
         P /= P.sum(axis=1, keepdims=True)
@@ -212,16 +216,17 @@ def pama(Q, q_labels, NQ, CK, k_counts, scale, row_block=8192):
     return I
 
 
-def pama_centroid_query(CQ, q_counts, CK, k_counts, scale):
+def pama_centroid_query(CQ, q_counts, CK, k_counts, scale, size_prior=False):
     """"w/o PAMA" ablation (PARK Table 3; Figure 1(a)): the query centroid is
     scored instead of every query, i.e. queries are averaged before Softmax:
-    I_rm = softmax_m(s c_r^Q . c_m) for non-empty r, m."""
+    I_rm = softmax_m(s c_r^Q . c_m) for non-empty r, m (size_prior as in pama)."""
     live = np.nonzero(np.asarray(k_counts) > 0)[0]
     I = np.zeros((CQ.shape[0], CK.shape[0]))
+    prior = np.log(np.asarray(k_counts, dtype=np.float64)[live]) if size_prior else 0.0
     for r in range(CQ.shape[0]):
         if q_counts[r] == 0:
             continue
-        z = scale * (np.asarray(CK, dtype=np.float64)[live] @ np.asarray(CQ[r], dtype=np.float64))
+        z = scale * (np.asarray(CK, dtype=np.float64)[live] @ np.asarray(CQ[r], dtype=np.float64)) + prior
         z -= z.max()
         e = np.exp(z)
         I[r, live] = e / e.sum()
@@ -316,11 +321,14 @@ def sparse_attention(Q, K, V, q_labels, k_labels, mask, scale, rows=None):
 # ----------------------------------------------------------------------------
 
 
-def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full"):
+def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", topk_ratio=None,
+                  size_prior=False):
     """PARK retrieval for one (b, h): query K-means (Euclidean), key K-means
     with the query-derived metric (QRKC), PAMA importance, top-p mask
     (PARK Figure 2).  qrkc=False is the "w/o QRKC" ablation (M = I);
-    pama_mode="centroid" is "w/o PAMA"."""
+    pama_mode="centroid" is "w/o PAMA" (PARK Table 3); topk_ratio selects the
+    top-k at that retrieval ratio instead of top-p (PARK Table 10);
+    size_prior adds log |B_m| to the PAMA logits (a variant, see pama)."""
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
     d = Q.shape[1]
@@ -331,10 +339,13 @@ def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full"):
     q_counts = np.bincount(q_labels, minlength=NQ)
     k_counts = np.bincount(k_labels, minlength=NK)
     if pama_mode == "full":
-        I = pama(Q, q_labels, NQ, CK, k_counts, scale)
+        I = pama(Q, q_labels, NQ, CK, k_counts, scale, size_prior=size_prior)
     else:
-        I = pama_centroid_query(CQ, q_counts, CK, k_counts, scale)
-    mask = top_p(I, p, q_counts, k_counts)
+        I = pama_centroid_query(CQ, q_counts, CK, k_counts, scale, size_prior=size_prior)
+    if topk_ratio is None:
+        mask = top_p(I, p, q_counts, k_counts)
+    else:
+        mask = top_k_ratio(I, topk_ratio, q_counts, k_counts)
     q_perm, q_off = stable_permutation(q_labels, NQ)
     k_perm, k_off = stable_permutation(k_labels, NK)
     return dict(M=M, q_labels=q_labels, k_labels=k_labels, q_centroids=CQ, k_centroids=CK,

@@ -355,6 +355,53 @@ def test_top_k_ratio():
     assert m[0].tolist() == [False, True, False, True]
 
 
+def test_size_prior_pama_is_exact_block_mass_for_tight_clusters():
+    # Every key of cluster m equal to its centroid: the attention mass of block m
+    # is |B_m| exp(s q.c_m) / sum_m' |B_m'| exp(s q.c_m'), which the size-weighted
+    # PAMA must reproduce through the independently pinned exact block mass.
+    rng = np.random.default_rng(11)
+    d, NK = 8, 5
+    protos = np.round(rng.standard_normal((NK, d)) * 4) / 4
+    sizes = np.array([1, 3, 7, 2, 5])
+    K = np.repeat(protos, sizes, axis=0)
+    k_labels = np.repeat(np.arange(NK), sizes)
+    Q = np.round(rng.standard_normal((12, d)) * 4) / 4
+    q_labels = np.arange(12) % 3
+    s = 1 / math.sqrt(d)
+    I = po.pama(Q, q_labels, 3, protos, sizes, s, size_prior=True)
+    A, _ = po.exact_block_mass(Q, K, q_labels, 3, k_labels, NK, s)
+    assert np.allclose(I, A, rtol=1e-12, atol=1e-15)
+    # without the prior the unequal sizes make it differ
+    assert not np.allclose(po.pama(Q, q_labels, 3, protos, sizes, s), A, rtol=1e-3)
+
+
+def test_size_prior_with_equal_sizes_changes_nothing():
+    Q, K, V, ql, CQ, kl, CK = _tiny_case(seed=12)
+    s = 1 / math.sqrt(Q.shape[1])
+    counts = np.where(np.bincount(kl, minlength=CK.shape[0]) > 0, 6, 0)
+    a = po.pama(Q, ql, CQ.shape[0], CK, counts, s)
+    b = po.pama(Q, ql, CQ.shape[0], CK, counts, s, size_prior=True)
+    assert np.allclose(a, b, rtol=1e-13, atol=1e-16)
+
+
+def test_retrieve_topk_keeps_ceil_ratio_blocks():
+    rng = np.random.default_rng(13)
+    Q, K = rng.standard_normal((96, 16)), rng.standard_normal((96, 16))
+    r = po.retrieve_head(Q, K, 6, 10, 0.9, 3, "bf16", topk_ratio=0.25)
+    live = int((r["k_counts"] > 0).sum())
+    k = max(1, math.ceil(0.25 * live))
+    for q in range(6):
+        if r["q_counts"][q] == 0:
+            assert not r["mask"][q].any()
+            continue
+        kept = np.nonzero(r["mask"][q])[0]
+        assert kept.size == k
+        # every kept block is at least as important as every dropped live block
+        dropped = [m for m in range(10) if r["k_counts"][m] > 0 and not r["mask"][q, m]]
+        if dropped:
+            assert r["importance"][q, kept].min() >= r["importance"][q, dropped].max()
+
+
 def test_key_errors_qk_term_is_metric_distance():
     rng = np.random.default_rng(10)
     Q, K = rng.standard_normal((64, 8)), rng.standard_normal((50, 8))
