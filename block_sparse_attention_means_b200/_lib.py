@@ -20,6 +20,10 @@ PARK_F32 = 1
 
 PARK_FLAG_WARM_START_Q = 0x1
 PARK_FLAG_WARM_START_K = 0x2
+PARK_FLAG_NO_QRKC = 0x4
+PARK_FLAG_CENTROID_QUERY = 0x8
+PARK_FLAG_TOPK = 0x10
+PARK_FLAG_SIZE_PRIOR = 0x20
 
 PARK_CNT_Q_RECHECK = 0
 PARK_CNT_K_RECHECK = 1

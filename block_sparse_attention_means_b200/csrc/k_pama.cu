@@ -29,7 +29,7 @@ __global__ __launch_bounds__(128) void k_pama_mma(const uint16_t* __restrict__ Q
                                                   const int32_t* __restrict__ q_off, const uint16_t* __restrict__ CK,
                                                   const int32_t* __restrict__ k_off, const float* __restrict__ qnorm,
                                                   const float* __restrict__ ckmax, int N, int NQ, int NK, float sl2e,
-                                                  float delta_scale, float* __restrict__ importance,
+                                                  float delta_scale, int size_prior, float* __restrict__ importance,
                                                   float* __restrict__ rho) {
     constexpr int D = 128, CH = 64, LDS = D + 8;
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -50,7 +50,9 @@ __global__ __launch_bounds__(128) void k_pama_mma(const uint16_t* __restrict__ Q
     }
     const int32_t* ko = k_off + (size_t)bh * (NK + 1);
     for (int m = threadIdx.x; m < nch * CH; m += blockDim.x) {
-        live[m] = (m < NK && ko[m + 1] > ko[m]) ? 0.f : __int_as_float(0xff800000);
+        // additive logit term in log2 units: 0 (or log2 |B_m| with the size prior), -inf for empty m
+        const int nm = m < NK ? ko[m + 1] - ko[m] : 0;
+        live[m] = nm > 0 ? (size_prior ? (float)log2((double)nm) : 0.f) : __int_as_float(0xff800000);
         for (int w = 0; w < 4; ++w) colsum[w * nch * CH + m] = 0.f;
     }
     const uint16_t* Ch = CK + (size_t)bh * NK * D;
@@ -195,14 +197,16 @@ __global__ __launch_bounds__(128) void k_pama_mma(const uint16_t* __restrict__ Q
         // relative each, numerator and denominator), products, and the float32
         // column sums (within-warp adds, one add per tile, warp sum, division)
         double delta = (double)delta_scale * qm * cmax;
+        // the size prior's log2 |B_m| is rounded to float once: half an ulp of at most log2 N
+        if (size_prior) delta += 0.6931471805599453 * 5.9604644775390625e-8 * log2((double)N + 1.0);
         double rr = expm1(2.0 * delta) + 4.0 * 4.76837158203125e-7 + (16.0 + nr / 64.0) * 5.9604644775390625e-8;
         rho[(size_t)bh * NQ + r] = (float)(rr * 1.001);
     }
 }
 
 int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t* q_perm, const int32_t* q_off,
-                    const void* CK, const int32_t* k_off, const float* qnorm, float* importance, float* rho,
-                    float* ckmax, cudaStream_t st) {
+                    const void* CK, const int32_t* k_off, const float* qnorm, int size_prior, float* importance,
+                    float* rho, float* ckmax, cudaStream_t st) {
     const int D = 128;
     int nch = (NK + 63) / 64;
     size_t sm = 2 * 64 * (D + 8) * 2 + (size_t)nch * 64 * 4 * 5;
@@ -220,7 +224,7 @@ int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t*
         (float)((1.0 / sqrt((double)D)) * (kappa * 5.9604644775390625e-8 + 1.1920928955078125e-7) * 1.01);
     ::park::prof_begin(st);
     k_pama_mma<<<dim3(NQ, BH), 128, sm, st>>>((const uint16_t*)Q, q_perm, q_off, (const uint16_t*)CK, k_off, qnorm,
-                                              ckmax, N, NQ, NK, sl2e, delta_scale, importance, rho);
+                                              ckmax, N, NQ, NK, sl2e, delta_scale, size_prior, importance, rho);
     PARK_TRY_LAUNCH("k_pama_mma", st);
     return PARK_OK;
 }
@@ -262,7 +266,7 @@ static int next_pow2(int x) {
 // ---------------------------------------------------------------- top-p (certified)
 __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importance, const float* __restrict__ rho,
                                               const int32_t* __restrict__ q_off, const int32_t* __restrict__ k_off,
-                                              int NQ, int NK, int NKP, float p, uint8_t* __restrict__ mask,
+                                              int NQ, int NK, int NKP, float p, int topk, uint8_t* __restrict__ mask,
                                               int32_t* __restrict__ kept_cnt, float* __restrict__ importance_bound,
                                               int32_t* __restrict__ flag_list, int32_t* __restrict__ flag_count) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -339,7 +343,12 @@ __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importan
     __syncthreads();
     int cut = s_cut;
     bool ok;
-    if (p >= 1.0f) {
+    if (topk) {  // the ceil(p L) most important; certified when the last kept is clear of the next
+        const int kk = max(1, (int)ceil((double)p * (double)L));
+        cut = min(kk, L) - 1;
+        const double rh = (double)rho[row];
+        ok = cut + 1 >= L || (double)sv[cut] * (1.0 - rh) > (double)sv[cut + 1] * (1.0 + 2.0 * rh) + 1e-300;
+    } else if (p >= 1.0f) {
         cut = L - 1;
         ok = true;
     } else if (cut < 0) {
@@ -370,14 +379,14 @@ __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importan
 }
 
 int launch_topp(const float* importance, const float* rho, int BH, int NQ, int NK, const int32_t* q_off,
-                const int32_t* k_off, float p, uint8_t* mask, int32_t* kept_cnt, float* importance_bound,
+                const int32_t* k_off, float p, int topk, uint8_t* mask, int32_t* kept_cnt, float* importance_bound,
                 int32_t* flag_list, int32_t* flag_count, cudaStream_t st) {
     int NKP = next_pow2(NK);
     if (NKP < 512) NKP = 512;
     size_t sm = (size_t)NKP * (8 + 4 + 4 + 1) + 16;
     cudaFuncSetAttribute(k_topp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     ::park::prof_begin(st);
-    k_topp<<<dim3(NQ, BH), 512, sm, st>>>(importance, rho, q_off, k_off, NQ, NK, NKP, p, mask, kept_cnt,
+    k_topp<<<dim3(NQ, BH), 512, sm, st>>>(importance, rho, q_off, k_off, NQ, NK, NKP, p, topk, mask, kept_cnt,
                                           importance_bound, flag_list, flag_count);
     PARK_TRY_LAUNCH("k_topp", st);
     return PARK_OK;
@@ -405,7 +414,8 @@ template <typename T, int RPT>
 __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, const int32_t* __restrict__ q_perm,
                                                      const int32_t* __restrict__ q_off, const T* __restrict__ CK,
                                                      const int32_t* __restrict__ k_off, int N, int D, int NQ, int NK,
-                                                     int NKP, double scale, float p, const int32_t* __restrict__ list,
+                                                     int NKP, double scale, float p, int topk, int size_prior,
+                                                     const int32_t* __restrict__ list,
                                                      const int32_t* __restrict__ count_ptr, int all_clusters,
                                                      int BHNQ, int32_t* __restrict__ work_ctr,
                                                      double* __restrict__ zscratch, float* __restrict__ importance,
@@ -418,7 +428,8 @@ __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, co
     double* Cs = Qs + DM * RT;                                 // [DM][F64_CH]
     double* Isum = Cs + DM * F64_CH;                           // [NKP]
     double* part = Isum + NKP;                                 // [16][F64_CH]
-    int32_t* si = reinterpret_cast<int32_t*>(part + 16 * F64_CH);  // [NKP]
+    double* lsz = part + 16 * F64_CH;                          // [NKP] additive logit term per column
+    int32_t* si = reinterpret_cast<int32_t*>(lsz + NKP);       // [NKP]
     uint8_t* live = reinterpret_cast<uint8_t*>(si + NKP);      // [NKP]
     __shared__ int s_cut, s_e;
     const double NEG_INF = __longlong_as_double(0xfff0000000000000ll);
@@ -455,7 +466,9 @@ __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, co
         }
         for (int m = t; m < NKP; m += blockDim.x) {
             Isum[m] = 0.0;
-            live[m] = (m < NK && ko[m + 1] > ko[m]) ? 1 : 0;
+            const int nm = m < NK ? ko[m + 1] - ko[m] : 0;
+            live[m] = nm > 0 ? 1 : 0;
+            lsz[m] = (size_prior && nm > 0) ? log((double)nm) : 0.0;  // the size prior log |B_m|
         }
         const T* Ch = CK + (size_t)bh * NK * D;
         const T* Qh = Q + (size_t)bh * N * D;
@@ -522,7 +535,7 @@ __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, co
                     const bool lv = col < NK && live[col];
 #pragma unroll
                     for (int i = 0; i < RPT; ++i) {
-                        z[i][u] = lv ? scale * z[i][u] : NEG_INF;
+                        z[i][u] = lv ? scale * z[i][u] + lsz[col] : NEG_INF;
                         mx[i] = fmax(mx[i], z[i][u]);
                     }
                 }
@@ -598,10 +611,16 @@ __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, co
         if (t == 0) {
             double run = 0.0;
             int cut = -1;
-            for (int q = 0; q < NKP && Isum[q] >= 0.0; ++q) {
-                cut = q;
-                run += Isum[q];
-                if (p < 1.0f && run >= (double)p) break;
+            if (topk) {  // the ceil(p L) most important of the L non-empty key clusters
+                int L = 0;
+                while (L < NKP && Isum[L] >= 0.0) ++L;
+                cut = L > 0 ? min(max(1, (int)ceil((double)p * (double)L)), L) - 1 : -1;
+            } else {
+                for (int q = 0; q < NKP && Isum[q] >= 0.0; ++q) {
+                    cut = q;
+                    run += Isum[q];
+                    if (p < 1.0f && run >= (double)p) break;
+                }
             }
             s_cut = cut;
             kept_cnt[row] = cut + 1;
@@ -622,25 +641,27 @@ size_t pama_f64_scratch_bytes(int NK) {
 template <typename T, int RPT>
 static void pama_f64_launch(const void* Q, const int32_t* q_perm, const int32_t* q_off, const void* CK,
                             const int32_t* k_off, int N, int D, int NQ, int NK, int NKP, double scale, float p,
-                            const int32_t* list, const int32_t* count, int all_clusters, int BHNQ, int32_t* work_ctr,
+                            int topk, int size_prior, const int32_t* list, const int32_t* count, int all_clusters, int BHNQ, int32_t* work_ctr,
                             double* zscratch, float* importance, float* importance_bound, uint8_t* mask,
                             int32_t* kept_cnt, int64_t* counters, size_t sm, int blocks, cudaStream_t st) {
     cudaFuncSetAttribute(k_pama_f64<T, RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     k_pama_f64<T, RPT><<<blocks, 256, sm, st>>>((const T*)Q, q_perm, q_off, (const T*)CK, k_off, N, D, NQ, NK, NKP,
-                                                scale, p, list, count, all_clusters, BHNQ, work_ctr, zscratch,
+                                                scale, p, topk, size_prior, list, count, all_clusters, BHNQ,
+                                                work_ctr, zscratch,
                                                 importance, importance_bound, mask, kept_cnt, counters);
 }
 
 int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int NK, const int32_t* q_perm,
-                    const int32_t* q_off, const void* CK, const int32_t* k_off, float p, const int32_t* list,
+                    const int32_t* q_off, const void* CK, const int32_t* k_off, float p, int topk, int size_prior,
+                    const int32_t* list,
                     const int32_t* count, int all_clusters, int num_sms, int32_t* work_ctr, double* zscratch,
                     float* importance, float* importance_bound, uint8_t* mask, int32_t* kept_cnt, int64_t* counters,
                     cudaStream_t st) {
     if (NK > 4096 || D > 128) return PARK_ERR_UNSUPPORTED;
     const int NKP = next_pow2(NK);
     auto smem = [&](int RT) {
-        return (size_t)128 * RT * 8 + (size_t)128 * F64_CH * 8 + (size_t)NKP * 8 + 16 * F64_CH * 8 + (size_t)NKP * 4 +
-               NKP;
+        return (size_t)128 * RT * 8 + (size_t)128 * F64_CH * 8 + (size_t)NKP * 8 + 16 * F64_CH * 8 + (size_t)NKP * 8 +
+               (size_t)NKP * 4 + NKP;
     };
     const bool big = smem(128) <= 227 * 1024;  // 128-row tiles when the sort buffers leave room
     const size_t sm = smem(big ? 128 : 64);
@@ -649,24 +670,73 @@ int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int 
     ::park::prof_begin(st);
     if (dtype == PARK_BF16) {
         if (big)
-            pama_f64_launch<bf16_t, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, list, count,
+            pama_f64_launch<bf16_t, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, topk, size_prior, list, count,
                                        all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
                                        kept_cnt, counters, sm, blocks, st);
         else
-            pama_f64_launch<bf16_t, 4>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, list, count,
+            pama_f64_launch<bf16_t, 4>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, topk, size_prior, list, count,
                                        all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
                                        kept_cnt, counters, sm, blocks, st);
     } else {
         if (big)
-            pama_f64_launch<float, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, list, count,
+            pama_f64_launch<float, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, topk, size_prior, list, count,
                                       all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
                                       kept_cnt, counters, sm, blocks, st);
         else
-            pama_f64_launch<float, 4>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, list, count,
+            pama_f64_launch<float, 4>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, topk, size_prior, list, count,
                                       all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
                                       kept_cnt, counters, sm, blocks, st);
     }
     PARK_TRY_LAUNCH("k_pama_f64", st);
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- "w/o PAMA" rows
+// Rows for the float64 PAMA kernel when the query centroid stands for its
+// cluster: cluster r has one row (centroid r) if it is non-empty, none
+// otherwise.  off[r] = number of non-empty clusters before r, perm[off[r]] = r.
+__global__ __launch_bounds__(1024) void k_centroid_rows(const int32_t* __restrict__ q_off, int NQ,
+                                                        int32_t* __restrict__ perm, int32_t* __restrict__ off) {
+    __shared__ int32_t wsum[32];
+    const int bh = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int32_t* qo = q_off + (size_t)bh * (NQ + 1);
+    int32_t* po = off + (size_t)bh * (NQ + 1);
+    int32_t* pp = perm + (size_t)bh * NQ;
+    const int seg = (NQ + 1023) / 1024, b0 = t * seg, b1 = min(NQ, b0 + seg);
+    int loc = 0;
+    for (int r = b0; r < b1; ++r) loc += qo[r + 1] > qo[r];
+    int incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        const int x = wsum[lane];
+        int xi = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, xi, o);
+            if (lane >= o) xi += y;
+        }
+        wsum[lane] = xi - x;
+    }
+    __syncthreads();
+    int run = wsum[w] + incl - loc;
+    for (int r = b0; r < b1; ++r) {
+        po[r] = run;
+        if (qo[r + 1] > qo[r]) pp[run++] = r;
+    }
+    if (b0 < NQ && b1 == NQ) po[NQ] = run;
+    if (NQ == 0 && t == 0) po[0] = 0;
+}
+
+int launch_centroid_rows(const int32_t* q_off, int BH, int NQ, int32_t* perm, int32_t* off, cudaStream_t st) {
+    ::park::prof_begin(st);
+    k_centroid_rows<<<BH, 1024, 0, st>>>(q_off, NQ, perm, off);
+    PARK_TRY_LAUNCH("k_centroid_rows", st);
     return PARK_OK;
 }
 

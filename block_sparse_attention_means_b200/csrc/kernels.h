@@ -53,19 +53,23 @@ int launch_update(const void* X, int dtype, int BH, int N, int D, int K, const i
                   const int32_t* offsets, void* C, cudaStream_t st);
 
 // ---- k_pama.cu
+// size_prior: logits gain log |B_m|; topk: keep the ceil(p L) most important (p a ratio)
 int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t* q_perm, const int32_t* q_off,
-                    const void* CK, const int32_t* k_off, const float* qnorm, float* importance, float* rho,
-                    float* ckmax, cudaStream_t st);
+                    const void* CK, const int32_t* k_off, const float* qnorm, int size_prior, float* importance,
+                    float* rho, float* ckmax, cudaStream_t st);
 int launch_topp(const float* importance, const float* rho, int BH, int NQ, int NK, const int32_t* q_off,
-                const int32_t* k_off, float p, uint8_t* mask, int32_t* kept_cnt, float* importance_bound,
+                const int32_t* k_off, float p, int topk, uint8_t* mask, int32_t* kept_cnt, float* importance_bound,
                 int32_t* flag_list, int32_t* flag_count, cudaStream_t st);
+// one row per non-empty query cluster (its centroid), for "w/o PAMA" through launch_pama_f64
+int launch_centroid_rows(const int32_t* q_off, int BH, int NQ, int32_t* perm, int32_t* off, cudaStream_t st);
 // Float64 PAMA + top-p for the listed clusters (or all): at most kPamaF64Slots
 // CTAs, each with pama_f64_scratch_bytes(NK) / kPamaF64Slots bytes of float64
 // scratch; work_ctr (zeroed by the caller) hands out the clusters.
 constexpr int kPamaF64Slots = 160;
 size_t pama_f64_scratch_bytes(int NK);
 int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int NK, const int32_t* q_perm,
-                    const int32_t* q_off, const void* CK, const int32_t* k_off, float p, const int32_t* list,
+                    const int32_t* q_off, const void* CK, const int32_t* k_off, float p, int topk, int size_prior,
+                    const int32_t* list,
                     const int32_t* count, int all_clusters, int num_sms, int32_t* work_ctr, double* zscratch,
                     float* importance, float* importance_bound, uint8_t* mask, int32_t* kept_cnt, int64_t* counters,
                     cudaStream_t st);

@@ -118,7 +118,7 @@ int metric_chunks(const Dims& d) {
 
 struct RetrievalWs {
     size_t M, Mpart, xnorm_q, xnorm_k, wop, b32, b64, w64, wmax, bmax, lfull, lcnt, hist, rho, plist,
-        pcnt, kcnt, f64z, total;
+        pcnt, kcnt, f64z, cperm, coff, total;
 };
 
 RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
@@ -144,6 +144,8 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
     w.pcnt = c.take(16 * 4);
     w.kcnt = c.take(BH * NQ * 4);
     w.f64z = c.take(pama_f64_scratch_bytes(NK));
+    w.cperm = c.take(BH * NQ * 4);
+    w.coff = c.take(BH * (NQ + 1) * 4);
     w.total = c.off;
     return w;
 }
@@ -283,6 +285,14 @@ size_t ws_bytes_for(const Dims& d, int NQ, int NK) {
     return a > b ? a : b;
 }
 
+// Known flag bits only; with PARK_FLAG_TOPK, p is a ratio in (0, 1].
+bool flags_ok(uint32_t flags, float p) {
+    const uint32_t known = PARK_FLAG_WARM_START_Q | PARK_FLAG_WARM_START_K | PARK_FLAG_NO_QRKC |
+                           PARK_FLAG_CENTROID_QUERY | PARK_FLAG_TOPK | PARK_FLAG_SIZE_PRIOR;
+    if (flags & ~known) return false;
+    return !(flags & PARK_FLAG_TOPK) || p <= 1.0f;
+}
+
 int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, float p, int iters,
                   park_retrieval* out, void* ws, cudaStream_t st) {
     const RetrievalWs w = plan_retrieval(d, NQ, NK);
@@ -294,20 +304,33 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
     PARK_CHECK(memset_async(at<int32_t>(ws, w.pcnt), 16 * 4, st));
     PARK_CHECK(launch_input_check(Q, nel, d.dtype, out->status, st));
     PARK_CHECK(launch_input_check(K, nel, d.dtype, out->status, st));
+    const uint32_t fl = out->flags;
+    const bool qrkc = (fl & PARK_FLAG_NO_QRKC) == 0;
+    const int topk = (fl & PARK_FLAG_TOPK) != 0, size_prior = (fl & PARK_FLAG_SIZE_PRIOR) != 0;
     double* M = at<double>(ws, w.M);
-    PARK_CHECK(launch_metric(Q, d.dtype, BH, N, D, at<double>(ws, w.Mpart), metric_chunks(d), M, out->metric, st));
+    if (qrkc || out->metric)
+        PARK_CHECK(launch_metric(Q, d.dtype, BH, N, D, at<double>(ws, w.Mpart), metric_chunks(d), M, out->metric, st));
 
     Side sq{Q, NQ, out->q_centroids, out->q_labels, out->q_perm, out->q_offsets, nullptr,
             (out->flags & PARK_FLAG_WARM_START_Q) != 0, PARK_CNT_Q_RECHECK, at<float>(ws, w.xnorm_q),
             NQ > NK ? NQ : NK, out->status};
-    Side sk{K, NK, out->k_centroids, out->k_labels, out->k_perm, out->k_offsets, M,
+    Side sk{K, NK, out->k_centroids, out->k_labels, out->k_perm, out->k_offsets, qrkc ? M : nullptr,
             (out->flags & PARK_FLAG_WARM_START_K) != 0, PARK_CNT_K_RECHECK, at<float>(ws, w.xnorm_k),
             NQ > NK ? NQ : NK, out->status};
     PARK_CHECK(run_kmeans(d, sq, iters, w, ws, out->counters, num_sms, st));
     PARK_CHECK(run_kmeans(d, sk, iters, w, ws, out->counters, num_sms, st));
 
     int32_t* kcnt = at<int32_t>(ws, w.kcnt);
-    if (d.dtype == PARK_BF16) {
+    if (fl & PARK_FLAG_CENTROID_QUERY) {
+        // "w/o PAMA": each non-empty query cluster is one row, its centroid, through the float64 kernel
+        int32_t* cperm = at<int32_t>(ws, w.cperm);
+        int32_t* coff = at<int32_t>(ws, w.coff);
+        PARK_CHECK(launch_centroid_rows(out->q_offsets, BH, NQ, cperm, coff, st));
+        PARK_CHECK(launch_pama_f64(out->q_centroids, d.dtype, BH, NQ, D, NQ, NK, cperm, coff, out->k_centroids,
+                                   out->k_offsets, p, topk, size_prior, nullptr, nullptr, 1, num_sms,
+                                   at<int32_t>(ws, w.pcnt) + 4, at<double>(ws, w.f64z), out->importance,
+                                   out->importance_bound, out->mask, kcnt, out->counters, st));
+    } else if (d.dtype == PARK_BF16) {
         // max ||c_m|| over the final key centroids, for the PAMA bound
         CentroidOps ops{nullptr, D, at<float>(ws, w.b32), (int)align_up((size_t)(NQ > NK ? NQ : NK), 128),
                         at<double>(ws, w.b64), nullptr, at<float>(ws, w.wmax), at<float>(ws, w.bmax)};
@@ -315,17 +338,20 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
         PARK_CHECK(memset_async(ops.bmax, (size_t)BH * 4, st));
         PARK_CHECK(launch_centroid_prep(out->k_centroids, d.dtype, BH, NK, D, nullptr, ops, st));
         PARK_CHECK(launch_pama_mma(Q, BH, N, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids, out->k_offsets,
-                                   at<float>(ws, w.xnorm_q), out->importance, at<float>(ws, w.rho), ops.wmax, st));
+                                   at<float>(ws, w.xnorm_q), size_prior, out->importance, at<float>(ws, w.rho),
+                                   ops.wmax, st));
         PARK_CHECK(launch_topp(out->importance, at<float>(ws, w.rho), BH, NQ, NK, out->q_offsets, out->k_offsets, p,
-                               out->mask, kcnt, out->importance_bound, at<int32_t>(ws, w.plist),
+                               topk, out->mask, kcnt, out->importance_bound, at<int32_t>(ws, w.plist),
                                at<int32_t>(ws, w.pcnt), st));
         PARK_CHECK(launch_pama_f64(Q, d.dtype, BH, N, D, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids,
-                                   out->k_offsets, p, at<int32_t>(ws, w.plist), at<int32_t>(ws, w.pcnt), 0, num_sms,
+                                   out->k_offsets, p, topk, size_prior, at<int32_t>(ws, w.plist),
+                                   at<int32_t>(ws, w.pcnt), 0, num_sms,
                                    at<int32_t>(ws, w.pcnt) + 4, at<double>(ws, w.f64z), out->importance,
                                    out->importance_bound, out->mask, kcnt, out->counters, st));
     } else {
         PARK_CHECK(launch_pama_f64(Q, d.dtype, BH, N, D, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids,
-                                   out->k_offsets, p, nullptr, nullptr, 1, num_sms, at<int32_t>(ws, w.pcnt) + 4,
+                                   out->k_offsets, p, topk, size_prior, nullptr, nullptr, 1, num_sms,
+                                   at<int32_t>(ws, w.pcnt) + 4,
                                    at<double>(ws, w.f64z), out->importance, out->importance_bound, out->mask, kcnt,
                                    out->counters, st));
     }
@@ -387,6 +413,7 @@ int park_retrieve(const void* Q, const void* K, const park_shape* shape, int NQ,
     PARK_CHECK(check_shape(shape, NQ, NK, &d));
     if (!Q || !K || !ws || !retrieval_ptrs_ok(out)) return PARK_ERR_INVALID_ARG;
     if (!(p > 0.0f) || !std::isfinite(p) || iters < 1) return PARK_ERR_INVALID_ARG;
+    if (!flags_ok(out->flags, p)) return PARK_ERR_INVALID_ARG;
     if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
     return retrieve_impl(Q, K, d, NQ, NK, p, iters, out, ws, static_cast<cudaStream_t>(stream));
 }
@@ -406,6 +433,7 @@ int park_layer(const void* Q, const void* K, const void* V, const park_shape* sh
     PARK_CHECK(check_shape(shape, NQ, NK, &d));
     if (!Q || !K || !V || !O || !ws || !retrieval_ptrs_ok(out)) return PARK_ERR_INVALID_ARG;
     if (!(p > 0.0f) || !std::isfinite(p) || iters < 1) return PARK_ERR_INVALID_ARG;
+    if (!flags_ok(out->flags, p)) return PARK_ERR_INVALID_ARG;
     if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     PARK_CHECK(retrieve_impl(Q, K, d, NQ, NK, p, iters, out, ws, st));

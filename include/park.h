@@ -75,6 +75,23 @@ extern "C" {
  * across denoising steps, PARK Appendix Table 9). */
 #define PARK_FLAG_WARM_START_Q 0x1u
 #define PARK_FLAG_WARM_START_K 0x2u
+/* Selection variants (PARK Table 3 ablations, Table 10 top-k, and a size prior
+ * that the pages do not have); any combination may be set:
+ *   NO_QRKC          "w/o QRKC": key K-means is Euclidean (M = I); out->metric,
+ *                    when non-NULL, is still written.
+ *   CENTROID_QUERY   "w/o PAMA": I_rm = softmax_m(s c_r . c_m) with the query
+ *                    centroid c_r in place of every member query; computed in
+ *                    float64 (importance_bound rows are 0).
+ *   TOPK             keep the ceil(p * L_r) most important key clusters of each
+ *                    non-empty query cluster (L_r = non-empty key clusters; ties:
+ *                    lower m; at least one), p read as the retrieval ratio in
+ *                    (0, 1] (the float32 value passed).
+ *   SIZE_PRIOR       PAMA logits gain log |B_m|: P_im proportional to
+ *                    |B_m| exp(s q_i . c_m). */
+#define PARK_FLAG_NO_QRKC 0x4u
+#define PARK_FLAG_CENTROID_QUERY 0x8u
+#define PARK_FLAG_TOPK 0x10u
+#define PARK_FLAG_SIZE_PRIOR 0x20u
 
 /* ---- park_retrieval.counters indices (outputs, int64) ------------------ */
 #define PARK_CNT_Q_RECHECK 0    /* query rows whose bf16 score margin was not

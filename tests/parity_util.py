@@ -32,6 +32,16 @@ def oracle_layer(name: str, seed: int = 0, p: float | None = None, NQ: int | Non
                     cfg.p if p is None else p, iters or cfg.iters, cfg.dtype)
 
 
+@functools.lru_cache(maxsize=None)
+def oracle_layer_variant(name: str, p: float, variant: tuple):
+    """The oracle layer with retrieval options (qrkc, pama_mode, topk_ratio,
+    size_prior) given as a sorted tuple of (key, value) pairs."""
+    cfg = CONFIGS[name]
+    Q, K, V = inputs(name)
+    return po.layer(Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64), cfg.NQ, cfg.NK, p, cfg.iters,
+                    cfg.dtype, **dict(variant))
+
+
 def to_device(x: np.ndarray, dtype: torch.dtype, device="cuda:0") -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(x)).to(device=device).to(dtype).contiguous()
 

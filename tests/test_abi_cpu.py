@@ -36,7 +36,8 @@ def test_struct_layout_matches_header():
     assert re.search(r"#define PARK_NUM_COUNTERS 8", text)
     for name in ("PARK_OK", "PARK_ERR_INVALID_ARG", "PARK_ERR_UNSUPPORTED", "PARK_ERR_WORKSPACE", "PARK_ERR_CUDA",
                  "PARK_ERR_RANGE", "PARK_ERR_TIMEOUT", "PARK_BF16", "PARK_F32", "PARK_FLAG_WARM_START_Q",
-                 "PARK_FLAG_WARM_START_K", "PARK_CNT_KEPT_PAIRS"):
+                 "PARK_FLAG_WARM_START_K", "PARK_FLAG_NO_QRKC", "PARK_FLAG_CENTROID_QUERY", "PARK_FLAG_TOPK",
+                 "PARK_FLAG_SIZE_PRIOR", "PARK_CNT_KEPT_PAIRS"):
         m = re.search(rf"#define {name} (\w+)", text)
         assert m and int(m.group(1).rstrip("u"), 0) == getattr(_lib, name), name
 
@@ -103,6 +104,14 @@ def test_host_argument_errors_enqueue_nothing():
     r2 = _fake_retrieval()
     r2.mask = None
     cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.9, 10, ctypes.byref(r2), fake, need,
+                                    None), _lib.PARK_ERR_INVALID_ARG))
+    r3 = _fake_retrieval()
+    r3.flags = 0x40                               # unknown flag bit
+    cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.9, 10, ctypes.byref(r3), fake, need,
+                                    None), _lib.PARK_ERR_INVALID_ARG))
+    r4 = _fake_retrieval()
+    r4.flags = _lib.PARK_FLAG_TOPK                # a top-k ratio above 1
+    cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 1.5, 10, ctypes.byref(r4), fake, need,
                                     None), _lib.PARK_ERR_INVALID_ARG))
     for got, want in cases:
         assert got == want

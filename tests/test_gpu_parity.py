@@ -75,6 +75,48 @@ def test_layer_matches_oracle(park, name):
     assert int(cnt[4]) == sum(int(h["mask"].sum()) for h in ref)
 
 
+# Selection variants (PARK Table 3 ablations, Table 10 top-k, the size prior):
+# flag bits, oracle options, and the p passed (a retrieval ratio for top-k).
+_RATIO = float(np.float32(0.3))  # the float32 value the C ABI receives
+VARIANTS = {
+    "no_qrkc": (0x4, (("qrkc", False),), None),
+    "centroid_query": (0x8, (("pama_mode", "centroid"),), None),
+    "topk": (0x10, (("topk_ratio", _RATIO),), _RATIO),
+    "size_prior": (0x20, (("size_prior", True),), None),
+    "all": (0x3C, (("pama_mode", "centroid"), ("qrkc", False), ("size_prior", True), ("topk_ratio", _RATIO)),
+            _RATIO),
+}
+
+
+@pytest.mark.parametrize("variant", sorted(VARIANTS))
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_selection_variants_match_oracle(park, name, variant):
+    flags, opts, p = VARIANTS[variant]
+    cfg = CONFIGS[name]
+    p = cfg.p if p is None else p
+    Q, K, V = pu.inputs(name)
+    ref = pu.oracle_layer_variant(name, p, opts)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    shape = park.Shape.of(cfg, dt)
+    q, k, v = (pu.to_device(x, dt) for x in (Q, K, V))
+    out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, q.device)
+    out.flags = flags
+    O, r = park.layer(q, k, v, shape, cfg.NQ, cfg.NK, p, cfg.iters, out=out)
+    torch.cuda.synchronize()
+    assert r.status_code() == 0, f"device status {r.status_code()}"
+    fails = pu.compare_retrieval(r, ref, cfg.NQ, cfg.NK)
+    assert not fails, "\n".join(fails[:20])
+    check_importance_bound(r, ref)
+    pu.assert_output_close(O, ref, cfg.dtype == "f32")
+    if "topk_ratio" in dict(opts):
+        mask = r.mask.cpu().numpy().reshape(-1, cfg.NQ, cfg.NK)
+        for bh, h in enumerate(ref):
+            live = int((h["k_counts"] > 0).sum())
+            want = max(1, int(np.ceil(_RATIO * live)))
+            rows = h["q_counts"] > 0
+            assert np.all(mask[bh][rows].sum(axis=1) == want)
+
+
 def test_per_step_injection_small(park):
     """Feed the oracle's iteration-t centroids as a warm start and run one
     iteration: labels and updated centroids must match the oracle's step t."""
