@@ -226,6 +226,11 @@ def workload_config(cfg) -> dict:
             "l2": "inputs larger than L2 (Q, K, V 731 MB each vs 126 MB L2); no flush"}
 
 
+# Retrieval variants: flag bits of park_retrieval.flags and the p passed (a ratio for top-k).
+VARIANTS = {"park": (0, None), "no_qrkc": (0x4, None), "centroid_query": (0x8, None), "topk_0.3": (0x10, 0.3),
+            "size_prior": (0x20, None)}
+
+
 # ----------------------------------------------------------------------------- roofline of one kernel
 
 KERNEL_SOURCES = {"k_sparse_attn_tc": ["block_sparse_attention_means_b200/csrc/k_attn_tc.cu"],
@@ -280,6 +285,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override H (small cases for profiler captures)")
+    ap.add_argument("--variant", default="park", choices=sorted(VARIANTS),
+                    help="retrieval variant (PARK Table 3 ablations, Table 10 top-k, size prior)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warmup must be >= 3", file=sys.stderr)
@@ -325,12 +332,15 @@ def main():
     Q, K, V = (host[n].to(dev, non_blocking=True) for n in ("Q", "K", "V"))
     shape = park.Shape.of(cfg)
     out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, dev)
+    vflags, vp = VARIANTS[args.variant]
+    out.flags = vflags
+    p_arg = cfg.p if vp is None else vp
     ws = park.alloc_workspace(shape, cfg.NQ, cfg.NK, dev)
     O = torch.empty_like(Q)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        park.layer(Q, K, V, shape, cfg.NQ, cfg.NK, cfg.p, cfg.iters, O=O, out=out, ws=ws, stream=stream)
+        park.layer(Q, K, V, shape, cfg.NQ, cfg.NK, p_arg, cfg.iters, O=O, out=out, ws=ws, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -409,7 +419,8 @@ def main():
     line = {"metric": METRIC, "value": round(value, 3), "unit": "ms", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(worst_ms, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(cfg), "roofline": roof, "attention_roofline": attn_roof,
+            "config": {**workload_config(cfg), **({"variant": args.variant} if args.variant != "park" else {})},
+            "roofline": roof, "attention_roofline": attn_roof,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches), "clocks": clocks,
             "status": status,
             "retrieval_ms_per_layer": round(retrieval_ms, 3),

@@ -1,0 +1,52 @@
+"""Selection variants measured against dense attention on one HunyuanVideo-shaped
+head (N = 119056, NQ = NK = 930): the attention recall of the kept blocks (PARK
+Table 1's quantity) and the PAMA-to-block-mass total variation (PARK Table 4's
+quantity), both on 1024 sampled query rows, computed by the oracle's float64
+diagnostics from the labels, centroids and masks that the GPU produced.  The
+values are printed (pytest -s); the assertions are sanity bounds only, since the
+pages' absolute recalls are on real activations."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import park_oracle as po
+from synth import CONFIGS
+from synth.generator import gen_layer
+
+import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+# flag bits of park_retrieval.flags and the p passed (a retrieval ratio for top-k)
+VARIANTS = {"park (top-p 0.9)": (0x0, 0.9), "w/o QRKC": (0x4, 0.9), "w/o PAMA": (0x8, 0.9),
+            "top-k 0.3": (0x10, 0.3), "size prior": (0x20, 0.9)}
+
+
+def test_variant_recall_and_tv():
+    import block_sparse_attention_means_b200 as park
+    cfg = CONFIGS["hunyuan"].replace(H=1, name="hunyuan_h1")
+    Q, K, _ = gen_layer(cfg, 0)
+    Q0, K0 = Q[0, 0].astype(np.float64), K[0, 0].astype(np.float64)
+    s = 1.0 / math.sqrt(cfg.D)
+    rows = np.sort(np.random.default_rng(0).choice(cfg.N, 1024, replace=False))
+    shape = park.Shape.of(cfg, torch.bfloat16)
+    q, k = pu.to_device(Q, torch.bfloat16), pu.to_device(K, torch.bfloat16)
+    print()
+    for name, (flags, p) in VARIANTS.items():
+        out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, q.device)
+        out.flags = flags
+        park.retrieve(q, k, shape, cfg.NQ, cfg.NK, p, cfg.iters, out=out)
+        torch.cuda.synchronize()
+        assert out.status_code() == 0
+        ql, kl = out.q_labels.cpu().numpy()[0, 0], out.k_labels.cpu().numpy()[0, 0]
+        mask = out.mask.cpu().numpy()[0, 0].astype(bool)
+        CK = pu.np64(out.k_centroids)[0, 0]
+        recall = po.block_recall(Q0, K0, ql, kl, mask, s, rows)
+        tv = po.attention_tv(Q0[rows], K0, kl, cfg.NK, CK, s)
+        live = np.bincount(kl, minlength=cfg.NK) > 0
+        kept = mask[:, live].mean()
+        print(f"{name:18s} recall {recall:.4f}  TV {tv:.4f}  kept block fraction {kept:.4f}")
+        assert 0.0 < recall <= 1.0 + 1e-9
+        assert 0.0 <= tv <= 1.0
