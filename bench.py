@@ -220,10 +220,12 @@ def run_reference(args, cfg):
 
 
 def workload_config(cfg) -> dict:
-    return {"workload": f"HunyuanVideo-shaped PARK layer ({cfg.name})", "B": cfg.B, "H": cfg.H, "N": cfg.N,
+    shaped = "Wan2.1-14B" if cfg.name.startswith("wan") else "HunyuanVideo"
+    return {"workload": f"{shaped}-shaped PARK layer ({cfg.name})", "B": cfg.B, "H": cfg.H, "N": cfg.N,
             "grid": [cfg.T, cfg.Hg, cfg.W], "n_text": cfg.n_text, "D": cfg.D, "NQ": cfg.NQ, "NK": cfg.NK,
             "kmeans_iters": cfg.iters, "p": cfg.p, "parallelism": "replicas",
-            "l2": "inputs larger than L2 (Q, K, V 731 MB each vs 126 MB L2); no flush"}
+            "l2": f"inputs larger than L2 (Q, K, V {cfg.B * cfg.H * cfg.N * cfg.D * 2 / 1e6:.0f} MB each vs 126 MB L2); "
+                  "no flush"}
 
 
 # Retrieval variants: flag bits of park_retrieval.flags and the p passed (a ratio for top-k).
@@ -293,7 +295,12 @@ def main():
         args.warmup = 3
 
     from synth import CONFIGS
-    cfg = CONFIGS[args.config]
+    from synth.generator import sweep_configs
+    all_cfgs = {**CONFIGS, **{c.name: c for c in sweep_configs()}}
+    if args.config not in all_cfgs:
+        print(f"unknown config {args.config}; one of {sorted(all_cfgs)}", file=sys.stderr)
+        return 2
+    cfg = all_cfgs[args.config]
     if args.heads:
         cfg = cfg.replace(H=args.heads, name=f"{cfg.name}_h{args.heads}")
     if args.impl == "reference":
