@@ -78,14 +78,28 @@ __global__ __launch_bounds__(272) void k_metric_partial(const T* __restrict__ Q,
     for (int u = 0; u < 4; ++u)
 #pragma unroll
         for (int v = 0; v < 8; ++v) acc[u][v] = 0.0;
+    // the next block of rows is fetched into registers while the current one is used
+    constexpr int PER = (kMetricRB * 128 + 271) / 272;
+    float pre[PER];  // inputs are exact in float32
+    auto fetch = [&](int base) {
+#pragma unroll
+        for (int v = 0; v < PER; ++v) {
+            const int e = t + 272 * v, rr = e >> 7, jj = e & 127;
+            pre[v] = (e < kMetricRB * 128 && base + rr < r1 && jj < D)
+                         ? Elem<T>::to_float(X + (size_t)(base + rr) * D, jj) : 0.f;
+        }
+    };
+    if (r0 < r1) fetch(r0);
     for (int base = r0; base < r1; base += kMetricRB) {
         const int nr = min(kMetricRB, r1 - base);
         __syncthreads();
-        for (int e = t; e < kMetricRB * 128; e += blockDim.x) {
-            const int rr = e >> 7, jj = e & 127;
-            qs[rr][jj] = (rr < nr && jj < D) ? Elem<T>::to_double(X + (size_t)(base + rr) * D, jj) : 0.0;
+#pragma unroll
+        for (int v = 0; v < PER; ++v) {
+            const int e = t + 272 * v;
+            if (e < kMetricRB * 128) qs[e >> 7][e & 127] = (double)pre[v];
         }
         __syncthreads();
+        if (base + kMetricRB < r1) fetch(base + kMetricRB);
         if (active) {
             for (int rr = 0; rr < nr; ++rr) {
                 double qa[4], qb[8];

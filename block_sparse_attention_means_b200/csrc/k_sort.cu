@@ -175,23 +175,34 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
     }
     const int32_t* pm = perm + (size_t)bh * N + start;
     const T* Xh = X + (size_t)bh * N * D;
-    if (slot < RPI) {
-        for (int j = slot; j < n; j += RPI) {
-            int tok = pm[j];
-            uint4 v = *reinterpret_cast<const uint4*>(Xh + (size_t)tok * D + piece * VEC);
-            uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            if (!TWO_LIMBS) {
+    auto add_piece = [&](const uint4& v) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        if (!TWO_LIMBS) {
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) acc_hi[e] += fixed_bf16((uint16_t)(w[e >> 1] >> (16 * (e & 1))));
-            } else {
+            for (int e = 0; e < VEC; ++e) acc_hi[e] += fixed_bf16((uint16_t)(w[e >> 1] >> (16 * (e & 1))));
+        } else {
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    long long f = fixed_f32(w[e]);
-                    acc_lo[e] += (unsigned long long)(f & 0xFFFFFFFFll);
-                    acc_hi[e] += f >> 32;
-                }
+            for (int e = 0; e < VEC; ++e) {
+                const long long f = fixed_f32(w[e]);
+                acc_lo[e] += (unsigned long long)(f & 0xFFFFFFFFll);
+                acc_hi[e] += f >> 32;
             }
         }
+    };
+    if (slot < RPI) {
+        // four member rows in flight per thread (integer sums: the order does not matter)
+        int j = slot;
+        for (; j + 3 * RPI < n; j += 4 * RPI) {
+            int tok[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) tok[u] = pm[j + u * RPI];
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const uint4*>(Xh + (size_t)tok[u] * D + piece * VEC);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) add_piece(v[u]);
+        }
+        for (; j < n; j += RPI) add_piece(*reinterpret_cast<const uint4*>(Xh + (size_t)pm[j] * D + piece * VEC));
     }
     long long* red_hi = red;
     long long* red_lo = red + RPI * D;
