@@ -279,6 +279,64 @@ def top_k_ratio(I, rho, q_counts, k_counts):
 
 
 # ----------------------------------------------------------------------------
+# sampling with inclusion-probability weighting
+# ----------------------------------------------------------------------------
+
+
+def sip_probabilities(values, budget):
+    """Inclusion probabilities proportional to importance, capped at 1, with
+    expected sample size `budget` ("AB-Attention Brings More Accurate Sparse
+    Attention to Video Diffusion", paragraph on SIP: blocks are sampled according
+    to their estimated importance).  READING: pi_m = min(1, c v_m) with c such
+    that sum_m pi_m = budget; the blocks whose c v_m would exceed 1 are taken with
+    certainty, found in descending order of v (ties: lower index first).
+    values: importances of the candidate blocks (> 0); returns pi in their order."""
+    v = np.asarray(values, dtype=np.float64)
+    L = v.size
+    if budget >= L:
+        return np.ones(L)
+    order = sorted(range(L), key=lambda m: (-v[m], m))
+    sv = v[order]
+    tail = np.cumsum(sv[::-1])[::-1]           # tail[t] = sum of sv[t:]
+    t = 0
+    while (budget - t) * sv[t] > tail[t]:      # c_t v_(t) > 1: the t-th largest is certain
+        t += 1
+    c = (budget - t) / tail[t]
+    pi = np.empty(L)
+    for pos, m in enumerate(order):
+        pi[m] = 1.0 if pos < t else c * sv[pos]
+    return pi
+
+
+def sip_select(I, ratio, u, q_counts, k_counts):
+    """SIP selection ("AB-Attention ...", paragraph on SIP).  READING: per
+    non-empty query cluster r, expected budget B = ceil(ratio L_r) (L_r
+    non-empty key clusters); pi from sip_probabilities(I_r., B); block m is kept
+    when u[r, m] < pi_m (independent draws, u uniform on [0, 1) given as input);
+    kept blocks get the weight 1 / pi_m (the inverse inclusion probability).  If no
+    block is drawn, the most important block is kept (with its weight).  Returns
+    (mask, weight), weight 0 where not kept."""
+    NQ, NK = I.shape
+    mask = np.zeros((NQ, NK), dtype=bool)
+    weight = np.zeros((NQ, NK))
+    live = [m for m in range(NK) if k_counts[m] > 0]
+    B = max(1, int(math.ceil(ratio * len(live))))
+    for r in range(NQ):
+        if q_counts[r] == 0:
+            continue
+        pi = sip_probabilities(I[r, live], B)
+        for m, pm in zip(live, pi):
+            if u[r, m] < pm:
+                mask[r, m] = True
+                weight[r, m] = 1.0 / pm
+        if not mask[r].any():
+            best = min(live, key=lambda m: (-I[r, m], m))
+            mask[r, best] = True
+            weight[r, best] = 1.0 / pi[live.index(best)]
+    return mask, weight
+
+
+# ----------------------------------------------------------------------------
 # attention
 # ----------------------------------------------------------------------------
 
@@ -295,11 +353,14 @@ def dense_attention(Q, K, V, scale):
     return O
 
 
-def sparse_attention(Q, K, V, q_labels, k_labels, mask, scale, rows=None):
+def sparse_attention(Q, K, V, q_labels, k_labels, mask, scale, rows=None, weight=None):
     """Block-sparse attention: query i attends, with a renormalised Softmax,
     only to keys whose cluster is kept for its query cluster a(i) ("computing
     attention only within" the retrieved blocks, PARK abstract).  Returns
-    float64 [N, d] in original token order (or only the listed rows)."""
+    float64 [N, d] in original token order (or only the listed rows).
+    weight[r, m] (SIP): every exp term of key cluster m is multiplied by it, in
+    the numerator and in the normaliser (a ratio of two inverse-probability
+    weighted sums, each an unbiased estimate of its dense counterpart)."""
     Q, K, V = (np.asarray(a, dtype=np.float64) for a in (Q, K, V))
     q_labels = np.asarray(q_labels)
     k_labels = np.asarray(k_labels)
@@ -310,6 +371,8 @@ def sparse_attention(Q, K, V, q_labels, k_labels, mask, scale, rows=None):
         sel = np.nonzero(lab == r)[0]
         keys = np.nonzero(mask[r][k_labels])[0]
         S = scale * (Q[want[sel]] @ K[keys].T)
+        if weight is not None:
+            S += np.log(weight[r][k_labels[keys]])[None, :]
         S -= S.max(axis=1, keepdims=True)
         P = np.exp(S)
         O[sel] = (P @ V[keys]) / P.sum(axis=1, keepdims=True)
@@ -322,13 +385,15 @@ def sparse_attention(Q, K, V, q_labels, k_labels, mask, scale, rows=None):
 
 
 def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", topk_ratio=None,
-                  size_prior=False):
+                  size_prior=False, sip_ratio=None, sip_u=None):
     """PARK retrieval for one (b, h): query K-means (Euclidean), key K-means
     with the query-derived metric (QRKC), PAMA importance, top-p mask
     (PARK Figure 2).  qrkc=False is the "w/o QRKC" ablation (M = I);
     pama_mode="centroid" is "w/o PAMA" (PARK Table 3); topk_ratio selects the
     top-k at that retrieval ratio instead of top-p (PARK Table 10);
-    size_prior adds log |B_m| to the PAMA logits (a variant, see pama)."""
+    size_prior adds log |B_m| to the PAMA logits (a variant, see pama);
+    sip_ratio with the uniforms sip_u [NQ, NK] selects by SIP (see sip_select)
+    and adds the weights to the result."""
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
     d = Q.shape[1]
@@ -342,14 +407,17 @@ def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", to
         I = pama(Q, q_labels, NQ, CK, k_counts, scale, size_prior=size_prior)
     else:
         I = pama_centroid_query(CQ, q_counts, CK, k_counts, scale, size_prior=size_prior)
-    if topk_ratio is None:
+    weight = None
+    if sip_ratio is not None:
+        mask, weight = sip_select(I, sip_ratio, sip_u, q_counts, k_counts)
+    elif topk_ratio is None:
         mask = top_p(I, p, q_counts, k_counts)
     else:
         mask = top_k_ratio(I, topk_ratio, q_counts, k_counts)
     q_perm, q_off = stable_permutation(q_labels, NQ)
     k_perm, k_off = stable_permutation(k_labels, NK)
     return dict(M=M, q_labels=q_labels, k_labels=k_labels, q_centroids=CQ, k_centroids=CK,
-                q_counts=q_counts, k_counts=k_counts, importance=I, mask=mask,
+                q_counts=q_counts, k_counts=k_counts, importance=I, mask=mask, weight=weight,
                 q_perm=q_perm, q_offsets=q_off, k_perm=k_perm, k_offsets=k_off)
 
 
@@ -357,14 +425,16 @@ def layer_head(Q, K, V, NQ, NK, p, iters, dtype, **kw):
     """Retrieval followed by block-sparse attention for one (b, h)."""
     r = retrieve_head(Q, K, NQ, NK, p, iters, dtype, **kw)
     scale = 1.0 / math.sqrt(np.asarray(Q).shape[1])
-    r["O"] = sparse_attention(Q, K, V, r["q_labels"], r["k_labels"], r["mask"], scale)
+    r["O"] = sparse_attention(Q, K, V, r["q_labels"], r["k_labels"], r["mask"], scale, weight=r["weight"])
     return r
 
 
 def layer(Q, K, V, NQ, NK, p, iters, dtype, **kw):
     """All (b, h) of [B, H, N, d] inputs; returns a list (row-major over b, h)."""
     B, H = Q.shape[:2]
-    return [layer_head(Q[b, h], K[b, h], V[b, h], NQ, NK, p, iters, dtype, **kw)
+    u = kw.pop("sip_u", None)  # [B, H, NQ, NK] uniforms for SIP, one slice per head
+    return [layer_head(Q[b, h], K[b, h], V[b, h], NQ, NK, p, iters, dtype,
+                       **kw, **({} if u is None else {"sip_u": np.asarray(u)[b, h]}))
             for b in range(B) for h in range(H)]
 
 

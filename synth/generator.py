@@ -36,7 +36,7 @@ import os
 
 import numpy as np
 
-TENSOR_IDS = {"Q": 0, "K": 1, "V": 2}
+TENSOR_IDS = {"Q": 0, "K": 1, "V": 2, "U": 3}
 FLUSH_BELOW = 2.0 ** -20
 
 
@@ -206,3 +206,15 @@ def gen_integer_blobs(n: int, d: int, k: int, seed: int, spread: int = 2, sep: i
     centers = rng.integers(-3, 4, size=(k, d)) * sep
     lab = rng.integers(0, k, size=n)
     return (centers[lab] + rng.integers(-spread, spread + 1, size=(n, d))).astype(np.float64)
+
+
+def gen_uniform(cfg: LayerConfig, seed: int = 0) -> np.ndarray:
+    """Uniforms on [0, 1) for randomised block selection, float32 [B, H, NQ, NK]
+    (one stream per (b, h), like the tensors).  Values are float32 so that the
+    oracle and the GPU compare against the same numbers."""
+    out = np.empty((cfg.B, cfg.H, cfg.NQ, cfg.NK), dtype=np.float32)
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            rng = np.random.default_rng([seed, TENSOR_IDS["U"], b, h])
+            out[b, h] = rng.random((cfg.NQ, cfg.NK), dtype=np.float32)
+    return out

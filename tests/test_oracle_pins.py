@@ -402,6 +402,66 @@ def test_retrieve_topk_keeps_ceil_ratio_blocks():
             assert r["importance"][q, kept].min() >= r["importance"][q, dropped].max()
 
 
+def test_sip_probabilities_worked_examples():
+    # budget 2 over [0.5, 0.3, 0.1, 0.1]: c = 2, nothing capped (c * 0.5 = 1)
+    assert np.allclose(po.sip_probabilities([0.5, 0.3, 0.1, 0.1], 2), [1.0, 0.6, 0.2, 0.2], rtol=1e-15)
+    # budget 2 over [0.7, 0.1, 0.1, 0.1]: 0.7 is certain, the rest share 1 -> 1/3 each
+    assert np.allclose(po.sip_probabilities([0.7, 0.1, 0.1, 0.1], 2), [1.0, 1 / 3, 1 / 3, 1 / 3], rtol=1e-15)
+    # budget >= count: everything is certain
+    assert np.array_equal(po.sip_probabilities([0.2, 0.8], 2), [1.0, 1.0])
+
+
+def test_sip_probabilities_sum_to_budget_and_are_proportional():
+    rng = np.random.default_rng(14)
+    for _ in range(50):
+        L = int(rng.integers(2, 40))
+        v = rng.random(L) ** 4 + 1e-6
+        B = int(rng.integers(1, L))
+        pi = po.sip_probabilities(v, B)
+        assert abs(pi.sum() - B) < 1e-12 * B
+        assert np.all(pi > 0) and np.all(pi <= 1.0)
+        free = pi < 1.0
+        if free.sum() > 1:
+            ratio = pi[free] / v[free]
+            assert np.allclose(ratio, ratio[0], rtol=1e-12)
+        # certain blocks are the largest ones
+        if (~free).any() and free.any():
+            assert v[~free].min() >= v[free].max()
+
+
+def test_sip_weighting_is_unbiased_by_enumeration():
+    # E over independent draws of sum_{m drawn} X_m / pi_m equals sum_m X_m: enumerate
+    # every inclusion pattern with its probability (a wrong weight, e.g. 1/pi^2, fails)
+    rng = np.random.default_rng(15)
+    v = rng.random(6) + 0.05
+    X = rng.random(6)
+    pi = po.sip_probabilities(v, 3)
+    expect = 0.0
+    for pattern in itertools.product([0, 1], repeat=6):
+        prob = np.prod([p if z else 1 - p for z, p in zip(pattern, pi)])
+        expect += prob * sum(X[m] / pi[m] for m in range(6) if pattern[m])
+    assert abs(expect - X.sum()) < 1e-12
+
+
+def test_sip_select_full_budget_is_dense_and_empty_draw_keeps_best():
+    Q, K, V, ql, CQ, kl, CK = _tiny_case(seed=16)
+    s = 1 / math.sqrt(Q.shape[1])
+    qc, kc = np.bincount(ql, minlength=CQ.shape[0]), np.bincount(kl, minlength=CK.shape[0])
+    I = po.pama(Q, ql, CQ.shape[0], CK, kc, s)
+    u = np.random.default_rng(16).random(I.shape)
+    mask, w = po.sip_select(I, 1.0, u, qc, kc)       # budget = every live block: all certain
+    assert np.array_equal(mask, (qc[:, None] > 0) & (kc[None, :] > 0))
+    assert np.all(w[mask] == 1.0)
+    O = po.sparse_attention(Q, K, V, ql, kl, mask, s, weight=w)
+    assert np.allclose(O, po.dense_attention(Q, K, V, s), rtol=1e-12, atol=1e-12)
+    # uniforms that draw nothing: the most important block is kept alone
+    mask, w = po.sip_select(I, 0.1, np.full(I.shape, 0.999999), qc, kc)
+    for r in np.nonzero(qc)[0]:
+        live = np.nonzero(kc)[0]
+        best = live[np.argmax(I[r, live])]
+        assert mask[r].sum() == 1 and mask[r, best] and w[r, best] >= 1.0
+
+
 def test_key_errors_qk_term_is_metric_distance():
     rng = np.random.default_rng(10)
     Q, K = rng.standard_normal((64, 8)), rng.standard_normal((50, 8))
