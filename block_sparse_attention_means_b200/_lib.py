@@ -24,6 +24,7 @@ PARK_FLAG_NO_QRKC = 0x4
 PARK_FLAG_CENTROID_QUERY = 0x8
 PARK_FLAG_TOPK = 0x10
 PARK_FLAG_SIZE_PRIOR = 0x20
+PARK_FLAG_SIP = 0x40
 
 PARK_CNT_Q_RECHECK = 0
 PARK_CNT_K_RECHECK = 1
@@ -55,7 +56,8 @@ class ParkRetrieval(ctypes.Structure):
                 ("importance", ctypes.c_void_p), ("mask", ctypes.c_void_p),
                 ("kept_ptr", ctypes.c_void_p), ("kept_idx", ctypes.c_void_p),
                 ("metric", ctypes.c_void_p), ("importance_bound", ctypes.c_void_p),
-                ("counters", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+                ("counters", ctypes.c_void_p), ("status", ctypes.c_void_p),
+                ("sip_uniform", ctypes.c_void_p), ("block_weight", ctypes.c_void_p)]
 
 
 class ParkKernelTime(ctypes.Structure):

@@ -53,7 +53,8 @@ __global__ __launch_bounds__(256) void k_attn_schedule(int NQ, int NK, const int
                                                        WorkItem* __restrict__ items, int32_t* __restrict__ item_count,
                                                        int64_t* __restrict__ counters, int tile_rows, int pad8,
                                                        const int32_t* __restrict__ poff, int Npad,
-                                                       int2* __restrict__ segs) {
+                                                       int2* __restrict__ segs, const float* __restrict__ bweight,
+                                                       float* __restrict__ segw) {
     __shared__ int wsum[8], wsum_u[8];
     const int r = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int qs = q_off[(size_t)bh * (NQ + 1) + r], nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - qs;
@@ -90,6 +91,9 @@ __global__ __launch_bounds__(256) void k_attn_schedule(int NQ, int NK, const int
         const int m = kl[e], sz = ko[m + 1] - ko[m];
         pre[e] = run;
         if (segs) segs[(size_t)bh * NQ * NK + kp0 + e] = make_int2(bh * Npad + poff[(size_t)bh * (NK + 1) + m], sz);
+        // additive logit term of the segment (log2 of its SIP weight; 0 without weights)
+        if (segw) segw[(size_t)bh * NQ * NK + kp0 + e] =
+                      bweight ? (float)log2((double)bweight[((size_t)bh * NQ + r) * NK + m]) : 0.f;
         run += padded(sz);
     }
     if (t == 0) {
@@ -120,10 +124,12 @@ __global__ __launch_bounds__(256) void k_attn_schedule(int NQ, int NK, const int
 int launch_attn_schedule(int BH, int NQ, int NK, const int32_t* q_off, const int32_t* k_off,
                          const int32_t* kept_ptr, const int32_t* kept_idx, int32_t* kv_pre, int32_t* kv_len,
                          WorkItem* items, int32_t* item_count, int64_t* counters, int tile_rows, int pad8,
-                         const int32_t* poff, int Npad, int2* segs, cudaStream_t st) {
+                         const int32_t* poff, int Npad, int2* segs, const float* bweight, float* segw,
+                         cudaStream_t st) {
     ::park::prof_begin(st);
     k_attn_schedule<<<dim3(NQ, BH), 256, 0, st>>>(NQ, NK, q_off, k_off, kept_ptr, kept_idx, kv_pre, kv_len, items,
-                                                  item_count, counters, tile_rows, pad8, poff, Npad, segs);
+                                                  item_count, counters, tile_rows, pad8, poff, Npad, segs, bweight,
+                                                  segw);
     PARK_TRY_LAUNCH("k_attn_schedule", st);
     return PARK_OK;
 }
@@ -232,7 +238,7 @@ __global__ void k_sparse_attn_simt(const T* __restrict__ Q, const T* __restrict_
                                    int D, int NQ, int NK, const int32_t* __restrict__ q_labels,
                                    const int32_t* __restrict__ k_perm, const int32_t* __restrict__ k_off,
                                    const int32_t* __restrict__ kept_ptr, const int32_t* __restrict__ kept_idx,
-                                   T* __restrict__ O, size_t rows, float scale) {
+                                   const float* __restrict__ bweight, T* __restrict__ O, size_t rows, float scale) {
     const int lane = threadIdx.x & 31;
     const size_t nw = ((size_t)gridDim.x * blockDim.x) >> 5;
     for (size_t row = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += nw) {
@@ -250,6 +256,7 @@ __global__ void k_sparse_attn_simt(const T* __restrict__ Q, const T* __restrict_
         const int32_t* ko = k_off + bh * (NK + 1);
         for (int e = p0; e < p1; ++e) {
             int mk = kept_idx[bh * NQ * NK + e];
+            const float lw = bweight ? logf(bweight[(bh * NQ + r) * NK + mk]) : 0.f;  // SIP weight, natural log
             for (int pos = ko[mk]; pos < ko[mk + 1]; ++pos) {
                 size_t tok = bh * N + k_perm[bh * N + pos];
                 float sdot = 0.f;
@@ -258,7 +265,7 @@ __global__ void k_sparse_attn_simt(const T* __restrict__ Q, const T* __restrict_
                     int j = lane + 32 * u;
                     if (j < D) sdot = fmaf(q[u], Elem<T>::to_float(K + tok * D, j), sdot);
                 }
-                float sc = warp_sum(sdot) * scale;
+                float sc = warp_sum(sdot) * scale + lw;
                 float mn = fmaxf(m, sc);
                 float corr = expf(m - mn), pw = expf(sc - mn);
                 l = l * corr + pw;
@@ -281,14 +288,16 @@ __global__ void k_sparse_attn_simt(const T* __restrict__ Q, const T* __restrict_
 
 int launch_sparse_attn_simt(const void* Q, const void* K, const void* V, int dtype, int BH, int N, int D, int NQ,
                             int NK, const int32_t* q_labels, const int32_t* k_perm, const int32_t* k_off,
-                            const int32_t* kept_ptr, const int32_t* kept_idx, void* O, cudaStream_t st) {
+                            const int32_t* kept_ptr, const int32_t* kept_idx, const float* bweight, void* O,
+                            cudaStream_t st) {
     if (dtype != PARK_F32 || D > 128) return PARK_ERR_UNSUPPORTED;
     size_t rows = (size_t)BH * N;
     int blocks = (int)((rows * 32 + 255) / 256);
     ::park::prof_begin(st);
     if (blocks > 148 * 64) blocks = 148 * 64;
     k_sparse_attn_simt<float><<<blocks, 256, 0, st>>>((const float*)Q, (const float*)K, (const float*)V, N, D, NQ, NK,
-                                                      q_labels, k_perm, k_off, kept_ptr, kept_idx, (float*)O, rows,
+                                                      q_labels, k_perm, k_off, kept_ptr, kept_idx, bweight, (float*)O,
+                                                      rows,
                                                       1.0f / sqrtf((float)D));
     PARK_TRY_LAUNCH("k_sparse_attn_simt", st);
     return PARK_OK;

@@ -1,5 +1,7 @@
 // Block-sparse attention on the 5th-generation tensor cores (tcgen05 + TMEM +
-// TMA), bf16 inputs, D = 128.
+// TMA), bf16 inputs, D = 128.  With SIP block weights (AB-Attention's inverse
+// inclusion probabilities) the per-column bias of a real key row is log2 of its
+// block's weight instead of 0, which weights both Softmax sums.
 //
 // Layout: Q is gathered into cluster order (rows of a query cluster are
 // contiguous).  K and V are gathered into cluster order with every key
@@ -80,7 +82,8 @@ __device__ __forceinline__ float fast_ex2(float x) {
 __global__ void __launch_bounds__(320, 1)
     k_sparse_attn_tc(const __grid_constant__ CUtensorMap tmQ, const uint8_t* __restrict__ Kimg,
                      const uint8_t* __restrict__ Vimg, int N, int NQ, int NK, const int32_t* __restrict__ q_perm,
-                     const int2* __restrict__ segs, const int32_t* __restrict__ kept_ptr,
+                     const int2* __restrict__ segs, const float* __restrict__ segw,
+                     const int32_t* __restrict__ kept_ptr,
                      const int32_t* __restrict__ kv_pre, const int32_t* __restrict__ kv_len,
                      const WorkItem* __restrict__ items, const int32_t* __restrict__ item_count,
                      uint16_t* __restrict__ O, float sl2e, int32_t* __restrict__ status) {
@@ -142,6 +145,7 @@ __global__ void __launch_bounds__(320, 1)
             const int nk = kept_ptr[(size_t)wi.bh * (NQ + 1) + wi.r + 1] - kp0;
             const int32_t* pre = kv_pre + (size_t)wi.bh * NQ * NK + kp0;
             const int2* segs_item = segs + (size_t)wi.bh * NQ * NK + kp0;
+            const float* segw_item = segw ? segw + (size_t)wi.bh * NQ * NK + kp0 : nullptr;
             if (lane == 0) {
                 bool ok = I == 0 || mbar_wait(&sh.q_empty, (I - 1) & 1, abort);
                 if (ok) {
@@ -159,6 +163,7 @@ __global__ void __launch_bounds__(320, 1)
             // segments (prefix of padded sizes, first padded row, size); a tile
             // spans at most 17 segments (each is >= 8 rows), so 32 lanes cover it.
             int seg0 = 0, p_l = 0x7fffffff, src_l = 0, sz_l = 0;
+            float lw_l = 0.f;  // additive logit term of the segment (log2 of its block weight)
             auto load_entries = [&](int s0) {
                 const int idx = s0 + lane;
                 if (idx < nk) {
@@ -166,17 +171,20 @@ __global__ void __launch_bounds__(320, 1)
                     const int2 e = segs_item[idx];
                     src_l = e.x;
                     sz_l = e.y;
+                    lw_l = segw_item ? segw_item[idx] : 0.f;
                 } else {
                     p_l = 0x7fffffff;
                     src_l = 0;
                     sz_l = 0;
+                    lw_l = 0.f;
                 }
             };
             load_entries(0);
             bool ok = true;
             for (int j = 0; j < nkt && ok; ++j) {
                 const int stg = T & 1, round = T >> 1;
-                int nvalid = 0;  // real key rows of group `lane` (lanes 0..15)
+                int nvalid = 0;   // real key rows of group `lane` (lanes 0..15)
+                float lwv = 0.f;  // and the logit term of its segment
 #pragma unroll 4
                 for (int g = 0; g < 16; ++g) {
                     const int vg = j * TC_ROWS + 8 * g;
@@ -184,9 +192,11 @@ __global__ void __launch_bounds__(320, 1)
                     const int idx = (__popc(bal) - 1) & 31;
                     const int pp = __shfl_sync(0xffffffffu, p_l, idx);
                     const int sz = __shfl_sync(0xffffffffu, sz_l, idx);
+                    const float lw = __shfl_sync(0xffffffffu, lw_l, idx);
                     if (lane == g && vg < L) {
                         int nv = sz - (vg - pp);
                         nvalid = nv < 0 ? 0 : (nv > 8 ? 8 : nv);
+                        lwv = lw;
                     }
                 }
                 // this lane's segment (seg0 + lane) as one piece of whole 8-row groups of the tile
@@ -234,10 +244,10 @@ __global__ void __launch_bounds__(320, 1)
                 if (lane < 16) {
                     float4* bp = reinterpret_cast<float4*>(&sh.bias[stg][8 * lane]);
                     const float NI = __int_as_float(0xff800000);
-                    bp[0] = make_float4(nvalid > 0 ? 0.f : NI, nvalid > 1 ? 0.f : NI, nvalid > 2 ? 0.f : NI,
-                                        nvalid > 3 ? 0.f : NI);
-                    bp[1] = make_float4(nvalid > 4 ? 0.f : NI, nvalid > 5 ? 0.f : NI, nvalid > 6 ? 0.f : NI,
-                                        nvalid > 7 ? 0.f : NI);
+                    bp[0] = make_float4(nvalid > 0 ? lwv : NI, nvalid > 1 ? lwv : NI, nvalid > 2 ? lwv : NI,
+                                        nvalid > 3 ? lwv : NI);
+                    bp[1] = make_float4(nvalid > 4 ? lwv : NI, nvalid > 5 ? lwv : NI, nvalid > 6 ? lwv : NI,
+                                        nvalid > 7 ? lwv : NI);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive_expect_tx(&sh.v_full[stg], tile_bytes);
@@ -506,8 +516,8 @@ int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t
 size_t attn_tc_smem_bytes() { return (size_t)10 * TC_BLK + 1024; }  // Q, K x2, V x2
 
 int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
-                          const int32_t* q_perm, const int2* segs, const int32_t* kept_ptr, const int32_t* kv_pre,
-                          const int32_t* kv_len,
+                          const int32_t* q_perm, const int2* segs, const float* segw, const int32_t* kept_ptr,
+                          const int32_t* kv_pre, const int32_t* kv_len,
                           const WorkItem* items, const int32_t* item_count, void* O, int32_t* status, int num_sms,
                           cudaStream_t st) {
     CUtensorMap mQ;
@@ -517,7 +527,7 @@ int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, in
     const float sl2e = (1.0f / sqrtf(128.f)) * kLog2eT;
     ::park::prof_begin(st);
     k_sparse_attn_tc<<<num_sms, 320, sm, st>>>(mQ, (const uint8_t*)Kpad, (const uint8_t*)Vpad, N, NQ, NK, q_perm,
-                                                segs, kept_ptr, kv_pre, kv_len, items, item_count, (uint16_t*)O,
+                                                segs, segw, kept_ptr, kv_pre, kv_len, items, item_count, (uint16_t*)O,
                                                 sl2e, status);
     PARK_TRY_LAUNCH("k_sparse_attn_tc", st);
     return PARK_OK;

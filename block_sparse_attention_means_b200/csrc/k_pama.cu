@@ -266,23 +266,28 @@ static int next_pow2(int x) {
 // ---------------------------------------------------------------- top-p (certified)
 __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importance, const float* __restrict__ rho,
                                               const int32_t* __restrict__ q_off, const int32_t* __restrict__ k_off,
-                                              int NQ, int NK, int NKP, float p, int topk, uint8_t* __restrict__ mask,
-                                              int32_t* __restrict__ kept_cnt, float* __restrict__ importance_bound,
-                                              int32_t* __restrict__ flag_list, int32_t* __restrict__ flag_count) {
+                                              int NQ, int NK, int NKP, float p, int select,
+                                              const float* __restrict__ sip_u, float* __restrict__ weight,
+                                              uint8_t* __restrict__ mask, int32_t* __restrict__ kept_cnt,
+                                              float* __restrict__ importance_bound, int32_t* __restrict__ flag_list,
+                                              int32_t* __restrict__ flag_count) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     double* S = reinterpret_cast<double*>(smem_raw);       // [NKP] inclusive prefix sums
     float* sv = reinterpret_cast<float*>(S + NKP);         // [NKP]
     int32_t* si = reinterpret_cast<int32_t*>(sv + NKP);    // [NKP]
     uint8_t* keep = reinterpret_cast<uint8_t*>(si + NKP);  // [NKP]
     __shared__ double wsum[16];
-    __shared__ int s_cut, s_live;
+    __shared__ int s_cut, s_live, s_t, s_bad, s_kept;
 
     const int r = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
     const size_t row = (size_t)bh * NQ + r;
     uint8_t* mrow = mask + row * NK;
     const int nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - q_off[(size_t)bh * (NQ + 1) + r];
     if (nr == 0) {
-        for (int m = t; m < NK; m += blockDim.x) mrow[m] = 0;
+        for (int m = t; m < NK; m += blockDim.x) {
+            mrow[m] = 0;
+            if (select == 2) weight[row * NK + m] = 0.f;
+        }
         if (t == 0) {
             kept_cnt[row] = 0;
             if (importance_bound) importance_bound[row] = 0.f;
@@ -294,6 +299,9 @@ __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importan
     if (t == 0) {
         s_cut = -1;
         s_live = 0;
+        s_t = 0x7fffffff;
+        s_bad = 0;
+        s_kept = 0;
     }
     __syncthreads();
     int live_local = 0;
@@ -343,10 +351,61 @@ __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importan
     __syncthreads();
     int cut = s_cut;
     bool ok;
-    if (topk) {  // the ceil(p L) most important; certified when the last kept is clear of the next
+    const double rh = (double)rho[row];
+    if (select == 2) {
+        // SIP: pi_e = 1 for the first tc sorted blocks, c sv[e] after them, with
+        // sum pi = Bd; tc = first e with (Bd - e) sv[e] <= tail[e] (tail[e] = sum of
+        // sv[e..L-1]).  Every decision is certified against the relative bound rh of
+        // the float importances (a tail sum carries at most rh, c at most 2 rh), else
+        // the whole row goes to float64.
+        const int Bd = max(1, (int)ceil((double)p * (double)L));
+        const double total = S[L - 1];
+        auto tail = [&](int e) { return total - (e > 0 ? S[e - 1] : 0.0); };
+        if (Bd < L)
+            for (int e = t; e < L; e += blockDim.x)
+                if ((double)(Bd - e) * (double)sv[e] <= tail(e)) atomicMin(&s_t, e);
+        for (int m = t; m < NK; m += blockDim.x) weight[row * NK + m] = 0.f;
+        __syncthreads();
+        const int tc = Bd >= L ? L : s_t;
+        double c = 0.0;
+        if (tc < L) {
+            c = (double)(Bd - tc) / tail(tc);
+            if (t == 0) {
+                bool b = !((double)(Bd - tc) * (double)sv[tc] * (1.0 + rh) < tail(tc) * (1.0 - rh));
+                if (tc > 0) {
+                    b |= !((double)(Bd - tc + 1) * (double)sv[tc - 1] * (1.0 - rh) > tail(tc - 1) * (1.0 + rh));
+                    b |= !((double)sv[tc - 1] * (1.0 - rh) > (double)sv[tc] * (1.0 + 2.0 * rh));
+                }
+                if (b) s_bad = 1;
+            }
+        }
+        int kept_local = 0;
+        for (int e = t; e < L; e += blockDim.x) {
+            const double pi = e < tc ? 1.0 : c * (double)sv[e];
+            const int m = si[e];
+            const double u = (double)sip_u[row * NK + m];
+            if (e >= tc && fabs(u - pi) <= 4.0 * rh * pi + 1e-12) s_bad = 1;
+            if (u < pi) {
+                keep[m] = 1;
+                weight[row * NK + m] = (float)(1.0 / pi);
+                ++kept_local;
+            }
+        }
+        atomicAdd(&s_kept, kept_local);
+        __syncthreads();
+        if (t == 0 && s_kept == 0) {  // nothing drawn: the most important block
+            if (L > 1 && !((double)sv[0] * (1.0 - rh) > (double)sv[1] * (1.0 + 2.0 * rh))) s_bad = 1;
+            const double pi0 = 0 < tc ? 1.0 : c * (double)sv[0];
+            keep[si[0]] = 1;
+            weight[row * NK + si[0]] = (float)(1.0 / pi0);
+            s_kept = 1;
+        }
+        __syncthreads();
+        ok = s_bad == 0;
+        cut = s_kept - 1;
+    } else if (select == 1) {  // the ceil(p L) most important; certified when the last kept is clear of the next
         const int kk = max(1, (int)ceil((double)p * (double)L));
         cut = min(kk, L) - 1;
-        const double rh = (double)rho[row];
         ok = cut + 1 >= L || (double)sv[cut] * (1.0 - rh) > (double)sv[cut + 1] * (1.0 + 2.0 * rh) + 1e-300;
     } else if (p >= 1.0f) {
         cut = L - 1;
@@ -354,7 +413,6 @@ __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importan
     } else if (cut < 0) {
         ok = false;  // float sums fell short of p: let float64 decide
     } else {
-        const double rh = (double)rho[row];
         const double vc = (double)sv[cut];
         const double eps = 1e-12;
         bool ord = cut + 1 >= L || vc * (1.0 - rh) > (double)sv[cut + 1] * (1.0 + 2.0 * rh) + 1e-300;
@@ -369,7 +427,8 @@ __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importan
         }
         return;
     }
-    for (int e = t; e <= cut; e += blockDim.x) keep[si[e]] = 1;
+    if (select != 2)
+        for (int e = t; e <= cut; e += blockDim.x) keep[si[e]] = 1;
     __syncthreads();
     for (int m = t; m < NK; m += blockDim.x) mrow[m] = keep[m];
     if (t == 0) {
@@ -379,14 +438,16 @@ __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importan
 }
 
 int launch_topp(const float* importance, const float* rho, int BH, int NQ, int NK, const int32_t* q_off,
-                const int32_t* k_off, float p, int topk, uint8_t* mask, int32_t* kept_cnt, float* importance_bound,
-                int32_t* flag_list, int32_t* flag_count, cudaStream_t st) {
+                const int32_t* k_off, float p, int select, const float* sip_u, float* weight, uint8_t* mask,
+                int32_t* kept_cnt, float* importance_bound, int32_t* flag_list, int32_t* flag_count,
+                cudaStream_t st) {
     int NKP = next_pow2(NK);
     if (NKP < 512) NKP = 512;
     size_t sm = (size_t)NKP * (8 + 4 + 4 + 1) + 16;
     cudaFuncSetAttribute(k_topp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     ::park::prof_begin(st);
-    k_topp<<<dim3(NQ, BH), 512, sm, st>>>(importance, rho, q_off, k_off, NQ, NK, NKP, p, topk, mask, kept_cnt,
+    k_topp<<<dim3(NQ, BH), 512, sm, st>>>(importance, rho, q_off, k_off, NQ, NK, NKP, p, select, sip_u, weight,
+                                          mask, kept_cnt,
                                           importance_bound, flag_list, flag_count);
     PARK_TRY_LAUNCH("k_topp", st);
     return PARK_OK;
@@ -414,7 +475,8 @@ template <typename T, int RPT>
 __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, const int32_t* __restrict__ q_perm,
                                                      const int32_t* __restrict__ q_off, const T* __restrict__ CK,
                                                      const int32_t* __restrict__ k_off, int N, int D, int NQ, int NK,
-                                                     int NKP, double scale, float p, int topk, int size_prior,
+                                                     int NKP, double scale, float p, int select, int size_prior,
+                                                     const float* __restrict__ sip_u, float* __restrict__ weight,
                                                      const int32_t* __restrict__ list,
                                                      const int32_t* __restrict__ count_ptr, int all_clusters,
                                                      int BHNQ, int32_t* __restrict__ work_ctr,
@@ -431,7 +493,8 @@ __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, co
     double* lsz = part + 16 * F64_CH;                          // [NKP] additive logit term per column
     int32_t* si = reinterpret_cast<int32_t*>(lsz + NKP);       // [NKP]
     uint8_t* live = reinterpret_cast<uint8_t*>(si + NKP);      // [NKP]
-    __shared__ int s_cut, s_e;
+    __shared__ int s_cut, s_e, s_tc, s_kept;
+    __shared__ double s_c;
     const double NEG_INF = __longlong_as_double(0xfff0000000000000ll);
     const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
     const int count = all_clusters ? BHNQ : *count_ptr;
@@ -457,6 +520,7 @@ __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, co
             for (int m = t; m < NK; m += blockDim.x) {
                 mrow[m] = 0;
                 Irow[m] = 0.f;
+                if (select == 2) weight[(size_t)row * NK + m] = 0.f;
             }
             if (t == 0) {
                 kept_cnt[row] = 0;
@@ -608,10 +672,64 @@ __global__ __launch_bounds__(256, 1) void k_pama_f64(const T* __restrict__ Q, co
         }
         __syncthreads();
         bitonic_desc<double>(Isum, si, NKP);
+        if (select == 2) {
+            // SIP in float64, as the definition reads: tail sums from the smallest up,
+            // the first sorted position whose (Bd - t) v_t fits under its tail, then
+            // one draw per block against the caller's uniform
+            double* tail = lsz;  // free after the GEMM passes
+            if (t == 0) {
+                int L = 0;
+                while (L < NKP && Isum[L] >= 0.0) ++L;
+                const int Bd = max(1, (int)ceil((double)p * (double)L));
+                int tc = L;
+                double c = 0.0;
+                if (Bd < L) {
+                    tail[L - 1] = Isum[L - 1];
+                    for (int e = L - 2; e >= 0; --e) tail[e] = tail[e + 1] + Isum[e];
+                    tc = 0;
+                    while ((double)(Bd - tc) * Isum[tc] > tail[tc]) ++tc;
+                    c = (double)(Bd - tc) / tail[tc];
+                }
+                s_cut = L;
+                s_tc = tc;
+                s_c = c;
+                s_kept = 0;
+                if (importance_bound) importance_bound[row] = 0.f;
+            }
+            for (int m = t; m < NK; m += blockDim.x) {
+                mrow[m] = 0;
+                weight[(size_t)row * NK + m] = 0.f;
+            }
+            __syncthreads();
+            const int L = s_cut, tc = s_tc;
+            const double c = s_c;
+            int kept_local = 0;
+            for (int e = t; e < L; e += blockDim.x) {
+                const double pi = e < tc ? 1.0 : c * Isum[e];
+                const int m = si[e];
+                if ((double)sip_u[(size_t)row * NK + m] < pi) {
+                    mrow[m] = 1;
+                    weight[(size_t)row * NK + m] = (float)(1.0 / pi);
+                    ++kept_local;
+                }
+            }
+            atomicAdd(&s_kept, kept_local);
+            __syncthreads();
+            if (t == 0) {
+                if (s_kept == 0) {  // nothing drawn: the most important block
+                    const double pi0 = 0 < tc ? 1.0 : c * Isum[0];
+                    mrow[si[0]] = 1;
+                    weight[(size_t)row * NK + si[0]] = (float)(1.0 / pi0);
+                    s_kept = 1;
+                }
+                kept_cnt[row] = s_kept;
+            }
+            continue;
+        }
         if (t == 0) {
             double run = 0.0;
             int cut = -1;
-            if (topk) {  // the ceil(p L) most important of the L non-empty key clusters
+            if (select == 1) {  // the ceil(p L) most important of the L non-empty key clusters
                 int L = 0;
                 while (L < NKP && Isum[L] >= 0.0) ++L;
                 cut = L > 0 ? min(max(1, (int)ceil((double)p * (double)L)), L) - 1 : -1;
@@ -641,19 +759,21 @@ size_t pama_f64_scratch_bytes(int NK) {
 template <typename T, int RPT>
 static void pama_f64_launch(const void* Q, const int32_t* q_perm, const int32_t* q_off, const void* CK,
                             const int32_t* k_off, int N, int D, int NQ, int NK, int NKP, double scale, float p,
-                            int topk, int size_prior, const int32_t* list, const int32_t* count, int all_clusters, int BHNQ, int32_t* work_ctr,
+                            int select, int size_prior, const float* sip_u, float* weight, const int32_t* list,
+                            const int32_t* count, int all_clusters, int BHNQ, int32_t* work_ctr,
                             double* zscratch, float* importance, float* importance_bound, uint8_t* mask,
                             int32_t* kept_cnt, int64_t* counters, size_t sm, int blocks, cudaStream_t st) {
     cudaFuncSetAttribute(k_pama_f64<T, RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     k_pama_f64<T, RPT><<<blocks, 256, sm, st>>>((const T*)Q, q_perm, q_off, (const T*)CK, k_off, N, D, NQ, NK, NKP,
-                                                scale, p, topk, size_prior, list, count, all_clusters, BHNQ,
+                                                scale, p, select, size_prior, sip_u, weight, list, count,
+                                                all_clusters, BHNQ,
                                                 work_ctr, zscratch,
                                                 importance, importance_bound, mask, kept_cnt, counters);
 }
 
 int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int NK, const int32_t* q_perm,
-                    const int32_t* q_off, const void* CK, const int32_t* k_off, float p, int topk, int size_prior,
-                    const int32_t* list,
+                    const int32_t* q_off, const void* CK, const int32_t* k_off, float p, int select, int size_prior,
+                    const float* sip_u, float* weight, const int32_t* list,
                     const int32_t* count, int all_clusters, int num_sms, int32_t* work_ctr, double* zscratch,
                     float* importance, float* importance_bound, uint8_t* mask, int32_t* kept_cnt, int64_t* counters,
                     cudaStream_t st) {
@@ -670,20 +790,20 @@ int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int 
     ::park::prof_begin(st);
     if (dtype == PARK_BF16) {
         if (big)
-            pama_f64_launch<bf16_t, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, topk, size_prior, list, count,
+            pama_f64_launch<bf16_t, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, select, size_prior, sip_u, weight, list, count,
                                        all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
                                        kept_cnt, counters, sm, blocks, st);
         else
-            pama_f64_launch<bf16_t, 4>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, topk, size_prior, list, count,
+            pama_f64_launch<bf16_t, 4>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, select, size_prior, sip_u, weight, list, count,
                                        all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
                                        kept_cnt, counters, sm, blocks, st);
     } else {
         if (big)
-            pama_f64_launch<float, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, topk, size_prior, list, count,
+            pama_f64_launch<float, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, select, size_prior, sip_u, weight, list, count,
                                       all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
                                       kept_cnt, counters, sm, blocks, st);
         else
-            pama_f64_launch<float, 4>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, topk, size_prior, list, count,
+            pama_f64_launch<float, 4>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, select, size_prior, sip_u, weight, list, count,
                                       all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,
                                       kept_cnt, counters, sm, blocks, st);
     }

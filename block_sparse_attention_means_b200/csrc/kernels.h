@@ -53,13 +53,16 @@ int launch_update(const void* X, int dtype, int BH, int N, int D, int K, const i
                   const int32_t* offsets, void* C, cudaStream_t st);
 
 // ---- k_pama.cu
-// size_prior: logits gain log |B_m|; topk: keep the ceil(p L) most important (p a ratio)
+// size_prior: logits gain log |B_m|.  select: 0 top-p; 1 top-k, the ceil(p L) most
+// important (p a ratio); 2 SIP with the uniforms sip_u, writing weight = 1/pi for
+// kept blocks and 0 elsewhere.
 int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t* q_perm, const int32_t* q_off,
                     const void* CK, const int32_t* k_off, const float* qnorm, int size_prior, float* importance,
                     float* rho, float* ckmax, cudaStream_t st);
 int launch_topp(const float* importance, const float* rho, int BH, int NQ, int NK, const int32_t* q_off,
-                const int32_t* k_off, float p, int topk, uint8_t* mask, int32_t* kept_cnt, float* importance_bound,
-                int32_t* flag_list, int32_t* flag_count, cudaStream_t st);
+                const int32_t* k_off, float p, int select, const float* sip_u, float* weight, uint8_t* mask,
+                int32_t* kept_cnt, float* importance_bound, int32_t* flag_list, int32_t* flag_count,
+                cudaStream_t st);
 // one row per non-empty query cluster (its centroid), for "w/o PAMA" through launch_pama_f64
 int launch_centroid_rows(const int32_t* q_off, int BH, int NQ, int32_t* perm, int32_t* off, cudaStream_t st);
 // Float64 PAMA + top-p for the listed clusters (or all): at most kPamaF64Slots
@@ -68,8 +71,8 @@ int launch_centroid_rows(const int32_t* q_off, int BH, int NQ, int32_t* perm, in
 constexpr int kPamaF64Slots = 160;
 size_t pama_f64_scratch_bytes(int NK);
 int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int NK, const int32_t* q_perm,
-                    const int32_t* q_off, const void* CK, const int32_t* k_off, float p, int topk, int size_prior,
-                    const int32_t* list,
+                    const int32_t* q_off, const void* CK, const int32_t* k_off, float p, int select, int size_prior,
+                    const float* sip_u, float* weight, const int32_t* list,
                     const int32_t* count, int all_clusters, int num_sms, int32_t* work_ctr, double* zscratch,
                     float* importance, float* importance_bound, uint8_t* mask, int32_t* kept_cnt, int64_t* counters,
                     cudaStream_t st);
@@ -88,7 +91,8 @@ int launch_gather(const void* X, int dtype, int BH, int N, int D, const int32_t*
 int launch_attn_schedule(int BH, int NQ, int NK, const int32_t* q_off, const int32_t* k_off,
                          const int32_t* kept_ptr, const int32_t* kept_idx, int32_t* kv_pre, int32_t* kv_len,
                          WorkItem* items, int32_t* item_count, int64_t* counters, int tile_rows, int pad8,
-                         const int32_t* poff, int Npad, int2* segs, cudaStream_t st);
+                         const int32_t* poff, int Npad, int2* segs, const float* bweight, float* segw,
+                         cudaStream_t st);
 // K and V in key-cluster order with every cluster padded to a multiple of 8
 // rows (zeros): poff[bh][m] = first padded row of cluster m; Npad rows per head.
 int launch_kv_pad_gather(const void* K, const void* V, int BH, int N, int NK, int Npad, const int32_t* k_perm,
@@ -99,12 +103,13 @@ size_t attn_tc_smem_bytes();
 // box_rows, 128-byte swizzle (k_attn_tc.cu).
 int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t cols, uint32_t box_rows);
 int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
-                          const int32_t* q_perm, const int2* segs, const int32_t* kept_ptr, const int32_t* kv_pre,
-                          const int32_t* kv_len,
+                          const int32_t* q_perm, const int2* segs, const float* segw, const int32_t* kept_ptr,
+                          const int32_t* kv_pre, const int32_t* kv_len,
                           const WorkItem* items, const int32_t* item_count, void* O, int32_t* status, int num_sms,
                           cudaStream_t st);
 int launch_sparse_attn_simt(const void* Q, const void* K, const void* V, int dtype, int BH, int N, int D, int NQ,
                             int NK, const int32_t* q_labels, const int32_t* k_perm, const int32_t* k_off,
-                            const int32_t* kept_ptr, const int32_t* kept_idx, void* O, cudaStream_t st);
+                            const int32_t* kept_ptr, const int32_t* kept_idx, const float* bweight, void* O,
+                            cudaStream_t st);
 
 }  // namespace park

@@ -151,7 +151,7 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
 }
 
 struct AttnWs {
-    size_t Qp, Kp, Vp, poff, segs, items, icnt, kvpre, kvlen, total;
+    size_t Qp, Kp, Vp, poff, segs, segw, items, icnt, kvpre, kvlen, total;
     int Npad;
 };
 
@@ -171,8 +171,9 @@ AttnWs plan_attn(const Dims& d, int NQ, int NK) {
         w.Vp = c.take(BH * (size_t)w.Npad * rowbytes);
         w.poff = c.take(BH * (size_t)(NK + 1) * 4);
         w.segs = c.take(BH * (size_t)NQ * NK * 8);
+        w.segw = c.take(BH * (size_t)NQ * NK * 4);
     } else {
-        w.Qp = w.Kp = w.Vp = w.poff = w.segs = 0;
+        w.Qp = w.Kp = w.Vp = w.poff = w.segs = w.segw = 0;
     }
     size_t max_items = BH * ((N + kAttnTile - 1) / kAttnTile + (size_t)NQ);
     w.items = c.take(max_items * sizeof(WorkItem));
@@ -286,11 +287,14 @@ size_t ws_bytes_for(const Dims& d, int NQ, int NK) {
 }
 
 // Known flag bits only; with PARK_FLAG_TOPK, p is a ratio in (0, 1].
-bool flags_ok(uint32_t flags, float p) {
+bool flags_ok(const park_retrieval* r, float p) {
+    const uint32_t flags = r->flags;
     const uint32_t known = PARK_FLAG_WARM_START_Q | PARK_FLAG_WARM_START_K | PARK_FLAG_NO_QRKC |
-                           PARK_FLAG_CENTROID_QUERY | PARK_FLAG_TOPK | PARK_FLAG_SIZE_PRIOR;
+                           PARK_FLAG_CENTROID_QUERY | PARK_FLAG_TOPK | PARK_FLAG_SIZE_PRIOR | PARK_FLAG_SIP;
     if (flags & ~known) return false;
-    return !(flags & PARK_FLAG_TOPK) || p <= 1.0f;
+    if ((flags & (PARK_FLAG_TOPK | PARK_FLAG_SIP)) && p > 1.0f) return false;
+    if ((flags & PARK_FLAG_TOPK) && (flags & PARK_FLAG_SIP)) return false;
+    return !(flags & PARK_FLAG_SIP) || (r->sip_uniform && r->block_weight);
 }
 
 int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, float p, int iters,
@@ -306,7 +310,10 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
     PARK_CHECK(launch_input_check(K, nel, d.dtype, out->status, st));
     const uint32_t fl = out->flags;
     const bool qrkc = (fl & PARK_FLAG_NO_QRKC) == 0;
-    const int topk = (fl & PARK_FLAG_TOPK) != 0, size_prior = (fl & PARK_FLAG_SIZE_PRIOR) != 0;
+    const int select = (fl & PARK_FLAG_SIP) ? 2 : ((fl & PARK_FLAG_TOPK) ? 1 : 0);
+    const int size_prior = (fl & PARK_FLAG_SIZE_PRIOR) != 0;
+    const float* sip_u = select == 2 ? out->sip_uniform : nullptr;
+    float* bw = select == 2 ? out->block_weight : nullptr;
     double* M = at<double>(ws, w.M);
     if (qrkc || out->metric)
         PARK_CHECK(launch_metric(Q, d.dtype, BH, N, D, at<double>(ws, w.Mpart), metric_chunks(d), M, out->metric, st));
@@ -327,7 +334,7 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
         int32_t* coff = at<int32_t>(ws, w.coff);
         PARK_CHECK(launch_centroid_rows(out->q_offsets, BH, NQ, cperm, coff, st));
         PARK_CHECK(launch_pama_f64(out->q_centroids, d.dtype, BH, NQ, D, NQ, NK, cperm, coff, out->k_centroids,
-                                   out->k_offsets, p, topk, size_prior, nullptr, nullptr, 1, num_sms,
+                                   out->k_offsets, p, select, size_prior, sip_u, bw, nullptr, nullptr, 1, num_sms,
                                    at<int32_t>(ws, w.pcnt) + 4, at<double>(ws, w.f64z), out->importance,
                                    out->importance_bound, out->mask, kcnt, out->counters, st));
     } else if (d.dtype == PARK_BF16) {
@@ -341,16 +348,16 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
                                    at<float>(ws, w.xnorm_q), size_prior, out->importance, at<float>(ws, w.rho),
                                    ops.wmax, st));
         PARK_CHECK(launch_topp(out->importance, at<float>(ws, w.rho), BH, NQ, NK, out->q_offsets, out->k_offsets, p,
-                               topk, out->mask, kcnt, out->importance_bound, at<int32_t>(ws, w.plist),
+                               select, sip_u, bw, out->mask, kcnt, out->importance_bound, at<int32_t>(ws, w.plist),
                                at<int32_t>(ws, w.pcnt), st));
         PARK_CHECK(launch_pama_f64(Q, d.dtype, BH, N, D, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids,
-                                   out->k_offsets, p, topk, size_prior, at<int32_t>(ws, w.plist),
+                                   out->k_offsets, p, select, size_prior, sip_u, bw, at<int32_t>(ws, w.plist),
                                    at<int32_t>(ws, w.pcnt), 0, num_sms,
                                    at<int32_t>(ws, w.pcnt) + 4, at<double>(ws, w.f64z), out->importance,
                                    out->importance_bound, out->mask, kcnt, out->counters, st));
     } else {
         PARK_CHECK(launch_pama_f64(Q, d.dtype, BH, N, D, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids,
-                                   out->k_offsets, p, topk, size_prior, nullptr, nullptr, 1, num_sms,
+                                   out->k_offsets, p, select, size_prior, sip_u, bw, nullptr, nullptr, 1, num_sms,
                                    at<int32_t>(ws, w.pcnt) + 4,
                                    at<double>(ws, w.f64z), out->importance, out->importance_bound, out->mask, kcnt,
                                    out->counters, st));
@@ -368,12 +375,13 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
     PARK_CHECK(memset_async(r->counters + PARK_CNT_KEPT_PAIRS, 3 * sizeof(int64_t), st));
     int32_t* icnt = at<int32_t>(ws, w.icnt);
     PARK_CHECK(memset_async(icnt, 16 * 4, st));
+    const float* bw = (r->flags & PARK_FLAG_SIP) ? r->block_weight : nullptr;  // SIP weights
     if (!bf16) {
         PARK_CHECK(launch_attn_schedule(BH, NQ, NK, r->q_offsets, r->k_offsets, r->kept_ptr, r->kept_idx,
                                         at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
-                                        icnt, r->counters, kAttnTile, 0, nullptr, 0, nullptr, st));
+                                        icnt, r->counters, kAttnTile, 0, nullptr, 0, nullptr, nullptr, nullptr, st));
         return launch_sparse_attn_simt(Q, K, V, d.dtype, BH, N, D, NQ, NK, r->q_labels, r->k_perm, r->k_offsets,
-                                       r->kept_ptr, r->kept_idx, O, st);
+                                       r->kept_ptr, r->kept_idx, bw, O, st);
     }
     const int num_sms = num_sms_current();
     void* Qp = at<void>(ws, w.Qp);
@@ -381,12 +389,14 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
     void* Vp = at<void>(ws, w.Vp);
     int32_t* poff = at<int32_t>(ws, w.poff);
     int2* segs = at<int2>(ws, w.segs);
+    float* segw = at<float>(ws, w.segw);
     PARK_CHECK(launch_gather(Q, d.dtype, BH, N, D, r->q_perm, Qp, st));
     PARK_CHECK(launch_kv_pad_gather(K, V, BH, N, NK, w.Npad, r->k_perm, r->k_labels, r->k_offsets, poff, Kp, Vp, st));
     PARK_CHECK(launch_attn_schedule(BH, NQ, NK, r->q_offsets, r->k_offsets, r->kept_ptr, r->kept_idx,
                                     at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
-                                    icnt, r->counters, kAttnTileTc, 1, poff, w.Npad, segs, st));
-    PARK_CHECK(launch_sparse_attn_tc(Qp, Kp, Vp, BH, N, w.Npad, NQ, NK, r->q_perm, segs, r->kept_ptr,
+                                    icnt, r->counters, kAttnTileTc, 1, poff, w.Npad, segs, bw, segw, st));
+    PARK_CHECK(launch_sparse_attn_tc(Qp, Kp, Vp, BH, N, w.Npad, NQ, NK, r->q_perm, segs, bw ? segw : nullptr,
+                                     r->kept_ptr,
                                      at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
                                      icnt, O, r->status, num_sms, st));
     return PARK_OK;
@@ -413,7 +423,7 @@ int park_retrieve(const void* Q, const void* K, const park_shape* shape, int NQ,
     PARK_CHECK(check_shape(shape, NQ, NK, &d));
     if (!Q || !K || !ws || !retrieval_ptrs_ok(out)) return PARK_ERR_INVALID_ARG;
     if (!(p > 0.0f) || !std::isfinite(p) || iters < 1) return PARK_ERR_INVALID_ARG;
-    if (!flags_ok(out->flags, p)) return PARK_ERR_INVALID_ARG;
+    if (!flags_ok(out, p)) return PARK_ERR_INVALID_ARG;
     if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
     return retrieve_impl(Q, K, d, NQ, NK, p, iters, out, ws, static_cast<cudaStream_t>(stream));
 }
@@ -423,6 +433,7 @@ int park_sparse_attn(const void* Q, const void* K, const void* V, const park_sha
     Dims d;
     PARK_CHECK(check_shape(shape, NQ, NK, &d));
     if (!Q || !K || !V || !O || !ws || !retrieval_ptrs_ok(r)) return PARK_ERR_INVALID_ARG;
+    if ((r->flags & PARK_FLAG_SIP) && !r->block_weight) return PARK_ERR_INVALID_ARG;
     if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
     return attn_impl(Q, K, V, d, NQ, NK, r, O, ws, static_cast<cudaStream_t>(stream));
 }
@@ -433,7 +444,7 @@ int park_layer(const void* Q, const void* K, const void* V, const park_shape* sh
     PARK_CHECK(check_shape(shape, NQ, NK, &d));
     if (!Q || !K || !V || !O || !ws || !retrieval_ptrs_ok(out)) return PARK_ERR_INVALID_ARG;
     if (!(p > 0.0f) || !std::isfinite(p) || iters < 1) return PARK_ERR_INVALID_ARG;
-    if (!flags_ok(out->flags, p)) return PARK_ERR_INVALID_ARG;
+    if (!flags_ok(out, p)) return PARK_ERR_INVALID_ARG;
     if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     PARK_CHECK(retrieve_impl(Q, K, d, NQ, NK, p, iters, out, ws, st));

@@ -64,22 +64,35 @@ class Retrieval:
     counters: torch.Tensor
     status: torch.Tensor
     flags: int = 0
+    sip_uniform: torch.Tensor | None = None   # float32 [B,H,NQ,NK], input with PARK_FLAG_SIP
+    block_weight: torch.Tensor | None = None  # float32 [B,H,NQ,NK], output with PARK_FLAG_SIP
 
     def c(self) -> _lib.ParkRetrieval:
         p = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)  # noqa: E731
         return _lib.ParkRetrieval(self.flags, p(self.q_labels), p(self.k_labels), p(self.q_perm), p(self.k_perm),
                                   p(self.q_offsets), p(self.k_offsets), p(self.q_centroids), p(self.k_centroids),
                                   p(self.importance), p(self.mask), p(self.kept_ptr), p(self.kept_idx),
-                                  p(self.metric), p(self.importance_bound), p(self.counters), p(self.status))
+                                  p(self.metric), p(self.importance_bound), p(self.counters), p(self.status),
+                                  p(self.sip_uniform), p(self.block_weight))
 
     def status_code(self) -> int:
         return int(self.status.item())
 
 
-def alloc_retrieval(shape: Shape, NQ: int, NK: int, device, with_metric: bool = False) -> Retrieval:
+def alloc_retrieval(shape: Shape, NQ: int, NK: int, device, with_metric: bool = False,
+                    sip_uniform: torch.Tensor | None = None) -> Retrieval:
+    """Outputs of park_retrieve on `device`.  With sip_uniform (float32
+    [B,H,NQ,NK] uniforms on the device) the result is set up for PARK_FLAG_SIP:
+    the flag is set and block_weight is allocated."""
     B, H, N, D = shape.B, shape.H, shape.N, shape.D
     i32 = dict(dtype=torch.int32, device=device)
-    return Retrieval(
+    sip = {}
+    if sip_uniform is not None:
+        if tuple(sip_uniform.shape) != (B, H, NQ, NK) or sip_uniform.dtype != torch.float32:
+            raise ValueError("sip_uniform must be float32 [B, H, NQ, NK]")
+        sip = dict(flags=_lib.PARK_FLAG_SIP, sip_uniform=sip_uniform.contiguous(),
+                   block_weight=torch.empty(B, H, NQ, NK, dtype=torch.float32, device=device))
+    return Retrieval(**sip,
         q_labels=torch.empty(B, H, N, **i32), k_labels=torch.empty(B, H, N, **i32),
         q_perm=torch.empty(B, H, N, **i32), k_perm=torch.empty(B, H, N, **i32),
         q_offsets=torch.empty(B, H, NQ + 1, **i32), k_offsets=torch.empty(B, H, NK + 1, **i32),

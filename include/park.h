@@ -87,11 +87,21 @@ extern "C" {
  *                    lower m; at least one), p read as the retrieval ratio in
  *                    (0, 1] (the float32 value passed).
  *   SIZE_PRIOR       PAMA logits gain log |B_m|: P_im proportional to
- *                    |B_m| exp(s q_i . c_m). */
+ *                    |B_m| exp(s q_i . c_m).
+ *   SIP              sampling with inclusion-probability weighting ("AB-Attention
+ *                    Brings More Accurate Sparse Attention to Video Diffusion",
+ *                    SIP paragraph), p read as a ratio in (0, 1]: per non-empty
+ *                    query cluster, pi_m = min(1, c I_rm) with sum_m pi_m =
+ *                    ceil(p L_r) (the largest blocks become certain first); block
+ *                    m is kept when sip_uniform[r][m] < pi_m, with weight 1 / pi_m
+ *                    in both Softmax sums of the attention; if none is drawn the
+ *                    most important block is kept.  Needs sip_uniform and
+ *                    block_weight; not combinable with TOPK. */
 #define PARK_FLAG_NO_QRKC 0x4u
 #define PARK_FLAG_CENTROID_QUERY 0x8u
 #define PARK_FLAG_TOPK 0x10u
 #define PARK_FLAG_SIZE_PRIOR 0x20u
+#define PARK_FLAG_SIP 0x40u
 
 /* ---- park_retrieval.counters indices (outputs, int64) ------------------ */
 #define PARK_CNT_Q_RECHECK 0    /* query rows whose bf16 score margin was not
@@ -139,6 +149,9 @@ typedef struct {
                               computed in float64                              */
     int64_t *counters;     /* [PARK_NUM_COUNTERS], zeroed by park_retrieve        */
     int32_t *status;       /* [1] device status word, zeroed by park_retrieve     */
+    const float *sip_uniform; /* [B,H,NQ,NK] in, with PARK_FLAG_SIP: uniforms on [0,1) */
+    float *block_weight;   /* [B,H,NQ,NK] out, with PARK_FLAG_SIP: 1/pi_m for kept
+                              blocks, 0 elsewhere; read by park_sparse_attn     */
 } park_retrieval;
 
 /* Bytes of device workspace that park_retrieve, park_sparse_attn and

@@ -29,15 +29,15 @@ def test_library_exports_every_declared_function():
 
 
 def test_struct_layout_matches_header():
-    # park_shape: 8 ints; park_retrieval: uint32 flags + 16 pointers (padded)
+    # park_shape: 8 ints; park_retrieval: uint32 flags + 18 pointers (padded)
     assert ctypes.sizeof(_lib.ParkShape) == 32
-    assert ctypes.sizeof(_lib.ParkRetrieval) == 8 + 16 * 8
+    assert ctypes.sizeof(_lib.ParkRetrieval) == 8 + 18 * 8
     text = open(os.path.join(ROOT, "include", "park.h")).read()
     assert re.search(r"#define PARK_NUM_COUNTERS 8", text)
     for name in ("PARK_OK", "PARK_ERR_INVALID_ARG", "PARK_ERR_UNSUPPORTED", "PARK_ERR_WORKSPACE", "PARK_ERR_CUDA",
                  "PARK_ERR_RANGE", "PARK_ERR_TIMEOUT", "PARK_BF16", "PARK_F32", "PARK_FLAG_WARM_START_Q",
                  "PARK_FLAG_WARM_START_K", "PARK_FLAG_NO_QRKC", "PARK_FLAG_CENTROID_QUERY", "PARK_FLAG_TOPK",
-                 "PARK_FLAG_SIZE_PRIOR", "PARK_CNT_KEPT_PAIRS"):
+                 "PARK_FLAG_SIZE_PRIOR", "PARK_FLAG_SIP", "PARK_CNT_KEPT_PAIRS"):
         m = re.search(rf"#define {name} (\w+)", text)
         assert m and int(m.group(1).rstrip("u"), 0) == getattr(_lib, name), name
 
@@ -106,12 +106,22 @@ def test_host_argument_errors_enqueue_nothing():
     cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.9, 10, ctypes.byref(r2), fake, need,
                                     None), _lib.PARK_ERR_INVALID_ARG))
     r3 = _fake_retrieval()
-    r3.flags = 0x40                               # unknown flag bit
+    r3.flags = 0x80                               # unknown flag bit
     cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.9, 10, ctypes.byref(r3), fake, need,
                                     None), _lib.PARK_ERR_INVALID_ARG))
     r4 = _fake_retrieval()
     r4.flags = _lib.PARK_FLAG_TOPK                # a top-k ratio above 1
     cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 1.5, 10, ctypes.byref(r4), fake, need,
+                                    None), _lib.PARK_ERR_INVALID_ARG))
+    r5 = _fake_retrieval()
+    r5.flags = _lib.PARK_FLAG_SIP                 # SIP without its uniforms
+    r5.sip_uniform = None
+    cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.5, 10, ctypes.byref(r5), fake, need,
+                                    None), _lib.PARK_ERR_INVALID_ARG))
+    r6 = _fake_retrieval()
+    r6.flags = _lib.PARK_FLAG_SIP | _lib.PARK_FLAG_TOPK
+    r6.sip_uniform = r6.block_weight = 0x1000
+    cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.5, 10, ctypes.byref(r6), fake, need,
                                     None), _lib.PARK_ERR_INVALID_ARG))
     for got, want in cases:
         assert got == want

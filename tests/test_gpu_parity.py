@@ -117,6 +117,34 @@ def test_selection_variants_match_oracle(park, name, variant):
             assert np.all(mask[bh][rows].sum(axis=1) == want)
 
 
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_sip_matches_oracle(park, name):
+    """SIP selection (caller-given uniforms) and the weighted attention: masks
+    bit-exact, weights within the float32 / fast-path bound, outputs within the
+    attention tolerance."""
+    from synth.generator import gen_uniform
+    cfg = CONFIGS[name]
+    ratio = float(np.float32(0.4))
+    Q, K, V = pu.inputs(name)
+    U = gen_uniform(cfg)
+    ref = po.layer(Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64), cfg.NQ, cfg.NK, ratio,
+                   cfg.iters, cfg.dtype, sip_ratio=ratio, sip_u=U.astype(np.float64))
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    shape = park.Shape.of(cfg, dt)
+    q, k, v = (pu.to_device(x, dt) for x in (Q, K, V))
+    out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, q.device, sip_uniform=torch.from_numpy(U).to(q.device))
+    O, r = park.layer(q, k, v, shape, cfg.NQ, cfg.NK, ratio, cfg.iters, out=out)
+    torch.cuda.synchronize()
+    assert r.status_code() == 0, f"device status {r.status_code()}"
+    fails = pu.compare_retrieval(r, ref, cfg.NQ, cfg.NK)
+    assert not fails, "\n".join(fails[:20])
+    W = r.block_weight.cpu().numpy().astype(np.float64).reshape(-1, cfg.NQ, cfg.NK)
+    for bh, h in enumerate(ref):
+        assert np.array_equal(W[bh] > 0, h["mask"])
+        assert np.allclose(W[bh], h["weight"], rtol=1e-4, atol=0)
+    pu.assert_output_close(O, ref, cfg.dtype == "f32")
+
+
 def test_per_step_injection_small(park):
     """Feed the oracle's iteration-t centroids as a warm start and run one
     iteration: labels and updated centroids must match the oracle's step t."""
