@@ -230,7 +230,7 @@ def workload_config(cfg) -> dict:
 
 # Retrieval variants: flag bits of park_retrieval.flags and the p passed (a ratio for top-k).
 VARIANTS = {"park": (0, None), "no_qrkc": (0x4, None), "centroid_query": (0x8, None), "topk_0.3": (0x10, 0.3),
-            "size_prior": (0x20, None)}
+            "size_prior": (0x20, None), "sip_0.3": (0x40, 0.3)}
 
 
 # ----------------------------------------------------------------------------- roofline of one kernel
@@ -338,8 +338,12 @@ def main():
         host[name] = torch.from_numpy(gen_tensor(cfg, name, seed=rank)).to(torch.bfloat16).pin_memory()
     Q, K, V = (host[n].to(dev, non_blocking=True) for n in ("Q", "K", "V"))
     shape = park.Shape.of(cfg)
-    out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, dev)
     vflags, vp = VARIANTS[args.variant]
+    sip_u = None
+    if vflags & 0x40:  # SIP draws against seeded uniforms, uploaded once
+        from synth.generator import gen_uniform
+        sip_u = torch.from_numpy(gen_uniform(cfg, seed=rank)).to(dev)
+    out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, dev, sip_uniform=sip_u)
     out.flags = vflags
     p_arg = cfg.p if vp is None else vp
     ws = park.alloc_workspace(shape, cfg.NQ, cfg.NK, dev)
