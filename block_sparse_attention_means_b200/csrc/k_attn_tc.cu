@@ -55,12 +55,13 @@ using namespace sm100;
 namespace {
 constexpr int TC_ROWS = 128;            // query rows and key rows per tile
 constexpr int TC_BLK = 16384;           // 128 rows x 128 bytes
+constexpr int TC_KST = 3;  // K ring stages (V: 2)
 constexpr uint32_t TC_TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256,384)
 constexpr float kLog2eT = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
 
 struct TcSmem {
-    uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], pv_done[2],
+    uint64_t q_full, q_empty, k_full[TC_KST], k_empty[TC_KST], v_full[2], v_empty[2], s_full[2], p_full[2], pv_done[2],
         o_empty, final_bar;
     uint32_t tmem_base;
     int abort;
@@ -79,7 +80,7 @@ __device__ __forceinline__ float fast_ex2(float x) {
     return y;
 }
 
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     k_sparse_attn_tc(const __grid_constant__ CUtensorMap tmQ, const uint8_t* __restrict__ Kimg,
                      const uint8_t* __restrict__ Vimg, int N, int NQ, int NK, const int32_t* __restrict__ q_perm,
                      const int2* __restrict__ segs, const float* __restrict__ segw,
@@ -93,16 +94,18 @@ __global__ void __launch_bounds__(320, 1)
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* Qs = base;
     uint8_t* Ks = base + 2 * TC_BLK;
-    uint8_t* Vs = Ks + 4 * TC_BLK;
+    uint8_t* Vs = Ks + 2 * TC_KST * TC_BLK;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort = &sh.abort;
     if (threadIdx.x == 0) {
         mbar_init(&sh.q_full, 1);
         mbar_init(&sh.q_empty, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < TC_KST; ++s) {
             mbar_init(&sh.k_full[s], 1);
             mbar_init(&sh.k_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&sh.v_full[s], 1);
             mbar_init(&sh.v_empty[s], 1);
             mbar_init(&sh.s_full[s], 1);
@@ -120,7 +123,7 @@ __global__ void __launch_bounds__(320, 1)
         tmem_relinquish();
     }
     // K/V stages start as zeros: groups that are never loaded must hold finite values
-    for (int i = threadIdx.x; i < 8 * TC_BLK / 16; i += blockDim.x)
+    for (int i = threadIdx.x; i < 2 * (TC_KST + 2) * TC_BLK / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(Ks)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
     tc_fence_before();
@@ -131,10 +134,15 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t idS = idesc_bf16(128, 128, 0, 0);   // S = Q K^T: both K-major
     const uint32_t idPV = idesc_bf16(128, 128, 0, 1);  // O += P V: P K-major (TMEM), V MN-major
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 0 || warp == 10) {
+        // ------------------------------------------------------------ producers
+        // Warp 0: Q and K (3-stage ring); warp 10: V and the column bias (2-stage
+        // ring).  Both walk the same items and tiles with the same segment cursor,
+        // so a V stage that waits for its PV never holds up the K loads.
+        const bool isK = warp == 0;
         int T = 0, I = 0;
-        int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
+        int k_last[TC_KST], v_last[2] = {-1, -1};
+        for (int q = 0; q < TC_KST; ++q) k_last[q] = -1;
         int q_pending = 0, q_parity = 0;
         for (int it = blockIdx.x; it < n_items && !warp_abort(abort); it += gridDim.x) {
             const WorkItem wi = items[it];
@@ -146,7 +154,7 @@ __global__ void __launch_bounds__(320, 1)
             const int32_t* pre = kv_pre + (size_t)wi.bh * NQ * NK + kp0;
             const int2* segs_item = segs + (size_t)wi.bh * NQ * NK + kp0;
             const float* segw_item = segw ? segw + (size_t)wi.bh * NQ * NK + kp0 : nullptr;
-            if (lane == 0) {
+            if (isK && lane == 0) {
                 bool ok = I == 0 || mbar_wait(&sh.q_empty, (I - 1) & 1, abort);
                 if (ok) {
                     mbar_arrive_expect_tx(&sh.q_full, 2 * TC_BLK);
@@ -183,10 +191,10 @@ __global__ void __launch_bounds__(320, 1)
             bool ok = true;
             for (int j = 0; j < nkt && ok; ++j) {
                 const int stg = T & 1, round = T >> 1;
-                int nvalid = 0;   // real key rows of group `lane` (lanes 0..15)
+                int nvalid = 0;   // real key rows of group `lane` (lanes 0..15; V warp)
                 float lwv = 0.f;  // and the logit term of its segment
 #pragma unroll 4
-                for (int g = 0; g < 16; ++g) {
+                for (int g = 0; g < 16 && !isK; ++g) {
                     const int vg = j * TC_ROWS + 8 * g;
                     const unsigned bal = __ballot_sync(0xffffffffu, p_l <= vg);
                     const int idx = (__popc(bal) - 1) & 31;
@@ -222,39 +230,45 @@ __global__ void __launch_bounds__(320, 1)
                         load_entries(seg0);
                     }
                 }
-                // K of tile j: stage free once S_{j-2} has completed
-                bool w = true;
-                if (lane == 0 && round > 0) w = mbar_wait(&sh.k_empty[stg], (round - 1) & 1, abort);
-                if (__shfl_sync(0xffffffffu, w ? 1 : 0, 0) == 0 || warp_abort(abort)) {
-                    ok = false;
-                    break;
+                if (isK) {
+                    // K of tile j: stage free once S_{j-3} has completed
+                    const int ks = T % TC_KST, kround = T / TC_KST;
+                    bool w = true;
+                    if (lane == 0 && kround > 0) w = mbar_wait(&sh.k_empty[ks], (kround - 1) & 1, abort);
+                    if (__shfl_sync(0xffffffffu, w ? 1 : 0, 0) == 0 || warp_abort(abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) mbar_arrive_expect_tx(&sh.k_full[ks], tile_bytes);
+                    __syncwarp();
+                    if (pc_groups > 0)
+                        bulk_load(Ks + ks * 2 * TC_BLK + (pc_start >> 3) * 2048, Kimg + src_off, bytes,
+                                  &sh.k_full[ks]);
+                    k_last[ks] = kround & 1;
+                } else {
+                    // V of tile j and its column bias: free once PV_{j-2} has completed
+                    bool w = true;
+                    if (lane == 0 && round > 0) w = mbar_wait(&sh.v_empty[stg], (round - 1) & 1, abort);
+                    if (__shfl_sync(0xffffffffu, w ? 1 : 0, 0) == 0 || warp_abort(abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane < 16) {
+                        float4* bp = reinterpret_cast<float4*>(&sh.bias[stg][8 * lane]);
+                        const float NI = __int_as_float(0xff800000);
+                        bp[0] = make_float4(nvalid > 0 ? lwv : NI, nvalid > 1 ? lwv : NI, nvalid > 2 ? lwv : NI,
+                                            nvalid > 3 ? lwv : NI);
+                        bp[1] = make_float4(nvalid > 4 ? lwv : NI, nvalid > 5 ? lwv : NI, nvalid > 6 ? lwv : NI,
+                                            nvalid > 7 ? lwv : NI);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_expect_tx(&sh.v_full[stg], tile_bytes);
+                    __syncwarp();
+                    if (pc_groups > 0)
+                        bulk_load(Vs + stg * 2 * TC_BLK + (pc_start >> 3) * 2048, Vimg + src_off, bytes,
+                                  &sh.v_full[stg]);
+                    v_last[stg] = round & 1;
                 }
-                if (lane == 0) mbar_arrive_expect_tx(&sh.k_full[stg], tile_bytes);
-                __syncwarp();
-                if (pc_groups > 0) bulk_load(Ks + stg * 2 * TC_BLK + (pc_start >> 3) * 2048, Kimg + src_off, bytes,
-                                             &sh.k_full[stg]);
-                k_last[stg] = round & 1;
-                // V of tile j and its column bias: free once PV_{j-2} has completed
-                w = true;
-                if (lane == 0 && round > 0) w = mbar_wait(&sh.v_empty[stg], (round - 1) & 1, abort);
-                if (__shfl_sync(0xffffffffu, w ? 1 : 0, 0) == 0 || warp_abort(abort)) {
-                    ok = false;
-                    break;
-                }
-                if (lane < 16) {
-                    float4* bp = reinterpret_cast<float4*>(&sh.bias[stg][8 * lane]);
-                    const float NI = __int_as_float(0xff800000);
-                    bp[0] = make_float4(nvalid > 0 ? lwv : NI, nvalid > 1 ? lwv : NI, nvalid > 2 ? lwv : NI,
-                                        nvalid > 3 ? lwv : NI);
-                    bp[1] = make_float4(nvalid > 4 ? lwv : NI, nvalid > 5 ? lwv : NI, nvalid > 6 ? lwv : NI,
-                                        nvalid > 7 ? lwv : NI);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive_expect_tx(&sh.v_full[stg], tile_bytes);
-                __syncwarp();
-                if (pc_groups > 0) bulk_load(Vs + stg * 2 * TC_BLK + (pc_start >> 3) * 2048, Vimg + src_off, bytes,
-                                             &sh.v_full[stg]);
-                v_last[stg] = round & 1;
                 ++T;
             }
             if (!ok) break;
@@ -263,10 +277,10 @@ __global__ void __launch_bounds__(320, 1)
         // drain: copies still in flight complete before the CTA may exit
         if (lane == 0) {
             int dummy = 0;
-            for (int s = 0; s < 2; ++s) {
+            for (int s = 0; s < TC_KST; ++s)
                 if (k_last[s] >= 0) mbar_wait(&sh.k_full[s], k_last[s], &dummy, 100000000ull);
+            for (int s = 0; s < 2; ++s)
                 if (v_last[s] >= 0) mbar_wait(&sh.v_full[s], v_last[s], &dummy, 100000000ull);
-            }
             if (q_pending) mbar_wait(&sh.q_full, q_parity, &dummy, 100000000ull);
         }
     } else if (warp == 1) {
@@ -275,11 +289,11 @@ __global__ void __launch_bounds__(320, 1)
             int G = 0, I = 0;
             const uint32_t qa = smem_u32(Qs);
             auto issue_S = [&](int g) -> bool {
-                const int b = g & 1, round = g >> 1;
+                const int b = g & 1, ks = g % TC_KST;
                 // buffer b is free: its last reader, PV_{g-2}, was issued before this MMA
-                if (!mbar_wait(&sh.k_full[b], round & 1, abort)) return false;
+                if (!mbar_wait(&sh.k_full[ks], (g / TC_KST) & 1, abort)) return false;
                 tc_fence_after();
-                const uint32_t ka = smem_u32(Ks + b * 2 * TC_BLK);
+                const uint32_t ka = smem_u32(Ks + ks * 2 * TC_BLK);
                 const uint32_t d = tmem + (uint32_t)(b * 128);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -288,7 +302,7 @@ __global__ void __launch_bounds__(320, 1)
                     umma_bf16(d, sdesc_sw128(qa + qoff, 16, 1024), sdesc_sw128(ka + koff, 16, 2048), idS, kk > 0);
                 }
                 umma_commit(&sh.s_full[b]);
-                umma_commit(&sh.k_empty[b]);
+                umma_commit(&sh.k_empty[ks]);
                 return true;
             };
             for (int it = blockIdx.x; it < n_items && !*abort; it += gridDim.x) {
@@ -513,7 +527,7 @@ int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t
     return r == CUDA_SUCCESS ? PARK_OK : PARK_ERR_CUDA;
 }
 
-size_t attn_tc_smem_bytes() { return (size_t)10 * TC_BLK + 1024; }  // Q, K x2, V x2
+size_t attn_tc_smem_bytes() { return (size_t)(2 + 2 * TC_KST + 4) * TC_BLK + 1024; }  // Q, K ring, V x2
 
 int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
                           const int32_t* q_perm, const int2* segs, const float* segw, const int32_t* kept_ptr,
@@ -526,7 +540,7 @@ int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, in
     cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     const float sl2e = (1.0f / sqrtf(128.f)) * kLog2eT;
     ::park::prof_begin(st);
-    k_sparse_attn_tc<<<num_sms, 320, sm, st>>>(mQ, (const uint8_t*)Kpad, (const uint8_t*)Vpad, N, NQ, NK, q_perm,
+    k_sparse_attn_tc<<<num_sms, 352, sm, st>>>(mQ, (const uint8_t*)Kpad, (const uint8_t*)Vpad, N, NQ, NK, q_perm,
                                                 segs, segw, kept_ptr, kv_pre, kv_len, items, item_count, (uint16_t*)O,
                                                 sl2e, status);
     PARK_TRY_LAUNCH("k_sparse_attn_tc", st);
