@@ -385,7 +385,8 @@ def sparse_attention(Q, K, V, q_labels, k_labels, mask, scale, rows=None, weight
 
 
 def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", topk_ratio=None,
-                  size_prior=False, sip_ratio=None, sip_u=None):
+                  size_prior=False, sip_ratio=None, sip_u=None, grid=None, window=None, merge=False,
+                  merge_rounds=8):
     """PARK retrieval for one (b, h): query K-means (Euclidean), key K-means
     with the query-derived metric (QRKC), PAMA importance, top-p mask
     (PARK Figure 2).  qrkc=False is the "w/o QRKC" ablation (M = I);
@@ -393,14 +394,22 @@ def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", to
     top-k at that retrieval ratio instead of top-p (PARK Table 10);
     size_prior adds log |B_m| to the PAMA logits (a variant, see pama);
     sip_ratio with the uniforms sip_u [NQ, NK] selects by SIP (see sip_select)
-    and adds the weights to the result."""
+    and adds the weights to the result.  window = (wt, wh, ww) with grid =
+    (T, Hg, W) runs both K-means with HVA's local-window assign, and merge=True
+    merges query clusters after the selection (hva_oracle); importance stays
+    the one the selection used."""
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
     d = Q.shape[1]
     scale = 1.0 / math.sqrt(d)
     M = metric(Q)
-    q_labels, CQ = kmeans(Q, NQ, iters, None, dtype)
-    k_labels, CK = kmeans(K, NK, iters, M if qrkc else None, dtype)
+    if window is None:
+        q_labels, CQ = kmeans(Q, NQ, iters, None, dtype)
+        k_labels, CK = kmeans(K, NK, iters, M if qrkc else None, dtype)
+    else:
+        from . import hva_oracle as hva
+        q_labels, CQ = hva.local_kmeans(Q, NQ, iters, grid, window, None, dtype)
+        k_labels, CK = hva.local_kmeans(K, NK, iters, grid, window, M if qrkc else None, dtype)
     q_counts = np.bincount(q_labels, minlength=NQ)
     k_counts = np.bincount(k_labels, minlength=NK)
     if pama_mode == "full":
@@ -414,6 +423,13 @@ def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", to
         mask = top_p(I, p, q_counts, k_counts)
     else:
         mask = top_k_ratio(I, topk_ratio, q_counts, k_counts)
+    if merge:
+        if weight is not None:
+            raise ValueError("merging is not defined for SIP weights")
+        from . import hva_oracle as hva
+        root = hva.merge_clusters(q_counts, mask, k_counts, merge_rounds)
+        q_labels, CQ, mask = hva.apply_merge(Q, q_labels, CQ, mask, root, dtype)
+        q_counts = np.bincount(q_labels, minlength=NQ)
     q_perm, q_off = stable_permutation(q_labels, NQ)
     k_perm, k_off = stable_permutation(k_labels, NK)
     return dict(M=M, q_labels=q_labels, k_labels=k_labels, q_centroids=CQ, k_centroids=CK,
