@@ -230,7 +230,15 @@ def workload_config(cfg) -> dict:
 
 # Retrieval variants: flag bits of park_retrieval.flags and the p passed (a ratio for top-k).
 VARIANTS = {"park": (0, None), "no_qrkc": (0x4, None), "centroid_query": (0x8, None), "topk_0.3": (0x10, 0.3),
-            "size_prior": (0x20, None), "sip_0.3": (0x40, 0.3)}
+            "size_prior": (0x20, None), "sip_0.3": (0x40, 0.3), "hva_merge": (0x80, None),
+            "hva_local": (0x100, None), "hva": (0x180, None)}
+# HyperVAttention local windows: boxes of 3 frames x 15 rows x 20 columns (900 tokens,
+# about seven clusters of the mean size 128), clipped to the grid
+HVA_WINDOW = (3, 15, 20)
+
+
+def hva_window(cfg):
+    return tuple(min(a, b) for a, b in zip(HVA_WINDOW, (cfg.T, cfg.Hg, cfg.W)))
 
 
 # ----------------------------------------------------------------------------- roofline of one kernel
@@ -288,7 +296,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override H (small cases for profiler captures)")
     ap.add_argument("--variant", default="park", choices=sorted(VARIANTS),
-                    help="retrieval variant (PARK Table 3 ablations, Table 10 top-k, size prior)")
+                    help="retrieval variant (PARK Table 3 ablations, Table 10 top-k, size prior, AB-Attention "
+                         "SIP, HyperVAttention cluster merging and local windows)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warmup must be >= 3", file=sys.stderr)
@@ -343,7 +352,8 @@ def main():
     if vflags & 0x40:  # SIP draws against seeded uniforms, uploaded once
         from synth.generator import gen_uniform
         sip_u = torch.from_numpy(gen_uniform(cfg, seed=rank)).to(dev)
-    out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, dev, sip_uniform=sip_u)
+    out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, dev, sip_uniform=sip_u,
+                               window=hva_window(cfg) if vflags & 0x100 else None)
     out.flags = vflags
     p_arg = cfg.p if vp is None else vp
     ws = park.alloc_workspace(shape, cfg.NQ, cfg.NK, dev)
@@ -430,7 +440,8 @@ def main():
     line = {"metric": METRIC, "value": round(value, 3), "unit": "ms", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(worst_ms, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {**workload_config(cfg), **({"variant": args.variant} if args.variant != "park" else {})},
+            "config": {**workload_config(cfg), **({"variant": args.variant} if args.variant != "park" else {}),
+                       **({"window": list(hva_window(cfg))} if vflags & 0x100 else {})},
             "roofline": roof, "attention_roofline": attn_roof,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches), "clocks": clocks,
             "status": status,

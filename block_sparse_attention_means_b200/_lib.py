@@ -25,6 +25,8 @@ PARK_FLAG_CENTROID_QUERY = 0x8
 PARK_FLAG_TOPK = 0x10
 PARK_FLAG_SIZE_PRIOR = 0x20
 PARK_FLAG_SIP = 0x40
+PARK_FLAG_MERGE_Q = 0x80
+PARK_FLAG_LOCAL_WINDOW = 0x100
 
 PARK_CNT_Q_RECHECK = 0
 PARK_CNT_K_RECHECK = 1
@@ -57,7 +59,9 @@ class ParkRetrieval(ctypes.Structure):
                 ("kept_ptr", ctypes.c_void_p), ("kept_idx", ctypes.c_void_p),
                 ("metric", ctypes.c_void_p), ("importance_bound", ctypes.c_void_p),
                 ("counters", ctypes.c_void_p), ("status", ctypes.c_void_p),
-                ("sip_uniform", ctypes.c_void_p), ("block_weight", ctypes.c_void_p)]
+                ("sip_uniform", ctypes.c_void_p), ("block_weight", ctypes.c_void_p),
+                ("window_t", ctypes.c_int32), ("window_h", ctypes.c_int32), ("window_w", ctypes.c_int32),
+                ("merge_rounds", ctypes.c_int32)]
 
 
 class ParkKernelTime(ctypes.Structure):

@@ -164,6 +164,11 @@ __device__ inline uint16_t double_to_bf16_bits(double x) {
 }
 
 // ---------------------------------------------------------------- warp helpers
+__device__ inline int warp_sum_int(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
 __device__ inline float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

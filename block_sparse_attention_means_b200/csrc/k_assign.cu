@@ -18,15 +18,18 @@ namespace park {
 // input path, which has no tensor-core filter).  Euclidean distance:
 // sum_j (x_j - c_j)^2.  QRKC: c^T M c - 2 x . (M c), the distance minus the row
 // constant x^T M x.  Ties go to the lowest index.
+// Rows row0 .. N-1 of every head (row0 = 0: all rows).
 template <typename T, bool METRIC>
 __global__ void k_recheck(const T* __restrict__ X, const T* __restrict__ C, const double* __restrict__ w64,
                           const double* __restrict__ b64, int N, int D, int K, int32_t* __restrict__ labels,
-                          int total_rows) {
+                          int BH, int row0) {
     const int lane = threadIdx.x & 31;
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nw = (gridDim.x * blockDim.x) >> 5;
-    for (int gr = gw; gr < total_rows; gr += nw) {
-        const int bh = gr / N;
+    const int per_head = N - row0, total_rows = BH * per_head;
+    for (int e = gw; e < total_rows; e += nw) {
+        const int bh = e / per_head;
+        const int gr = bh * N + row0 + (e - bh * per_head);
         const T* x = X + (size_t)gr * D;
         double xv[4];
 #pragma unroll
@@ -160,32 +163,39 @@ __global__ __launch_bounds__(256) void k_rescore_full(const T* __restrict__ X, c
     }
 }
 
+int launch_recheck_rows(const void* X, int dtype, int BH, int N, int D, int K, const void* C, const double* w64,
+                        const double* b64, int32_t* labels, int row0, int num_sms, cudaStream_t st) {
+    if (D > 128) return PARK_ERR_UNSUPPORTED;
+    if (row0 >= N) return PARK_OK;
+    const bool metric = w64 != nullptr;
+    const int blocks = num_sms * 8;
+    ::park::prof_begin(st);
+    if (dtype == PARK_BF16) {
+        if (metric)
+            k_recheck<bf16_t, true><<<blocks, 256, 0, st>>>((const bf16_t*)X, (const bf16_t*)C, w64, b64, N, D, K,
+                                                            labels, BH, row0);
+        else
+            k_recheck<bf16_t, false><<<blocks, 256, 0, st>>>((const bf16_t*)X, (const bf16_t*)C, w64, b64, N, D, K,
+                                                             labels, BH, row0);
+    } else {
+        if (metric)
+            k_recheck<float, true><<<blocks, 256, 0, st>>>((const float*)X, (const float*)C, w64, b64, N, D, K,
+                                                           labels, BH, row0);
+        else
+            k_recheck<float, false><<<blocks, 256, 0, st>>>((const float*)X, (const float*)C, w64, b64, N, D, K,
+                                                            labels, BH, row0);
+    }
+    PARK_TRY_LAUNCH("k_recheck", st);
+    return PARK_OK;
+}
+
 int launch_recheck(const void* X, int dtype, int BH, int N, int D, int K, const void* C, const double* w64,
                    const double* b64, int32_t* labels, Lists lists, int all_rows, int num_sms,
                    int64_t* counters, int cnt_slot, cudaStream_t st) {
     if (D > 128) return PARK_ERR_UNSUPPORTED;
     const bool metric = w64 != nullptr;
+    if (all_rows) return launch_recheck_rows(X, dtype, BH, N, D, K, C, w64, b64, labels, 0, num_sms, st);
     ::park::prof_begin(st);
-    if (all_rows) {
-        const int blocks = num_sms * 8, total = BH * N;
-        if (dtype == PARK_BF16) {
-            if (metric)
-                k_recheck<bf16_t, true><<<blocks, 256, 0, st>>>((const bf16_t*)X, (const bf16_t*)C, w64, b64, N, D,
-                                                                K, labels, total);
-            else
-                k_recheck<bf16_t, false><<<blocks, 256, 0, st>>>((const bf16_t*)X, (const bf16_t*)C, w64, b64, N, D,
-                                                                 K, labels, total);
-        } else {
-            if (metric)
-                k_recheck<float, true><<<blocks, 256, 0, st>>>((const float*)X, (const float*)C, w64, b64, N, D, K,
-                                                               labels, total);
-            else
-                k_recheck<float, false><<<blocks, 256, 0, st>>>((const float*)X, (const float*)C, w64, b64, N, D, K,
-                                                                labels, total);
-        }
-        PARK_TRY_LAUNCH("k_recheck", st);
-        return PARK_OK;
-    }
     const int fb = num_sms * 4;
     if (dtype == PARK_BF16) {
         if (metric)

@@ -45,6 +45,9 @@ int launch_assign_tc(const void* X, int BH, int N, int K, const CentroidOps& ops
 int launch_recheck(const void* X, int dtype, int BH, int N, int D, int K, const void* C, const double* w64,
                    const double* b64, int32_t* labels, Lists lists, int all_rows, int num_sms,
                    int64_t* counters, int cnt_slot, cudaStream_t st);
+// float64 assign of rows row0 .. N-1 of every head against every centroid
+int launch_recheck_rows(const void* X, int dtype, int BH, int N, int D, int K, const void* C, const double* w64,
+                        const double* b64, int32_t* labels, int row0, int num_sms, cudaStream_t st);
 
 // ---- k_sort.cu
 int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist, int nchunks, int32_t* perm,
@@ -78,6 +81,34 @@ int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int 
                     cudaStream_t st);
 int launch_kept_csr(const uint8_t* mask, const int32_t* kept_cnt, int BH, int NQ, int NK, int32_t* kept_ptr,
                     int32_t* kept_idx, int64_t* counters, cudaStream_t st);
+
+// ---- k_hva.cu
+// Video-grid windows for the local-window K-means: wt x wh x ww tokens, nWt x
+// nWh x nWw of them (nW in all), maxwin tokens in the largest; nvideo = T Hg W.
+struct WinGeom {
+    int T, Hg, W, wt, wh, ww, nWt, nWh, nWw, nW, nvideo, maxwin;
+};
+int launch_local_init(const void* X, int dtype, int BH, int N, int D, int K, const WinGeom& g, void* C,
+                      cudaStream_t st);
+// Grid tokens against their window's centroids; text tokens are left to
+// launch_recheck_rows.  C: centroids (Euclidean); w64/b64/wmax/bmax from
+// launch_centroid_prep (w64 null: Euclidean).
+int launch_assign_local(const void* X, int dtype, int BH, int N, int D, int K, const WinGeom& g, const void* C,
+                        const double* w64, const double* b64, const float* wmax, const float* bmax, int32_t* labels,
+                        int64_t* counters, int cnt_slot, cudaStream_t st);
+size_t local_assign_smem(int K, int nW, int D);
+// Query-cluster merging state, per head: S [NQ][Wd] kept-set bitsets, P
+// [kMergePlanes][Wd] bit planes of the key clusters' 8-row unit counts.
+constexpr int kMergePlanes = 18;  // unit counts are below 2^18 (N <= 2^20)
+struct MergeWs {
+    uint32_t* S;
+    uint32_t* P;
+    int32_t *n, *L, *alive, *root, *best, *rootf, *done, *nb;
+};
+// Rewrites mask rows and kept counts of the merged groups and moves q_labels to
+// the groups' roots; `rounds` parallel rounds at most.
+int launch_merge(uint8_t* mask, int32_t* kept_cnt, const int32_t* q_off, const int32_t* k_off, int BH, int N, int NQ,
+                 int NK, int rounds, const MergeWs& m, int32_t* q_labels, int num_sms, cudaStream_t st);
 
 // ---- k_attn.cu
 struct WorkItem {

@@ -65,6 +65,7 @@ namespace {
 
 struct Dims {
     int B, H, N, D, dtype, BH, elt;
+    int T, Hg, W, nvideo;  // video grid; nvideo = T Hg W tokens precede the text tokens
 };
 
 int check_shape(const park_shape* s, int NQ, int NK, Dims* d) {
@@ -92,6 +93,10 @@ int check_shape(const park_shape* s, int NQ, int NK, Dims* d) {
     d->dtype = s->dtype;
     d->BH = (int)BH;
     d->elt = s->dtype == PARK_BF16 ? 2 : 4;
+    d->T = s->T;
+    d->Hg = s->Hg;
+    d->W = s->W;
+    d->nvideo = (int)nv;
     return PARK_OK;
 }
 
@@ -118,7 +123,7 @@ int metric_chunks(const Dims& d) {
 
 struct RetrievalWs {
     size_t M, Mpart, xnorm_q, xnorm_k, wop, b32, b64, w64, wmax, bmax, lfull, lcnt, hist, rho, plist,
-        pcnt, kcnt, f64z, cperm, coff, total;
+        pcnt, kcnt, f64z, cperm, coff, mS, mP, mI, mH, total;
 };
 
 RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
@@ -146,9 +151,15 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
     w.f64z = c.take(pama_f64_scratch_bytes(NK));
     w.cperm = c.take(BH * NQ * 4);
     w.coff = c.take(BH * (NQ + 1) * 4);
+    const size_t Wd = (NK + 31) / 32;
+    w.mS = c.take(BH * NQ * Wd * 4);
+    w.mP = c.take(BH * kMergePlanes * Wd * 4);
+    w.mI = c.take(6 * BH * NQ * 4);  // n, L, alive, root, best, rootf
+    w.mH = c.take(2 * BH * 4);       // done, nb
     w.total = c.off;
     return w;
 }
+
 
 struct AttnWs {
     size_t Qp, Kp, Vp, poff, segs, segw, items, icnt, kvpre, kvlen, total;
@@ -198,6 +209,23 @@ P* at(void* ws, size_t off) {
     return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
 }
 
+MergeWs merge_ws(void* ws, const RetrievalWs& w, int BH, int NQ) {
+    MergeWs m;
+    m.S = at<uint32_t>(ws, w.mS);
+    m.P = at<uint32_t>(ws, w.mP);
+    int32_t* a = at<int32_t>(ws, w.mI);
+    const size_t s = (size_t)BH * NQ;
+    m.n = a;
+    m.L = a + s;
+    m.alive = a + 2 * s;
+    m.root = a + 3 * s;
+    m.best = a + 4 * s;
+    m.rootf = a + 5 * s;
+    m.done = at<int32_t>(ws, w.mH);
+    m.nb = m.done + BH;
+    return m;
+}
+
 int memset_async(void* p, size_t n, cudaStream_t st) {
     if (cudaMemsetAsync(p, 0, n, st) != cudaSuccess) {
         cudaGetLastError();
@@ -229,6 +257,8 @@ struct Side {
     float* xnorm;
     int Kmax;          // max(NQ, NK): leading dimension of the shared bias buffer
     int32_t* status;
+    const WinGeom* win;  // non-null: HVA local-window assign
+    int n_text;
 };
 
 int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, void* ws, int64_t* counters,
@@ -253,6 +283,25 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
     Lists lists;
     lists.full_row = at<int32_t>(ws, w.lfull);
     lists.counts = at<int32_t>(ws, w.lcnt);
+    if (s.win) {
+        // HVA local windows: float32-certified scores against the window's centroids,
+        // float64 for text tokens and for rows the bound cannot decide
+        ops.w = nullptr;
+        if (!s.warm) PARK_CHECK(launch_local_init(s.X, d.dtype, BH, N, D, K, *s.win, s.C, st));
+        for (int it = 0; it < iters; ++it) {
+            PARK_CHECK(memset_async(ops.wmax, (size_t)BH * 4, st));
+            PARK_CHECK(memset_async(ops.bmax, (size_t)BH * 4, st));
+            PARK_CHECK(launch_centroid_prep(s.C, d.dtype, BH, K, D, s.M, ops, st));
+            PARK_CHECK(launch_assign_local(s.X, d.dtype, BH, N, D, K, *s.win, s.C, ops.w64, ops.bias64, ops.wmax,
+                                           ops.bmax, s.labels, counters, s.cnt_slot, st));
+            if (s.n_text > 0)
+                PARK_CHECK(launch_recheck_rows(s.X, d.dtype, BH, N, D, K, s.C, ops.w64, ops.bias64, s.labels,
+                                               s.win->nvideo, num_sms, st));
+            PARK_CHECK(launch_label_sort(s.labels, BH, N, K, at<int32_t>(ws, w.hist), nchunks, s.perm, s.offsets, st));
+            PARK_CHECK(launch_update(s.X, d.dtype, BH, N, D, K, s.perm, s.offsets, s.C, st));
+        }
+        return PARK_OK;
+    }
     if (bf16) PARK_CHECK(launch_row_norms(s.X, d.dtype, BH, N, D, s.xnorm, st));
     if (!s.warm) PARK_CHECK(launch_strided_init(s.X, d.dtype, BH, N, D, K, s.C, st));
     const float gamma = gamma_for(ops.kw, s.M != nullptr);
@@ -290,11 +339,43 @@ size_t ws_bytes_for(const Dims& d, int NQ, int NK) {
 bool flags_ok(const park_retrieval* r, float p) {
     const uint32_t flags = r->flags;
     const uint32_t known = PARK_FLAG_WARM_START_Q | PARK_FLAG_WARM_START_K | PARK_FLAG_NO_QRKC |
-                           PARK_FLAG_CENTROID_QUERY | PARK_FLAG_TOPK | PARK_FLAG_SIZE_PRIOR | PARK_FLAG_SIP;
+                           PARK_FLAG_CENTROID_QUERY | PARK_FLAG_TOPK | PARK_FLAG_SIZE_PRIOR | PARK_FLAG_SIP |
+                           PARK_FLAG_MERGE_Q | PARK_FLAG_LOCAL_WINDOW;
     if (flags & ~known) return false;
     if ((flags & (PARK_FLAG_TOPK | PARK_FLAG_SIP)) && p > 1.0f) return false;
     if ((flags & PARK_FLAG_TOPK) && (flags & PARK_FLAG_SIP)) return false;
+    if ((flags & PARK_FLAG_MERGE_Q) && ((flags & PARK_FLAG_SIP) || r->merge_rounds < 0 || r->merge_rounds > 64))
+        return false;
     return !(flags & PARK_FLAG_SIP) || (r->sip_uniform && r->block_weight);
+}
+
+constexpr int kDefaultMergeRounds = 8;
+constexpr int kMaxWindowCentroids = 256;
+
+// Window geometry of PARK_FLAG_LOCAL_WINDOW: every extent within the grid, every
+// window owning at least one query and one key centroid, at most 256 each.
+int window_geometry(const park_retrieval* r, const Dims& d, int NQ, int NK, WinGeom* g) {
+    if (!(r->flags & PARK_FLAG_LOCAL_WINDOW)) return PARK_OK;
+    if (d.nvideo < 1 || r->window_t < 1 || r->window_h < 1 || r->window_w < 1 || r->window_t > d.T ||
+        r->window_h > d.Hg || r->window_w > d.W)
+        return PARK_ERR_INVALID_ARG;
+    g->T = d.T;
+    g->Hg = d.Hg;
+    g->W = d.W;
+    g->wt = r->window_t;
+    g->wh = r->window_h;
+    g->ww = r->window_w;
+    g->nWt = (d.T + g->wt - 1) / g->wt;
+    g->nWh = (d.Hg + g->wh - 1) / g->wh;
+    g->nWw = (d.W + g->ww - 1) / g->ww;
+    const long long nW = (long long)g->nWt * g->nWh * g->nWw;
+    if (nW > NQ || nW > NK) return PARK_ERR_INVALID_ARG;
+    g->nW = (int)nW;
+    g->nvideo = d.nvideo;
+    g->maxwin = g->wt * g->wh * g->ww;
+    const int kmax = ((NQ > NK ? NQ : NK) + g->nW - 1) / g->nW;
+    if (kmax > kMaxWindowCentroids) return PARK_ERR_UNSUPPORTED;
+    return PARK_OK;
 }
 
 int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, float p, int iters,
@@ -318,12 +399,15 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
     if (qrkc || out->metric)
         PARK_CHECK(launch_metric(Q, d.dtype, BH, N, D, at<double>(ws, w.Mpart), metric_chunks(d), M, out->metric, st));
 
+    WinGeom geo{};
+    PARK_CHECK(window_geometry(out, d, NQ, NK, &geo));
+    const WinGeom* win = (fl & PARK_FLAG_LOCAL_WINDOW) ? &geo : nullptr;
     Side sq{Q, NQ, out->q_centroids, out->q_labels, out->q_perm, out->q_offsets, nullptr,
             (out->flags & PARK_FLAG_WARM_START_Q) != 0, PARK_CNT_Q_RECHECK, at<float>(ws, w.xnorm_q),
-            NQ > NK ? NQ : NK, out->status};
+            NQ > NK ? NQ : NK, out->status, win, N - d.nvideo};
     Side sk{K, NK, out->k_centroids, out->k_labels, out->k_perm, out->k_offsets, qrkc ? M : nullptr,
             (out->flags & PARK_FLAG_WARM_START_K) != 0, PARK_CNT_K_RECHECK, at<float>(ws, w.xnorm_k),
-            NQ > NK ? NQ : NK, out->status};
+            NQ > NK ? NQ : NK, out->status, win, N - d.nvideo};
     PARK_CHECK(run_kmeans(d, sq, iters, w, ws, out->counters, num_sms, st));
     PARK_CHECK(run_kmeans(d, sk, iters, w, ws, out->counters, num_sms, st));
 
@@ -361,6 +445,16 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
                                    at<int32_t>(ws, w.pcnt) + 4,
                                    at<double>(ws, w.f64z), out->importance, out->importance_bound, out->mask, kcnt,
                                    out->counters, st));
+    }
+    if (fl & PARK_FLAG_MERGE_Q) {
+        // HVA cluster merging; the merged clustering's permutation and centroids follow
+        const int rounds = out->merge_rounds > 0 ? out->merge_rounds : kDefaultMergeRounds;
+        PARK_CHECK(launch_merge(out->mask, kcnt, out->q_offsets, out->k_offsets, BH, N, NQ, NK, rounds,
+                                merge_ws(ws, w, BH, NQ), out->q_labels, num_sms, st));
+        const int nchunks = (N + kSortChunk - 1) / kSortChunk;
+        PARK_CHECK(launch_label_sort(out->q_labels, BH, N, NQ, at<int32_t>(ws, w.hist), nchunks, out->q_perm,
+                                     out->q_offsets, st));
+        PARK_CHECK(launch_update(Q, d.dtype, BH, N, D, NQ, out->q_perm, out->q_offsets, out->q_centroids, st));
     }
     PARK_CHECK(launch_kept_csr(out->mask, kcnt, BH, NQ, NK, out->kept_ptr, out->kept_idx, out->counters, st));
     return PARK_OK;
@@ -424,6 +518,8 @@ int park_retrieve(const void* Q, const void* K, const park_shape* shape, int NQ,
     if (!Q || !K || !ws || !retrieval_ptrs_ok(out)) return PARK_ERR_INVALID_ARG;
     if (!(p > 0.0f) || !std::isfinite(p) || iters < 1) return PARK_ERR_INVALID_ARG;
     if (!flags_ok(out, p)) return PARK_ERR_INVALID_ARG;
+    WinGeom geo;
+    PARK_CHECK(window_geometry(out, d, NQ, NK, &geo));
     if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
     return retrieve_impl(Q, K, d, NQ, NK, p, iters, out, ws, static_cast<cudaStream_t>(stream));
 }
@@ -445,6 +541,8 @@ int park_layer(const void* Q, const void* K, const void* V, const park_shape* sh
     if (!Q || !K || !V || !O || !ws || !retrieval_ptrs_ok(out)) return PARK_ERR_INVALID_ARG;
     if (!(p > 0.0f) || !std::isfinite(p) || iters < 1) return PARK_ERR_INVALID_ARG;
     if (!flags_ok(out, p)) return PARK_ERR_INVALID_ARG;
+    WinGeom geo;
+    PARK_CHECK(window_geometry(out, d, NQ, NK, &geo));
     if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     PARK_CHECK(retrieve_impl(Q, K, d, NQ, NK, p, iters, out, ws, st));

@@ -66,6 +66,8 @@ class Retrieval:
     flags: int = 0
     sip_uniform: torch.Tensor | None = None   # float32 [B,H,NQ,NK], input with PARK_FLAG_SIP
     block_weight: torch.Tensor | None = None  # float32 [B,H,NQ,NK], output with PARK_FLAG_SIP
+    window: tuple = (0, 0, 0)                 # (frames, rows, columns) of a box, with PARK_FLAG_LOCAL_WINDOW
+    merge_rounds: int = 0                     # with PARK_FLAG_MERGE_Q (0 = the library's default)
 
     def c(self) -> _lib.ParkRetrieval:
         p = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)  # noqa: E731
@@ -73,17 +75,21 @@ class Retrieval:
                                   p(self.q_offsets), p(self.k_offsets), p(self.q_centroids), p(self.k_centroids),
                                   p(self.importance), p(self.mask), p(self.kept_ptr), p(self.kept_idx),
                                   p(self.metric), p(self.importance_bound), p(self.counters), p(self.status),
-                                  p(self.sip_uniform), p(self.block_weight))
+                                  p(self.sip_uniform), p(self.block_weight), *[int(x) for x in self.window],
+                                  int(self.merge_rounds))
 
     def status_code(self) -> int:
         return int(self.status.item())
 
 
 def alloc_retrieval(shape: Shape, NQ: int, NK: int, device, with_metric: bool = False,
-                    sip_uniform: torch.Tensor | None = None) -> Retrieval:
+                    sip_uniform: torch.Tensor | None = None, window: tuple | None = None,
+                    merge: bool = False, merge_rounds: int = 0) -> Retrieval:
     """Outputs of park_retrieve on `device`.  With sip_uniform (float32
     [B,H,NQ,NK] uniforms on the device) the result is set up for PARK_FLAG_SIP:
-    the flag is set and block_weight is allocated."""
+    the flag is set and block_weight is allocated.  window = (frames, rows,
+    columns) sets PARK_FLAG_LOCAL_WINDOW with that box; merge sets
+    PARK_FLAG_MERGE_Q."""
     B, H, N, D = shape.B, shape.H, shape.N, shape.D
     i32 = dict(dtype=torch.int32, device=device)
     sip = {}
@@ -92,7 +98,14 @@ def alloc_retrieval(shape: Shape, NQ: int, NK: int, device, with_metric: bool = 
             raise ValueError("sip_uniform must be float32 [B, H, NQ, NK]")
         sip = dict(flags=_lib.PARK_FLAG_SIP, sip_uniform=sip_uniform.contiguous(),
                    block_weight=torch.empty(B, H, NQ, NK, dtype=torch.float32, device=device))
-    return Retrieval(**sip,
+    flags = sip.pop("flags", 0)
+    if window is not None:
+        flags |= _lib.PARK_FLAG_LOCAL_WINDOW
+        sip["window"] = tuple(int(x) for x in window)
+    if merge:
+        flags |= _lib.PARK_FLAG_MERGE_Q
+        sip["merge_rounds"] = int(merge_rounds)
+    return Retrieval(flags=flags, **sip,
         q_labels=torch.empty(B, H, N, **i32), k_labels=torch.empty(B, H, N, **i32),
         q_perm=torch.empty(B, H, N, **i32), k_perm=torch.empty(B, H, N, **i32),
         q_offsets=torch.empty(B, H, NQ + 1, **i32), k_offsets=torch.empty(B, H, NK + 1, **i32),

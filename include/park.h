@@ -102,6 +102,35 @@ extern "C" {
 #define PARK_FLAG_TOPK 0x10u
 #define PARK_FLAG_SIZE_PRIOR 0x20u
 #define PARK_FLAG_SIP 0x40u
+/* HyperVAttention's clustering parts ("HyperVAttention: Efficient Sparse
+ * Attention with Spatio-Temporal Clustering for Video Diffusion", abstract):
+ *   MERGE_Q          after the selection, query clusters merge in parallel
+ *                    agglomerative rounds: each non-empty cluster g picks the
+ *                    partner h with the largest gain cost(g) + cost(h) -
+ *                    cost(g u h) > 0 (ties: lowest h), with cost(n, L) =
+ *                    ceil(n/128) ceil(L/128) the attention's (query tile, key
+ *                    tile) pairs for n query rows whose kept key clusters fill L
+ *                    key rows (each cluster rounded up to 8 rows), the merged
+ *                    cluster keeping the union of the kept sets; mutual pairs
+ *                    merge into the lower index; rounds repeat until one merges
+ *                    nothing, at most merge_rounds (0 = 8, at most 64).  The
+ *                    outputs then describe the merged clustering (labels, perm,
+ *                    offsets, centroids recomputed as exact means, mask and CSR
+ *                    rows of merged-away clusters empty) except importance and
+ *                    importance_bound, which keep the values the selection used.
+ *                    Not combinable with SIP.
+ *   LOCAL_WINDOW     both K-means run on 3D local windows: the video grid is tiled
+ *                    by boxes of window_t x window_h x window_w tokens (the last
+ *                    box of an axis may be shorter; nW boxes, numbered with the
+ *                    column box fastest); box w owns centroids floor(w K / nW) ..
+ *                    floor((w+1) K / nW) - 1, initialised at its members
+ *                    floor(j n_w / K_w) in token order (without WARM_START), and
+ *                    a video token is assigned among its box's centroids only;
+ *                    text tokens among all.  Needs 1 <= window extents <= grid
+ *                    extents and nW <= min(NQ, NK) (else PARK_ERR_INVALID_ARG),
+ *                    at most 256 centroids per box (else PARK_ERR_UNSUPPORTED). */
+#define PARK_FLAG_MERGE_Q 0x80u
+#define PARK_FLAG_LOCAL_WINDOW 0x100u
 
 /* ---- park_retrieval.counters indices (outputs, int64) ------------------ */
 #define PARK_CNT_Q_RECHECK 0    /* query rows whose bf16 score margin was not
@@ -152,6 +181,9 @@ typedef struct {
     const float *sip_uniform; /* [B,H,NQ,NK] in, with PARK_FLAG_SIP: uniforms on [0,1) */
     float *block_weight;   /* [B,H,NQ,NK] out, with PARK_FLAG_SIP: 1/pi_m for kept
                               blocks, 0 elsewhere; read by park_sparse_attn     */
+    int32_t window_t, window_h, window_w; /* in, with PARK_FLAG_LOCAL_WINDOW: box
+                              extent in frames, rows and columns of the grid    */
+    int32_t merge_rounds;  /* in, with PARK_FLAG_MERGE_Q: most merging rounds (0 = 8) */
 } park_retrieval;
 
 /* Bytes of device workspace that park_retrieve, park_sparse_attn and

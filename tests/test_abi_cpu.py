@@ -29,15 +29,16 @@ def test_library_exports_every_declared_function():
 
 
 def test_struct_layout_matches_header():
-    # park_shape: 8 ints; park_retrieval: uint32 flags + 18 pointers (padded)
+    # park_shape: 8 ints; park_retrieval: uint32 flags + 18 pointers (padded) + 4 int32
     assert ctypes.sizeof(_lib.ParkShape) == 32
-    assert ctypes.sizeof(_lib.ParkRetrieval) == 8 + 18 * 8
+    assert ctypes.sizeof(_lib.ParkRetrieval) == 8 + 18 * 8 + 4 * 4
     text = open(os.path.join(ROOT, "include", "park.h")).read()
     assert re.search(r"#define PARK_NUM_COUNTERS 8", text)
     for name in ("PARK_OK", "PARK_ERR_INVALID_ARG", "PARK_ERR_UNSUPPORTED", "PARK_ERR_WORKSPACE", "PARK_ERR_CUDA",
                  "PARK_ERR_RANGE", "PARK_ERR_TIMEOUT", "PARK_BF16", "PARK_F32", "PARK_FLAG_WARM_START_Q",
                  "PARK_FLAG_WARM_START_K", "PARK_FLAG_NO_QRKC", "PARK_FLAG_CENTROID_QUERY", "PARK_FLAG_TOPK",
-                 "PARK_FLAG_SIZE_PRIOR", "PARK_FLAG_SIP", "PARK_CNT_KEPT_PAIRS"):
+                 "PARK_FLAG_SIZE_PRIOR", "PARK_FLAG_SIP", "PARK_FLAG_MERGE_Q", "PARK_FLAG_LOCAL_WINDOW",
+                 "PARK_CNT_KEPT_PAIRS"):
         m = re.search(rf"#define {name} (\w+)", text)
         assert m and int(m.group(1).rstrip("u"), 0) == getattr(_lib, name), name
 
@@ -71,8 +72,9 @@ def test_workspace_size_and_shape_validation():
 def _fake_retrieval():
     # non-null placeholders: every call below fails validation before touching them
     r = _lib.ParkRetrieval()
-    for name, _ in _lib.ParkRetrieval._fields_[1:]:
-        setattr(r, name, ctypes.c_void_p(0x1000))
+    for name, kind in _lib.ParkRetrieval._fields_[1:]:
+        if kind is ctypes.c_void_p:
+            setattr(r, name, ctypes.c_void_p(0x1000))
     return r
 
 
@@ -106,7 +108,7 @@ def test_host_argument_errors_enqueue_nothing():
     cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.9, 10, ctypes.byref(r2), fake, need,
                                     None), _lib.PARK_ERR_INVALID_ARG))
     r3 = _fake_retrieval()
-    r3.flags = 0x80                               # unknown flag bit
+    r3.flags = 0x200                              # unknown flag bit
     cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.9, 10, ctypes.byref(r3), fake, need,
                                     None), _lib.PARK_ERR_INVALID_ARG))
     r4 = _fake_retrieval()
@@ -123,6 +125,23 @@ def test_host_argument_errors_enqueue_nothing():
     r6.sip_uniform = r6.block_weight = 0x1000
     cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.5, 10, ctypes.byref(r6), fake, need,
                                     None), _lib.PARK_ERR_INVALID_ARG))
+    # HVA options: merging with SIP, too many merging rounds, a box that is empty,
+    # larger than the grid (2 x 4 x 8 here), or more boxes than centroids
+    bad = [(_lib.PARK_FLAG_MERGE_Q | _lib.PARK_FLAG_SIP, dict(), 0.5),
+           (_lib.PARK_FLAG_MERGE_Q, dict(merge_rounds=65), 0.9),
+           (_lib.PARK_FLAG_MERGE_Q, dict(merge_rounds=-1), 0.9),
+           (_lib.PARK_FLAG_LOCAL_WINDOW, dict(window_t=0, window_h=1, window_w=1), 0.9),
+           (_lib.PARK_FLAG_LOCAL_WINDOW, dict(window_t=3, window_h=1, window_w=1), 0.9),
+           (_lib.PARK_FLAG_LOCAL_WINDOW, dict(window_t=1, window_h=1, window_w=1), 0.9)]   # 16 boxes > 4
+    for flags, fields, p in bad:
+        rb = _fake_retrieval()
+        rb.flags = flags
+        for k, v in fields.items():
+            setattr(rb, k, v)
+        cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, p, 10, ctypes.byref(rb), fake, need,
+                                        None), _lib.PARK_ERR_INVALID_ARG))
+        cases.append((lib.park_layer(fake, fake, fake, ctypes.byref(shape), 4, 4, p, 10, fake, ctypes.byref(rb),
+                                     fake, need, None), _lib.PARK_ERR_INVALID_ARG))
     for got, want in cases:
         assert got == want
     assert lib.park_launch_count() == before
