@@ -58,6 +58,44 @@ __device__ inline void load8<float>(const float* p, float* v) {
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
+// acc0[j] += x_a . w_j and acc1[j] += x_b . w_j (float32 FMA chains over the D
+// columns in order) for the KC rows w_j of wsm; the token rows are read 16
+// columns at a time, whole 32-byte sectors, so no sector is fetched twice.  With
+// NORM the squared norms of the two rows are accumulated too.
+template <typename T, int KC, bool NORM>
+__device__ inline void dot_rows(const T* xa_p, const T* xb_p, const float* wsm, int D, float* acc0, float* acc1,
+                                float& nxa, float& nxb) {
+    for (int d = 0; d < D; d += 16) {
+        float xa[16], xb[16];
+        load8<T>(xa_p + d, xa);
+        load8<T>(xa_p + d + 8, xa + 8);
+        load8<T>(xb_p + d, xb);
+        load8<T>(xb_p + d + 8, xb + 8);
+        if (NORM) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                nxa = fmaf(xa[e], xa[e], nxa);
+                nxb = fmaf(xb[e], xb[e], nxb);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < KC; ++j) {
+#pragma unroll
+            for (int h = 0; h < 16; h += 4) {
+                const float4 w = *reinterpret_cast<const float4*>(wsm + j * D + d + h);
+                acc0[j] = fmaf(xa[h], w.x, acc0[j]);
+                acc0[j] = fmaf(xa[h + 1], w.y, acc0[j]);
+                acc0[j] = fmaf(xa[h + 2], w.z, acc0[j]);
+                acc0[j] = fmaf(xa[h + 3], w.w, acc0[j]);
+                acc1[j] = fmaf(xb[h], w.x, acc1[j]);
+                acc1[j] = fmaf(xb[h + 1], w.y, acc1[j]);
+                acc1[j] = fmaf(xb[h + 2], w.z, acc1[j]);
+                acc1[j] = fmaf(xb[h + 3], w.w, acc1[j]);
+            }
+        }
+    }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- local init
@@ -135,39 +173,10 @@ __global__ __launch_bounds__(kLocalThreads) void k_assign_local(
         float acc0[KC], acc1[KC];
 #pragma unroll
         for (int j = 0; j < KC; ++j) acc0[j] = acc1[j] = 0.f;
-        for (int d = 0; d < D; d += 8) {
-            float xa[8], xb[8];
-            load8<T>(x0p + d, xa);
-            load8<T>(x1p + d, xb);
-            if (kc == 0) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    nx0 = fmaf(xa[e], xa[e], nx0);
-                    nx1 = fmaf(xb[e], xb[e], nx1);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < KC; ++j) {
-                const float4 wa = *reinterpret_cast<const float4*>(wsm + (kc + j) * D + d);
-                const float4 wb = *reinterpret_cast<const float4*>(wsm + (kc + j) * D + d + 4);
-                acc0[j] = fmaf(xa[0], wa.x, acc0[j]);
-                acc0[j] = fmaf(xa[1], wa.y, acc0[j]);
-                acc0[j] = fmaf(xa[2], wa.z, acc0[j]);
-                acc0[j] = fmaf(xa[3], wa.w, acc0[j]);
-                acc0[j] = fmaf(xa[4], wb.x, acc0[j]);
-                acc0[j] = fmaf(xa[5], wb.y, acc0[j]);
-                acc0[j] = fmaf(xa[6], wb.z, acc0[j]);
-                acc0[j] = fmaf(xa[7], wb.w, acc0[j]);
-                acc1[j] = fmaf(xb[0], wa.x, acc1[j]);
-                acc1[j] = fmaf(xb[1], wa.y, acc1[j]);
-                acc1[j] = fmaf(xb[2], wa.z, acc1[j]);
-                acc1[j] = fmaf(xb[3], wa.w, acc1[j]);
-                acc1[j] = fmaf(xb[4], wb.x, acc1[j]);
-                acc1[j] = fmaf(xb[5], wb.y, acc1[j]);
-                acc1[j] = fmaf(xb[6], wb.z, acc1[j]);
-                acc1[j] = fmaf(xb[7], wb.w, acc1[j]);
-            }
-        }
+        if (kc == 0)
+            dot_rows<T, KC, true>(x0p, x1p, wsm + kc * D, D, acc0, acc1, nx0, nx1);
+        else
+            dot_rows<T, KC, false>(x0p, x1p, wsm + kc * D, D, acc0, acc1, nx0, nx1);
 #pragma unroll
         for (int j = 0; j < KC; ++j) {
             if (kc + j < kw) {
@@ -242,6 +251,268 @@ __global__ __launch_bounds__(kLocalThreads) void k_assign_local(
         atomicAdd((unsigned long long*)(counters + cnt_slot), (unsigned long long)s_rescored);
 }
 
+// ---------------------------------------------------------------- text tokens
+// Text tokens have no box and search every centroid.  k_text_partial: one CTA
+// per (64 text tokens, split of the centroids, head); lane l holds tokens l and
+// l + 32, warp w scores candidates 16w .. 16w + 15 of each staged block of 128
+// centroids (float32 operands in shared memory, the same scores as the box
+// assign) and the CTA leaves each token's (best, index, runner-up) of its split.
+// k_text_finish: one warp per token merges the splits, certifies the winner with
+// the box assign's bound, else rescores it in float64 (lanes over the columns,
+// one centroid at a time, ties to the lowest index).
+constexpr int kTextTokens = 64;
+constexpr int kTextBlock = 128;
+
+int text_splits(int BH, int n_text, int K) {
+    const int nblk = (K + kTextBlock - 1) / kTextBlock;
+    const long long ctas = (long long)BH * ((n_text + kTextTokens - 1) / kTextTokens);
+    long long want = (4 * 148 + ctas - 1) / ctas;  // about four CTAs per SM of a B200
+    if (want < 1) want = 1;
+    const int bps = (int)((nblk + want - 1) / want);  // centroid blocks per split
+    return (nblk + bps - 1) / bps;
+}
+
+struct TextPart {
+    float best, sec;
+    int idx, pad;
+};
+
+template <typename T, bool METRIC>
+__global__ __launch_bounds__(256) void k_text_partial(const T* __restrict__ X, int N, int D, int K, int row0,
+                                                      int splits, const T* __restrict__ C,
+                                                      const double* __restrict__ w64, const double* __restrict__ b64,
+                                                      TextPart* __restrict__ part) {
+    extern __shared__ __align__(16) float tsm[];
+    float* wsm = tsm;                        // [kTextBlock][D]
+    float* bsm = tsm + kTextBlock * D;       // [kTextBlock]
+    __shared__ float r_best[8][kTextTokens], r_sec[8][kTextTokens];
+    __shared__ int r_idx[8][kTextTokens];
+    const int bh = blockIdx.z, sp = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n_text = N - row0;
+    const int nblk = (K + kTextBlock - 1) / kTextBlock, bps = (nblk + splits - 1) / splits;
+    const int kb = sp * bps * kTextBlock, ke = min(K, (sp + 1) * bps * kTextBlock);
+    const int ta = blockIdx.x * kTextTokens + lane, tb = ta + 32;
+    const T* xa_p = X + ((size_t)bh * N + row0 + min(ta, n_text - 1)) * D;
+    const T* xb_p = X + ((size_t)bh * N + row0 + min(tb, n_text - 1)) * D;
+    const float INF = __int_as_float(0x7f800000);
+    float best0 = INF, sec0 = INF, best1 = INF, sec1 = INF;
+    int bi0 = kb, bi1 = kb;
+    for (int cb = kb; cb < ke; cb += kTextBlock) {
+        __syncthreads();  // the previous block is consumed
+        const int nb = min(kTextBlock, ke - cb);
+        for (int i = tid; i < kTextBlock * D; i += blockDim.x) {
+            const int j = i / D, d = i - j * D;
+            float v = 0.f;
+            if (j < nb) {
+                const size_t row = (size_t)bh * K + cb + j;
+                v = METRIC ? (float)w64[row * D + d] : Elem<T>::to_float(C + row * D, d);
+            }
+            wsm[i] = v;
+        }
+        for (int j = tid; j < kTextBlock; j += blockDim.x) bsm[j] = j < nb ? (float)b64[(size_t)bh * K + cb + j] : INF;
+        __syncthreads();
+        const int c0 = 16 * warp;
+        if (c0 >= nb) continue;
+        float acc0[16], acc1[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc0[j] = acc1[j] = 0.f;
+        float na = 0.f, nb2 = 0.f;
+        dot_rows<T, 16, false>(xa_p, xb_p, wsm + c0 * D, D, acc0, acc1, na, nb2);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (c0 + j < nb) {
+                const float b = bsm[c0 + j];
+                const float s0 = fmaf(-2.f, acc0[j], b), s1 = fmaf(-2.f, acc1[j], b);
+                const int k = cb + c0 + j;
+                if (s0 < best0) {
+                    sec0 = best0;
+                    best0 = s0;
+                    bi0 = k;
+                } else if (s0 < sec0) {
+                    sec0 = s0;
+                }
+                if (s1 < best1) {
+                    sec1 = best1;
+                    best1 = s1;
+                    bi1 = k;
+                } else if (s1 < sec1) {
+                    sec1 = s1;
+                }
+            }
+        }
+    }
+    r_best[warp][lane] = best0;
+    r_sec[warp][lane] = sec0;
+    r_idx[warp][lane] = bi0;
+    r_best[warp][lane + 32] = best1;
+    r_sec[warp][lane + 32] = sec1;
+    r_idx[warp][lane + 32] = bi1;
+    __syncthreads();
+    if (tid < kTextTokens) {
+        const int t = blockIdx.x * kTextTokens + tid;
+        int ww = 0;  // winner over the warps (ties: lowest index), runner-up over the rest
+        for (int w = 1; w < 8; ++w)
+            if (r_best[w][tid] < r_best[ww][tid] || (r_best[w][tid] == r_best[ww][tid] && r_idx[w][tid] < r_idx[ww][tid]))
+                ww = w;
+        float sec = r_sec[ww][tid];
+        for (int w = 0; w < 8; ++w)
+            if (w != ww) sec = fminf(sec, r_best[w][tid]);
+        if (t < n_text) part[((size_t)bh * n_text + t) * splits + sp] = TextPart{r_best[ww][tid], sec, r_idx[ww][tid], 0};
+    }
+}
+
+template <typename T, bool METRIC>
+__global__ __launch_bounds__(256) void k_text_finish(const T* __restrict__ X, int N, int D, int K, int row0,
+                                                     int splits, const T* __restrict__ C,
+                                                     const double* __restrict__ w64, const double* __restrict__ b64,
+                                                     const float* __restrict__ wmax, const float* __restrict__ bmax,
+                                                     const TextPart* __restrict__ part, int32_t* __restrict__ labels,
+                                                     int64_t* __restrict__ counters, int cnt_slot) {
+    __shared__ int s_list[8], s_n;
+    __shared__ double s_x[128];
+    __shared__ double s_bd[8];
+    __shared__ int s_bk[8];
+    const int bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n_text = N - row0;
+    const int t = blockIdx.x * 8 + warp;
+    if (tid == 0) s_n = 0;
+    __syncthreads();
+    if (t < n_text) {  // warp-uniform
+        const float INF = __int_as_float(0x7f800000);
+        float best = INF, sec = INF;
+        int idx = K;
+        if (lane < splits) {
+            const TextPart pp = part[((size_t)bh * n_text + t) * splits + lane];
+            best = pp.best;
+            sec = pp.sec;
+            idx = pp.idx;
+        }
+        for (int o = 16; o > 0; o >>= 1) {  // merge (best, idx, sec) over the splits
+            const float ob = __shfl_xor_sync(0xffffffffu, best, o), os = __shfl_xor_sync(0xffffffffu, sec, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, idx, o);
+            if (ob < best || (ob == best && oi < idx)) {
+                sec = fminf(best, os);
+                best = ob;
+                idx = oi;
+            } else {
+                sec = fminf(sec, ob);
+            }
+        }
+        const T* xp = X + ((size_t)bh * N + row0 + t) * D;
+        float nx = 0.f;
+        for (int j = lane; j < D; j += 32) {
+            const float v = Elem<T>::to_float(xp, j);
+            nx = fmaf(v, v, nx);
+        }
+        nx = warp_sum(nx);
+        const float u = 5.9604645e-8f;  // 2^-24
+        const float beta = 1.05f * (2.f * u * bmax[bh] + (2.f * D + 7.f) * u * sqrtf(nx) * 1.001f * wmax[bh]);
+        if (lane == 0) {
+            if (K == 1 || sec - best > 2.f * beta)
+                labels[(size_t)bh * N + row0 + t] = idx < K ? idx : 0;
+            else
+                s_list[atomicAdd(&s_n, 1)] = t;
+        }
+    }
+    __syncthreads();
+    // float64 rescore of the undecided tokens with the whole CTA: thread i scores
+    // centroids i, i + 256, ... (ascending), then a CTA argmin, ties to the lowest index
+    const int nlist = s_n;
+    for (int e = 0; e < nlist; ++e) {
+        const int tt = s_list[e];
+        const T* xp = X + ((size_t)bh * N + row0 + tt) * D;
+        for (int j = tid; j < D; j += blockDim.x) s_x[j] = Elem<T>::to_double(xp, j);
+        __syncthreads();
+        double bd = __longlong_as_double(0x7ff0000000000000ll);
+        int bk = 0;
+        for (int k = tid; k < K; k += blockDim.x) {
+            const size_t row = (size_t)bh * K + k;
+            double sc = 0.0;
+            if (METRIC) {
+                const double* wr = w64 + row * D;
+                for (int d = 0; d < D; ++d) sc = __fma_rn(s_x[d], wr[d], sc);
+                sc = b64[row] - 2.0 * sc;
+            } else {
+                const T* cr = C + row * D;
+                for (int d = 0; d < D; ++d) {
+                    const double df = s_x[d] - Elem<T>::to_double(cr, d);
+                    sc = __fma_rn(df, df, sc);
+                }
+            }
+            if (sc < bd) {
+                bd = sc;
+                bk = k;
+            }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            const double od = __shfl_xor_sync(0xffffffffu, bd, o);
+            const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
+            if (od < bd || (od == bd && ok < bk)) {
+                bd = od;
+                bk = ok;
+            }
+        }
+        if (lane == 0) {
+            s_bd[warp] = bd;
+            s_bk[warp] = bk;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            for (int w = 1; w < 8; ++w)
+                if (s_bd[w] < bd || (s_bd[w] == bd && s_bk[w] < bk)) {
+                    bd = s_bd[w];
+                    bk = s_bk[w];
+                }
+            labels[(size_t)bh * N + row0 + tt] = bk;
+        }
+        __syncthreads();
+    }
+    if (tid == 0 && nlist && counters)
+        atomicAdd((unsigned long long*)(counters + cnt_slot), (unsigned long long)nlist);
+}
+
+// enough for any K' <= K (the split count is not monotone in K)
+size_t text_scratch_bytes(int BH, int n_text, int K) {
+    if (n_text <= 0) return 0;
+    int most = 1;
+    for (int k = 1; k <= K; k += kTextBlock) most = max(most, text_splits(BH, n_text, k));
+    most = max(most, text_splits(BH, n_text, K));
+    return (size_t)BH * n_text * most * sizeof(TextPart);
+}
+
+int launch_assign_text(const void* X, int dtype, int BH, int N, int D, int K, int row0, const void* C,
+                       const double* w64, const double* b64, const float* wmax, const float* bmax, void* scratch,
+                       int32_t* labels, int64_t* counters, int cnt_slot, cudaStream_t st) {
+    if (D % 16 != 0 || D > 128) return PARK_ERR_UNSUPPORTED;
+    const int n_text = N - row0;
+    if (n_text <= 0) return PARK_OK;
+    const int splits = text_splits(BH, n_text, K);
+    const dim3 g1((n_text + kTextTokens - 1) / kTextTokens, splits, BH), g2((n_text + 7) / 8, BH);
+    const size_t sm = (size_t)kTextBlock * (D + 1) * sizeof(float);
+    TextPart* part = static_cast<TextPart*>(scratch);
+    const bool metric = w64 != nullptr;
+#define PARK_TEXT_LAUNCH(T, M)                                                                                     \
+    do {                                                                                                           \
+        cudaFuncSetAttribute(k_text_partial<T, M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);         \
+        ::park::prof_begin(st);                                                                                    \
+        k_text_partial<T, M><<<g1, 256, sm, st>>>((const T*)X, N, D, K, row0, splits, (const T*)C, w64, b64, part); \
+        PARK_TRY_LAUNCH("k_text_partial", st);                                                                     \
+        ::park::prof_begin(st);                                                                                    \
+        k_text_finish<T, M><<<g2, 256, 0, st>>>((const T*)X, N, D, K, row0, splits, (const T*)C, w64, b64, wmax,   \
+                                                bmax, part, labels, counters, cnt_slot);                            \
+        PARK_TRY_LAUNCH("k_text_finish", st);                                                                      \
+    } while (0)
+    if (dtype == PARK_BF16) {
+        if (metric) PARK_TEXT_LAUNCH(bf16_t, true);
+        else PARK_TEXT_LAUNCH(bf16_t, false);
+    } else {
+        if (metric) PARK_TEXT_LAUNCH(float, true);
+        else PARK_TEXT_LAUNCH(float, false);
+    }
+#undef PARK_TEXT_LAUNCH
+    return PARK_OK;
+}
+
 int launch_local_init(const void* X, int dtype, int BH, int N, int D, int K, const WinGeom& g, void* C,
                       cudaStream_t st) {
     ::park::prof_begin(st);
@@ -287,7 +558,7 @@ static void launch_local_t(dim3 grid, size_t sm, int kmax, cudaStream_t st, cons
 int launch_assign_local(const void* X, int dtype, int BH, int N, int D, int K, const WinGeom& g, const void* C,
                         const double* w64, const double* b64, const float* wmax, const float* bmax, int32_t* labels,
                         int64_t* counters, int cnt_slot, cudaStream_t st) {
-    if (D % 8 != 0 || D > 128) return PARK_ERR_UNSUPPORTED;
+    if (D % 16 != 0 || D > 128) return PARK_ERR_UNSUPPORTED;
     const int chunks = (g.maxwin + kLocalTokens - 1) / kLocalTokens;
     const dim3 grid(g.nW * chunks, BH);
     const size_t sm = local_assign_smem(K, g.nW, D);
@@ -393,111 +664,123 @@ __global__ void k_merge_planes(const int32_t* __restrict__ k_off, int NQ, int NK
     if (tid == 0) m.nb[bh] = 32 - __clz(s_max);
 }
 
-// One CTA per 8 groups g of a head: the best partner h of each (largest positive
-// gain, ties to the lowest h), -1 when no merge gains.  A pair is skipped
-// without counting when even a union adding no key rows could not gain:
-// ceil((n_g + n_h)/128) * max(T_g, T_h) >= cost_g + cost_h.
+// Kept units shared by groups g and h, I[g][h] = sum_b 2^b popc(S[g] & S[h] & P[b])
+// (symmetric), for the groups flagged in todo (first round: every live group,
+// each pair once from its lower index).  A pair that cannot gain whatever it
+// shares is stored as -1 without counting: ceil((n_g + n_h)/128) * max(T_g, T_h)
+// >= cost_g + cost_h, since the union keeps at least as many key tiles as
+// either group.  That test depends only on the two groups, so it stays true
+// until one of them merges, which puts it back in todo.
 constexpr int kMergeGroups = 8;
 
-__global__ __launch_bounds__(256) void k_merge_best(int NQ, int Wd, MergeWs m) {
+__global__ __launch_bounds__(256) void k_merge_inter(int NQ, int Wd, int first, MergeWs m) {
     extern __shared__ uint32_t gp[];  // [kMergeGroups][nb][Wd]: S[g] & P[b]
     __shared__ int sg_n[kMergeGroups], sg_L[kMergeGroups], sg_cost[kMergeGroups], sg_T[kMergeGroups];
-    __shared__ int red_gain[8][kMergeGroups], red_h[8][kMergeGroups];
+    __shared__ int s_any;
     const int bh = blockIdx.y, g0 = blockIdx.x * kMergeGroups, tid = threadIdx.x;
     if (m.done[bh]) return;
     const int nb = m.nb[bh];
     const size_t hb = (size_t)bh * NQ;
+    if (tid == 0) s_any = 0;
+    __syncthreads();
     if (tid < kMergeGroups) {
         const int g = g0 + tid;
-        const bool ok = g < NQ && m.alive[hb + g];
+        const bool ok = g < NQ && m.alive[hb + g] && (first || m.todo[hb + g]);
         sg_n[tid] = ok ? m.n[hb + g] : 0;
         sg_L[tid] = ok ? m.L[hb + g] : 0;
         sg_cost[tid] = ok ? merge_cost(sg_n[tid], sg_L[tid]) : -1;
         sg_T[tid] = ok ? (sg_L[tid] + 15) >> 4 : 0;
+        if (ok) atomicOr(&s_any, 1);
     }
+    __syncthreads();
+    if (!s_any) return;  // uniform
     for (int i = tid; i < kMergeGroups * nb * Wd; i += blockDim.x) {
         const int q = i / (nb * Wd), rem = i - q * nb * Wd, b = rem / Wd, w = rem - b * Wd;
         const int g = g0 + q;
-        gp[i] = g < NQ ? m.S[(hb + g) * Wd + w] & m.P[((size_t)bh * kMergePlanes + b) * Wd + w] : 0u;
+        gp[i] = (g < NQ && sg_cost[q] >= 0) ? m.S[(hb + g) * Wd + w] & m.P[((size_t)bh * kMergePlanes + b) * Wd + w]
+                                             : 0u;
     }
     __syncthreads();
-    int bgain[kMergeGroups], bh_idx[kMergeGroups];
-#pragma unroll
-    for (int q = 0; q < kMergeGroups; ++q) {
-        bgain[q] = 0;
-        bh_idx[q] = -1;
-    }
+    int32_t* I = m.inter + hb * NQ;
     for (int h = tid; h < NQ; h += blockDim.x) {
         if (!m.alive[hb + h]) continue;
         const int nh = m.n[hb + h], Lh = m.L[hb + h];
         const int Th = (Lh + 15) >> 4, ch = merge_cost(nh, Lh);
-        unsigned need = 0;
+        unsigned want = 0, need = 0;
 #pragma unroll
         for (int q = 0; q < kMergeGroups; ++q) {
-            if (sg_cost[q] >= 0 && g0 + q != h) {
+            const int g = g0 + q;
+            if (sg_cost[q] >= 0 && g != h && (!first || h > g)) {
+                want |= 1u << q;
                 const int A = (sg_n[q] + nh + 127) >> 7;
                 if (A * max(sg_T[q], Th) < sg_cost[q] + ch) need |= 1u << q;
             }
         }
-        if (!need) continue;
+        if (!want) continue;
         int inter[kMergeGroups];
 #pragma unroll
         for (int q = 0; q < kMergeGroups; ++q) inter[q] = 0;
-        const uint32_t* Sh = m.S + (hb + h) * Wd;
-        for (int w = 0; w < Wd; ++w) {
-            const uint32_t s = Sh[w];
-            if (!s) continue;
+        if (need) {
+            const uint32_t* Sh = m.S + (hb + h) * Wd;
+            for (int w = 0; w < Wd; ++w) {
+                const uint32_t sw = Sh[w];
+                if (!sw) continue;
 #pragma unroll
-            for (int q = 0; q < kMergeGroups; ++q) {
-                if ((need >> q) & 1u) {
-                    const uint32_t* gq = gp + (size_t)q * nb * Wd + w;
-                    int acc = 0;
-                    for (int b = 0; b < nb; ++b) acc += __popc(s & gq[b * Wd]) << b;
-                    inter[q] += acc;
+                for (int q = 0; q < kMergeGroups; ++q) {
+                    if ((need >> q) & 1u) {
+                        const uint32_t* gq = gp + (size_t)q * nb * Wd + w;
+                        int acc = 0;
+                        for (int b = 0; b < nb; ++b) acc += __popc(sw & gq[b * Wd]) << b;
+                        inter[q] += acc;
+                    }
                 }
             }
         }
 #pragma unroll
         for (int q = 0; q < kMergeGroups; ++q) {
-            if ((need >> q) & 1u) {
-                const int Lu = sg_L[q] + Lh - inter[q];
-                const int gain = sg_cost[q] + ch - merge_cost(sg_n[q] + nh, Lu);
-                if (gain > bgain[q]) {  // h ascends within a thread: strict keeps the lowest
-                    bgain[q] = gain;
-                    bh_idx[q] = h;
-                }
+            if ((want >> q) & 1u) {
+                const int g = g0 + q;
+                const int v = ((need >> q) & 1u) ? inter[q] : -1;
+                I[(size_t)g * NQ + h] = v;
+                I[(size_t)h * NQ + g] = v;
             }
         }
     }
-    // block argmax per group: largest gain, then lowest h
-    const int lane = tid & 31, warp = tid >> 5;
-#pragma unroll
-    for (int q = 0; q < kMergeGroups; ++q) {
-        int gq = bgain[q], hq = bh_idx[q];
-        for (int o = 16; o > 0; o >>= 1) {
-            const int go = __shfl_xor_sync(0xffffffffu, gq, o), ho = __shfl_xor_sync(0xffffffffu, hq, o);
-            if (go > gq || (go == gq && ho >= 0 && (hq < 0 || ho < hq))) {
-                gq = go;
-                hq = ho;
-            }
-        }
-        if (lane == 0) {
-            red_gain[warp][q] = gq;
-            red_h[warp][q] = hq;
+}
+
+// One warp per group g: the partner h with the largest gain
+// cost(g) + cost(h) - cost(g u h) > 0, ties to the lowest h; -1 if none.
+__global__ __launch_bounds__(256) void k_merge_pick(int NQ, MergeWs m) {
+    const int bh = blockIdx.y, lane = threadIdx.x & 31;
+    const int g = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (m.done[bh] || g >= NQ) return;  // warp-uniform
+    const size_t hb = (size_t)bh * NQ;
+    if (!m.alive[hb + g]) {
+        if (lane == 0) m.best[hb + g] = -1;
+        return;
+    }
+    const int ng = m.n[hb + g], Lg = m.L[hb + g], cg = merge_cost(ng, Lg);
+    const int32_t* I = m.inter + (hb + g) * NQ;
+    int bgain = 0, bidx = -1;
+    for (int h = lane; h < NQ; h += 32) {
+        if (h == g || !m.alive[hb + h]) continue;
+        const int it = I[h];
+        if (it < 0) continue;
+        const int nh = m.n[hb + h], Lh = m.L[hb + h];
+        const int gain = cg + merge_cost(nh, Lh) - merge_cost(ng + nh, Lg + Lh - it);
+        if (gain > bgain) {  // h ascends within a lane: strict keeps the lowest
+            bgain = gain;
+            bidx = h;
         }
     }
-    __syncthreads();
-    if (tid < kMergeGroups && g0 + tid < NQ) {
-        int gq = 0, hq = -1;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-            const int go = red_gain[w][tid], ho = red_h[w][tid];
-            if (go > gq || (go == gq && ho >= 0 && (hq < 0 || ho < hq))) {
-                gq = go;
-                hq = ho;
-            }
+    for (int o = 16; o > 0; o >>= 1) {
+        const int go = __shfl_xor_sync(0xffffffffu, bgain, o), ho = __shfl_xor_sync(0xffffffffu, bidx, o);
+        if (go > bgain || (go == bgain && ho >= 0 && (bidx < 0 || ho < bidx))) {
+            bgain = go;
+            bidx = ho;
         }
-        m.best[hb + g0 + tid] = gq > 0 ? hq : -1;
     }
+    if (lane == 0) m.best[hb + g] = bgain > 0 ? bidx : -1;
 }
 
 // Mutual best pairs merge into the lower index; a head with no merge is done.
@@ -511,7 +794,9 @@ __global__ void k_merge_apply(int NQ, int Wd, MergeWs m) {
     const int nb = m.nb[bh];
     for (int g = tid; g < NQ; g += blockDim.x) {
         const int h = m.best[hb + g];
-        if (h > g && m.best[hb + h] == g) {
+        const bool merge = h > g && m.best[hb + h] == g;
+        m.todo[hb + g] = merge;
+        if (merge) {
             uint32_t* Sg = m.S + (hb + g) * Wd;
             uint32_t* Sh = m.S + (hb + h) * Wd;
             int L = 0;
@@ -574,14 +859,18 @@ int launch_merge(uint8_t* mask, int32_t* kept_cnt, const int32_t* q_off, const i
     k_merge_planes<<<BH, 128, 0, st>>>(k_off, NQ, NK, Wd, m);
     PARK_TRY_LAUNCH("k_merge_planes", st);
     const size_t sm = (size_t)kMergeGroups * kMergePlanes * Wd * 4;
-    if (cudaFuncSetAttribute(k_merge_best, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess) {
+    if (cudaFuncSetAttribute(k_merge_inter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess) {
         cudaGetLastError();
         return PARK_ERR_CUDA;
     }
+    const dim3 gg((NQ + kMergeGroups - 1) / kMergeGroups, BH);
     for (int it = 0; it < rounds; ++it) {
         ::park::prof_begin(st);
-        k_merge_best<<<dim3((NQ + kMergeGroups - 1) / kMergeGroups, BH), 256, sm, st>>>(NQ, Wd, m);
-        PARK_TRY_LAUNCH("k_merge_best", st);
+        k_merge_inter<<<gg, 256, sm, st>>>(NQ, Wd, it == 0, m);
+        PARK_TRY_LAUNCH("k_merge_inter", st);
+        ::park::prof_begin(st);
+        k_merge_pick<<<dim3((NQ + 7) / 8, BH), 256, 0, st>>>(NQ, m);
+        PARK_TRY_LAUNCH("k_merge_pick", st);
         ::park::prof_begin(st);
         k_merge_apply<<<BH, 1024, 0, st>>>(NQ, Wd, m);
         PARK_TRY_LAUNCH("k_merge_apply", st);

@@ -97,13 +97,23 @@ int launch_assign_local(const void* X, int dtype, int BH, int N, int D, int K, c
                         const double* w64, const double* b64, const float* wmax, const float* bmax, int32_t* labels,
                         int64_t* counters, int cnt_slot, cudaStream_t st);
 size_t local_assign_smem(int K, int nW, int D);
+// Rows row0 .. N-1 of every head (the text tokens) against every centroid, with
+// the same float32 bound and float64 fallback as launch_assign_local; scratch
+// holds text_scratch_bytes(BH, N - row0, K).
+size_t text_scratch_bytes(int BH, int n_text, int K);
+int launch_assign_text(const void* X, int dtype, int BH, int N, int D, int K, int row0, const void* C,
+                       const double* w64, const double* b64, const float* wmax, const float* bmax, void* scratch,
+                       int32_t* labels, int64_t* counters, int cnt_slot, cudaStream_t st);
 // Query-cluster merging state, per head: S [NQ][Wd] kept-set bitsets, P
-// [kMergePlanes][Wd] bit planes of the key clusters' 8-row unit counts.
+// [kMergePlanes][Wd] bit planes of the key clusters' 8-row unit counts, inter
+// [NQ][NQ] the kept units two groups share (-1: the pair cannot gain).
 constexpr int kMergePlanes = 18;  // unit counts are below 2^18 (N <= 2^20)
+constexpr int kMergeMaxNQ = 2048;
 struct MergeWs {
     uint32_t* S;
     uint32_t* P;
-    int32_t *n, *L, *alive, *root, *best, *rootf, *done, *nb;
+    int32_t* inter;
+    int32_t *n, *L, *alive, *root, *best, *rootf, *todo, *done, *nb;
 };
 // Rewrites mask rows and kept counts of the merged groups and moves q_labels to
 // the groups' roots; `rounds` parallel rounds at most.

@@ -123,7 +123,7 @@ int metric_chunks(const Dims& d) {
 
 struct RetrievalWs {
     size_t M, Mpart, xnorm_q, xnorm_k, wop, b32, b64, w64, wmax, bmax, lfull, lcnt, hist, rho, plist,
-        pcnt, kcnt, f64z, cperm, coff, mS, mP, mI, mH, total;
+        pcnt, kcnt, f64z, cperm, coff, mS, mP, mI, mX, mH, txt, total;
 };
 
 RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
@@ -154,8 +154,10 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
     const size_t Wd = (NK + 31) / 32;
     w.mS = c.take(BH * NQ * Wd * 4);
     w.mP = c.take(BH * kMergePlanes * Wd * 4);
-    w.mI = c.take(6 * BH * NQ * 4);  // n, L, alive, root, best, rootf
+    w.mI = c.take(7 * BH * NQ * 4);  // n, L, alive, root, best, rootf, todo
+    w.mX = c.take(NQ <= kMergeMaxNQ ? BH * NQ * NQ * 4 : 0);
     w.mH = c.take(2 * BH * 4);       // done, nb
+    w.txt = c.take(text_scratch_bytes(d.BH, d.N - d.nvideo, (int)Km));
     w.total = c.off;
     return w;
 }
@@ -221,6 +223,8 @@ MergeWs merge_ws(void* ws, const RetrievalWs& w, int BH, int NQ) {
     m.root = a + 3 * s;
     m.best = a + 4 * s;
     m.rootf = a + 5 * s;
+    m.todo = a + 6 * s;
+    m.inter = at<int32_t>(ws, w.mX);
     m.done = at<int32_t>(ws, w.mH);
     m.nb = m.done + BH;
     return m;
@@ -284,8 +288,8 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
     lists.full_row = at<int32_t>(ws, w.lfull);
     lists.counts = at<int32_t>(ws, w.lcnt);
     if (s.win) {
-        // HVA local windows: float32-certified scores against the window's centroids,
-        // float64 for text tokens and for rows the bound cannot decide
+        // HVA local windows: float32-certified scores against the box's centroids (text
+        // tokens: against all), float64 for the rows the bound cannot decide
         ops.w = nullptr;
         if (!s.warm) PARK_CHECK(launch_local_init(s.X, d.dtype, BH, N, D, K, *s.win, s.C, st));
         for (int it = 0; it < iters; ++it) {
@@ -295,8 +299,9 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
             PARK_CHECK(launch_assign_local(s.X, d.dtype, BH, N, D, K, *s.win, s.C, ops.w64, ops.bias64, ops.wmax,
                                            ops.bmax, s.labels, counters, s.cnt_slot, st));
             if (s.n_text > 0)
-                PARK_CHECK(launch_recheck_rows(s.X, d.dtype, BH, N, D, K, s.C, ops.w64, ops.bias64, s.labels,
-                                               s.win->nvideo, num_sms, st));
+                PARK_CHECK(launch_assign_text(s.X, d.dtype, BH, N, D, K, s.win->nvideo, s.C, ops.w64, ops.bias64,
+                                              ops.wmax, ops.bmax, at<void>(ws, w.txt), s.labels, counters,
+                                              s.cnt_slot, st));
             PARK_CHECK(launch_label_sort(s.labels, BH, N, K, at<int32_t>(ws, w.hist), nchunks, s.perm, s.offsets, st));
             PARK_CHECK(launch_update(s.X, d.dtype, BH, N, D, K, s.perm, s.offsets, s.C, st));
         }
@@ -518,6 +523,7 @@ int park_retrieve(const void* Q, const void* K, const park_shape* shape, int NQ,
     if (!Q || !K || !ws || !retrieval_ptrs_ok(out)) return PARK_ERR_INVALID_ARG;
     if (!(p > 0.0f) || !std::isfinite(p) || iters < 1) return PARK_ERR_INVALID_ARG;
     if (!flags_ok(out, p)) return PARK_ERR_INVALID_ARG;
+    if ((out->flags & PARK_FLAG_MERGE_Q) && NQ > kMergeMaxNQ) return PARK_ERR_UNSUPPORTED;
     WinGeom geo;
     PARK_CHECK(window_geometry(out, d, NQ, NK, &geo));
     if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;
@@ -541,6 +547,7 @@ int park_layer(const void* Q, const void* K, const void* V, const park_shape* sh
     if (!Q || !K || !V || !O || !ws || !retrieval_ptrs_ok(out)) return PARK_ERR_INVALID_ARG;
     if (!(p > 0.0f) || !std::isfinite(p) || iters < 1) return PARK_ERR_INVALID_ARG;
     if (!flags_ok(out, p)) return PARK_ERR_INVALID_ARG;
+    if ((out->flags & PARK_FLAG_MERGE_Q) && NQ > kMergeMaxNQ) return PARK_ERR_UNSUPPORTED;
     WinGeom geo;
     PARK_CHECK(window_geometry(out, d, NQ, NK, &geo));
     if (ws_bytes < ws_bytes_for(d, NQ, NK)) return PARK_ERR_WORKSPACE;

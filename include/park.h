@@ -118,7 +118,8 @@ extern "C" {
  *                    offsets, centroids recomputed as exact means, mask and CSR
  *                    rows of merged-away clusters empty) except importance and
  *                    importance_bound, which keep the values the selection used.
- *                    Not combinable with SIP.
+ *                    Not combinable with SIP; NQ <= 2048 (else
+ *                    PARK_ERR_UNSUPPORTED).
  *   LOCAL_WINDOW     both K-means run on 3D local windows: the video grid is tiled
  *                    by boxes of window_t x window_h x window_w tokens (the last
  *                    box of an axis may be shorter; nW boxes, numbered with the
