@@ -22,7 +22,9 @@ pytestmark = pytest.mark.gpu
 
 # flag bits of park_retrieval.flags and the p passed (a retrieval ratio for top-k and SIP)
 VARIANTS = {"park (top-p 0.9)": (0x0, 0.9), "w/o QRKC": (0x4, 0.9), "w/o PAMA": (0x8, 0.9),
-            "top-k 0.3": (0x10, 0.3), "SIP 0.3": (0x40, 0.3), "size prior": (0x20, 0.9)}
+            "top-k 0.3": (0x10, 0.3), "SIP 0.3": (0x40, 0.3), "size prior": (0x20, 0.9),
+            "HVA merge": (0x80, 0.9), "HVA local 3x15x20": (0x100, 0.9), "HVA both": (0x180, 0.9)}
+WINDOW = (3, 15, 20)
 
 
 def test_variant_recall_tv_and_output_error():
@@ -38,7 +40,8 @@ def test_variant_recall_tv_and_output_error():
     U = torch.from_numpy(gen_uniform(cfg)).to(q.device)
     print()
     for name, (flags, p) in VARIANTS.items():
-        out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, q.device, sip_uniform=U if flags & 0x40 else None)
+        out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, q.device, sip_uniform=U if flags & 0x40 else None,
+                                   window=WINDOW if flags & 0x100 else None)
         out.flags = flags
         O, _ = park.layer(q, k, v, shape, cfg.NQ, cfg.NK, p, cfg.iters, out=out)
         torch.cuda.synchronize()
@@ -49,10 +52,12 @@ def test_variant_recall_tv_and_output_error():
         recall = po.block_recall(Q0, K0, ql, kl, mask, s, rows)
         tv = po.attention_tv(Q0[rows], K0, kl, cfg.NK, CK, s)
         live = np.bincount(kl, minlength=cfg.NK) > 0
-        kept = mask[:, live].mean()
+        qlive = np.bincount(ql, minlength=cfg.NQ) > 0
+        kept = mask[qlive][:, live].mean()
         Og = O[0, 0].float().cpu().numpy().astype(np.float64)[rows]
         err = np.linalg.norm(Og - dense) / np.linalg.norm(dense)
-        print(f"{name:18s} recall {recall:.4f}  TV {tv:.4f}  kept {kept:.4f}  output rel. error {err:.4f}")
+        print(f"{name:18s} recall {recall:.4f}  TV {tv:.4f}  kept {kept:.4f}  output rel. error {err:.4f}  "
+              f"key tiles {int(out.counters[7].item())}")
         assert 0.0 < recall <= 1.0 + 1e-9
         assert 0.0 <= tv <= 1.0
         assert np.isfinite(err)
