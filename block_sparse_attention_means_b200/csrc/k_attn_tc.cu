@@ -55,17 +55,18 @@ using namespace sm100;
 namespace {
 constexpr int TC_ROWS = 128;            // query rows and key rows per tile
 constexpr int TC_BLK = 16384;           // 128 rows x 128 bytes
-constexpr int TC_KST = 3;  // K ring stages (V: 2)
+constexpr int TC_KST = 3;  // K ring stages
+constexpr int TC_VST = 2;  // V ring stages (with the column bias)
 constexpr uint32_t TC_TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256,384)
 constexpr float kLog2eT = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
 
 struct TcSmem {
-    uint64_t q_full, q_empty, k_full[TC_KST], k_empty[TC_KST], v_full[2], v_empty[2], s_full[2], p_full[2], pv_done[2],
+    uint64_t q_full, q_empty, k_full[TC_KST], k_empty[TC_KST], v_full[TC_VST], v_empty[TC_VST], s_full[2], p_full[2], pv_done[2],
         o_empty, final_bar;
     uint32_t tmem_base;
     int abort;
-    alignas(16) float bias[2][TC_ROWS];  // per stage: 0 for a real key row, -inf for a pad row or past the end
+    alignas(16) float bias[TC_VST][TC_ROWS];  // per stage: 0 for a real key row, -inf for a pad row or past the end
     float xmax[2][2][TC_ROWS];           // [tile parity][column half][row]: tile maxima of the two halves
     float xl[2][TC_ROWS];                // [column half][row]: partial row sums
 };
@@ -94,7 +95,7 @@ __global__ void __launch_bounds__(352, 1)
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* Qs = base;
     uint8_t* Ks = base + 2 * TC_BLK;
-    uint8_t* Vs = Ks + 2 * TC_KST * TC_BLK;
+    uint8_t* Vs = Ks + 2 * TC_KST * TC_BLK;  // TC_VST stages follow
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort = &sh.abort;
@@ -105,9 +106,11 @@ __global__ void __launch_bounds__(352, 1)
             mbar_init(&sh.k_full[s], 1);
             mbar_init(&sh.k_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < TC_VST; ++s) {
             mbar_init(&sh.v_full[s], 1);
             mbar_init(&sh.v_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&sh.s_full[s], 1);
             mbar_init(&sh.p_full[s], 256);
             mbar_init(&sh.pv_done[s], 1);
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(352, 1)
         tmem_relinquish();
     }
     // K/V stages start as zeros: groups that are never loaded must hold finite values
-    for (int i = threadIdx.x; i < 2 * (TC_KST + 2) * TC_BLK / 16; i += blockDim.x)
+    for (int i = threadIdx.x; i < 2 * (TC_KST + TC_VST) * TC_BLK / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(Ks)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
     tc_fence_before();
@@ -141,8 +144,9 @@ __global__ void __launch_bounds__(352, 1)
         // so a V stage that waits for its PV never holds up the K loads.
         const bool isK = warp == 0;
         int T = 0, I = 0;
-        int k_last[TC_KST], v_last[2] = {-1, -1};
+        int k_last[TC_KST], v_last[TC_VST];
         for (int q = 0; q < TC_KST; ++q) k_last[q] = -1;
+        for (int q = 0; q < TC_VST; ++q) v_last[q] = -1;
         int q_pending = 0, q_parity = 0;
         for (int it = blockIdx.x; it < n_items && !warp_abort(abort); it += gridDim.x) {
             const WorkItem wi = items[it];
@@ -190,7 +194,7 @@ __global__ void __launch_bounds__(352, 1)
             load_entries(0);
             bool ok = true;
             for (int j = 0; j < nkt && ok; ++j) {
-                const int stg = T & 1, round = T >> 1;
+                const int stg = T % TC_VST, round = T / TC_VST;
                 int nvalid = 0;   // real key rows of group `lane` (lanes 0..15; V warp)
                 float lwv = 0.f;  // and the logit term of its segment
 #pragma unroll 4
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(352, 1)
             int dummy = 0;
             for (int s = 0; s < TC_KST; ++s)
                 if (k_last[s] >= 0) mbar_wait(&sh.k_full[s], k_last[s], &dummy, 100000000ull);
-            for (int s = 0; s < 2; ++s)
+            for (int s = 0; s < TC_VST; ++s)
                 if (v_last[s] >= 0) mbar_wait(&sh.v_full[s], v_last[s], &dummy, 100000000ull);
             if (q_pending) mbar_wait(&sh.q_full, q_parity, &dummy, 100000000ull);
         }
@@ -314,21 +318,21 @@ __global__ void __launch_bounds__(352, 1)
                 tc_fence_after();
                 bool ok = issue_S(G) && (nkt < 2 || issue_S(G + 1));
                 for (int j = 0; j < nkt && ok; ++j) {
-                    const int g = G + j, b = g & 1, ph = (g >> 1) & 1;
+                    const int g = G + j, b = g & 1, ph = (g >> 1) & 1, vs = g % TC_VST;
                     if (!mbar_wait(&sh.p_full[b], ph, abort) ||
                         (j == 0 && I > 0 && !mbar_wait(&sh.o_empty, (I - 1) & 1, abort)) ||
-                        !mbar_wait(&sh.v_full[b], ph, abort)) {
+                        !mbar_wait(&sh.v_full[vs], (g / TC_VST) & 1, abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t va = smem_u32(Vs + b * 2 * TC_BLK);
+                    const uint32_t va = smem_u32(Vs + vs * 2 * TC_BLK);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         umma_bf16_ts(tmem + 256, tmem + (uint32_t)(b * 128 + 8 * kk),
                                      sdesc_sw128(va + (uint32_t)kk * 4096, 1024, 2048), idPV, (j > 0 || kk > 0));
                     umma_commit(&sh.pv_done[b]);
-                    umma_commit(&sh.v_empty[b]);
+                    umma_commit(&sh.v_empty[vs]);
                     if (j + 2 < nkt && !issue_S(g + 2)) ok = false;
                 }
                 if (!ok) break;
@@ -365,8 +369,8 @@ __global__ void __launch_bounds__(352, 1)
             if (nkt == 0) continue;
             float m_ref = __int_as_float(0xff800000), l = 0.f;
             for (int j = 0; j < nkt; ++j) {
-                const int g = G + j, b = g & 1, ph = (g >> 1) & 1;
-                const bool live = wwait(&sh.s_full[b], ph) && wwait(&sh.v_full[b], ph);
+                const int g = G + j, b = g & 1, ph = (g >> 1) & 1, vs = g % TC_VST;
+                const bool live = wwait(&sh.s_full[b], ph) && wwait(&sh.v_full[vs], (g / TC_VST) & 1);
                 uint32_t s[2][32];
                 float tm[4] = {__int_as_float(0xff800000), __int_as_float(0xff800000), __int_as_float(0xff800000),
                                __int_as_float(0xff800000)};
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(352, 1)
                     tmem_ld_wait();
                     tmem_ld_dep(s[0]);
                     tmem_ld_dep(s[1]);
-                    const float4* bz = reinterpret_cast<const float4*>(sh.bias[b] + 64 * hc);
+                    const float4* bz = reinterpret_cast<const float4*>(sh.bias[vs] + 64 * hc);
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
 #pragma unroll
@@ -527,7 +531,7 @@ int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t
     return r == CUDA_SUCCESS ? PARK_OK : PARK_ERR_CUDA;
 }
 
-size_t attn_tc_smem_bytes() { return (size_t)(2 + 2 * TC_KST + 4) * TC_BLK + 1024; }  // Q, K ring, V x2
+size_t attn_tc_smem_bytes() { return (size_t)(2 + 2 * TC_KST + 2 * TC_VST) * TC_BLK + 1024; }  // Q, K and V rings
 
 int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
                           const int32_t* q_perm, const int2* segs, const float* segw, const int32_t* kept_ptr,
