@@ -776,19 +776,30 @@ int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int 
                     const float* sip_u, float* weight, const int32_t* list,
                     const int32_t* count, int all_clusters, int num_sms, int32_t* work_ctr, double* zscratch,
                     float* importance, float* importance_bound, uint8_t* mask, int32_t* kept_cnt, int64_t* counters,
-                    cudaStream_t st) {
+                    cudaStream_t st, int one_row) {
     if (NK > 4096 || D > 128) return PARK_ERR_UNSUPPORTED;
     const int NKP = next_pow2(NK);
     auto smem = [&](int RT) {
         return (size_t)128 * RT * 8 + (size_t)128 * F64_CH * 8 + (size_t)NKP * 8 + 16 * F64_CH * 8 + (size_t)NKP * 8 +
                (size_t)NKP * 4 + NKP;
     };
-    const bool big = smem(128) <= 227 * 1024;  // 128-row tiles when the sort buffers leave room
-    const size_t sm = smem(big ? 128 : 64);
+    // 128-row tiles when the sort buffers leave room; 32-row tiles when every
+    // cluster is a single row (the query centroids of "w/o PAMA")
+    const bool big = smem(128) <= 227 * 1024 && !one_row;
+    const size_t sm = smem(one_row ? 32 : big ? 128 : 64);
     const int blocks = num_sms < kPamaF64Slots ? num_sms : kPamaF64Slots;
     const double scale = 1.0 / sqrt((double)D);
     ::park::prof_begin(st);
-    if (dtype == PARK_BF16) {
+    if (one_row) {
+        if (dtype == PARK_BF16)
+            pama_f64_launch<bf16_t, 2>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, select, size_prior,
+                                       sip_u, weight, list, count, all_clusters, BH * NQ, work_ctr, zscratch,
+                                       importance, importance_bound, mask, kept_cnt, counters, sm, blocks, st);
+        else
+            pama_f64_launch<float, 2>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, select, size_prior,
+                                      sip_u, weight, list, count, all_clusters, BH * NQ, work_ctr, zscratch,
+                                      importance, importance_bound, mask, kept_cnt, counters, sm, blocks, st);
+    } else if (dtype == PARK_BF16) {
         if (big)
             pama_f64_launch<bf16_t, 8>(Q, q_perm, q_off, CK, k_off, N, D, NQ, NK, NKP, scale, p, select, size_prior, sip_u, weight, list, count,
                                        all_clusters, BH * NQ, work_ctr, zscratch, importance, importance_bound, mask,

@@ -70,7 +70,8 @@ int launch_topp(const float* importance, const float* rho, int BH, int NQ, int N
 int launch_centroid_rows(const int32_t* q_off, int BH, int NQ, int32_t* perm, int32_t* off, cudaStream_t st);
 // Float64 PAMA + top-p for the listed clusters (or all): at most kPamaF64Slots
 // CTAs, each with pama_f64_scratch_bytes(NK) / kPamaF64Slots bytes of float64
-// scratch; work_ctr (zeroed by the caller) hands out the clusters.
+// scratch; work_ctr (zeroed by the caller) hands out the clusters.  one_row:
+// every cluster has at most one row (32-row tiles instead of 128).
 constexpr int kPamaF64Slots = 160;
 size_t pama_f64_scratch_bytes(int NK);
 int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int NK, const int32_t* q_perm,
@@ -78,7 +79,7 @@ int launch_pama_f64(const void* Q, int dtype, int BH, int N, int D, int NQ, int 
                     const float* sip_u, float* weight, const int32_t* list,
                     const int32_t* count, int all_clusters, int num_sms, int32_t* work_ctr, double* zscratch,
                     float* importance, float* importance_bound, uint8_t* mask, int32_t* kept_cnt, int64_t* counters,
-                    cudaStream_t st);
+                    cudaStream_t st, int one_row = 0);
 int launch_kept_csr(const uint8_t* mask, const int32_t* kept_cnt, int BH, int NQ, int NK, int32_t* kept_ptr,
                     int32_t* kept_idx, int64_t* counters, cudaStream_t st);
 

@@ -425,7 +425,7 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
         PARK_CHECK(launch_pama_f64(out->q_centroids, d.dtype, BH, NQ, D, NQ, NK, cperm, coff, out->k_centroids,
                                    out->k_offsets, p, select, size_prior, sip_u, bw, nullptr, nullptr, 1, num_sms,
                                    at<int32_t>(ws, w.pcnt) + 4, at<double>(ws, w.f64z), out->importance,
-                                   out->importance_bound, out->mask, kcnt, out->counters, st));
+                                   out->importance_bound, out->mask, kcnt, out->counters, st, 1));
     } else if (d.dtype == PARK_BF16) {
         // max ||c_m|| over the final key centroids, for the PAMA bound
         CentroidOps ops{nullptr, D, at<float>(ws, w.b32), (int)align_up((size_t)(NQ > NK ? NQ : NK), 128),
