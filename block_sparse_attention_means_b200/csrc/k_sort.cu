@@ -175,11 +175,30 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
     }
     const int32_t* pm = perm + (size_t)bh * N + start;
     const T* Xh = X + (size_t)bh * N * D;
+    // bf16: float64 partial sums, exact for up to 1024 rows (members are multiples
+    // of 2^-27 below 2^16, so 1024 of them need at most 53 bits), moved into the
+    // int64 fixed-point accumulators every 1024 rows and at the end
+    double part[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) part[e] = 0.0;
+    int rows_in_part = 0;
+    auto flush = [&]() {
+        if (!TWO_LIMBS) {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                acc_hi[e] += __double2ll_rn(ldexp(part[e], Elem<T>::frac_bits));
+                part[e] = 0.0;
+            }
+        }
+        rows_in_part = 0;
+    };
     auto add_piece = [&](const uint4& v) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         if (!TWO_LIMBS) {
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) acc_hi[e] += fixed_bf16((uint16_t)(w[e >> 1] >> (16 * (e & 1))));
+            for (int e = 0; e < VEC; ++e)
+                part[e] += (double)__uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+            if (++rows_in_part == 1024) flush();
         } else {
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
@@ -203,6 +222,7 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
             for (int u = 0; u < 4; ++u) add_piece(v[u]);
         }
         for (; j < n; j += RPI) add_piece(*reinterpret_cast<const uint4*>(Xh + (size_t)pm[j] * D + piece * VEC));
+        flush();
     }
     long long* red_hi = red;
     long long* red_lo = red + RPI * D;

@@ -78,6 +78,10 @@ CONFIGS = {
                        _nclusters(75600, 128), _nclusters(75600, 128), 10, 0.9, True, "normal"),
     "hunyuan": LayerConfig("hunyuan", 1, 24, 33, 45, 80, 256, 128, "bf16",
                            _nclusters(119056, 128), _nclusters(119056, 128), 10, 0.9, True, "normal"),
+    # the PARK paper's own HunyuanVideo setting (its Table 7 row matching Table 3's PARK row):
+    # 128 query centroids, 1024 key centroids; context beside the pages' PAMA timings
+    "hunyuan_nq128_nk1024": LayerConfig("hunyuan_nq128_nk1024", 1, 24, 33, 45, 80, 256, 128, "bf16",
+                                        128, 1024, 10, 0.9, True, "normal"),
 }
 
 
