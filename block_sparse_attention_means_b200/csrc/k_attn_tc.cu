@@ -352,6 +352,7 @@ __global__ void __launch_bounds__(352, 1)
         const int row = 32 * quad + lane;
         const uint32_t trow = tmem + ((uint32_t)(32 * quad) << 16);
         const int pair_bar = 1 + quad;  // named barrier of warps w and w+4 (64 threads)
+        const float2 sl2e2 = make_float2(sl2e, sl2e);
         int G = 0;
         // Waits are decided per warp (tcgen05.ld/st and shuffles are warp-collective).
         // The two warps of a pair pass their named barrier the same number of times
@@ -367,7 +368,8 @@ __global__ void __launch_bounds__(352, 1)
             const int L = kv_len[(size_t)wi.bh * NQ + wi.r];
             const int nkt = (L + TC_ROWS - 1) / TC_ROWS;
             if (nkt == 0) continue;
-            float m_ref = __int_as_float(0xff800000), l = 0.f;
+            float m_ref = __int_as_float(0xff800000);
+            float2 l2 = make_float2(0.f, 0.f);  // partial row sums of the even and odd columns
             for (int j = 0; j < nkt; ++j) {
                 const int g = G + j, b = g & 1, ph = (g >> 1) & 1, vs = g % TC_VST;
                 const bool live = wwait(&sh.s_full[b], ph) && wwait(&sh.v_full[vs], (g / TC_VST) & 1);
@@ -386,19 +388,21 @@ __global__ void __launch_bounds__(352, 1)
                     for (int c = 0; c < 2; ++c) {
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
+                            // packed float32 pairs: one FMA instruction per two elements
                             const float4 bb = bz[c * 8 + q];
-                            const float x0 = fmaf(bits_f(s[c][4 * q + 0]), sl2e, bb.x);
-                            const float x1 = fmaf(bits_f(s[c][4 * q + 1]), sl2e, bb.y);
-                            const float x2 = fmaf(bits_f(s[c][4 * q + 2]), sl2e, bb.z);
-                            const float x3 = fmaf(bits_f(s[c][4 * q + 3]), sl2e, bb.w);
-                            s[c][4 * q + 0] = __float_as_uint(x0);
-                            s[c][4 * q + 1] = __float_as_uint(x1);
-                            s[c][4 * q + 2] = __float_as_uint(x2);
-                            s[c][4 * q + 3] = __float_as_uint(x3);
-                            tm[0] = fmaxf(tm[0], x0);
-                            tm[1] = fmaxf(tm[1], x1);
-                            tm[2] = fmaxf(tm[2], x2);
-                            tm[3] = fmaxf(tm[3], x3);
+                            const float2 x01 = __ffma2_rn(make_float2(bits_f(s[c][4 * q]), bits_f(s[c][4 * q + 1])),
+                                                          sl2e2, make_float2(bb.x, bb.y));
+                            const float2 x23 = __ffma2_rn(
+                                make_float2(bits_f(s[c][4 * q + 2]), bits_f(s[c][4 * q + 3])), sl2e2,
+                                make_float2(bb.z, bb.w));
+                            s[c][4 * q + 0] = __float_as_uint(x01.x);
+                            s[c][4 * q + 1] = __float_as_uint(x01.y);
+                            s[c][4 * q + 2] = __float_as_uint(x23.x);
+                            s[c][4 * q + 3] = __float_as_uint(x23.y);
+                            tm[0] = fmaxf(tm[0], x01.x);
+                            tm[1] = fmaxf(tm[1], x01.y);
+                            tm[2] = fmaxf(tm[2], x23.x);
+                            tm[3] = fmaxf(tm[3], x23.y);
                         }
                     }
                 }
@@ -431,19 +435,22 @@ __global__ void __launch_bounds__(352, 1)
                         tmem_st32(trow + 256u + (uint32_t)(64 * hc + 32 * c), o);
                     }
                     tmem_st_wait();
-                    l *= alpha;
+                    l2.x *= alpha;
+                    l2.y *= alpha;
                     m_ref = m_new;
                 }
                 // P (bf16 pairs) over the first 64 columns of buffer b: this half's 64
                 // keys are packed columns [32 hc, 32 hc + 32)
                 uint32_t pk[32];
+                const float2 nm2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = fast_ex2(bits_f(s[c][2 * e]) - m_ref);
-                        const float p1 = fast_ex2(bits_f(s[c][2 * e + 1]) - m_ref);
-                        l += p0 + p1;
+                        const float2 d = __fadd2_rn(make_float2(bits_f(s[c][2 * e]), bits_f(s[c][2 * e + 1])), nm2);
+                        const float p0 = fast_ex2(d.x);
+                        const float p1 = fast_ex2(d.y);
+                        l2 = __fadd2_rn(l2, make_float2(p0, p1));
                         __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
                         pk[16 * c + e] = *reinterpret_cast<uint32_t*>(&h);
                     }
@@ -455,7 +462,7 @@ __global__ void __launch_bounds__(352, 1)
             // epilogue: O / l, original token order; each thread writes its 64 columns.
             // The partner overwrites xl only after its next item's first pair barrier,
             // which this thread reaches after reading xl.
-            sh.xl[hc][row] = l;
+            sh.xl[hc][row] = l2.x + l2.y;
             named_bar_sync(pair_bar, 64);
             const float lt = sh.xl[0][row] + sh.xl[1][row];
             const int gl = G + nkt - 1;
