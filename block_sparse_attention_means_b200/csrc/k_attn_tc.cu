@@ -15,12 +15,13 @@
 // the part of a kept cluster that falls in a tile arrives with one bulk copy
 // for K and one for V; pad rows and groups past the end are masked.
 //
-// One CTA per SM (persistent, work items round-robin), 10 warps:
-//   warp 0     producer: Q tile (128 x 128, TMA) per item; K and V tiles (bulk
-//              copies, one per kept-cluster piece) into two 2-stage rings with
-//              separate barriers, so K of tile j+2 may arrive while V of tile
-//              j is still in use; a per-tile column bias (0 or -inf) for the
-//              masked rows;
+// One CTA per SM (persistent, work items round-robin), 11 warps:
+//   warp 0     producer: Q tile (128 x 128, TMA) per item and each key tile's K
+//              (bulk copies, one per kept-cluster piece) into a 3-stage ring;
+//   warp 10    producer: each key tile's V into a 2-stage ring, with the
+//              per-tile column bias (0, log2 w, or -inf for masked rows).  The
+//              two producers walk the same segment cursor, so K of tile j+3
+//              may arrive while V of tile j is still in use;
 //   warp 1     TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into TMEM
 //              buffer j%2 (128 x 128 fp32), O += P_j V_j into a TMEM
 //              accumulator (128 x 128 fp32) with P_j read from TMEM, in the
@@ -29,14 +30,15 @@
 //              read P_j from it.
 //   warps 2-9  Softmax, two threads per query row (= TMEM lane; warps w and
 //              w+4 share a lane quadrant), each owning 64 of a tile's 128
-//              columns.  Online Softmax in the log2 domain with a lazily
-//              updated reference max (O is rescaled in TMEM only when a row max
-//              grows by more than 2^8); the two halves exchange their tile
-//              maxima through shared memory so both use the same reference.
-//              P_j is written as bf16 pairs over the first 64 columns of S_j's
-//              TMEM buffer (the A operand of the PV MMA).  At the end the two
-//              partial row sums are added, and each thread normalises and
-//              writes its half of the O row in original token order.
+//              columns, with packed float32 pair arithmetic.  Online Softmax in
+//              the log2 domain with a lazily updated reference max (O is
+//              rescaled in TMEM only when a row max grows by more than 2^8);
+//              the two halves exchange their tile maxima through shared memory
+//              so both use the same reference.  P_j is written as bf16 pairs
+//              over the first 64 columns of S_j's TMEM buffer (the A operand of
+//              the PV MMA).  At the end the two partial row sums are added, and
+//              each thread normalises and writes its half of the O row in
+//              original token order.
 // Every wait is time-bounded; a timeout sets PARK_ERR_TIMEOUT in the status
 // word, the roles leave their loops, outstanding copies and MMAs are waited
 // for (bounded) and TMEM is freed before the CTA exits.  Decisions that guard
