@@ -86,18 +86,9 @@ __device__ inline bool in_range_exp(int e, uint32_t magnitude_bits) {
 }
 
 // ---------------------------------------------------------------- fixed point
-// Exact fixed-point image of an input element: F = x * 2^frac_bits (integer).
-// For both bf16 and f32 the left shift of the integer significand is e - 107.
-__device__ inline long long fixed_bf16(uint16_t b) {
-    int e = (b >> 7) & 0xFF;
-    if (e == 0) return 0;
-    long long m = (long long)(0x80 | (b & 0x7F));
-    int sh = e - 107;
-    sh = sh < 0 ? 0 : (sh > 40 ? 40 : sh);  // out-of-range inputs are reported, not summed exactly
-    long long v = m << sh;
-    return (b & 0x8000) ? -v : v;
-}
-
+// Exact fixed-point image of a float32 input element: F = x * 2^43 (integer);
+// the left shift of the integer significand is e - 107.  Out-of-range inputs
+// are reported by the input check, not summed exactly.
 __device__ inline long long fixed_f32(uint32_t u) {
     int e = (u >> 23) & 0xFF;
     if (e == 0) return 0;
