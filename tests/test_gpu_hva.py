@@ -16,7 +16,7 @@ import parity_util as pu
 pytestmark = pytest.mark.gpu
 
 # box (frames, rows, columns) per config: 8 boxes each
-WINDOWS = {"tiny": (2, 4, 4), "small": (4, 8, 8), "small_text": (4, 8, 8)}
+WINDOWS = {"tiny": (2, 4, 4), "small": (4, 8, 8), "small_text": (4, 8, 8), "small_ragged": (3, 5, 6)}
 
 
 @pytest.fixture(scope="module")
@@ -30,30 +30,36 @@ def park():
 def _cfg(name):
     if name == "small_text":
         return CONFIGS["small"].replace(name="small_text", H=2, n_text=64)
+    if name == "small_ragged":  # boxes clipped at every grid edge, 1-2 centroids per box, text tokens
+        return CONFIGS["small"].replace(name="small_ragged", H=2, n_text=24, NQ=48, NK=40)
     return CONFIGS[name]
 
 
-def _run(park, name, window=None, merge=False, rounds=0):
+def _run(park, name, window=None, merge=False, rounds=0, flags=0, p=None):
     cfg = _cfg(name)
     Q, K, V = gen_layer(cfg, 0)
     kw = {}
+    if flags & 0x10:
+        kw.update(topk_ratio=p)
     if window is not None:
         kw.update(grid=(cfg.T, cfg.Hg, cfg.W), window=window)
     if merge:
         kw.update(merge=True, merge_rounds=rounds or 8)
-    ref = po.layer(Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64), cfg.NQ, cfg.NK, cfg.p,
+    p = cfg.p if p is None else p
+    ref = po.layer(Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64), cfg.NQ, cfg.NK, p,
                    cfg.iters, cfg.dtype, **kw)
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     shape = park.Shape.of(cfg, dt)
     q, k, v = (pu.to_device(x, dt) for x in (Q, K, V))
     out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, q.device, window=window, merge=merge, merge_rounds=rounds)
-    O, r = park.layer(q, k, v, shape, cfg.NQ, cfg.NK, cfg.p, cfg.iters, out=out)
+    out.flags |= flags
+    O, r = park.layer(q, k, v, shape, cfg.NQ, cfg.NK, p, cfg.iters, out=out)
     torch.cuda.synchronize()
     assert r.status_code() == 0, f"device status {r.status_code()}"
     return cfg, ref, O, r
 
 
-@pytest.mark.parametrize("name", ["tiny", "small", "small_text"])
+@pytest.mark.parametrize("name", ["tiny", "small", "small_text", "small_ragged"])
 def test_local_window_matches_oracle(park, name):
     cfg, ref, O, r = _run(park, name, window=WINDOWS[name])
     fails = pu.compare_retrieval(r, ref, cfg.NQ, cfg.NK)
@@ -85,6 +91,14 @@ def test_merge_round_cap_matches_oracle(park):
     cfg, ref, O, r = _run(park, "small", merge=True, rounds=1)
     fails = pu.compare_retrieval(r, ref, cfg.NQ, cfg.NK)
     assert not fails, "\n".join(fails[:20])
+
+
+def test_merge_with_topk_and_ragged_windows(park):
+    ratio = float(np.float32(0.3))
+    cfg, ref, O, r = _run(park, "small_ragged", window=WINDOWS["small_ragged"], merge=True, flags=0x10, p=ratio)
+    fails = pu.compare_retrieval(r, ref, cfg.NQ, cfg.NK)
+    assert not fails, "\n".join(fails[:20])
+    pu.assert_output_close(O, ref, False)
 
 
 def test_local_window_and_merge_together(park):
