@@ -245,7 +245,7 @@ def hva_window(cfg):
 
 KERNEL_SOURCES = {"k_sparse_attn_tc": ["block_sparse_attention_means_b200/csrc/k_attn_tc.cu"],
                   "k_assign_tc": ["block_sparse_attention_means_b200/csrc/k_assign_tc.cu"],
-                  "k_pama_mma": ["block_sparse_attention_means_b200/csrc/k_pama.cu"],
+                  "k_pama_tc": ["block_sparse_attention_means_b200/csrc/k_pama_tc.cu"],
                   "k_pama_f64": ["block_sparse_attention_means_b200/csrc/k_pama.cu"],
                   "k_metric_partial": ["block_sparse_attention_means_b200/csrc/k_prep.cu"]}
 ATTENTION_KERNELS = ("k_sparse_attn_tc", "k_gather_rows", "k_attn_schedule", "k_kv_pad_gather", "k_kv_pad_offsets")
@@ -259,7 +259,7 @@ def kernel_roofline(name: str, ms_per_launch: float, cfg, counters, peaks, peak_
         work, bound, peak, unit = 4.0 * D * counters[5], "tensor", sustained, "TFLOP/s"
     elif name == "k_assign_tc":
         work, bound, peak, unit = 2.0 * BH * N * ((NQ + NK) / 2) * D, "tensor", sustained, "TFLOP/s"
-    elif name == "k_pama_mma":
+    elif name == "k_pama_tc":  # one pass of the score GEMM (the second pass is overhead)
         work, bound, peak, unit = 2.0 * BH * N * NK * D, "tensor", sustained, "TFLOP/s"
     elif name == "k_metric_partial":
         work, bound, peak, unit = 2.0 * BH * N * D * D, "alu", FP64_PEAK_TFLOPS, "TFLOP/s"

@@ -4,13 +4,10 @@
 // over the non-empty key clusters, P_im = softmax_m(q_i . c_m / sqrt(D)), and
 // I_rm is the mean of P_im over the members i of query cluster r.
 //
-// Fast path (bf16): one CTA per (query cluster, head) streams the cluster's
-// rows in 64-row tiles through two tensor-core passes over the key centroids:
-// pass 1 finds each row's max logit and Softmax denominator, pass 2 adds the
-// normalised probabilities into per-warp column sums.  Only the NQ x NK map is
-// written; per-query scores never reach memory (O(NQ*NK) extra memory, the
-// streamed form of PARK Appendix Table 6).  The kernel also writes a relative
-// error bound rho_r for the row of I.
+// Fast path (bf16): k_pama_tc.cu computes the NQ x NK importance map on the
+// tcgen05 tensor cores, streamed over the key centroids (per-query scores never
+// reach memory: O(NQ*NK) extra memory, the streamed form of PARK Appendix
+// Table 6), with a relative error bound rho_r for each row of I.
 //
 // top-p: per (query cluster, head) a bitonic sort (I descending, ties: lower m
 // first) and a float64 prefix sum give the shortest prefix reaching p.  The
@@ -18,216 +15,8 @@
 // recomputed entirely in float64 (k_pama_f64), which also serves the float32
 // input path for every row.
 #include "kernels.h"
-#include "mma_sync.cuh"
 
 namespace park {
-
-constexpr float kLog2e = 1.4426950408889634f;
-
-// ---------------------------------------------------------------- PAMA (bf16)
-__global__ __launch_bounds__(128) void k_pama_mma(const uint16_t* __restrict__ Q, const int32_t* __restrict__ q_perm,
-                                                  const int32_t* __restrict__ q_off, const uint16_t* __restrict__ CK,
-                                                  const int32_t* __restrict__ k_off, const float* __restrict__ qnorm,
-                                                  const float* __restrict__ ckmax, int N, int NQ, int NK, float sl2e,
-                                                  float delta_scale, int size_prior, float* __restrict__ importance,
-                                                  float* __restrict__ rho) {
-    constexpr int D = 128, CH = 64, LDS = D + 8;
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    uint16_t* Cs = reinterpret_cast<uint16_t*>(smem_raw);                       // [2][CH][LDS]
-    float* live = reinterpret_cast<float*>(smem_raw + 2 * CH * LDS * 2);        // [nch*CH] 0 or -inf
-    const int nch = (NK + CH - 1) / CH;
-    float* colsum = live + nch * CH;                                             // [4][nch*CH]
-    __shared__ float s_dmax[4];
-
-    const int r = blockIdx.x, bh = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-    const int qs = q_off[(size_t)bh * (NQ + 1) + r], nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - qs;
-    float* Irow = importance + ((size_t)bh * NQ + r) * NK;
-    if (nr == 0) {
-        for (int m = threadIdx.x; m < NK; m += blockDim.x) Irow[m] = 0.f;
-        if (threadIdx.x == 0) rho[(size_t)bh * NQ + r] = 0.f;
-        return;
-    }
-    const int32_t* ko = k_off + (size_t)bh * (NK + 1);
-    for (int m = threadIdx.x; m < nch * CH; m += blockDim.x) {
-        // additive logit term in log2 units: 0 (or log2 |B_m| with the size prior), -inf for empty m
-        const int nm = m < NK ? ko[m + 1] - ko[m] : 0;
-        live[m] = nm > 0 ? (size_prior ? (float)log2((double)nm) : 0.f) : __int_as_float(0xff800000);
-        for (int w = 0; w < 4; ++w) colsum[w * nch * CH + m] = 0.f;
-    }
-    const uint16_t* Ch = CK + (size_t)bh * NK * D;
-    const uint16_t* Qh = Q + (size_t)bh * N * D;
-    const int32_t* pm = q_perm + (size_t)bh * N + qs;
-    const float cmax = ckmax[bh];
-    float dmax = 0.f;
-
-    auto load_chunk = [&](int c, int stg) {
-        for (int e = threadIdx.x; e < CH * 16; e += 128) {
-            int rr = e >> 4, pc = e & 15, ci = c * CH + rr;
-            cp_async16(Cs + (stg * CH + rr) * LDS + pc * 8, Ch + (size_t)(ci < NK ? ci : NK - 1) * D + pc * 8,
-                       ci < NK ? 16 : 0);
-        }
-    };
-    auto scores = [&](int stg, const uint32_t (&a)[8][4], float (&acc)[8][4]) {
-        const uint16_t* Cst = Cs + stg * CH * LDS;
-        const int mi = lane >> 3, rr = lane & 7;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[nt][j] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4(b0, b1, b2, b3, Cst + (np * 16 + (mi >> 1) * 8 + rr) * LDS + kk * 16 + (mi & 1) * 8);
-                mma_bf16_16816(acc[2 * np], a[kk], b0, b1);
-                mma_bf16_16816(acc[2 * np + 1], a[kk], b2, b3);
-            }
-    };
-
-    for (int t0 = 0; t0 < nr; t0 += 64) {
-        const int lr0 = t0 + warp * 16 + g, lr1 = lr0 + 8;  // rows within the cluster
-        const bool v0 = lr0 < nr, v1 = lr1 < nr;
-        const int tok0 = v0 ? pm[lr0] : 0, tok1 = v1 ? pm[lr1] : 0;
-        uint32_t a[8][4];
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            int c0 = kk * 16 + 2 * tq;
-            a[kk][0] = v0 ? ld_u32(Qh + (size_t)tok0 * D + c0) : 0u;
-            a[kk][1] = v1 ? ld_u32(Qh + (size_t)tok1 * D + c0) : 0u;
-            a[kk][2] = v0 ? ld_u32(Qh + (size_t)tok0 * D + c0 + 8) : 0u;
-            a[kk][3] = v1 ? ld_u32(Qh + (size_t)tok1 * D + c0 + 8) : 0u;
-        }
-        if (tq == 0) {
-            if (v0) dmax = fmaxf(dmax, qnorm[(size_t)bh * N + tok0]);
-            if (v1) dmax = fmaxf(dmax, qnorm[(size_t)bh * N + tok1]);
-        }
-        // pass 1: row max and Softmax denominator (log2 domain)
-        float mrow[2] = {__int_as_float(0xff800000), __int_as_float(0xff800000)};
-        double lrow[2] = {0.0, 0.0};
-        __syncthreads();
-        load_chunk(0, 0);
-        cp_async_commit();
-        for (int c = 0; c < nch; ++c) {
-            const int stg = c & 1;
-            if (c + 1 < nch) load_chunk(c + 1, stg ^ 1);
-            cp_async_commit();
-            cp_async_wait<1>();
-            __syncthreads();
-            float acc[8][4];
-            scores(stg, a, acc);
-            float mloc[2] = {__int_as_float(0xff800000), __int_as_float(0xff800000)};
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float s = acc[nt][j] * sl2e + live[c * CH + nt * 8 + 2 * tq + (j & 1)];
-                    acc[nt][j] = s;
-                    mloc[j >> 1] = fmaxf(mloc[j >> 1], s);
-                }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], 1));
-                mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], 2));
-                float mn = fmaxf(mrow[h], mloc[h]);
-                if (mn != __int_as_float(0xff800000)) {
-                    lrow[h] *= (double)exp2f(mrow[h] - mn);
-                    mrow[h] = mn;
-                }
-            }
-            // rows whose max is still -inf have seen only empty clusters: nothing to add
-            const float mr0 = mrow[0] == __int_as_float(0xff800000) ? 0.f : mrow[0];
-            const float mr1 = mrow[1] == __int_as_float(0xff800000) ? 0.f : mrow[1];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) lrow[j >> 1] += (double)exp2f(acc[nt][j] - (j < 2 ? mr0 : mr1));
-            __syncthreads();
-        }
-        float inv[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
-            lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
-            inv[h] = (float)(1.0 / lrow[h]);
-        }
-        if (!v0) inv[0] = 0.f;
-        if (!v1) inv[1] = 0.f;
-        // pass 2: normalised probabilities summed over the tile's rows
-        load_chunk(0, 0);
-        cp_async_commit();
-        for (int c = 0; c < nch; ++c) {
-            const int stg = c & 1;
-            if (c + 1 < nch) load_chunk(c + 1, stg ^ 1);
-            cp_async_commit();
-            cp_async_wait<1>();
-            __syncthreads();
-            float acc[8][4];
-            scores(stg, a, acc);
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    int cl = nt * 8 + 2 * tq + j;
-                    float lv = live[c * CH + cl];
-                    float p0 = exp2f(acc[nt][j] * sl2e + lv - mrow[0]) * inv[0];
-                    float p1 = exp2f(acc[nt][j + 2] * sl2e + lv - mrow[1]) * inv[1];
-                    float s = p0 + p1;
-                    s += __shfl_xor_sync(0xffffffffu, s, 4);
-                    s += __shfl_xor_sync(0xffffffffu, s, 8);
-                    s += __shfl_xor_sync(0xffffffffu, s, 16);
-                    if (g == 0) colsum[warp * nch * CH + c * CH + cl] += s;
-                }
-            __syncthreads();
-        }
-    }
-    // importance row and its bound
-    dmax = warp_max(dmax);
-    if (lane == 0) s_dmax[warp] = dmax;
-    __syncthreads();
-    const float invn = 1.0f / (float)nr;
-    for (int m = threadIdx.x; m < NK; m += blockDim.x) {
-        float s = colsum[m] + colsum[nch * CH + m] + colsum[2 * nch * CH + m] + colsum[3 * nch * CH + m];
-        Irow[m] = s * invn;
-    }
-    if (threadIdx.x == 0) {
-        float qm = fmaxf(fmaxf(s_dmax[0], s_dmax[1]), fmaxf(s_dmax[2], s_dmax[3]));
-        // logit error bound (natural log units); then exp2 approximations (2^-21
-        // relative each, numerator and denominator), products, and the float32
-        // column sums (within-warp adds, one add per tile, warp sum, division)
-        double delta = (double)delta_scale * qm * cmax;
-        // the size prior's log2 |B_m| is rounded to float once: half an ulp of at most log2 N
-        if (size_prior) delta += 0.6931471805599453 * 5.9604644775390625e-8 * log2((double)N + 1.0);
-        double rr = expm1(2.0 * delta) + 4.0 * 4.76837158203125e-7 + (16.0 + nr / 64.0) * 5.9604644775390625e-8;
-        rho[(size_t)bh * NQ + r] = (float)(rr * 1.001);
-    }
-}
-
-int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t* q_perm, const int32_t* q_off,
-                    const void* CK, const int32_t* k_off, const float* qnorm, int size_prior, float* importance,
-                    float* rho, float* ckmax, cudaStream_t st) {
-    const int D = 128;
-    int nch = (NK + 63) / 64;
-    size_t sm = 2 * 64 * (D + 8) * 2 + (size_t)nch * 64 * 4 * 5;
-    cudaFuncSetAttribute(k_pama_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    float scale = 1.0f / sqrtf((float)D);
-    float sl2e = scale * kLog2e;
-    // |logit~ - logit| <= s (kappa 2^-24 + 2^-23) ||q|| max||c||: tensor-core fp32
-    // accumulation modelled as at most 2 half-ulps of the partial-sum bound per
-    // k-step (kappa = 2 D / 16 = 16 for D = 128; five times the largest error
-    // measured on this GPU over 8.4M bf16 dot products), plus the rounding of
-    // the scaled logit.  The GPU tests check the oracle's importance lies
-    // inside the resulting per-row bound.
-    const double kappa = 2.0 * D / 16.0;
-    float delta_scale =
-        (float)((1.0 / sqrt((double)D)) * (kappa * 5.9604644775390625e-8 + 1.1920928955078125e-7) * 1.01);
-    ::park::prof_begin(st);
-    k_pama_mma<<<dim3(NQ, BH), 128, sm, st>>>((const uint16_t*)Q, q_perm, q_off, (const uint16_t*)CK, k_off, qnorm,
-                                              ckmax, N, NQ, NK, sl2e, delta_scale, size_prior, importance, rho);
-    PARK_TRY_LAUNCH("k_pama_mma", st);
-    return PARK_OK;
-}
 
 // ---------------------------------------------------------------- sort helpers
 // Bitonic sort of n (power of two) (value, index) pairs: value descending,

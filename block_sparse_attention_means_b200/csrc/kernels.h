@@ -59,9 +59,12 @@ int launch_update(const void* X, int dtype, int BH, int N, int D, int K, const i
 // size_prior: logits gain log |B_m|.  select: 0 top-p; 1 top-k, the ceil(p L) most
 // important (p a ratio); 2 SIP with the uniforms sip_u, writing weight = 1/pi for
 // kept blocks and 0 elsewhere.
-int launch_pama_mma(const void* Q, int BH, int N, int NQ, int NK, const int32_t* q_perm, const int32_t* q_off,
-                    const void* CK, const int32_t* k_off, const float* qnorm, int size_prior, float* importance,
-                    float* rho, float* ckmax, cudaStream_t st);
+// k_pama_tc.cu: the importance map and its per-row relative bound rho on tcgen05,
+// from Q already gathered into cluster order (Qg [BH][N][128] bf16)
+int launch_pama_tc(const void* Qg, int BH, int N, int NQ, int NK, const int32_t* q_perm, const int32_t* q_off,
+                   const void* CK, const int32_t* k_off, const float* qnorm, int size_prior, float* importance,
+                   float* rho, const float* ckmax, int32_t* status, int num_sms, cudaStream_t st);
+size_t pama_tc_smem_bytes(int NK);
 int launch_topp(const float* importance, const float* rho, int BH, int NQ, int NK, const int32_t* q_off,
                 const int32_t* k_off, float p, int select, const float* sip_u, float* weight, uint8_t* mask,
                 int32_t* kept_cnt, float* importance_bound, int32_t* flag_list, int32_t* flag_count,

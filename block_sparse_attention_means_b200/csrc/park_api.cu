@@ -123,7 +123,7 @@ int metric_chunks(const Dims& d) {
 
 struct RetrievalWs {
     size_t M, Mpart, xnorm_q, xnorm_k, wop, b32, b64, w64, wmax, bmax, lfull, lcnt, hist, rho, plist,
-        pcnt, kcnt, f64z, cperm, coff, mS, mP, mI, mX, mH, txt, total;
+        pcnt, kcnt, f64z, cperm, coff, mS, mP, mI, mX, mH, txt, qg, total;
 };
 
 RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
@@ -158,6 +158,7 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
     w.mX = c.take(NQ <= kMergeMaxNQ ? BH * NQ * NQ * 4 : 0);
     w.mH = c.take(2 * BH * 4);       // done, nb
     w.txt = c.take(text_scratch_bytes(d.BH, d.N - d.nvideo, (int)Km));
+    w.qg = c.take(d.dtype == PARK_BF16 ? BH * N * D * 2 : 0);  // Q in query-cluster order, for PAMA
     w.total = c.off;
     return w;
 }
@@ -433,9 +434,11 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
         PARK_CHECK(memset_async(ops.wmax, (size_t)BH * 4, st));
         PARK_CHECK(memset_async(ops.bmax, (size_t)BH * 4, st));
         PARK_CHECK(launch_centroid_prep(out->k_centroids, d.dtype, BH, NK, D, nullptr, ops, st));
-        PARK_CHECK(launch_pama_mma(Q, BH, N, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids, out->k_offsets,
-                                   at<float>(ws, w.xnorm_q), size_prior, out->importance, at<float>(ws, w.rho),
-                                   ops.wmax, st));
+        void* Qg = at<void>(ws, w.qg);
+        PARK_CHECK(launch_gather(Q, d.dtype, BH, N, D, out->q_perm, Qg, st));
+        PARK_CHECK(launch_pama_tc(Qg, BH, N, NQ, NK, out->q_perm, out->q_offsets, out->k_centroids, out->k_offsets,
+                                  at<float>(ws, w.xnorm_q), size_prior, out->importance, at<float>(ws, w.rho),
+                                  ops.wmax, out->status, num_sms, st));
         PARK_CHECK(launch_topp(out->importance, at<float>(ws, w.rho), BH, NQ, NK, out->q_offsets, out->k_offsets, p,
                                select, sip_u, bw, out->mask, kcnt, out->importance_bound, at<int32_t>(ws, w.plist),
                                at<int32_t>(ws, w.pcnt), st));
