@@ -107,6 +107,9 @@ __global__ __launch_bounds__(256) void k_attn_schedule(int NQ, int NK, const int
                 it.r = r;
                 it.q_start = qs + q * tile_rows;
                 it.rows = min(tile_rows, nr - q * tile_rows);
+                it.g = -1;
+                it.g_start = 0;
+                it.g_rows = 0;
                 items[base + q] = it;
             }
             atomicAdd((unsigned long long*)(counters + PARK_CNT_KEPT_PAIRS),
@@ -131,6 +134,257 @@ int launch_attn_schedule(int BH, int NQ, int NK, const int32_t* q_off, const int
                                                   item_count, counters, tile_rows, pad8, poff, Npad, segs, bweight,
                                                   segw);
     PARK_TRY_LAUNCH("k_attn_schedule", st);
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- query-tile packing
+// One CTA per head, guests in cluster order.  A guest g (more than one 128-row
+// tile, last tile of rem rows) may join the single tile of a host h (1 <= n_h <=
+// 128 - rem, not yet taken): gain = T_g + T_h - T(g u h) key tiles, T(L) =
+// ceil(L / 16) for L kept 8-row groups, the shared groups counted from the bit
+// planes as in the merge.  The best positive gain wins, ties to the lowest h.
+__global__ __launch_bounds__(1024) void k_pack_pairs(int NQ, int Wd, MergeWs m, int32_t* __restrict__ pack_host,
+                                                     int32_t* __restrict__ pack_guest) {
+    extern __shared__ uint32_t pk_sm[];
+    uint32_t* sg = pk_sm;                           // [nb][Wd] guest S & P_b
+    uint32_t* taken = pk_sm + kMergePlanes * Wd;    // [ceil(NQ / 32)] hosts already used
+    __shared__ int red_gain[32], red_h[32];
+    const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t hb = (size_t)bh * NQ;
+    const int nb = m.nb[bh];
+    for (int r = tid; r < NQ; r += blockDim.x) {
+        pack_host[hb + r] = -1;
+        pack_guest[hb + r] = -1;
+    }
+    for (int i = tid; i < (NQ + 31) / 32; i += blockDim.x) taken[i] = 0u;
+    __syncthreads();
+    for (int g = 0; g < NQ; ++g) {
+        const int ng = m.n[hb + g];
+        if (ng <= 128) continue;  // uniform: not a guest
+        const int rem = ((ng - 1) & 127) + 1;
+        const int Lg = m.L[hb + g], Tg = (Lg + 15) >> 4;
+        for (int i = tid; i < nb * Wd; i += blockDim.x) {
+            const int b = i / Wd, w = i - b * Wd;
+            sg[i] = m.S[(hb + g) * Wd + w] & m.P[((size_t)bh * kMergePlanes + b) * Wd + w];
+        }
+        __syncthreads();
+        int bgain = 0, bidx = -1;
+        for (int h = tid; h < NQ; h += blockDim.x) {
+            const int nh = m.n[hb + h];
+            if (nh < 1 || nh > 128 - rem || ((taken[h >> 5] >> (h & 31)) & 1u)) continue;
+            const int Lh = m.L[hb + h], Th = (Lh + 15) >> 4;
+            int inter = 0;
+            const uint32_t* Sh = m.S + (hb + h) * Wd;
+            for (int w = 0; w < Wd; ++w) {
+                const uint32_t x = Sh[w];
+                if (!x) continue;
+                for (int b = 0; b < nb; ++b) inter += __popc(x & sg[b * Wd + w]) << b;
+            }
+            const int gain = Tg + Th - ((Lg + Lh - inter + 15) >> 4);
+            if (gain > bgain) {  // h ascends within a thread: strict keeps the lowest
+                bgain = gain;
+                bidx = h;
+            }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            const int go = __shfl_xor_sync(0xffffffffu, bgain, o), ho = __shfl_xor_sync(0xffffffffu, bidx, o);
+            if (go > bgain || (go == bgain && ho >= 0 && (bidx < 0 || ho < bidx))) {
+                bgain = go;
+                bidx = ho;
+            }
+        }
+        if (lane == 0) {
+            red_gain[warp] = bgain;
+            red_h[warp] = bidx;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int gq = 0, hq = -1;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+                const int go = red_gain[w], ho = red_h[w];
+                if (go > gq || (go == gq && ho >= 0 && (hq < 0 || ho < hq))) {
+                    gq = go;
+                    hq = ho;
+                }
+            }
+            if (gq > 0) {
+                pack_host[hb + g] = hq;
+                pack_guest[hb + hq] = g;
+                taken[hq >> 5] |= 1u << (hq & 31);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+int launch_pack_pairs(int BH, int NQ, int NK, const uint8_t* mask, const int32_t* q_off, const int32_t* k_off,
+                      const MergeWs& m, int32_t* pack_host, int32_t* pack_guest, cudaStream_t st) {
+    const int Wd = (NK + 31) / 32;
+    PARK_CHECK(launch_merge_setup(mask, q_off, k_off, BH, NQ, NK, m, st));
+    const size_t sm = (size_t)kMergePlanes * Wd * 4 + (size_t)((NQ + 31) / 32) * 4;
+    if (cudaFuncSetAttribute(k_pack_pairs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess) {
+        cudaGetLastError();
+        return PARK_ERR_CUDA;
+    }
+    ::park::prof_begin(st);
+    k_pack_pairs<<<BH, 1024, sm, st>>>(NQ, Wd, m, pack_host, pack_guest);
+    PARK_TRY_LAUNCH("k_pack_pairs", st);
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- schedule (tensor cores)
+// One CTA per (query cluster, head).  The slot's key list is the cluster's kept
+// set, or for a host the union with its guest's; entries in ascending m.
+__global__ __launch_bounds__(256) void k_attn_schedule_tc(int NQ, int NK, int Npad, const int32_t* __restrict__ q_off,
+                                                          const int32_t* __restrict__ k_off,
+                                                          const uint8_t* __restrict__ mask,
+                                                          const float* __restrict__ bweight,
+                                                          const int32_t* __restrict__ poff,
+                                                          const int32_t* __restrict__ pack_host,
+                                                          const int32_t* __restrict__ pack_guest,
+                                                          int32_t* __restrict__ kv_pre, int32_t* __restrict__ kv_len,
+                                                          int32_t* __restrict__ kv_nseg, int2* __restrict__ segs,
+                                                          float* __restrict__ segwA, float* __restrict__ segwB,
+                                                          WorkItem* __restrict__ items, int32_t* __restrict__ item_count,
+                                                          int64_t* __restrict__ counters) {
+    __shared__ int wcnt[8], wpad[8];
+    __shared__ long long wown[8];
+    const int r = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const size_t slot = (size_t)bh * NQ + r;
+    const int qs = q_off[(size_t)bh * (NQ + 1) + r], nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - qs;
+    const int g = pack_guest ? pack_guest[slot] : -1;  // guest hosted in r's tile
+    const int h = pack_host ? pack_host[slot] : -1;    // host of r's last tile
+    const uint8_t* mA = mask + slot * NK;
+    const uint8_t* mB = g >= 0 ? mask + ((size_t)bh * NQ + g) * NK : nullptr;
+    const int32_t* ko = k_off + (size_t)bh * (NK + 1);
+    const int32_t* po = poff + (size_t)bh * (NK + 1);
+    const int per = (NK + 255) / 256, m0 = t * per;
+    int cnt = 0, pad = 0;
+    long long own = 0;
+    for (int m = m0; m < m0 + per && m < NK; ++m) {
+        const bool a = mA[m] != 0, b = mB && mB[m] != 0;
+        if (a || b) {
+            const int sz = ko[m + 1] - ko[m];
+            ++cnt;
+            pad += (sz + 7) & ~7;
+            if (a) own += sz;
+        }
+    }
+    // block exclusive scans of the entry count and the padded rows
+    int ic = cnt, ip = pad;
+    long long so = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int yc = __shfl_up_sync(0xffffffffu, ic, o), yp = __shfl_up_sync(0xffffffffu, ip, o);
+        if (lane >= o) {
+            ic += yc;
+            ip += yp;
+        }
+        so += __shfl_xor_sync(0xffffffffu, so, o);
+    }
+    if (lane == 31) {
+        wcnt[w] = ic;
+        wpad[w] = ip;
+    }
+    if (lane == 0) wown[w] = so;
+    __syncthreads();
+    int ec = ic - cnt, ep = ip - pad, tot_c = 0, tot_p = 0;
+    long long tot_own = 0;
+    for (int q = 0; q < 8; ++q) {
+        if (q < w) {
+            ec += wcnt[q];
+            ep += wpad[q];
+        }
+        tot_c += wcnt[q];
+        tot_p += wpad[q];
+        tot_own += wown[q];
+    }
+    const float NI = __int_as_float(0xff800000);
+    const float* wA = bweight ? bweight + slot * NK : nullptr;
+    const float* wB = (bweight && g >= 0) ? bweight + ((size_t)bh * NQ + g) * NK : nullptr;
+    for (int m = m0; m < m0 + per && m < NK; ++m) {
+        const bool a = mA[m] != 0, b = mB && mB[m] != 0;
+        if (!(a || b)) continue;
+        const int sz = ko[m + 1] - ko[m];
+        const size_t e = slot * NK + ec;
+        kv_pre[e] = ep;
+        segs[e] = make_int2(bh * Npad + po[m], sz);
+        segwA[e] = a ? (wA ? (float)log2((double)wA[m]) : 0.f) : NI;
+        segwB[e] = b ? (wB ? (float)log2((double)wB[m]) : 0.f) : NI;
+        ++ec;
+        ep += (sz + 7) & ~7;
+    }
+    if (t == 0) {
+        kv_len[slot] = nr > 0 ? tot_p : 0;
+        kv_nseg[slot] = tot_c;
+        if (nr > 0 && tot_p > 0) {
+            const int tiles = (nr + 127) / 128;
+            const int own_items = h >= 0 ? tiles - 1 : tiles;  // a guest's last tile is in its host's item
+            int gs = 0, gr = 0;
+            if (g >= 0) {
+                const int gq = q_off[(size_t)bh * (NQ + 1) + g], gn = q_off[(size_t)bh * (NQ + 1) + g + 1] - gq;
+                gs = gq + 128 * ((gn - 1) / 128);
+                gr = gn - 128 * ((gn - 1) / 128);
+            }
+            const int base = atomicAdd(item_count, own_items);
+            for (int q = 0; q < own_items; ++q) {
+                WorkItem it;
+                it.bh = bh;
+                it.r = r;
+                it.q_start = qs + q * 128;
+                it.rows = min(128, nr - q * 128);
+                it.g = g;
+                it.g_start = gs;
+                it.g_rows = gr;
+                items[base + q] = it;
+            }
+            atomicAdd((unsigned long long*)(counters + PARK_CNT_KEPT_PAIRS),
+                      (unsigned long long)nr * (unsigned long long)tot_own);
+            atomicAdd((unsigned long long*)(counters + PARK_CNT_WORK_ITEMS), (unsigned long long)own_items);
+            atomicAdd((unsigned long long*)(counters + PARK_CNT_KEY_TILES),
+                      (unsigned long long)own_items * (unsigned long long)((tot_p + 127) / 128));
+        }
+    }
+}
+
+int launch_attn_schedule_tc(int BH, int NQ, int NK, int Npad, const int32_t* q_off, const int32_t* k_off,
+                            const uint8_t* mask, const float* bweight, const int32_t* poff, const int32_t* pack_host,
+                            const int32_t* pack_guest, int32_t* kv_pre, int32_t* kv_len, int32_t* kv_nseg,
+                            int2* segs, float* segwA, float* segwB, WorkItem* items, int32_t* item_count,
+                            int64_t* counters, cudaStream_t st) {
+    ::park::prof_begin(st);
+    k_attn_schedule_tc<<<dim3(NQ, BH), 256, 0, st>>>(NQ, NK, Npad, q_off, k_off, mask, bweight, poff, pack_host,
+                                                     pack_guest, kv_pre, kv_len, kv_nseg, segs, segwA, segwB, items,
+                                                     item_count, counters);
+    PARK_TRY_LAUNCH("k_attn_schedule", st);
+    return PARK_OK;
+}
+
+// ---------------------------------------------------------------- item-major Q
+__global__ void k_item_gather(const uint4* __restrict__ Q, int N, const int32_t* __restrict__ q_perm,
+                              const WorkItem* __restrict__ items, const int32_t* __restrict__ item_count,
+                              size_t item_cap, uint4* __restrict__ Qimg) {
+    constexpr int VPR = 16;  // 16-byte chunks per 128-element bf16 row
+    const size_t n = (size_t)min((size_t)*item_count, item_cap) * 128 * VPR;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+        const size_t rowi = e / VPR;
+        const int c = (int)(e - rowi * VPR);
+        const size_t it = rowi / 128;
+        const int row = (int)(rowi - it * 128);
+        const WorkItem wi = items[it];
+        const int grow = row - wi.rows;
+        int tok = -1;
+        if (row < wi.rows) tok = q_perm[(size_t)wi.bh * N + wi.q_start + row];
+        else if (grow < wi.g_rows) tok = q_perm[(size_t)wi.bh * N + wi.g_start + grow];
+        Qimg[e] = tok >= 0 ? Q[((size_t)wi.bh * N + tok) * VPR + c] : make_uint4(0, 0, 0, 0);
+    }
+}
+
+int launch_item_gather(const void* Q, int N, const int32_t* q_perm, const WorkItem* items, const int32_t* item_count,
+                       size_t item_cap, void* Qimg, int num_sms, cudaStream_t st) {
+    ::park::prof_begin(st);
+    k_item_gather<<<num_sms * 8, 256, 0, st>>>((const uint4*)Q, N, q_perm, items, item_count, item_cap, (uint4*)Qimg);
+    PARK_TRY_LAUNCH("k_item_gather", st);
     return PARK_OK;
 }
 

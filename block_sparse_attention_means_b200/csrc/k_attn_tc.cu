@@ -68,7 +68,9 @@ struct TcSmem {
         o_empty, final_bar;
     uint32_t tmem_base;
     int abort;
-    alignas(16) float bias[TC_VST][TC_ROWS];  // per stage: 0 for a real key row, -inf for a pad row or past the end
+    alignas(16) float bias[TC_VST][2][TC_ROWS];  // per stage, for the item's own rows [0] and its guest rows [1]:
+                                                 // the logit term of a real key row, -inf for a pad row, a row
+                                                 // past the end or a key cluster those query rows do not keep
     float xmax[2][2][TC_ROWS];           // [tile parity][column half][row]: tile maxima of the two halves
     float xl[2][TC_ROWS];                // [column half][row]: partial row sums
 };
@@ -86,8 +88,8 @@ __device__ __forceinline__ float fast_ex2(float x) {
 __global__ void __launch_bounds__(352, 1)
     k_sparse_attn_tc(const __grid_constant__ CUtensorMap tmQ, const uint8_t* __restrict__ Kimg,
                      const uint8_t* __restrict__ Vimg, int N, int NQ, int NK, const int32_t* __restrict__ q_perm,
-                     const int2* __restrict__ segs, const float* __restrict__ segw,
-                     const int32_t* __restrict__ kept_ptr,
+                     const int2* __restrict__ segs, const float* __restrict__ segwA,
+                     const float* __restrict__ segwB, const int32_t* __restrict__ kv_nseg,
                      const int32_t* __restrict__ kv_pre, const int32_t* __restrict__ kv_len,
                      const WorkItem* __restrict__ items, const int32_t* __restrict__ item_count,
                      uint16_t* __restrict__ O, float sl2e, int32_t* __restrict__ status) {
@@ -155,16 +157,17 @@ __global__ void __launch_bounds__(352, 1)
             const int L = kv_len[(size_t)wi.bh * NQ + wi.r];
             const int nkt = (L + TC_ROWS - 1) / TC_ROWS;
             if (nkt == 0) continue;
-            const int kp0 = kept_ptr[(size_t)wi.bh * (NQ + 1) + wi.r];
-            const int nk = kept_ptr[(size_t)wi.bh * (NQ + 1) + wi.r + 1] - kp0;
-            const int32_t* pre = kv_pre + (size_t)wi.bh * NQ * NK + kp0;
-            const int2* segs_item = segs + (size_t)wi.bh * NQ * NK + kp0;
-            const float* segw_item = segw ? segw + (size_t)wi.bh * NQ * NK + kp0 : nullptr;
+            const size_t slot = (size_t)wi.bh * NQ + wi.r;  // the item's key list, NK entries per slot
+            const int nk = kv_nseg[slot];
+            const int32_t* pre = kv_pre + slot * NK;
+            const int2* segs_item = segs + slot * NK;
+            const float* segwA_item = segwA + slot * NK;
+            const float* segwB_item = segwB + slot * NK;
             if (isK && lane == 0) {
                 bool ok = I == 0 || mbar_wait(&sh.q_empty, (I - 1) & 1, abort);
                 if (ok) {
                     mbar_arrive_expect_tx(&sh.q_full, 2 * TC_BLK);
-                    const int y = wi.bh * N + wi.q_start;
+                    const int y = it * TC_ROWS;  // the item's rows in the item-major Q image
                     tma_load_2d(Qs, &tmQ, &sh.q_full, 0, y);
                     tma_load_2d(Qs + TC_BLK, &tmQ, &sh.q_full, 64, y);
                     q_pending = 1;
@@ -177,7 +180,9 @@ __global__ void __launch_bounds__(352, 1)
             // segments (prefix of padded sizes, first padded row, size); a tile
             // spans at most 17 segments (each is >= 8 rows), so 32 lanes cover it.
             int seg0 = 0, p_l = 0x7fffffff, src_l = 0, sz_l = 0;
-            float lw_l = 0.f;  // additive logit term of the segment (log2 of its block weight)
+            // additive logit terms of the segment for the own and the guest rows (log2
+            // of the block weight, 0 without weights, -inf where those rows do not keep it)
+            float lwA_l = 0.f, lwB_l = 0.f;
             auto load_entries = [&](int s0) {
                 const int idx = s0 + lane;
                 if (idx < nk) {
@@ -185,20 +190,21 @@ __global__ void __launch_bounds__(352, 1)
                     const int2 e = segs_item[idx];
                     src_l = e.x;
                     sz_l = e.y;
-                    lw_l = segw_item ? segw_item[idx] : 0.f;
+                    lwA_l = segwA_item[idx];
+                    lwB_l = segwB_item[idx];
                 } else {
                     p_l = 0x7fffffff;
                     src_l = 0;
                     sz_l = 0;
-                    lw_l = 0.f;
+                    lwA_l = lwB_l = 0.f;
                 }
             };
             load_entries(0);
             bool ok = true;
             for (int j = 0; j < nkt && ok; ++j) {
                 const int stg = T % TC_VST, round = T / TC_VST;
-                int nvalid = 0;   // real key rows of group `lane` (lanes 0..15; V warp)
-                float lwv = 0.f;  // and the logit term of its segment
+                int nvalid = 0;                // real key rows of group `lane` (lanes 0..15; V warp)
+                float lwvA = 0.f, lwvB = 0.f;  // and the logit terms of its segment
 #pragma unroll 4
                 for (int g = 0; g < 16 && !isK; ++g) {
                     const int vg = j * TC_ROWS + 8 * g;
@@ -206,11 +212,13 @@ __global__ void __launch_bounds__(352, 1)
                     const int idx = (__popc(bal) - 1) & 31;
                     const int pp = __shfl_sync(0xffffffffu, p_l, idx);
                     const int sz = __shfl_sync(0xffffffffu, sz_l, idx);
-                    const float lw = __shfl_sync(0xffffffffu, lw_l, idx);
+                    const float lwa = __shfl_sync(0xffffffffu, lwA_l, idx);
+                    const float lwb = __shfl_sync(0xffffffffu, lwB_l, idx);
                     if (lane == g && vg < L) {
                         int nv = sz - (vg - pp);
                         nvalid = nv < 0 ? 0 : (nv > 8 ? 8 : nv);
-                        lwv = lw;
+                        lwvA = lwa;
+                        lwvB = lwb;
                     }
                 }
                 // this lane's segment (seg0 + lane) as one piece of whole 8-row groups of the tile
@@ -260,12 +268,16 @@ __global__ void __launch_bounds__(352, 1)
                         break;
                     }
                     if (lane < 16) {
-                        float4* bp = reinterpret_cast<float4*>(&sh.bias[stg][8 * lane]);
                         const float NI = __int_as_float(0xff800000);
-                        bp[0] = make_float4(nvalid > 0 ? lwv : NI, nvalid > 1 ? lwv : NI, nvalid > 2 ? lwv : NI,
-                                            nvalid > 3 ? lwv : NI);
-                        bp[1] = make_float4(nvalid > 4 ? lwv : NI, nvalid > 5 ? lwv : NI, nvalid > 6 ? lwv : NI,
-                                            nvalid > 7 ? lwv : NI);
+#pragma unroll
+                        for (int v = 0; v < 2; ++v) {
+                            const float lwv = v == 0 ? lwvA : lwvB;
+                            float4* bp = reinterpret_cast<float4*>(&sh.bias[stg][v][8 * lane]);
+                            bp[0] = make_float4(nvalid > 0 ? lwv : NI, nvalid > 1 ? lwv : NI, nvalid > 2 ? lwv : NI,
+                                                nvalid > 3 ? lwv : NI);
+                            bp[1] = make_float4(nvalid > 4 ? lwv : NI, nvalid > 5 ? lwv : NI, nvalid > 6 ? lwv : NI,
+                                                nvalid > 7 ? lwv : NI);
+                        }
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive_expect_tx(&sh.v_full[stg], tile_bytes);
@@ -385,7 +397,8 @@ __global__ void __launch_bounds__(352, 1)
                     tmem_ld_wait();
                     tmem_ld_dep(s[0]);
                     tmem_ld_dep(s[1]);
-                    const float4* bz = reinterpret_cast<const float4*>(sh.bias[vs] + 64 * hc);
+                    // the guest rows of a packed item [rows, rows + g_rows) keep their own key clusters
+                    const float4* bz = reinterpret_cast<const float4*>(sh.bias[vs][row < wi.rows ? 0 : 1] + 64 * hc);
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
 #pragma unroll
@@ -444,7 +457,10 @@ __global__ void __launch_bounds__(352, 1)
                 // P (bf16 pairs) over the first 64 columns of buffer b: this half's 64
                 // keys are packed columns [32 hc, 32 hc + 32)
                 uint32_t pk[32];
-                const float2 nm2 = make_float2(-m_ref, -m_ref);
+                // a row that has met only masked keys so far (the guest rows of a packed item
+                // can) keeps m_ref = -inf: its P is 0, and the first real maximum rescales O by 0
+                const float mr = m_ref == __int_as_float(0xff800000) ? 0.f : m_ref;
+                const float2 nm2 = make_float2(-mr, -mr);
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -479,9 +495,11 @@ __global__ void __launch_bounds__(352, 1)
             tmem_ld_dep(o[1]);
             tc_fence_before();
             mbar_arrive(&sh.o_empty);
-            if (row < wi.rows) {
+            const int grow = row - wi.rows;  // row of the guest part, if any
+            if (row < wi.rows || grow < wi.g_rows) {
                 const float inv = lt > 0.f ? 1.f / lt : 0.f;
-                const int tok = q_perm[(size_t)wi.bh * N + wi.q_start + row];
+                const int tok = row < wi.rows ? q_perm[(size_t)wi.bh * N + wi.q_start + row]
+                                              : q_perm[(size_t)wi.bh * N + wi.g_start + grow];
                 uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)wi.bh * N + tok) * 128 + 64 * hc);
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
@@ -542,19 +560,20 @@ int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t
 
 size_t attn_tc_smem_bytes() { return (size_t)(2 + 2 * TC_KST + 2 * TC_VST) * TC_BLK + 1024; }  // Q, K and V rings
 
-int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
-                          const int32_t* q_perm, const int2* segs, const float* segw, const int32_t* kept_ptr,
-                          const int32_t* kv_pre, const int32_t* kv_len,
+int launch_sparse_attn_tc(const void* Qimg, size_t item_cap, const void* Kpad, const void* Vpad, int BH, int N, int Npad,
+                          int NQ, int NK, const int32_t* q_perm, const int2* segs, const float* segwA,
+                          const float* segwB, const int32_t* kv_nseg, const int32_t* kv_pre, const int32_t* kv_len,
                           const WorkItem* items, const int32_t* item_count, void* O, int32_t* status, int num_sms,
                           cudaStream_t st) {
     CUtensorMap mQ;
-    PARK_CHECK(make_tma_map_bf16(&mQ, Qp, (uint64_t)BH * N, 128, 128));
+    PARK_CHECK(make_tma_map_bf16(&mQ, Qimg, (uint64_t)item_cap * TC_ROWS, 128, 128));
     const size_t sm = attn_tc_smem_bytes();
     cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     const float sl2e = (1.0f / sqrtf(128.f)) * kLog2eT;
     ::park::prof_begin(st);
     k_sparse_attn_tc<<<num_sms, 352, sm, st>>>(mQ, (const uint8_t*)Kpad, (const uint8_t*)Vpad, N, NQ, NK, q_perm,
-                                                segs, segw, kept_ptr, kv_pre, kv_len, items, item_count, (uint16_t*)O,
+                                                segs, segwA, segwB, kv_nseg, kv_pre, kv_len, items, item_count,
+                                                (uint16_t*)O,
                                                 sl2e, status);
     PARK_TRY_LAUNCH("k_sparse_attn_tc", st);
     return PARK_OK;

@@ -849,8 +849,8 @@ __global__ void k_merge_relabel(int BH, int N, int NQ, const int32_t* __restrict
     }
 }
 
-int launch_merge(uint8_t* mask, int32_t* kept_cnt, const int32_t* q_off, const int32_t* k_off, int BH, int N, int NQ,
-                 int NK, int rounds, const MergeWs& m, int32_t* q_labels, int num_sms, cudaStream_t st) {
+int launch_merge_setup(const uint8_t* mask, const int32_t* q_off, const int32_t* k_off, int BH, int NQ, int NK,
+                       const MergeWs& m, cudaStream_t st) {
     const int Wd = (NK + 31) / 32;
     ::park::prof_begin(st);
     k_merge_init<<<dim3(NQ, BH), 128, 0, st>>>(mask, q_off, k_off, NQ, NK, Wd, m);
@@ -858,6 +858,13 @@ int launch_merge(uint8_t* mask, int32_t* kept_cnt, const int32_t* q_off, const i
     ::park::prof_begin(st);
     k_merge_planes<<<BH, 128, 0, st>>>(k_off, NQ, NK, Wd, m);
     PARK_TRY_LAUNCH("k_merge_planes", st);
+    return PARK_OK;
+}
+
+int launch_merge(uint8_t* mask, int32_t* kept_cnt, const int32_t* q_off, const int32_t* k_off, int BH, int N, int NQ,
+                 int NK, int rounds, const MergeWs& m, int32_t* q_labels, int num_sms, cudaStream_t st) {
+    const int Wd = (NK + 31) / 32;
+    PARK_CHECK(launch_merge_setup(mask, q_off, k_off, BH, NQ, NK, m, st));
     const size_t sm = (size_t)kMergeGroups * kMergePlanes * Wd * 4;
     if (cudaFuncSetAttribute(k_merge_inter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess) {
         cudaGetLastError();

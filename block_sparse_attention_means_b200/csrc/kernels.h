@@ -119,14 +119,22 @@ struct MergeWs {
     int32_t* inter;
     int32_t *n, *L, *alive, *root, *best, *rootf, *todo, *done, *nb;
 };
+// S, n, L, alive, root, best, P and nb of a MergeWs from the masks (k_merge_init,
+// k_merge_planes).
+int launch_merge_setup(const uint8_t* mask, const int32_t* q_off, const int32_t* k_off, int BH, int NQ, int NK,
+                       const MergeWs& m, cudaStream_t st);
 // Rewrites mask rows and kept counts of the merged groups and moves q_labels to
 // the groups' roots; `rounds` parallel rounds at most.
 int launch_merge(uint8_t* mask, int32_t* kept_cnt, const int32_t* q_off, const int32_t* k_off, int BH, int N, int NQ,
                  int NK, int rounds, const MergeWs& m, int32_t* q_labels, int num_sms, cudaStream_t st);
 
 // ---- k_attn.cu
+// One query tile of the attention: rows [q_start, q_start + rows) of cluster r in
+// cluster order, and on the tensor-core path optionally the last tile of a guest
+// cluster g packed into the same tile (rows [g_start, g_start + g_rows), g = -1
+// when none).
 struct WorkItem {
-    int bh, r, q_start, rows;
+    int bh, r, q_start, rows, g, g_start, g_rows;
 };
 int launch_gather(const void* X, int dtype, int BH, int N, int D, const int32_t* perm, void* Xp, cudaStream_t st);
 // pad8: key cluster sizes rounded up to multiples of 8 in kv_pre / kv_len (the
@@ -147,9 +155,29 @@ size_t attn_tc_smem_bytes();
 // TMA descriptor for a row-major bf16 [rows][cols] tensor, boxes of 64 columns x
 // box_rows, 128-byte swizzle (k_attn_tc.cu).
 int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t cols, uint32_t box_rows);
-int launch_sparse_attn_tc(const void* Qp, const void* Kpad, const void* Vpad, int BH, int N, int Npad, int NQ, int NK,
-                          const int32_t* q_perm, const int2* segs, const float* segw, const int32_t* kept_ptr,
-                          const int32_t* kv_pre, const int32_t* kv_len,
+// Query-tile packing for the tensor-core path: the last tile of a query cluster
+// with several tiles (a guest) shares the single tile of a cluster with enough
+// free rows (its host) when the host tile's key list, the union of both kept
+// sets, needs fewer key tiles than the two tiles apart.  Greedy per head in
+// cluster order (best gain, ties to the lowest host).  Needs m.S / n / L / P / nb
+// from the merge initialisation (k_merge_init, k_merge_planes).
+int launch_pack_pairs(int BH, int NQ, int NK, const uint8_t* mask, const int32_t* q_off, const int32_t* k_off,
+                      const MergeWs& m, int32_t* pack_host, int32_t* pack_guest, cudaStream_t st);
+// Tensor-core schedule: per slot (bh, r) the key list at slot * NK (ascending m: padded prefix kv_pre, segs,
+// logit terms segwA for the own rows and segwB for the guest rows, -inf where not kept), kv_len, kv_nseg;
+// 128-row work items with their guests.  pack_host / pack_guest may be null (no packing).
+int launch_attn_schedule_tc(int BH, int NQ, int NK, int Npad, const int32_t* q_off, const int32_t* k_off,
+                            const uint8_t* mask, const float* bweight, const int32_t* poff, const int32_t* pack_host,
+                            const int32_t* pack_guest, int32_t* kv_pre, int32_t* kv_len, int32_t* kv_nseg,
+                            int2* segs, float* segwA, float* segwB, WorkItem* items, int32_t* item_count,
+                            int64_t* counters, cudaStream_t st);
+// Q rows of every work item into an item-major image: item i occupies rows
+// [128 i, 128 i + 128) (own rows, then guest rows, then zeros).
+int launch_item_gather(const void* Q, int N, const int32_t* q_perm, const WorkItem* items, const int32_t* item_count,
+                       size_t item_cap, void* Qimg, int num_sms, cudaStream_t st);
+int launch_sparse_attn_tc(const void* Qimg, size_t item_cap, const void* Kpad, const void* Vpad, int BH, int N, int Npad,
+                          int NQ, int NK, const int32_t* q_perm, const int2* segs, const float* segwA,
+                          const float* segwB, const int32_t* kv_nseg, const int32_t* kv_pre, const int32_t* kv_len,
                           const WorkItem* items, const int32_t* item_count, void* O, int32_t* status, int num_sms,
                           cudaStream_t st);
 int launch_sparse_attn_simt(const void* Q, const void* K, const void* V, int dtype, int BH, int N, int D, int NQ,

@@ -165,7 +165,8 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
 
 
 struct AttnWs {
-    size_t Qp, Kp, Vp, poff, segs, segw, items, icnt, kvpre, kvlen, total;
+    size_t Qimg, Kp, Vp, poff, segs, segw, segwB, kvnseg, pack, mS, mP, mI, mH, items, icnt, kvpre, kvlen, total;
+    size_t item_cap;  // tensor-core work items at most: sum_r ceil(n_r / 128) <= ceil(N / 128) + NQ per head
     int Npad;
 };
 
@@ -179,15 +180,26 @@ AttnWs plan_attn(const Dims& d, int NQ, int NK) {
     size_t BH = d.BH, N = d.N, D = d.D;
     size_t rowbytes = D * d.elt;
     w.Npad = padded_rows(d, NK);
+    w.item_cap = BH * ((N + kAttnTileTc - 1) / kAttnTileTc + (size_t)NQ);
     if (d.dtype == PARK_BF16) {
-        w.Qp = c.take(BH * N * rowbytes);
+        w.Qimg = c.take(w.item_cap * kAttnTileTc * rowbytes);
         w.Kp = c.take(BH * (size_t)w.Npad * rowbytes);
         w.Vp = c.take(BH * (size_t)w.Npad * rowbytes);
         w.poff = c.take(BH * (size_t)(NK + 1) * 4);
         w.segs = c.take(BH * (size_t)NQ * NK * 8);
         w.segw = c.take(BH * (size_t)NQ * NK * 4);
+        w.segwB = c.take(BH * (size_t)NQ * NK * 4);
+        w.kvnseg = c.take(BH * (size_t)NQ * 4);
+        const bool pk = NQ <= kMergeMaxNQ;  // query-tile packing (its state as in the merge)
+        const size_t Wd = (NK + 31) / 32;
+        w.pack = c.take(pk ? 2 * BH * (size_t)NQ * 4 : 0);
+        w.mS = c.take(pk ? BH * (size_t)NQ * Wd * 4 : 0);
+        w.mP = c.take(pk ? BH * kMergePlanes * Wd * 4 : 0);
+        w.mI = c.take(pk ? 7 * BH * (size_t)NQ * 4 : 0);
+        w.mH = c.take(pk ? 2 * BH * 4 : 0);
     } else {
-        w.Qp = w.Kp = w.Vp = w.poff = w.segs = w.segw = 0;
+        w.Qimg = w.Kp = w.Vp = w.poff = w.segs = w.segw = w.segwB = w.kvnseg = 0;
+        w.pack = w.mS = w.mP = w.mI = w.mH = 0;
     }
     size_t max_items = BH * ((N + kAttnTile - 1) / kAttnTile + (size_t)NQ);
     w.items = c.take(max_items * sizeof(WorkItem));
@@ -346,7 +358,7 @@ bool flags_ok(const park_retrieval* r, float p) {
     const uint32_t flags = r->flags;
     const uint32_t known = PARK_FLAG_WARM_START_Q | PARK_FLAG_WARM_START_K | PARK_FLAG_NO_QRKC |
                            PARK_FLAG_CENTROID_QUERY | PARK_FLAG_TOPK | PARK_FLAG_SIZE_PRIOR | PARK_FLAG_SIP |
-                           PARK_FLAG_MERGE_Q | PARK_FLAG_LOCAL_WINDOW;
+                           PARK_FLAG_MERGE_Q | PARK_FLAG_LOCAL_WINDOW | PARK_FLAG_NO_TILE_PACKING;
     if (flags & ~known) return false;
     if ((flags & (PARK_FLAG_TOPK | PARK_FLAG_SIP)) && p > 1.0f) return false;
     if ((flags & PARK_FLAG_TOPK) && (flags & PARK_FLAG_SIP)) return false;
@@ -486,21 +498,47 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
                                        r->kept_ptr, r->kept_idx, bw, O, st);
     }
     const int num_sms = num_sms_current();
-    void* Qp = at<void>(ws, w.Qp);
+    void* Qimg = at<void>(ws, w.Qimg);
     void* Kp = at<void>(ws, w.Kp);
     void* Vp = at<void>(ws, w.Vp);
     int32_t* poff = at<int32_t>(ws, w.poff);
     int2* segs = at<int2>(ws, w.segs);
-    float* segw = at<float>(ws, w.segw);
-    PARK_CHECK(launch_gather(Q, d.dtype, BH, N, D, r->q_perm, Qp, st));
+    float* segwA = at<float>(ws, w.segw);
+    float* segwB = at<float>(ws, w.segwB);
+    int32_t* kvnseg = at<int32_t>(ws, w.kvnseg);
+    WorkItem* items = at<WorkItem>(ws, w.items);
     PARK_CHECK(launch_kv_pad_gather(K, V, BH, N, NK, w.Npad, r->k_perm, r->k_labels, r->k_offsets, poff, Kp, Vp, st));
-    PARK_CHECK(launch_attn_schedule(BH, NQ, NK, r->q_offsets, r->k_offsets, r->kept_ptr, r->kept_idx,
-                                    at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
-                                    icnt, r->counters, kAttnTileTc, 1, poff, w.Npad, segs, bw, segw, st));
-    PARK_CHECK(launch_sparse_attn_tc(Qp, Kp, Vp, BH, N, w.Npad, NQ, NK, r->q_perm, segs, bw ? segw : nullptr,
-                                     r->kept_ptr,
-                                     at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
-                                     icnt, O, r->status, num_sms, st));
+    // query-tile packing: a guest's last tile shares its host's single tile (exact: every row keeps
+    // only its own cluster's key blocks)
+    int32_t* pack_host = nullptr;
+    int32_t* pack_guest = nullptr;
+    if (!(r->flags & PARK_FLAG_NO_TILE_PACKING) && NQ <= kMergeMaxNQ) {
+        pack_host = at<int32_t>(ws, w.pack);
+        pack_guest = pack_host + (size_t)BH * NQ;
+        MergeWs m;
+        m.S = at<uint32_t>(ws, w.mS);
+        m.P = at<uint32_t>(ws, w.mP);
+        m.inter = nullptr;
+        int32_t* a = at<int32_t>(ws, w.mI);
+        const size_t sN = (size_t)BH * NQ;
+        m.n = a;
+        m.L = a + sN;
+        m.alive = a + 2 * sN;
+        m.root = a + 3 * sN;
+        m.best = a + 4 * sN;
+        m.rootf = a + 5 * sN;
+        m.todo = a + 6 * sN;
+        m.done = at<int32_t>(ws, w.mH);
+        m.nb = m.done + BH;
+        PARK_CHECK(launch_pack_pairs(BH, NQ, NK, r->mask, r->q_offsets, r->k_offsets, m, pack_host, pack_guest, st));
+    }
+    PARK_CHECK(launch_attn_schedule_tc(BH, NQ, NK, w.Npad, r->q_offsets, r->k_offsets, r->mask, bw, poff, pack_host,
+                                       pack_guest, at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), kvnseg, segs,
+                                       segwA, segwB, items, icnt, r->counters, st));
+    PARK_CHECK(launch_item_gather(Q, N, r->q_perm, items, icnt, w.item_cap, Qimg, num_sms, st));
+    PARK_CHECK(launch_sparse_attn_tc(Qimg, w.item_cap, Kp, Vp, BH, N, w.Npad, NQ, NK, r->q_perm, segs, segwA, segwB,
+                                     kvnseg, at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), items, icnt, O,
+                                     r->status, num_sms, st));
     return PARK_OK;
 }
 

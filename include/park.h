@@ -132,6 +132,12 @@ extern "C" {
  *                    at most 256 centroids per box (else PARK_ERR_UNSUPPORTED). */
 #define PARK_FLAG_MERGE_Q 0x80u
 #define PARK_FLAG_LOCAL_WINDOW 0x100u
+/* Implementation switch, no change to the result (up to float32 summation
+ * order): on the bf16 path park_sparse_attn packs the last 128-row tile of a
+ * query cluster with several tiles into the single tile of a cluster with
+ * enough free rows when that needs fewer key tiles (every row still attends
+ * only to its own cluster's kept key clusters); this flag turns it off. */
+#define PARK_FLAG_NO_TILE_PACKING 0x200u
 
 /* ---- park_retrieval.counters indices (outputs, int64) ------------------ */
 #define PARK_CNT_Q_RECHECK 0    /* query rows whose bf16 score margin was not
