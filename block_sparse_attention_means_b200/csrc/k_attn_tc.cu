@@ -3,8 +3,12 @@
 // inclusion probabilities) the per-column bias of a real key row is log2 of its
 // block's weight instead of 0, which weights both Softmax sums.
 //
-// Layout: Q is gathered into cluster order (rows of a query cluster are
-// contiguous).  K and V are gathered into cluster order with every key
+// Work items are 128-row query tiles.  Q is gathered into an item-major image
+// (item i owns rows 128 i .. 128 i + 127).  Exact query-tile packing: the last
+// tile of a query cluster with several tiles (a guest) may share the single tile
+// of a smaller cluster (its host); the item's key list is then the union of both
+// kept sets, and each row masks the key clusters its own cluster does not keep
+// (two column-bias vectors per key tile: own rows, guest rows).  K and V are gathered into cluster order with every key
 // cluster padded to a multiple of 8 rows (zero rows), so a kept key cluster is
 // a run of whole 8-row groups.  For a query cluster, its kept key clusters are
 // concatenated (padded sizes) into one virtual key sequence that is cut into
@@ -19,7 +23,8 @@
 //   warp 0     producer: Q tile (128 x 128, TMA) per item and each key tile's K
 //              (bulk copies, one per kept-cluster piece) into a 3-stage ring;
 //   warp 10    producer: each key tile's V into a 2-stage ring, with the
-//              per-tile column bias (0, log2 w, or -inf for masked rows).  The
+//              per-tile column biases (0, log2 w, or -inf for masked rows) for
+//              the own and the guest rows.  The
 //              two producers walk the same segment cursor, so K of tile j+3
 //              may arrive while V of tile j is still in use;
 //   warp 1     TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into TMEM
