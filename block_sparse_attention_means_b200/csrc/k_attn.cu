@@ -138,40 +138,39 @@ int launch_attn_schedule(int BH, int NQ, int NK, const int32_t* q_off, const int
 }
 
 // ---------------------------------------------------------------- query-tile packing
-// One CTA per head, guests in cluster order.  A guest g (more than one 128-row
-// tile, last tile of rem rows) may join the single tile of a host h (1 <= n_h <=
-// 128 - rem, not yet taken): gain = T_g + T_h - T(g u h) key tiles, T(L) =
-// ceil(L / 16) for L kept 8-row groups, the shared groups counted from the bit
-// planes as in the merge.  The best positive gain wins, ties to the lowest h.
-__global__ __launch_bounds__(1024) void k_pack_pairs(int NQ, int Wd, MergeWs m, int32_t* __restrict__ pack_host,
-                                                     int32_t* __restrict__ pack_guest) {
+// A guest g (more than one 128-row tile, last tile of rem rows) may join the
+// single tile of a host h (1 <= n_h <= 128 - rem): gain = T_g + T_h - T(g u h)
+// key tiles, T(L) = ceil(L / 16) for L kept 8-row groups, the shared groups
+// counted from the bit planes as in the merge.  k_pack_cand: one CTA per
+// (cluster, head) lists a guest's kPackCand best hosts (gain, then lowest h);
+// k_pack_select: one thread per head takes the guests in cluster order, each
+// joining its best listed host not yet taken.
+constexpr int kPackCand = kPackCandidates;
+
+__global__ __launch_bounds__(256) void k_pack_cand(int NQ, int Wd, MergeWs m, int2* __restrict__ cand) {
     extern __shared__ uint32_t pk_sm[];
-    uint32_t* sg = pk_sm;                           // [nb][Wd] guest S & P_b
-    uint32_t* taken = pk_sm + kMergePlanes * Wd;    // [ceil(NQ / 32)] hosts already used
-    __shared__ int red_gain[32], red_h[32];
-    const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t* sg = pk_sm;                                   // [nb][Wd] guest S & P_b
+    int* gain = reinterpret_cast<int*>(pk_sm + kMergePlanes * Wd);  // [NQ]
+    const int g = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const size_t hb = (size_t)bh * NQ;
-    const int nb = m.nb[bh];
-    for (int r = tid; r < NQ; r += blockDim.x) {
-        pack_host[hb + r] = -1;
-        pack_guest[hb + r] = -1;
+    int2* out = cand + (hb + g) * kPackCand;
+    const int ng = m.n[hb + g];
+    if (ng <= 128) {  // not a guest
+        if (tid < kPackCand) out[tid] = make_int2(0, -1);
+        return;
     }
-    for (int i = tid; i < (NQ + 31) / 32; i += blockDim.x) taken[i] = 0u;
+    const int nb = m.nb[bh];
+    const int rem = ((ng - 1) & 127) + 1;
+    const int Lg = m.L[hb + g], Tg = (Lg + 15) >> 4;
+    for (int i = tid; i < nb * Wd; i += blockDim.x) {
+        const int b = i / Wd, w = i - b * Wd;
+        sg[i] = m.S[(hb + g) * Wd + w] & m.P[((size_t)bh * kMergePlanes + b) * Wd + w];
+    }
     __syncthreads();
-    for (int g = 0; g < NQ; ++g) {
-        const int ng = m.n[hb + g];
-        if (ng <= 128) continue;  // uniform: not a guest
-        const int rem = ((ng - 1) & 127) + 1;
-        const int Lg = m.L[hb + g], Tg = (Lg + 15) >> 4;
-        for (int i = tid; i < nb * Wd; i += blockDim.x) {
-            const int b = i / Wd, w = i - b * Wd;
-            sg[i] = m.S[(hb + g) * Wd + w] & m.P[((size_t)bh * kMergePlanes + b) * Wd + w];
-        }
-        __syncthreads();
-        int bgain = 0, bidx = -1;
-        for (int h = tid; h < NQ; h += blockDim.x) {
-            const int nh = m.n[hb + h];
-            if (nh < 1 || nh > 128 - rem || ((taken[h >> 5] >> (h & 31)) & 1u)) continue;
+    for (int h = tid; h < NQ; h += blockDim.x) {
+        const int nh = m.n[hb + h];
+        int gv = 0;
+        if (nh >= 1 && nh <= 128 - rem) {
             const int Lh = m.L[hb + h], Th = (Lh + 15) >> 4;
             int inter = 0;
             const uint32_t* Sh = m.S + (hb + h) * Wd;
@@ -180,55 +179,76 @@ __global__ __launch_bounds__(1024) void k_pack_pairs(int NQ, int Wd, MergeWs m, 
                 if (!x) continue;
                 for (int b = 0; b < nb; ++b) inter += __popc(x & sg[b * Wd + w]) << b;
             }
-            const int gain = Tg + Th - ((Lg + Lh - inter + 15) >> 4);
-            if (gain > bgain) {  // h ascends within a thread: strict keeps the lowest
-                bgain = gain;
-                bidx = h;
-            }
+            gv = Tg + Th - ((Lg + Lh - inter + 15) >> 4);
         }
-        for (int o = 16; o > 0; o >>= 1) {
-            const int go = __shfl_xor_sync(0xffffffffu, bgain, o), ho = __shfl_xor_sync(0xffffffffu, bidx, o);
-            if (go > bgain || (go == bgain && ho >= 0 && (bidx < 0 || ho < bidx))) {
-                bgain = go;
-                bidx = ho;
-            }
-        }
-        if (lane == 0) {
-            red_gain[warp] = bgain;
-            red_h[warp] = bidx;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            int gq = 0, hq = -1;
-            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-                const int go = red_gain[w], ho = red_h[w];
-                if (go > gq || (go == gq && ho >= 0 && (hq < 0 || ho < hq))) {
-                    gq = go;
-                    hq = ho;
+        gain[h] = gv;
+    }
+    __syncthreads();
+    if (tid < 32) {  // one warp: the kPackCand largest positive gains, ties to the lowest h
+        const int lane = tid;
+        for (int k = 0; k < kPackCand; ++k) {
+            int bg = 0, bi = -1;
+            for (int h = lane; h < NQ; h += 32)
+                if (gain[h] > bg) {
+                    bg = gain[h];
+                    bi = h;
+                }
+            for (int o = 16; o > 0; o >>= 1) {
+                const int go = __shfl_xor_sync(0xffffffffu, bg, o), ho = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (go > bg || (go == bg && ho >= 0 && (bi < 0 || ho < bi))) {
+                    bg = go;
+                    bi = ho;
                 }
             }
-            if (gq > 0) {
-                pack_host[hb + g] = hq;
-                pack_guest[hb + hq] = g;
-                taken[hq >> 5] |= 1u << (hq & 31);
-            }
+            if (lane == 0) out[k] = make_int2(bg, bi);
+            if (bi >= 0 && lane == (bi & 31)) gain[bi] = 0;  // taken out of the next round
+            __syncwarp();
         }
-        __syncthreads();
+    }
+}
+
+__global__ void k_pack_select(int NQ, const MergeWs m, const int2* __restrict__ cand, int32_t* __restrict__ pack_host,
+                              int32_t* __restrict__ pack_guest) {
+    extern __shared__ uint32_t taken[];  // [ceil(NQ / 32)]
+    const int bh = blockIdx.x, tid = threadIdx.x;
+    const size_t hb = (size_t)bh * NQ;
+    for (int r = tid; r < NQ; r += blockDim.x) {
+        pack_host[hb + r] = -1;
+        pack_guest[hb + r] = -1;
+    }
+    for (int i = tid; i < (NQ + 31) / 32; i += blockDim.x) taken[i] = 0u;
+    __syncthreads();
+    if (tid != 0) return;
+    for (int g = 0; g < NQ; ++g) {
+        if (m.n[hb + g] <= 128) continue;
+        const int2* c = cand + (hb + g) * kPackCand;
+        for (int k = 0; k < kPackCand; ++k) {
+            const int2 e = c[k];
+            if (e.y < 0 || e.x <= 0) break;
+            if ((taken[e.y >> 5] >> (e.y & 31)) & 1u) continue;
+            taken[e.y >> 5] |= 1u << (e.y & 31);
+            pack_host[hb + g] = e.y;
+            pack_guest[hb + e.y] = g;
+            break;
+        }
     }
 }
 
 int launch_pack_pairs(int BH, int NQ, int NK, const uint8_t* mask, const int32_t* q_off, const int32_t* k_off,
-                      const MergeWs& m, int32_t* pack_host, int32_t* pack_guest, cudaStream_t st) {
+                      const MergeWs& m, int2* cand, int32_t* pack_host, int32_t* pack_guest, cudaStream_t st) {
     const int Wd = (NK + 31) / 32;
     PARK_CHECK(launch_merge_setup(mask, q_off, k_off, BH, NQ, NK, m, st));
-    const size_t sm = (size_t)kMergePlanes * Wd * 4 + (size_t)((NQ + 31) / 32) * 4;
-    if (cudaFuncSetAttribute(k_pack_pairs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess) {
+    const size_t sm = (size_t)kMergePlanes * Wd * 4 + (size_t)NQ * 4;
+    if (cudaFuncSetAttribute(k_pack_cand, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess) {
         cudaGetLastError();
         return PARK_ERR_CUDA;
     }
     ::park::prof_begin(st);
-    k_pack_pairs<<<BH, 1024, sm, st>>>(NQ, Wd, m, pack_host, pack_guest);
-    PARK_TRY_LAUNCH("k_pack_pairs", st);
+    k_pack_cand<<<dim3(NQ, BH), 256, sm, st>>>(NQ, Wd, m, cand);
+    PARK_TRY_LAUNCH("k_pack_cand", st);
+    ::park::prof_begin(st);
+    k_pack_select<<<BH, 256, (size_t)((NQ + 31) / 32) * 4, st>>>(NQ, m, cand, pack_host, pack_guest);
+    PARK_TRY_LAUNCH("k_pack_select", st);
     return PARK_OK;
 }
 

@@ -158,11 +158,12 @@ int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t
 // Query-tile packing for the tensor-core path: the last tile of a query cluster
 // with several tiles (a guest) shares the single tile of a cluster with enough
 // free rows (its host) when the host tile's key list, the union of both kept
-// sets, needs fewer key tiles than the two tiles apart.  Greedy per head in
-// cluster order (best gain, ties to the lowest host).  Needs m.S / n / L / P / nb
-// from the merge initialisation (k_merge_init, k_merge_planes).
+// sets, needs fewer key tiles than the two tiles apart.  Each guest lists its
+// best hosts in parallel; then per head, guests in cluster order take the best
+// listed host still free.  Uses a MergeWs (S / n / L / P / nb) and cand [BH][NQ][8].
+constexpr int kPackCandidates = 8;
 int launch_pack_pairs(int BH, int NQ, int NK, const uint8_t* mask, const int32_t* q_off, const int32_t* k_off,
-                      const MergeWs& m, int32_t* pack_host, int32_t* pack_guest, cudaStream_t st);
+                      const MergeWs& m, int2* cand, int32_t* pack_host, int32_t* pack_guest, cudaStream_t st);
 // Tensor-core schedule: per slot (bh, r) the key list at slot * NK (ascending m: padded prefix kv_pre, segs,
 // logit terms segwA for the own rows and segwB for the guest rows, -inf where not kept), kv_len, kv_nseg;
 // 128-row work items with their guests.  pack_host / pack_guest may be null (no packing).

@@ -165,7 +165,8 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
 
 
 struct AttnWs {
-    size_t Qimg, Kp, Vp, poff, segs, segw, segwB, kvnseg, pack, mS, mP, mI, mH, items, icnt, kvpre, kvlen, total;
+    size_t Qimg, Kp, Vp, poff, segs, segw, segwB, kvnseg, pack, pcand, mS, mP, mI, mH, items, icnt, kvpre, kvlen,
+        total;
     size_t item_cap;  // tensor-core work items at most: sum_r ceil(n_r / 128) <= ceil(N / 128) + NQ per head
     int Npad;
 };
@@ -193,13 +194,14 @@ AttnWs plan_attn(const Dims& d, int NQ, int NK) {
         const bool pk = NQ <= kMergeMaxNQ;  // query-tile packing (its state as in the merge)
         const size_t Wd = (NK + 31) / 32;
         w.pack = c.take(pk ? 2 * BH * (size_t)NQ * 4 : 0);
+        w.pcand = c.take(pk ? BH * (size_t)NQ * kPackCandidates * 8 : 0);
         w.mS = c.take(pk ? BH * (size_t)NQ * Wd * 4 : 0);
         w.mP = c.take(pk ? BH * kMergePlanes * Wd * 4 : 0);
         w.mI = c.take(pk ? 7 * BH * (size_t)NQ * 4 : 0);
         w.mH = c.take(pk ? 2 * BH * 4 : 0);
     } else {
         w.Qimg = w.Kp = w.Vp = w.poff = w.segs = w.segw = w.segwB = w.kvnseg = 0;
-        w.pack = w.mS = w.mP = w.mI = w.mH = 0;
+        w.pack = w.pcand = w.mS = w.mP = w.mI = w.mH = 0;
     }
     size_t max_items = BH * ((N + kAttnTile - 1) / kAttnTile + (size_t)NQ);
     w.items = c.take(max_items * sizeof(WorkItem));
@@ -530,7 +532,8 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
         m.todo = a + 6 * sN;
         m.done = at<int32_t>(ws, w.mH);
         m.nb = m.done + BH;
-        PARK_CHECK(launch_pack_pairs(BH, NQ, NK, r->mask, r->q_offsets, r->k_offsets, m, pack_host, pack_guest, st));
+        PARK_CHECK(launch_pack_pairs(BH, NQ, NK, r->mask, r->q_offsets, r->k_offsets, m, at<int2>(ws, w.pcand),
+                                     pack_host, pack_guest, st));
     }
     PARK_CHECK(launch_attn_schedule_tc(BH, NQ, NK, w.Npad, r->q_offsets, r->k_offsets, r->mask, bw, poff, pack_host,
                                        pack_guest, at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), kvnseg, segs,
