@@ -248,7 +248,11 @@ KERNEL_SOURCES = {"k_sparse_attn_tc": ["block_sparse_attention_means_b200/csrc/k
                   "k_pama_tc": ["block_sparse_attention_means_b200/csrc/k_pama_tc.cu"],
                   "k_pama_f64": ["block_sparse_attention_means_b200/csrc/k_pama.cu"],
                   "k_metric_partial": ["block_sparse_attention_means_b200/csrc/k_prep.cu"]}
-ATTENTION_KERNELS = ("k_sparse_attn_tc", "k_gather_rows", "k_attn_schedule", "k_kv_pad_gather", "k_kv_pad_offsets")
+# kernels of park_sparse_attn; the rest of a layer is the retrieval (k_merge_init / k_merge_planes set up
+# the query-tile packing here, and also the cluster merging of the merge variant)
+ATTENTION_KERNELS = ("k_sparse_attn_tc", "k_attn_schedule", "k_kv_pad_gather", "k_kv_pad_offsets",
+                     "k_pack_cand", "k_pack_select", "k_items_emit", "k_item_gather", "k_merge_init",
+                     "k_merge_planes")
 
 
 def kernel_roofline(name: str, ms_per_launch: float, cfg, counters, peaks, peak_kind) -> dict:

@@ -265,7 +265,7 @@ __global__ __launch_bounds__(256) void k_attn_schedule_tc(int NQ, int NK, int Np
                                                           int32_t* __restrict__ kv_pre, int32_t* __restrict__ kv_len,
                                                           int32_t* __restrict__ kv_nseg, int2* __restrict__ segs,
                                                           float* __restrict__ segwA, float* __restrict__ segwB,
-                                                          WorkItem* __restrict__ items, int32_t* __restrict__ item_count,
+                                                          int32_t* __restrict__ slot_items,
                                                           int64_t* __restrict__ counters) {
     __shared__ int wcnt[8], wpad[8];
     __shared__ long long wown[8];
@@ -337,17 +337,61 @@ __global__ __launch_bounds__(256) void k_attn_schedule_tc(int NQ, int NK, int Np
     if (t == 0) {
         kv_len[slot] = nr > 0 ? tot_p : 0;
         kv_nseg[slot] = tot_c;
+        slot_items[slot] = 0;
         if (nr > 0 && tot_p > 0) {
             const int tiles = (nr + 127) / 128;
             const int own_items = h >= 0 ? tiles - 1 : tiles;  // a guest's last tile is in its host's item
+            slot_items[slot] = own_items;  // k_items_emit writes them, head by head in cluster order
+            atomicAdd((unsigned long long*)(counters + PARK_CNT_KEPT_PAIRS),
+                      (unsigned long long)nr * (unsigned long long)tot_own);
+            atomicAdd((unsigned long long*)(counters + PARK_CNT_WORK_ITEMS), (unsigned long long)own_items);
+            atomicAdd((unsigned long long*)(counters + PARK_CNT_KEY_TILES),
+                      (unsigned long long)own_items * (unsigned long long)((tot_p + 127) / 128));
+        }
+    }
+}
+
+// Work items in slot order (head by head, clusters in order, so that the
+// persistent attention CTAs, which take consecutive items, work on one head's
+// key images at a time): one CTA scans the per-slot item counts.
+__global__ __launch_bounds__(1024) void k_items_emit(int BH, int NQ, const int32_t* __restrict__ q_off,
+                                                     const int32_t* __restrict__ pack_guest,
+                                                     const int32_t* __restrict__ slot_items,
+                                                     WorkItem* __restrict__ items, int32_t* __restrict__ item_count) {
+    __shared__ int wsum[32];
+    __shared__ int s_base;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const long long nslot = (long long)BH * NQ;
+    if (t == 0) s_base = 0;
+    __syncthreads();
+    for (long long s0 = 0; s0 < nslot; s0 += 1024) {
+        const long long slot = s0 + t;
+        const int cnt = slot < nslot ? slot_items[slot] : 0;
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[w] = incl;
+        __syncthreads();
+        int woff = 0, tot = 0;
+        for (int q = 0; q < 32; ++q) {
+            if (q < w) woff += wsum[q];
+            tot += wsum[q];
+        }
+        const int base = s_base + woff + incl - cnt;
+        if (cnt > 0) {
+            const int bh = (int)(slot / NQ), r = (int)(slot - (long long)bh * NQ);
+            const int qs = q_off[(size_t)bh * (NQ + 1) + r], nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - qs;
+            const int g = pack_guest ? pack_guest[slot] : -1;
             int gs = 0, gr = 0;
             if (g >= 0) {
                 const int gq = q_off[(size_t)bh * (NQ + 1) + g], gn = q_off[(size_t)bh * (NQ + 1) + g + 1] - gq;
                 gs = gq + 128 * ((gn - 1) / 128);
                 gr = gn - 128 * ((gn - 1) / 128);
             }
-            const int base = atomicAdd(item_count, own_items);
-            for (int q = 0; q < own_items; ++q) {
+            for (int q = 0; q < cnt; ++q) {
                 WorkItem it;
                 it.bh = bh;
                 it.r = r;
@@ -358,25 +402,27 @@ __global__ __launch_bounds__(256) void k_attn_schedule_tc(int NQ, int NK, int Np
                 it.g_rows = gr;
                 items[base + q] = it;
             }
-            atomicAdd((unsigned long long*)(counters + PARK_CNT_KEPT_PAIRS),
-                      (unsigned long long)nr * (unsigned long long)tot_own);
-            atomicAdd((unsigned long long*)(counters + PARK_CNT_WORK_ITEMS), (unsigned long long)own_items);
-            atomicAdd((unsigned long long*)(counters + PARK_CNT_KEY_TILES),
-                      (unsigned long long)own_items * (unsigned long long)((tot_p + 127) / 128));
         }
+        __syncthreads();
+        if (t == 0) s_base += tot;
+        __syncthreads();
     }
+    if (t == 0) *item_count = s_base;
 }
 
 int launch_attn_schedule_tc(int BH, int NQ, int NK, int Npad, const int32_t* q_off, const int32_t* k_off,
                             const uint8_t* mask, const float* bweight, const int32_t* poff, const int32_t* pack_host,
                             const int32_t* pack_guest, int32_t* kv_pre, int32_t* kv_len, int32_t* kv_nseg,
-                            int2* segs, float* segwA, float* segwB, WorkItem* items, int32_t* item_count,
-                            int64_t* counters, cudaStream_t st) {
+                            int2* segs, float* segwA, float* segwB, int32_t* slot_items, WorkItem* items,
+                            int32_t* item_count, int64_t* counters, cudaStream_t st) {
     ::park::prof_begin(st);
     k_attn_schedule_tc<<<dim3(NQ, BH), 256, 0, st>>>(NQ, NK, Npad, q_off, k_off, mask, bweight, poff, pack_host,
-                                                     pack_guest, kv_pre, kv_len, kv_nseg, segs, segwA, segwB, items,
-                                                     item_count, counters);
+                                                     pack_guest, kv_pre, kv_len, kv_nseg, segs, segwA, segwB,
+                                                     slot_items, counters);
     PARK_TRY_LAUNCH("k_attn_schedule", st);
+    ::park::prof_begin(st);
+    k_items_emit<<<1, 1024, 0, st>>>(BH, NQ, q_off, pack_guest, slot_items, items, item_count);
+    PARK_TRY_LAUNCH("k_items_emit", st);
     return PARK_OK;
 }
 

@@ -161,17 +161,18 @@ int make_tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t
 // sets, needs fewer key tiles than the two tiles apart.  Each guest lists its
 // best hosts in parallel; then per head, guests in cluster order take the best
 // listed host still free.  Uses a MergeWs (S / n / L / P / nb) and cand [BH][NQ][8].
-constexpr int kPackCandidates = 8;
+constexpr int kPackCandidates = 32;
 int launch_pack_pairs(int BH, int NQ, int NK, const uint8_t* mask, const int32_t* q_off, const int32_t* k_off,
                       const MergeWs& m, int2* cand, int32_t* pack_host, int32_t* pack_guest, cudaStream_t st);
 // Tensor-core schedule: per slot (bh, r) the key list at slot * NK (ascending m: padded prefix kv_pre, segs,
 // logit terms segwA for the own rows and segwB for the guest rows, -inf where not kept), kv_len, kv_nseg;
-// 128-row work items with their guests.  pack_host / pack_guest may be null (no packing).
+// 128-row work items with their guests, head by head in cluster order (slot_items [BH][NQ]
+// scratch).  pack_host / pack_guest may be null (no packing).
 int launch_attn_schedule_tc(int BH, int NQ, int NK, int Npad, const int32_t* q_off, const int32_t* k_off,
                             const uint8_t* mask, const float* bweight, const int32_t* poff, const int32_t* pack_host,
                             const int32_t* pack_guest, int32_t* kv_pre, int32_t* kv_len, int32_t* kv_nseg,
-                            int2* segs, float* segwA, float* segwB, WorkItem* items, int32_t* item_count,
-                            int64_t* counters, cudaStream_t st);
+                            int2* segs, float* segwA, float* segwB, int32_t* slot_items, WorkItem* items,
+                            int32_t* item_count, int64_t* counters, cudaStream_t st);
 // Q rows of every work item into an item-major image: item i occupies rows
 // [128 i, 128 i + 128) (own rows, then guest rows, then zeros).
 int launch_item_gather(const void* Q, int N, const int32_t* q_perm, const WorkItem* items, const int32_t* item_count,

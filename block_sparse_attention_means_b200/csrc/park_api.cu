@@ -165,8 +165,8 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
 
 
 struct AttnWs {
-    size_t Qimg, Kp, Vp, poff, segs, segw, segwB, kvnseg, pack, pcand, mS, mP, mI, mH, items, icnt, kvpre, kvlen,
-        total;
+    size_t Qimg, Kp, Vp, poff, segs, segw, segwB, kvnseg, sitems, pack, pcand, mS, mP, mI, mH, items, icnt, kvpre,
+        kvlen, total;
     size_t item_cap;  // tensor-core work items at most: sum_r ceil(n_r / 128) <= ceil(N / 128) + NQ per head
     int Npad;
 };
@@ -191,6 +191,7 @@ AttnWs plan_attn(const Dims& d, int NQ, int NK) {
         w.segw = c.take(BH * (size_t)NQ * NK * 4);
         w.segwB = c.take(BH * (size_t)NQ * NK * 4);
         w.kvnseg = c.take(BH * (size_t)NQ * 4);
+        w.sitems = c.take(BH * (size_t)NQ * 4);
         const bool pk = NQ <= kMergeMaxNQ;  // query-tile packing (its state as in the merge)
         const size_t Wd = (NK + 31) / 32;
         w.pack = c.take(pk ? 2 * BH * (size_t)NQ * 4 : 0);
@@ -200,7 +201,7 @@ AttnWs plan_attn(const Dims& d, int NQ, int NK) {
         w.mI = c.take(pk ? 7 * BH * (size_t)NQ * 4 : 0);
         w.mH = c.take(pk ? 2 * BH * 4 : 0);
     } else {
-        w.Qimg = w.Kp = w.Vp = w.poff = w.segs = w.segw = w.segwB = w.kvnseg = 0;
+        w.Qimg = w.Kp = w.Vp = w.poff = w.segs = w.segw = w.segwB = w.kvnseg = w.sitems = 0;
         w.pack = w.pcand = w.mS = w.mP = w.mI = w.mH = 0;
     }
     size_t max_items = BH * ((N + kAttnTile - 1) / kAttnTile + (size_t)NQ);
@@ -537,7 +538,7 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
     }
     PARK_CHECK(launch_attn_schedule_tc(BH, NQ, NK, w.Npad, r->q_offsets, r->k_offsets, r->mask, bw, poff, pack_host,
                                        pack_guest, at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), kvnseg, segs,
-                                       segwA, segwB, items, icnt, r->counters, st));
+                                       segwA, segwB, at<int32_t>(ws, w.sitems), items, icnt, r->counters, st));
     PARK_CHECK(launch_item_gather(Q, N, r->q_perm, items, icnt, w.item_cap, Qimg, num_sms, st));
     PARK_CHECK(launch_sparse_attn_tc(Qimg, w.item_cap, Kp, Vp, BH, N, w.Npad, NQ, NK, r->q_perm, segs, segwA, segwB,
                                      kvnseg, at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), items, icnt, O,
