@@ -136,7 +136,8 @@ extern "C" {
  * order): on the bf16 path park_sparse_attn packs the last 128-row tile of a
  * query cluster with several tiles into the single tile of a cluster with
  * enough free rows when that needs fewer key tiles (every row still attends
- * only to its own cluster's kept key clusters); this flag turns it off. */
+ * only to its own cluster's kept key clusters; done only for NQ <= 2048);
+ * this flag turns it off. */
 #define PARK_FLAG_NO_TILE_PACKING 0x200u
 
 /* ---- park_retrieval.counters indices (outputs, int64) ------------------ */
