@@ -140,6 +140,18 @@ def test_merge_ties_and_round_cap():
     assert hva.merge_clusters(n, mask, [128], rounds=1).tolist() == [0, 0, 2]
 
 
+def test_merge_pairs_only_mutual_choices():
+    # three 40-row clusters over five 128-row key blocks, A {0,1}, B {0,1,2,3},
+    # C {1,2,3,4}: the gain of a pair is the number of shared blocks (a second query
+    # tile never arises: 40 + 40 + 40 <= 128), so A -> B (2), B -> C (3), C -> B (3).
+    # Only the mutual pair B, C merges in the first round; A joins in the second.
+    n = [40, 40, 40]
+    mask = np.array([[1, 1, 0, 0, 0], [1, 1, 1, 1, 0], [0, 1, 1, 1, 1]], dtype=bool)
+    k = [128] * 5
+    assert hva.merge_clusters(n, mask, k, rounds=1).tolist() == [0, 1, 1]
+    assert hva.merge_clusters(n, mask, k).tolist() == [0, 0, 0]
+
+
 def _gain_bruteforce(na, Sa, nb, Sb, wk):
     # the tile cost written with Python sets, independent of merge_clusters
     def cost(n, S):

@@ -31,6 +31,7 @@ def _read_golden(name):
 def test_round_bf16_matches_torch_on_f32_values():
     rng = np.random.default_rng(1)
     x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-8, 8, 20000),
+                        rng.standard_normal(2000) * 2.0 ** -127,      # bf16 subnormals: fixed ulp 2^-133
                         [0.0, -0.0, 1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 2.0 ** -130]]).astype(np.float32)
     want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
     got = po.round_to_bf16(x.astype(np.float64))
@@ -246,6 +247,23 @@ def test_pama_against_per_query_loop():
     assert np.allclose(I[qc > 0].sum(1), 1.0, atol=1e-12)
 
 
+def test_pama_ignores_empty_key_clusters():
+    # an empty key cluster stands for no keys (PAMA over non-empty clusters only): its
+    # column is 0, and its centroid, however strongly it would score, changes nothing
+    Q, K, V, ql, CQ, kl, CK = _tiny_case(seed=3)
+    NQ, NK = CQ.shape[0], CK.shape[0]
+    kc = np.bincount(kl, minlength=NK)
+    kc[2] = 0
+    s = 1 / math.sqrt(Q.shape[1])
+    I = po.pama(Q, ql, NQ, CK, kc, s)
+    CK2 = CK.copy()
+    CK2[2] = 50.0 * Q.mean(axis=0)
+    I2 = po.pama(Q, ql, NQ, CK2, kc, s)
+    qc = np.bincount(ql, minlength=NQ)
+    assert np.all(I[:, 2] == 0.0) and np.array_equal(I, I2)
+    assert np.allclose(I[qc > 0].sum(1), 1.0, atol=1e-12)
+
+
 def test_identity_clustering_gives_exact_attention_mass():
     rng = np.random.default_rng(8)
     N, d = 24, 8
@@ -304,6 +322,8 @@ def test_top_p_rules():
     assert m1[1].tolist() == [True, False, False, False, False]  # 0.5 >= 0.5 with one block
     mall = po.top_p(I, 1.0, qc, kc)
     assert mall[0].tolist() == [True, True, True, False, True]
+    # p = 1 keeps every non-empty block even when the running sum reaches 1 early
+    assert po.top_p(np.array([[0.5, 0.5, 1e-20]]), 1.0, np.array([1]), np.array([1, 1, 1]))[0].all()
     # tiny p keeps exactly one block
     assert po.top_p(I, 1e-9, qc, kc).sum(1).tolist() == [1, 1, 0, 1]
 
@@ -338,6 +358,19 @@ def test_full_full_tv_is_zero():
     assert po.attention_tv(Q, K, kl, 4, CK, 1 / math.sqrt(8)) > 1e-3
 
 
+def test_recall_and_tv_hand_cases():
+    # one query, two single-key clusters with equal scores: the dense attention is
+    # (1/2, 1/2), so keeping one block recalls 1/2 and keeping both recalls 1
+    Q, K = np.array([[1.0]]), np.array([[0.0], [0.0]])
+    kl = np.array([0, 1])
+    assert po.block_recall(Q, K, np.array([0]), kl, np.array([[True, False]]), 1.0) == 0.5
+    assert po.block_recall(Q, K, np.array([0]), kl, np.array([[True, True]]), 1.0) == 1.0
+    # centroids scoring ln 3 and 0 give P = (3/4, 1/4) against the block mass (1/2, 1/2):
+    # total variation (1/2)(1/4 + 1/4) = 1/4
+    CK = np.array([[math.log(3.0)], [0.0]])
+    assert abs(po.attention_tv(Q, K, kl, 2, CK, 1.0) - 0.25) < 1e-15
+
+
 def test_centroid_query_ablation_is_softmax_of_centroid():
     Q, K, V, ql, CQ, kl, CK = _tiny_case(seed=4)
     s = 1 / math.sqrt(Q.shape[1])
@@ -353,6 +386,10 @@ def test_top_k_ratio():
     I = np.array([[0.1, 0.3, 0.2, 0.4]])
     m = po.top_k_ratio(I, 0.5, np.array([1]), np.array([1, 1, 1, 1]))
     assert m[0].tolist() == [False, True, False, True]
+    # ties go to the lower index: k = 1 of two equal leaders, k = 3 of two equal last ones
+    I = np.array([[0.2, 0.3, 0.3, 0.2]])
+    assert po.top_k_ratio(I, 0.25, np.array([1]), np.ones(4, int))[0].tolist() == [False, True, False, False]
+    assert po.top_k_ratio(I, 0.75, np.array([1]), np.ones(4, int))[0].tolist() == [True, True, True, False]
 
 
 def test_size_prior_pama_is_exact_block_mass_for_tight_clusters():
@@ -441,6 +478,58 @@ def test_sip_weighting_is_unbiased_by_enumeration():
         prob = np.prod([p if z else 1 - p for z, p in zip(pattern, pi)])
         expect += prob * sum(X[m] / pi[m] for m in range(6) if pattern[m])
     assert abs(expect - X.sum()) < 1e-12
+
+
+def test_sip_select_inclusion_thresholds_and_weights():
+    # Block m is drawn exactly when its uniform lies below pi_m, so pi_m is the
+    # threshold at which a constant uniform stops drawing m; found by bisection on
+    # sip_select alone.  The thresholds must add up to the expected budget
+    # ceil(0.3 * 7) = 3 (a fractional ratio * L), and every drawn block must carry
+    # the inverse of its threshold as its weight.
+    I = np.array([[0.5, 0.1, 0.1, 0.08, 0.07, 0.1, 0.05]])
+    qc, kc = np.array([4]), np.ones(7, dtype=np.int64)
+
+    def drawn(c):
+        mask, w = po.sip_select(I, 0.3, np.full(I.shape, c), qc, kc)
+        return mask[0], w[0]
+
+    thr = np.zeros(7)
+    for m in range(7):
+        lo, hi = 0.0, 1.0
+        for _ in range(60):
+            mid = 0.5 * (lo + hi)
+            if drawn(mid)[0][m]:
+                lo = mid
+            else:
+                hi = mid
+        thr[m] = lo
+    assert abs(thr.sum() - 3.0) < 1e-9
+    assert abs(thr[0] - 1.0) < 1e-12                        # the dominant block is certain
+    assert np.allclose(thr[1:] / I[0, 1:], thr[1] / I[0, 1], rtol=1e-9)   # the rest in proportion
+    for m in range(1, 7):
+        mask, w = drawn(thr[m] * (1 - 1e-9))
+        assert mask[m] and abs(w[m] * thr[m] - 1.0) < 1e-6
+
+
+def test_integer_block_weights_equal_duplicated_keys():
+    # A key block with weight n in both Softmax sums acts as if its keys were
+    # present n times: the weighted sparse attention of one query cluster equals
+    # plain attention over the kept keys, each repeated by its block's weight.
+    Q, K, V, ql, CQ, kl, CK = _tiny_case(seed=17)
+    NQ, NK = CQ.shape[0], CK.shape[0]
+    s = 1 / math.sqrt(Q.shape[1])
+    rng = np.random.default_rng(17)
+    mask = rng.random((NQ, NK)) < 0.7
+    mask[:, 0] = True
+    weight = np.where(mask, rng.integers(1, 4, size=(NQ, NK)).astype(np.float64), 0.0)
+    O = po.sparse_attention(Q, K, V, ql, kl, mask, s, weight=weight)
+    for r in np.unique(ql):
+        rows = np.nonzero(ql == r)[0]
+        keys = [j for j in range(K.shape[0]) if mask[r, kl[j]] for _ in range(int(weight[r, kl[j]]))]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Q[rows])[None], torch.from_numpy(K[keys])[None], torch.from_numpy(V[keys])[None],
+            scale=s)[0].numpy()
+        assert np.allclose(O[rows], ref, rtol=1e-10, atol=1e-12)
 
 
 def test_sip_select_full_budget_is_dense_and_empty_draw_keeps_best():
