@@ -84,6 +84,14 @@ MUTS2 = [
     ("merge_rounds_plus", H, "    for _ in range(rounds):", "    for _ in range(rounds + 1):"),
     ("merge_root_nofollow", H, "        while root[g] != g:\n            g = root[g]", "        pass"),
     ("padded_floor", H, "return KEY_GROUP * ((k_counts + KEY_GROUP - 1) // KEY_GROUP)", "return KEY_GROUP * (k_counts // KEY_GROUP)"),
+    ("q_kmeans_metric", P, "        q_labels, CQ = kmeans(Q, NQ, iters, None, dtype)", "        q_labels, CQ = kmeans(Q, NQ, iters, M, dtype)"),
+    ("k_kmeans_euclid", P, "        k_labels, CK = kmeans(K, NK, iters, M if qrkc else None, dtype)",
+     "        k_labels, CK = kmeans(K, NK, iters, None, dtype)"),
+    ("pama_query_centroids", P, "        I = pama(Q, q_labels, NQ, CK, k_counts, scale, size_prior=size_prior)",
+     "        I = pama(Q, q_labels, NQ, CQ, k_counts, scale, size_prior=size_prior)"),
+    ("layer_scale_n", P, "    scale = 1.0 / math.sqrt(np.asarray(Q).shape[1])\n    r[\"O\"]", "    scale = 1.0 / math.sqrt(np.asarray(Q).shape[0])\n    r[\"O\"]"),
+    ("local_assign_euclid", H, "labels[rows] = k0[w] + po.assign(X[rows], C[k0[w]:k0[w + 1]], M)",
+     "labels[rows] = k0[w] + po.assign(X[rows], C[k0[w]:k0[w + 1]], None)"),
     ("local_update_local", H, "        C = po.update(X, labels, C, dtype)\n    return (labels, C, hist)", "        C = po.update(X, labels, C, None)\n    return (labels, C, hist)"),
 ]
 

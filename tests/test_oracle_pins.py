@@ -123,6 +123,23 @@ def test_qrkc_changes_clustering_when_metric_is_anisotropic():
     assert lab_q.tolist() == [0, 0, 1, 1] or lab_q.tolist() == [1, 1, 0, 0]
 
 
+def test_retrieval_clusters_queries_euclidean_and_keys_under_the_query_metric():
+    # PARK Figure 2 caption: standard K-means on the queries, the query-derived metric
+    # on the keys.  Anisotropic inputs on which the two metrics give different
+    # clusterings on both sides, so swapping or dropping the metric is visible.
+    rng = np.random.default_rng(4)
+    Q = rng.standard_normal((40, 4)) * np.array([20, 1, 1, 1])
+    K = rng.standard_normal((40, 4)) * np.array([1, 1, 5, 1])
+    M = po.metric(Q)
+    qe, _ = po.kmeans(Q, 4, 3, None, None)
+    ke, _ = po.kmeans(K, 4, 3, None, None)
+    km, _ = po.kmeans(K, 4, 3, M, None)
+    assert (qe != po.kmeans(Q, 4, 3, M, None)[0]).any() and (ke != km).any()
+    r = po.retrieve_head(Q, K, 4, 4, 0.9, 3, None)
+    assert np.array_equal(r["q_labels"], qe) and np.array_equal(r["k_labels"], km)
+    assert np.array_equal(po.retrieve_head(Q, K, 4, 4, 0.9, 3, None, qrkc=False)["k_labels"], ke)
+
+
 # --------------------------------------------------------------------------- K-means brute force
 
 
