@@ -97,7 +97,7 @@ MUTS2 = [
 
 
 def run(name, f, old, new):
-    with tempfile.TemporaryDirectory() as dst:
+    with tempfile.TemporaryDirectory(prefix=".oracle_mutants_", dir=ROOT) as dst:
         for d in ("oracle", "tests", "synth"):
             shutil.copytree(os.path.join(ROOT, d), os.path.join(dst, d), ignore=shutil.ignore_patterns("__pycache__"))
         shutil.copy(os.path.join(ROOT, "pytest.ini"), dst)
