@@ -568,6 +568,24 @@ def test_sip_select_full_budget_is_dense_and_empty_draw_keeps_best():
         assert mask[r].sum() == 1 and mask[r, best] and w[r, best] >= 1.0
 
 
+def test_qrkc_trades_raw_key_error_for_qk_score_error():
+    # PARK Appendix Table 5: clustering the keys under the query-derived metric lowers
+    # the QK-score squared error and raises the raw-key MSE against Euclidean K-means
+    # (there -36.6 % / -22.8 % and +8.5 % / +14.8 % on real activations).  A direction
+    # check on every head of the small synthetic layer.
+    from synth.generator import gen_tensor
+    cfg = CONFIGS["small"]
+    Q, K = (gen_tensor(cfg, t).astype(np.float64)[0] for t in "QK")
+    for h in range(cfg.H):
+        M = po.metric(Q[h])
+        le, Ce = po.kmeans(K[h], cfg.NK, cfg.iters, None, cfg.dtype)
+        lm, Cm = po.kmeans(K[h], cfg.NK, cfg.iters, M, cfg.dtype)
+        raw_e, qk_e = po.key_errors(Q[h], K[h], le, Ce)
+        raw_m, qk_m = po.key_errors(Q[h], K[h], lm, Cm)
+        print(f"head {h}: raw-key MSE {100 * (raw_m / raw_e - 1):+.1f} %, QK-score error {100 * (qk_m / qk_e - 1):+.1f} %")
+        assert qk_m < qk_e and raw_m > raw_e
+
+
 def test_key_errors_qk_term_is_metric_distance():
     rng = np.random.default_rng(10)
     Q, K = rng.standard_normal((64, 8)), rng.standard_normal((50, 8))
