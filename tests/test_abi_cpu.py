@@ -53,7 +53,7 @@ def test_status_strings():
 def test_workspace_size_and_shape_validation():
     hy = P.Shape(1, 24, 33, 45, 80, 256, 128)
     n = P.workspace_size(hy, 930, 930)
-    assert 2.0e9 < n < 4.0e9                     # permuted Q/K/V dominate: 3 x 731 MB
+    assert 2.0e9 < n < 4.0e9                     # the item-major Q image and the K/V tile images dominate
     # streamed PAMA: workspace does not grow with N * NK (PARK Appendix Table 6)
     n2 = P.workspace_size(P.Shape(1, 24, 66, 45, 80, 256, 128), 930, 930)
     assert n2 < 2.2 * n
