@@ -1,5 +1,5 @@
 // Block-sparse attention over the kept (query cluster, key cluster) pairs
-// (PARK abstract: attention "only within" the retrieved blocks).
+// (PARK abstract: attention is computed inside the retrieved blocks alone).
 //
 // Layout: Q, K, V are first gathered into cluster-contiguous order (q_perm /
 // k_perm), so every query cluster is a run of rows and every key cluster a run

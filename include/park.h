@@ -5,11 +5,12 @@
  * The operation is the one described in "PARK: Accurate Block Retrieval for
  * Sparse Attention in Video Diffusion Transformers" (abstract; Figure 2
  * caption; Table 1 caption): for one attention layer, cluster the queries with
- * Euclidean K-means, cluster the keys with K-means under a metric derived from
- * the current queries (QRKC), give every original query a Softmax over the key
- * centroids and average these within each query cluster (PAMA), keep key
- * clusters per query cluster up to cumulative importance p (top-p), and compute
- * attention only on the kept (query-cluster, key-cluster) pairs.
+ * Euclidean K-means, cluster the keys with K-means under a metric computed from
+ * this layer's queries (QRKC), give every original query its own Softmax over
+ * the key centroids and take the mean of those within each query cluster
+ * (PAMA), keep key clusters per query cluster up to cumulative importance p
+ * (top-p), and compute attention only on the kept (query-cluster,
+ * key-cluster) pairs.
  *
  * Definitions fixed by this library where the pages are silent:
  *   metric       M = (1/N) sum_i q_i q_i^T (float64); key distance
@@ -206,7 +207,7 @@ int park_retrieve(const void *Q, const void *K, const park_shape *shape, int NQ,
                   int iters, park_retrieval *out, void *ws, size_t ws_bytes, void *stream);
 
 /* Block-sparse attention over the kept blocks of a retrieval result (PARK
- * abstract: "computing attention only within" the retrieved blocks).  Reads
+ * abstract: attention is computed inside the retrieved blocks alone).  Reads
  * labels, perms, offsets and the CSR of *r; writes O [B,H,N,D] in the input
  * dtype, original token order.  Also sets r->counters[PARK_CNT_WORK_ITEMS] and
  * may set *r->status. */

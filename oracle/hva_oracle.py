@@ -73,8 +73,8 @@ def local_init(X, K, win, nW):
 
 def local_assign(X, C, win, nW, M=None):
     """Each grid token searches only the centroids of its own window (READING of
-    "restrict centroid search to fixed local neighborhoods": the neighbourhood
-    of a token is its window); a text token has no grid position and searches
+    the abstract's centroid search limited to a fixed neighbourhood around each
+    token: that neighbourhood is the token's window); a text token has no grid position and searches
     every centroid.  Distances and ties as in the global assign (lowest index)."""
     K = C.shape[0]
     k0 = window_starts(K, nW)

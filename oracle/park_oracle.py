@@ -54,9 +54,9 @@ def round_to(x, dtype):
 def metric(Q):
     """M = (1/N) sum_i q_i q_i^T, the queries' second-moment matrix.
 
-    READING of "transforms keys using a metric derived from the current
-    queries, so that keys receiving similar QK scores are grouped together"
-    (PARK, Figure 2 caption): for any key k and centroid c,
+    READING of PARK's Figure 2 caption, where the keys are clustered under a
+    metric computed from this layer's queries, which should put keys that get
+    alike scores from those queries in one cluster: for any key k and centroid c,
     (k - c)^T M (k - c) = mean_i (q_i.k - q_i.c)^2, the mean squared QK-score
     difference under the current queries, which is what the pages want small
     inside a key cluster.  A library matmul forms the sum."""
@@ -110,8 +110,8 @@ def exact_mean(rows, dtype):
 
     The column sums are exact and rounded once to float64 (math.fsum is
     correctly rounded), then divided by n in IEEE float64, then rounded to the
-    storage dtype.  READING: the pages only say clusters are represented by
-    their averages (PARK abstract, "averaged representations")."""
+    storage dtype.  READING: the pages only say that a cluster is represented
+    by the mean of its members (PARK abstract)."""
     n = rows.shape[0]
     sums = np.array([math.fsum(col) for col in np.asarray(rows, dtype=np.float64).T.tolist()])
     return round_to(sums / float(n), dtype)
@@ -355,8 +355,8 @@ def dense_attention(Q, K, V, scale):
 
 def sparse_attention(Q, K, V, q_labels, k_labels, mask, scale, rows=None, weight=None):
     """Block-sparse attention: query i attends, with a renormalised Softmax,
-    only to keys whose cluster is kept for its query cluster a(i) ("computing
-    attention only within" the retrieved blocks, PARK abstract).  Returns
+    only to keys whose cluster is kept for its query cluster a(i) (PARK
+    abstract: attention is computed inside the retrieved blocks alone).  Returns
     float64 [N, d] in original token order (or only the listed rows).
     weight[r, m] (SIP): every exp term of key cluster m is multiplied by it, in
     the numerator and in the normaliser (a ratio of two inverse-probability
