@@ -42,7 +42,7 @@ PARK_NUM_COUNTERS = 8
 # Every symbol include/park.h declares (checked by the CPU tests).
 EXPORTS = ("park_workspace_size", "park_retrieve", "park_sparse_attn", "park_layer", "park_status_string",
            "park_launch_count", "park_version", "park_profile_enable", "park_profile_collect",
-           "park_qrkc_metric_static")
+           "park_qrkc_metric_static", "park_set_wait_limit_ns")
 
 
 class ParkShape(ctypes.Structure):
@@ -108,6 +108,8 @@ def load() -> ctypes.CDLL:
     lib.park_profile_collect.restype = i32
     lib.park_qrkc_metric_static.argtypes = [vp, shp, vp, vp]
     lib.park_qrkc_metric_static.restype = i32
+    lib.park_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.park_set_wait_limit_ns.restype = i32
     _lib = lib
     return lib
 

@@ -13,6 +13,8 @@ namespace park {
 
 // ---------------------------------------------------------------- host side
 void note_launch(int n = 1);  // counts kernels for park_launch_count()
+// Limit of every bounded device wait on the hot path, in ns (park_set_wait_limit_ns).
+uint64_t wait_limit_ns();
 // Per-kernel event timing (park_profile_enable): begin before a launch, end
 // (with the kernel's name) right after it, on the launch stream.
 void prof_begin(cudaStream_t st);
@@ -48,10 +50,6 @@ template <>
 struct Elem<bf16_t> {
     static constexpr int bytes = 2;
     static constexpr int dtype = PARK_BF16;
-    // Inputs meeting the range precondition are multiples of 2^-27 below 2^16,
-    // so x * 2^27 is an integer below 2^43: sums of up to 2^20 of them are exact
-    // in int64.
-    static constexpr int frac_bits = 27;
     __device__ static inline double to_double(const bf16_t* p, int j) {
         return (double)__uint_as_float(((uint32_t)p[j].bits) << 16);
     }
@@ -66,9 +64,6 @@ template <>
 struct Elem<float> {
     static constexpr int bytes = 4;
     static constexpr int dtype = PARK_F32;
-    // Multiples of 2^-43 below 2^16: x * 2^43 < 2^59 per element; sums are kept
-    // in two int64 limbs (see FixedAcc).
-    static constexpr int frac_bits = 43;
     __device__ static inline double to_double(const float* p, int j) { return (double)p[j]; }
     __device__ static inline float to_float(const float* p, int j) { return p[j]; }
     __device__ static inline int biased_exp(uint32_t bits) { return (bits >> 23) & 0xFF; }
@@ -79,24 +74,49 @@ __device__ inline void set_status(int32_t* status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
-// Range precondition: x == 0, or finite with 2^-20 <= |x| < 2^16
-// (biased exponent 107..142 in the IEEE single layout that bf16 shares).
+// Range precondition: x == 0, or finite with 2^-40 <= |x| < 2^40
+// (biased exponent 87..166 in the IEEE single layout that bf16 shares).
+constexpr int kRangeExpMin = 87, kRangeExpMax = 166;
 __device__ inline bool in_range_exp(int e, uint32_t magnitude_bits) {
-    return magnitude_bits == 0 || (e >= 107 && e <= 142);
+    return magnitude_bits == 0 || (e >= kRangeExpMin && e <= kRangeExpMax);
 }
 
 // ---------------------------------------------------------------- fixed point
-// Exact fixed-point image of a float32 input element: F = x * 2^43 (integer);
-// the left shift of the integer significand is e - 107.  Out-of-range inputs
-// are reported by the input check, not summed exactly.
-__device__ inline long long fixed_f32(uint32_t u) {
-    int e = (u >> 23) & 0xFF;
-    if (e == 0) return 0;
-    long long m = (long long)(0x800000u | (u & 0x7FFFFFu));
-    int sh = e - 107;
-    sh = sh < 0 ? 0 : (sh > 38 ? 38 : sh);
-    long long v = m << sh;
-    return (u & 0x80000000u) ? -v : v;
+// Exact centroid sums: every element in range is an integer multiple of 2^-64
+// (bf16: 8-bit significand, ulp >= 2^-47; float32: 24-bit significand, ulp >=
+// 2^-63) below 2^40, so F = x * 2^64 is an integer with |F| < 2^104, and a sum
+// of up to 2^20 of them fits a signed 128-bit integer (hi * 2^64 + lo, two's
+// complement).  Integer sums do not depend on the order of the terms.
+__device__ inline void acc128_add(unsigned long long& lo, long long& hi, unsigned long long a_lo, long long a_hi) {
+    const unsigned long long n = lo + a_lo;
+    hi += a_hi + (long long)(n < lo);
+    lo = n;
+}
+
+// Adds F = x * 2^64 for the element with IEEE-single-layout bits `u` (a bf16
+// element passed as its bits << 16): x = (-1)^s m 2^(e - 150) with the 24-bit
+// significand m, so F = m << (e - 86), a shift of 1..80 inside the range.
+// Zero adds nothing; elements outside the range (reported by the input check)
+// are clamped, not summed exactly.
+__device__ inline void fixed64_add(unsigned long long& lo, long long& hi, uint32_t u) {
+    const int e = (u >> 23) & 0xFF;
+    if (e == 0) return;
+    const unsigned long long m = 0x800000ull | (u & 0x7FFFFFull);
+    int sh = e - 86;
+    sh = sh < 0 ? 0 : (sh > 80 ? 80 : sh);
+    unsigned long long a_lo, a_hi;
+    if (sh >= 64) {
+        a_lo = 0ull;
+        a_hi = m << (sh - 64);
+    } else {
+        a_lo = m << sh;
+        a_hi = sh == 0 ? 0ull : (m >> (64 - sh));
+    }
+    if (u & 0x80000000u) {  // two's complement negation of the 128-bit value
+        a_lo = ~a_lo + 1ull;
+        a_hi = ~a_hi + (a_lo == 0ull ? 1ull : 0ull);
+    }
+    acc128_add(lo, hi, a_lo, (long long)a_hi);
 }
 
 // Correctly rounded (nearest, ties to even) conversion of the signed 128-bit
@@ -133,8 +153,8 @@ __device__ inline double i128_to_double_rn(long long hi, unsigned long long lo) 
 
 // Round a double to bf16 (nearest, ties to even) directly, without passing
 // through float.  Finite inputs whose magnitude is at most 2^127; values
-// below the bf16 normal range flush to zero (never reached by means of inputs
-// meeting the range precondition, which are >= 2^-47 or 0).
+// below the bf16 normal range (2^-126) flush to zero (never reached by means of
+// inputs meeting the range precondition, which are >= 2^-67 or 0).
 __device__ inline uint16_t double_to_bf16_bits(double x) {
     unsigned long long u = (unsigned long long)__double_as_longlong(x);
     unsigned long long sign = u >> 63;

@@ -45,7 +45,8 @@ __global__ void __launch_bounds__(320, 1)
     k_assign_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int N, int K,
                 int BH, const float* __restrict__ bias, int bias_ld, const float* __restrict__ xnorm,
                 const float* __restrict__ wmax, const float* __restrict__ bmax, float gamma,
-                int32_t* __restrict__ labels, Lists lists, int32_t* __restrict__ status) {
+                int32_t* __restrict__ labels, Lists lists, int32_t* __restrict__ status,
+                uint64_t wait_ns) {
     constexpr int WB = KW / 64;  // 64-column blocks per centroid chunk
     extern __shared__ __align__(1024) uint8_t dsmem_raw[];
     __shared__ AsSmem sh;
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(320, 1)
             int G = 0, I = 0, w_last[2] = {-1, -1}, x_last = -1;
             for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
                 const int bh = t / tpr, r0 = (t - bh * tpr) * AS_ROWS;
-                if (I > 0 && !mbar_wait(&sh.x_empty, (I - 1) & 1, abort)) break;
+                if (I > 0 && !mbar_wait(&sh.x_empty, (I - 1) & 1, abort, wait_ns)) break;
                 mbar_arrive_expect_tx(&sh.x_full, 4 * AS_BLK);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(320, 1)
                 bool ok = true;
                 for (int c = 0; c < nch; ++c) {
                     const int s = G & 1, round = G >> 1;
-                    if (round > 0 && !mbar_wait(&sh.w_empty[s], (round - 1) & 1, abort)) {
+                    if (round > 0 && !mbar_wait(&sh.w_empty[s], (round - 1) & 1, abort, wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -124,12 +125,12 @@ __global__ void __launch_bounds__(320, 1)
             int G = 0, I = 0;
             const uint32_t xa = smem_u32(Xs);
             for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
-                if (!mbar_wait(&sh.x_full, I & 1, abort)) break;
+                if (!mbar_wait(&sh.x_full, I & 1, abort, wait_ns)) break;
                 bool ok = true;
                 for (int c = 0; c < nch; ++c) {
                     const int s = G & 1, round = G >> 1;
-                    if (!mbar_wait(&sh.w_full[s], round & 1, abort) ||
-                        (round > 0 && !mbar_wait(&sh.acc_empty[s], (round - 1) & 1, abort))) {
+                    if (!mbar_wait(&sh.w_full[s], round & 1, abort, wait_ns) ||
+                        (round > 0 && !mbar_wait(&sh.acc_empty[s], (round - 1) & 1, abort, wait_ns))) {
                         ok = false;
                         break;
                     }
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int c = 0; c < nch; ++c) {
                 const int s = G & 1, round = G >> 1;
                 if (!failed) {
-                    const bool ok = mbar_wait(&sh.acc_full[s], round & 1, abort);
+                    const bool ok = mbar_wait(&sh.acc_full[s], round & 1, abort, wait_ns);
                     failed = !__all_sync(0xffffffffu, ok);
                 }
                 tc_fence_after();
@@ -227,7 +228,13 @@ __global__ void __launch_bounds__(320, 1)
                 if (g != w) second = fminf(second, v0[g]);
             if (r0 + row < N && !failed) {
                 const size_t gr = (size_t)bh * N + r0 + row;
-                const float beta = gamma * xnorm[gr] * wmax[bh] + 4.8e-7f * bmax[bh] + 1e-30f;
+                // relative terms (accumulation, split residual, bias rounding) plus two
+                // absolute ones for magnitudes below the float32/bf16 normal range: bf16
+                // hi/lo parts of M c that flush to zero (< 2^-126 each, summed against
+                // |x|: <= 2^-121.5 ||x||) and products or partial sums that the tensor
+                // core flushes (< 2^-126 each over 256 terms, doubled: covered by 1e-30)
+                const float xn = xnorm[gr];
+                const float beta = gamma * xn * wmax[bh] + 4.8e-7f * bmax[bh] + xn * 0x1p-118f + 1e-30f;
                 labels[gr] = i0[w];
                 if (!(second - best > 2.f * beta)) {
                     const int pos = atomicAdd(lists.counts + 1, 1);
@@ -260,10 +267,10 @@ int launch_assign_tc(const void* X, int BH, int N, int K, const CentroidOps& ops
     ::park::prof_begin(st);
     if (ops.kw == 128)
         k_assign_tc<128><<<num_sms, 320, sm, st>>>(mX, mW, N, K, BH, ops.bias32, ops.bias_ld, xnorm, ops.wmax,
-                                                   ops.bmax, gamma, labels, lists, status);
+                                                   ops.bmax, gamma, labels, lists, status, wait_limit_ns());
     else
         k_assign_tc<256><<<num_sms, 320, sm, st>>>(mX, mW, N, K, BH, ops.bias32, ops.bias_ld, xnorm, ops.wmax,
-                                                   ops.bmax, gamma, labels, lists, status);
+                                                   ops.bmax, gamma, labels, lists, status, wait_limit_ns());
     PARK_TRY_LAUNCH("k_assign_tc", st);
     return PARK_OK;
 }

@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(352, 1)
                      const float* __restrict__ segwB, const int32_t* __restrict__ kv_nseg,
                      const int32_t* __restrict__ kv_pre, const int32_t* __restrict__ kv_len,
                      const WorkItem* __restrict__ items, const int32_t* __restrict__ item_count,
-                     uint16_t* __restrict__ O, float sl2e, int32_t* __restrict__ status) {
+                     uint16_t* __restrict__ O, float sl2e, int32_t* __restrict__ status, uint64_t wait_ns) {
     extern __shared__ __align__(1024) uint8_t dsmem_raw[];
     __shared__ TcSmem sh;
     // 1024-byte aligned operand area: Q | K0 K1 | V0 V1 (each 32 KB)
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(352, 1)
             const float* segwA_item = segwA + slot * NK;
             const float* segwB_item = segwB + slot * NK;
             if (isK && lane == 0) {
-                bool ok = I == 0 || mbar_wait(&sh.q_empty, (I - 1) & 1, abort);
+                bool ok = I == 0 || mbar_wait(&sh.q_empty, (I - 1) & 1, abort, wait_ns);
                 if (ok) {
                     mbar_arrive_expect_tx(&sh.q_full, 2 * TC_BLK);
                     const int y = it * TC_ROWS;  // the item's rows in the item-major Q image
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(352, 1)
                     // K of tile j: stage free once S_{j-3} has completed
                     const int ks = T % TC_KST, kround = T / TC_KST;
                     bool w = true;
-                    if (lane == 0 && kround > 0) w = mbar_wait(&sh.k_empty[ks], (kround - 1) & 1, abort);
+                    if (lane == 0 && kround > 0) w = mbar_wait(&sh.k_empty[ks], (kround - 1) & 1, abort, wait_ns);
                     if (__shfl_sync(0xffffffffu, w ? 1 : 0, 0) == 0 || warp_abort(abort)) {
                         ok = false;
                         break;
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(352, 1)
                 } else {
                     // V of tile j and its column bias: free once PV_{j-2} has completed
                     bool w = true;
-                    if (lane == 0 && round > 0) w = mbar_wait(&sh.v_empty[stg], (round - 1) & 1, abort);
+                    if (lane == 0 && round > 0) w = mbar_wait(&sh.v_empty[stg], (round - 1) & 1, abort, wait_ns);
                     if (__shfl_sync(0xffffffffu, w ? 1 : 0, 0) == 0 || warp_abort(abort)) {
                         ok = false;
                         break;
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(352, 1)
             auto issue_S = [&](int g) -> bool {
                 const int b = g & 1, ks = g % TC_KST;
                 // buffer b is free: its last reader, PV_{g-2}, was issued before this MMA
-                if (!mbar_wait(&sh.k_full[ks], (g / TC_KST) & 1, abort)) return false;
+                if (!mbar_wait(&sh.k_full[ks], (g / TC_KST) & 1, abort, wait_ns)) return false;
                 tc_fence_after();
                 const uint32_t ka = smem_u32(Ks + ks * 2 * TC_BLK);
                 const uint32_t d = tmem + (uint32_t)(b * 128);
@@ -333,14 +333,14 @@ __global__ void __launch_bounds__(352, 1)
                 const int L = kv_len[(size_t)wi.bh * NQ + wi.r];
                 const int nkt = (L + TC_ROWS - 1) / TC_ROWS;
                 if (nkt == 0) continue;
-                if (!mbar_wait(&sh.q_full, I & 1, abort)) break;
+                if (!mbar_wait(&sh.q_full, I & 1, abort, wait_ns)) break;
                 tc_fence_after();
                 bool ok = issue_S(G) && (nkt < 2 || issue_S(G + 1));
                 for (int j = 0; j < nkt && ok; ++j) {
                     const int g = G + j, b = g & 1, ph = (g >> 1) & 1, vs = g % TC_VST;
-                    if (!mbar_wait(&sh.p_full[b], ph, abort) ||
-                        (j == 0 && I > 0 && !mbar_wait(&sh.o_empty, (I - 1) & 1, abort)) ||
-                        !mbar_wait(&sh.v_full[vs], (g / TC_VST) & 1, abort)) {
+                    if (!mbar_wait(&sh.p_full[b], ph, abort, wait_ns) ||
+                        (j == 0 && I > 0 && !mbar_wait(&sh.o_empty, (I - 1) & 1, abort, wait_ns)) ||
+                        !mbar_wait(&sh.v_full[vs], (g / TC_VST) & 1, abort, wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(352, 1)
         // tensor-memory work but still walks the items and meets its barriers.
         bool failed = false;
         auto wwait = [&](uint64_t* bar, uint32_t parity) {
-            if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+            if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(bar, parity, abort, wait_ns));
             return !failed;
         };
         for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
@@ -579,7 +579,7 @@ int launch_sparse_attn_tc(const void* Qimg, size_t item_cap, const void* Kpad, c
     k_sparse_attn_tc<<<num_sms, 352, sm, st>>>(mQ, (const uint8_t*)Kpad, (const uint8_t*)Vpad, N, NQ, NK, q_perm,
                                                 segs, segwA, segwB, kv_nseg, kv_pre, kv_len, items, item_count,
                                                 (uint16_t*)O,
-                                                sl2e, status);
+                                                sl2e, status, wait_limit_ns());
     PARK_TRY_LAUNCH("k_sparse_attn_tc", st);
     return PARK_OK;
 }

@@ -121,10 +121,11 @@ __global__ void k_local_init(const T* __restrict__ X, int N, int D, int K, WinGe
 // memory as float32: s_k = fl32(bias_k) - 2 x . fl32(w_k) with w = c (Euclidean)
 // or M c (QRKC).  The float32 winner is certified when the runner-up is more
 // than 2 beta above it, with
-//   beta = 1.05 (2 u Bmax + (2 D + 7) u ||x|| Wmax),  u = 2^-24,
+//   beta = 1.05 (2 u Bmax + (2 D + 7) u ||x|| Wmax) + 2^-120 (||x|| + 1),  u = 2^-24,
 // which bounds the error of each float32 score against the exact one (the
-// roundings of bias and w, the D-term FMA chain, the final subtraction); Wmax and
-// Bmax are the head's max ||w_k|| and |bias_k|.  Otherwise the token is
+// roundings of bias and w, the D-term FMA chain, the final subtraction, and
+// gradual underflow below 2^-126); Wmax and Bmax are the head's max ||w_k|| and
+// |bias_k|.  Otherwise the token is
 // rescored in float64 (Euclidean sum_j (x_j - c_j)^2; QRKC bias - 2 x . (M c)),
 // ties to the lowest index.
 constexpr int kLocalThreads = 256;
@@ -203,7 +204,9 @@ __global__ __launch_bounds__(kLocalThreads) void k_assign_local(
     const float Wm = wmax[bh], Bm = bmax[bh];
     auto certified = [&](float best, float sec, float nx) {
         const float xn = sqrtf(nx) * 1.001f;  // covers the float32 rounding of ||x||^2
-        const float beta = 1.05f * (2.f * u * Bm + (2.f * D + 7.f) * u * xn * Wm);
+        // + absolute terms for results below the float32 normal range (gradual
+        // underflow: <= 2^-150 per rounding, generously covered)
+        const float beta = 1.05f * (2.f * u * Bm + (2.f * D + 7.f) * u * xn * Wm) + xn * 0x1p-120f + 0x1p-120f;
         return kw == 1 || (sec - best > 2.f * beta);  // false for NaN
     };
     auto rescore = [&](const T* xp) -> int {
@@ -406,7 +409,9 @@ __global__ __launch_bounds__(256) void k_text_finish(const T* __restrict__ X, in
         }
         nx = warp_sum(nx);
         const float u = 5.9604645e-8f;  // 2^-24
-        const float beta = 1.05f * (2.f * u * bmax[bh] + (2.f * D + 7.f) * u * sqrtf(nx) * 1.001f * wmax[bh]);
+        const float xn = sqrtf(nx) * 1.001f;
+        const float beta = 1.05f * (2.f * u * bmax[bh] + (2.f * D + 7.f) * u * xn * wmax[bh]) + xn * 0x1p-120f +
+                           0x1p-120f;
         if (lane == 0) {
             if (K == 1 || sec - best > 2.f * beta)
                 labels[(size_t)bh * N + row0 + t] = idx < K ? idx : 0;

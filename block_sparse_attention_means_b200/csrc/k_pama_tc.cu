@@ -71,7 +71,8 @@ __global__ void __launch_bounds__(320, 1)
               const int32_t* __restrict__ q_perm, const int32_t* __restrict__ q_off,
               const int32_t* __restrict__ k_off, const float* __restrict__ qnorm, const float* __restrict__ ckmax,
               int N, int NQ, int NK, int BH, float sl2e, float delta_scale, int size_prior,
-              float* __restrict__ importance, float* __restrict__ rho, int32_t* __restrict__ status) {
+              float* __restrict__ importance, float* __restrict__ rho, int32_t* __restrict__ status,
+              uint64_t wait_ns) {
     extern __shared__ __align__(1024) uint8_t dsmem_raw[];
     __shared__ PtSmem sh;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(320, 1)
                 const int bh = it / NQ, r = it - bh * NQ;
                 const int qs = q_off[(size_t)bh * (NQ + 1) + r], nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - qs;
                 for (int t0 = 0; t0 < nr && ok; t0 += PT_ROWS) {
-                    if (I > 0 && !mbar_wait(&sh.q_empty, (I - 1) & 1, abort)) {
+                    if (I > 0 && !mbar_wait(&sh.q_empty, (I - 1) & 1, abort, wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(320, 1)
                     for (int c2 = 0; c2 < 2 * nch; ++c2) {  // both passes
                         const int c = c2 < nch ? c2 : c2 - nch;
                         const int s = G & 1, round = G >> 1;
-                        if (round > 0 && !mbar_wait(&sh.c_empty[s], (round - 1) & 1, abort)) {
+                        if (round > 0 && !mbar_wait(&sh.c_empty[s], (round - 1) & 1, abort, wait_ns)) {
                             ok = false;
                             break;
                         }
@@ -157,14 +158,14 @@ __global__ void __launch_bounds__(320, 1)
                 const int bh = it / NQ, r = it - bh * NQ;
                 const int nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - q_off[(size_t)bh * (NQ + 1) + r];
                 for (int t0 = 0; t0 < nr && ok; t0 += PT_ROWS) {
-                    if (!mbar_wait(&sh.q_full, I & 1, abort)) {
+                    if (!mbar_wait(&sh.q_full, I & 1, abort, wait_ns)) {
                         ok = false;
                         break;
                     }
                     for (int c2 = 0; c2 < 2 * nch; ++c2) {
                         const int s = G & 1, b = G % PT_NB;
-                        if (!mbar_wait(&sh.c_full[s], (G >> 1) & 1, abort) ||
-                            (G >= PT_NB && !mbar_wait(&sh.acc_empty[b], (G / PT_NB - 1) & 1, abort))) {
+                        if (!mbar_wait(&sh.c_full[s], (G >> 1) & 1, abort, wait_ns) ||
+                            (G >= PT_NB && !mbar_wait(&sh.acc_empty[b], (G / PT_NB - 1) & 1, abort, wait_ns))) {
                             ok = false;
                             break;
                         }
@@ -200,7 +201,7 @@ __global__ void __launch_bounds__(320, 1)
         bool failed = false;
         int G = 0;
         auto wait_acc = [&](int b, int g) {
-            if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(&sh.acc_full[b], (g / PT_NB) & 1, abort));
+            if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(&sh.acc_full[b], (g / PT_NB) & 1, abort, wait_ns));
             tc_fence_after();
         };
         for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
@@ -327,7 +328,9 @@ __global__ void __launch_bounds__(320, 1)
                 // (numerator and denominator); the float32 row-sum partials (8 x 8
                 // terms per 64 columns, relative error <= 10 2^-24; 12 counted) and the
                 // float32 column sums
-                double delta = (double)delta_scale * qm * ckmax[bh];
+                // (+ products and partial sums that the tensor core may flush below
+                // 2^-126: at most 2D of them, 2^-118 in all, times the scale)
+                double delta = (double)delta_scale * qm * ckmax[bh] + 0x1p-118;
                 if (size_prior) delta += 0.6931471805599453 * 5.9604644775390625e-8 * log2((double)N + 1.0);
                 const double rr = expm1(2.0 * delta) + 4.0 * 4.76837158203125e-7 +
                                   (12.0 + 16.0 + nr / 64.0) * 5.9604644775390625e-8;
@@ -368,7 +371,7 @@ int launch_pama_tc(const void* Qg, int BH, int N, int NQ, int NK, const int32_t*
         (float)((1.0 / sqrt((double)D)) * (kappa * 5.9604644775390625e-8 + 1.1920928955078125e-7) * 1.01);
     ::park::prof_begin(st);
     k_pama_tc<<<num_sms, 320, sm, st>>>(mQ, mC, q_perm, q_off, k_off, qnorm, ckmax, N, NQ, NK, BH, sl2e, delta_scale,
-                                        size_prior, importance, rho, status);
+                                        size_prior, importance, rho, status, wait_limit_ns());
     PARK_TRY_LAUNCH("k_pama_tc", st);
     return PARK_OK;
 }

@@ -6,7 +6,7 @@ namespace park {
 
 // ---------------------------------------------------------------- input check
 // One pass over the tensor with 16-byte loads: every element must be 0 or a
-// finite value with 2^-20 <= |x| < 2^16 (the library's range precondition).
+// finite value with 2^-40 <= |x| < 2^40 (the library's range precondition).
 template <int BYTES>
 __global__ void k_input_check(const uint4* __restrict__ x, size_t n16, int32_t* status) {
     size_t stride = (size_t)gridDim.x * blockDim.x;
@@ -214,55 +214,31 @@ int launch_strided_init(const void* X, int dtype, int BH, int N, int D, int K, v
 }
 
 // ---------------------------------------------------------------- centroid operands
-// Per centroid: bias = ||c||^2 (Euclidean) or c^T M c with w = M c (QRKC),
-// w split as bf16 hi + lo (|w - hi - lo| <= 2^-16 |w|) for the score GEMM,
-// and the per-head maxima ||w|| and |bias| used by the certified bound.
-// One CTA of D threads per (centroid, head); float64 sums in a fixed tree.
-template <typename T, bool METRIC>
-__global__ void k_centroid_prep(const T* __restrict__ C, int K, int D, const double* __restrict__ Mall,
-                                uint16_t* __restrict__ wop, float* __restrict__ bias32, int bias_ld,
-                                double* __restrict__ bias64, double* __restrict__ w64, float* __restrict__ wmax,
-                                float* __restrict__ bmax) {
-    __shared__ double cs[128];
-    __shared__ double red[2][128];
+// Euclidean operands, per centroid: bias = ||c||^2 and the per-head maxima
+// ||c|| and |bias| used by the certified bound (the score GEMM reads the
+// centroids themselves, w = c).  One CTA of D threads per (centroid, head);
+// float64 sums in a fixed tree.
+template <typename T>
+__global__ void k_centroid_prep(const T* __restrict__ C, int K, int D, float* __restrict__ bias32, int bias_ld,
+                                double* __restrict__ bias64, float* __restrict__ wmax, float* __restrict__ bmax) {
+    __shared__ double red[128];
     int k = blockIdx.x, bh = blockIdx.y, a = threadIdx.x;
     const T* c = C + ((size_t)bh * K + k) * D;
-    double ca = Elem<T>::to_double(c, a);
-    cs[a] = ca;
-    __syncthreads();
-    double wa = ca;
-    if (METRIC) {
-        const double* M = Mall + (size_t)bh * D * D + (size_t)a * D;
-        double s = 0.0;
-        for (int b = 0; b < D; ++b) s = __fma_rn(M[b], cs[b], s);
-        wa = s;
-        w64[((size_t)bh * K + k) * D + a] = wa;
-        if (wop != nullptr) {
-            uint16_t hi = double_to_bf16_bits(wa);
-            double hid = (double)__uint_as_float(((uint32_t)hi) << 16);
-            uint16_t lo = double_to_bf16_bits(wa - hid);  // wa - hid is exact
-            wop[((size_t)bh * K + k) * (2 * D) + a] = hi;
-            wop[((size_t)bh * K + k) * (2 * D) + D + a] = lo;
-        }
-    }
-    red[0][a] = ca * wa;
-    red[1][a] = wa * wa;
+    const double ca = Elem<T>::to_double(c, a);
+    red[a] = ca * ca;
     __syncthreads();
     for (int s = 64; s > 0; s >>= 1) {
-        if (a < s && a + s < D) {
-            red[0][a] += red[0][a + s];
-            red[1][a] += red[1][a + s];
-        }
+        if (a < s && a + s < D) red[a] += red[a + s];
         __syncthreads();
     }
     if (k == 0)  // columns past K read +inf, so a score GEMM over whole 128-column chunks never picks them
         for (int j = K + a; j < ((K + 127) & ~127); j += blockDim.x)
             bias32[(size_t)bh * bias_ld + j] = __int_as_float(0x7f800000);
     if (a == 0) {
-        double b = red[0][0];
+        const double b = red[0];
         bias64[(size_t)bh * K + k] = b;
         bias32[(size_t)bh * bias_ld + k] = __double2float_rn(b);
-        atomic_max_nonneg(wmax + bh, round_up_f(__double2float_ru(sqrt(red[1][0]))));
+        atomic_max_nonneg(wmax + bh, round_up_f(__double2float_ru(sqrt(b))));
         atomic_max_nonneg(bmax + bh, round_up_f(__double2float_ru(fabs(b))));
     }
 }
@@ -271,6 +247,11 @@ __global__ void k_centroid_prep(const T* __restrict__ C, int K, int D, const dou
 // in shared memory, thread (a, half) forms w_a = sum_b M[b][a] c_b for eight
 // centroids (row b of M: conflict-free), then per centroid bias = c . w and
 // ||w||^2 are reduced over the 128 threads of its half in a fixed order.
+// w and the bias are taken for 2^-e M, e the binary exponent of the head's
+// largest diagonal entry (|M_ab| <= max_a M_aa), so that the float32 scores stay
+// far from overflow over the whole input range (|x| < 2^40 gives M up to 2^80).
+// A power-of-two scale is exact in float64 and multiplies every score of the
+// head by the same factor, so it changes no argmin.
 constexpr int kPrepCents = 16;
 
 template <typename T>
@@ -284,6 +265,7 @@ __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restric
     double* Ms = reinterpret_cast<double*>(smem_raw);  // [D][D]
     double* Cs = Ms + D * D;                          // [kPrepCents][D]
     __shared__ double red[kPrepCents][4][2];
+    __shared__ double s_scale;
     const int bh = blockIdx.y, k0 = blockIdx.x * kPrepCents, t = threadIdx.x;
     const int a = t & 127, half = t >> 7, lane = t & 31, wq = (t >> 5) & 3;
     const double* M = Mall + (size_t)bh * D * D;
@@ -296,6 +278,14 @@ __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restric
         for (int j = K + t; j < ((K + 127) & ~127); j += blockDim.x)
             bias32[(size_t)bh * bias_ld + j] = __int_as_float(0x7f800000);
     __syncthreads();
+    if (t < 32) {
+        double dm = 0.0;
+        for (int j = t; j < D; j += 32) dm = fmax(dm, Ms[j * D + j]);
+        dm = warp_max(dm);
+        if (t == 0) s_scale = dm > 0.0 ? ldexp(1.0, -ilogb(dm)) : 1.0;
+    }
+    __syncthreads();
+    const double scale = s_scale;
     double w[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) w[c] = 0.0;
@@ -306,6 +296,8 @@ __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restric
             for (int c = 0; c < 8; ++c) w[c] = __fma_rn(m, Cs[(half * 8 + c) * D + b], w[c]);
         }
     }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) w[c] *= scale;  // exact
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         const int cc = half * 8 + c, k = k0 + cc;
@@ -361,21 +353,12 @@ int launch_centroid_prep(const void* C, int dtype, int BH, int K, int D, const d
         return PARK_OK;
     }
     ::park::prof_begin(st);
-    if (dtype == PARK_BF16) {
-        if (metric)
-            k_centroid_prep<bf16_t, true><<<g, D, 0, st>>>((const bf16_t*)C, K, D, M, (uint16_t*)ops.w, ops.bias32, ops.bias_ld,
-                                                          ops.bias64, ops.w64, ops.wmax, ops.bmax);
-        else
-            k_centroid_prep<bf16_t, false><<<g, D, 0, st>>>((const bf16_t*)C, K, D, M, nullptr, ops.bias32, ops.bias_ld,
-                                                           ops.bias64, ops.w64, ops.wmax, ops.bmax);
-    } else {
-        if (metric)
-            k_centroid_prep<float, true><<<g, D, 0, st>>>((const float*)C, K, D, M, (uint16_t*)ops.w, ops.bias32, ops.bias_ld,
-                                                         ops.bias64, ops.w64, ops.wmax, ops.bmax);
-        else
-            k_centroid_prep<float, false><<<g, D, 0, st>>>((const float*)C, K, D, M, nullptr, ops.bias32, ops.bias_ld,
-                                                          ops.bias64, ops.w64, ops.wmax, ops.bmax);
-    }
+    if (dtype == PARK_BF16)
+        k_centroid_prep<bf16_t><<<g, D, 0, st>>>((const bf16_t*)C, K, D, ops.bias32, ops.bias_ld, ops.bias64, ops.wmax,
+                                                 ops.bmax);
+    else
+        k_centroid_prep<float><<<g, D, 0, st>>>((const float*)C, K, D, ops.bias32, ops.bias_ld, ops.bias64, ops.wmax,
+                                                ops.bmax);
     PARK_TRY_LAUNCH("k_centroid_prep", st);
     return PARK_OK;
 }

@@ -8,12 +8,11 @@
 // warps in sequence) and scatters them.  The result equals a stable argsort of
 // the labels.
 //
-// Update: one CTA per (cluster, head) sums its members' rows exactly in fixed
-// point (x * 2^27 for bf16, x * 2^43 for float32 inputs; integer sums are exact
-// and independent of order), converts the exact sum to float64 with one
-// correct rounding, divides by the member count in IEEE float64 and rounds to
-// the storage dtype (nearest, ties to even).  Empty clusters keep their
-// centroid.
+// Update: one CTA per (cluster, head) sums its members' rows exactly in 128-bit
+// fixed point (x * 2^64; integer sums are exact and independent of order),
+// converts the exact sum to float64 with one correct rounding, divides by the
+// member count in IEEE float64 and rounds to the storage dtype (nearest, ties
+// to even).  Empty clusters keep their centroid.
 #include "kernels.h"
 
 namespace park {
@@ -153,13 +152,20 @@ int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist
 // ---------------------------------------------------------------- update
 // 128 threads.  Each thread owns one 16-byte piece of a row: VEC elements at
 // piece p = t % CPR, and rows s, s + RPI, ... of the cluster (s = t / CPR).
+// Every element goes into a signed 128-bit fixed-point sum of x * 2^64
+// (fixed64_add, exact for the whole range precondition).  bf16 elements with
+// 2^-20 <= |x| < 2^16 -- all of them on unit-scale data -- first go through a
+// float64 partial sum per element that is exact for 1024 rows (such values are
+// multiples of 2^-27 below 2^16, so 1024 of them need at most 53 bits) and is
+// moved into the 128-bit sum every 1024 rows; the rest take the integer path
+// directly.
 template <typename T>
 __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const int32_t* __restrict__ perm,
                                                 const int32_t* __restrict__ offsets, int N, int D, int K,
                                                 T* __restrict__ C) {
     constexpr int VEC = 16 / sizeof(T);
-    constexpr bool TWO_LIMBS = sizeof(T) == 4;
-    extern __shared__ long long red[];  // [RPI][D] (x2 for two limbs)
+    constexpr bool BF16 = sizeof(T) == 2;
+    extern __shared__ long long red[];  // [2][RPI][D]: high and low words of the 128-bit sums
     int k = blockIdx.x, bh = blockIdx.y;
     const int32_t* off = offsets + (size_t)bh * (K + 1);
     int start = off[k], n = off[k + 1] - start;
@@ -168,25 +174,23 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
     int t = threadIdx.x, piece = t % CPR, slot = t / CPR;
     long long acc_hi[VEC];
     unsigned long long acc_lo[VEC];
+    double part[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
         acc_hi[e] = 0;
         acc_lo[e] = 0;
+        part[e] = 0.0;
     }
     const int32_t* pm = perm + (size_t)bh * N + start;
     const T* Xh = X + (size_t)bh * N * D;
-    // bf16: float64 partial sums, exact for up to 1024 rows (members are multiples
-    // of 2^-27 below 2^16, so 1024 of them need at most 53 bits), moved into the
-    // int64 fixed-point accumulators every 1024 rows and at the end
-    double part[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) part[e] = 0.0;
     int rows_in_part = 0;
     auto flush = [&]() {
-        if (!TWO_LIMBS) {
+        if (BF16) {
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
-                acc_hi[e] += __double2ll_rn(ldexp(part[e], Elem<T>::frac_bits));
+                // part * 2^27 is an integer below 2^53; as x * 2^64 it is that integer << 37
+                const long long v = __double2ll_rn(ldexp(part[e], 27));
+                acc128_add(acc_lo[e], acc_hi[e], (unsigned long long)v << 37, v >> 27);
                 part[e] = 0.0;
             }
         }
@@ -194,18 +198,19 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
     };
     auto add_piece = [&](const uint4& v) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        if (!TWO_LIMBS) {
+        if (BF16) {
 #pragma unroll
-            for (int e = 0; e < VEC; ++e)
-                part[e] += (double)__uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+            for (int e = 0; e < VEC; ++e) {
+                const uint32_t b = (e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16);
+                const uint32_t ex = (b >> 23) & 0xFFu;
+                const bool fast = (ex - 107u) <= 35u || ex == 0u;  // 2^-20 <= |x| < 2^16, or 0
+                part[e] += fast ? (double)__uint_as_float(b) : 0.0;
+                if (!fast) fixed64_add(acc_lo[e], acc_hi[e], b);
+            }
             if (++rows_in_part == 1024) flush();
         } else {
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                const long long f = fixed_f32(w[e]);
-                acc_lo[e] += (unsigned long long)(f & 0xFFFFFFFFll);
-                acc_hi[e] += f >> 32;
-            }
+            for (int e = 0; e < VEC; ++e) fixed64_add(acc_lo[e], acc_hi[e], w[e]);
         }
     };
     if (slot < RPI) {
@@ -230,29 +235,16 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
             red_hi[slot * D + piece * VEC + e] = acc_hi[e];
-            if (TWO_LIMBS) red_lo[slot * D + piece * VEC + e] = (long long)acc_lo[e];
+            red_lo[slot * D + piece * VEC + e] = (long long)acc_lo[e];
         }
     }
     __syncthreads();
     if (t < D) {
-        double mean;
-        if (!TWO_LIMBS) {
-            long long s = 0;
-            for (int q = 0; q < RPI; ++q) s += red_hi[q * D + t];
-            mean = ldexp(__ll2double_rn(s), -Elem<T>::frac_bits) / (double)n;
-        } else {
-            long long sh = 0;
-            unsigned long long sl = 0;
-            for (int q = 0; q < RPI; ++q) {
-                sh += red_hi[q * D + t];
-                sl += (unsigned long long)red_lo[q * D + t];
-            }
-            // exact value = sh * 2^32 + sl (sl < 2^52, |sh| < 2^48): form it in 128 bits
-            __int128 v = ((__int128)sh << 32) + (__int128)sl;
-            long long hi = (long long)(v >> 64);
-            unsigned long long lo = (unsigned long long)v;
-            mean = ldexp(i128_to_double_rn(hi, lo), -Elem<T>::frac_bits) / (double)n;
-        }
+        long long sh = 0;
+        unsigned long long sl = 0;
+        for (int q = 0; q < RPI; ++q) acc128_add(sl, sh, (unsigned long long)red_lo[q * D + t], red_hi[q * D + t]);
+        // one correct rounding of the exact sum to float64, then the IEEE division by n
+        const double mean = ldexp(i128_to_double_rn(sh, sl), -64) / (double)n;
         T* c = C + ((size_t)bh * K + k) * D + t;
         if (sizeof(T) == 2)
             reinterpret_cast<uint16_t*>(c)[0] = double_to_bf16_bits(mean);
@@ -269,7 +261,7 @@ int launch_update(const void* X, int dtype, int BH, int N, int D, int K, const i
     ::park::prof_begin(st);
     if (dtype == PARK_BF16) {
         int rpi = 128 / (D / 8);
-        k_update<bf16_t><<<g, 128, (size_t)rpi * D * 8, st>>>((const bf16_t*)X, perm, offsets, N, D, K, (bf16_t*)C);
+        k_update<bf16_t><<<g, 128, (size_t)rpi * D * 16, st>>>((const bf16_t*)X, perm, offsets, N, D, K, (bf16_t*)C);
     } else {
         int rpi = 128 / (D / 4);
         k_update<float><<<g, 128, (size_t)rpi * D * 16, st>>>((const float*)X, perm, offsets, N, D, K, (float*)C);

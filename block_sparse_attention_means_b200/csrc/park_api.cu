@@ -14,6 +14,10 @@ namespace park {
 static std::atomic<unsigned long long> g_launches{0};
 void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s
+static std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+
 // ---------------------------------------------------------------- per-kernel timing
 namespace {
 struct ProfRec {
@@ -323,6 +327,9 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
         }
         return PARK_OK;
     }
+    // labels start valid (cluster 0), so that a kernel that gave up on a bounded
+    // wait (status PARK_ERR_TIMEOUT) leaves nothing out of range for the later steps
+    PARK_CHECK(memset_async(s.labels, (size_t)BH * N * 4, st));
     if (bf16) PARK_CHECK(launch_row_norms(s.X, d.dtype, BH, N, D, s.xnorm, st));
     if (!s.warm) PARK_CHECK(launch_strided_init(s.X, d.dtype, BH, N, D, K, s.C, st));
     const float gamma = gamma_for(ops.kw, s.M != nullptr);
@@ -608,7 +615,7 @@ const char* park_status_string(int code) {
         case PARK_ERR_UNSUPPORTED: return "unsupported shape or dtype";
         case PARK_ERR_WORKSPACE: return "workspace too small";
         case PARK_ERR_CUDA: return "CUDA launch failed";
-        case PARK_ERR_RANGE: return "input outside the range precondition (0 or 2^-20 <= |x| < 2^16, finite)";
+        case PARK_ERR_RANGE: return "input outside the range precondition (0 or 2^-40 <= |x| < 2^40, finite)";
         case PARK_ERR_TIMEOUT: return "a bounded device wait ran out";
         default: return "unknown status";
     }
@@ -651,6 +658,11 @@ int park_profile_collect(park_kernel_time* out, int cap, int* n) {
     return rc;
 }
 
-int park_version(void) { return 100; }
+int park_version(void) { return 200; }
+
+int park_set_wait_limit_ns(uint64_t ns) {
+    g_wait_ns.store(ns ? ns : kDefaultWaitNs, std::memory_order_relaxed);
+    return PARK_OK;
+}
 
 }  // extern "C"

@@ -9,7 +9,7 @@
 // workspace; this entry point takes it from a fixed array compiled into the
 // library instead, so the caller passes nothing but Q and the output M.
 //
-// The scratch is a file-scope __device__ array of PARK_STATIC_SCRATCH_BYTES
+// The scratch is a file-scope __device__ array of kStaticScratchBytes
 // (16 MiB).  Every GPU that loads the library holds it until the process exits.
 // It holds the per-chunk partial sums of the metric: one D x D float64 matrix
 // per (head, row chunk), so at most 16 MiB / (8 D^2) partials (128 at D = 128):
@@ -22,8 +22,9 @@
 // the entry point looks the address up once with cudaGetSymbolAddress and
 // caches it; make that first call before any stream capture.  Every call
 // shares the one array: calls that overlap on the GPU (different streams, or
-// several host threads) race on it.  The partial sums are fully overwritten by
-// each call, so nothing has to start at zero.  No cudaMalloc, cudaFree or
+// several host threads) race on it.  Each call writes every entry of the
+// partials that its reduction reads (the upper-triangle 8 x 8 blocks of each
+// D x D partial), so nothing has to start at zero.  No cudaMalloc, cudaFree or
 // allocating library routine is called.
 #include <mutex>
 

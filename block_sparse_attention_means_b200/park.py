@@ -205,3 +205,9 @@ def profile_collect() -> dict:
     n = ctypes.c_int(0)
     _lib.check(_lib.load().park_profile_collect(buf, cap, ctypes.byref(n)), "park_profile_collect")
     return {buf[i].name.decode(): (buf[i].total_ms, int(buf[i].launches)) for i in range(n.value)}
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Limit of every bounded device wait inside the library's kernels (0 = the
+    default, 2 s).  Only the tests of the timeout path change it."""
+    _lib.check(_lib.load().park_set_wait_limit_ns(int(ns)), "park_set_wait_limit_ns")

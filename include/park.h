@@ -38,9 +38,11 @@
  *   - Layout: Q, K, V, O are [B, H, N, D] contiguous, N = T*Hg*W + n_text
  *     (video tokens in (t, y, w) order, text tokens last).  dtype PARK_BF16
  *     requires D == 128; PARK_F32 requires D % 32 == 0 and D <= 128.
- *   - Range precondition: every input element is 0 or has 2^-20 <= |x| < 2^16
- *     (and is finite).  N <= 2^20, B*H*N < 2^31, 1 <= NQ, NK <= N,
- *     NK <= 4096, NQ <= 65536, p > 0, iters >= 1.
+ *   - Range precondition: every input element is 0 or has 2^-40 <= |x| < 2^40
+ *     (and is finite).  Inside it the centroid sums are exact (128-bit fixed
+ *     point at 2^-64), whatever the order of the terms.
+ *   - Sizes: N <= 2^20, B*H*N < 2^31, 1 <= NQ, NK <= N, NK <= 4096,
+ *     NQ <= 65536, p > 0, iters >= 1.
  *   - Errors: argument errors are returned synchronously (nothing is enqueued).
  *     Conditions only the device can see (an input outside the range
  *     precondition, a bounded wait that ran out) are written to *status; the
@@ -228,6 +230,16 @@ uint64_t park_launch_count(void);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int park_version(void);
+
+/* Limit, in nanoseconds of device time, of every bounded wait inside this
+ * library's kernels (a wait for a tensor-memory-access copy or a tensor-core
+ * result; default 2 s; ns = 0 restores the default).  Host state, read at each
+ * launch.  A wait that runs out sets *status to PARK_ERR_TIMEOUT; the kernel
+ * then lets its copies and MMAs in flight finish, frees its tensor memory and
+ * returns, so the context stays usable and later calls are unaffected.  A tiny
+ * limit (1 ns) makes the waits run out on purpose: that is how the timeout path
+ * is tested.  Never needed in normal use. */
+int park_set_wait_limit_ns(uint64_t ns);
 
 /* ---- per-kernel timing for measurement tools --------------------------- */
 typedef struct {

@@ -100,9 +100,40 @@ def distances(X, C, M=None, row_block=4096):
     return D
 
 
+_CLIB = None
+
+
+def _clib():
+    """The oracle's C part (oracle/assign.c), compiled on first use."""
+    global _CLIB
+    if _CLIB is None:
+        import ctypes
+        from . import build_oracle
+        lib = ctypes.CDLL(build_oracle.build())
+        lib.oracle_assign.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                      ctypes.c_int64, ctypes.c_void_p]
+        lib.oracle_assign.restype = None
+        _CLIB = lib
+    return _CLIB
+
+
 def assign(X, C, M=None):
-    """a(i) = argmin_k D(x_i, c_k); ties go to the lowest k (READING)."""
-    return np.argmin(distances(X, C, M), axis=1).astype(np.int64)
+    """a(i) = argmin_k D(x_i, c_k); ties go to the lowest k (READING).
+
+    The same distances as `distances` (rows and centroids transformed by F^T
+    for a metric, then sum_j (x_j - c_j)^2), each summed in j order by the C
+    loop in assign.c, which keeps full-size heads within seconds."""
+    X = np.asarray(X, dtype=np.float64)
+    C = np.asarray(C, dtype=np.float64)
+    if M is not None:
+        F = metric_factor(M)
+        X = X @ F
+        C = C @ F
+    X = np.ascontiguousarray(X)
+    C = np.ascontiguousarray(C)
+    labels = np.empty(X.shape[0], dtype=np.int64)
+    _clib().oracle_assign(X.ctypes.data, C.ctypes.data, X.shape[0], C.shape[0], X.shape[1], labels.ctypes.data)
+    return labels
 
 
 def exact_mean(rows, dtype):
@@ -386,7 +417,7 @@ def sparse_attention(Q, K, V, q_labels, k_labels, mask, scale, rows=None, weight
 
 def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", topk_ratio=None,
                   size_prior=False, sip_ratio=None, sip_u=None, grid=None, window=None, merge=False,
-                  merge_rounds=8):
+                  merge_rounds=8, q_init=None, k_init=None):
     """PARK retrieval for one (b, h): query K-means (Euclidean), key K-means
     with the query-derived metric (QRKC), PAMA importance, top-p mask
     (PARK Figure 2).  qrkc=False is the "w/o QRKC" ablation (M = I);
@@ -397,15 +428,18 @@ def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", to
     and adds the weights to the result.  window = (wt, wh, ww) with grid =
     (T, Hg, W) runs both K-means with HVA's local-window assign, and merge=True
     merges query clusters after the selection (hva_oracle); importance stays
-    the one the selection used."""
+    the one the selection used.  q_init / k_init: centroids to start K-means
+    from instead of the strided initialisation (a warm start).  The result also
+    holds q_hist / k_hist, the centroids entering each K-means iteration."""
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
     d = Q.shape[1]
     scale = 1.0 / math.sqrt(d)
     M = metric(Q)
+    q_hist = k_hist = None
     if window is None:
-        q_labels, CQ = kmeans(Q, NQ, iters, None, dtype)
-        k_labels, CK = kmeans(K, NK, iters, M if qrkc else None, dtype)
+        q_labels, CQ, q_hist = kmeans(Q, NQ, iters, None, dtype, init=q_init, history=True)
+        k_labels, CK, k_hist = kmeans(K, NK, iters, M if qrkc else None, dtype, init=k_init, history=True)
     else:
         from . import hva_oracle as hva
         q_labels, CQ = hva.local_kmeans(Q, NQ, iters, grid, window, None, dtype)
@@ -434,7 +468,8 @@ def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", to
     k_perm, k_off = stable_permutation(k_labels, NK)
     return dict(M=M, q_labels=q_labels, k_labels=k_labels, q_centroids=CQ, k_centroids=CK,
                 q_counts=q_counts, k_counts=k_counts, importance=I, mask=mask, weight=weight,
-                q_perm=q_perm, q_offsets=q_off, k_perm=k_perm, k_offsets=k_off)
+                q_perm=q_perm, q_offsets=q_off, k_perm=k_perm, k_offsets=k_off, q_hist=q_hist, k_hist=k_hist,
+                qrkc=qrkc)
 
 
 def layer_head(Q, K, V, NQ, NK, p, iters, dtype, **kw):

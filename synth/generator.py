@@ -19,10 +19,7 @@ shape; real activations are not available):
 * V is positional (tiny, small) or i.i.d. N(0, 1) (Wan- and HunyuanVideo-shaped).
   Text tokens are i.i.d. N(0, 1) in Q, K and V.
 * Values are computed in float64, rounded to float32 and then, for bf16
-  configs, to bf16 with round-to-nearest-even.  Magnitudes below 2^-20 are
-  flushed to zero so every input meets the library's range precondition
-  (x = 0 or 2^-20 <= |x| < 2^16); with unit-scale data this touches about one
-  element in a million.
+  configs, to bf16 with round-to-nearest-even.  Nothing else is changed.
 * Every (tensor, batch, head) slice has its own stream
   ``numpy.random.default_rng([seed, tensor_id, b, h])`` so slices can be made
   in any order, in parallel, and one at a time for large configs.
@@ -37,7 +34,6 @@ import os
 import numpy as np
 
 TENSOR_IDS = {"Q": 0, "K": 1, "V": 2, "U": 3}
-FLUSH_BELOW = 2.0 ** -20
 
 
 @dataclasses.dataclass(frozen=True)
@@ -153,7 +149,6 @@ def _finish(x64: np.ndarray, dtype: str) -> np.ndarray:
     x32 = x64.astype(np.float32)
     if dtype == "bf16":
         x32 = round_bf16_from_f32(x32)
-    x32[np.abs(x32) < FLUSH_BELOW] = 0.0
     return x32
 
 
@@ -221,4 +216,35 @@ def gen_uniform(cfg: LayerConfig, seed: int = 0) -> np.ndarray:
         for h in range(cfg.H):
             rng = np.random.default_rng([seed, TENSOR_IDS["U"], b, h])
             out[b, h] = rng.random((cfg.NQ, cfg.NK), dtype=np.float32)
+    return out
+
+
+def with_extreme_magnitudes(x: np.ndarray, dtype: str, seed: int, frac_small: float = 0.01,
+                            frac_zero: float = 0.002, frac_large: float = 0.0, large_exp=(16.0, 39.9)) -> np.ndarray:
+    """A copy of ``x`` with a seeded fraction of its elements replaced by values
+    at the ends of the library's input range (0 or 2^-40 <= |x| < 2^40):
+    magnitudes 2^u with u ~ U[-40, -20) (``frac_small``), exact zeros
+    (``frac_zero``) and magnitudes 2^u with u ~ U[large_exp) (``frac_large``),
+    random signs, rounded to ``dtype`` (a rounding that reaches 2^40 is pulled
+    back one ulp).  Only an input generator: it holds none of the method's
+    arithmetic."""
+    rng = np.random.default_rng([seed, 7])
+    out = np.array(x, dtype=np.float32, copy=True)
+    flat = out.reshape(-1)
+    n = flat.size
+    pick = rng.random(n)
+    sign = np.where(rng.random(n) < 0.5, -1.0, 1.0)
+    u_small = rng.uniform(-40.0, -20.0, size=n)
+    u_large = rng.uniform(large_exp[0], large_exp[1], size=n)
+    small = pick < frac_small
+    zero = (pick >= frac_small) & (pick < frac_small + frac_zero)
+    large = (pick >= frac_small + frac_zero) & (pick < frac_small + frac_zero + frac_large)
+    vals = np.where(small, sign * np.exp2(u_small), np.where(large, sign * np.exp2(u_large), 0.0))
+    v32 = _finish(vals, dtype)
+    top = np.float32(2.0 ** 40)
+    v32 = np.where(np.abs(v32) >= top, np.nextafter(np.float32(np.abs(v32)), np.float32(0)) * np.sign(v32), v32)
+    v32 = np.where(np.abs(v32) < np.float32(2.0 ** -40), np.sign(v32) * np.float32(2.0 ** -40), v32)
+    v32 = _finish(v32.astype(np.float64), dtype)
+    flat[small | zero | large] = v32[small | zero | large]
+    flat[zero] = 0.0
     return out

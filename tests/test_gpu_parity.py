@@ -58,7 +58,7 @@ def test_layer_matches_oracle(park, name):
     Q, K, V = pu.inputs(name)
     ref = pu.oracle_layer(name)
     O, r = run_layer(park, cfg, Q, K, V)
-    fails = pu.compare_retrieval(r, ref, cfg.NQ, cfg.NK)
+    fails = pu.compare_retrieval(r, ref, cfg.NQ, cfg.NK, Q, K, cfg.p)
     M = pu.np64(r.metric)
     for bh, h in enumerate(ref):
         rel = np.abs(M[0, bh] - h["M"]).max() / np.abs(h["M"]).max()
@@ -260,17 +260,61 @@ def test_large_logits_many_key_tiles(park):
     pu.assert_output_close(O, ref, False)
 
 
-def test_range_precondition_reported(park):
+@pytest.mark.parametrize("where,value", [("Q", 2.0 ** -41), ("K", -(2.0 ** 40)), ("V", 2.0 ** -41)])
+def test_range_precondition_reported(park, where, value):
+    """One finite element outside 0 or 2^-40 <= |x| < 2^40 in any of Q, K, V
+    sets PARK_ERR_RANGE; the extreme values inside it do not."""
     cfg = RAGGED
     Q, K, V = gen_layer(cfg, seed=6)
-    Q = Q.copy()
-    Q[0, 1, 7, 3] = 1e-7  # below 2^-20 and not zero
+    X = {"Q": Q.copy(), "K": K.copy(), "V": V.copy()}
+    X[where][0, 1, 7, 3] = value
     dt = torch.bfloat16
     shape = park.Shape.of(cfg, dt)
-    q, k, v = (pu.to_device(x, dt) for x in (Q, K, V))
+    q, k, v = (pu.to_device(X[t], dt) for t in "QKV")
     _, r = park.layer(q, k, v, shape, cfg.NQ, cfg.NK, cfg.p, cfg.iters)
     torch.cuda.synchronize()
     assert r.status_code() == park._lib.PARK_ERR_RANGE
+    for edge in (2.0 ** -40, -(2.0 ** 40 - 2.0 ** 32), 0.0):  # the ends of the range: accepted
+        X[where][0, 1, 7, 3] = edge
+        q, k, v = (pu.to_device(X[t], dt) for t in "QKV")
+        _, r = park.layer(q, k, v, shape, cfg.NQ, cfg.NK, cfg.p, cfg.iters)
+        torch.cuda.synchronize()
+        assert r.status_code() == 0, edge
+
+
+def test_cached_retrieval_reused_on_new_inputs(park):
+    """Mask reuse across denoising steps (PARK Appendix Table 9): a retrieval
+    computed on one step's Q, K is kept, and park_sparse_attn alone runs on the
+    next step's Q, K, V with it; the output equals the oracle's block-sparse
+    attention of the new tensors under the cached labels and mask."""
+    cfg = CONFIGS["small"]
+    Q0, K0, _ = pu.inputs("small", 0)
+    Q1, K1, V1 = pu.inputs("small", 1)
+    dt = torch.bfloat16
+    shape = park.Shape.of(cfg, dt)
+    q0, k0 = pu.to_device(Q0, dt), pu.to_device(K0, dt)
+    r = park.retrieve(q0, k0, shape, cfg.NQ, cfg.NK, cfg.p, cfg.iters)
+    torch.cuda.synchronize()
+    assert r.status_code() == 0
+    ref = pu.oracle_layer("small", 0)
+    assert not pu.compare_retrieval(r, ref, cfg.NQ, cfg.NK, Q0, K0, cfg.p)
+    q1, k1, v1 = (pu.to_device(x, dt) for x in (Q1, K1, V1))
+    O = park.sparse_attn(q1, k1, v1, shape, cfg.NQ, cfg.NK, r)
+    torch.cuda.synchronize()
+    assert r.status_code() == 0
+    got = pu.np64(O)
+    worst = 0.0
+    for h, hr in enumerate(ref):
+        want = po.sparse_attention(Q1[0, h], K1[0, h], V1[0, h], hr["q_labels"], hr["k_labels"], hr["mask"],
+                                   pu.scale_of(cfg.D))
+        d = np.abs(got[0, h] - want)
+        assert d.max() <= pu.O_MAX_ABS and d.mean() <= pu.O_MEAN_ABS, (h, d.max(), d.mean())
+        worst = max(worst, float(d.max()))
+        # and it is not the output of the retrieval's own step
+        same = po.sparse_attention(Q0[0, h], K0[0, h], V1[0, h], hr["q_labels"], hr["k_labels"], hr["mask"],
+                                   pu.scale_of(cfg.D))
+        assert np.abs(got[0, h] - same).max() > 10 * pu.O_MAX_ABS
+    print(f"cached retrieval on new inputs: max abs {worst:.3g}")
 
 
 def test_stream_and_repeat_determinism(park):

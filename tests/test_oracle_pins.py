@@ -595,3 +595,23 @@ def test_key_errors_qk_term_is_metric_distance():
     assert abs(qk - D.mean()) <= 1e-12 * qk
     Deu = po.distances(K, CK, None)[np.arange(50), kl]
     assert abs(raw - Deu.mean()) <= 1e-12 * raw
+
+
+def test_c_assign_is_the_distance_argmin():
+    """The oracle's C assign loop equals the argmin of the written-out distance
+    matrix: on integer inputs (exact sums, real ties resolved to the lowest
+    index) bit for bit, with and without a metric; on random floats up to
+    rounding-order near-ties, of which there are none here."""
+    rng = np.random.default_rng(5)
+    for trial in range(30):
+        N, K, D = int(rng.integers(1, 200)), int(rng.integers(1, 23)), int(rng.integers(1, 40))
+        X = rng.integers(-2, 3, size=(N, D)).astype(float)
+        C = rng.integers(-2, 3, size=(K, D)).astype(float)
+        D_ = po.distances(X, C)
+        want = np.array([min(range(K), key=lambda k: (D_[i, k], k)) for i in range(N)])
+        assert np.array_equal(po.assign(X, C), want), trial
+    X = rng.standard_normal((3000, 64))
+    C = rng.standard_normal((70, 64))
+    M = po.metric(rng.standard_normal((400, 64)))
+    assert np.array_equal(po.assign(X, C), np.argmin(po.distances(X, C), axis=1))
+    assert np.array_equal(po.assign(X, C, M), np.argmin(po.distances(X, C, M), axis=1))

@@ -30,7 +30,7 @@ def test_values_are_bf16_and_inside_the_range_precondition():
         x = g.gen_slice(cfg, t, 0, 0)
         assert np.array_equal(torch.from_numpy(x).to(torch.bfloat16).float().numpy(), x)
         a = np.abs(x[x != 0])
-        assert a.min() >= 2.0 ** -20 and a.max() < 2.0 ** 16 and np.all(np.isfinite(x))
+        assert a.min() >= 2.0 ** -40 and a.max() < 2.0 ** 40 and np.all(np.isfinite(x))
 
 
 def test_normal_v_and_text_tokens():
@@ -60,3 +60,16 @@ def test_rope_rotates_22_21_21_pairs_and_keeps_norms():
     assert moved_pairs(idx(1, 0, 0)).tolist() == list(range(0, 22))
     assert moved_pairs(idx(0, 1, 0)).tolist() == list(range(22, 43))
     assert moved_pairs(idx(0, 0, 1)).tolist() == list(range(43, 64))
+
+
+def test_extreme_magnitudes_stay_inside_the_range():
+    cfg = _small_hunyuan()
+    x = g.gen_slice(cfg, "Q", 0, 0)
+    y = g.with_extreme_magnitudes(x, "bf16", 3, frac_small=0.02, frac_zero=0.01, frac_large=0.01)
+    assert np.array_equal(torch.from_numpy(y).to(torch.bfloat16).float().numpy(), y)
+    a = np.abs(y[y != 0])
+    assert a.min() >= 2.0 ** -40 and a.max() < 2.0 ** 40
+    assert a.min() < 2.0 ** -38 and a.max() > 2.0 ** 38  # both ends are reached
+    assert 0.005 < np.mean(y == 0) < 0.02
+    assert np.array_equal(y, g.with_extreme_magnitudes(x, "bf16", 3, frac_small=0.02, frac_zero=0.01,
+                                                       frac_large=0.01))
