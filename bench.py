@@ -202,10 +202,10 @@ def run_reference(args, cfg):
     if rank != 0:
         return 0
     for _ in range(args.warmup):
-        oracle_layer_estimate(cfg, rows=256, attn_rows=128)
+        oracle_layer_estimate(cfg)
     vals, last = [], None
     for _ in range(args.steps):
-        last = oracle_layer_estimate(cfg, rows=256, attn_rows=128)
+        last = oracle_layer_estimate(cfg)
         vals.append(last["ms_per_layer"])
     v = statistics.median(vals)
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": "ms", "n_gpus": args.gpus,
@@ -286,6 +286,78 @@ def kernel_roofline(name: str, ms_per_launch: float, cfg, counters, peaks, peak_
                                         " bf16_tflops_sustained")}
 
 
+# ----------------------------------------------------------------------------- dense reference, recall
+
+
+def dense_reference(park, torch, cfg, shape, Q, K, V, ws, stream, reps: int = 3) -> dict:
+    """Dense attention on the same tensors, two ways: the library's own
+    block-sparse attention with every block kept (a retrieval at p = 1; the
+    attention kernel's time per launch and the whole park_sparse_attn call), and
+    torch's scaled_dot_product_attention (library flash kernel) for context."""
+    dev = Q.device
+    r1 = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, dev)
+    park.retrieve(Q, K, shape, cfg.NQ, cfg.NK, 1.0, cfg.iters, out=r1, ws=ws, stream=stream)
+    O1 = torch.empty_like(Q)
+    park.sparse_attn(Q, K, V, shape, cfg.NQ, cfg.NK, r1, O=O1, ws=ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    park.profile_enable(True)
+    park.profile_collect()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        park.sparse_attn(Q, K, V, shape, cfg.NQ, cfg.NK, r1, O=O1, ws=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    park.profile_enable(False)
+    prof = park.profile_collect()
+    call_ms = e0.elapsed_time(e1) / reps
+    kt, kn = prof.get("k_sparse_attn_tc", (float("nan"), 1))
+    counters = r1.counters.cpu().tolist()
+    flops = 4.0 * cfg.D * counters[5]
+    del O1
+    import torch.nn.functional as F
+    out = F.scaled_dot_product_attention(Q, K, V)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(reps):
+        out = F.scaled_dot_product_attention(Q, K, V)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    sdpa_ms = e0.elapsed_time(e1) / reps
+    del out
+    torch.cuda.empty_cache()
+    return {"k10_p1_attention_kernel_ms": round(kt / kn, 3), "k10_p1_sparse_attn_call_ms": round(call_ms, 3),
+            "k10_p1_tflops": round(flops / (kt / kn * 1e-3) / 1e12, 1), "torch_sdpa_ms": round(sdpa_ms, 3),
+            "torch_sdpa_tflops": round(4.0 * cfg.D * cfg.B * cfg.H * cfg.N ** 2 / (sdpa_ms * 1e-3) / 1e12, 1),
+            "kept_pair_fraction_p1": round(counters[5] / (cfg.B * cfg.H * cfg.N ** 2), 4)}
+
+
+def recall_per_head(torch, cfg, Q, K, r, rows: int = 1024, seed: int = 0) -> dict:
+    """Attention recall of the kept blocks per head (PARK Table 1): for `rows`
+    query rows per head drawn uniformly (seeded), the share of each row's dense
+    attention mass (float64 softmax(Q K^T / sqrt(D)) over all keys) that falls
+    on keys of the key clusters its query cluster kept; mean over the rows.  A
+    measurement on the library's outputs, outside the timed region."""
+    g = torch.Generator().manual_seed(seed)
+    scale = 1.0 / math.sqrt(cfg.D)
+    vals = []
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            idx = torch.randperm(cfg.N, generator=g)[:rows].to(Q.device)
+            S = (Q[b, h, idx].double() @ K[b, h].double().T) * scale
+            A = torch.softmax(S, dim=1)
+            ql = r.q_labels[b, h, idx].long()
+            kl = r.k_labels[b, h].long()
+            keep = r.mask[b, h][ql][:, kl].bool()
+            vals.append(float((A * keep).sum(1).mean()))
+            del S, A, keep
+    v = np.array(vals)
+    return {"per_head": [round(x, 5) for x in vals], "mean": round(float(v.mean()), 5),
+            "p05": round(float(np.percentile(v, 5)), 5), "worst": round(float(v.min()), 5),
+            "sample": f"{rows} uniformly drawn query rows per head (seed {seed}), dense float64 attention over "
+                      f"all {cfg.N} keys"}
+
+
 # ----------------------------------------------------------------------------- main (our arm)
 
 
@@ -298,6 +370,8 @@ def main():
     ap.add_argument("--config", default=WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention reference")
+    ap.add_argument("--no-quality", action="store_true", help="skip the recall measurement")
     ap.add_argument("--heads", type=int, default=0, help="override H (small cases for profiler captures)")
     ap.add_argument("--variant", default="park", choices=sorted(VARIANTS),
                     help="retrieval variant (PARK Table 3 ablations, Table 10 top-k, size prior, AB-Attention "
@@ -372,10 +446,9 @@ def main():
     torch.cuda.synchronize(dev)
     status = out.status_code()
 
-    # ---- device-resident timing (inputs already in HBM)
+    # ---- device-resident timing (inputs already in HBM), no per-kernel events
     sampler = ClockSampler(dev.index)
-    park.profile_enable(True)
-    park.profile_collect()
+    park.profile_enable(False)
     launches0 = park.launch_count()
     barrier()
     torch.cuda.synchronize(dev)
@@ -389,11 +462,26 @@ def main():
     barrier()
     clocks = sampler.stop()
     launches = park.launch_count() - launches0
-    park.profile_enable(False)
-    prof = park.profile_collect()
     step_ms = e0.elapsed_time(e1) / args.steps
     worst_ms, value = aggregate_ms(step_ms, world, reduce_max)
     counters = out.counters.cpu().tolist()
+
+    # ---- per-kernel breakdown: a separate pass of the same steps with an event pair
+    # around every launch (on the launch stream); the rooflines below use it
+    park.profile_enable(True)
+    park.profile_collect()
+    barrier()
+    torch.cuda.synchronize(dev)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for _ in range(args.steps):
+        step()
+    p1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    park.profile_enable(False)
+    prof = park.profile_collect()
+    profiled_step_ms = p0.elapsed_time(p1) / args.steps
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -418,6 +506,11 @@ def main():
         e2e = {"value": round(e2e_val, 3), "unit": "ms", "h2d_bytes_per_step": int(nbytes),
                "d2h_bytes_per_step": int(O.numel() * O.element_size())}
 
+    # ---- quality and the dense reference (outside the timed regions; every rank
+    # takes the same steps, rank 0 reports)
+    recall = None if args.no_quality else recall_per_head(torch, cfg, Q, K, out)
+    dense = None if args.no_dense else dense_reference(park, torch, cfg, shape, Q, K, V, ws, stream)
+
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
@@ -434,6 +527,11 @@ def main():
         if attn else None
     retrieval_ms = sum(v[0] for k, v in prof.items()
                        if k not in ATTENTION_KERNELS) / args.steps
+    attention_ms = sum(v[0] for k, v in prof.items() if k in ATTENTION_KERNELS) / args.steps
+    if dense:
+        denom = min(dense["k10_p1_attention_kernel_ms"], dense["torch_sdpa_ms"])
+        dense["retrieval_frac_of_dense"] = round(retrieval_ms / denom, 4)
+        dense["layer_vs_dense"] = round(value / denom, 4)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -450,6 +548,9 @@ def main():
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches), "clocks": clocks,
             "status": status,
             "retrieval_ms_per_layer": round(retrieval_ms, 3),
+            "attention_ms_per_layer": round(attention_ms, 3),
+            "profiled_ms_per_step": round(profiled_step_ms, 3),
+            "dense": dense, "recall": recall,
             "kept_block_fraction": round(counters[4] / (cfg.B * cfg.H * cfg.NQ * cfg.NK), 4),
             "kept_pair_fraction": round(counters[5] / (cfg.B * cfg.H * cfg.N ** 2), 4),
             "rechecks": {"query_rows": counters[0], "key_rows": counters[1], "full_rescore_rows": counters[2],

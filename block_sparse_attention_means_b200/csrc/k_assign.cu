@@ -8,6 +8,8 @@
 // winner is certified when the runner-up is more than 2 beta above it;
 // otherwise the row is listed for a float64 rescore against every centroid
 // (k_rescore_full), so labels agree with a float64 evaluation of the definition.
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace park {
@@ -74,90 +76,112 @@ __global__ void k_recheck(const T* __restrict__ X, const T* __restrict__ C, cons
     }
 }
 
-// Full rescore (mode 1) with one CTA per listed row: warp w takes centroids
-// w, w + 8, ..., two at a time; the CTA keeps the smallest distance, ties to the
-// lowest index.
+// Full rescore of the rows the tensor-core assign could not certify, listed per
+// head.  CTA (s, bh) takes groups of up to eight listed rows of head bh (groups
+// s, s + gridDim.x, ...); warp w scores centroids w, w + 8, ... against every row
+// of the group (lane l holds elements l, l + 32, l + 64, l + 96 of each row), so
+// every centroid operand is read once per group instead of once per row.  Each
+// distance is the same float64 expression, summed in the same order, as a
+// one-row evaluation; ties go to the lowest index.
+constexpr int kRescoreRows = 8;
+
 template <typename T, bool METRIC>
 __global__ __launch_bounds__(256) void k_rescore_full(const T* __restrict__ X, const T* __restrict__ C,
                                                       const double* __restrict__ w64, const double* __restrict__ b64,
                                                       int N, int D, int K, int32_t* __restrict__ labels,
                                                       const int32_t* __restrict__ rows,
-                                                      const int32_t* __restrict__ count_ptr,
+                                                      const int32_t* __restrict__ counts,
                                                       int64_t* __restrict__ counters, int cnt_slot) {
-    __shared__ double s_best[8];
-    __shared__ int s_idx[8];
+    constexpr int R = kRescoreRows;
+    __shared__ double s_best[8][R];
+    __shared__ int s_idx[8][R];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int count = *count_ptr;
-    if (blockIdx.x == 0 && threadIdx.x == 0 && counters != nullptr) {
+    const int bh = blockIdx.y;
+    const int count = counts[bh];
+    if (blockIdx.x == 0 && threadIdx.x == 0 && counters != nullptr && count > 0) {
         atomicAdd((unsigned long long*)(counters + cnt_slot), (unsigned long long)count);
         atomicAdd((unsigned long long*)(counters + PARK_CNT_FULL_RESCORE), (unsigned long long)count);
     }
-    for (int e = blockIdx.x; e < count; e += gridDim.x) {
-        const int gr = rows[e];
-        const int bh = gr / N;
-        const T* x = X + (size_t)gr * D;
-        double xv[4];
+    const int32_t* list = rows + (size_t)bh * N;
+    for (int g0 = blockIdx.x * R; g0 < count; g0 += gridDim.x * R) {
+        const int nr = min(R, count - g0);
+        double xv[R][4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int j = lane + 32 * u;
-            xv[u] = j < D ? Elem<T>::to_double(x, j) : 0.0;
+        for (int r = 0; r < R; ++r) {
+            const int gr = list[g0 + (r < nr ? r : 0)];  // rows past the group repeat its first row
+            const T* x = X + (size_t)gr * D;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = lane + 32 * u;
+                xv[r][u] = j < D ? Elem<T>::to_double(x, j) : 0.0;
+            }
         }
-        auto partial = [&](int k) -> double {  // this lane's share of distance k
-            double s = 0.0;
+        double bd[R];
+        int best[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            bd[r] = __longlong_as_double(0x7ff0000000000000ll);
+            best[r] = K;
+        }
+        for (int k = warp; k < K; k += 8) {
+            double cv[4];
             if (METRIC) {
                 const double* w = w64 + ((size_t)bh * K + k) * D;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int j = lane + 32 * u;
-                    if (j < D) s = __fma_rn(xv[u], w[j], s);
+                    cv[u] = j < D ? w[j] : 0.0;
                 }
             } else {
                 const T* c = C + ((size_t)bh * K + k) * D;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int j = lane + 32 * u;
-                    if (j < D) {
-                        const double d = xv[u] - Elem<T>::to_double(c, j);
-                        s = __fma_rn(d, d, s);
-                    }
+                    cv[u] = j < D ? Elem<T>::to_double(c, j) : 0.0;
                 }
             }
-            return s;
-        };
-        double bd = __longlong_as_double(0x7ff0000000000000ll);
-        int best = K;
-        for (int k = warp; k < K; k += 16) {  // centroids k and k + 8 in flight together
-            const int k2 = k + 8;
-            double s1 = partial(k), s2 = k2 < K ? partial(k2) : 0.0;
-            s1 = warp_sum(s1);
-            s2 = warp_sum(s2);
-            const double d1 = METRIC ? b64[(size_t)bh * K + k] - 2.0 * s1 : s1;
-            if (d1 < bd) {
-                bd = d1;
-                best = k;
-            }
-            if (k2 < K) {
-                const double d2 = METRIC ? b64[(size_t)bh * K + k2] - 2.0 * s2 : s2;
-                if (d2 < bd) {  // k2 > every index seen so far by this warp
-                    bd = d2;
-                    best = k2;
+            const double bk = METRIC ? b64[(size_t)bh * K + k] : 0.0;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                double s = 0.0;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = lane + 32 * u;
+                    if (j < D) {
+                        if (METRIC) {
+                            s = __fma_rn(xv[r][u], cv[u], s);
+                        } else {
+                            const double d = xv[r][u] - cv[u];
+                            s = __fma_rn(d, d, s);
+                        }
+                    }
+                }
+                s = warp_sum(s);
+                const double d = METRIC ? bk - 2.0 * s : s;
+                if (d < bd[r]) {  // k grows within the warp: the first of equal distances stays
+                    bd[r] = d;
+                    best[r] = k;
                 }
             }
         }
         if (lane == 0) {
-            s_best[warp] = bd;
-            s_idx[warp] = best;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                s_best[warp][r] = bd[r];
+                s_idx[warp][r] = best[r];
+            }
         }
         __syncthreads();
-        if (threadIdx.x == 0) {
-            double b = s_best[0];
-            int bi = s_idx[0];
+        if (threadIdx.x < nr) {
+            const int r = threadIdx.x;
+            double b = s_best[0][r];
+            int bi = s_idx[0][r];
             for (int q = 1; q < 8; ++q)
-                if (s_best[q] < b || (s_best[q] == b && s_idx[q] < bi)) {
-                    b = s_best[q];
-                    bi = s_idx[q];
+                if (s_best[q][r] < b || (s_best[q][r] == b && s_idx[q][r] < bi)) {
+                    b = s_best[q][r];
+                    bi = s_idx[q][r];
                 }
-            labels[gr] = bi;
+            labels[list[g0 + r]] = bi;
         }
         __syncthreads();
     }
@@ -196,24 +220,25 @@ int launch_recheck(const void* X, int dtype, int BH, int N, int D, int K, const 
     const bool metric = w64 != nullptr;
     if (all_rows) return launch_recheck_rows(X, dtype, BH, N, D, K, C, w64, b64, labels, 0, num_sms, st);
     ::park::prof_begin(st);
-    const int fb = num_sms * 4;
+    // per head: enough CTAs for about four per SM over all heads
+    const dim3 fb((unsigned)std::max(1, (num_sms * 4 + BH - 1) / BH), (unsigned)BH);
     if (dtype == PARK_BF16) {
         if (metric)
             k_rescore_full<bf16_t, true><<<fb, 256, 0, st>>>((const bf16_t*)X, (const bf16_t*)C, w64, b64, N, D, K,
-                                                             labels, lists.full_row, lists.counts + 1, counters,
+                                                             labels, lists.full_row, lists.counts, counters,
                                                              cnt_slot);
         else
             k_rescore_full<bf16_t, false><<<fb, 256, 0, st>>>((const bf16_t*)X, (const bf16_t*)C, w64, b64, N, D, K,
-                                                              labels, lists.full_row, lists.counts + 1, counters,
+                                                              labels, lists.full_row, lists.counts, counters,
                                                               cnt_slot);
     } else {
         if (metric)
             k_rescore_full<float, true><<<fb, 256, 0, st>>>((const float*)X, (const float*)C, w64, b64, N, D, K,
-                                                            labels, lists.full_row, lists.counts + 1, counters,
+                                                            labels, lists.full_row, lists.counts, counters,
                                                             cnt_slot);
         else
             k_rescore_full<float, false><<<fb, 256, 0, st>>>((const float*)X, (const float*)C, w64, b64, N, D, K,
-                                                             labels, lists.full_row, lists.counts + 1, counters,
+                                                             labels, lists.full_row, lists.counts, counters,
                                                              cnt_slot);
     }
     PARK_TRY_LAUNCH("k_rescore_full", st);

@@ -237,8 +237,8 @@ __global__ void __launch_bounds__(320, 1)
                 const float beta = gamma * xn * wmax[bh] + 4.8e-7f * bmax[bh] + xn * 0x1p-118f + 1e-30f;
                 labels[gr] = i0[w];
                 if (!(second - best > 2.f * beta)) {
-                    const int pos = atomicAdd(lists.counts + 1, 1);
-                    lists.full_row[pos] = (int32_t)gr;
+                    const int pos = atomicAdd(lists.counts + bh, 1);
+                    lists.full_row[(size_t)bh * N + pos] = (int32_t)gr;
                 }
             }
         }

@@ -243,16 +243,18 @@ __global__ void k_centroid_prep(const T* __restrict__ C, int K, int D, float* __
     }
 }
 
-// QRKC operands for 16 centroids per CTA: M (symmetric, float64) is staged once
-// in shared memory, thread (a, half) forms w_a = sum_b M[b][a] c_b for eight
-// centroids (row b of M: conflict-free), then per centroid bias = c . w and
-// ||w||^2 are reduced over the 128 threads of its half in a fixed order.
+// QRKC operands for 64 centroids per CTA: M (symmetric, float64) is staged once
+// in shared memory, thread (a, half) forms w_a = sum_b M[b][a] c_b for 32
+// centroids (row b of M: conflict-free; the centroids' pairs c_b, c_b+1 as one
+// 16-byte broadcast), then per centroid bias = c . w and ||w||^2 are reduced
+// over the 128 threads of its half in a fixed order.
 // w and the bias are taken for 2^-e M, e the binary exponent of the head's
 // largest diagonal entry (|M_ab| <= max_a M_aa), so that the float32 scores stay
 // far from overflow over the whole input range (|x| < 2^40 gives M up to 2^80).
 // A power-of-two scale is exact in float64 and multiplies every score of the
 // head by the same factor, so it changes no argmin.
-constexpr int kPrepCents = 16;
+constexpr int kPrepPerThread = 32;
+constexpr int kPrepCents = 2 * kPrepPerThread;
 
 template <typename T>
 __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restrict__ C, int K, int D,
@@ -268,8 +270,18 @@ __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restric
     __shared__ double s_scale;
     const int bh = blockIdx.y, k0 = blockIdx.x * kPrepCents, t = threadIdx.x;
     const int a = t & 127, half = t >> 7, lane = t & 31, wq = (t >> 5) & 3;
-    const double* M = Mall + (size_t)bh * D * D;
-    for (int i = t; i < D * D; i += blockDim.x) Ms[i] = M[i];
+    const double2* M2 = reinterpret_cast<const double2*>(Mall + (size_t)bh * D * D);
+    double2* Ms2 = reinterpret_cast<double2*>(Ms);
+    const int n2 = D * D / 2;
+    for (int i0 = t; i0 < n2; i0 += 256 * 8) {  // eight 16-byte loads in flight per thread
+        double2 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (i0 + 256 * u < n2) v[u] = M2[i0 + 256 * u];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (i0 + 256 * u < n2) Ms2[i0 + 256 * u] = v[u];
+    }
     for (int i = t; i < kPrepCents * D; i += blockDim.x) {
         const int c = i / D, j = i - c * D, k = k0 + c;
         Cs[i] = k < K ? Elem<T>::to_double(C + ((size_t)bh * K + k) * D, j) : 0.0;
@@ -286,21 +298,26 @@ __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restric
     }
     __syncthreads();
     const double scale = s_scale;
-    double w[8];
+    double w[kPrepPerThread];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) w[c] = 0.0;
+    for (int c = 0; c < kPrepPerThread; ++c) w[c] = 0.0;
     if (a < D) {
-        for (int b = 0; b < D; ++b) {
-            const double m = Ms[b * D + a];
+        const double* cbase = Cs + half * kPrepPerThread * D;
+        for (int b = 0; b < D; b += 2) {  // D is even
+            const double m0 = Ms[b * D + a], m1 = Ms[(b + 1) * D + a];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) w[c] = __fma_rn(m, Cs[(half * 8 + c) * D + b], w[c]);
+            for (int c = 0; c < kPrepPerThread; ++c) {
+                const double2 cv = *reinterpret_cast<const double2*>(cbase + c * D + b);
+                w[c] = __fma_rn(m0, cv.x, w[c]);
+                w[c] = __fma_rn(m1, cv.y, w[c]);
+            }
         }
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c) w[c] *= scale;  // exact
+    for (int c = 0; c < kPrepPerThread; ++c) w[c] *= scale;  // exact
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const int cc = half * 8 + c, k = k0 + cc;
+    for (int c = 0; c < kPrepPerThread; ++c) {
+        const int cc = half * kPrepPerThread + c, k = k0 + cc;
         const double ca = a < D ? Cs[cc * D + a] : 0.0;
         if (a < D && k < K) {
             w64[((size_t)bh * K + k) * D + a] = w[c];
@@ -322,10 +339,10 @@ __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restric
     if (t < kPrepCents && k0 + t < K) {
         const int k = k0 + t;
         const double b = ((red[t][0][0] + red[t][1][0]) + red[t][2][0]) + red[t][3][0];
-        const double n2 = ((red[t][0][1] + red[t][1][1]) + red[t][2][1]) + red[t][3][1];
+        const double n2w = ((red[t][0][1] + red[t][1][1]) + red[t][2][1]) + red[t][3][1];
         bias64[(size_t)bh * K + k] = b;
         bias32[(size_t)bh * bias_ld + k] = __double2float_rn(b);
-        atomic_max_nonneg(wmax + bh, round_up_f(__double2float_ru(sqrt(n2))));
+        atomic_max_nonneg(wmax + bh, round_up_f(__double2float_ru(sqrt(n2w))));
         atomic_max_nonneg(bmax + bh, round_up_f(__double2float_ru(fabs(b))));
     }
 }

@@ -25,8 +25,8 @@ struct CentroidOps {
 };
 
 struct Lists {
-    int32_t* full_row;  // [BH*N] bh*N + i of rows rescored against every centroid
-    int32_t* counts;    // [4]: (spare), full count, (spare)
+    int32_t* full_row;  // [BH][N]: per head, bh*N + i of the rows to rescore against every centroid
+    int32_t* counts;    // [BH]: rows listed per head (zeroed before each assign)
 };
 
 // ---- k_prep.cu

@@ -146,7 +146,7 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
     w.wmax = c.take(BH * 4);
     w.bmax = c.take(BH * 4);
     w.lfull = c.take(BH * N * 4);
-    w.lcnt = c.take(16 * 4);
+    w.lcnt = c.take(BH * 4);
     w.hist = c.take(BH * Km * nchunks * 4);
     w.rho = c.take(BH * NQ * 4);
     w.plist = c.take(BH * NQ * 4);
@@ -336,7 +336,7 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
     for (int it = 0; it < iters; ++it) {
         PARK_CHECK(memset_async(ops.wmax, (size_t)BH * 4, st));
         PARK_CHECK(memset_async(ops.bmax, (size_t)BH * 4, st));
-        PARK_CHECK(memset_async(lists.counts, 16 * 4, st));
+        PARK_CHECK(memset_async(lists.counts, (size_t)BH * 4, st));
         PARK_CHECK(launch_centroid_prep(s.C, d.dtype, BH, K, D, s.M, ops, st));
         if (bf16) {
             PARK_CHECK(launch_assign_tc(s.X, BH, N, K, ops, s.xnorm, gamma, s.labels, lists, s.status, num_sms, st));

@@ -64,10 +64,29 @@ def metric(Q):
     return (Q.T @ Q) / Q.shape[0]
 
 
+class QueryMetric:
+    """The QRKC metric of a set of queries, M = Q^T Q / N, together with a
+    factor F = R^T / sqrt(N) from the QR decomposition Q = Q_1 R (so that
+    M = F F^T): keys are transformed by F^T before clustering, as the pages put
+    it (PARK abstract).  Taking F from the queries themselves keeps every
+    direction in which the queries are small; a factor of M from its
+    eigendecomposition loses the directions whose eigenvalues fall below
+    float64 rounding of the largest one, which inputs spanning many binades
+    reach."""
+
+    def __init__(self, Q):
+        Q = np.asarray(Q, dtype=np.float64)
+        self.M = metric(Q)
+        R = np.linalg.qr(Q, mode="r")
+        self.F = R.T / math.sqrt(Q.shape[0])
+
+
 def metric_factor(M):
-    """F with M = F F^T (eigendecomposition, clipped at 0 for a PSD M), so that
-    (x - c)^T M (x - c) = ||F^T x - F^T c||^2: keys transformed before
-    clustering, as the pages put it (PARK abstract)."""
+    """F with M = F F^T, so that (x - c)^T M (x - c) = ||F^T x - F^T c||^2.
+    A QueryMetric carries its own factor; a plain matrix M is factored by its
+    eigendecomposition (clipped at 0 for a PSD M)."""
+    if isinstance(M, QueryMetric):
+        return M.F
     lam, V = np.linalg.eigh(np.asarray(M, dtype=np.float64))
     return V * np.sqrt(np.clip(lam, 0.0, None))
 
@@ -85,8 +104,9 @@ def strided_init(X, K):
 
 def distances(X, C, M=None, row_block=4096):
     """D[i, k] = (x_i - c_k)^T M (x_i - c_k); M = None means the identity
-    (standard Euclidean K-means, PARK Figure 2 caption).  For a metric the keys
-    and centroids are first transformed by F^T with M = F F^T."""
+    (standard Euclidean K-means, PARK Figure 2 caption).  For a metric (a
+    matrix or a QueryMetric) the keys and centroids are first transformed by
+    F^T with M = F F^T."""
     X = np.asarray(X, dtype=np.float64)
     C = np.asarray(C, dtype=np.float64)
     if M is not None:
@@ -435,15 +455,17 @@ def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", to
     K = np.asarray(K, dtype=np.float64)
     d = Q.shape[1]
     scale = 1.0 / math.sqrt(d)
-    M = metric(Q)
+    qm = QueryMetric(Q)
+    M = qm.M
+    km = qm if qrkc else None
     q_hist = k_hist = None
     if window is None:
         q_labels, CQ, q_hist = kmeans(Q, NQ, iters, None, dtype, init=q_init, history=True)
-        k_labels, CK, k_hist = kmeans(K, NK, iters, M if qrkc else None, dtype, init=k_init, history=True)
+        k_labels, CK, k_hist = kmeans(K, NK, iters, km, dtype, init=k_init, history=True)
     else:
         from . import hva_oracle as hva
         q_labels, CQ = hva.local_kmeans(Q, NQ, iters, grid, window, None, dtype)
-        k_labels, CK = hva.local_kmeans(K, NK, iters, grid, window, M if qrkc else None, dtype)
+        k_labels, CK = hva.local_kmeans(K, NK, iters, grid, window, km, dtype)
     q_counts = np.bincount(q_labels, minlength=NQ)
     k_counts = np.bincount(k_labels, minlength=NK)
     if pama_mode == "full":
@@ -469,7 +491,7 @@ def retrieve_head(Q, K, NQ, NK, p, iters, dtype, qrkc=True, pama_mode="full", to
     return dict(M=M, q_labels=q_labels, k_labels=k_labels, q_centroids=CQ, k_centroids=CK,
                 q_counts=q_counts, k_counts=k_counts, importance=I, mask=mask, weight=weight,
                 q_perm=q_perm, q_offsets=q_off, k_perm=k_perm, k_offsets=k_off, q_hist=q_hist, k_hist=k_hist,
-                qrkc=qrkc)
+                qrkc=qrkc, k_metric=km)
 
 
 def layer_head(Q, K, V, NQ, NK, p, iters, dtype, **kw):

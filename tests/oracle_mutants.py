@@ -19,9 +19,11 @@ MUTS = [
     ("metric_n1", P, "return (Q.T @ Q) / Q.shape[0]", "return (Q.T @ Q) / (Q.shape[0] - 1)"),
     ("init_offset", P, "[(np.arange(K) * N) // K]", "[(np.arange(K) * N + N // (2 * K)) // K]"),
     ("dist_l1", P, "np.sum(diff * diff, axis=2)", "np.sum(np.abs(diff), axis=2)"),
-    ("metric_transpose", P, "        X = X @ F\n        C = C @ F", "        X = X @ F.T\n        C = C @ F.T"),
-    ("tie_last", P, "return np.argmin(distances(X, C, M), axis=1).astype(np.int64)",
-     "Dm = distances(X, C, M)\n    return (Dm.shape[1] - 1 - np.argmin(Dm[:, ::-1], axis=1)).astype(np.int64)"),
+    ("metric_transpose", P, "        X = X @ F\n        C = C @ F\n    X = np.ascontiguousarray(X)",
+     "        X = X @ F.T\n        C = C @ F.T\n    X = np.ascontiguousarray(X)"),
+    ("query_factor_T", P, "self.F = R.T / math.sqrt(Q.shape[0])", "self.F = R / math.sqrt(Q.shape[0])"),
+    ("assign_c_l1", "oracle/assign.c", "                s[0] = s[0] + d0 * d0;", "                s[0] = s[0] + (d0 < 0 ? -d0 : d0);"),
+    ("tie_last", "oracle/assign.c", "if (arg < 0 || s[u] < best) { /* strict", "if (arg < 0 || s[u] <= best) { /* strict"),
     ("mean_double_round", P, "return round_to(sums / float(n), dtype)",
      "return round_to(np.float64(np.float32(sums / float(n))), dtype)"),
     ("empty_zero", P, "        if n:\n            C[k] = exact_mean(X[order[start:start + n]], dtype)",
@@ -84,9 +86,10 @@ MUTS2 = [
     ("merge_rounds_plus", H, "    for _ in range(rounds):", "    for _ in range(rounds + 1):"),
     ("merge_root_nofollow", H, "        while root[g] != g:\n            g = root[g]", "        pass"),
     ("padded_floor", H, "return KEY_GROUP * ((k_counts + KEY_GROUP - 1) // KEY_GROUP)", "return KEY_GROUP * (k_counts // KEY_GROUP)"),
-    ("q_kmeans_metric", P, "        q_labels, CQ = kmeans(Q, NQ, iters, None, dtype)", "        q_labels, CQ = kmeans(Q, NQ, iters, M, dtype)"),
-    ("k_kmeans_euclid", P, "        k_labels, CK = kmeans(K, NK, iters, M if qrkc else None, dtype)",
-     "        k_labels, CK = kmeans(K, NK, iters, None, dtype)"),
+    ("q_kmeans_metric", P, "q_labels, CQ, q_hist = kmeans(Q, NQ, iters, None, dtype,",
+     "q_labels, CQ, q_hist = kmeans(Q, NQ, iters, qm, dtype,"),
+    ("k_kmeans_euclid", P, "k_labels, CK, k_hist = kmeans(K, NK, iters, km, dtype,",
+     "k_labels, CK, k_hist = kmeans(K, NK, iters, None, dtype,"),
     ("pama_query_centroids", P, "        I = pama(Q, q_labels, NQ, CK, k_counts, scale, size_prior=size_prior)",
      "        I = pama(Q, q_labels, NQ, CQ, k_counts, scale, size_prior=size_prior)"),
     ("layer_scale_n", P, "    scale = 1.0 / math.sqrt(np.asarray(Q).shape[1])\n    r[\"O\"]", "    scale = 1.0 / math.sqrt(np.asarray(Q).shape[0])\n    r[\"O\"]"),
@@ -99,7 +102,7 @@ MUTS2 = [
 def run(name, f, old, new):
     with tempfile.TemporaryDirectory(prefix=".oracle_mutants_", dir=ROOT) as dst:
         for d in ("oracle", "tests", "synth"):
-            shutil.copytree(os.path.join(ROOT, d), os.path.join(dst, d), ignore=shutil.ignore_patterns("__pycache__"))
+            shutil.copytree(os.path.join(ROOT, d), os.path.join(dst, d), ignore=shutil.ignore_patterns("__pycache__", "*.so"))
         shutil.copy(os.path.join(ROOT, "pytest.ini"), dst)
         path = os.path.join(dst, f)
         s = open(path).read()

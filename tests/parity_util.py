@@ -135,7 +135,7 @@ def compare_retrieval(gpu, ref_heads, NQ: int, NK: int, Q=None, K=None, p=None, 
             got, want = lab[b, h], ref[f"{side}_labels"]
             bad = np.nonzero(got != want)[0]
             if bad.size and ties and ref.get(f"{side}_hist") is not None:
-                M = ref["M"] if (side == "k" and ref.get("qrkc", True)) else None
+                M = ref.get("k_metric") if side == "k" else None
                 X = Qh[bh] if side == "q" else Kh[bh]
                 bad, excused = label_ties(X, ref[f"{side}_hist"][-1], M, got, want)
                 rep[f"{side}_label_ties"] += int(excused.size)

@@ -155,14 +155,15 @@ def test_step_injection_matches_oracle(park, name, step):
         for h, ref in enumerate(refs):
             x, y = Q[0, h].astype(np.float64), K[0, h].astype(np.float64)
             ql = po.assign(x, ref["q_hist"][0])
-            kl = po.assign(y, ref["k_hist"][0], ref["M"])
+            kl = po.assign(y, ref["k_hist"][0], ref["k_metric"])
             want.append(dict(ref, q_labels=ql, k_labels=kl, q_centroids=ref["q_hist"][1],
                              k_centroids=ref["k_hist"][1], q_hist=ref["q_hist"][:1], k_hist=ref["k_hist"][:1]))
         ql, kl = r.q_labels.cpu().numpy()[0], r.k_labels.cpu().numpy()[0]
         qc, kc = pu.np64(r.q_centroids)[0], pu.np64(r.k_centroids)[0]
         ties = 0
         for h, w in enumerate(want):
-            for side, got, cen, X, M in (("q", ql[h], qc[h], Q[0, h], None), ("k", kl[h], kc[h], K[0, h], w["M"])):
+            for side, got, cen, X, M in (("q", ql[h], qc[h], Q[0, h], None),
+                                         ("k", kl[h], kc[h], K[0, h], w["k_metric"])):
                 bad, exc = pu.label_ties(X, w[f"{side}_hist"][0], M, got, w[f"{side}_labels"])
                 assert np.setdiff1d(bad, exc).size == 0, f"head {h} {side}: labels differ not at a tie"
                 ties += exc.size

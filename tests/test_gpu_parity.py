@@ -163,10 +163,10 @@ def test_per_step_injection_small(park):
             x = Q[b, h].astype(np.float64)
             y = K[b, h].astype(np.float64)
             _, _, hq = po.kmeans(x, cfg.NQ, t + 1, None, "bf16", history=True)
-            _, _, hk = po.kmeans(y, cfg.NK, t + 1, po.metric(x), "bf16", history=True)
+            _, _, hk = po.kmeans(y, cfg.NK, t + 1, po.QueryMetric(x), "bf16", history=True)
             qc[0, h], kc[0, h] = hq[t], hk[t]
             lq, cq = po.kmeans(x, cfg.NQ, 1, None, "bf16", init=hq[t])
-            lk, ck = po.kmeans(y, cfg.NK, 1, po.metric(x), "bf16", init=hk[t])
+            lk, ck = po.kmeans(y, cfg.NK, 1, po.QueryMetric(x), "bf16", init=hk[t])
             want.append((lq, cq, lk, ck))
         out.q_centroids.copy_(pu.to_device(qc, dt))
         out.k_centroids.copy_(pu.to_device(kc, dt))
