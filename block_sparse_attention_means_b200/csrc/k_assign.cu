@@ -123,44 +123,58 @@ __global__ __launch_bounds__(256) void k_rescore_full(const T* __restrict__ X, c
             bd[r] = __longlong_as_double(0x7ff0000000000000ll);
             best[r] = K;
         }
-        for (int k = warp; k < K; k += 8) {
-            double cv[4];
-            if (METRIC) {
-                const double* w = w64 + ((size_t)bh * K + k) * D;
+        // four centroids per warp step (k, k + 8, k + 16, k + 24): their operand loads
+        // are in flight together
+        constexpr int U = 4;
+        for (int k0 = warp; k0 < K; k0 += 8 * U) {
+            double cv[U][4], bk[U];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int j = lane + 32 * u;
-                    cv[u] = j < D ? w[j] : 0.0;
-                }
-            } else {
-                const T* c = C + ((size_t)bh * K + k) * D;
+            for (int v = 0; v < U; ++v) {
+                const int k = k0 + 8 * v;
+                const bool kin = k < K;
+                if (METRIC) {
+                    const double* w = w64 + ((size_t)bh * K + (kin ? k : 0)) * D;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int j = lane + 32 * u;
-                    cv[u] = j < D ? Elem<T>::to_double(c, j) : 0.0;
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = lane + 32 * u;
+                        cv[v][u] = (kin && j < D) ? w[j] : 0.0;
+                    }
+                    bk[v] = kin ? b64[(size_t)bh * K + k] : 0.0;
+                } else {
+                    const T* c = C + ((size_t)bh * K + (kin ? k : 0)) * D;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = lane + 32 * u;
+                        cv[v][u] = (kin && j < D) ? Elem<T>::to_double(c, j) : 0.0;
+                    }
+                    bk[v] = 0.0;
                 }
             }
-            const double bk = METRIC ? b64[(size_t)bh * K + k] : 0.0;
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                double s = 0.0;
+            for (int v = 0; v < U; ++v) {
+                const int k = k0 + 8 * v;
+                if (k >= K) break;  // uniform over the warp
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int j = lane + 32 * u;
-                    if (j < D) {
-                        if (METRIC) {
-                            s = __fma_rn(xv[r][u], cv[u], s);
-                        } else {
-                            const double d = xv[r][u] - cv[u];
-                            s = __fma_rn(d, d, s);
+                for (int r = 0; r < R; ++r) {
+                    double s = 0.0;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = lane + 32 * u;
+                        if (j < D) {
+                            if (METRIC) {
+                                s = __fma_rn(xv[r][u], cv[v][u], s);
+                            } else {
+                                const double d = xv[r][u] - cv[v][u];
+                                s = __fma_rn(d, d, s);
+                            }
                         }
                     }
-                }
-                s = warp_sum(s);
-                const double d = METRIC ? bk - 2.0 * s : s;
-                if (d < bd[r]) {  // k grows within the warp: the first of equal distances stays
-                    bd[r] = d;
-                    best[r] = k;
+                    s = warp_sum(s);
+                    const double d = METRIC ? bk[v] - 2.0 * s : s;
+                    if (d < bd[r]) {  // k grows within the warp: the first of equal distances stays
+                        bd[r] = d;
+                        best[r] = k;
+                    }
                 }
             }
         }

@@ -202,12 +202,23 @@ __global__ __launch_bounds__(512) void k_topp(const float* __restrict__ importan
     } else if (cut < 0) {
         ok = false;  // float sums fell short of p: let float64 decide
     } else {
+        // The exact importances of a row sum to 1 (every query's Softmax does), so the
+        // error of a running sum is minus the error of what lies after it: with
+        // T = sum of every computed value and each value within rh of the exact one
+        // (relative), the exact running sum through sorted position e lies within
+        // rh / (1 - rh) (T - S[e]) of S[e] - (T - 1).  After the cut only about 1 - p
+        // of the mass is left, so this is about (1 - p) / p times the plain bound.
+        // The order of the last kept and the first dropped value is certain when
+        // the exact values, each within re of the computed one, cannot swap.
         const double vc = (double)sv[cut];
         const double eps = 1e-12;
-        bool ord = cut + 1 >= L || vc * (1.0 - rh) > (double)sv[cut + 1] * (1.0 + 2.0 * rh) + 1e-300;
-        bool hi = S[cut] * (1.0 - 2.0 * rh) - eps >= (double)p;
-        bool lo = S[cut] * (1.0 + 2.0 * rh) + eps - vc * (1.0 - rh) < (double)p;
-        ok = ord && hi && lo;
+        const double re = rh + 0x1p-23;  // + the float rounding of the stored values
+        const double T = S[L - 1], E = T - 1.0, rp = re / (1.0 - re);
+        const double Sc = S[cut], Sb = cut > 0 ? S[cut - 1] : 0.0;
+        bool ord = cut + 1 >= L || vc * (1.0 - re) > (double)sv[cut + 1] * (1.0 + re) + 1e-300;
+        bool hi = Sc - E - rp * (T - Sc) - eps >= (double)p;  // the exact sum through the cut reaches p
+        bool lo = Sb - E + rp * (T - Sb) + eps < (double)p;   // and the one before it does not
+        ok = rh < 0.5 && ord && hi && lo;
     }
     if (!ok) {
         if (t == 0) {

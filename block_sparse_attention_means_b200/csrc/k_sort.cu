@@ -199,13 +199,29 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
     auto add_piece = [&](const uint4& v) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         if (BF16) {
+            // the common case, decided once per 16-byte piece with 16-bit SIMD compares:
+            // every element is 0 or has 2^-20 <= |x| < 2^16 (biased exponent 107..142)
+            uint32_t bad = 0;
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                const uint32_t b = (e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16);
-                const uint32_t ex = (b >> 23) & 0xFFu;
-                const bool fast = (ex - 107u) <= 35u || ex == 0u;  // 2^-20 <= |x| < 2^16, or 0
-                part[e] += fast ? (double)__uint_as_float(b) : 0.0;
-                if (!fast) fixed64_add(acc_lo[e], acc_hi[e], b);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t ex = (w[q] >> 7) & 0x00FF00FFu;
+                const uint32_t in = __vcmpgeu2(ex, 0x006B006Bu) & __vcmpleu2(ex, 0x008E008Eu);
+                bad |= ~(in | __vcmpeq2(w[q] & 0x7FFF7FFFu, 0u));
+            }
+            if (bad == 0) {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    part[e] += (double)__uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+            } else {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    const uint32_t b = (e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16);
+                    const uint32_t ex = (b >> 23) & 0xFFu;
+                    if ((ex - 107u) <= 35u || (b & 0x7FFFFFFFu) == 0u)
+                        part[e] += (double)__uint_as_float(b);
+                    else
+                        fixed64_add(acc_lo[e], acc_hi[e], b);
+                }
             }
             if (++rows_in_part == 1024) flush();
         } else {
