@@ -38,23 +38,6 @@ struct AsSmem {
     int abort;
 };
 
-__device__ __forceinline__ float fmin3(float a, float b, float c) {
-    float d;
-    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-
-// Scores s1 (column col) and s2 (column col + 1) into a tracker (v0: smallest,
-// i0: its column, v1: second smallest).  The second smallest of {v0, v1, s1, s2}
-// with v0 <= v1 is min(v1, max(v0, min(s1, s2)), max(s1, s2)).
-__device__ __forceinline__ void track_pair(float s1, float s2, int col, float& v0, float& v1, int& i0) {
-    const float mn = fminf(s1, s2), mx = fmaxf(s1, s2);
-    const int ic = s2 < s1 ? col + 1 : col;
-    i0 = mn < v0 ? ic : i0;
-    v1 = fmin3(v1, fmaxf(v0, mn), mx);
-    v0 = fminf(v0, mn);
-}
-
 }  // namespace
 
 template <int KW>
@@ -222,18 +205,14 @@ __global__ void __launch_bounds__(320, 1)
                             const int g = 2 * gp + h;
                             const int cb = c * AS_CH + 32 * g + 4 * q;
                             const float4 b4 = *reinterpret_cast<const float4*>(sbias + cb);
-                            const float2 m2 = make_float2(-2.f, -2.f);
-                            const float2 s01 = __ffma2_rn(make_float2(__uint_as_float(acc[h][4 * q]),
-                                                                      __uint_as_float(acc[h][4 * q + 1])),
-                                                          m2, make_float2(b4.x, b4.y));
-                            const float2 s23 = __ffma2_rn(make_float2(__uint_as_float(acc[h][4 * q + 2]),
-                                                                      __uint_as_float(acc[h][4 * q + 3])),
-                                                          m2, make_float2(b4.z, b4.w));
-                            // two scores at a time; the same (smallest, its column, second
-                            // smallest) as taking them one by one, strict comparisons keeping
-                            // the first of equal scores
-                            track_pair(s01.x, s01.y, cb, v0[g], v1[g], i0[g]);
-                            track_pair(s23.x, s23.y, cb + 2, v0[g], v1[g], i0[g]);
+                            const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float sc = fmaf(-2.f, __uint_as_float(acc[h][4 * q + e]), bv[e]);
+                                v1[g] = fminf(v1[g], fmaxf(v0[g], sc));
+                                i0[g] = sc < v0[g] ? cb + e : i0[g];  // strict: the first of equal scores stays
+                                v0[g] = fminf(v0[g], sc);
+                            }
                         }
                 }
                 ++G;

@@ -152,13 +152,29 @@ int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist
 // ---------------------------------------------------------------- update
 // 128 threads.  Each thread owns one 16-byte piece of a row: VEC elements at
 // piece p = t % CPR, and rows s, s + RPI, ... of the cluster (s = t / CPR).
-// Every element goes into a signed 128-bit fixed-point sum of x * 2^64
-// (fixed64_add, exact for the whole range precondition).  bf16 elements with
-// 2^-20 <= |x| < 2^16 -- all of them on unit-scale data -- first go through a
-// float64 partial sum per element that is exact for 1024 rows (such values are
-// multiples of 2^-27 below 2^16, so 1024 of them need at most 53 bits) and is
-// moved into the 128-bit sum every 1024 rows; the rest take the integer path
-// directly.
+// The sum is exact: every element is taken as the integer x * 2^64 (exact for
+// the whole range precondition) and summed in a signed 128-bit integer.
+// bf16 elements with 2^-20 <= |x| < 2^16 -- all of them on unit-scale data --
+// go through a float64 partial sum per element that is exact for 1024 rows
+// (such values are multiples of 2^-27 below 2^16, so 1024 of them need at most
+// 53 bits); every 1024 rows it moves, as the integer part * 2^27 (below 2^53),
+// into an int64 sum (at most 128 moves per thread: below 2^60), which counts
+// x * 2^64 in units of 2^37.  A piece holding any other element (rare) adds
+// all its elements as x * 2^64 directly to 128-bit sums kept in shared memory.  float32 elements all take the 128-bit
+// path, in registers.
+// Adds the eight bf16 elements of a 16-byte piece, as x * 2^64, to 128-bit sums.
+__device__ __noinline__ void update_slow_piece(uint4 v, unsigned long long* lo, long long* hi) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        unsigned long long l = lo[e];
+        long long h = hi[e];
+        fixed64_add(l, h, (e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+        lo[e] = l;
+        hi[e] = h;
+    }
+}
+
 template <typename T>
 __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const int32_t* __restrict__ perm,
                                                 const int32_t* __restrict__ offsets, int N, int D, int K,
@@ -166,20 +182,34 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
     constexpr int VEC = 16 / sizeof(T);
     constexpr bool BF16 = sizeof(T) == 2;
     extern __shared__ long long red[];  // [2][RPI][D]: high and low words of the 128-bit sums
+    __shared__ unsigned long long slow_lo[BF16 ? 128 * VEC : 1];
+    __shared__ long long slow_hi[BF16 ? 128 * VEC : 1];
     int k = blockIdx.x, bh = blockIdx.y;
     const int32_t* off = offsets + (size_t)bh * (K + 1);
     int start = off[k], n = off[k + 1] - start;
     if (n == 0) return;  // empty cluster keeps its centroid
     const int CPR = D / VEC, RPI = 128 / CPR;
     int t = threadIdx.x, piece = t % CPR, slot = t / CPR;
-    long long acc_hi[VEC];
-    unsigned long long acc_lo[VEC];
-    double part[VEC];
+    long long acc_hi[BF16 ? 1 : VEC];             // float32: 128-bit sums in registers
+    unsigned long long acc_lo[BF16 ? 1 : VEC];
+    long long mid[BF16 ? VEC : 1];                // bf16: flushed partials, units of 2^37
+    double part[BF16 ? VEC : 1];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
+    for (int e = 0; e < (BF16 ? 1 : VEC); ++e) {
         acc_hi[e] = 0;
         acc_lo[e] = 0;
+    }
+#pragma unroll
+    for (int e = 0; e < (BF16 ? VEC : 1); ++e) {
+        mid[e] = 0;
         part[e] = 0.0;
+    }
+    if (BF16) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            slow_lo[t * VEC + e] = 0ull;
+            slow_hi[t * VEC + e] = 0;
+        }
     }
     const int32_t* pm = perm + (size_t)bh * N + start;
     const T* Xh = X + (size_t)bh * N * D;
@@ -188,9 +218,7 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
         if (BF16) {
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
-                // part * 2^27 is an integer below 2^53; as x * 2^64 it is that integer << 37
-                const long long v = __double2ll_rn(ldexp(part[e], 27));
-                acc128_add(acc_lo[e], acc_hi[e], (unsigned long long)v << 37, v >> 27);
+                mid[e] += __double2ll_rn(ldexp(part[e], 27));  // exact: a multiple of 2^-27 below 2^26
                 part[e] = 0.0;
             }
         }
@@ -212,16 +240,8 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
 #pragma unroll
                 for (int e = 0; e < VEC; ++e)
                     part[e] += (double)__uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
-            } else {
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    const uint32_t b = (e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16);
-                    const uint32_t ex = (b >> 23) & 0xFFu;
-                    if ((ex - 107u) <= 35u || (b & 0x7FFFFFFFu) == 0u)
-                        part[e] += (double)__uint_as_float(b);
-                    else
-                        fixed64_add(acc_lo[e], acc_hi[e], b);
-                }
+            } else {  // rare: the whole piece goes to the 128-bit sums, out of line
+                update_slow_piece(v, slow_lo + t * VEC, slow_hi + t * VEC);
             }
             if (++rows_in_part == 1024) flush();
         } else {
@@ -250,8 +270,18 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
     if (slot < RPI) {
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-            red_hi[slot * D + piece * VEC + e] = acc_hi[e];
-            red_lo[slot * D + piece * VEC + e] = (long long)acc_lo[e];
+            unsigned long long lo;
+            long long hi;
+            if (BF16) {  // mid * 2^37 plus the directly added elements
+                lo = (unsigned long long)mid[e] << 37;
+                hi = mid[e] >> 27;
+                acc128_add(lo, hi, slow_lo[t * VEC + e], slow_hi[t * VEC + e]);
+            } else {
+                lo = acc_lo[e];
+                hi = acc_hi[e];
+            }
+            red_hi[slot * D + piece * VEC + e] = hi;
+            red_lo[slot * D + piece * VEC + e] = (long long)lo;
         }
     }
     __syncthreads();
