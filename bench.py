@@ -253,13 +253,14 @@ KERNEL_SOURCES = {"k_sparse_attn_tc": ["block_sparse_attention_means_b200/csrc/k
 ATTENTION_KERNELS = ("k_sparse_attn_tc", "k_attn_schedule", "k_kv_pad_gather", "k_kv_pad_offsets",
                      "k_pack_cand", "k_pack_select", "k_items_emit", "k_item_gather", "k_merge_init",
                      "k_merge_planes")
+ATTENTION_MAIN = ("k_sparse_attn_tc",)
 
 
 def kernel_roofline(name: str, ms_per_launch: float, cfg, counters, peaks, peak_kind) -> dict:
     """Algorithmic work per launch of the named kernel and its roofline."""
     BH, N, D, NQ, NK = cfg.B * cfg.H, cfg.N, cfg.D, cfg.NQ, cfg.NK
     sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    if name == "k_sparse_attn_tc":
+    if name in ATTENTION_MAIN:
         work, bound, peak, unit = 4.0 * D * counters[5], "tensor", sustained, "TFLOP/s"
     elif name == "k_assign_tc":
         work, bound, peak, unit = 2.0 * BH * N * ((NQ + NK) / 2) * D, "tensor", sustained, "TFLOP/s"
@@ -276,7 +277,7 @@ def kernel_roofline(name: str, ms_per_launch: float, cfg, counters, peaks, peak_
     achieved = work / (ms_per_launch * 1e-3) / 1e12
     traffic = committed_traffic(name)
     extra = {}
-    if name == "k_sparse_attn_tc":
+    if name in ATTENTION_MAIN:
         # tensor work actually issued: every (128-row query tile, 128-row key tile) pair, padding included
         tile_tf = 4.0 * 128 * 128 * D * counters[7] / (ms_per_launch * 1e-3) / 1e12
         extra = {"tile_tflops": round(tile_tf, 2), "tensor_pipe_frac_on_tiles": round(tile_tf / peak, 4)}
@@ -372,6 +373,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention reference")
     ap.add_argument("--no-quality", action="store_true", help="skip the recall measurement")
+    ap.add_argument("--extra-flags", type=lambda x: int(x, 0), default=0,
+                    help="park_retrieval flag bits added to the variant's (e.g. 0x200: no query-tile packing)")
     ap.add_argument("--heads", type=int, default=0, help="override H (small cases for profiler captures)")
     ap.add_argument("--variant", default="park", choices=sorted(VARIANTS),
                     help="retrieval variant (PARK Table 3 ablations, Table 10 top-k, size prior, AB-Attention "
@@ -432,7 +435,7 @@ def main():
         sip_u = torch.from_numpy(gen_uniform(cfg, seed=rank)).to(dev)
     out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, dev, sip_uniform=sip_u,
                                window=hva_window(cfg) if vflags & 0x100 else None)
-    out.flags = vflags
+    out.flags = vflags | args.extra_flags
     p_arg = cfg.p if vp is None else vp
     ws = park.alloc_workspace(shape, cfg.NQ, cfg.NK, dev)
     O = torch.empty_like(Q)
@@ -522,8 +525,9 @@ def main():
                for k, v in sorted(prof.items(), key=lambda kv: -kv[1][0])}
     top = next(iter(kernels)) if kernels else None
     roof = kernel_roofline(top, prof[top][0] / prof[top][1], cfg, counters, peaks, peak_kind) if top else None
-    attn = prof.get("k_sparse_attn_tc")
-    attn_roof = kernel_roofline("k_sparse_attn_tc", attn[0] / attn[1], cfg, counters, peaks, peak_kind) \
+    attn_name = next((k for k in ATTENTION_MAIN if k in prof), None)
+    attn = prof.get(attn_name) if attn_name else None
+    attn_roof = kernel_roofline(attn_name, attn[0] / attn[1], cfg, counters, peaks, peak_kind) \
         if attn else None
     retrieval_ms = sum(v[0] for k, v in prof.items()
                        if k not in ATTENTION_KERNELS) / args.steps
@@ -543,6 +547,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": round(worst_ms, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {**workload_config(cfg), **({"variant": args.variant} if args.variant != "park" else {}),
+                       **({"extra_flags": hex(args.extra_flags)} if args.extra_flags else {}),
                        **({"window": list(hva_window(cfg))} if vflags & 0x100 else {})},
             "roofline": roof, "attention_roofline": attn_roof,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches), "clocks": clocks,

@@ -28,7 +28,6 @@ PARK_FLAG_SIP = 0x40
 PARK_FLAG_MERGE_Q = 0x80
 PARK_FLAG_LOCAL_WINDOW = 0x100
 PARK_FLAG_NO_TILE_PACKING = 0x200
-PARK_FLAG_NO_TILE_PAIRING = 0x400
 
 PARK_CNT_Q_RECHECK = 0
 PARK_CNT_K_RECHECK = 1

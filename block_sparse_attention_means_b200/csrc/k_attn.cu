@@ -266,7 +266,7 @@ __global__ __launch_bounds__(256) void k_attn_schedule_tc(int NQ, int NK, int Np
                                                           int32_t* __restrict__ kv_nseg, int2* __restrict__ segs,
                                                           float* __restrict__ segwA, float* __restrict__ segwB,
                                                           int32_t* __restrict__ slot_items,
-                                                          int64_t* __restrict__ counters, int write_lists) {
+                                                          int64_t* __restrict__ counters) {
     __shared__ int wcnt[8], wpad[8];
     __shared__ long long wown[8];
     const int r = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, lane = t & 31, w = t >> 5;
@@ -322,7 +322,7 @@ __global__ __launch_bounds__(256) void k_attn_schedule_tc(int NQ, int NK, int Np
     const float NI = __int_as_float(0xff800000);
     const float* wA = bweight ? bweight + slot * NK : nullptr;
     const float* wB = (bweight && g >= 0) ? bweight + ((size_t)bh * NQ + g) * NK : nullptr;
-    for (int m = m0; m < m0 + per && m < NK && write_lists; ++m) {
+    for (int m = m0; m < m0 + per && m < NK; ++m) {
         const bool a = mA[m] != 0, b = mB && mB[m] != 0;
         if (!(a || b)) continue;
         const int sz = ko[m + 1] - ko[m];
@@ -345,9 +345,8 @@ __global__ __launch_bounds__(256) void k_attn_schedule_tc(int NQ, int NK, int Np
             atomicAdd((unsigned long long*)(counters + PARK_CNT_KEPT_PAIRS),
                       (unsigned long long)nr * (unsigned long long)tot_own);
             atomicAdd((unsigned long long*)(counters + PARK_CNT_WORK_ITEMS), (unsigned long long)own_items);
-            if (write_lists)  // (the paired schedule counts its own key tiles)
-                atomicAdd((unsigned long long*)(counters + PARK_CNT_KEY_TILES),
-                          (unsigned long long)own_items * (unsigned long long)((tot_p + 127) / 128));
+            atomicAdd((unsigned long long*)(counters + PARK_CNT_KEY_TILES),
+                      (unsigned long long)own_items * (unsigned long long)((tot_p + 127) / 128));
         }
     }
 }
@@ -358,8 +357,7 @@ __global__ __launch_bounds__(256) void k_attn_schedule_tc(int NQ, int NK, int Np
 __global__ __launch_bounds__(1024) void k_items_emit(int BH, int NQ, const int32_t* __restrict__ q_off,
                                                      const int32_t* __restrict__ pack_guest,
                                                      const int32_t* __restrict__ slot_items,
-                                                     WorkItem* __restrict__ items, int32_t* __restrict__ item_count,
-                                                     int32_t* __restrict__ slot_base) {
+                                                     WorkItem* __restrict__ items, int32_t* __restrict__ item_count) {
     __shared__ int wsum[32];
     __shared__ int s_base;
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
@@ -383,7 +381,6 @@ __global__ __launch_bounds__(1024) void k_items_emit(int BH, int NQ, const int32
             tot += wsum[q];
         }
         const int base = s_base + woff + incl - cnt;
-        if (slot_base && slot < nslot) slot_base[slot] = base;  // index of the slot's first item
         if (cnt > 0) {
             const int bh = (int)(slot / NQ), r = (int)(slot - (long long)bh * NQ);
             const int qs = q_off[(size_t)bh * (NQ + 1) + r], nr = q_off[(size_t)bh * (NQ + 1) + r + 1] - qs;
@@ -417,14 +414,14 @@ int launch_attn_schedule_tc(int BH, int NQ, int NK, int Npad, const int32_t* q_o
                             const uint8_t* mask, const float* bweight, const int32_t* poff, const int32_t* pack_host,
                             const int32_t* pack_guest, int32_t* kv_pre, int32_t* kv_len, int32_t* kv_nseg,
                             int2* segs, float* segwA, float* segwB, int32_t* slot_items, WorkItem* items,
-                            int32_t* item_count, int64_t* counters, int32_t* slot_base, cudaStream_t st) {
+                            int32_t* item_count, int64_t* counters, cudaStream_t st) {
     ::park::prof_begin(st);
     k_attn_schedule_tc<<<dim3(NQ, BH), 256, 0, st>>>(NQ, NK, Npad, q_off, k_off, mask, bweight, poff, pack_host,
                                                      pack_guest, kv_pre, kv_len, kv_nseg, segs, segwA, segwB,
-                                                     slot_items, counters, slot_base == nullptr);
+                                                     slot_items, counters);
     PARK_TRY_LAUNCH("k_attn_schedule", st);
     ::park::prof_begin(st);
-    k_items_emit<<<1, 1024, 0, st>>>(BH, NQ, q_off, pack_guest, slot_items, items, item_count, slot_base);
+    k_items_emit<<<1, 1024, 0, st>>>(BH, NQ, q_off, pack_guest, slot_items, items, item_count);
     PARK_TRY_LAUNCH("k_items_emit", st);
     return PARK_OK;
 }

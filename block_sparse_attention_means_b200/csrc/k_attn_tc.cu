@@ -84,6 +84,11 @@ struct TcSmem {
 __device__ __forceinline__ float bits_f(uint32_t u) { return __uint_as_float(u); }
 // warp-uniform view of the abort flag
 __device__ __forceinline__ bool warp_abort(volatile int* abort) { return __any_sync(0xffffffffu, *abort != 0); }
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
 __device__ __forceinline__ float fast_ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -393,8 +398,7 @@ __global__ void __launch_bounds__(352, 1)
                 const int g = G + j, b = g & 1, ph = (g >> 1) & 1, vs = g % TC_VST;
                 const bool live = wwait(&sh.s_full[b], ph) && wwait(&sh.v_full[vs], (g / TC_VST) & 1);
                 uint32_t s[2][32];
-                float tm[4] = {__int_as_float(0xff800000), __int_as_float(0xff800000), __int_as_float(0xff800000),
-                               __int_as_float(0xff800000)};
+                float tm[2] = {__int_as_float(0xff800000), __int_as_float(0xff800000)};
                 if (live) {
                     tc_fence_after();
                     tmem_ld32(trow + (uint32_t)(b * 128 + 64 * hc), s[0]);
@@ -419,16 +423,14 @@ __global__ void __launch_bounds__(352, 1)
                             s[c][4 * q + 1] = __float_as_uint(x01.y);
                             s[c][4 * q + 2] = __float_as_uint(x23.x);
                             s[c][4 * q + 3] = __float_as_uint(x23.y);
-                            tm[0] = fmaxf(tm[0], x01.x);
-                            tm[1] = fmaxf(tm[1], x01.y);
-                            tm[2] = fmaxf(tm[2], x23.x);
-                            tm[3] = fmaxf(tm[3], x23.y);
+                            tm[0] = fmax3f(tm[0], x01.x, x01.y);
+                            tm[1] = fmax3f(tm[1], x23.x, x23.y);
                         }
                     }
                 }
                 // Both halves of the row agree on the tile max.  The barrier also orders
                 // the partner's S loads before this thread's P stores over them.
-                sh.xmax[j & 1][hc][row] = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+                sh.xmax[j & 1][hc][row] = fmaxf(tm[0], tm[1]);
                 tc_fence_before();
                 named_bar_sync(pair_bar, 64);
                 tc_fence_after();
@@ -443,7 +445,7 @@ __global__ void __launch_bounds__(352, 1)
                     if (!wwait(&sh.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) continue;
                     tc_fence_after();
                     const float m_new = tmax > m_ref + kRescaleThreshold ? tmax : m_ref;
-                    const float alpha = fast_ex2(m_ref - m_new);
+                    const float alpha = m_new == m_ref ? 1.f : fast_ex2(m_ref - m_new);  // (m_ref may be -inf)
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         uint32_t o[32];

@@ -130,6 +130,113 @@ __global__ __launch_bounds__(272) void k_metric_partial(const T* __restrict__ Q,
         for (int v = 0; v < 8; ++v) P[(a0 + u) * D + b0 + v] = acc[u][v];
 }
 
+// D = 128: the same partials on the float64 tensor cores (mma.sync m8n8k4 f64,
+// exact products and float64 accumulation).  256 threads; warp w owns the block
+// rows w and 15 - w of the upper triangle of 8 x 8 blocks (17 blocks, the B
+// fragments of row 15 - w are those of row w's last w + 1 blocks).  Rows are
+// staged 32 at a time in shared memory as float64 (row pitch 136 doubles: the
+// four rows of a fragment load fall in different bank halves); k-steps of 4
+// rows.  Fragment layouts (PTX ISA, m8n8k4 .f64): A[r][k] and B[k][c] are held
+// by lane 4 r + k and 4 c + k, D[r][2 (l % 4) + {0, 1}] by lane l = 4 r + ...
+constexpr int kMetricPitch = 136;
+
+__device__ __forceinline__ void dmma_m8n8k4(double& d0, double& d1, double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d0), "+d"(d1)
+                 : "d"(a), "d"(b));
+}
+
+// Warp W's part: rows W and 15 - W (compile-time, so that every accumulator
+// index is static).
+template <int W>
+__device__ __forceinline__ void metric_mma_rows(const double* __restrict__ qs, int nk, double (&acc)[17][2],
+                                                int lane) {
+    constexpr int ta0 = W, ta1 = 15 - W;
+    const int fr = lane >> 2, fk = lane & 3;
+#pragma unroll 2
+    for (int k0 = 0; k0 < nk; k0 += 4) {
+        const double* rowp = qs + (k0 + fk) * kMetricPitch + fr;
+        const double a0 = rowp[8 * ta0], a1 = rowp[8 * ta1];
+#pragma unroll
+        for (int q = 0; q < 16 - W; ++q) {  // blocks (ta0, ta0 + q); (ta1, ta0 + q) when ta0 + q >= ta1
+            const double b = rowp[8 * (ta0 + q)];
+            dmma_m8n8k4(acc[q][0], acc[q][1], a0, b);
+            if (ta0 + q >= ta1) dmma_m8n8k4(acc[16 - W + (ta0 + q - ta1)][0], acc[16 - W + (ta0 + q - ta1)][1], a1, b);
+        }
+    }
+}
+
+template <int W>
+__device__ __forceinline__ void metric_mma_store(double* __restrict__ P, const double (&acc)[17][2], int lane) {
+    constexpr int D = 128, ta0 = W, ta1 = 15 - W;
+    const int cr = lane >> 2, cc = 2 * (lane & 3);
+#pragma unroll
+    for (int q = 0; q < 16 - W; ++q) {
+        const int tb = ta0 + q;
+        P[(8 * ta0 + cr) * D + 8 * tb + cc] = acc[q][0];
+        P[(8 * ta0 + cr) * D + 8 * tb + cc + 1] = acc[q][1];
+        if (tb >= ta1) {
+            P[(8 * ta1 + cr) * D + 8 * tb + cc] = acc[16 - W + (tb - ta1)][0];
+            P[(8 * ta1 + cr) * D + 8 * tb + cc + 1] = acc[16 - W + (tb - ta1)][1];
+        }
+    }
+}
+
+template <typename T>
+__global__ __launch_bounds__(256) void k_metric_partial_mma(const T* __restrict__ Q, int N, int rows_per_chunk,
+                                                            double* __restrict__ part) {
+    constexpr int D = 128, RB = 32;
+    __shared__ __align__(16) double qs[RB * kMetricPitch];
+    const int bh = blockIdx.y, c = blockIdx.x, nch = gridDim.x;
+    const T* X = Q + (size_t)bh * N * D;
+    const int r0 = c * rows_per_chunk, r1 = min(N, r0 + rows_per_chunk);
+    const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+    double acc[17][2];
+#pragma unroll
+    for (int b = 0; b < 17; ++b) acc[b][0] = acc[b][1] = 0.0;
+    constexpr int PER = RB * D / 256;  // 16 elements per thread per block of rows
+    float pre[PER];                    // inputs are exact in float32
+    auto fetch = [&](int base) {
+#pragma unroll
+        for (int v = 0; v < PER; ++v) {
+            const int e = t + 256 * v, rr = e >> 7, jj = e & 127;
+            pre[v] = base + rr < r1 ? Elem<T>::to_float(X + (size_t)(base + rr) * D, jj) : 0.f;
+        }
+    };
+    if (r0 < r1) fetch(r0);
+    for (int base = r0; base < r1; base += RB) {
+        __syncthreads();
+#pragma unroll
+        for (int v = 0; v < PER; ++v) {
+            const int e = t + 256 * v;
+            qs[(e >> 7) * kMetricPitch + (e & 127)] = (double)pre[v];  // rows past the end are 0
+        }
+        __syncthreads();
+        if (base + RB < r1) fetch(base + RB);
+        switch (w) {  // warp-uniform
+            case 0: metric_mma_rows<0>(qs, RB, acc, lane); break;
+            case 1: metric_mma_rows<1>(qs, RB, acc, lane); break;
+            case 2: metric_mma_rows<2>(qs, RB, acc, lane); break;
+            case 3: metric_mma_rows<3>(qs, RB, acc, lane); break;
+            case 4: metric_mma_rows<4>(qs, RB, acc, lane); break;
+            case 5: metric_mma_rows<5>(qs, RB, acc, lane); break;
+            case 6: metric_mma_rows<6>(qs, RB, acc, lane); break;
+            default: metric_mma_rows<7>(qs, RB, acc, lane); break;
+        }
+    }
+    double* P = part + ((size_t)bh * nch + c) * D * D;
+    switch (w) {
+        case 0: metric_mma_store<0>(P, acc, lane); break;
+        case 1: metric_mma_store<1>(P, acc, lane); break;
+        case 2: metric_mma_store<2>(P, acc, lane); break;
+        case 3: metric_mma_store<3>(P, acc, lane); break;
+        case 4: metric_mma_store<4>(P, acc, lane); break;
+        case 5: metric_mma_store<5>(P, acc, lane); break;
+        case 6: metric_mma_store<6>(P, acc, lane); break;
+        default: metric_mma_store<7>(P, acc, lane); break;
+    }
+}
+
 __global__ void k_metric_reduce(const double* __restrict__ part, int nch, int N, int D, double* __restrict__ M,
                                 double* __restrict__ M_out) {
     const int bh = blockIdx.y;
@@ -152,8 +259,10 @@ int launch_metric(const void* Q, int dtype, int BH, int N, int D, double* part, 
     int rpc = (N + nchunks - 1) / nchunks;
     dim3 g1(nchunks, BH);
     ::park::prof_begin(st);
-    if (dtype == PARK_BF16)
-        k_metric_partial<bf16_t><<<g1, 272, 0, st>>>((const bf16_t*)Q, N, D, rpc, part);
+    if (dtype == PARK_BF16 && D == 128)
+        k_metric_partial_mma<bf16_t><<<g1, 256, 0, st>>>((const bf16_t*)Q, N, rpc, part);
+    else if (D == 128)
+        k_metric_partial_mma<float><<<g1, 256, 0, st>>>((const float*)Q, N, rpc, part);
     else
         k_metric_partial<float><<<g1, 272, 0, st>>>((const float*)Q, N, D, rpc, part);
     PARK_TRY_LAUNCH("k_metric_partial", st);

@@ -168,39 +168,15 @@ int launch_pack_pairs(int BH, int NQ, int NK, const uint8_t* mask, const int32_t
 // logit terms segwA for the own rows and segwB for the guest rows, -inf where not kept), kv_len, kv_nseg;
 // 128-row work items with their guests, head by head in cluster order (slot_items [BH][NQ]
 // scratch).  pack_host / pack_guest may be null (no packing).
-// slot_base (non-null: the paired schedule follows) receives each slot's first
-// item index; the per-slot key lists are then not written (only kv_len).
 int launch_attn_schedule_tc(int BH, int NQ, int NK, int Npad, const int32_t* q_off, const int32_t* k_off,
                             const uint8_t* mask, const float* bweight, const int32_t* poff, const int32_t* pack_host,
                             const int32_t* pack_guest, int32_t* kv_pre, int32_t* kv_len, int32_t* kv_nseg,
                             int2* segs, float* segwA, float* segwB, int32_t* slot_items, WorkItem* items,
-                            int32_t* item_count, int64_t* counters, int32_t* slot_base, cudaStream_t st);
+                            int32_t* item_count, int64_t* counters, cudaStream_t st);
 // Q rows of every work item into an item-major image: item i occupies rows
 // [128 i, 128 i + 128) (own rows, then guest rows, then zeros).
 int launch_item_gather(const void* Q, int N, const int32_t* q_perm, const WorkItem* items, const int32_t* item_count,
                        size_t item_cap, void* Qimg, int num_sms, cudaStream_t st);
-// ---- k_attn_pair.cu
-// Two work items walking one key list: ia, ib (ib = -1: ia alone) index the
-// work items; lead is the slot (bh * NQ + cluster) holding the pair's key list.
-struct PairItem {
-    int ia, ib, lead;
-};
-// Pairing of the tensor-core schedule's items (pairing = 0: every item alone
-// except the tiles of one cluster, which always pair); per-lead key lists with
-// four row-group logit terms; the pair list.  cand [BH*NQ*8], partner [BH*NQ],
-// pl_* [BH*NQ*NK] / [BH*NQ], pairs [item capacity].
-int launch_pair_schedule(int BH, int NQ, int NK, int Npad, const uint8_t* mask, const int32_t* k_off,
-                         const float* bweight, const int32_t* poff, const int32_t* pack_guest,
-                         const int32_t* slot_items, const int32_t* slot_base, const int32_t* kv_len, int pairing,
-                         int2* cand, int32_t* partner, int32_t* pl_pre, int2* pl_seg, float4* pl_bias,
-                         int32_t* pl_len, int32_t* pl_nseg, PairItem* pairs, int32_t* pair_count, int64_t* counters,
-                         cudaStream_t st);
-constexpr int kPairCandStride = 8;  // candidates stored per slot
-size_t attn_pair_smem_bytes();
-int launch_sparse_attn_pair(const void* Qimg, size_t item_cap, const void* Kpad, const void* Vpad, int N, int NK,
-                            const int32_t* q_perm, const int2* pl_seg, const float4* pl_bias, const int32_t* pl_nseg,
-                            const int32_t* pl_pre, const int32_t* pl_len, const WorkItem* items, const PairItem* pairs,
-                            const int32_t* pair_count, void* O, int32_t* status, int num_sms, cudaStream_t st);
 int launch_sparse_attn_tc(const void* Qimg, size_t item_cap, const void* Kpad, const void* Vpad, int BH, int N, int Npad,
                           int NQ, int NK, const int32_t* q_perm, const int2* segs, const float* segwA,
                           const float* segwB, const int32_t* kv_nseg, const int32_t* kv_pre, const int32_t* kv_len,

@@ -170,7 +170,7 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
 
 struct AttnWs {
     size_t Qimg, Kp, Vp, poff, segs, segw, segwB, kvnseg, sitems, pack, pcand, mS, mP, mI, mH, items, icnt, kvpre,
-        kvlen, sbase, pcand2, partner, plbias, pllen, pairs, pcnt, total;
+        kvlen, total;
     size_t item_cap;  // tensor-core work items at most: sum_r ceil(n_r / 128) <= ceil(N / 128) + NQ per head
     int Npad;
 };
@@ -204,20 +204,9 @@ AttnWs plan_attn(const Dims& d, int NQ, int NK) {
         w.mP = c.take(pk ? BH * kMergePlanes * Wd * 4 : 0);
         w.mI = c.take(pk ? 7 * BH * (size_t)NQ * 4 : 0);
         w.mH = c.take(pk ? 2 * BH * 4 : 0);
-        // paired schedule: per-slot first item, pairing candidates and partners, the
-        // per-lead key lists' four logit terms and lengths (prefixes, segments and
-        // segment counts reuse kvpre / segs / kvnseg), the pair list
-        w.sbase = c.take(BH * (size_t)NQ * 4);
-        w.pcand2 = c.take(BH * (size_t)NQ * kPairCandStride * 8);
-        w.partner = c.take(BH * (size_t)NQ * 4);
-        w.plbias = c.take(BH * (size_t)NQ * NK * 16);
-        w.pllen = c.take(BH * (size_t)NQ * 4);
-        w.pairs = c.take(w.item_cap * sizeof(PairItem));
-        w.pcnt = c.take(16 * 4);
     } else {
         w.Qimg = w.Kp = w.Vp = w.poff = w.segs = w.segw = w.segwB = w.kvnseg = w.sitems = 0;
         w.pack = w.pcand = w.mS = w.mP = w.mI = w.mH = 0;
-        w.sbase = w.pcand2 = w.partner = w.plbias = w.pllen = w.pairs = w.pcnt = 0;
     }
     size_t max_items = BH * ((N + kAttnTile - 1) / kAttnTile + (size_t)NQ);
     w.items = c.take(max_items * sizeof(WorkItem));
@@ -379,8 +368,7 @@ bool flags_ok(const park_retrieval* r, float p) {
     const uint32_t flags = r->flags;
     const uint32_t known = PARK_FLAG_WARM_START_Q | PARK_FLAG_WARM_START_K | PARK_FLAG_NO_QRKC |
                            PARK_FLAG_CENTROID_QUERY | PARK_FLAG_TOPK | PARK_FLAG_SIZE_PRIOR | PARK_FLAG_SIP |
-                           PARK_FLAG_MERGE_Q | PARK_FLAG_LOCAL_WINDOW | PARK_FLAG_NO_TILE_PACKING |
-                           PARK_FLAG_NO_TILE_PAIRING;
+                           PARK_FLAG_MERGE_Q | PARK_FLAG_LOCAL_WINDOW | PARK_FLAG_NO_TILE_PACKING;
     if (flags & ~known) return false;
     if ((flags & (PARK_FLAG_TOPK | PARK_FLAG_SIP)) && p > 1.0f) return false;
     if ((flags & PARK_FLAG_TOPK) && (flags & PARK_FLAG_SIP)) return false;
@@ -555,29 +543,10 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
         PARK_CHECK(launch_pack_pairs(BH, NQ, NK, r->mask, r->q_offsets, r->k_offsets, m, at<int2>(ws, w.pcand),
                                      pack_host, pack_guest, st));
     }
-    // two query tiles per CTA sharing each K/V tile (tiles of one cluster always; clusters with
-    // similar kept sets when pairing is on), unless turned off
-    const bool paired = !(r->flags & PARK_FLAG_NO_TILE_PAIRING);
-    int32_t* slot_base = paired ? at<int32_t>(ws, w.sbase) : nullptr;
     PARK_CHECK(launch_attn_schedule_tc(BH, NQ, NK, w.Npad, r->q_offsets, r->k_offsets, r->mask, bw, poff, pack_host,
                                        pack_guest, at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), kvnseg, segs,
-                                       segwA, segwB, at<int32_t>(ws, w.sitems), items, icnt, r->counters, slot_base,
-                                       st));
+                                       segwA, segwB, at<int32_t>(ws, w.sitems), items, icnt, r->counters, st));
     PARK_CHECK(launch_item_gather(Q, N, r->q_perm, items, icnt, w.item_cap, Qimg, num_sms, st));
-    if (paired) {
-        PairItem* pairs = at<PairItem>(ws, w.pairs);
-        int32_t* pcnt = at<int32_t>(ws, w.pcnt);
-        int32_t* pl_len = at<int32_t>(ws, w.pllen);
-        float4* pl_bias = at<float4>(ws, w.plbias);
-        PARK_CHECK(launch_pair_schedule(BH, NQ, NK, w.Npad, r->mask, r->k_offsets, bw, poff, pack_guest,
-                                        at<int32_t>(ws, w.sitems), slot_base, at<int32_t>(ws, w.kvlen),
-                                        NQ <= kMergeMaxNQ, at<int2>(ws, w.pcand2), at<int32_t>(ws, w.partner),
-                                        at<int32_t>(ws, w.kvpre), segs, pl_bias, pl_len, kvnseg, pairs, pcnt,
-                                        r->counters, st));
-        return launch_sparse_attn_pair(Qimg, w.item_cap, Kp, Vp, N, NK, r->q_perm, segs, pl_bias, kvnseg,
-                                       at<int32_t>(ws, w.kvpre), pl_len, items, pairs, pcnt, O, r->status, num_sms,
-                                       st);
-    }
     PARK_CHECK(launch_sparse_attn_tc(Qimg, w.item_cap, Kp, Vp, BH, N, w.Npad, NQ, NK, r->q_perm, segs, segwA, segwB,
                                      kvnseg, at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), items, icnt, O,
                                      r->status, num_sms, st));

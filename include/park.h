@@ -142,14 +142,6 @@ extern "C" {
  * only to its own cluster's kept key clusters; done only for NQ <= 2048);
  * this flag turns it off. */
 #define PARK_FLAG_NO_TILE_PACKING 0x200u
-/* Implementation switch, no change to the result (up to float32 summation
- * order): on the bf16 path park_sparse_attn runs two 128-row query tiles per
- * CTA that share each K/V tile -- the tiles of one query cluster, and (for
- * NQ <= 2048) two single-tile clusters of a head whose kept sets overlap enough
- * that the union of their key lists costs fewer key-tile loads than the two
- * lists apart (every row still attends only to its own cluster's kept key
- * clusters); this flag runs every query tile alone instead. */
-#define PARK_FLAG_NO_TILE_PAIRING 0x400u
 
 /* ---- park_retrieval.counters indices (outputs, int64) ------------------ */
 #define PARK_CNT_Q_RECHECK 0    /* query rows whose bf16 score margin was not

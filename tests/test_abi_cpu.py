@@ -38,7 +38,7 @@ def test_struct_layout_matches_header():
                  "PARK_ERR_RANGE", "PARK_ERR_TIMEOUT", "PARK_BF16", "PARK_F32", "PARK_FLAG_WARM_START_Q",
                  "PARK_FLAG_WARM_START_K", "PARK_FLAG_NO_QRKC", "PARK_FLAG_CENTROID_QUERY", "PARK_FLAG_TOPK",
                  "PARK_FLAG_SIZE_PRIOR", "PARK_FLAG_SIP", "PARK_FLAG_MERGE_Q", "PARK_FLAG_LOCAL_WINDOW",
-                 "PARK_FLAG_NO_TILE_PACKING", "PARK_FLAG_NO_TILE_PAIRING",
+                 "PARK_FLAG_NO_TILE_PACKING",
                  "PARK_CNT_KEPT_PAIRS"):
         m = re.search(rf"#define {name} (\w+)", text)
         assert m and int(m.group(1).rstrip("u"), 0) == getattr(_lib, name), name
@@ -109,7 +109,7 @@ def test_host_argument_errors_enqueue_nothing():
     cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.9, 10, ctypes.byref(r2), fake, need,
                                     None), _lib.PARK_ERR_INVALID_ARG))
     r3 = _fake_retrieval()
-    r3.flags = 0x800                              # unknown flag bit
+    r3.flags = 0x400                              # unknown flag bit
     cases.append((lib.park_retrieve(fake, fake, ctypes.byref(shape), 4, 4, 0.9, 10, ctypes.byref(r3), fake, need,
                                     None), _lib.PARK_ERR_INVALID_ARG))
     r4 = _fake_retrieval()

@@ -52,7 +52,7 @@ def _run(park, name, window=None, merge=False, rounds=0, flags=0, p=None):
     shape = park.Shape.of(cfg, dt)
     q, k, v = (pu.to_device(x, dt) for x in (Q, K, V))
     out = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, q.device, window=window, merge=merge, merge_rounds=rounds)
-    out.flags |= flags | 0x600  # no query-tile packing or pairing: tile pairs follow the merge cost model
+    out.flags |= flags | 0x200  # no query-tile packing: the tile-pair counter follows the merge cost model
     O, r = park.layer(q, k, v, shape, cfg.NQ, cfg.NK, p, cfg.iters, out=out)
     torch.cuda.synchronize()
     assert r.status_code() == 0, f"device status {r.status_code()}"
@@ -121,10 +121,10 @@ def test_hva_properties_at_hunyuan_shape(park):
     q, k, v = (pu.to_device(x, torch.bfloat16) for x in (Q, K, V))
     dev = q.device
     plain = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, dev)
-    plain.flags |= 0x600  # no query-tile packing or pairing: tile pairs as the merge cost model counts them
+    plain.flags |= 0x200  # no query-tile packing: tile pairs as the merge cost model counts them
     _, r0 = park.layer(q, k, v, shape, cfg.NQ, cfg.NK, cfg.p, cfg.iters, out=plain)
     merged = park.alloc_retrieval(shape, cfg.NQ, cfg.NK, dev, merge=True)
-    merged.flags |= 0x600
+    merged.flags |= 0x200
     _, r1 = park.layer(q, k, v, shape, cfg.NQ, cfg.NK, cfg.p, cfg.iters, out=merged)
     torch.cuda.synchronize()
     assert r0.status_code() == 0 and r1.status_code() == 0

@@ -15,8 +15,7 @@ import parity_util as pu
 
 pytestmark = pytest.mark.gpu
 
-NO_PAIR = 0x400  # packing is compared with query tiles running alone (no pairing)
-NO_PACK = 0x200 | NO_PAIR
+NO_PACK = 0x200
 
 
 @pytest.fixture(scope="module")
@@ -49,7 +48,7 @@ def test_packing_matches_oracle_and_saves_tiles(park):
     Q, K, V = gen_layer(cfg, 0)
     ref = po.layer(Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64), cfg.NQ, cfg.NK, cfg.p,
                    cfg.iters, cfg.dtype)
-    O1, r1 = _layer(park, cfg, NO_PAIR, cfg.p)
+    O1, r1 = _layer(park, cfg, 0, cfg.p)
     fails = pu.compare_retrieval(r1, ref, cfg.NQ, cfg.NK)
     assert not fails, "\n".join(fails[:20])
     pu.assert_output_close(O1, ref, False)
@@ -68,7 +67,7 @@ def test_packing_with_sip_weights(park):
     U = gen_uniform(cfg)
     ref = po.layer(Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64), cfg.NQ, cfg.NK, ratio,
                    cfg.iters, cfg.dtype, sip_ratio=ratio, sip_u=U.astype(np.float64))
-    O1, r1 = _layer(park, cfg, NO_PAIR, ratio, sip=U)
+    O1, r1 = _layer(park, cfg, 0, ratio, sip=U)
     fails = pu.compare_retrieval(r1, ref, cfg.NQ, cfg.NK)
     assert not fails, "\n".join(fails[:20])
     pu.assert_output_close(O1, ref, False)
@@ -80,7 +79,7 @@ def test_packing_at_hunyuan_shape(park):
     """Two HunyuanVideo-shaped heads: packed and unpacked outputs agree and the
     packing removes work items and tile pairs."""
     cfg = CONFIGS["hunyuan"].replace(H=2, name="hunyuan_h2")
-    O1, r1 = _layer(park, cfg, NO_PAIR, cfg.p)
+    O1, r1 = _layer(park, cfg, 0, cfg.p)
     O0, r0 = _layer(park, cfg, NO_PACK, cfg.p)
     c1, c0 = r1.counters.cpu().tolist(), r0.counters.cpu().tolist()
     assert c1[5] == c0[5]
