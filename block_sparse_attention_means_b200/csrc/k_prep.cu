@@ -7,13 +7,21 @@ namespace park {
 // ---------------------------------------------------------------- input check
 // One pass over the tensor with 16-byte loads: every element must be 0 or a
 // finite value with 2^-40 <= |x| < 2^40 (the library's range precondition).
+// For bf16, wide[h] (when given) is set for every head h holding an element
+// with |x| >= 2^16 (none in unit-scale data): the centroid update of such a
+// head takes its general 128-bit path instead of the float64 partial sums
+// (k_sort.cu); and tiny_rows[r] (when given) for every row r holding a nonzero
+// element with |x| < 2^-20 (about one row in ten thousand in unit-scale data),
+// which the float64 partial sums cannot take exactly either.
 template <int BYTES>
-__global__ void k_input_check(const uint4* __restrict__ x, size_t n16, int32_t* status) {
+__global__ void k_input_check(const uint4* __restrict__ x, size_t n16, int32_t* status, size_t per_head16,
+                              int32_t* __restrict__ wide, uint8_t* __restrict__ tiny_rows, size_t row16) {
     size_t stride = (size_t)gridDim.x * blockDim.x;
     bool bad = false;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += stride) {
         uint4 v = x[i];
         uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        bool narrow = true, tiny = false;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             if (BYTES == 2) {
@@ -23,6 +31,8 @@ __global__ void k_input_check(const uint4* __restrict__ x, size_t n16, int32_t* 
                     uint32_t mag = b & 0x7FFFu;
                     int e = (b >> 7) & 0xFF;
                     bad |= !in_range_exp(e, mag);
+                    narrow &= e <= 142;
+                    tiny |= mag != 0u && e < 107;
                 }
             } else {
                 uint32_t mag = w[q] & 0x7FFFFFFFu;
@@ -30,21 +40,27 @@ __global__ void k_input_check(const uint4* __restrict__ x, size_t n16, int32_t* 
                 bad |= !in_range_exp(e, mag);
             }
         }
+        if (BYTES == 2 && !narrow && wide) atomicOr(wide + i / per_head16, 1);  // rare
+        if (BYTES == 2 && tiny && tiny_rows) tiny_rows[i / row16] = 1;            // rare
     }
     if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) set_status(status, PARK_ERR_RANGE);
 }
 
-int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status, cudaStream_t st) {
+int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status, int32_t* wide,
+                       size_t per_head_elems, uint8_t* tiny_rows, size_t row_elems, cudaStream_t st) {
     int eb = dtype == PARK_BF16 ? 2 : 4;
     size_t n16 = n_elems * eb / 16;
     int blocks = (int)((n16 + 255) / 256);
     ::park::prof_begin(st);
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (blocks < 1) blocks = 1;
+    const size_t ph16 = per_head_elems * eb / 16;  // a head is a whole number of 16-byte pieces (D % 8 == 0)
+    const size_t r16 = row_elems * eb / 16;          // and so is a row
     if (eb == 2)
-        k_input_check<2><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status);
+        k_input_check<2><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status, ph16 ? ph16 : 1, wide,
+                                                 r16 ? tiny_rows : nullptr, r16 ? r16 : 1);
     else
-        k_input_check<4><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status);
+        k_input_check<4><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status, ph16 ? ph16 : 1, nullptr, nullptr, 1);
     PARK_TRY_LAUNCH("k_input_check", st);
     return PARK_OK;
 }

@@ -126,6 +126,52 @@ __global__ __launch_bounds__(1024) void k_label_scatter(const int32_t* __restric
     if (valid) perm[(size_t)bh * N + pos] = i;
 }
 
+// (3), for K <= kScatterMaxK: each warp's leaders record the counts of their
+// labels in a [warp][label] table in shared memory; one pass per label turns the
+// table into the number of earlier tokens of the chunk with that label (the
+// warps in order), so the ranks need three block barriers instead of one per
+// warp.
+constexpr int kScatterMaxK = 1536;
+
+__global__ __launch_bounds__(1024) void k_label_scatter_tab(const int32_t* __restrict__ labels, int N, int K,
+                                                            int KP, int nchunks, const int32_t* __restrict__ hist,
+                                                            const int32_t* __restrict__ offsets,
+                                                            int32_t* __restrict__ perm) {
+    extern __shared__ uint16_t tab[];  // [32][KP]: counts, then exclusive starts over the warps
+    const int c = blockIdx.x, bh = blockIdx.y;
+    uint32_t* tab32 = reinterpret_cast<uint32_t*>(tab);
+    for (int e = threadIdx.x; e < 16 * KP; e += blockDim.x) tab32[e] = 0u;  // 32 KP uint16 (KP even)
+    const int i = c * SORT_CHUNK + threadIdx.x;
+    const bool valid = i < N;
+    const int lab = valid ? labels[(size_t)bh * N + i] : -1;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned peers = __match_any_sync(0xffffffffu, lab);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    __syncthreads();
+    if (valid && rank == 0) tab[warp * KP + lab] = (uint16_t)__popc(peers);
+    __syncthreads();
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+        uint32_t run = 0;
+#pragma unroll
+        for (int h = 0; h < 32; h += 16) {  // sixteen loads in flight
+            uint32_t v[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) v[w] = tab[(h + w) * KP + k];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+                tab[(h + w) * KP + k] = (uint16_t)run;
+                run += v[w];
+            }
+        }
+    }
+    __syncthreads();
+    if (valid) {
+        const int pos = offsets[(size_t)bh * (K + 1) + lab] + hist[((size_t)bh * K + lab) * nchunks + c] +
+                        tab[warp * KP + lab] + rank;
+        perm[(size_t)bh * N + pos] = i;
+    }
+}
+
 int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist, int nchunks, int32_t* perm,
                       int32_t* offsets, cudaStream_t st) {
     size_t sm = (size_t)K * sizeof(int32_t);
@@ -144,7 +190,15 @@ int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist
     k_label_scan<<<BH, 1024, 0, st>>>(N, K, offsets);
     PARK_TRY_LAUNCH("k_label_scan", st);
     ::park::prof_begin(st);
-    k_label_scatter<<<g, 1024, sm, st>>>(labels, N, K, nchunks, hist, offsets, perm);
+    if (K <= kScatterMaxK) {
+        const int KP = (K + 1) & ~1;  // even row pitch: the table is zeroed in 32-bit words
+        const size_t tsm = (size_t)32 * KP * sizeof(uint16_t);
+        if (tsm > 48 * 1024)
+            cudaFuncSetAttribute(k_label_scatter_tab, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+        k_label_scatter_tab<<<g, 1024, tsm, st>>>(labels, N, K, KP, nchunks, hist, offsets, perm);
+    } else {
+        k_label_scatter<<<g, 1024, sm, st>>>(labels, N, K, nchunks, hist, offsets, perm);
+    }
     PARK_TRY_LAUNCH("k_label_scatter", st);
     return PARK_OK;
 }
@@ -152,136 +206,188 @@ int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist
 // ---------------------------------------------------------------- update
 // 128 threads.  Each thread owns one 16-byte piece of a row: VEC elements at
 // piece p = t % CPR, and rows s, s + RPI, ... of the cluster (s = t / CPR).
-// The sum is exact: every element is taken as the integer x * 2^64 (exact for
-// the whole range precondition) and summed in a signed 128-bit integer.
-// bf16 elements with 2^-20 <= |x| < 2^16 -- all of them on unit-scale data --
-// go through a float64 partial sum per element that is exact for 1024 rows
-// (such values are multiples of 2^-27 below 2^16, so 1024 of them need at most
-// 53 bits); every 1024 rows it moves, as the integer part * 2^27 (below 2^53),
-// into an int64 sum (at most 128 moves per thread: below 2^60), which counts
-// x * 2^64 in units of 2^37.  A piece holding any other element (rare) adds
-// all its elements as x * 2^64 directly to 128-bit sums kept in shared memory.  float32 elements all take the 128-bit
-// path, in registers.
-// Adds the eight bf16 elements of a 16-byte piece, as x * 2^64, to 128-bit sums.
-__device__ __noinline__ void update_slow_piece(uint4 v, unsigned long long* lo, long long* hi) {
+// Every sum is exact: the integer x * 2^64, summed in a signed 128-bit integer
+// (exact over the whole range precondition; fixed64_add).  On a bf16 head
+// without elements of magnitude 2^16 or more (the input check flags the others;
+// unit-scale data has none) the same integer is reached faster:
+//   * rows without a nonzero element below 2^-20 (the input check flags the
+//     others, one byte per row) go into float64 partial sums per element,
+//     exact for 1024 rows (every element is a multiple of 2^-27 below 2^16:
+//     1024 of them need at most 53 bits), moved every 1024 rows into an int64
+//     sum of x * 2^27 (at most 128 moves per thread: below 2^60);
+//   * a flagged row's piece goes, out of line, to int64 sums in shared memory:
+//     x * 2^47 for its elements below 2^-20 (below 2^27 inside the range),
+//     x * 2^27 for the others.
+// Other heads, and float32 inputs, take the general path, out of line.
+
+// The general path of one thread: 128-bit sums of its VEC elements over rows
+// slot, slot + RPI, ..., written to red_hi / red_lo.
+template <typename T>
+__device__ __noinline__ void update_exact_rows(const T* __restrict__ Xh, const int32_t* __restrict__ pm, int n,
+                                               int D, int piece, int slot, int RPI, long long* red_hi,
+                                               long long* red_lo) {
+    constexpr int VEC = 16 / sizeof(T);
+    long long hi[VEC];
+    unsigned long long lo[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        hi[e] = 0;
+        lo[e] = 0;
+    }
+    for (int j = slot; j < n; j += RPI) {
+        const uint4 v = *reinterpret_cast<const uint4*>(Xh + (size_t)pm[j] * D + piece * VEC);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            const uint32_t u = sizeof(T) == 2 ? ((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16)) : w[e];
+            fixed64_add(lo[e], hi[e], u);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        red_hi[slot * D + piece * VEC + e] = hi[e];
+        red_lo[slot * D + piece * VEC + e] = (long long)lo[e];
+    }
+}
+
+// x * 2^47 of a bf16 element (IEEE-single bits u) with 2^-40 <= |x| < 2^-20:
+// the significand m (8 bits with the leading one) shifted by e - 87 (0 .. 19);
+// lower exponents (outside the range precondition, reported by the input check)
+// are clamped.
+__device__ inline long long tiny_fixed47(uint32_t u) {
+    const int e = (u >> 23) & 0xFF;
+    const long long m = (long long)(0x80u | ((u >> 16) & 0x7Fu));
+    const int sh = e - 87;
+    const long long v = sh >= 0 ? (m << sh) : (m >> min(-sh, 63));
+    return (u & 0x80000000u) ? -v : v;
+}
+
+// A piece of a flagged bf16 row: elements below 2^-20 add x * 2^47 to tiny[e],
+// the others (2^-20 <= |x| < 2^16 on a head without larger values, or 0) add
+// the integer x * 2^27 to norm[e].
+__device__ __noinline__ void update_tiny_piece(uint4 v, long long* tiny, long long* norm) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-        unsigned long long l = lo[e];
-        long long h = hi[e];
-        fixed64_add(l, h, (e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
-        lo[e] = l;
-        hi[e] = h;
+        const uint32_t b = (e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16);
+        const uint32_t mag = b & 0x7FFFFFFFu;
+        if (mag == 0u) continue;
+        if (mag < 0x35800000u) {
+            tiny[e] += tiny_fixed47(b);
+        } else {  // m << (e - 107): an integer below 2^43
+            const int ex = (b >> 23) & 0xFF;
+            const long long m = (long long)(0x80u | ((b >> 16) & 0x7Fu)) << min(max(ex - 107, 0), 35);
+            norm[e] += (b & 0x80000000u) ? -m : m;
+        }
     }
 }
+
+constexpr int kUpdStage = 1024;  // member tokens staged in shared memory at a time
 
 template <typename T>
 __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const int32_t* __restrict__ perm,
                                                 const int32_t* __restrict__ offsets, int N, int D, int K,
-                                                T* __restrict__ C) {
+                                                T* __restrict__ C, const int32_t* __restrict__ wide,
+                                                const uint8_t* __restrict__ tiny_rows) {
     constexpr int VEC = 16 / sizeof(T);
-    constexpr bool BF16 = sizeof(T) == 2;
     extern __shared__ long long red[];  // [2][RPI][D]: high and low words of the 128-bit sums
-    __shared__ unsigned long long slow_lo[BF16 ? 128 * VEC : 1];
-    __shared__ long long slow_hi[BF16 ? 128 * VEC : 1];
+    __shared__ int32_t stok[sizeof(T) == 2 ? kUpdStage : 1];  // member tokens of the current stage
     int k = blockIdx.x, bh = blockIdx.y;
     const int32_t* off = offsets + (size_t)bh * (K + 1);
     int start = off[k], n = off[k + 1] - start;
     if (n == 0) return;  // empty cluster keeps its centroid
     const int CPR = D / VEC, RPI = 128 / CPR;
     int t = threadIdx.x, piece = t % CPR, slot = t / CPR;
-    long long acc_hi[BF16 ? 1 : VEC];             // float32: 128-bit sums in registers
-    unsigned long long acc_lo[BF16 ? 1 : VEC];
-    long long mid[BF16 ? VEC : 1];                // bf16: flushed partials, units of 2^37
-    double part[BF16 ? VEC : 1];
-#pragma unroll
-    for (int e = 0; e < (BF16 ? 1 : VEC); ++e) {
-        acc_hi[e] = 0;
-        acc_lo[e] = 0;
-    }
-#pragma unroll
-    for (int e = 0; e < (BF16 ? VEC : 1); ++e) {
-        mid[e] = 0;
-        part[e] = 0.0;
-    }
-    if (BF16) {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-            slow_lo[t * VEC + e] = 0ull;
-            slow_hi[t * VEC + e] = 0;
-        }
-    }
-    const int32_t* pm = perm + (size_t)bh * N + start;
-    const T* Xh = X + (size_t)bh * N * D;
-    int rows_in_part = 0;
-    auto flush = [&]() {
-        if (BF16) {
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                mid[e] += __double2ll_rn(ldexp(part[e], 27));  // exact: a multiple of 2^-27 below 2^26
-                part[e] = 0.0;
-            }
-        }
-        rows_in_part = 0;
-    };
-    auto add_piece = [&](const uint4& v) {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        if (BF16) {
-            // the common case, decided once per 16-byte piece with 16-bit SIMD compares:
-            // every element is 0 or has 2^-20 <= |x| < 2^16 (biased exponent 107..142)
-            uint32_t bad = 0;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t ex = (w[q] >> 7) & 0x00FF00FFu;
-                const uint32_t in = __vcmpgeu2(ex, 0x006B006Bu) & __vcmpleu2(ex, 0x008E008Eu);
-                bad |= ~(in | __vcmpeq2(w[q] & 0x7FFF7FFFu, 0u));
-            }
-            if (bad == 0) {
-#pragma unroll
-                for (int e = 0; e < VEC; ++e)
-                    part[e] += (double)__uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
-            } else {  // rare: the whole piece goes to the 128-bit sums, out of line
-                update_slow_piece(v, slow_lo + t * VEC, slow_hi + t * VEC);
-            }
-            if (++rows_in_part == 1024) flush();
-        } else {
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) fixed64_add(acc_lo[e], acc_hi[e], w[e]);
-        }
-    };
-    if (slot < RPI) {
-        // four member rows in flight per thread (integer sums: the order does not matter)
-        int j = slot;
-        for (; j + 3 * RPI < n; j += 4 * RPI) {
-            int tok[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) tok[u] = pm[j + u * RPI];
-            uint4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const uint4*>(Xh + (size_t)tok[u] * D + piece * VEC);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) add_piece(v[u]);
-        }
-        for (; j < n; j += RPI) add_piece(*reinterpret_cast<const uint4*>(Xh + (size_t)pm[j] * D + piece * VEC));
-        flush();
-    }
     long long* red_hi = red;
     long long* red_lo = red + RPI * D;
-    if (slot < RPI) {
+    const int32_t* pm = perm + (size_t)bh * N + start;
+    const T* Xh = X + (size_t)bh * N * D;
+    // uniform over the CTA
+    const bool fast = sizeof(T) == 2 && wide != nullptr && tiny_rows != nullptr && wide[bh] == 0 && RPI * CPR == 128;
+    if (!fast) {
+        if (slot < RPI) update_exact_rows<T>(Xh, pm, n, D, piece, slot, RPI, red_hi, red_lo);
+    } else {
+        const uint8_t* trow = tiny_rows + (size_t)bh * N;
+        // this thread's entries of red (slot * D + piece * VEC = t * VEC) hold, until the
+        // end, the flagged rows' int64 sums: x * 2^27 in red_hi, x * 2^47 in red_lo
+        long long* norm = red_hi + t * VEC;
+        long long* tiny = red_lo + t * VEC;
+        long long acc[VEC];  // sums of x * 2^27
+        double part[VEC];
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-            unsigned long long lo;
-            long long hi;
-            if (BF16) {  // mid * 2^37 plus the directly added elements
-                lo = (unsigned long long)mid[e] << 37;
-                hi = mid[e] >> 27;
-                acc128_add(lo, hi, slow_lo[t * VEC + e], slow_hi[t * VEC + e]);
-            } else {
-                lo = acc_lo[e];
-                hi = acc_hi[e];
+            acc[e] = 0;
+            part[e] = 0.0;
+            norm[e] = 0;
+            tiny[e] = 0;
+        }
+        auto flush = [&]() {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                acc[e] += __double2ll_rn(ldexp(part[e], 27));  // exact: a multiple of 2^-27 below 2^26
+                part[e] = 0.0;
             }
-            red_hi[slot * D + piece * VEC + e] = hi;
-            red_lo[slot * D + piece * VEC + e] = (long long)lo;
+        };
+        auto add_fast = [&](const uint4& v) {
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < VEC; ++e)
+                part[e] += (double)__uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+        };
+        // The cluster's member tokens are staged in shared memory (kUpdStage at a time,
+        // one coalesced load), so each member row costs one dependent global load; eight
+        // rows in flight per thread (integer sums: the order does not matter).  A thread
+        // takes kUpdStage / RPI <= 1024 rows per stage: one flush per stage keeps every
+        // float64 partial sum within 1024 rows.
+        for (int base = 0; base < n; base += kUpdStage) {
+            const int cnt = min(kUpdStage, n - base);
+            __syncthreads();  // the previous stage's tokens have been read
+            for (int i = t; i < cnt; i += blockDim.x) stok[i] = pm[base + i];
+            __syncthreads();
+            int j = slot;
+            for (; j + 7 * RPI < cnt; j += 8 * RPI) {
+                uint4 v[8];
+                uint32_t fl = 0;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int tk = stok[j + u * RPI];
+                    v[u] = *reinterpret_cast<const uint4*>(Xh + (size_t)tk * D + piece * VEC);
+                    fl |= (uint32_t)trow[tk] << u;
+                }
+                if (fl == 0u) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) add_fast(v[u]);
+                } else {  // rare
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        if (fl >> u & 1u)
+                            update_tiny_piece(v[u], tiny, norm);
+                        else
+                            add_fast(v[u]);
+                    }
+                }
+            }
+            for (; j < cnt; j += RPI) {
+                const int tk = stok[j];
+                const uint4 v = *reinterpret_cast<const uint4*>(Xh + (size_t)tk * D + piece * VEC);
+                if (trow[tk])
+                    update_tiny_piece(v, tiny, norm);
+                else
+                    add_fast(v);
+            }
+            flush();
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            // x * 2^64 = (acc + norm) * 2^37 + tiny * 2^17 as a 128-bit integer (|acc + norm| < 2^61,
+            // |tiny| < 2^47)
+            const long long a = acc[e] + norm[e];
+            unsigned long long lo = (unsigned long long)a << 37;
+            long long hi = a >> 27;
+            const long long ts = tiny[e];
+            acc128_add(lo, hi, (unsigned long long)ts << 17, ts >> 47);
+            norm[e] = hi;  // = red_hi[slot * D + piece * VEC + e]
+            tiny[e] = (long long)lo;
         }
     }
     __syncthreads();
@@ -300,18 +406,19 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
 }
 
 int launch_update(const void* X, int dtype, int BH, int N, int D, int K, const int32_t* perm,
-                  const int32_t* offsets, void* C, cudaStream_t st) {
+                  const int32_t* offsets, void* C, const int32_t* wide, const uint8_t* tiny_rows,
+                  cudaStream_t st) {
     dim3 g(K, BH);
     const int vec = dtype == PARK_BF16 ? 8 : 4;
     if (D % vec || D / vec > 128) return PARK_ERR_UNSUPPORTED;
+    const int rpi = 128 / (D / vec);
     ::park::prof_begin(st);
-    if (dtype == PARK_BF16) {
-        int rpi = 128 / (D / 8);
-        k_update<bf16_t><<<g, 128, (size_t)rpi * D * 16, st>>>((const bf16_t*)X, perm, offsets, N, D, K, (bf16_t*)C);
-    } else {
-        int rpi = 128 / (D / 4);
-        k_update<float><<<g, 128, (size_t)rpi * D * 16, st>>>((const float*)X, perm, offsets, N, D, K, (float*)C);
-    }
+    if (dtype == PARK_BF16)
+        k_update<bf16_t><<<g, 128, (size_t)rpi * D * 16, st>>>((const bf16_t*)X, perm, offsets, N, D, K, (bf16_t*)C,
+                                                                wide, tiny_rows);
+    else
+        k_update<float><<<g, 128, (size_t)rpi * D * 16, st>>>((const float*)X, perm, offsets, N, D, K, (float*)C,
+                                                               nullptr, nullptr);
     PARK_TRY_LAUNCH("k_update", st);
     return PARK_OK;
 }

@@ -30,7 +30,12 @@ struct Lists {
 };
 
 // ---- k_prep.cu
-int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status, cudaStream_t st);
+// wide (bf16, may be null): per-head flags, set where an element has
+// |x| >= 2^16 (zeroed by the caller); per_head_elems = N * D.  tiny_rows (bf16,
+// may be null): one byte per row of row_elems elements, set to 1 where the row
+// holds a nonzero element with |x| < 2^-20 (zeroed by the caller).
+int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status, int32_t* wide,
+                       size_t per_head_elems, uint8_t* tiny_rows, size_t row_elems, cudaStream_t st);
 int launch_metric(const void* Q, int dtype, int BH, int N, int D, double* part, int nchunks, double* M,
                   double* M_out, cudaStream_t st);
 int launch_row_norms(const void* X, int dtype, int BH, int N, int D, float* xnorm, cudaStream_t st);
@@ -52,8 +57,11 @@ int launch_recheck_rows(const void* X, int dtype, int BH, int N, int D, int K, c
 // ---- k_sort.cu
 int launch_label_sort(const int32_t* labels, int BH, int N, int K, int32_t* hist, int nchunks, int32_t* perm,
                       int32_t* offsets, cudaStream_t st);
+// wide, tiny_rows: the per-head and per-row flags of launch_input_check for X
+// (either null: every head takes the general path).
 int launch_update(const void* X, int dtype, int BH, int N, int D, int K, const int32_t* perm,
-                  const int32_t* offsets, void* C, cudaStream_t st);
+                  const int32_t* offsets, void* C, const int32_t* wide, const uint8_t* tiny_rows,
+                  cudaStream_t st);
 
 // ---- k_pama.cu
 // size_prior: logits gain log |B_m|.  select: 0 top-p; 1 top-k, the ceil(p L) most

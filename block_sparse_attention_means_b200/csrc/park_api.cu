@@ -127,7 +127,7 @@ int metric_chunks(const Dims& d) {
 
 struct RetrievalWs {
     size_t M, Mpart, xnorm_q, xnorm_k, wop, b32, b64, w64, wmax, bmax, lfull, lcnt, hist, rho, plist,
-        pcnt, kcnt, f64z, cperm, coff, mS, mP, mI, mX, mH, txt, qg, total;
+        pcnt, kcnt, f64z, cperm, coff, mS, mP, mI, mX, mH, txt, qg, wide, tiny, total;
 };
 
 RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
@@ -151,6 +151,8 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
     w.rho = c.take(BH * NQ * 4);
     w.plist = c.take(BH * NQ * 4);
     w.pcnt = c.take(16 * 4);
+    w.wide = c.take(2 * BH * 4);  // per-head flags of Q and K: an element with |x| >= 2^16
+    w.tiny = c.take(2 * BH * N);  // per-row flags of Q and K: a nonzero element with |x| < 2^-20
     w.kcnt = c.take(BH * NQ * 4);
     w.f64z = c.take(pama_f64_scratch_bytes(NK));
     w.cperm = c.take(BH * NQ * 4);
@@ -283,6 +285,8 @@ struct Side {
     int32_t* status;
     const WinGeom* win;  // non-null: HVA local-window assign
     int n_text;
+    const int32_t* wide;       // per-head flags of X from the input check (general update path)
+    const uint8_t* tiny_rows;  // per-row flags of X from the input check (out-of-line update rows)
 };
 
 int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, void* ws, int64_t* counters,
@@ -323,7 +327,7 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
                                               ops.wmax, ops.bmax, at<void>(ws, w.txt), s.labels, counters,
                                               s.cnt_slot, st));
             PARK_CHECK(launch_label_sort(s.labels, BH, N, K, at<int32_t>(ws, w.hist), nchunks, s.perm, s.offsets, st));
-            PARK_CHECK(launch_update(s.X, d.dtype, BH, N, D, K, s.perm, s.offsets, s.C, st));
+            PARK_CHECK(launch_update(s.X, d.dtype, BH, N, D, K, s.perm, s.offsets, s.C, s.wide, s.tiny_rows, st));
         }
         return PARK_OK;
     }
@@ -347,7 +351,7 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
                                       num_sms, counters, s.cnt_slot, st));
         }
         PARK_CHECK(launch_label_sort(s.labels, BH, N, K, at<int32_t>(ws, w.hist), nchunks, s.perm, s.offsets, st));
-        PARK_CHECK(launch_update(s.X, d.dtype, BH, N, D, K, s.perm, s.offsets, s.C, st));
+        PARK_CHECK(launch_update(s.X, d.dtype, BH, N, D, K, s.perm, s.offsets, s.C, s.wide, s.tiny_rows, st));
     }
     return PARK_OK;
 }
@@ -415,8 +419,13 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
     PARK_CHECK(memset_async(out->status, 4, st));
     PARK_CHECK(memset_async(out->counters, PARK_NUM_COUNTERS * 8, st));
     PARK_CHECK(memset_async(at<int32_t>(ws, w.pcnt), 16 * 4, st));
-    PARK_CHECK(launch_input_check(Q, nel, d.dtype, out->status, st));
-    PARK_CHECK(launch_input_check(K, nel, d.dtype, out->status, st));
+    int32_t* wide = at<int32_t>(ws, w.wide);
+    uint8_t* tiny = at<uint8_t>(ws, w.tiny);
+    PARK_CHECK(memset_async(wide, (size_t)2 * BH * 4, st));
+    PARK_CHECK(memset_async(tiny, (size_t)2 * BH * N, st));
+    PARK_CHECK(launch_input_check(Q, nel, d.dtype, out->status, wide, (size_t)N * D, tiny, D, st));
+    PARK_CHECK(launch_input_check(K, nel, d.dtype, out->status, wide + BH, (size_t)N * D, tiny + (size_t)BH * N, D,
+                                  st));
     const uint32_t fl = out->flags;
     const bool qrkc = (fl & PARK_FLAG_NO_QRKC) == 0;
     const int select = (fl & PARK_FLAG_SIP) ? 2 : ((fl & PARK_FLAG_TOPK) ? 1 : 0);
@@ -432,10 +441,10 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
     const WinGeom* win = (fl & PARK_FLAG_LOCAL_WINDOW) ? &geo : nullptr;
     Side sq{Q, NQ, out->q_centroids, out->q_labels, out->q_perm, out->q_offsets, nullptr,
             (out->flags & PARK_FLAG_WARM_START_Q) != 0, PARK_CNT_Q_RECHECK, at<float>(ws, w.xnorm_q),
-            NQ > NK ? NQ : NK, out->status, win, N - d.nvideo};
+            NQ > NK ? NQ : NK, out->status, win, N - d.nvideo, wide, tiny};
     Side sk{K, NK, out->k_centroids, out->k_labels, out->k_perm, out->k_offsets, qrkc ? M : nullptr,
             (out->flags & PARK_FLAG_WARM_START_K) != 0, PARK_CNT_K_RECHECK, at<float>(ws, w.xnorm_k),
-            NQ > NK ? NQ : NK, out->status, win, N - d.nvideo};
+            NQ > NK ? NQ : NK, out->status, win, N - d.nvideo, wide + BH, tiny + (size_t)BH * N};
     PARK_CHECK(run_kmeans(d, sq, iters, w, ws, out->counters, num_sms, st));
     PARK_CHECK(run_kmeans(d, sk, iters, w, ws, out->counters, num_sms, st));
 
@@ -484,7 +493,8 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
         const int nchunks = (N + kSortChunk - 1) / kSortChunk;
         PARK_CHECK(launch_label_sort(out->q_labels, BH, N, NQ, at<int32_t>(ws, w.hist), nchunks, out->q_perm,
                                      out->q_offsets, st));
-        PARK_CHECK(launch_update(Q, d.dtype, BH, N, D, NQ, out->q_perm, out->q_offsets, out->q_centroids, st));
+        PARK_CHECK(launch_update(Q, d.dtype, BH, N, D, NQ, out->q_perm, out->q_offsets, out->q_centroids, wide, tiny,
+                                 st));
     }
     PARK_CHECK(launch_kept_csr(out->mask, kcnt, BH, NQ, NK, out->kept_ptr, out->kept_idx, out->counters, st));
     return PARK_OK;
@@ -495,7 +505,7 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
     const AttnWs w = plan_attn(d, NQ, NK);
     const int BH = d.BH, N = d.N, D = d.D;
     const bool bf16 = d.dtype == PARK_BF16;
-    PARK_CHECK(launch_input_check(V, (size_t)BH * N * D, d.dtype, r->status, st));
+    PARK_CHECK(launch_input_check(V, (size_t)BH * N * D, d.dtype, r->status, nullptr, (size_t)N * D, nullptr, D, st));
     PARK_CHECK(memset_async(r->counters + PARK_CNT_KEPT_PAIRS, 3 * sizeof(int64_t), st));
     int32_t* icnt = at<int32_t>(ws, w.icnt);
     PARK_CHECK(memset_async(icnt, 16 * 4, st));
