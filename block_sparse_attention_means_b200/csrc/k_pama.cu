@@ -20,28 +20,36 @@ namespace park {
 
 // ---------------------------------------------------------------- sort helpers
 // Bitonic sort of n (power of two) (value, index) pairs: value descending,
-// ties by index ascending.  All threads of the block take part.
+// ties by index ascending.  All threads of the block take part (a multiple of
+// 32).  Each stage (k, j) compares n / 2 pairs (i, i + j), pair q taking
+// i = 2 (q - q mod j) + q mod j, so no thread only tests its index.  The 32
+// pairs of a warp then touch one aligned block of 64 elements whenever j <= 32,
+// so consecutive stages with j <= 32 need only a warp barrier; a block barrier
+// separates every stage that crosses warps.
 template <typename V>
 __device__ void bitonic_desc(V* v, int32_t* idx, int n) {
     for (int k = 2; k <= n; k <<= 1) {
         for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = threadIdx.x; i < n; i += blockDim.x) {
-                int ixj = i ^ j;
-                if (ixj > i) {
-                    V a = v[i], b = v[ixj];
-                    int ia = idx[i], ib = idx[ixj];
-                    bool b_first = (b > a) || (b == a && ib < ia);
-                    bool a_first = (a > b) || (a == b && ia < ib);
-                    bool up = (i & k) == 0;
-                    if (up ? b_first : a_first) {
-                        v[i] = b;
-                        v[ixj] = a;
-                        idx[i] = ib;
-                        idx[ixj] = ia;
-                    }
+            for (int q = threadIdx.x; q < (n >> 1); q += blockDim.x) {
+                const int i = ((q & ~(j - 1)) << 1) | (q & (j - 1));
+                const int ixj = i | j;
+                const V a = v[i], b = v[ixj];
+                const int ia = idx[i], ib = idx[ixj];
+                const bool b_first = (b > a) || (b == a && ib < ia);
+                const bool a_first = (a > b) || (a == b && ia < ib);
+                const bool up = (i & k) == 0;
+                if (up ? b_first : a_first) {
+                    v[i] = b;
+                    v[ixj] = a;
+                    idx[i] = ib;
+                    idx[ixj] = ia;
                 }
             }
-            __syncthreads();
+            const int jn = j > 1 ? j >> 1 : k;  // the next stage's j
+            if (j > 32 || jn > 32 || (j == 1 && k == n))
+                __syncthreads();
+            else
+                __syncwarp();
         }
     }
 }

@@ -12,15 +12,35 @@ namespace park {
 // head takes its general 128-bit path instead of the float64 partial sums
 // (k_sort.cu); and tiny_rows[r] (when given) for every row r holding a nonzero
 // element with |x| < 2^-20 (about one row in ten thousand in unit-scale data),
-// which the float64 partial sums cannot take exactly either.
+// which the float64 partial sums cannot take exactly either.  With xnorm given
+// (bf16 rows of 128 elements: 16 pieces, one per lane of a half warp) it also
+// writes every row's ||x||, as k_row_norms does (float64 sum of squares, square
+// root rounded up to float), so the K-means needs no second pass over X.
 template <int BYTES>
 __global__ void k_input_check(const uint4* __restrict__ x, size_t n16, int32_t* status, size_t per_head16,
-                              int32_t* __restrict__ wide, uint8_t* __restrict__ tiny_rows, size_t row16) {
-    size_t stride = (size_t)gridDim.x * blockDim.x;
+                              int32_t* __restrict__ wide, uint8_t* __restrict__ tiny_rows, size_t row16,
+                              float* __restrict__ xnorm) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;  // a multiple of 32
+    const int lane = threadIdx.x & 31;
     bool bad = false;
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += stride) {
-        uint4 v = x[i];
+    // warp-uniform trip count: the half-warp reductions below need every lane
+    for (size_t i0 = (size_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31u); i0 < n16; i0 += stride) {
+        const size_t i = i0 + lane;
+        const bool in = i < n16;
+        uint4 v = in ? x[i] : make_uint4(0u, 0u, 0u, 0u);
         uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        if (BYTES == 2 && xnorm != nullptr) {
+            double ss = 0.0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const double lo = (double)__uint_as_float(w[q] << 16), hi = (double)__uint_as_float(w[q] & 0xffff0000u);
+                ss = fma(lo, lo, ss);
+                ss = fma(hi, hi, ss);
+            }
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            if (in && (lane & 15) == 0) xnorm[i >> 4] = round_up_f(__double2float_ru(sqrt(ss)));
+        }
         bool narrow = true, tiny = false;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -40,14 +60,15 @@ __global__ void k_input_check(const uint4* __restrict__ x, size_t n16, int32_t* 
                 bad |= !in_range_exp(e, mag);
             }
         }
-        if (BYTES == 2 && !narrow && wide) atomicOr(wide + i / per_head16, 1);  // rare
-        if (BYTES == 2 && tiny && tiny_rows) tiny_rows[i / row16] = 1;            // rare
+        if (in && BYTES == 2 && !narrow && wide) atomicOr(wide + i / per_head16, 1);  // rare
+        if (in && BYTES == 2 && tiny && tiny_rows) tiny_rows[i / row16] = 1;            // rare
     }
     if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) set_status(status, PARK_ERR_RANGE);
 }
 
 int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status, int32_t* wide,
-                       size_t per_head_elems, uint8_t* tiny_rows, size_t row_elems, cudaStream_t st) {
+                       size_t per_head_elems, uint8_t* tiny_rows, size_t row_elems, float* xnorm,
+                       cudaStream_t st) {
     int eb = dtype == PARK_BF16 ? 2 : 4;
     size_t n16 = n_elems * eb / 16;
     int blocks = (int)((n16 + 255) / 256);
@@ -58,9 +79,11 @@ int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status
     const size_t r16 = row_elems * eb / 16;          // and so is a row
     if (eb == 2)
         k_input_check<2><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status, ph16 ? ph16 : 1, wide,
-                                                 r16 ? tiny_rows : nullptr, r16 ? r16 : 1);
+                                                 r16 ? tiny_rows : nullptr, r16 ? r16 : 1,
+                                                 r16 == 16 ? xnorm : nullptr);
     else
-        k_input_check<4><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status, ph16 ? ph16 : 1, nullptr, nullptr, 1);
+        k_input_check<4><<<blocks, 256, 0, st>>>((const uint4*)x, n16, status, ph16 ? ph16 : 1, nullptr, nullptr, 1,
+                                                 nullptr);
     PARK_TRY_LAUNCH("k_input_check", st);
     return PARK_OK;
 }

@@ -243,10 +243,11 @@ __device__ __noinline__ void update_exact_rows(const T* __restrict__ Xh, const i
             fixed64_add(lo[e], hi[e], u);
         }
     }
+    const int CPR = D / VEC;
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-        red_hi[slot * D + piece * VEC + e] = hi[e];
-        red_lo[slot * D + piece * VEC + e] = (long long)lo[e];
+    for (int e = 0; e < VEC; ++e) {  // layout [slot][e][piece]
+        red_hi[slot * D + e * CPR + piece] = hi[e];
+        red_lo[slot * D + e * CPR + piece] = (long long)lo[e];
     }
 }
 
@@ -262,10 +263,10 @@ __device__ inline long long tiny_fixed47(uint32_t u) {
     return (u & 0x80000000u) ? -v : v;
 }
 
-// A piece of a flagged bf16 row: elements below 2^-20 add x * 2^47 to tiny[e],
-// the others (2^-20 <= |x| < 2^16 on a head without larger values, or 0) add
-// the integer x * 2^27 to norm[e].
-__device__ __noinline__ void update_tiny_piece(uint4 v, long long* tiny, long long* norm) {
+// A piece of a flagged bf16 row: elements below 2^-20 add x * 2^47 to
+// tiny[e * stride], the others (2^-20 <= |x| < 2^16 on a head without larger
+// values, or 0) add the integer x * 2^27 to norm[e * stride].
+__device__ __noinline__ void update_tiny_piece(uint4 v, long long* tiny, long long* norm, int stride) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -273,19 +274,30 @@ __device__ __noinline__ void update_tiny_piece(uint4 v, long long* tiny, long lo
         const uint32_t mag = b & 0x7FFFFFFFu;
         if (mag == 0u) continue;
         if (mag < 0x35800000u) {
-            tiny[e] += tiny_fixed47(b);
+            tiny[e * stride] += tiny_fixed47(b);
         } else {  // m << (e - 107): an integer below 2^43
             const int ex = (b >> 23) & 0xFF;
             const long long m = (long long)(0x80u | ((b >> 16) & 0x7Fu)) << min(max(ex - 107, 0), 35);
-            norm[e] += (b & 0x80000000u) ? -m : m;
+            norm[e * stride] += (b & 0x80000000u) ? -m : m;
         }
     }
 }
 
 constexpr int kUpdStage = 1024;  // member tokens staged in shared memory at a time
 
+// The float64 value of a bf16 element given as IEEE-single bits f (low 16 bits
+// zero), for 0 and normal values, built with integer operations: the sign, the
+// exponent rebiased by 1023 - 127 and the 7 stored significand bits in the high
+// word, a zero low word.  (The float32 -> float64 conversion instruction runs at a
+// fraction of the integer rate and bounded the update.)
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t f) {
+    const uint32_t mag = f & 0x7FFFFFFFu;
+    const uint32_t hi = mag ? (((mag >> 3) + 0x38000000u) | (f & 0x80000000u)) : f;
+    return __hiloint2double((int)hi, 0);
+}
+
 template <typename T>
-__global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const int32_t* __restrict__ perm,
+__global__ __launch_bounds__(128, 5) void k_update(const T* __restrict__ X, const int32_t* __restrict__ perm,
                                                 const int32_t* __restrict__ offsets, int N, int D, int K,
                                                 T* __restrict__ C, const int32_t* __restrict__ wide,
                                                 const uint8_t* __restrict__ tiny_rows) {
@@ -308,23 +320,24 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
         if (slot < RPI) update_exact_rows<T>(Xh, pm, n, D, piece, slot, RPI, red_hi, red_lo);
     } else {
         const uint8_t* trow = tiny_rows + (size_t)bh * N;
-        // this thread's entries of red (slot * D + piece * VEC = t * VEC) hold, until the
-        // end, the flagged rows' int64 sums: x * 2^27 in red_hi, x * 2^47 in red_lo
-        long long* norm = red_hi + t * VEC;
-        long long* tiny = red_lo + t * VEC;
-        long long acc[VEC];  // sums of x * 2^27
+        // until the end, red holds the flagged rows' int64 sums element-major ([e][t]:
+        // consecutive threads, consecutive words): x * 2^27 in red_hi for their elements of
+        // 2^-20 and above, x * 2^47 in red_lo for those below
+        long long* norm = red_hi + t;
+        long long* tiny = red_lo + t;
+        long long acc[VEC];  // x * 2^27: the flushed float64 partial sums
         double part[VEC];
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
             acc[e] = 0;
             part[e] = 0.0;
-            norm[e] = 0;
-            tiny[e] = 0;
+            norm[e * 128] = 0;
+            tiny[e * 128] = 0;
         }
         auto flush = [&]() {
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
-                acc[e] += __double2ll_rn(ldexp(part[e], 27));  // exact: a multiple of 2^-27 below 2^26
+                acc[e] += __double2ll_rn(part[e] * 0x1p27);  // exact: a multiple of 2^-27 below 2^26
                 part[e] = 0.0;
             }
         };
@@ -332,27 +345,38 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int e = 0; e < VEC; ++e)
-                part[e] += (double)__uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+                part[e] += bf16_bits_to_f64((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
         };
         // The cluster's member tokens are staged in shared memory (kUpdStage at a time,
-        // one coalesced load), so each member row costs one dependent global load; eight
-        // rows in flight per thread (integer sums: the order does not matter).  A thread
+        // one coalesced load), each with its row's flag in the sign bit (one flag load per
+        // row instead of one per 16-byte piece: those cost 40 % of the kernel), so each
+        // member row costs one dependent global load; eight rows in flight per thread
+        // (integer sums: the order does not matter).  A thread
         // takes kUpdStage / RPI <= 1024 rows per stage: one flush per stage keeps every
         // float64 partial sum within 1024 rows.
         for (int base = 0; base < n; base += kUpdStage) {
             const int cnt = min(kUpdStage, n - base);
             __syncthreads();  // the previous stage's tokens have been read
-            for (int i = t; i < cnt; i += blockDim.x) stok[i] = pm[base + i];
+            for (int i = t; i < cnt; i += blockDim.x) {
+                const int tk = pm[base + i];
+                stok[i] = trow[tk] ? (tk | (int)0x80000000u) : tk;
+            }
             __syncthreads();
-            int j = slot;
-            for (; j + 7 * RPI < cnt; j += 8 * RPI) {
+            // every batch, the last one included, keeps its eight loads in flight: rows past
+            // the stage read as zero, which adds nothing to the exact sums
+            for (int j = slot; j < cnt; j += 8 * RPI) {
                 uint4 v[8];
                 uint32_t fl = 0;
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const int tk = stok[j + u * RPI];
-                    v[u] = *reinterpret_cast<const uint4*>(Xh + (size_t)tk * D + piece * VEC);
-                    fl |= (uint32_t)trow[tk] << u;
+                    const int r = j + u * RPI;
+                    v[u] = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < cnt) {
+                        const int sv = stok[r];
+                        const int tk = sv & 0x7FFFFFFF;
+                        v[u] = *reinterpret_cast<const uint4*>(Xh + (size_t)tk * D + piece * VEC);
+                        fl |= (uint32_t)(sv < 0) << u;
+                    }
                 }
                 if (fl == 0u) {
 #pragma unroll
@@ -361,43 +385,44 @@ __global__ __launch_bounds__(128) void k_update(const T* __restrict__ X, const i
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         if (fl >> u & 1u)
-                            update_tiny_piece(v[u], tiny, norm);
+                            update_tiny_piece(v[u], tiny, norm, 128);
                         else
                             add_fast(v[u]);
                     }
                 }
             }
-            for (; j < cnt; j += RPI) {
-                const int tk = stok[j];
-                const uint4 v = *reinterpret_cast<const uint4*>(Xh + (size_t)tk * D + piece * VEC);
-                if (trow[tk])
-                    update_tiny_piece(v, tiny, norm);
-                else
-                    add_fast(v);
-            }
             flush();
         }
+        long long hv[VEC];
+        unsigned long long lv[VEC];
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
             // x * 2^64 = (acc + norm) * 2^37 + tiny * 2^17 as a 128-bit integer (|acc + norm| < 2^61,
             // |tiny| < 2^47)
-            const long long a = acc[e] + norm[e];
-            unsigned long long lo = (unsigned long long)a << 37;
-            long long hi = a >> 27;
-            const long long ts = tiny[e];
-            acc128_add(lo, hi, (unsigned long long)ts << 17, ts >> 47);
-            norm[e] = hi;  // = red_hi[slot * D + piece * VEC + e]
-            tiny[e] = (long long)lo;
+            const long long a = acc[e] + norm[e * 128];
+            lv[e] = (unsigned long long)a << 37;
+            hv[e] = a >> 27;
+            const long long ts = tiny[e * 128];
+            acc128_add(lv[e], hv[e], (unsigned long long)ts << 17, ts >> 47);
+        }
+        __syncthreads();  // every thread has read its element-major entries
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {  // layout [slot][e][piece]
+            red_hi[slot * D + e * CPR + piece] = hv[e];
+            red_lo[slot * D + e * CPR + piece] = (long long)lv[e];
         }
     }
     __syncthreads();
     if (t < D) {
+        // thread t reduces column piece * VEC + e with piece = t % CPR, e = t / CPR: its
+        // slot partials sit at q * D + t in the [slot][e][piece] layout
+        const int col = (t % CPR) * VEC + t / CPR;
         long long sh = 0;
         unsigned long long sl = 0;
         for (int q = 0; q < RPI; ++q) acc128_add(sl, sh, (unsigned long long)red_lo[q * D + t], red_hi[q * D + t]);
         // one correct rounding of the exact sum to float64, then the IEEE division by n
         const double mean = ldexp(i128_to_double_rn(sh, sl), -64) / (double)n;
-        T* c = C + ((size_t)bh * K + k) * D + t;
+        T* c = C + ((size_t)bh * K + k) * D + col;
         if (sizeof(T) == 2)
             reinterpret_cast<uint16_t*>(c)[0] = double_to_bf16_bits(mean);
         else

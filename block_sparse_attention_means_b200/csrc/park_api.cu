@@ -334,7 +334,8 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
     // labels start valid (cluster 0), so that a kernel that gave up on a bounded
     // wait (status PARK_ERR_TIMEOUT) leaves nothing out of range for the later steps
     PARK_CHECK(memset_async(s.labels, (size_t)BH * N * 4, st));
-    if (bf16) PARK_CHECK(launch_row_norms(s.X, d.dtype, BH, N, D, s.xnorm, st));
+    // (bf16 with D = 128: the input check has written them)
+    if (bf16 && D != 128) PARK_CHECK(launch_row_norms(s.X, d.dtype, BH, N, D, s.xnorm, st));
     if (!s.warm) PARK_CHECK(launch_strided_init(s.X, d.dtype, BH, N, D, K, s.C, st));
     const float gamma = gamma_for(ops.kw, s.M != nullptr);
     for (int it = 0; it < iters; ++it) {
@@ -423,9 +424,12 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
     uint8_t* tiny = at<uint8_t>(ws, w.tiny);
     PARK_CHECK(memset_async(wide, (size_t)2 * BH * 4, st));
     PARK_CHECK(memset_async(tiny, (size_t)2 * BH * N, st));
-    PARK_CHECK(launch_input_check(Q, nel, d.dtype, out->status, wide, (size_t)N * D, tiny, D, st));
+    // bf16 with D = 128: the checks also write the row norms the certified assign bound uses
+    const bool norms = d.dtype == PARK_BF16 && D == 128;
+    PARK_CHECK(launch_input_check(Q, nel, d.dtype, out->status, wide, (size_t)N * D, tiny, D,
+                                  norms ? at<float>(ws, w.xnorm_q) : nullptr, st));
     PARK_CHECK(launch_input_check(K, nel, d.dtype, out->status, wide + BH, (size_t)N * D, tiny + (size_t)BH * N, D,
-                                  st));
+                                  norms ? at<float>(ws, w.xnorm_k) : nullptr, st));
     const uint32_t fl = out->flags;
     const bool qrkc = (fl & PARK_FLAG_NO_QRKC) == 0;
     const int select = (fl & PARK_FLAG_SIP) ? 2 : ((fl & PARK_FLAG_TOPK) ? 1 : 0);
@@ -505,7 +509,8 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
     const AttnWs w = plan_attn(d, NQ, NK);
     const int BH = d.BH, N = d.N, D = d.D;
     const bool bf16 = d.dtype == PARK_BF16;
-    PARK_CHECK(launch_input_check(V, (size_t)BH * N * D, d.dtype, r->status, nullptr, (size_t)N * D, nullptr, D, st));
+    PARK_CHECK(launch_input_check(V, (size_t)BH * N * D, d.dtype, r->status, nullptr, (size_t)N * D, nullptr, D,
+                                  nullptr, st));
     PARK_CHECK(memset_async(r->counters + PARK_CNT_KEPT_PAIRS, 3 * sizeof(int64_t), st));
     int32_t* icnt = at<int32_t>(ws, w.icnt);
     PARK_CHECK(memset_async(icnt, 16 * 4, st));
