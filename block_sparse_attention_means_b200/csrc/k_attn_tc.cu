@@ -28,22 +28,25 @@
 //              two producers walk the same segment cursor, so K of tile j+3
 //              may arrive while V of tile j is still in use;
 //   warp 1     TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into TMEM
-//              buffer j%2 (128 x 128 fp32), O += P_j V_j into a TMEM
-//              accumulator (128 x 128 fp32) with P_j read from TMEM, in the
-//              order S0 S1 PV0 S2 PV1 S3 ...; tcgen05 MMAs of one thread run in
-//              issue order, so S_{j+2} overwrites buffer j%2 only after PV_j has
-//              read P_j from it.
+//              buffer j%2 (128 x 128 fp32), and for each column half h of the
+//              tile O_h += P_j,h V_j,h (K = 64) into that half's own TMEM
+//              accumulator (128 x 128 fp32), issued as soon as the half's P is
+//              in TMEM, in the order S0 S1 PV0 S2 PV1 S3 ...; tcgen05 MMAs of
+//              one thread run in issue order, so S_{j+2} overwrites buffer j%2
+//              only after PV_j has read P_j from it.
 //   warps 2-9  Softmax, two threads per query row (= TMEM lane; warps w and
 //              w+4 share a lane quadrant), each owning 64 of a tile's 128
 //              columns, with packed float32 pair arithmetic.  Online Softmax in
-//              the log2 domain with a lazily updated reference max (O is
-//              rescaled in TMEM only when a row max grows by more than 2^8);
-//              the two halves exchange their tile maxima through shared memory
-//              so both use the same reference.  P_j is written as bf16 pairs
-//              over the first 64 columns of S_j's TMEM buffer (the A operand of
-//              the PV MMA).  At the end the two partial row sums are added, and
-//              each thread normalises and writes its half of the O row in
-//              original token order.
+//              the log2 domain with a lazily updated reference max (the half's
+//              O is rescaled in TMEM only when its max grows by more than 2^8).
+//              Each half keeps its own reference, row sum and O accumulator, so
+//              the two threads of a row never wait for each other within an
+//              item.  P_j of a half is written as bf16 pairs over the first 32
+//              of the half's own 64 columns of S_j's TMEM buffer (the A operand
+//              of that half's PV MMA).  At the end of the item the two halves
+//              meet once: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M)
+//              + l_1 2^(m_1 - M)) with M = max(m_0, m_1), and each thread writes
+//              its half of the O row in original token order.
 // Every wait is time-bounded; a timeout sets PARK_ERR_TIMEOUT in the status
 // word, the roles leave their loops, outstanding copies and MMAs are waited
 // for (bounded) and TMEM is freed before the CTA exits.  Decisions that guard
@@ -64,20 +67,20 @@ constexpr int TC_ROWS = 128;            // query rows and key rows per tile
 constexpr int TC_BLK = 16384;           // 128 rows x 128 bytes
 constexpr int TC_KST = 3;  // K ring stages
 constexpr int TC_VST = 2;  // V ring stages (with the column bias)
-constexpr uint32_t TC_TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256,384)
+constexpr uint32_t TC_TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O_0 [256,384), O_1 [384,512)
 constexpr float kLog2eT = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
 
 struct TcSmem {
-    uint64_t q_full, q_empty, k_full[TC_KST], k_empty[TC_KST], v_full[TC_VST], v_empty[TC_VST], s_full[2], p_full[2], pv_done[2],
-        o_empty, final_bar;
+    uint64_t q_full, q_empty, k_full[TC_KST], k_empty[TC_KST], v_full[TC_VST], v_empty[TC_VST], s_full[2],
+        p_full[2][2], pv_done[2], o_empty, final_bar;  // p_full[column half][S buffer]
     uint32_t tmem_base;
     int abort;
     alignas(16) float bias[TC_VST][2][TC_ROWS];  // per stage, for the item's own rows [0] and its guest rows [1]:
                                                  // the logit term of a real key row, -inf for a pad row, a row
                                                  // past the end or a key cluster those query rows do not keep
-    float xmax[2][2][TC_ROWS];           // [tile parity][column half][row]: tile maxima of the two halves
-    float xl[2][TC_ROWS];                // [column half][row]: partial row sums
+    float xm[2][2][TC_ROWS];             // [item parity][column half][row]: the half's reference max
+    float xl[2][2][TC_ROWS];             // [item parity][column half][row]: the half's row sum
 };
 }  // namespace
 
@@ -126,7 +129,8 @@ __global__ void __launch_bounds__(352, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sh.s_full[s], 1);
-            mbar_init(&sh.p_full[s], 256);
+            mbar_init(&sh.p_full[0][s], 128);
+            mbar_init(&sh.p_full[1][s], 128);
             mbar_init(&sh.pv_done[s], 1);
         }
         mbar_init(&sh.o_empty, 256);
@@ -343,18 +347,27 @@ __global__ void __launch_bounds__(352, 1)
                 bool ok = issue_S(G) && (nkt < 2 || issue_S(G + 1));
                 for (int j = 0; j < nkt && ok; ++j) {
                     const int g = G + j, b = g & 1, ph = (g >> 1) & 1, vs = g % TC_VST;
-                    if (!mbar_wait(&sh.p_full[b], ph, abort, wait_ns) ||
-                        (j == 0 && I > 0 && !mbar_wait(&sh.o_empty, (I - 1) & 1, abort, wait_ns)) ||
+                    if ((j == 0 && I > 0 && !mbar_wait(&sh.o_empty, (I - 1) & 1, abort, wait_ns)) ||
                         !mbar_wait(&sh.v_full[vs], (g / TC_VST) & 1, abort, wait_ns)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
                     const uint32_t va = smem_u32(Vs + vs * 2 * TC_BLK);
+                    // each column half's keys (V rows 64 h .. 64 h + 63) into its own O_h, as
+                    // soon as that half's P is in TMEM (columns 64 h .. 64 h + 31 of buffer b)
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        if (!mbar_wait(&sh.p_full[h][b], ph, abort, wait_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16_ts(tmem + 256, tmem + (uint32_t)(b * 128 + 8 * kk),
-                                     sdesc_sw128(va + (uint32_t)kk * 4096, 1024, 2048), idPV, (j > 0 || kk > 0));
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16_ts(tmem + 256u + 128u * h, tmem + (uint32_t)(b * 128 + 64 * h + 8 * kk),
+                                         sdesc_sw128(va + (uint32_t)(4 * h + kk) * 4096, 1024, 2048), idPV,
+                                         (j > 0 || kk > 0));
+                    }
+                    if (!ok) break;
                     umma_commit(&sh.pv_done[b]);
                     umma_commit(&sh.v_empty[vs]);
                     if (j + 2 < nkt && !issue_S(g + 2)) ok = false;
@@ -376,12 +389,13 @@ __global__ void __launch_bounds__(352, 1)
         const int row = 32 * quad + lane;
         const uint32_t trow = tmem + ((uint32_t)(32 * quad) << 16);
         const int pair_bar = 1 + quad;  // named barrier of warps w and w+4 (64 threads)
+        const uint32_t o_col = 256u + 128u * (uint32_t)hc;  // this half's O accumulator
         const float2 sl2e2 = make_float2(sl2e, sl2e);
-        int G = 0;
+        int G = 0, I = 0;
         // Waits are decided per warp (tcgen05.ld/st and shuffles are warp-collective).
-        // The two warps of a pair pass their named barrier the same number of times
-        // whatever happens: after a failed wait a warp skips every later wait and all
-        // tensor-memory work but still walks the items and meets its barriers.
+        // The two warps of a pair pass their named barrier (once per item) the same number
+        // of times whatever happens: after a failed wait a warp skips every later wait and
+        // all tensor-memory work but still walks the items and meets its barriers.
         bool failed = false;
         auto wwait = [&](uint64_t* bar, uint32_t parity) {
             if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(bar, parity, abort, wait_ns));
@@ -428,41 +442,34 @@ __global__ void __launch_bounds__(352, 1)
                         }
                     }
                 }
-                // Both halves of the row agree on the tile max.  The barrier also orders
-                // the partner's S loads before this thread's P stores over them.
-                sh.xmax[j & 1][hc][row] = fmaxf(tm[0], tm[1]);
-                tc_fence_before();
-                named_bar_sync(pair_bar, 64);
-                tc_fence_after();
                 if (!live) continue;
-                const float tmax = fmaxf(sh.xmax[j & 1][0][row], sh.xmax[j & 1][1][row]);
+                const float tmax = fmaxf(tm[0], tm[1]);  // this half's tile max
                 if (j == 0) {
                     m_ref = tmax;
                 } else if (__any_sync(0xffffffffu, tmax > m_ref + kRescaleThreshold)) {
-                    // decided per warp, identically in both warps of the pair (same rows,
-                    // same maxima); rows that keep their reference get alpha = 1.  O must
-                    // hold PV_{j-1}.
+                    // decided per warp; rows that keep their reference get alpha = 1.  O_h
+                    // must hold PV_{j-1}.
                     if (!wwait(&sh.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) continue;
                     tc_fence_after();
                     const float m_new = tmax > m_ref + kRescaleThreshold ? tmax : m_ref;
                     const float alpha = m_new == m_ref ? 1.f : fast_ex2(m_ref - m_new);  // (m_ref may be -inf)
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
+                    for (int c = 0; c < 4; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(trow + 256u + (uint32_t)(64 * hc + 32 * c), o);
+                        tmem_ld32(trow + o_col + (uint32_t)(32 * c), o);
                         tmem_ld_wait();
                         tmem_ld_dep(o);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(bits_f(o[e]) * alpha);
-                        tmem_st32(trow + 256u + (uint32_t)(64 * hc + 32 * c), o);
+                        tmem_st32(trow + o_col + (uint32_t)(32 * c), o);
                     }
                     tmem_st_wait();
                     l2.x *= alpha;
                     l2.y *= alpha;
                     m_ref = m_new;
                 }
-                // P (bf16 pairs) over the first 64 columns of buffer b: this half's 64
-                // keys are packed columns [32 hc, 32 hc + 32)
+                // P (bf16 pairs) over the first 32 of this half's own 64 columns of buffer b
+                // (S values this thread has already read)
                 uint32_t pk[32];
                 // a row that has met only masked keys so far (the guest rows of a packed item
                 // can) keeps m_ref = -inf: its P is 0, and the first real maximum rescales O by 0
@@ -479,48 +486,64 @@ __global__ void __launch_bounds__(352, 1)
                         __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
                         pk[16 * c + e] = *reinterpret_cast<uint32_t*>(&h);
                     }
-                tmem_st32(trow + (uint32_t)(b * 128 + 32 * hc), pk);
+                tmem_st32(trow + (uint32_t)(b * 128 + 64 * hc), pk);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&sh.p_full[b]);
+                mbar_arrive(&sh.p_full[hc][b]);
             }
-            // epilogue: O / l, original token order; each thread writes its 64 columns.
-            // The partner overwrites xl only after its next item's first pair barrier,
-            // which this thread reaches after reading xl.
-            sh.xl[hc][row] = l2.x + l2.y;
+            // epilogue: the two halves meet once per item.  O = (O_0 a_0 + O_1 a_1) / l with
+            // a_h = 2^(m_h - M), M = max(m_0, m_1), l = l_0 a_0 + l_1 a_1; original token order;
+            // each thread writes its 64 columns.  The shared slots alternate by item, so the
+            // partner overwrites them only after the next item's barrier, which this thread
+            // reaches after reading them.
+            sh.xm[I & 1][hc][row] = m_ref;
+            sh.xl[I & 1][hc][row] = l2.x + l2.y;
             named_bar_sync(pair_bar, 64);
-            const float lt = sh.xl[0][row] + sh.xl[1][row];
+            const float m0 = sh.xm[I & 1][0][row], m1 = sh.xm[I & 1][1][row];
+            const float M = fmaxf(m0, m1);
+            const float a0 = m0 == __int_as_float(0xff800000) ? 0.f : fast_ex2(m0 - M);
+            const float a1 = m1 == __int_as_float(0xff800000) ? 0.f : fast_ex2(m1 - M);
+            const float lt = sh.xl[I & 1][0][row] * a0 + sh.xl[I & 1][1][row] * a1;
             const int gl = G + nkt - 1;
             G += nkt;
+            ++I;
             if (!wwait(&sh.pv_done[gl & 1], (gl >> 1) & 1)) continue;
             tc_fence_after();
-            uint32_t o[2][32];
-            tmem_ld32(trow + 256u + (uint32_t)(64 * hc), o[0]);
-            tmem_ld32(trow + 256u + (uint32_t)(64 * hc + 32), o[1]);
-            tmem_ld_wait();
-            tmem_ld_dep(o[0]);
-            tmem_ld_dep(o[1]);
-            tc_fence_before();
-            mbar_arrive(&sh.o_empty);
             const int grow = row - wi.rows;  // row of the guest part, if any
-            if (row < wi.rows || grow < wi.g_rows) {
-                const float inv = lt > 0.f ? 1.f / lt : 0.f;
-                const int tok = row < wi.rows ? q_perm[(size_t)wi.bh * N + wi.q_start + row]
-                                              : q_perm[(size_t)wi.bh * N + wi.g_start + grow];
-                uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)wi.bh * N + tok) * 128 + 64 * hc);
+            const bool wr = row < wi.rows || grow < wi.g_rows;
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            const int tok = !wr ? 0
+                                : (row < wi.rows ? q_perm[(size_t)wi.bh * N + wi.q_start + row]
+                                                 : q_perm[(size_t)wi.bh * N + wi.g_start + grow]);
+            uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)wi.bh * N + tok) * 128 + 64 * hc);
+            const float s0 = a0 * inv, s1 = a1 * inv;
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < 2; ++c) {
+                uint32_t o0[32], o1[32];
+                tmem_ld32(trow + 256u + (uint32_t)(64 * hc + 32 * c), o0);
+                tmem_ld32(trow + 384u + (uint32_t)(64 * hc + 32 * c), o1);
+                tmem_ld_wait();
+                tmem_ld_dep(o0);
+                tmem_ld_dep(o1);
+                if (c == 1) {
+                    tc_fence_before();
+                    mbar_arrive(&sh.o_empty);
+                }
+                if (wr) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint32_t w4[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            __nv_bfloat162 h = __floats2bfloat162_rn(bits_f(o[c][8 * q + 2 * e]) * inv,
-                                                                     bits_f(o[c][8 * q + 2 * e + 1]) * inv);
+                            const int k = 8 * q + 2 * e;
+                            __nv_bfloat162 h =
+                                __floats2bfloat162_rn(fmaf(bits_f(o0[k]), s0, bits_f(o1[k]) * s1),
+                                                      fmaf(bits_f(o0[k + 1]), s0, bits_f(o1[k + 1]) * s1));
                             w4[e] = *reinterpret_cast<uint32_t*>(&h);
                         }
                         dst[c * 4 + q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
+                }
             }
         }
     }
