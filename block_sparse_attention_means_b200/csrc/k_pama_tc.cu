@@ -48,6 +48,11 @@ struct PtSmem {
 };
 
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
 
 // Sum of v[0..31] over the 32 lanes of the warp: lane j returns the total of
 // element j (31 shuffles, recursive halving).
@@ -198,6 +203,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t trow = tmem + ((uint32_t)(32 * quad) << 16);
         const int et = threadIdx.x - 64;  // 0..255
         const float NEG = __int_as_float(0xff800000);
+        const float2 sl2e2 = make_float2(sl2e, sl2e);
         bool failed = false;
         int G = 0;
         auto wait_acc = [&](int b, int g) {
@@ -252,10 +258,14 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                         for (int q = 0; q < 2; ++q)
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                const float v = fmaf(__uint_as_float(a[q][e]), sl2e, live[c * PT_CH + 64 * h + 32 * q + e]);
-                                x[q][e] = v;
-                                cm = fmaxf(cm, v);
+                            for (int e = 0; e < 32; e += 2) {
+                                // packed float32 pairs: the same per-element rounding as fmaf
+                                const float2 lv = *reinterpret_cast<const float2*>(live + c * PT_CH + 64 * h + 32 * q + e);
+                                const float2 v = __ffma2_rn(make_float2(__uint_as_float(a[q][e]), __uint_as_float(a[q][e + 1])),
+                                                            sl2e2, lv);
+                                x[q][e] = v.x;
+                                x[q][e + 1] = v.y;
+                                cm = fmax3f(cm, v.x, v.y);
                             }
                         const float mn = fmaxf(m, cm);
                         if (mn != NEG) {
@@ -265,10 +275,17 @@ __global__ void __launch_bounds__(320, 1)
                             }
 #pragma unroll
                             for (int k = 0; k < 8; ++k) part[k] = 0.f;
+                            const float2 nm2 = make_float2(-m, -m);
 #pragma unroll
                             for (int q = 0; q < 2; ++q)
 #pragma unroll
-                                for (int e = 0; e < 32; ++e) part[e & 7] += fast_exp2(x[q][e] - m);
+                                for (int e = 0; e < 32; e += 2) {
+                                    const float2 d = __fadd2_rn(make_float2(x[q][e], x[q][e + 1]), nm2);
+                                    const float2 pp = __fadd2_rn(make_float2(part[e & 7], part[(e + 1) & 7]),
+                                                                 make_float2(fast_exp2(d.x), fast_exp2(d.y)));
+                                    part[e & 7] = pp.x;
+                                    part[(e + 1) & 7] = pp.y;
+                                }
                             l += (double)(((part[0] + part[1]) + (part[2] + part[3])) +
                                           ((part[4] + part[5]) + (part[6] + part[7])));
                         }
@@ -283,6 +300,7 @@ __global__ void __launch_bounds__(320, 1)
                 const double L = (m0 == NEG ? 0.0 : sh.xl[0][row] * (double)fast_exp2(m0 - M)) +
                                  (m1 == NEG ? 0.0 : sh.xl[1][row] * (double)fast_exp2(m1 - M));
                 const float inv = valid && L > 0.0 ? (float)(1.0 / L) : 0.f;
+                const float2 inv2 = make_float2(inv, inv), nM2 = make_float2(-M, -M);
                 named_bar_sync(2 + quad, 64);  // both read before the next tile overwrites
                 // pass 2: normalised probabilities, column sums over the warp's 32 rows
                 for (int c = 0; c < nch; ++c, ++G) {
@@ -302,10 +320,16 @@ __global__ void __launch_bounds__(320, 1)
                         }
                         float v[32];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const float pe =
-                                fast_exp2(fmaf(__uint_as_float(a[e]), sl2e, live[c * PT_CH + 32 * q + e]) - M) * inv;
-                            v[e] = valid ? pe : 0.f;  // rows past the cluster add nothing
+                        for (int e = 0; e < 32; e += 2) {
+                            // packed float32 pairs: the same per-element roundings as fmaf, - and *
+                            const float2 lv = *reinterpret_cast<const float2*>(live + c * PT_CH + 32 * q + e);
+                            const float2 xx =
+                                __fadd2_rn(__ffma2_rn(make_float2(__uint_as_float(a[e]), __uint_as_float(a[e + 1])),
+                                                      sl2e2, lv),
+                                           nM2);
+                            const float2 pe = __fmul2_rn(make_float2(fast_exp2(xx.x), fast_exp2(xx.y)), inv2);
+                            v[e] = valid ? pe.x : 0.f;  // rows past the cluster add nothing
+                            v[e + 1] = valid ? pe.y : 0.f;
                         }
                         cs[32 * q + lane] += transpose_sum32(v, lane);
                     }
