@@ -601,7 +601,13 @@ __global__ void k_sparse_attn_simt(const T* __restrict__ Q, const T* __restrict_
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             int j = lane + 32 * u;
-            if (j < D) reinterpret_cast<float*>(O)[row * D + j] = l > 0.f ? o[u] / l : 0.f;
+            if (j < D) {
+                const float out = l > 0.f ? o[u] / l : 0.f;
+                if (sizeof(T) == 2)
+                    reinterpret_cast<uint16_t*>(O)[row * D + j] = __bfloat16_as_ushort(__float2bfloat16_rn(out));
+                else
+                    reinterpret_cast<float*>(O)[row * D + j] = out;
+            }
         }
     }
 }
@@ -610,15 +616,19 @@ int launch_sparse_attn_simt(const void* Q, const void* K, const void* V, int dty
                             int NK, const int32_t* q_labels, const int32_t* k_perm, const int32_t* k_off,
                             const int32_t* kept_ptr, const int32_t* kept_idx, const float* bweight, void* O,
                             cudaStream_t st) {
-    if (dtype != PARK_F32 || D > 128) return PARK_ERR_UNSUPPORTED;
+    if (D > 128) return PARK_ERR_UNSUPPORTED;
     size_t rows = (size_t)BH * N;
     int blocks = (int)((rows * 32 + 255) / 256);
     ::park::prof_begin(st);
     if (blocks > 148 * 64) blocks = 148 * 64;
-    k_sparse_attn_simt<float><<<blocks, 256, 0, st>>>((const float*)Q, (const float*)K, (const float*)V, N, D, NQ, NK,
-                                                      q_labels, k_perm, k_off, kept_ptr, kept_idx, bweight, (float*)O,
-                                                      rows,
-                                                      1.0f / sqrtf((float)D));
+    if (dtype == PARK_BF16)
+        k_sparse_attn_simt<bf16_t><<<blocks, 256, 0, st>>>((const bf16_t*)Q, (const bf16_t*)K, (const bf16_t*)V, N, D,
+                                                           NQ, NK, q_labels, k_perm, k_off, kept_ptr, kept_idx, bweight,
+                                                           (bf16_t*)O, rows, 1.0f / sqrtf((float)D));
+    else
+        k_sparse_attn_simt<float><<<blocks, 256, 0, st>>>((const float*)Q, (const float*)K, (const float*)V, N, D, NQ,
+                                                          NK, q_labels, k_perm, k_off, kept_ptr, kept_idx, bweight,
+                                                          (float*)O, rows, 1.0f / sqrtf((float)D));
     PARK_TRY_LAUNCH("k_sparse_attn_simt", st);
     return PARK_OK;
 }

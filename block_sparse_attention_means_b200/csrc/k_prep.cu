@@ -302,6 +302,8 @@ int launch_metric(const void* Q, int dtype, int BH, int N, int D, double* part, 
         k_metric_partial_mma<bf16_t><<<g1, 256, 0, st>>>((const bf16_t*)Q, N, rpc, part);
     else if (D == 128)
         k_metric_partial_mma<float><<<g1, 256, 0, st>>>((const float*)Q, N, rpc, part);
+    else if (dtype == PARK_BF16)
+        k_metric_partial<bf16_t><<<g1, 272, 0, st>>>((const bf16_t*)Q, N, D, rpc, part);
     else
         k_metric_partial<float><<<g1, 272, 0, st>>>((const float*)Q, N, D, rpc, part);
     PARK_TRY_LAUNCH("k_metric_partial", st);

@@ -72,6 +72,9 @@ struct Dims {
     int T, Hg, W, nvideo;  // video grid; nvideo = T Hg W tokens precede the text tokens
 };
 
+// bf16 with D = 128: the tcgen05 kernels (assign, PAMA, attention)
+inline bool tensor_path(const Dims& d) { return d.dtype == PARK_BF16 && d.D == 128; }
+
 int check_shape(const park_shape* s, int NQ, int NK, Dims* d) {
     if (!s) return PARK_ERR_INVALID_ARG;
     if (s->B < 1 || s->H < 1 || s->T < 0 || s->Hg < 0 || s->W < 0 || s->n_text < 0 || s->D < 1)
@@ -83,13 +86,10 @@ int check_shape(const park_shape* s, int NQ, int NK, Dims* d) {
     if (BH * N >= (1ll << 31) || BH > 65535) return PARK_ERR_UNSUPPORTED;
     if (NQ < 1 || NK < 1 || NQ > N || NK > N) return PARK_ERR_INVALID_ARG;
     if (NK > 4096 || NQ > 65536) return PARK_ERR_UNSUPPORTED;
-    if (s->dtype == PARK_BF16) {
-        if (s->D != 128) return PARK_ERR_UNSUPPORTED;
-    } else if (s->dtype == PARK_F32) {
-        if (s->D % 32 != 0 || s->D > 128) return PARK_ERR_UNSUPPORTED;
-    } else {
-        return PARK_ERR_INVALID_ARG;
-    }
+    // bf16 with D = 128 takes the tensor-core kernels; bf16 with another D, and float32,
+    // take the float64 and SIMT kernels (the same certified results, slower)
+    if (s->dtype != PARK_BF16 && s->dtype != PARK_F32) return PARK_ERR_INVALID_ARG;
+    if (s->D % 32 != 0 || s->D > 128) return PARK_ERR_UNSUPPORTED;
     d->B = s->B;
     d->H = s->H;
     d->N = (int)N;
@@ -164,7 +164,7 @@ RetrievalWs plan_retrieval(const Dims& d, int NQ, int NK) {
     w.mX = c.take(NQ <= kMergeMaxNQ ? BH * NQ * NQ * 4 : 0);
     w.mH = c.take(2 * BH * 4);       // done, nb
     w.txt = c.take(text_scratch_bytes(d.BH, d.N - d.nvideo, (int)Km));
-    w.qg = c.take(d.dtype == PARK_BF16 ? BH * N * D * 2 : 0);  // Q in query-cluster order, for PAMA
+    w.qg = c.take(tensor_path(d) ? BH * N * D * 2 : 0);  // Q in query-cluster order, for PAMA
     w.total = c.off;
     return w;
 }
@@ -188,7 +188,7 @@ AttnWs plan_attn(const Dims& d, int NQ, int NK) {
     size_t rowbytes = D * d.elt;
     w.Npad = padded_rows(d, NK);
     w.item_cap = BH * ((N + kAttnTileTc - 1) / kAttnTileTc + (size_t)NQ);
-    if (d.dtype == PARK_BF16) {
+    if (tensor_path(d)) {
         w.Qimg = c.take(w.item_cap * kAttnTileTc * rowbytes);
         w.Kp = c.take(BH * (size_t)w.Npad * rowbytes);
         w.Vp = c.take(BH * (size_t)w.Npad * rowbytes);
@@ -291,7 +291,7 @@ struct Side {
 
 int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, void* ws, int64_t* counters,
                int num_sms, cudaStream_t st) {
-    const bool bf16 = d.dtype == PARK_BF16;
+    const bool tc = tensor_path(d);
     const int BH = d.BH, N = d.N, D = d.D, K = s.K;
     const int nchunks = (N + kSortChunk - 1) / kSortChunk;
     CentroidOps ops;
@@ -302,7 +302,7 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
     ops.wmax = at<float>(ws, w.wmax);
     ops.bmax = at<float>(ws, w.bmax);
     if (s.M) {
-        ops.w = bf16 ? at<uint16_t>(ws, w.wop) : nullptr;
+        ops.w = tc ? at<uint16_t>(ws, w.wop) : nullptr;
         ops.kw = 2 * D;
     } else {
         ops.w = static_cast<const uint16_t*>(s.C);
@@ -334,8 +334,7 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
     // labels start valid (cluster 0), so that a kernel that gave up on a bounded
     // wait (status PARK_ERR_TIMEOUT) leaves nothing out of range for the later steps
     PARK_CHECK(memset_async(s.labels, (size_t)BH * N * 4, st));
-    // (bf16 with D = 128: the input check has written them)
-    if (bf16 && D != 128) PARK_CHECK(launch_row_norms(s.X, d.dtype, BH, N, D, s.xnorm, st));
+    // (the row norms of the tensor-core assign bound come from the input check)
     if (!s.warm) PARK_CHECK(launch_strided_init(s.X, d.dtype, BH, N, D, K, s.C, st));
     const float gamma = gamma_for(ops.kw, s.M != nullptr);
     for (int it = 0; it < iters; ++it) {
@@ -343,7 +342,7 @@ int run_kmeans(const Dims& d, const Side& s, int iters, const RetrievalWs& w, vo
         PARK_CHECK(memset_async(ops.bmax, (size_t)BH * 4, st));
         PARK_CHECK(memset_async(lists.counts, (size_t)BH * 4, st));
         PARK_CHECK(launch_centroid_prep(s.C, d.dtype, BH, K, D, s.M, ops, st));
-        if (bf16) {
+        if (tc) {
             PARK_CHECK(launch_assign_tc(s.X, BH, N, K, ops, s.xnorm, gamma, s.labels, lists, s.status, num_sms, st));
             PARK_CHECK(launch_recheck(s.X, d.dtype, BH, N, D, K, s.C, ops.w64, ops.bias64, s.labels, lists, 0,
                                       num_sms, counters, s.cnt_slot, st));
@@ -462,7 +461,7 @@ int retrieve_impl(const void* Q, const void* K, const Dims& d, int NQ, int NK, f
                                    out->k_offsets, p, select, size_prior, sip_u, bw, nullptr, nullptr, 1, num_sms,
                                    at<int32_t>(ws, w.pcnt) + 4, at<double>(ws, w.f64z), out->importance,
                                    out->importance_bound, out->mask, kcnt, out->counters, st, 1));
-    } else if (d.dtype == PARK_BF16) {
+    } else if (tensor_path(d)) {
         // max ||c_m|| over the final key centroids, for the PAMA bound
         CentroidOps ops{nullptr, D, at<float>(ws, w.b32), (int)align_up((size_t)(NQ > NK ? NQ : NK), 128),
                         at<double>(ws, w.b64), nullptr, at<float>(ws, w.wmax), at<float>(ws, w.bmax)};
@@ -508,14 +507,14 @@ int attn_impl(const void* Q, const void* K, const void* V, const Dims& d, int NQ
               void* O, void* ws, cudaStream_t st) {
     const AttnWs w = plan_attn(d, NQ, NK);
     const int BH = d.BH, N = d.N, D = d.D;
-    const bool bf16 = d.dtype == PARK_BF16;
+    const bool tc = tensor_path(d);
     PARK_CHECK(launch_input_check(V, (size_t)BH * N * D, d.dtype, r->status, nullptr, (size_t)N * D, nullptr, D,
                                   nullptr, st));
     PARK_CHECK(memset_async(r->counters + PARK_CNT_KEPT_PAIRS, 3 * sizeof(int64_t), st));
     int32_t* icnt = at<int32_t>(ws, w.icnt);
     PARK_CHECK(memset_async(icnt, 16 * 4, st));
     const float* bw = (r->flags & PARK_FLAG_SIP) ? r->block_weight : nullptr;  // SIP weights
-    if (!bf16) {
+    if (!tc) {
         PARK_CHECK(launch_attn_schedule(BH, NQ, NK, r->q_offsets, r->k_offsets, r->kept_ptr, r->kept_idx,
                                         at<int32_t>(ws, w.kvpre), at<int32_t>(ws, w.kvlen), at<WorkItem>(ws, w.items),
                                         icnt, r->counters, kAttnTile, 0, nullptr, 0, nullptr, nullptr, nullptr, st));

@@ -3,7 +3,8 @@ every step of the computation runs in the library's CUDA kernels.
 
 The names follow the C ABI: ``workspace_size``, ``retrieve``, ``sparse_attn``,
 ``layer``.  Tensors are [B, H, N, D], contiguous, on one CUDA device, in
-torch.bfloat16 (D = 128) or torch.float32.
+torch.bfloat16 or torch.float32 with D a multiple of 32 up to 128 (bf16 with
+D = 128 runs the tensor-core kernels).
 """
 from __future__ import annotations
 

@@ -36,8 +36,10 @@
  *     allocates, frees or synchronises; all work is enqueued on `stream` (a
  *     cudaStream_t passed as void*, NULL = legacy default stream).
  *   - Layout: Q, K, V, O are [B, H, N, D] contiguous, N = T*Hg*W + n_text
- *     (video tokens in (t, y, w) order, text tokens last).  dtype PARK_BF16
- *     requires D == 128; PARK_F32 requires D % 32 == 0 and D <= 128.
+ *     (video tokens in (t, y, w) order, text tokens last).  Both dtypes
+ *     require D % 32 == 0 and D <= 128; PARK_BF16 with D == 128 runs the
+ *     tensor-core kernels, every other shape the float64 / SIMT kernels (the
+ *     same results, certified the same way, slower).
  *   - Range precondition: every input element is 0 or has 2^-40 <= |x| < 2^40
  *     (and is finite).  Inside it the centroid sums are exact (128-bit fixed
  *     point at 2^-64), whatever the order of the terms.

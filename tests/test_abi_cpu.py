@@ -57,7 +57,9 @@ def test_workspace_size_and_shape_validation():
     # streamed PAMA: workspace does not grow with N * NK (PARK Appendix Table 6)
     n2 = P.workspace_size(P.Shape(1, 24, 66, 45, 80, 256, 128), 930, 930)
     assert n2 < 2.2 * n
-    bad = [(P.Shape(1, 8, 8, 16, 16, 0, 64), 32, 32, _lib.PARK_ERR_UNSUPPORTED),    # bf16 needs D = 128
+    assert P.workspace_size(P.Shape(1, 8, 8, 16, 16, 0, 64), 32, 32) > 0         # bf16 with D = 64
+    bad = [(P.Shape(1, 8, 8, 16, 16, 0, 48), 32, 32, _lib.PARK_ERR_UNSUPPORTED),    # D % 32 != 0
+           (P.Shape(1, 8, 8, 16, 16, 0, 160), 32, 32, _lib.PARK_ERR_UNSUPPORTED),   # D > 128
            (P.Shape(1, 8, 8, 32, 32, 0, 128, dtype=__import__("torch").float32), 32, 5000,
             _lib.PARK_ERR_UNSUPPORTED),                                              # NK > 4096
            (P.Shape(1, 8, 8, 16, 16, 0, 128), 0, 32, _lib.PARK_ERR_INVALID_ARG),

@@ -202,9 +202,11 @@ def test_all_blocks_kept_is_dense(park):
 
 RAGGED = LayerConfig("ragged", 2, 3, 3, 7, 11, 5, 128, "bf16", 9, 13, 4, 0.85, True, "normal")
 RAGGED_F32 = LayerConfig("ragged32", 2, 2, 3, 5, 7, 3, 64, "f32", 6, 9, 3, 0.8, False, "positional")
+# bf16 with D = 64: the float64 / SIMT kernels instead of the tensor-core ones
+RAGGED_D64 = LayerConfig("ragged64", 2, 3, 3, 7, 11, 5, 64, "bf16", 9, 13, 4, 0.85, True, "normal")
 
 
-@pytest.mark.parametrize("cfg", [RAGGED, RAGGED_F32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("cfg", [RAGGED, RAGGED_F32, RAGGED_D64], ids=["bf16", "f32", "bf16_d64"])
 def test_ragged_batch_shapes(park, cfg):
     """B = 2, ragged N (not a multiple of any tile), text tokens."""
     Q, K, V = gen_layer(cfg, seed=3)
