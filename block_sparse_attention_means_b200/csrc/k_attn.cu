@@ -143,8 +143,9 @@ int launch_attn_schedule(int BH, int NQ, int NK, const int32_t* q_off, const int
 // key tiles, T(L) = ceil(L / 16) for L kept 8-row groups, the shared groups
 // counted from the bit planes as in the merge.  k_pack_cand: one CTA per
 // (cluster, head) lists a guest's kPackCand best hosts (gain, then lowest h);
-// k_pack_select: one thread per head takes the guests in cluster order, each
-// joining its best listed host not yet taken.
+// k_pack_select: one warp per head takes the guests in cluster order, each
+// joining its best listed host not yet taken (lane k holds the guest's k-th
+// listed host; a ballot finds the first one free, before the end of the list).
 constexpr int kPackCand = kPackCandidates;
 
 __global__ __launch_bounds__(256) void k_pack_cand(int NQ, int Wd, MergeWs m, int2* __restrict__ cand) {
@@ -209,28 +210,43 @@ __global__ __launch_bounds__(256) void k_pack_cand(int NQ, int Wd, MergeWs m, in
 
 __global__ void k_pack_select(int NQ, const MergeWs m, const int2* __restrict__ cand, int32_t* __restrict__ pack_host,
                               int32_t* __restrict__ pack_guest) {
-    extern __shared__ uint32_t taken[];  // [ceil(NQ / 32)]
-    const int bh = blockIdx.x, tid = threadIdx.x;
+    static_assert(kPackCand == 32, "one listed host per lane");
+    extern __shared__ uint32_t taken[];                    // [ceil(NQ / 32)] hosts already taken
+    uint8_t* guest = reinterpret_cast<uint8_t*>(taken + (NQ + 31) / 32);  // [NQ] cluster spills over a tile
+    const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
     const size_t hb = (size_t)bh * NQ;
     for (int r = tid; r < NQ; r += blockDim.x) {
         pack_host[hb + r] = -1;
         pack_guest[hb + r] = -1;
+        guest[r] = m.n[hb + r] > 128 ? 1 : 0;
     }
     for (int i = tid; i < (NQ + 31) / 32; i += blockDim.x) taken[i] = 0u;
     __syncthreads();
-    if (tid != 0) return;
-    for (int g = 0; g < NQ; ++g) {
-        if (m.n[hb + g] <= 128) continue;
-        const int2* c = cand + (hb + g) * kPackCand;
-        for (int k = 0; k < kPackCand; ++k) {
-            const int2 e = c[k];
-            if (e.y < 0 || e.x <= 0) break;
-            if ((taken[e.y >> 5] >> (e.y & 31)) & 1u) continue;
-            taken[e.y >> 5] |= 1u << (e.y & 31);
-            pack_host[hb + g] = e.y;
-            pack_guest[hb + e.y] = g;
-            break;
+    if (tid >= 32) return;
+    int g = 0;
+    while (g < NQ && !guest[g]) ++g;
+    int2 e = g < NQ ? cand[(hb + g) * kPackCand + lane] : make_int2(0, -1);
+    while (g < NQ) {
+        // the next guest's list is loaded while this one is decided
+        int gn = g + 1;
+        while (gn < NQ && !guest[gn]) ++gn;
+        const int2 en = gn < NQ ? cand[(hb + gn) * kPackCand + lane] : make_int2(0, -1);
+        const unsigned end = __ballot_sync(0xffffffffu, e.y < 0 || e.x <= 0);
+        const int first_end = end ? __ffs(end) - 1 : 32;
+        const int hy = e.y < 0 ? 0 : e.y;  // (entries past the end of the list are not read as hosts)
+        const bool free_host = lane < first_end && !((taken[hy >> 5] >> (hy & 31)) & 1u);
+        const unsigned ok = __ballot_sync(0xffffffffu, free_host);
+        if (ok) {
+            const int h = __shfl_sync(0xffffffffu, e.y, __ffs(ok) - 1);
+            if (lane == 0) {
+                taken[h >> 5] |= 1u << (h & 31);
+                pack_host[hb + g] = h;
+                pack_guest[hb + h] = g;
+            }
         }
+        __syncwarp();
+        g = gn;
+        e = en;
     }
 }
 
@@ -247,7 +263,7 @@ int launch_pack_pairs(int BH, int NQ, int NK, const uint8_t* mask, const int32_t
     k_pack_cand<<<dim3(NQ, BH), 256, sm, st>>>(NQ, Wd, m, cand);
     PARK_TRY_LAUNCH("k_pack_cand", st);
     ::park::prof_begin(st);
-    k_pack_select<<<BH, 256, (size_t)((NQ + 31) / 32) * 4, st>>>(NQ, m, cand, pack_host, pack_guest);
+    k_pack_select<<<BH, 256, (size_t)((NQ + 31) / 32) * 4 + (size_t)NQ, st>>>(NQ, m, cand, pack_host, pack_guest);
     PARK_TRY_LAUNCH("k_pack_select", st);
     return PARK_OK;
 }

@@ -42,19 +42,27 @@ __global__ void k_input_check(const uint4* __restrict__ x, size_t n16, int32_t* 
             if (in && (lane & 15) == 0) xnorm[i >> 4] = round_up_f(__double2float_ru(sqrt(ss)));
         }
         bool narrow = true, tiny = false;
+        if (BYTES == 2) {
+            // both bf16 halves of a word at once: with x the two 15-bit magnitudes, x + c
+            // sets bit 15 of a half exactly when its magnitude is >= 0x8000 - c (no carry
+            // reaches the other half): nonzero (>= 1), exponent >= 87 (0x2B80), >= 167
+            // (0x5380: beyond the range, or inf / NaN), >= 143 (0x4780: |x| >= 2^16) and
+            // >= 107 (0x3580: |x| >= 2^-20)
+            uint32_t a_bad = 0, a_wide = 0, a_tiny = 0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            if (BYTES == 2) {
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t x = w[q] & 0x7FFF7FFFu;
+                const uint32_t nz = x + 0x7FFF7FFFu;
+                a_bad |= nz & (~(x + 0x54805480u) | (x + 0x2C802C80u));
+                a_wide |= x + 0x38803880u;
+                a_tiny |= nz & ~(x + 0x4A804A80u);
+            }
+            bad |= (a_bad & 0x80008000u) != 0u;
+            narrow = (a_wide & 0x80008000u) == 0u;
+            tiny = (a_tiny & 0x80008000u) != 0u;
+        } else {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t b = (w[q] >> (16 * h)) & 0xFFFFu;
-                    uint32_t mag = b & 0x7FFFu;
-                    int e = (b >> 7) & 0xFF;
-                    bad |= !in_range_exp(e, mag);
-                    narrow &= e <= 142;
-                    tiny |= mag != 0u && e < 107;
-                }
-            } else {
+            for (int q = 0; q < 4; ++q) {
                 uint32_t mag = w[q] & 0x7FFFFFFFu;
                 int e = (w[q] >> 23) & 0xFF;
                 bad |= !in_range_exp(e, mag);
