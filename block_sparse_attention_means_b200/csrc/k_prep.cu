@@ -401,18 +401,19 @@ __global__ void k_centroid_prep(const T* __restrict__ C, int K, int D, float* __
     }
 }
 
-// QRKC operands for 64 centroids per CTA: M (symmetric, float64) is staged once
-// in shared memory, thread (a, half) forms w_a = sum_b M[b][a] c_b for 32
-// centroids (row b of M: conflict-free; the centroids' pairs c_b, c_b+1 as one
-// 16-byte broadcast), then per centroid bias = c . w and ||w||^2 are reduced
-// over the 128 threads of its half in a fixed order.
+// QRKC operands for 64 centroids per CTA: M (symmetric, float64) and the
+// centroids (transposed: Cs[b][c]) are staged once in shared memory; thread t
+// owns columns 4 (t % 32) .. + 3 and centroids 8 (t / 32) .. + 7 and forms
+// w_a = sum_b M[b][a] c_b for them, summing over b in order (four M values and
+// eight centroid values per step: 32 FMAs per 6 shared loads).  A warp holds whole
+// rows w of its eight centroids, so bias = c . w and ||w||^2 are reduced within
+// the warp in a fixed order.
 // w and the bias are taken for 2^-e M, e the binary exponent of the head's
 // largest diagonal entry (|M_ab| <= max_a M_aa), so that the float32 scores stay
 // far from overflow over the whole input range (|x| < 2^40 gives M up to 2^80).
 // A power-of-two scale is exact in float64 and multiplies every score of the
 // head by the same factor, so it changes no argmin.
-constexpr int kPrepPerThread = 32;
-constexpr int kPrepCents = 2 * kPrepPerThread;
+constexpr int kPrepCents = 64;
 
 template <typename T>
 __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restrict__ C, int K, int D,
@@ -423,11 +424,11 @@ __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restric
                                                               float* __restrict__ bmax) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     double* Ms = reinterpret_cast<double*>(smem_raw);  // [D][D]
-    double* Cs = Ms + D * D;                          // [kPrepCents][D]
-    __shared__ double red[kPrepCents][4][2];
+    double* Cs = Ms + D * D;                          // [D][kPrepCents]: Cs[b][c]
     __shared__ double s_scale;
     const int bh = blockIdx.y, k0 = blockIdx.x * kPrepCents, t = threadIdx.x;
-    const int a = t & 127, half = t >> 7, lane = t & 31, wq = (t >> 5) & 3;
+    const int lane = t & 31, cb = t >> 5;  // column block (4 columns), centroid block (8 centroids)
+    const int a0 = 4 * lane, c0 = 8 * cb;
     const double2* M2 = reinterpret_cast<const double2*>(Mall + (size_t)bh * D * D);
     double2* Ms2 = reinterpret_cast<double2*>(Ms);
     const int n2 = D * D / 2;
@@ -442,7 +443,7 @@ __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restric
     }
     for (int i = t; i < kPrepCents * D; i += blockDim.x) {
         const int c = i / D, j = i - c * D, k = k0 + c;
-        Cs[i] = k < K ? Elem<T>::to_double(C + ((size_t)bh * K + k) * D, j) : 0.0;
+        Cs[j * kPrepCents + c] = k < K ? Elem<T>::to_double(C + ((size_t)bh * K + k) * D, j) : 0.0;
     }
     if (blockIdx.x == 0)  // columns past K read +inf, so a score GEMM over whole 128-column chunks never picks them
         for (int j = K + t; j < ((K + 127) & ~127); j += blockDim.x)
@@ -456,52 +457,71 @@ __global__ __launch_bounds__(256) void k_centroid_prep_metric(const T* __restric
     }
     __syncthreads();
     const double scale = s_scale;
-    double w[kPrepPerThread];
+    const bool act = a0 < D;  // D is a multiple of 32: a thread's four columns are all in or all out
+    double w[8][4];
 #pragma unroll
-    for (int c = 0; c < kPrepPerThread; ++c) w[c] = 0.0;
-    if (a < D) {
-        const double* cbase = Cs + half * kPrepPerThread * D;
-        for (int b = 0; b < D; b += 2) {  // D is even
-            const double m0 = Ms[b * D + a], m1 = Ms[(b + 1) * D + a];
+    for (int c = 0; c < 8; ++c)
 #pragma unroll
-            for (int c = 0; c < kPrepPerThread; ++c) {
-                const double2 cv = *reinterpret_cast<const double2*>(cbase + c * D + b);
-                w[c] = __fma_rn(m0, cv.x, w[c]);
-                w[c] = __fma_rn(m1, cv.y, w[c]);
+        for (int j = 0; j < 4; ++j) w[c][j] = 0.0;
+    if (act) {
+        for (int b = 0; b < D; ++b) {
+            const double2 m01 = *reinterpret_cast<const double2*>(Ms + b * D + a0);
+            const double2 m23 = *reinterpret_cast<const double2*>(Ms + b * D + a0 + 2);
+            const double mv[4] = {m01.x, m01.y, m23.x, m23.y};
+#pragma unroll
+            for (int c2 = 0; c2 < 4; ++c2) {
+                const double2 cv = *reinterpret_cast<const double2*>(Cs + b * kPrepCents + c0 + 2 * c2);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    w[2 * c2][j] = __fma_rn(mv[j], cv.x, w[2 * c2][j]);
+                    w[2 * c2 + 1][j] = __fma_rn(mv[j], cv.y, w[2 * c2 + 1][j]);
+                }
             }
         }
     }
 #pragma unroll
-    for (int c = 0; c < kPrepPerThread; ++c) w[c] *= scale;  // exact
+    for (int c = 0; c < 8; ++c) {
+        const int k = k0 + c0 + c;
+        double pb = 0.0, pn = 0.0;
 #pragma unroll
-    for (int c = 0; c < kPrepPerThread; ++c) {
-        const int cc = half * kPrepPerThread + c, k = k0 + cc;
-        const double ca = a < D ? Cs[cc * D + a] : 0.0;
-        if (a < D && k < K) {
-            w64[((size_t)bh * K + k) * D + a] = w[c];
+        for (int j = 0; j < 4; ++j) {
+            w[c][j] *= scale;  // exact
+            if (act) {
+                pb = __fma_rn(Cs[(a0 + j) * kPrepCents + c0 + c], w[c][j], pb);
+                pn = __fma_rn(w[c][j], w[c][j], pn);
+            }
+        }
+        if (act && k < K) {
+            double* wd = w64 + ((size_t)bh * K + k) * D + a0;
+            reinterpret_cast<double2*>(wd)[0] = make_double2(w[c][0], w[c][1]);
+            reinterpret_cast<double2*>(wd)[1] = make_double2(w[c][2], w[c][3]);
             if (wop != nullptr) {
-                const uint16_t hi = double_to_bf16_bits(w[c]);
-                const double hid = (double)__uint_as_float(((uint32_t)hi) << 16);
-                const uint16_t lo = double_to_bf16_bits(w[c] - hid);  // w - hi is exact
-                wop[((size_t)bh * K + k) * (2 * D) + a] = hi;
-                wop[((size_t)bh * K + k) * (2 * D) + D + a] = lo;
+                uint32_t hi2[2], lo2[2];
+#pragma unroll
+                for (int j = 0; j < 4; j += 2) {
+                    uint16_t h[2], l[2];
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        h[q] = double_to_bf16_bits(w[c][j + q]);
+                        const double hid = (double)__uint_as_float(((uint32_t)h[q]) << 16);
+                        l[q] = double_to_bf16_bits(w[c][j + q] - hid);  // w - hi is exact
+                    }
+                    hi2[j >> 1] = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
+                    lo2[j >> 1] = (uint32_t)l[0] | ((uint32_t)l[1] << 16);
+                }
+                uint16_t* row = wop + ((size_t)bh * K + k) * (2 * D);
+                *reinterpret_cast<uint2*>(row + a0) = make_uint2(hi2[0], hi2[1]);
+                *reinterpret_cast<uint2*>(row + D + a0) = make_uint2(lo2[0], lo2[1]);
             }
         }
-        const double pb = warp_sum(ca * w[c]), pn = warp_sum(w[c] * w[c]);
-        if (lane == 0) {
-            red[cc][wq][0] = pb;
-            red[cc][wq][1] = pn;
+        pb = warp_sum(pb);
+        pn = warp_sum(pn);
+        if (lane == 0 && k < K) {
+            bias64[(size_t)bh * K + k] = pb;
+            bias32[(size_t)bh * bias_ld + k] = __double2float_rn(pb);
+            atomic_max_nonneg(wmax + bh, round_up_f(__double2float_ru(sqrt(pn))));
+            atomic_max_nonneg(bmax + bh, round_up_f(__double2float_ru(fabs(pb))));
         }
-    }
-    __syncthreads();
-    if (t < kPrepCents && k0 + t < K) {
-        const int k = k0 + t;
-        const double b = ((red[t][0][0] + red[t][1][0]) + red[t][2][0]) + red[t][3][0];
-        const double n2w = ((red[t][0][1] + red[t][1][1]) + red[t][2][1]) + red[t][3][1];
-        bias64[(size_t)bh * K + k] = b;
-        bias32[(size_t)bh * bias_ld + k] = __double2float_rn(b);
-        atomic_max_nonneg(wmax + bh, round_up_f(__double2float_ru(sqrt(n2w))));
-        atomic_max_nonneg(bmax + bh, round_up_f(__double2float_ru(fabs(b))));
     }
 }
 
