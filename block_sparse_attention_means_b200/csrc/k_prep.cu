@@ -14,8 +14,9 @@ namespace park {
 // element with |x| < 2^-20 (about one row in ten thousand in unit-scale data),
 // which the float64 partial sums cannot take exactly either.  With xnorm given
 // (bf16 rows of 128 elements: 16 pieces, one per lane of a half warp) it also
-// writes every row's ||x||, as k_row_norms does (float64 sum of squares, square
-// root rounded up to float), so the K-means needs no second pass over X.
+// writes every row's ||x|| for the certified assign bound (float64 sum of
+// squares, square root rounded up to float), so the K-means needs no second pass
+// over X.
 template <int BYTES>
 __global__ void k_input_check(const uint4* __restrict__ x, size_t n16, int32_t* status, size_t per_head16,
                               int32_t* __restrict__ wide, uint8_t* __restrict__ tiny_rows, size_t row16,
@@ -319,36 +320,6 @@ int launch_metric(const void* Q, int dtype, int BH, int N, int D, double* part, 
     ::park::prof_begin(st);
     k_metric_reduce<<<g2, 256, 0, st>>>(part, nchunks, N, D, M, M_out);
     PARK_TRY_LAUNCH("k_metric_reduce", st);
-    return PARK_OK;
-}
-
-// ---------------------------------------------------------------- row norms
-// ||x_i|| (float64 sum of squares, square root rounded up to float): one warp
-// per row.  Used only inside the certified score bound.
-template <typename T>
-__global__ void k_row_norms(const T* __restrict__ X, size_t rows, int D, float* __restrict__ out) {
-    size_t w = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    int lane = threadIdx.x & 31;
-    if (w >= rows) return;
-    const T* x = X + w * D;
-    double s = 0.0;
-    for (int j = lane; j < D; j += 32) {
-        double v = Elem<T>::to_double(x, j);
-        s += v * v;
-    }
-    s = warp_sum(s);
-    if (lane == 0) out[w] = round_up_f(__double2float_ru(sqrt(s)));
-}
-
-int launch_row_norms(const void* X, int dtype, int BH, int N, int D, float* xnorm, cudaStream_t st) {
-    size_t rows = (size_t)BH * N;
-    int blocks = (int)((rows * 32 + 255) / 256);
-    ::park::prof_begin(st);
-    if (dtype == PARK_BF16)
-        k_row_norms<bf16_t><<<blocks, 256, 0, st>>>((const bf16_t*)X, rows, D, xnorm);
-    else
-        k_row_norms<float><<<blocks, 256, 0, st>>>((const float*)X, rows, D, xnorm);
-    PARK_TRY_LAUNCH("k_row_norms", st);
     return PARK_OK;
 }
 

@@ -34,13 +34,12 @@ struct Lists {
 // |x| >= 2^16 (zeroed by the caller); per_head_elems = N * D.  tiny_rows (bf16,
 // may be null): one byte per row of row_elems elements, set to 1 where the row
 // holds a nonzero element with |x| < 2^-20 (zeroed by the caller).  xnorm (bf16
-// with row_elems = 128, may be null): every row's norm, as launch_row_norms.
+// with row_elems = 128, may be null): every row's norm, rounded up to float.
 int launch_input_check(const void* x, size_t n_elems, int dtype, int32_t* status, int32_t* wide,
                        size_t per_head_elems, uint8_t* tiny_rows, size_t row_elems, float* xnorm,
                        cudaStream_t st);
 int launch_metric(const void* Q, int dtype, int BH, int N, int D, double* part, int nchunks, double* M,
                   double* M_out, cudaStream_t st);
-int launch_row_norms(const void* X, int dtype, int BH, int N, int D, float* xnorm, cudaStream_t st);
 int launch_strided_init(const void* X, int dtype, int BH, int N, int D, int K, void* C, cudaStream_t st);
 int launch_centroid_prep(const void* C, int dtype, int BH, int K, int D, const double* M, CentroidOps ops,
                          cudaStream_t st);
