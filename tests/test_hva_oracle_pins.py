@@ -133,7 +133,7 @@ def test_merge_worked_example():
 
 def test_merge_ties_and_round_cap():
     # three 10-row clusters keeping the same 128-row block: every pair gains 1;
-    # round 1 pairs 0 with 1 (lowest partner on ties), round 2 adds 2
+    # the first merge round pairs 0 with 1 (lowest partner on ties), the second adds 2
     n = [10, 10, 10]
     mask = np.ones((3, 1), dtype=bool)
     assert hva.merge_clusters(n, mask, [128]).tolist() == [0, 0, 0]
