@@ -138,11 +138,11 @@ extern "C" {
 #define PARK_FLAG_MERGE_Q 0x80u
 #define PARK_FLAG_LOCAL_WINDOW 0x100u
 /* Implementation switch, no change to the result (up to float32 summation
- * order): on the bf16 path park_sparse_attn packs the last 128-row tile of a
- * query cluster with several tiles into the single tile of a cluster with
- * enough free rows when that needs fewer key tiles (every row still attends
- * only to its own cluster's kept key clusters; done only for NQ <= 2048);
- * this flag turns it off. */
+ * order): on the tensor-core path (bf16, D == 128) park_sparse_attn packs the
+ * last 128-row tile of a query cluster with several tiles into the single
+ * tile of a cluster with enough free rows when that needs fewer key tiles
+ * (every row still attends only to its own cluster's kept key clusters; done
+ * only for NQ <= 2048); this flag turns it off. */
 #define PARK_FLAG_NO_TILE_PACKING 0x200u
 
 /* ---- park_retrieval.counters indices (outputs, int64) ------------------ */
